@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark of the JetBlock token mixer on B200.
+
+One step = one serving iteration of the mixer on 2B shapes (H=12, dk=96,
+dv=256, d_model=1536, bf16 inputs, float32 state):
+  prefill  generator+conv (K1) and chunked GDN prefill (K2) over one new
+           4096-token sequence (zero initial state);
+  decode   generator+conv with history (K1, T=1) and the GDN decode step (K3)
+           for 256 running sequences, one token each; the state advances in
+           place from step to step (64 pre-drawn token sets, cycled).
+Tokens per step = 4096 + 256. Every rank runs its own copy of this work
+(independent shards, no collective on the data path): weak scaling.
+
+Prints one JSON line (rank 0). `--impl reference` times the float64 CPU
+oracle on the same workload instead (bounded sample per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+PREFILL = synth.CONFIGS["prefill_2b_t4096"]
+DECODE = synth.CONFIGS["decode_2b_b256"]
+TOKENS_PER_STEP = PREFILL.B * PREFILL.T + DECODE.B
+METRIC = "JetBlock prefill & decode tokens/s (2B/4B shapes); % of HBM/BF16 roofline"
+WORKLOAD = ("mixed serving step on 2B JetBlock shapes: prefill of one 4096-token sequence "
+            "(prefill_2b_t4096) + one decode token for each of 256 sequences (decode_2b_b256)")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ------------------------------------------------------------------ algorithmic traffic per launch
+def model_bytes():
+    """Algorithmic HBM bytes (and flops) per launch of each kernel of a step:
+    every input read once, every output written once."""
+    P, Dc = PREFILL, DECODE
+    e = 2  # bf16
+    T = P.B * P.T
+    k1p = T * (P.D * e + 2 * P.H * P.dv * e) + (P.D * 32 + 32 * P.H * 4) * e
+    k2p = (T * P.H * (2 * P.dk * e + 2 * P.dv * e + 8) + P.B * P.H * P.dv * P.dk * 4)
+    C = 64
+    k2p_flops = T * P.H * (2 * C * (3 * P.dk + 2 * P.dv) + 6 * P.dk * P.dv + C * C / 3)
+    k1d = Dc.B * (Dc.D * e + 2 * Dc.H * Dc.dv * e + 2 * 3 * Dc.H * Dc.dv * e) + (Dc.D * 32 + 32 * Dc.H * 4) * e
+    k3d = Dc.B * Dc.H * (2 * Dc.dv * Dc.dk * 4 + 2 * Dc.dk * e + 2 * Dc.dv * e + 8)
+    k3d_flops = Dc.B * Dc.H * 7 * Dc.dk * Dc.dv
+    return {
+        "genconv_prefill": dict(bytes=k1p, flops=T * (2 * P.D * 32 + 2 * 32 * P.H * 4 + 8 * P.H * P.dv)),
+        "gdn_prefill": dict(bytes=k2p, flops=k2p_flops),
+        "genconv_decode": dict(bytes=k1d, flops=Dc.B * (2 * Dc.D * 32 + 8 * Dc.H * Dc.dv)),
+        "gdn_decode": dict(bytes=k3d, flops=k3d_flops),
+    }
+
+
+def csrc_digest():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "linear_attention_lm_gen_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        h.update(f.encode())
+        h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, only if it was taken
+    on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    ent = d.get(kernel)
+    if not ent or ent.get("csrc_sha") != csrc_digest():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu=timestamp,{self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(index), "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self, t0: float, t1: float):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[4:9]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 - 1.0 <= r[0] <= t1 + 1.0] or rows
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ["active_mask", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i in range(1, 5) if r[3][i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ------------------------------------------------------------------ the GPU workload
+class Workload:
+    def __init__(self, device, seed: int):
+        import torch
+        import linear_attention_lm_gen_b200 as jet
+        self.torch, self.jet, self.dev = torch, jet, device
+
+        def T(a):
+            if a.dtype == np.uint16:
+                return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+            return torch.from_numpy(np.ascontiguousarray(a))
+
+        p = synth.prefill_inputs(PREFILL, seed=seed)
+        d = synth.decode_inputs(DECODE, seed=seed + 1)
+        self.host_p = {k: T(v).pin_memory() for k, v in p.items() if isinstance(v, np.ndarray)}
+        self.host_d = {k: T(v).pin_memory() for k, v in d.items() if isinstance(v, np.ndarray)}
+        self.p = {k: v.to(device) for k, v in self.host_p.items()}
+        self.d = {k: v.to(device) for k, v in self.host_d.items()}
+        P, Dc = PREFILL, DECODE
+        bf = torch.bfloat16
+        self.vc = torch.empty((P.B, P.T, P.H, P.dv), device=device, dtype=bf)
+        self.o = torch.empty_like(self.vc)
+        self.S_out = torch.empty((P.B, P.H, P.dv, P.dk), device=device, dtype=torch.float32)
+        self.S = self.d["S0"].clone()
+        self.hist = [self.d["hist"].clone(), torch.empty_like(self.d["hist"])]
+        self.vc_d = torch.empty((Dc.B, 1, Dc.H, Dc.dv), device=device, dtype=bf)
+        self.o_d = torch.empty((Dc.B, Dc.H, Dc.dv), device=device, dtype=bf)
+        ws = jet.jet_gdn_prefill_workspace_size(P.B, P.T, P.H, P.dk, P.dv)
+        self.ws = torch.empty(max(ws, 16), device=device, dtype=torch.uint8)
+        # pinned host buffers for the end-to-end pass
+        self.h_o = torch.empty(self.o.shape, dtype=bf).pin_memory()
+        self.h_o_d = torch.empty(self.o_d.shape, dtype=bf).pin_memory()
+        self.steps_done = 0
+
+    # four launches: K1 prefill, K2 prefill, K1 decode, K3 decode
+    def step(self, stream, i: int, ev=None):
+        jet, p, d = self.jet, self.p, self.d
+        if ev is not None:
+            ev[0].record(stream)
+        jet.jet_dyn_conv_v(p["x"], p["W1"], p["W2"], p["v"], None, self.vc, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        jet.jet_gdn_prefill(p["q"], p["k"], self.vc, p["g"], p["beta"], None, self.o, self.S_out, self.ws,
+                            stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        s = i % DECODE.steps
+        hin, hout = self.hist[i % 2], self.hist[(i + 1) % 2]
+        jet.jet_dyn_conv_v(d["x"][s][:, None], d["W1"], d["W2"], d["v"][s][:, None], hin, self.vc_d, hout,
+                           stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        jet.jet_gdn_decode_step(d["q"][s], d["k"][s], self.vc_d[:, 0], d["g"][s], d["beta"][s], self.S, self.o_d,
+                                stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    def h2d(self, stream, i: int) -> int:
+        """Copy one step's inputs from pinned host memory; returns bytes."""
+        n = 0
+        for k in ("x", "q", "k", "v", "g", "beta"):
+            self.p[k].copy_(self.host_p[k], non_blocking=True)
+            n += self.p[k].numel() * self.p[k].element_size()
+        s = i % DECODE.steps
+        for k in ("x", "q", "k", "v", "g", "beta"):
+            self.d[k][s].copy_(self.host_d[k][s], non_blocking=True)
+            n += self.d[k][s].numel() * self.d[k][s].element_size()
+        return n
+
+    def d2h(self, stream) -> int:
+        self.h_o.copy_(self.o, non_blocking=True)
+        self.h_o_d.copy_(self.o_d, non_blocking=True)
+        return self.o.numel() * 2 + self.o_d.numel() * 2
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+def oracle_step(orc, p64, d64, frac: float = 1.0, dstep: int = 0):
+    """The workload on the float64 oracle; `frac` < 1 takes the first frac of the
+    prefill tokens and of the decode sequences (same mix). Returns tokens done."""
+    Tp = max(1, int(round(PREFILL.T * frac)))
+    Bd = max(1, int(round(DECODE.B * frac)))
+    sl = lambda a: a[:, :Tp]
+    orc.jetblock_prefill(sl(p64["x"]), p64["W1"], p64["W2"], sl(p64["q"]), sl(p64["k"]), sl(p64["v"]),
+                         sl(p64["g"]), sl(p64["beta"]))
+    s = dstep % DECODE.steps
+    one = lambda a: a[s:s + 1, :Bd]
+    orc.jetblock_decode(one(d64["x"]), d64["W1"], d64["W2"], one(d64["q"]), one(d64["k"]), one(d64["v"]),
+                        one(d64["g"]), one(d64["beta"]), d64["S0"][:Bd], d64["hist"][:Bd])
+    return Tp * PREFILL.B + Bd
+
+
+def oracle_inputs(seed: int):
+    p = synth.prefill_inputs(PREFILL, seed=seed)
+    d = synth.decode_inputs(DECODE, seed=seed + 1)
+    f = lambda inp: {k: synth.to_f64(v, inp["dtype"]) if v.dtype == np.uint16 else v.astype(np.float64)
+                     for k, v in inp.items() if isinstance(v, np.ndarray)}
+    return f(p), f(d)
+
+
+def cpu_baseline(seed: int, budget_s: float = 15.0):
+    import oracle
+    orc = oracle.get()
+    p64, d64 = oracle_inputs(seed)
+    t0 = time.perf_counter()
+    tokens, reps = 0, 0
+    while True:
+        tokens += oracle_step(orc, p64, d64, 1.0, reps)
+        reps += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"{reps} full step(s) of the same workload (4096-token prefill + one decode token "
+                      f"for each of 256 sequences) on the float64 oracle, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    orc = oracle.get()
+    p64, d64 = oracle_inputs(args.seed)
+    t0 = time.perf_counter()
+    oracle_step(orc, p64, d64, 1.0, 0)
+    full = time.perf_counter() - t0
+    frac = min(1.0, 150.0 / max(1e-9, full * (args.steps + args.warmup)))
+    for i in range(args.warmup):
+        oracle_step(orc, p64, d64, frac, i)
+    t0 = time.perf_counter()
+    tokens = 0
+    for i in range(args.steps):
+        tokens += oracle_step(orc, p64, d64, frac, i)
+    dt = time.perf_counter() - t0
+    value = tokens / dt
+    sample = (f"each step: the first {frac:.3f} of the workload's prefill tokens and decode sequences "
+              f"(same 16:1 mix) on the float64 oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tokens_per_step_full": TOKENS_PER_STEP, "sample_fraction": frac},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": orc.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ main GPU arm
+def run_jet(args):
+    import torch
+    import torch.distributed as dist
+    from linear_attention_lm_gen_b200 import build as jbuild
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+
+    jbuild.build()
+    import linear_attention_lm_gen_b200 as jet
+    jet.load_library()
+    wl = Workload(device, seed=args.seed + 17 * rank)
+    stream = torch.cuda.Stream(device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            wl.step(stream, i)
+    if jet.jet_device_error(stream) != 0:
+        raise RuntimeError("device error word set after warm-up")
+
+    # ---- device-resident timed pass (per-kernel events inside it)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    barrier()
+    n0 = jet.jet_launch_count()
+    t_wall0 = time.time()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(args.steps):
+            wl.step(stream, args.warmup + i, evs[i])
+        stop.record(stream)
+    barrier()
+    t_wall1 = time.time()
+    launches = jet.jet_launch_count() - n0
+    clk = clocks.stop(t_wall0, t_wall1)
+    ms = max_over_ranks(start.elapsed_time(stop))
+    per_kernel = np.zeros(4)
+    for e in evs:
+        for j in range(4):
+            per_kernel[j] += e[j].elapsed_time(e[j + 1])
+    per_kernel /= args.steps                      # ms per launch
+    if jet.jet_device_error(stream) != 0:
+        raise RuntimeError("device error word set in the timed region")
+
+    # ---- end-to-end pass: host inputs in, results out, through the same calls
+    barrier()
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h2d = d2h = 0
+    with torch.cuda.stream(stream):
+        e_start.record(stream)
+        for i in range(args.steps):
+            h2d = wl.h2d(stream, i)
+            wl.step(stream, args.warmup + args.steps + i)
+            d2h = wl.d2h(stream)
+        e_stop.record(stream)
+    barrier()
+    e_ms = max_over_ranks(e_start.elapsed_time(e_stop))
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    pk = peaks()
+    mb = model_bytes()
+    names = ["genconv_prefill", "gdn_prefill", "genconv_decode", "gdn_decode"]
+    kern = {}
+    for j, n in enumerate(names):
+        t = per_kernel[j] * 1e-3
+        gbs = mb[n]["bytes"] / t / 1e9
+        kern[n] = {"us_per_launch": per_kernel[j] * 1e3, "algorithmic_bytes": mb[n]["bytes"],
+                   "algorithmic_flops": mb[n]["flops"], "achieved_gbs": gbs, "hbm_frac": gbs / pk["hbm_gbs"],
+                   "roofline_us": 1e6 * max(mb[n]["bytes"] / (pk["hbm_gbs"] * 1e9),
+                                            mb[n]["flops"] / (pk["bf16_tflops"] * 1e12))}
+    dom = names[int(np.argmax(per_kernel))]
+    ach = kern[dom]["achieved_gbs"]
+    tokens = TOKENS_PER_STEP * world
+    value = tokens * args.steps / (ms * 1e-3)
+    prefill_ms = per_kernel[0] + per_kernel[1]
+    decode_ms = per_kernel[2] + per_kernel[3]
+    roof_step_us = sum(k["roofline_us"] for k in kern.values())
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded numpy PCG64; shapes of the 2B JetBlock)",
+        "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": TOKENS_PER_STEP,
+                   "prefill": {"B": PREFILL.B, "T": PREFILL.T, "H": PREFILL.H, "dk": PREFILL.dk, "dv": PREFILL.dv,
+                               "d_model": PREFILL.D, "chunk": 64, "initial_state": "zero"},
+                   "decode": {"B": DECODE.B, "H": DECODE.H, "dk": DECODE.dk, "dv": DECODE.dv, "d_model": DECODE.D,
+                              "state": "float32, advanced in place every step", "token_sets": DECODE.steps},
+                   "l2": "inputs larger than L2: 608 MB of decode state streamed per step (L2 126 MB)",
+                   "parallelism": f"dp{world} (independent shard per GPU, no collective on the data path)"},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": ach / pk["hbm_gbs"], "traffic": ncu_traffic(dom),
+                     "peak_source": f"{pk['source']} (MEASURED_PEAKS.json hbm_gbs, burst copy)"},
+        "step_roofline": {"roofline_us": roof_step_us, "measured_us": 1e3 * ms / args.steps,
+                          "frac": roof_step_us / (1e3 * ms / args.steps)},
+        "phases": {
+            "prefill": {"tokens_per_s": PREFILL.T / (prefill_ms * 1e-3), "us": prefill_ms * 1e3,
+                        "roofline_us": kern["genconv_prefill"]["roofline_us"] + kern["gdn_prefill"]["roofline_us"]},
+            "decode": {"tokens_per_s": DECODE.B / (decode_ms * 1e-3), "us": decode_ms * 1e3,
+                       "roofline_us": kern["genconv_decode"]["roofline_us"] + kern["gdn_decode"]["roofline_us"]}},
+        "kernels": kern,
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "e2e": {"value": tokens * args.steps / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps},
+    }
+    for ph in line["phases"].values():
+        ph["roofline_frac"] = ph["roofline_us"] / ph["us"]
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.seed, args.cpu_budget)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="jet", choices=["jet", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)        # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_jet(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,138 @@
+/*
+ * jet.h — C ABI of the JetBlock token mixer on NVIDIA B200 (sm_100a).
+ *
+ * The mixer (Jet-Nemotron, "JetBlock"):
+ *   1. kernel generator   w_t = SiLU(x_t W1) W2          d_model -> 32 -> H*4
+ *   2. dynamic causal conv on V, width 4:
+ *        v'_t[h,:] = sum_{j=0..3} w_t[h,j] v_{t-j}[h,:]   (tap 0 = current token)
+ *   3. Gated DeltaNet on L2-normalised q, k (no 1/sqrt(dk) scale):
+ *        S_t = a_t (S_{t-1} - b_t (S_{t-1} k_t) k_t^T) + b_t v'_t k_t^T,
+ *        o_t = S_t q_t,   a_t = exp(g_t) (g_t <= 0),  b_t in (0,1),  S in R^{dv x dk}
+ * Sources: Jet-Nemotron paper (arXiv 2508.15884, Chinese translation on
+ * adg.csdn.net), section 2.3 "linear attention block selection" (Gated
+ * DeltaNet: data-dependent gate + delta rule) and section 2.4 "new attention
+ * block design" (kernel generator: linear reduction, SiLU, linear output of
+ * the conv taps; dynamic conv applied to V only; no static conv on Q/K); the
+ * xugj520.cn explainer, section 2.2 "JetBlock" (q/k dim 96 or 128, v dim 256,
+ * 12 or 16 heads, conv kernel 4, generator hidden 32).
+ *
+ * Conventions for every entry point
+ *   - Pointers are caller-owned DEVICE memory (except where stated). The
+ *     library never allocates or frees device memory and keeps no state
+ *     between calls except a per-device error word (see jet_device_error).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously. Argument checks are synchronous and
+ *     happen before any launch: on error nothing is enqueued.
+ *   - Layouts are dense row-major, token-major:
+ *       x [B,T,D];  q, k [B,T,H,dk];  v, v', o [B,T,H,dv];  g, beta [B,T,H];
+ *       W1 [D,hidden];  W2 [hidden,H*width] (column h*width+j = tap j of head h);
+ *       conv taps [B,T,H,width] float32;  state S [B,H,dv,dk] float32 (dk fastest);
+ *       conv history [B,width-1,H,dv] = raw V of positions -3,-2,-1 (oldest first).
+ *   - dtype JET_BF16: x, q, k, v, v', o, W1, W2 and the history are bf16; g, beta,
+ *     taps and states are float32; all arithmetic accumulates in float32.
+ *     dtype JET_F32: everything float32.
+ *   - Every pointer must be 16-byte aligned. Sizes must be > 0 (T may be any
+ *     length; no multiple of the chunk is needed) and the element counts must
+ *     fit in int64. Supported shapes: width == 4, hidden == 32, chunk == 64,
+ *     dk % 16 == 0 and dk <= 128, dv % 32 == 0 and dv <= 256, D % 16 == 0.
+ *     Anything else returns JET_ERR_UNSUPPORTED.
+ *   - Nothing aborts, exits or throws across the ABI. Thread-safe.
+ */
+#ifndef JET_H
+#define JET_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    JET_OK = 0,
+    JET_ERR_INVALID_ARG = 1,   /* null required pointer, size <= 0 or overflowing, aliasing */
+    JET_ERR_UNSUPPORTED = 2,   /* shape outside the supported set above */
+    JET_ERR_MISALIGNED = 3,    /* a pointer not 16-byte aligned */
+    JET_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    JET_ERR_TIMEOUT = 5,       /* a bounded in-kernel wait ran out (via jet_device_error) */
+    JET_ERR_DEVICE = 6,        /* a kernel flagged bad data (via jet_device_error) */
+    JET_ERR_WORKSPACE = 7      /* workspace pointer null or smaller than required */
+} jet_status;
+
+typedef enum { JET_F32 = 0, JET_BF16 = 1 } jet_dtype;
+
+/*
+ * Kernel generator only (step 1; paper section 2.4): conv_w[b,t,h,j] = w_t[h,j].
+ *   x [B,T,D], w1 [D,hidden], w2 [hidden,H*width] in `dt`; conv_w [B,T,H,width] float32 out.
+ */
+jet_status jet_kernel_gen(const void* x, const void* w1, const void* w2, float* conv_w,
+                          int B, int T, int D, int H, int hidden, int width,
+                          jet_dtype dt, void* stream);
+
+/*
+ * Generator fused with the dynamic causal conv on V (steps 1-2; paper section
+ * 2.4), one pass over V.
+ *   v [B,T,H,dv] raw values in; v_out [B,T,H,dv] conv output (v') out.
+ *   hist_in [B,width-1,H,dv] or NULL: raw V of the 3 positions before token 0
+ *     (NULL = zeros, i.e. the start of a sequence).
+ *   hist_out [B,width-1,H,dv] or NULL: receives the last 3 raw V positions of
+ *     [hist_in, v] (the history for the next call). Must not overlap hist_in.
+ *   conv_w_out [B,T,H,width] float32 or NULL: the generated taps.
+ * For decode call it with T = 1 and both histories.
+ */
+jet_status jet_dyn_conv_v(const void* x, const void* w1, const void* w2, const void* v,
+                          const void* hist_in, void* v_out, void* hist_out, float* conv_w_out,
+                          int B, int T, int D, int H, int dv, int hidden, int width,
+                          jet_dtype dt, void* stream);
+
+/*
+ * Bytes of device workspace jet_gdn_prefill needs for these sizes (may be 0).
+ */
+size_t jet_gdn_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt);
+
+/*
+ * Gated DeltaNet prefill over T tokens per sequence (step 3; paper section
+ * 2.3), chunkwise (chunk = 64) in the WY / UT-transform form; q and k are
+ * L2-normalised inside (eps 1e-6 under the square root).
+ *   q, k [B,T,H,dk]; v [B,T,H,dv] (normally v' from jet_dyn_conv_v); g, beta [B,T,H] float32.
+ *   S0 [B,H,dv,dk] float32 or NULL (zeros). o [B,T,H,dv] out.
+ *   S_out [B,H,dv,dk] float32 out: the state after token T-1; may alias S0.
+ *   workspace / ws_bytes: at least jet_gdn_prefill_workspace_size(...) bytes
+ *   (may be NULL when that is 0). Contents on entry are ignored.
+ * A prefill can be continued: pass its S_out as the next call's S0.
+ */
+jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const float* S0, void* o, float* S_out,
+                           void* workspace, size_t ws_bytes,
+                           int B, int T, int H, int dk, int dv, int chunk,
+                           jet_dtype dt, void* stream);
+
+/*
+ * One decode step (step 3 for a single new token per sequence), updating S in place:
+ *   u = S k,  S' = a S + (b v - a b u) k^T,  o = S' q.
+ *   q, k [B,H,dk]; v [B,H,dv] (v' of the new token); g, beta [B,H] float32;
+ *   S [B,H,dv,dk] float32 in/out; o [B,H,dv] out.
+ */
+jet_status jet_gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, float* S, void* o,
+                               int B, int H, int dk, int dv, jet_dtype dt, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's error
+ * word: JET_ERR_TIMEOUT if a bounded in-kernel wait ran out since the last
+ * call, JET_ERR_DEVICE if a kernel flagged bad data, JET_ERR_CUDA if the
+ * synchronisation itself failed, else JET_OK.
+ */
+jet_status jet_device_error(void* stream);
+
+/* Static string naming a status. */
+const char* jet_status_string(jet_status s);
+
+/* Number of kernels this library has launched in this process (all devices). */
+uint64_t jet_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JET_H */

@@ -1,0 +1,189 @@
+"""JetBlock token mixer on B200: Python binding of the C ABI in include/jet.h.
+
+Argument marshalling only: every step of the mixer runs in the CUDA kernels
+of ``libjet.so`` (built in-tree by ``build.py``). torch supplies device memory
+and the current stream. There is no CPU path: if the library is missing or
+no CUDA device is present, the calls raise.
+
+Function names match the C entry points:
+  jet_kernel_gen, jet_dyn_conv_v, jet_gdn_prefill_workspace_size,
+  jet_gdn_prefill, jet_gdn_decode_step, jet_device_error, jet_status_string,
+  jet_launch_count.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libjet.so")
+
+JET_F32, JET_BF16 = 0, 1
+STATUS = {0: "JET_OK", 1: "JET_ERR_INVALID_ARG", 2: "JET_ERR_UNSUPPORTED", 3: "JET_ERR_MISALIGNED",
+          4: "JET_ERR_CUDA", 5: "JET_ERR_TIMEOUT", 6: "JET_ERR_DEVICE", 7: "JET_ERR_WORKSPACE"}
+EXPORTS = ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill_workspace_size", "jet_gdn_prefill",
+           "jet_gdn_decode_step", "jet_device_error", "jet_status_string", "jet_launch_count")
+
+
+class JetError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libjet.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libjet.so not built at {path}: run linear_attention_lm_gen_b200/build.py")
+    L = ctypes.CDLL(path)
+    P, I, Z, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
+    L.jet_kernel_gen.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P]
+    L.jet_dyn_conv_v.argtypes = [P] * 8 + [I] * 8 + [P]
+    L.jet_gdn_prefill_workspace_size.argtypes = [I] * 7
+    L.jet_gdn_prefill_workspace_size.restype = Z
+    L.jet_gdn_prefill.argtypes = [P] * 9 + [Z] + [I] * 7 + [P]
+    L.jet_gdn_decode_step.argtypes = [P] * 7 + [I] * 5 + [P]
+    L.jet_device_error.argtypes = [P]
+    L.jet_status_string.argtypes = [I]
+    L.jet_status_string.restype = ctypes.c_char_p
+    L.jet_launch_count.argtypes = []
+    L.jet_launch_count.restype = U
+    for f in ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill", "jet_gdn_decode_step", "jet_device_error"):
+        getattr(L, f).restype = I
+    _lib = L
+    return L
+
+
+# ---------------------------------------------------------------- marshalling
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return JET_BF16
+    if t.dtype == torch.float32:
+        return JET_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or float32)")
+
+
+def _ptr(t, name, dtype=None, shape=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(fn, st):
+    if st != 0:
+        raise JetError(fn, st)
+
+
+# ---------------------------------------------------------------- entry points
+def jet_kernel_gen(x, W1, W2, H: int, conv_w=None, *, stream=None):
+    """x [B,T,D], W1 [D,32], W2 [32,H*4] -> conv taps [B,T,H,4] float32."""
+    L = load_library()
+    B, T, D = x.shape
+    dt = _dt(x)
+    if conv_w is None:
+        conv_w = torch.empty((B, T, H, 4), device=x.device, dtype=torch.float32)
+    st = L.jet_kernel_gen(_ptr(x, "x"), _ptr(W1, "W1", x.dtype, (D, 32)), _ptr(W2, "W2", x.dtype, (32, H * 4)),
+                          _ptr(conv_w, "conv_w", torch.float32, (B, T, H, 4)), B, T, D, H, 32, 4, dt, _stream(stream))
+    _check("jet_kernel_gen", st)
+    return conv_w
+
+
+def jet_dyn_conv_v(x, W1, W2, v, hist_in=None, v_out=None, hist_out=None, conv_w_out=None, *, stream=None):
+    """Generator + dynamic causal conv on V. v [B,T,H,dv] -> v' (same shape).
+    Returns (v_out, hist_out); hist_out is None unless a buffer is given."""
+    L = load_library()
+    B, T, D = x.shape
+    _, _, H, dv = v.shape
+    dt = _dt(x)
+    if v_out is None:
+        v_out = torch.empty_like(v)
+    st = L.jet_dyn_conv_v(_ptr(x, "x"), _ptr(W1, "W1", x.dtype, (D, 32)), _ptr(W2, "W2", x.dtype, (32, H * 4)),
+                          _ptr(v, "v", x.dtype, (B, T, H, dv)),
+                          _ptr(hist_in, "hist_in", x.dtype, (B, 3, H, dv)), _ptr(v_out, "v_out", x.dtype, (B, T, H, dv)),
+                          _ptr(hist_out, "hist_out", x.dtype, (B, 3, H, dv)),
+                          _ptr(conv_w_out, "conv_w_out", torch.float32, (B, T, H, 4)),
+                          B, T, D, H, dv, 32, 4, dt, _stream(stream))
+    _check("jet_dyn_conv_v", st)
+    return v_out, hist_out
+
+
+def jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
+    L = load_library()
+    return int(L.jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk,
+                                                JET_BF16 if dtype == torch.bfloat16 else JET_F32))
+
+
+def jet_gdn_prefill(q, k, v, g, beta, S0=None, o=None, S_out=None, workspace=None, *, stream=None):
+    """Chunked Gated DeltaNet prefill. q,k [B,T,H,dk], v [B,T,H,dv], g,beta [B,T,H]
+    float32, S0 [B,H,dv,dk] float32 or None. Returns (o, S_out)."""
+    L = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dt(q)
+    if o is None:
+        o = torch.empty((B, T, H, dv), device=q.device, dtype=q.dtype)
+    if S_out is None:
+        S_out = torch.empty((B, H, dv, dk), device=q.device, dtype=torch.float32)
+    need = jet_gdn_prefill_workspace_size(B, T, H, dk, dv, 64, q.dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = L.jet_gdn_prefill(_ptr(q, "q"), _ptr(k, "k", q.dtype, q.shape), _ptr(v, "v", q.dtype, (B, T, H, dv)),
+                           _ptr(g, "g", torch.float32, (B, T, H)), _ptr(beta, "beta", torch.float32, (B, T, H)),
+                           _ptr(S0, "S0", torch.float32, (B, H, dv, dk)), _ptr(o, "o", q.dtype, (B, T, H, dv)),
+                           _ptr(S_out, "S_out", torch.float32, (B, H, dv, dk)), _ptr(workspace, "workspace"),
+                           ws_bytes, B, T, H, dk, dv, 64, dt, _stream(stream))
+    _check("jet_gdn_prefill", st)
+    return o, S_out
+
+
+def jet_gdn_decode_step(q, k, v, g, beta, S, o=None, *, stream=None):
+    """One decode step, S [B,H,dv,dk] float32 updated in place. q,k [B,H,dk],
+    v [B,H,dv], g,beta [B,H]. Returns o [B,H,dv]."""
+    L = load_library()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dt(q)
+    if o is None:
+        o = torch.empty((B, H, dv), device=q.device, dtype=q.dtype)
+    st = L.jet_gdn_decode_step(_ptr(q, "q"), _ptr(k, "k", q.dtype, q.shape), _ptr(v, "v", q.dtype, (B, H, dv)),
+                               _ptr(g, "g", torch.float32, (B, H)), _ptr(beta, "beta", torch.float32, (B, H)),
+                               _ptr(S, "S", torch.float32, (B, H, dv, dk)), _ptr(o, "o", q.dtype, (B, H, dv)),
+                               B, H, dk, dv, dt, _stream(stream))
+    _check("jet_gdn_decode_step", st)
+    return o
+
+
+def jet_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status."""
+    return int(load_library().jet_device_error(_stream(stream)))
+
+
+def jet_status_string(status: int) -> str:
+    return load_library().jet_status_string(status).decode()
+
+
+def jet_launch_count() -> int:
+    return int(load_library().jet_launch_count())

@@ -1,0 +1,252 @@
+// C ABI of the JetBlock token mixer: argument checks, kernel selection and
+// launches. Declarations and the contract are in include/jet.h.
+#include "jet.h"
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "k_decode.cuh"
+#include "k_genconv.cuh"
+#include "k_prefill_simt.cuh"
+
+using namespace jet;
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+constexpr long long kMaxElems = (1LL << 62);
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool mul_ok(long long& acc, long long v) {
+    if (v <= 0) return false;
+    if (acc > kMaxElems / v) return false;
+    acc *= v;
+    return true;
+}
+
+// product of positive dimensions, or -1 on overflow / non-positive
+long long elems(std::initializer_list<long long> dims) {
+    long long acc = 1;
+    for (long long d : dims)
+        if (!mul_ok(acc, d)) return -1;
+    return acc;
+}
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+size_t esize(jet_dtype dt) { return dt == JET_BF16 ? 2 : 4; }
+
+jet_status launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? JET_OK : JET_ERR_CUDA;
+}
+
+// opt a kernel into more than 48 KB of dynamic shared memory
+template <typename K>
+jet_status smem_attr(K kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return JET_OK;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess
+               ? JET_OK : JET_ERR_CUDA;
+}
+
+bool dtype_ok(jet_dtype dt) { return dt == JET_F32 || dt == JET_BF16; }
+
+// ---------------------------------------------------------------- K1
+template <typename T>
+jet_status launch_genconv(const void* x, const void* w1, const void* w2, const void* v, const void* hin,
+                          void* vout, void* hout, float* cw, int B, int Tn, int D, int H, int dv,
+                          cudaStream_t s) {
+    const long long N = (long long)B * Tn;
+    const int HW4 = H * GC_W;
+    // small token counts (decode) use 16-token CTAs for more parallelism
+    if (N <= 148LL * 32) {
+        constexpr int TB = 16;
+        const size_t smem = sizeof(float) * gc_smem_floats(TB, HW4);
+        auto kern = genconv_kernel<T, TB>;
+        if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
+        kern<<<(unsigned)((N + TB - 1) / TB), GC_THREADS, smem, s>>>(
+            (const T*)x, (const T*)w1, (const T*)w2, (const T*)v, (const T*)hin, (T*)vout, (T*)hout, cw,
+            B, Tn, D, H, dv);
+    } else {
+        constexpr int TB = 32;
+        const size_t smem = sizeof(float) * gc_smem_floats(TB, HW4);
+        auto kern = genconv_kernel<T, TB>;
+        if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
+        kern<<<(unsigned)((N + TB - 1) / TB), GC_THREADS, smem, s>>>(
+            (const T*)x, (const T*)w1, (const T*)w2, (const T*)v, (const T*)hin, (T*)vout, (T*)hout, cw,
+            B, Tn, D, H, dv);
+    }
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return launch_status();
+}
+
+jet_status check_gen(const void* x, const void* w1, const void* w2, int B, int T, int D, int H,
+                     int hidden, int width, jet_dtype dt) {
+    if (!x || !w1 || !w2) return JET_ERR_INVALID_ARG;
+    if (!dtype_ok(dt)) return JET_ERR_INVALID_ARG;
+    if (elems({B, T, D}) < 0 || elems({B, T, H, 4}) < 0) return JET_ERR_INVALID_ARG;
+    if (hidden != GC_HID || width != GC_W || D % 16 != 0 || H > 64) return JET_ERR_UNSUPPORTED;
+    if ((long long)(B) * T / 16 + 1 > 0x7fffffffLL) return JET_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(w1) || !aligned16(w2)) return JET_ERR_MISALIGNED;
+    return JET_OK;
+}
+
+// ---------------------------------------------------------------- K2
+template <typename T, int DK>
+jet_status launch_prefill_simt(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                               const float* S0, void* o, float* S_out, int B, int Tn, int H, int dv,
+                               cudaStream_t s) {
+    const size_t smem = sizeof(float) * ps_smem_floats(DK);
+    auto kern = gdn_prefill_simt_kernel<T, DK>;
+    if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
+    dim3 grid(dv / PS_DVS, H, B);
+    kern<<<grid, PS_THREADS, smem, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta, S0, (T*)o, S_out, Tn, H, dv);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return launch_status();
+}
+
+template <typename T>
+jet_status dispatch_prefill(int dk, const void* q, const void* k, const void* v, const float* g,
+                            const float* beta, const float* S0, void* o, float* S_out, int B, int Tn,
+                            int H, int dv, cudaStream_t s) {
+    switch (dk) {
+#define JET_CASE(DK) case DK: return launch_prefill_simt<T, DK>(q, k, v, g, beta, S0, o, S_out, B, Tn, H, dv, s);
+        JET_CASE(16) JET_CASE(32) JET_CASE(48) JET_CASE(64)
+        JET_CASE(80) JET_CASE(96) JET_CASE(112) JET_CASE(128)
+#undef JET_CASE
+        default: return JET_ERR_UNSUPPORTED;
+    }
+}
+
+// ---------------------------------------------------------------- K3
+template <typename T, int NV>
+jet_status launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                         float* S, void* o, int B, int H, int dv, cudaStream_t s) {
+    dim3 grid((dv + DEC_ROWS - 1) / DEC_ROWS, H, B);
+    gdn_decode_kernel<T, NV><<<grid, DEC_THREADS, 0, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta, S,
+                                                        (T*)o, H, dv);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return launch_status();
+}
+
+template <typename T>
+jet_status dispatch_decode(int dk, const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, float* S, void* o, int B, int H, int dv, cudaStream_t s) {
+    switch (dk / 16) {
+#define JET_CASE(NV) case NV: return launch_decode<T, NV>(q, k, v, g, beta, S, o, B, H, dv, s);
+        JET_CASE(1) JET_CASE(2) JET_CASE(3) JET_CASE(4) JET_CASE(5) JET_CASE(6) JET_CASE(7) JET_CASE(8)
+#undef JET_CASE
+        default: return JET_ERR_UNSUPPORTED;
+    }
+}
+
+bool shape_ok(int dk, int dv) { return dk % 16 == 0 && dk >= 16 && dk <= 128 && dv % 32 == 0 && dv <= 256; }
+
+}  // namespace
+
+extern "C" {
+
+jet_status jet_kernel_gen(const void* x, const void* w1, const void* w2, float* conv_w, int B, int T, int D,
+                          int H, int hidden, int width, jet_dtype dt, void* stream) {
+    jet_status st = check_gen(x, w1, w2, B, T, D, H, hidden, width, dt);
+    if (st != JET_OK) return st;
+    if (!conv_w) return JET_ERR_INVALID_ARG;
+    if (!aligned16(conv_w)) return JET_ERR_MISALIGNED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == JET_BF16)
+        return launch_genconv<__nv_bfloat16>(x, w1, w2, nullptr, nullptr, nullptr, nullptr, conv_w, B, T, D, H, 32, s);
+    return launch_genconv<float>(x, w1, w2, nullptr, nullptr, nullptr, nullptr, conv_w, B, T, D, H, 32, s);
+}
+
+jet_status jet_dyn_conv_v(const void* x, const void* w1, const void* w2, const void* v, const void* hist_in,
+                          void* v_out, void* hist_out, float* conv_w_out, int B, int T, int D, int H, int dv,
+                          int hidden, int width, jet_dtype dt, void* stream) {
+    jet_status st = check_gen(x, w1, w2, B, T, D, H, hidden, width, dt);
+    if (st != JET_OK) return st;
+    if (!v || !v_out) return JET_ERR_INVALID_ARG;
+    const long long nv = elems({B, T, H, dv});
+    const long long nh = elems({B, 3, H, dv});
+    if (nv < 0 || nh < 0) return JET_ERR_INVALID_ARG;
+    if (dv % 32 != 0 || dv > 256) return JET_ERR_UNSUPPORTED;
+    for (const void* p : {v, (const void*)v_out, hist_in, (const void*)hist_out, (const void*)conv_w_out})
+        if (p && !aligned16(p)) return JET_ERR_MISALIGNED;
+    const size_t es = esize(dt);
+    if (overlap(v, nv * es, v_out, nv * es)) return JET_ERR_INVALID_ARG;
+    if (hist_in && hist_out && overlap(hist_in, nh * es, hist_out, nh * es)) return JET_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == JET_BF16)
+        return launch_genconv<__nv_bfloat16>(x, w1, w2, v, hist_in, v_out, hist_out, conv_w_out, B, T, D, H, dv, s);
+    return launch_genconv<float>(x, w1, w2, v, hist_in, v_out, hist_out, conv_w_out, B, T, D, H, dv, s);
+}
+
+size_t jet_gdn_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt) {
+    (void)B; (void)T; (void)H; (void)dk; (void)dv; (void)chunk; (void)dt;
+    return 0;
+}
+
+jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           const float* S0, void* o, float* S_out, void* workspace, size_t ws_bytes, int B,
+                           int T, int H, int dk, int dv, int chunk, jet_dtype dt, void* stream) {
+    if (!q || !k || !v || !g || !beta || !o || !S_out) return JET_ERR_INVALID_ARG;
+    if (!dtype_ok(dt)) return JET_ERR_INVALID_ARG;
+    if (elems({B, T, H, dk}) < 0 || elems({B, T, H, dv}) < 0 || elems({B, H, dv, dk}) < 0) return JET_ERR_INVALID_ARG;
+    if (!shape_ok(dk, dv) || chunk != 64 || B > 65535 || H > 65535) return JET_ERR_UNSUPPORTED;
+    for (const void* p : {q, k, v, (const void*)g, (const void*)beta, (const void*)S0, (const void*)o,
+                          (const void*)S_out, (const void*)workspace})
+        if (p && !aligned16(p)) return JET_ERR_MISALIGNED;
+    const size_t need = jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk, dt);
+    if (need > 0 && (!workspace || ws_bytes < need)) return JET_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == JET_BF16)
+        return dispatch_prefill<__nv_bfloat16>(dk, q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
+    return dispatch_prefill<float>(dk, q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
+}
+
+jet_status jet_gdn_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                               float* S, void* o, int B, int H, int dk, int dv, jet_dtype dt, void* stream) {
+    if (!q || !k || !v || !g || !beta || !S || !o) return JET_ERR_INVALID_ARG;
+    if (!dtype_ok(dt)) return JET_ERR_INVALID_ARG;
+    if (elems({B, H, dv, dk}) < 0) return JET_ERR_INVALID_ARG;
+    if (!shape_ok(dk, dv) || B > 65535 || H > 65535) return JET_ERR_UNSUPPORTED;
+    for (const void* p : {q, k, v, (const void*)g, (const void*)beta, (const void*)S, (const void*)o})
+        if (!aligned16(p)) return JET_ERR_MISALIGNED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == JET_BF16) return dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, B, H, dv, s);
+    return dispatch_decode<float>(dk, q, k, v, g, beta, S, o, B, H, dv, s);
+}
+
+jet_status jet_device_error(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return JET_ERR_CUDA;
+    int word = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&word, jet::g_dev_error, sizeof(int)) != cudaSuccess) return JET_ERR_CUDA;
+    if (cudaMemcpyToSymbol(jet::g_dev_error, &zero, sizeof(int)) != cudaSuccess) return JET_ERR_CUDA;
+    if (word & DEVERR_TIMEOUT) return JET_ERR_TIMEOUT;
+    if (word & DEVERR_DATA) return JET_ERR_DEVICE;
+    return JET_OK;
+}
+
+const char* jet_status_string(jet_status s) {
+    switch (s) {
+        case JET_OK: return "JET_OK";
+        case JET_ERR_INVALID_ARG: return "JET_ERR_INVALID_ARG";
+        case JET_ERR_UNSUPPORTED: return "JET_ERR_UNSUPPORTED";
+        case JET_ERR_MISALIGNED: return "JET_ERR_MISALIGNED";
+        case JET_ERR_CUDA: return "JET_ERR_CUDA";
+        case JET_ERR_TIMEOUT: return "JET_ERR_TIMEOUT";
+        case JET_ERR_DEVICE: return "JET_ERR_DEVICE";
+        case JET_ERR_WORKSPACE: return "JET_ERR_WORKSPACE";
+    }
+    return "JET_ERR_UNKNOWN";
+}
+
+uint64_t jet_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

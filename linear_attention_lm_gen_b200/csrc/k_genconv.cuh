@@ -1,0 +1,236 @@
+// K1: kernel generator fused with the dynamic causal conv on V.
+//
+// Jet-Nemotron paper, section 2.4: the generator shares the block input x,
+// reduces it linearly (d_model -> 32), applies SiLU, and a final linear layer
+// emits the conv taps (32 -> H*4). The taps of token t act on V only:
+//   v'_t[h,:] = sum_{j=0..3} w_t[h,j] v_{t-j}[h,:]   (tap 0 = current token)
+// with positions before token 0 taken from the history (or zero).
+//
+// One CTA owns TB consecutive tokens of the flattened [B*T] token axis:
+//   stage A  x[TB,D] . W1[D,32]: bf16 tensor-core mma (m16n8k16, fp32
+//            accumulate), the D reduction split over the 8 warps, partial
+//            sums reduced in shared memory; float32 inputs use FFMA.
+//   stage B  SiLU, then h[TB,32] . W2[32,H*4] in FFMA -> taps in shared memory
+//            (and optionally to global).
+//   stage C  conv: each work item is one 16-byte channel group of one head
+//            over a run of 8 tokens, holding a 3-token window in registers;
+//            loads and stores are 128-bit and consecutive threads touch
+//            consecutive 16-byte groups of a row (coalesced).
+// The x.W1 product is ~6.5 flop per HBM byte of the kernel, so the tensor
+// cores keep it in the shadow of the V stream.
+#pragma once
+#include "common.cuh"
+
+namespace jet {
+
+constexpr int GC_THREADS = 256;
+constexpr int GC_HID = 32;      // generator hidden width
+constexpr int GC_W = 4;         // conv width
+constexpr int GC_RUN = 8;       // tokens per conv work item
+
+// shared-memory layout (floats), TB tokens, HW4 = H*4 taps per token
+__host__ __device__ constexpr int gc_smem_floats(int TB, int HW4) {
+    return 8 * TB * GC_HID      // partial sums of the 8 warps (bf16 path)
+         + TB * (GC_HID + 1)    // hidden activations
+         + GC_HID * HW4         // W2 as float
+         + TB * HW4;            // taps
+}
+
+__device__ __forceinline__ uint32_t ld_u32(const void* p) { return *reinterpret_cast<const uint32_t*>(p); }
+__device__ __forceinline__ uint32_t pack_u16(uint16_t lo, uint16_t hi) { return (uint32_t)lo | ((uint32_t)hi << 16); }
+
+__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, const uint32_t* b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Stage A for bf16: z_part[warp][t][r] over the warp's share of the D axis.
+template <int TB>
+__device__ __forceinline__ void gen_stageA_bf16(const __nv_bfloat16* __restrict__ x,
+                                                const __nv_bfloat16* __restrict__ W1,
+                                                long long r0, long long N, int D, float* zpart) {
+    constexpr int MT = TB / 16;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, t4 = lane & 3;
+    const uint16_t* xs = reinterpret_cast<const uint16_t*>(x);
+    const uint16_t* ws = reinterpret_cast<const uint16_t*>(W1);
+    float acc[MT][4][4];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int n = 0; n < 4; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[m][n][e] = 0.f;
+
+    const int nks = D / 16;
+    for (int ks = warp; ks < nks; ks += 8) {
+        const int k0 = ks * 16 + t4 * 2;
+        uint32_t bfr[4][2];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            const int col = n * 8 + gid;
+            bfr[n][0] = pack_u16(__ldg(ws + (long long)k0 * GC_HID + col), __ldg(ws + (long long)(k0 + 1) * GC_HID + col));
+            bfr[n][1] = pack_u16(__ldg(ws + (long long)(k0 + 8) * GC_HID + col), __ldg(ws + (long long)(k0 + 9) * GC_HID + col));
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const long long ra = r0 + m * 16 + gid, rb = ra + 8;
+            uint32_t afr[4];
+            afr[0] = ra < N ? ld_u32(xs + ra * D + k0) : 0u;
+            afr[1] = rb < N ? ld_u32(xs + rb * D + k0) : 0u;
+            afr[2] = ra < N ? ld_u32(xs + ra * D + k0 + 8) : 0u;
+            afr[3] = rb < N ? ld_u32(xs + rb * D + k0 + 8) : 0u;
+#pragma unroll
+            for (int n = 0; n < 4; ++n) mma_bf16_16816(acc[m][n], afr, bfr[n]);
+        }
+    }
+    // accumulator fragment: rows gid / gid+8, cols t4*2, t4*2+1 of each n-tile
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            float* zp = zpart + (warp * TB + m * 16 + gid) * GC_HID + n * 8 + t4 * 2;
+            zp[0] = acc[m][n][0];
+            zp[1] = acc[m][n][1];
+            zp[8 * GC_HID] = acc[m][n][2];
+            zp[8 * GC_HID + 1] = acc[m][n][3];
+        }
+}
+
+template <typename T, int TB>
+__global__ void __launch_bounds__(GC_THREADS)
+genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __restrict__ W2,
+               const T* __restrict__ v, const T* __restrict__ hist_in, T* __restrict__ v_out,
+               T* __restrict__ hist_out, float* __restrict__ conv_w_out,
+               int Bn, int Tn, int D, int H, int dv) {
+    extern __shared__ float smem[];
+    const int HW4 = H * GC_W;
+    float* zpart = smem;                          // [8][TB][32]
+    float* hs = zpart + 8 * TB * GC_HID;          // [TB][33]
+    float* w2s = hs + TB * (GC_HID + 1);          // [32][HW4]
+    float* taps = w2s + GC_HID * HW4;             // [TB][HW4]
+
+    const int tid = threadIdx.x;
+    const long long N = (long long)Bn * Tn;
+    const long long r0 = (long long)blockIdx.x * TB;
+    const int nrows = (int)((N - r0) < TB ? (N - r0) : TB);
+
+    for (int i = tid; i < GC_HID * HW4; i += GC_THREADS) w2s[i] = Elem<T>::ld(W2 + i);
+
+    // ---- stage A: z = x . W1 ----
+    if constexpr (sizeof(T) == 2) {
+        gen_stageA_bf16<TB>(reinterpret_cast<const __nv_bfloat16*>(x),
+                            reinterpret_cast<const __nv_bfloat16*>(W1), r0, N, D, zpart);
+        __syncthreads();
+        for (int i = tid; i < TB * GC_HID; i += GC_THREADS) {
+            const int t = i / GC_HID, r = i % GC_HID;
+            float z = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) z += zpart[(w * TB + t) * GC_HID + r];
+            hs[t * (GC_HID + 1) + r] = z / (1.0f + expf(-z));
+        }
+    } else {
+        // float32: thread (t, 4 hidden units) in FFMA
+        for (int i = tid; i < TB * (GC_HID / 4); i += GC_THREADS) {
+            const int t = i / (GC_HID / 4), r4 = (i % (GC_HID / 4)) * 4;
+            float z[4] = {0.f, 0.f, 0.f, 0.f};
+            if (t < nrows) {
+                const T* xr = x + (r0 + t) * D;
+                for (int d = 0; d < D; ++d) {
+                    const float xv = Elem<T>::ld(xr + d);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) z[e] += xv * Elem<T>::ld(W1 + (long long)d * GC_HID + r4 + e);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) hs[t * (GC_HID + 1) + r4 + e] = z[e] / (1.0f + expf(-z[e]));
+        }
+    }
+    __syncthreads();
+
+    // ---- stage B: taps = h . W2 ----
+    for (int i = tid; i < TB * HW4; i += GC_THREADS) {
+        const int t = i / HW4, c = i % HW4;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int r = 0; r < GC_HID; ++r) acc += hs[t * (GC_HID + 1) + r] * w2s[r * HW4 + c];
+        taps[i] = acc;
+        if (conv_w_out && t < nrows) conv_w_out[(r0 + t) * HW4 + c] = acc;
+    }
+    if (v == nullptr) return;
+    __syncthreads();
+
+    // ---- stage C: causal conv over V ----
+    using V16 = Vec16<T>;
+    constexpr int VN = V16::N;                 // channels per 16-byte group
+    const int ngrp = dv / VN;                  // groups per head row
+    const int nruns = (nrows + GC_RUN - 1) / GC_RUN;
+    const int items = H * ngrp * nruns;
+    const long long rowstride = (long long)H * dv;   // elements per token
+    for (int it = tid; it < items; it += GC_THREADS) {
+        const int col = it % (H * ngrp);
+        const int run = it / (H * ngrp);
+        const int h = col / ngrp, cg = col % ngrp;
+        const long long coff = (long long)h * dv + (long long)cg * VN;
+        const int ta = run * GC_RUN;
+        const int tb = min(nrows, ta + GC_RUN);
+
+        // window: win[0] = v_{t-1}, win[1] = v_{t-2}, win[2] = v_{t-3}
+        float win[3][VN];
+        {
+            const long long rr = r0 + ta;
+            const int bseq = (int)(rr / Tn);
+            const long long tpos = rr % Tn;
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                const long long tau = tpos - 1 - j;
+                uint4 u = make_uint4(0, 0, 0, 0);
+                if (tau >= 0) {
+                    u = *reinterpret_cast<const uint4*>(v + (rr - 1 - j) * rowstride + coff);
+                } else if (hist_in) {
+                    u = *reinterpret_cast<const uint4*>(hist_in + ((long long)bseq * 3 + (3 + tau)) * rowstride + coff);
+                }
+                V16::unpack(u, win[j]);
+            }
+        }
+        uint4 cur[GC_RUN];
+#pragma unroll
+        for (int i = 0; i < GC_RUN; ++i)
+            if (ta + i < tb) cur[i] = *reinterpret_cast<const uint4*>(v + (r0 + ta + i) * rowstride + coff);
+#pragma unroll
+        for (int i = 0; i < GC_RUN; ++i) {
+            if (ta + i >= tb) break;
+            const long long rr = r0 + ta + i;
+            const long long tpos = rr % Tn;
+            const int bseq = (int)(rr / Tn);
+            if (tpos == 0 && i > 0) {           // a new sequence starts inside the run
+#pragma unroll
+                for (int j = 0; j < 3; ++j) {
+                    uint4 u = make_uint4(0, 0, 0, 0);
+                    if (hist_in) u = *reinterpret_cast<const uint4*>(hist_in + ((long long)bseq * 3 + (2 - j)) * rowstride + coff);
+                    V16::unpack(u, win[j]);
+                }
+            }
+            float cv[VN];
+            V16::unpack(cur[i], cv);
+            const float4 w4 = *reinterpret_cast<const float4*>(taps + (ta + i) * HW4 + h * GC_W);
+            float out[VN];
+#pragma unroll
+            for (int e = 0; e < VN; ++e)
+                out[e] = w4.x * cv[e] + w4.y * win[0][e] + w4.z * win[1][e] + w4.w * win[2][e];
+            *reinterpret_cast<uint4*>(v_out + rr * rowstride + coff) = V16::pack(out);
+#pragma unroll
+            for (int e = 0; e < VN; ++e) { win[2][e] = win[1][e]; win[1][e] = win[0][e]; win[0][e] = cv[e]; }
+            if (hist_out && tpos == Tn - 1) {
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    *reinterpret_cast<uint4*>(hist_out + ((long long)bseq * 3 + (2 - j)) * rowstride + coff) = V16::pack(win[j]);
+            }
+        }
+    }
+}
+
+}  // namespace jet

@@ -1,0 +1,132 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/jet.h declares, and rejects bad arguments before any CUDA call.
+
+Every call here that passes made-up pointer values also passes an argument
+that the host-side checks reject first, so no kernel is ever launched.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_lm_gen_b200 as jet
+from linear_attention_lm_gen_b200 import build as jbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "jet.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, WORKSPACE = 0, 1, 2, 3, 7
+A = 1 << 20          # an aligned, never-dereferenced address
+BF16, F32 = 1, 0
+
+
+@pytest.fixture(scope="module")
+def lib():
+    jbuild.build()
+    return jet.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(jet_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for f in ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill", "jet_gdn_decode_step",
+              "jet_gdn_prefill_workspace_size", "jet_device_error", "jet_status_string", "jet_launch_count"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libjet.so does not export {name}"
+    assert set(declared_functions()) == set(jet.EXPORTS)
+
+
+def test_status_strings(lib):
+    for code, name in jet.STATUS.items():
+        assert jet.jet_status_string(code) == name
+    assert jet.jet_status_string(99) == "JET_ERR_UNKNOWN"
+
+
+def test_launch_counter_is_readable(lib):
+    assert jet.jet_launch_count() >= 0
+
+
+def P(x):
+    return ctypes.c_void_p(x)
+
+
+def prefill(lib, q=A, k=A, v=A, g=A, b=A, S0=None, o=A, S=A, ws=None, wsb=0,
+            B=1, T=64, H=2, dk=16, dv=32, chunk=64, dt=BF16):
+    return lib.jet_gdn_prefill(P(q), P(k), P(v), P(g), P(b), P(S0), P(o), P(S), P(ws), wsb,
+                               B, T, H, dk, dv, chunk, dt, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), INVALID), (dict(o=None), INVALID), (dict(S=None), INVALID),
+    (dict(B=0), INVALID), (dict(T=-1), INVALID), (dict(H=0), INVALID),
+    (dict(dk=24), UNSUPPORTED), (dict(dk=144), UNSUPPORTED), (dict(dv=48), UNSUPPORTED),
+    (dict(dv=288), UNSUPPORTED), (dict(chunk=32), UNSUPPORTED), (dict(dt=7), INVALID),
+    (dict(q=A + 2), MISALIGNED), (dict(S0=A + 8), MISALIGNED), (dict(S=A + 4), MISALIGNED),
+    (dict(B=1 << 30, T=1 << 30, H=1 << 30), INVALID),
+])
+def test_prefill_rejects(lib, kw, expect):
+    assert prefill(lib, **kw) == expect
+
+
+def decode(lib, q=A, k=A, v=A, g=A, b=A, S=A, o=A, B=4, H=2, dk=16, dv=32, dt=BF16):
+    return lib.jet_gdn_decode_step(P(q), P(k), P(v), P(g), P(b), P(S), P(o), B, H, dk, dv, dt, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(S=None), INVALID), (dict(v=None), INVALID), (dict(B=0), INVALID),
+    (dict(dk=8), UNSUPPORTED), (dict(dv=40), UNSUPPORTED), (dict(o=A + 2), MISALIGNED),
+    (dict(dt=3), INVALID),
+])
+def test_decode_rejects(lib, kw, expect):
+    assert decode(lib, **kw) == expect
+
+
+def conv(lib, x=A, w1=A, w2=A, v=A, hin=None, vout=A + (1 << 24), hout=None, cw=None,
+         B=1, T=8, D=64, H=2, dv=32, hidden=32, width=4, dt=BF16):
+    return lib.jet_dyn_conv_v(P(x), P(w1), P(w2), P(v), P(hin), P(vout), P(hout), P(cw),
+                              B, T, D, H, dv, hidden, width, dt, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(x=None), INVALID), (dict(v=None), INVALID), (dict(vout=None), INVALID),
+    (dict(hidden=16), UNSUPPORTED), (dict(width=3), UNSUPPORTED), (dict(D=60), UNSUPPORTED),
+    (dict(dv=48), UNSUPPORTED), (dict(H=65), UNSUPPORTED),
+    (dict(v=A + 2), MISALIGNED), (dict(hout=A + 8 + (1 << 25)), MISALIGNED),
+    (dict(vout=A), INVALID),                                    # v_out overlaps v
+    (dict(hin=A + (1 << 26), hout=A + (1 << 26) + 16), INVALID),  # histories overlap
+    (dict(T=0), INVALID),
+])
+def test_dyn_conv_rejects(lib, kw, expect):
+    assert conv(lib, **kw) == expect
+
+
+def test_kernel_gen_rejects(lib):
+    f = lib.jet_kernel_gen
+    assert f(P(A), P(A), P(A), P(None), 1, 8, 64, 2, 32, 4, BF16, None) == INVALID
+    assert f(P(A), P(A), P(A), P(A + 4), 1, 8, 64, 2, 32, 4, BF16, None) == MISALIGNED
+    assert f(P(A), P(A), P(A), P(A), 1, 8, 64, 2, 8, 4, BF16, None) == UNSUPPORTED
+
+
+def test_workspace_query_is_host_only(lib):
+    n = jet.jet_gdn_prefill_workspace_size(1, 4096, 12, 96, 256)
+    assert n >= 0
+    if n > 0:
+        assert prefill(lib, B=1, T=4096, H=12, dk=96, dv=256, ws=None, wsb=0) == WORKSPACE
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises((TypeError, RuntimeError, AssertionError)):
+        jet.jet_kernel_gen(x, torch.zeros(64, 32, dtype=torch.bfloat16), torch.zeros(32, 8, dtype=torch.bfloat16),
+                           H=2, conv_w=torch.zeros(1, 4, 2, 4))

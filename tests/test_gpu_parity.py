@@ -1,0 +1,267 @@
+"""GPU parity: the CUDA library (through its C ABI) against the float64 oracle
+on identical seeded inputs.
+
+Pass criteria on outputs o and final states S (and conv history):
+bf16 inputs -> relative L2 <= 1e-2 and max-abs <= 5e-2; float32 -> relative
+L2 <= 1e-4. Stage checks of intermediate results use tighter bounds derived
+from their arithmetic (stated beside each). Outputs are poisoned with NaN
+before each call so unwritten elements fail the finiteness check.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from jet_testlib import TOL, assert_close, dev, errors, gpu_inputs, host64, to_oracle
+from oracle import get as get_oracle
+
+pytestmark = pytest.mark.gpu
+
+jet = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    global jet
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from linear_attention_lm_gen_b200 import build
+    build.build()
+    import linear_attention_lm_gen_b200 as m
+    m.load_library()
+    jet = m
+    yield
+    assert m.jet_device_error() == 0
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return get_oracle()
+
+
+def nan_like(t):
+    return torch.full_like(t, float("nan"))
+
+
+def shape(dtype, **kw):
+    base = dict(name="t", B=1, T=64, H=2, dk=16, dv=32, D=64, dtype=dtype)
+    base.update(kw)
+    return synth.JetShape(**base)
+
+
+# ------------------------------------------------------------------ K3 decode
+@pytest.mark.parametrize("dtype,H,dk,dv", [("f32", 2, 16, 32), ("bf16", 3, 96, 256), ("bf16", 2, 128, 256),
+                                           ("bf16", 2, 48, 64), ("f32", 3, 128, 96)])
+def test_decode_step_stage(orc, dtype, H, dk, dv):
+    s = shape(dtype, B=5, T=0, H=H, dk=dk, dv=dv, D=64, steps=2)
+    inp = synth.decode_inputs(s, seed=1)
+    d = gpu_inputs(inp)
+    ref = to_oracle(inp)
+    S = d["S0"].clone()
+    Sref = inp["S0"].astype(np.float64)
+    for step in range(2):
+        o = nan_like(d["v"][step])
+        jet.jet_gdn_decode_step(d["q"][step], d["k"][step], d["v"][step], d["g"][step], d["beta"][step], S, o)
+        ro, Sref = orc.gdn_decode_step(ref["q"][step], ref["k"][step], ref["v"][step], ref["g"][step],
+                                       ref["beta"][step], Sref)
+        assert_close(host64(o), ro, dtype, f"o step {step}")
+        # the state is float32 end to end: tight bound
+        assert_close(host64(S), Sref, dtype, f"S step {step}", tol=dict(rel_l2=1e-5, max_abs=1e-5))
+
+
+# ------------------------------------------------------------------ K1 generator + conv
+@pytest.mark.parametrize("dtype,B,T,H,dv,D,hist", [
+    ("f32", 1, 64, 2, 32, 64, False), ("f32", 2, 37, 2, 32, 64, True),
+    ("bf16", 1, 100, 12, 256, 1536, False), ("bf16", 3, 37, 12, 256, 1536, True),
+    ("bf16", 4, 1, 16, 256, 2048, True), ("bf16", 2, 2, 2, 64, 128, True), ("bf16", 1, 300, 2, 32, 64, False),
+])
+def test_generator_and_conv_stage(orc, dtype, B, T, H, dv, D, hist):
+    s = shape(dtype, B=B, T=T, H=H, dv=dv, D=D)
+    inp = synth.prefill_inputs(s, seed=2)
+    d = gpu_inputs(inp)
+    ref = to_oracle(inp)
+    hin_np = synth.jetblock._draw(np.random.default_rng(5), (B, 3, H, dv), dtype) if hist else None
+    hin = dev(hin_np, dtype) if hist else None
+    vout = nan_like(d["v"])
+    hout = torch.full((B, 3, H, dv), float("nan"), device="cuda", dtype=d["v"].dtype)
+    cw = torch.full((B, T, H, 4), float("nan"), device="cuda")
+    jet.jet_dyn_conv_v(d["x"], d["W1"], d["W2"], d["v"], hin, vout, hout, cw)
+    w = orc.kernel_gen(ref["x"], ref["W1"], ref["W2"], H)
+    vc, hist_ref = orc.dyn_conv(ref["v"], w, synth.to_f64(hin_np, dtype) if hist else None)
+    # taps: fp32 accumulation of bf16 / f32 products, no output rounding
+    assert_close(host64(cw), w, dtype, "taps", tol=dict(rel_l2=1e-5, max_abs=1e-4))
+    assert_close(host64(vout), vc, dtype, "v'")
+    # the new history is a copy of raw V: bit-exact
+    np.testing.assert_array_equal(host64(hout), hist_ref)
+    # the generator-only entry point gives the same taps bit for bit
+    cw2 = jet.jet_kernel_gen(d["x"], d["W1"], d["W2"], H)
+    assert torch.equal(cw2, cw)
+
+
+def test_identity_taps_via_conv_stage(orc):
+    # W2 = 0 gives zero taps: v' = 0 whatever V is (no hidden bias or tap offset)
+    s = shape("bf16", T=70, H=2, dv=64, D=128)
+    inp = synth.prefill_inputs(s, seed=3)
+    d = gpu_inputs(inp)
+    vout = nan_like(d["v"])
+    jet.jet_dyn_conv_v(d["x"], d["W1"], torch.zeros_like(d["W2"]), d["v"], None, vout)
+    assert torch.count_nonzero(vout.float()) == 0
+
+
+# ------------------------------------------------------------------ K2 prefill
+@pytest.mark.parametrize("dtype,H,dk,dv", [("f32", 2, 16, 32), ("bf16", 12, 96, 256), ("bf16", 2, 128, 256),
+                                           ("bf16", 3, 32, 64), ("f32", 2, 64, 64)])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 130])
+@pytest.mark.parametrize("s0", [False, True])
+def test_prefill_gdn_stage(orc, dtype, H, dk, dv, T, s0):
+    s = shape(dtype, B=2, T=T, H=H, dk=dk, dv=dv, D=64)
+    inp = synth.prefill_inputs(s, seed=T, s0_std=0.3 if s0 else None)
+    d = gpu_inputs(inp)
+    ref = to_oracle(inp)
+    o = nan_like(d["v"])
+    S_out = torch.full((2, H, dv, dk), float("nan"), device="cuda")
+    jet.jet_gdn_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d.get("S0"), o, S_out)
+    ro, rS = orc.gdn_sequential(ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"],
+                                inp["S0"].astype(np.float64) if s0 else None)
+    assert_close(host64(o), ro, dtype, "o")
+    assert_close(host64(S_out), rS, dtype, "S")
+
+
+@pytest.mark.parametrize("dtype,dk", [("bf16", 96), ("f32", 16)])
+def test_prefill_long_memory_gates(orc, dtype, dk):
+    # g = -0.01 softplus(N(0,1)): a ~ 0.99, so the state carries across many chunks
+    s = shape(dtype, B=1, T=400, H=2, dk=dk, dv=64, D=64)
+    inp = synth.prefill_inputs(s, seed=9, gate_scale=0.01, s0_std=0.1)
+    d = gpu_inputs(inp)
+    ref = to_oracle(inp)
+    o, S_out = jet.jet_gdn_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    ro, rS = orc.gdn_sequential(ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"], inp["S0"].astype(np.float64))
+    assert_close(host64(o), ro, dtype, "o")
+    assert_close(host64(S_out), rS, dtype, "S")
+
+
+def test_prefill_state_alias_and_continuation(orc):
+    # S_out may alias S0; prefill(T1) then prefill(T2) from its state = prefill(T1+T2)
+    s = shape("bf16", B=2, T=200, H=2, dk=64, dv=64, D=64)
+    inp = synth.prefill_inputs(s, seed=4, s0_std=0.2)
+    d = gpu_inputs(inp)
+    o_full, S_full = jet.jet_gdn_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    S = d["S0"].clone()
+    parts = []
+    for a, b in ((0, 77), (77, 200)):
+        sl = lambda t: t[:, a:b].contiguous()
+        o, _ = jet.jet_gdn_prefill(sl(d["q"]), sl(d["k"]), sl(d["v"]), sl(d["g"]), sl(d["beta"]), S, None, S)
+        parts.append(o)
+    e = errors(host64(torch.cat(parts, 1)), host64(o_full))
+    assert e["rel_l2"] < 1e-2
+    assert errors(host64(S), host64(S_full))["rel_l2"] < 1e-3
+
+
+# ------------------------------------------------------------------ whole mixer, stated configs
+def run_prefill(d, H, hist_out=False):
+    vc, hout = jet.jet_dyn_conv_v(d["x"], d["W1"], d["W2"], d["v"], None, None,
+                                  torch.empty((d["v"].shape[0], 3, H, d["v"].shape[-1]), device="cuda",
+                                              dtype=d["v"].dtype) if hist_out else None)
+    o, S = jet.jet_gdn_prefill(d["q"], d["k"], vc, d["g"], d["beta"])
+    return vc, o, S, hout
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "prefill_2b_t4096"])
+def test_config_prefill_full(orc, name):
+    s = synth.CONFIGS[name]
+    inp = synth.prefill_inputs(s, seed=0)
+    d = gpu_inputs(inp)
+    ref = to_oracle(inp)
+    vc, o, S, _ = run_prefill(d, s.H)
+    r = orc.jetblock_prefill(ref["x"], ref["W1"], ref["W2"], ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"])
+    assert_close(host64(o), r["o"], s.dtype, f"{name} o")
+    assert_close(host64(S), r["S"], s.dtype, f"{name} S")
+    assert_close(host64(vc), r["v_conv"], s.dtype, f"{name} v'")
+
+
+def sampled_prefill_reference(orc, inp, heads, rows, block=16384):
+    """Oracle outputs of chosen (head, state-row) chains over every token: the
+    generator for all tokens, then conv and recurrence restricted to those
+    value channels (rows of S are independent chains)."""
+    dt = inp["dtype"]
+    B, T, H, _ = inp["q"].shape
+    W1, W2 = synth.to_f64(inp["W1"], dt), synth.to_f64(inp["W2"], dt)
+    w = np.empty((B, T, H, 4))
+    for t0 in range(0, T, block):
+        w[:, t0:t0 + block] = orc.kernel_gen(synth.to_f64(inp["x"][:, t0:t0 + block], dt), W1, W2, H)
+    out = {}
+    for h in heads:
+        v = synth.to_f64(inp["v"][:, :, h:h + 1, rows], dt)
+        vc, _ = orc.dyn_conv(v, w[:, :, h:h + 1])
+        q = synth.to_f64(inp["q"][:, :, h:h + 1], dt)
+        k = synth.to_f64(inp["k"][:, :, h:h + 1], dt)
+        o, S = orc.gdn_sequential(q, k, vc, inp["g"][:, :, h:h + 1], inp["beta"][:, :, h:h + 1])
+        out[h] = (o[:, :, 0], S[:, 0], vc[:, :, 0])
+    return out
+
+
+@pytest.mark.parametrize("name", ["prefill_4b_t65536", "prefill_2b_t262144"])
+def test_config_long_prefill_sampled(orc, name):
+    s = synth.CONFIGS[name]
+    inp = synth.prefill_inputs(s, seed=0)
+    d = gpu_inputs(inp)
+    vc, o, S, _ = run_prefill(d, s.H)
+    heads, rows = [0, s.H - 3], [0, 1, 100, 255]
+    ref = sampled_prefill_reference(orc, inp, heads, rows)
+    for h in heads:
+        ro, rS, rvc = ref[h]
+        assert_close(host64(o[:, :, h, rows]), ro, s.dtype, f"{name} o head {h}")
+        assert_close(host64(S[:, h, rows]), rS, s.dtype, f"{name} S head {h}")
+        assert_close(host64(vc[:, :, h, rows]), rvc, s.dtype, f"{name} v' head {h}")
+
+
+def run_decode(d, steps, B, H, dv, dtype_t):
+    """Per step: generator + conv with history ping-pong (T = 1), then the GDN
+    decode step updating S in place. Returns outputs [n,B,H,dv], S, history."""
+    S = d["S0"].clone()
+    ha, hb = d["hist"].clone(), torch.empty_like(d["hist"])
+    outs = []
+    for t in range(steps):
+        vc, _ = jet.jet_dyn_conv_v(d["x"][t][:, None], d["W1"], d["W2"], d["v"][t][:, None], ha, None, hb)
+        o = jet.jet_gdn_decode_step(d["q"][t], d["k"][t], vc[:, 0], d["g"][t], d["beta"][t], S)
+        outs.append(o)
+        ha, hb = hb, ha
+    return torch.stack(outs), S, ha
+
+
+@pytest.mark.parametrize("name,steps,seqs", [
+    ("decode_2b_b256", 64, [0, 37, 128, 255]),
+    ("decode_4b_b1", 16, [0]), ("decode_4b_b16", 16, [0, 15]), ("decode_4b_b64", 8, [0, 63]),
+    ("decode_4b_b256", 8, [5, 200]), ("decode_4b_b1024", 4, [0, 511, 1023]),
+])
+def test_config_decode_sampled(orc, name, steps, seqs):
+    s = synth.CONFIGS[name]
+    inp = synth.decode_inputs(s, seed=0, steps=steps)
+    d = gpu_inputs(inp)
+    o, S, hist = run_decode(d, steps, s.B, s.H, s.dv, d["v"].dtype)
+    sel = lambda a: np.ascontiguousarray(a[:, seqs])
+    dt = s.dtype
+    r = orc.jetblock_decode(synth.to_f64(sel(inp["x"]), dt), synth.to_f64(inp["W1"], dt), synth.to_f64(inp["W2"], dt),
+                            synth.to_f64(sel(inp["q"]), dt), synth.to_f64(sel(inp["k"]), dt),
+                            synth.to_f64(sel(inp["v"]), dt), sel(inp["g"]), sel(inp["beta"]),
+                            inp["S0"][seqs].astype(np.float64), synth.to_f64(inp["hist"][seqs], dt))
+    assert_close(host64(o[:, seqs]), r["o"], dt, f"{name} o")
+    assert_close(host64(S[seqs]), r["S"], dt, f"{name} S")
+    np.testing.assert_array_equal(host64(hist[seqs]), r["hist"])
+
+
+def test_long_prefill_then_decode_continues(orc):
+    # prefill T tokens, then decode n more from its state and history = prefill of T+n
+    s = shape("bf16", B=2, T=150, H=12, dk=96, dv=256, D=1536)
+    n = 6
+    inp = synth.prefill_inputs(s, seed=11, T=s.T + n)
+    d = gpu_inputs(inp)
+    head = {k: v[:, :s.T].contiguous() for k, v in d.items() if k not in ("W1", "W2")}
+    head.update(W1=d["W1"], W2=d["W2"])
+    _, _, S, hist = run_prefill(head, s.H, hist_out=True)
+    tail = {k: v[:, s.T:].transpose(0, 1).contiguous() for k, v in d.items() if k not in ("W1", "W2")}
+    tail.update(W1=d["W1"], W2=d["W2"], S0=S, hist=hist)
+    o, S_end, _ = run_decode(tail, n, s.B, s.H, s.dv, d["v"].dtype)
+    ref = to_oracle(inp)
+    r = orc.jetblock_prefill(ref["x"], ref["W1"], ref["W2"], ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"])
+    assert_close(host64(o.transpose(0, 1)), r["o"][:, s.T:], "bf16", "decoded o")
+    assert_close(host64(S_end), r["S"], "bf16", "S after decode")
