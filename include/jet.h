@@ -31,10 +31,14 @@
  *   - dtype JET_BF16: x, q, k, v, v', o, W1, W2 and the history are bf16; g, beta,
  *     taps and states are float32; all arithmetic accumulates in float32.
  *     dtype JET_F32: everything float32.
- *   - Every pointer must be 16-byte aligned. Sizes must be > 0 (T may be any
- *     length; no multiple of the chunk is needed) and the element counts must
- *     fit in int64. Supported shapes: width == 4, hidden == 32, chunk == 64,
- *     dk % 16 == 0 and dk <= 128, dv % 32 == 0 and dv <= 256, D % 16 == 0.
+ *   - Alignment: the bulk tensors (x, q, k, v, v', o, histories, states,
+ *     workspace) must be 16-byte aligned; g, beta and conv taps 4-byte aligned;
+ *     W1 and W2 aligned to their element size. jet_gdn_decode_step needs 16
+ *     bytes only for S (its per-token q, k, v, o need element alignment).
+ *     Sizes must be > 0 (T may be any length; no multiple of the chunk is
+ *     needed) and the element counts must fit in int64.
+ *   - Supported shapes: width == 4, hidden == 32, chunk == 64, dk % 16 == 0
+ *     and dk <= 128, dv % 32 == 0 and dv <= 256, D % 16 == 0, H <= 64.
  *     Anything else returns JET_ERR_UNSUPPORTED.
  *   - Nothing aborts, exits or throws across the ABI. Thread-safe.
  */
@@ -52,7 +56,7 @@ typedef enum {
     JET_OK = 0,
     JET_ERR_INVALID_ARG = 1,   /* null required pointer, size <= 0 or overflowing, aliasing */
     JET_ERR_UNSUPPORTED = 2,   /* shape outside the supported set above */
-    JET_ERR_MISALIGNED = 3,    /* a pointer not 16-byte aligned */
+    JET_ERR_MISALIGNED = 3,    /* a pointer below its required alignment */
     JET_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
     JET_ERR_TIMEOUT = 5,       /* a bounded in-kernel wait ran out (via jet_device_error) */
     JET_ERR_DEVICE = 6,        /* a kernel flagged bad data (via jet_device_error) */

@@ -20,6 +20,7 @@ std::atomic<uint64_t> g_launches{0};
 constexpr long long kMaxElems = (1LL << 62);
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 bool mul_ok(long long& acc, long long v) {
     if (v <= 0) return false;
@@ -94,7 +95,8 @@ jet_status check_gen(const void* x, const void* w1, const void* w2, int B, int T
     if (elems({B, T, D}) < 0 || elems({B, T, H, 4}) < 0) return JET_ERR_INVALID_ARG;
     if (hidden != GC_HID || width != GC_W || D % 16 != 0 || H > 64) return JET_ERR_UNSUPPORTED;
     if ((long long)(B) * T / 16 + 1 > 0x7fffffffLL) return JET_ERR_UNSUPPORTED;
-    if (!aligned16(x) || !aligned16(w1) || !aligned16(w2)) return JET_ERR_MISALIGNED;
+    const size_t es = dt == JET_BF16 ? 2 : 4;
+    if (!aligned16(x) || !aligned_to(w1, es) || !aligned_to(w2, es)) return JET_ERR_MISALIGNED;
     return JET_OK;
 }
 
@@ -158,7 +160,7 @@ jet_status jet_kernel_gen(const void* x, const void* w1, const void* w2, float* 
     jet_status st = check_gen(x, w1, w2, B, T, D, H, hidden, width, dt);
     if (st != JET_OK) return st;
     if (!conv_w) return JET_ERR_INVALID_ARG;
-    if (!aligned16(conv_w)) return JET_ERR_MISALIGNED;
+    if (!aligned_to(conv_w, 4)) return JET_ERR_MISALIGNED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dt == JET_BF16)
         return launch_genconv<__nv_bfloat16>(x, w1, w2, nullptr, nullptr, nullptr, nullptr, conv_w, B, T, D, H, 32, s);
@@ -175,8 +177,9 @@ jet_status jet_dyn_conv_v(const void* x, const void* w1, const void* w2, const v
     const long long nh = elems({B, 3, H, dv});
     if (nv < 0 || nh < 0) return JET_ERR_INVALID_ARG;
     if (dv % 32 != 0 || dv > 256) return JET_ERR_UNSUPPORTED;
-    for (const void* p : {v, (const void*)v_out, hist_in, (const void*)hist_out, (const void*)conv_w_out})
+    for (const void* p : {v, (const void*)v_out, hist_in, (const void*)hist_out})
         if (p && !aligned16(p)) return JET_ERR_MISALIGNED;
+    if (conv_w_out && !aligned_to(conv_w_out, 4)) return JET_ERR_MISALIGNED;
     const size_t es = esize(dt);
     if (overlap(v, nv * es, v_out, nv * es)) return JET_ERR_INVALID_ARG;
     if (hist_in && hist_out && overlap(hist_in, nh * es, hist_out, nh * es)) return JET_ERR_INVALID_ARG;
@@ -198,9 +201,9 @@ jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const fl
     if (!dtype_ok(dt)) return JET_ERR_INVALID_ARG;
     if (elems({B, T, H, dk}) < 0 || elems({B, T, H, dv}) < 0 || elems({B, H, dv, dk}) < 0) return JET_ERR_INVALID_ARG;
     if (!shape_ok(dk, dv) || chunk != 64 || B > 65535 || H > 65535) return JET_ERR_UNSUPPORTED;
-    for (const void* p : {q, k, v, (const void*)g, (const void*)beta, (const void*)S0, (const void*)o,
-                          (const void*)S_out, (const void*)workspace})
+    for (const void* p : {q, k, v, (const void*)S0, (const void*)o, (const void*)S_out, (const void*)workspace})
         if (p && !aligned16(p)) return JET_ERR_MISALIGNED;
+    if (!aligned_to(g, 4) || !aligned_to(beta, 4)) return JET_ERR_MISALIGNED;
     const size_t need = jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk, dt);
     if (need > 0 && (!workspace || ws_bytes < need)) return JET_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -215,8 +218,10 @@ jet_status jet_gdn_decode_step(const void* q, const void* k, const void* v, cons
     if (!dtype_ok(dt)) return JET_ERR_INVALID_ARG;
     if (elems({B, H, dv, dk}) < 0) return JET_ERR_INVALID_ARG;
     if (!shape_ok(dk, dv) || B > 65535 || H > 65535) return JET_ERR_UNSUPPORTED;
-    for (const void* p : {q, k, v, (const void*)g, (const void*)beta, (const void*)S, (const void*)o})
-        if (!aligned16(p)) return JET_ERR_MISALIGNED;
+    const size_t es = esize(dt);
+    for (const void* p : {q, k, v, (const void*)o})
+        if (!aligned_to(p, es)) return JET_ERR_MISALIGNED;
+    if (!aligned_to(g, 4) || !aligned_to(beta, 4) || !aligned16(S)) return JET_ERR_MISALIGNED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dt == JET_BF16) return dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, B, H, dv, s);
     return dispatch_decode<float>(dk, q, k, v, g, beta, S, o, B, H, dv, s);

@@ -72,6 +72,7 @@ def prefill(lib, q=A, k=A, v=A, g=A, b=A, S0=None, o=A, S=A, ws=None, wsb=0,
     (dict(dk=24), UNSUPPORTED), (dict(dk=144), UNSUPPORTED), (dict(dv=48), UNSUPPORTED),
     (dict(dv=288), UNSUPPORTED), (dict(chunk=32), UNSUPPORTED), (dict(dt=7), INVALID),
     (dict(q=A + 2), MISALIGNED), (dict(S0=A + 8), MISALIGNED), (dict(S=A + 4), MISALIGNED),
+    (dict(g=A + 2), MISALIGNED),
     (dict(B=1 << 30, T=1 << 30, H=1 << 30), INVALID),
 ])
 def test_prefill_rejects(lib, kw, expect):
@@ -84,7 +85,8 @@ def decode(lib, q=A, k=A, v=A, g=A, b=A, S=A, o=A, B=4, H=2, dk=16, dv=32, dt=BF
 
 @pytest.mark.parametrize("kw,expect", [
     (dict(S=None), INVALID), (dict(v=None), INVALID), (dict(B=0), INVALID),
-    (dict(dk=8), UNSUPPORTED), (dict(dv=40), UNSUPPORTED), (dict(o=A + 2), MISALIGNED),
+    (dict(dk=8), UNSUPPORTED), (dict(dv=40), UNSUPPORTED), (dict(o=A + 1), MISALIGNED),
+    (dict(S=A + 4), MISALIGNED), (dict(g=A + 2), MISALIGNED),
     (dict(dt=3), INVALID),
 ])
 def test_decode_rejects(lib, kw, expect):
@@ -113,7 +115,7 @@ def test_dyn_conv_rejects(lib, kw, expect):
 def test_kernel_gen_rejects(lib):
     f = lib.jet_kernel_gen
     assert f(P(A), P(A), P(A), P(None), 1, 8, 64, 2, 32, 4, BF16, None) == INVALID
-    assert f(P(A), P(A), P(A), P(A + 4), 1, 8, 64, 2, 32, 4, BF16, None) == MISALIGNED
+    assert f(P(A), P(A), P(A), P(A + 2), 1, 8, 64, 2, 32, 4, BF16, None) == MISALIGNED
     assert f(P(A), P(A), P(A), P(A), 1, 8, 64, 2, 8, 4, BF16, None) == UNSUPPORTED
 
 
