@@ -2,6 +2,8 @@
 // launches. Declarations and the contract are in include/jet.h.
 #include "jet.h"
 
+#include <cuda.h>
+
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -10,6 +12,7 @@
 #include "k_decode.cuh"
 #include "k_genconv.cuh"
 #include "k_prefill_simt.cuh"
+#include "k_prefill_tc.cuh"
 
 using namespace jet;
 
@@ -114,6 +117,51 @@ jet_status launch_prefill_simt(const void* q, const void* k, const void* v, cons
     return launch_status();
 }
 
+// ---- TMA descriptors (driver entry point fetched once through the runtime)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (EncodeTiledFn) nullptr;
+        return (EncodeTiledFn)p;
+    }();
+    return fn;
+}
+
+// bf16 tensor [rows][H][d] viewed as 3-D (d, H, rows); box (64, 1, 64), 128-byte swizzle
+bool tile_map(CUtensorMap* m, const void* base, int d, int H, long long rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)rows};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * H * 2};
+    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DK>
+jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             const float* S0, void* o, float* S_out, int B, int Tn, int H, int dv, cudaStream_t s) {
+    CUtensorMap mq, mk, mv;
+    const long long rows = (long long)B * Tn;
+    if (!tile_map(&mq, q, DK, H, rows) || !tile_map(&mk, k, DK, H, rows) || !tile_map(&mv, v, dv, H, rows))
+        return JET_ERR_CUDA;
+    auto kern = pftc::gdn_prefill_tc_kernel<DK>;
+    if (smem_attr(kern, pftc::SMEM_BYTES) != JET_OK) return JET_ERR_CUDA;
+    dim3 grid(dv / pftc::ROWS, H, B);
+    kern<<<grid, pftc::THREADS, pftc::SMEM_BYTES, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return launch_status();
+}
+
 template <typename T>
 jet_status dispatch_prefill(int dk, const void* q, const void* k, const void* v, const float* g,
                             const float* beta, const float* S0, void* o, float* S_out, int B, int Tn,
@@ -207,6 +255,12 @@ jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const fl
     const size_t need = jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk, dt);
     if (need > 0 && (!workspace || ws_bytes < need)) return JET_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == JET_BF16 && dv % pftc::ROWS == 0 && (long long)B * T < (1LL << 31)) {
+        // tensor-core path: bf16, 128-row state slices, dk in {64, 96, 128}
+        if (dk == 64) return launch_prefill_tc<64>(q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
+        if (dk == 96) return launch_prefill_tc<96>(q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
+        if (dk == 128) return launch_prefill_tc<128>(q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
+    }
     if (dt == JET_BF16)
         return dispatch_prefill<__nv_bfloat16>(dk, q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
     return dispatch_prefill<float>(dk, q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);

@@ -109,8 +109,8 @@ def test_identity_taps_via_conv_stage(orc):
 
 # ------------------------------------------------------------------ K2 prefill
 @pytest.mark.parametrize("dtype,H,dk,dv", [("f32", 2, 16, 32), ("bf16", 12, 96, 256), ("bf16", 2, 128, 256),
-                                           ("bf16", 3, 32, 64), ("f32", 2, 64, 64)])
-@pytest.mark.parametrize("T", [1, 63, 64, 65, 130])
+                                           ("bf16", 3, 32, 64), ("f32", 2, 64, 64), ("bf16", 2, 64, 128)])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 130, 333])
 @pytest.mark.parametrize("s0", [False, True])
 def test_prefill_gdn_stage(orc, dtype, H, dk, dv, T, s0):
     s = shape(dtype, B=2, T=T, H=H, dk=dk, dv=dv, D=64)
