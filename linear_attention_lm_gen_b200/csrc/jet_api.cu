@@ -63,32 +63,34 @@ jet_status smem_attr(K kernel, size_t bytes) {
 bool dtype_ok(jet_dtype dt) { return dt == JET_F32 || dt == JET_BF16; }
 
 // ---------------------------------------------------------------- K1
+template <typename T, int TB, int RUN>
+jet_status launch_genconv_t(const void* x, const void* w1, const void* w2, const void* v, const void* hin,
+                            void* vout, void* hout, float* cw, int B, int Tn, int D, int H, int dv, int hpc,
+                            cudaStream_t s) {
+    const long long N = (long long)B * Tn;
+    const size_t smem = sizeof(float) * gc_smem_floats(TB, hpc * GC_W);
+    auto kern = genconv_kernel<T, TB, RUN>;
+    if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
+    dim3 grid((unsigned)((N + TB - 1) / TB), (unsigned)((H + hpc - 1) / hpc));
+    kern<<<grid, GC_THREADS, smem, s>>>((const T*)x, (const T*)w1, (const T*)w2, (const T*)v, (const T*)hin,
+                                        (T*)vout, (T*)hout, cw, B, Tn, D, H, dv, hpc);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return launch_status();
+}
+
 template <typename T>
 jet_status launch_genconv(const void* x, const void* w1, const void* w2, const void* v, const void* hin,
                           void* vout, void* hout, float* cw, int B, int Tn, int D, int H, int dv,
                           cudaStream_t s) {
-    const long long N = (long long)B * Tn;
-    const int HW4 = H * GC_W;
-    // small token counts (decode) use 16-token CTAs for more parallelism
-    if (N <= 148LL * 32) {
-        constexpr int TB = 16;
-        const size_t smem = sizeof(float) * gc_smem_floats(TB, HW4);
-        auto kern = genconv_kernel<T, TB>;
-        if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
-        kern<<<(unsigned)((N + TB - 1) / TB), GC_THREADS, smem, s>>>(
-            (const T*)x, (const T*)w1, (const T*)w2, (const T*)v, (const T*)hin, (T*)vout, (T*)hout, cw,
-            B, Tn, D, H, dv);
-    } else {
-        constexpr int TB = 32;
-        const size_t smem = sizeof(float) * gc_smem_floats(TB, HW4);
-        auto kern = genconv_kernel<T, TB>;
-        if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
-        kern<<<(unsigned)((N + TB - 1) / TB), GC_THREADS, smem, s>>>(
-            (const T*)x, (const T*)w1, (const T*)w2, (const T*)v, (const T*)hin, (T*)vout, (T*)hout, cw,
-            B, Tn, D, H, dv);
-    }
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return launch_status();
+    constexpr int TB = 16;
+    const long long nblk = ((long long)B * Tn + TB - 1) / TB;
+    // split heads across CTAs until the grid covers the SMs about twice
+    int groups = 1;
+    while (groups < H && nblk * groups < 296) ++groups;
+    const int hpc = (H + groups - 1) / groups;
+    if (Tn >= 8)
+        return launch_genconv_t<T, TB, 8>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, hpc, s);
+    return launch_genconv_t<T, TB, 1>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, hpc, s);
 }
 
 jet_status check_gen(const void* x, const void* w1, const void* w2, int B, int T, int D, int H,

@@ -6,14 +6,15 @@
 //   v'_t[h,:] = sum_{j=0..3} w_t[h,j] v_{t-j}[h,:]   (tap 0 = current token)
 // with positions before token 0 taken from the history (or zero).
 //
-// One CTA owns TB consecutive tokens of the flattened [B*T] token axis:
+// One CTA owns TB consecutive tokens of the flattened [B*T] token axis and a
+// group of heads:
 //   stage A  x[TB,D] . W1[D,32]: bf16 tensor-core mma (m16n8k16, fp32
 //            accumulate), the D reduction split over the 8 warps, partial
 //            sums reduced in shared memory; float32 inputs use FFMA.
 //   stage B  SiLU, then h[TB,32] . W2[32,H*4] in FFMA -> taps in shared memory
 //            (and optionally to global).
 //   stage C  conv: each work item is one 16-byte channel group of one head
-//            over a run of 8 tokens, holding a 3-token window in registers;
+//            over a run of tokens, holding a 3-token window in registers;
 //            loads and stores are 128-bit and consecutive threads touch
 //            consecutive 16-byte groups of a row (coalesced).
 // The x.W1 product is ~6.5 flop per HBM byte of the kernel, so the tensor
@@ -26,14 +27,13 @@ namespace jet {
 constexpr int GC_THREADS = 256;
 constexpr int GC_HID = 32;      // generator hidden width
 constexpr int GC_W = 4;         // conv width
-constexpr int GC_RUN = 8;       // tokens per conv work item
 
-// shared-memory layout (floats), TB tokens, HW4 = H*4 taps per token
-__host__ __device__ constexpr int gc_smem_floats(int TB, int HW4) {
+// shared-memory layout (floats), TB tokens, CW = tap columns per CTA
+__host__ __device__ constexpr int gc_smem_floats(int TB, int CW) {
     return 8 * TB * GC_HID      // partial sums of the 8 warps (bf16 path)
          + TB * (GC_HID + 1)    // hidden activations
-         + GC_HID * HW4         // W2 as float
-         + TB * HW4;            // taps
+         + GC_HID * CW          // W2 columns of the CTA's heads, as float
+         + TB * CW;             // taps
 }
 
 __device__ __forceinline__ uint32_t ld_u32(const void* p) { return *reinterpret_cast<const uint32_t*>(p); }
@@ -66,6 +66,7 @@ __device__ __forceinline__ void gen_stageA_bf16(const __nv_bfloat16* __restrict_
             for (int e = 0; e < 4; ++e) acc[m][n][e] = 0.f;
 
     const int nks = D / 16;
+#pragma unroll 4
     for (int ks = warp; ks < nks; ks += 8) {
         const int k0 = ks * 16 + t4 * 2;
         uint32_t bfr[4][2];
@@ -100,27 +101,39 @@ __device__ __forceinline__ void gen_stageA_bf16(const __nv_bfloat16* __restrict_
         }
 }
 
-template <typename T, int TB>
+// Grid: x = blocks of TB tokens, y = head groups of `hpc` heads. Every CTA of
+// a token block computes the (cheap) hidden activations of its tokens; the
+// taps and the conv are split across the head groups so that small token
+// counts (decode: one token per sequence) still spread over many SMs.
+// RUN = tokens per conv work item (8 keeps a sliding window in registers;
+// 1 makes every token an independent item with its 4 loads in flight).
+template <typename T, int TB, int RUN>
 __global__ void __launch_bounds__(GC_THREADS)
 genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __restrict__ W2,
                const T* __restrict__ v, const T* __restrict__ hist_in, T* __restrict__ v_out,
                T* __restrict__ hist_out, float* __restrict__ conv_w_out,
-               int Bn, int Tn, int D, int H, int dv) {
+               int Bn, int Tn, int D, int H, int dv, int hpc) {
     extern __shared__ float smem[];
     const int HW4 = H * GC_W;
+    const int h0 = blockIdx.y * hpc;
+    const int nh = min(hpc, H - h0);
+    const int CW = nh * GC_W;                     // tap columns of this CTA
     float* zpart = smem;                          // [8][TB][32]
     float* hs = zpart + 8 * TB * GC_HID;          // [TB][33]
-    float* w2s = hs + TB * (GC_HID + 1);          // [32][HW4]
-    float* taps = w2s + GC_HID * HW4;             // [TB][HW4]
+    float* w2s = hs + TB * (GC_HID + 1);          // [32][CW]
+    float* taps = w2s + GC_HID * CW;              // [TB][CW]
 
     const int tid = threadIdx.x;
     const long long N = (long long)Bn * Tn;
     const long long r0 = (long long)blockIdx.x * TB;
     const int nrows = (int)((N - r0) < TB ? (N - r0) : TB);
 
-    for (int i = tid; i < GC_HID * HW4; i += GC_THREADS) w2s[i] = Elem<T>::ld(W2 + i);
+    for (int i = tid; i < GC_HID * CW; i += GC_THREADS) {
+        const int r = i / CW, c = i % CW;
+        w2s[i] = Elem<T>::ld(W2 + (long long)r * HW4 + h0 * GC_W + c);
+    }
 
-    // ---- stage A: z = x . W1 ----
+    // ---- stage A: z = x . W1, SiLU ----
     if constexpr (sizeof(T) == 2) {
         gen_stageA_bf16<TB>(reinterpret_cast<const __nv_bfloat16*>(x),
                             reinterpret_cast<const __nv_bfloat16*>(W1), r0, N, D, zpart);
@@ -151,14 +164,14 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
     }
     __syncthreads();
 
-    // ---- stage B: taps = h . W2 ----
-    for (int i = tid; i < TB * HW4; i += GC_THREADS) {
-        const int t = i / HW4, c = i % HW4;
+    // ---- stage B: taps of this CTA's heads = h . W2 ----
+    for (int i = tid; i < TB * CW; i += GC_THREADS) {
+        const int t = i / CW, c = i % CW;
         float acc = 0.f;
 #pragma unroll 8
-        for (int r = 0; r < GC_HID; ++r) acc += hs[t * (GC_HID + 1) + r] * w2s[r * HW4 + c];
+        for (int r = 0; r < GC_HID; ++r) acc += hs[t * (GC_HID + 1) + r] * w2s[r * CW + c];
         taps[i] = acc;
-        if (conv_w_out && t < nrows) conv_w_out[(r0 + t) * HW4 + c] = acc;
+        if (conv_w_out && t < nrows) conv_w_out[(r0 + t) * HW4 + h0 * GC_W + c] = acc;
     }
     if (v == nullptr) return;
     __syncthreads();
@@ -167,19 +180,22 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
     using V16 = Vec16<T>;
     constexpr int VN = V16::N;                 // channels per 16-byte group
     const int ngrp = dv / VN;                  // groups per head row
-    const int nruns = (nrows + GC_RUN - 1) / GC_RUN;
-    const int items = H * ngrp * nruns;
+    const int nruns = (nrows + RUN - 1) / RUN;
+    const int cols = nh * ngrp;
+    const int items = cols * nruns;
     const long long rowstride = (long long)H * dv;   // elements per token
     for (int it = tid; it < items; it += GC_THREADS) {
-        const int col = it % (H * ngrp);
-        const int run = it / (H * ngrp);
-        const int h = col / ngrp, cg = col % ngrp;
+        const int col = it % cols;
+        const int run = it / cols;
+        const int hl = col / ngrp, cg = col % ngrp;
+        const int h = h0 + hl;
         const long long coff = (long long)h * dv + (long long)cg * VN;
-        const int ta = run * GC_RUN;
-        const int tb = min(nrows, ta + GC_RUN);
+        const int ta = run * RUN;
+        const int tb = min(nrows, ta + RUN);
 
         // window: win[0] = v_{t-1}, win[1] = v_{t-2}, win[2] = v_{t-3}
-        float win[3][VN];
+        uint4 wraw[3];
+        uint4 cur[RUN];
         {
             const long long rr = r0 + ta;
             const int bseq = (int)(rr / Tn);
@@ -187,26 +203,24 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
 #pragma unroll
             for (int j = 0; j < 3; ++j) {
                 const long long tau = tpos - 1 - j;
-                uint4 u = make_uint4(0, 0, 0, 0);
-                if (tau >= 0) {
-                    u = *reinterpret_cast<const uint4*>(v + (rr - 1 - j) * rowstride + coff);
-                } else if (hist_in) {
-                    u = *reinterpret_cast<const uint4*>(hist_in + ((long long)bseq * 3 + (3 + tau)) * rowstride + coff);
-                }
-                V16::unpack(u, win[j]);
+                wraw[j] = make_uint4(0, 0, 0, 0);
+                if (tau >= 0) wraw[j] = *reinterpret_cast<const uint4*>(v + (rr - 1 - j) * rowstride + coff);
+                else if (hist_in) wraw[j] = *reinterpret_cast<const uint4*>(hist_in + ((long long)bseq * 3 + (3 + tau)) * rowstride + coff);
             }
+#pragma unroll
+            for (int i = 0; i < RUN; ++i)
+                if (ta + i < tb) cur[i] = *reinterpret_cast<const uint4*>(v + (rr + i) * rowstride + coff);
         }
-        uint4 cur[GC_RUN];
+        float win[3][VN];
 #pragma unroll
-        for (int i = 0; i < GC_RUN; ++i)
-            if (ta + i < tb) cur[i] = *reinterpret_cast<const uint4*>(v + (r0 + ta + i) * rowstride + coff);
+        for (int j = 0; j < 3; ++j) V16::unpack(wraw[j], win[j]);
 #pragma unroll
-        for (int i = 0; i < GC_RUN; ++i) {
+        for (int i = 0; i < RUN; ++i) {
             if (ta + i >= tb) break;
             const long long rr = r0 + ta + i;
             const long long tpos = rr % Tn;
             const int bseq = (int)(rr / Tn);
-            if (tpos == 0 && i > 0) {           // a new sequence starts inside the run
+            if (RUN > 1 && tpos == 0 && i > 0) {   // a new sequence starts inside the run
 #pragma unroll
                 for (int j = 0; j < 3; ++j) {
                     uint4 u = make_uint4(0, 0, 0, 0);
@@ -216,7 +230,7 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
             }
             float cv[VN];
             V16::unpack(cur[i], cv);
-            const float4 w4 = *reinterpret_cast<const float4*>(taps + (ta + i) * HW4 + h * GC_W);
+            const float4 w4 = *reinterpret_cast<const float4*>(taps + (ta + i) * CW + hl * GC_W);
             float out[VN];
 #pragma unroll
             for (int e = 0; e < VN; ++e)

@@ -22,8 +22,9 @@
 // The L2 norms of q and k are folded into per-token scale factors, so the raw
 // bf16 q / k / v tiles from TMA serve directly as MMA operands. The float32
 // state lives in TMEM for the whole sequence; its bf16 copy is the A operand
-// of P3 / P5a. The UT inverse is a blocked (16 x 16) forward substitution in
-// float32 on the CUDA cores. Decay factors are formed as exp(G_r - G_i) <= 1.
+// of P3 / P5a. The UT inverse (I + A)^-1 is computed in float32 on the CUDA
+// cores by recursive doubling over 16 x 16 blocks. Decay factors are formed
+// as exp(G_r - G_i) <= 1.
 //
 // One CTA = (sequence, head, 128 state rows); 128 threads; thread 0 issues
 // TMA and MMA; the four warps read TMEM lanes 32w..32w+31 in the epilogues.
@@ -57,20 +58,23 @@ constexpr uint32_t OFF_AW = OFF_AS + 32768;             // 16K Wt^T
 constexpr uint32_t OFF_AWD = OFF_AW + 16384;            // 16K Wt^T diag(d/|k|)
 constexpr uint32_t OFF_AF = OFF_AS;                     // fp32 A [64][65] (aliases AS..AWD)
 constexpr uint32_t OFF_TF = OFF_AS + 64 * 65 * 4;       // fp32 T [64][65]
-constexpr uint32_t OFF_XB = OFF_TF + 64 * 65 * 4;       // fp32 block products [3][16][16]
+constexpr uint32_t OFF_XB = OFF_TF + 64 * 65 * 4;       // fp32 block products (1024 floats)
 constexpr uint32_t OFF_VEC = OFF_AWD + 16384;           // per-token vectors, 8 x 64 floats
 constexpr uint32_t OFF_BAR = OFF_VEC + 2048;
 constexpr uint32_t OFF_TSLOT = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = OFF_TSLOT + 64 + 1024;  // + alignment slack
-static_assert(OFF_XB + 3 * 256 * 4 <= OFF_VEC, "fp32 scratch overflows its alias region");
+static_assert(OFF_XB + 1024 * 4 <= OFF_VEC, "fp32 scratch overflows its alias region");
 
 // TMEM columns
 constexpr uint32_t TM_S = 0, TM_X1 = 128, TM_X2 = 192, TM_X3 = 256, TM_XP = 320, TM_XW = 384;
 constexpr uint32_t TM_COLS = 512;
 
+// per-token vectors of a chunk; G is kept in log2 units (G * log2 e) so that
+// every decay factor is one exp2 of a difference
 struct Vecs {
     float* G; float* gam; float* dcy; float* bet; float* ik; float* iq; float* graw;
 };
+constexpr float LOG2E = 1.4426950408889634f;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -100,42 +104,90 @@ __device__ __forceinline__ float row_sumsq(const uint8_t* tile, int row, int nch
     return s;
 }
 
-// T = (I + A)^-1 for strictly lower A [64][65] (fp32), blocked in 16 x 16.
-__device__ void invert_unit_lower(const float* A, float* T, float* Xb, int tid) {
-    // diagonal blocks: one thread per (block, column), forward substitution
+// T = (I + A)^-1 for strictly lower A [64][65] (fp32) by recursive doubling:
+// invert the four 16 x 16 diagonal blocks by forward substitution (one thread
+// per column, the column held in registers), then merge pairs with
+//   [[T11, 0], [X, T22]],  X = -T22 A21 T11
+// at 16 -> 32 and 32 -> 64. Every loop has a constant trip count and several
+// independent accumulators, so the shared-memory loads pipeline. Xs holds
+// 1024 floats of scratch.
+__device__ __forceinline__ void invert_unit_lower(const float* A, float* T, float* Xs, int tid) {
     if (tid < 64) {
-        const int blk = tid >> 4, col = tid;                  // global column
-        const int r0 = blk * 16;
-        for (int r = r0; r < r0 + 16; ++r) {
-            float x = (r == col) ? 1.f : 0.f;
-            if (r > col)
-                for (int i = col; i < r; ++i) x -= A[r * 65 + i] * T[i * 65 + col];
-            T[r * 65 + col] = x;
+        const int c = tid, j = c >> 4, cl = c & 15;
+        const float* Ab = A + (j * 16) * 65 + j * 16;
+        float t[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float x = (r == cl) ? 1.f : 0.f;
+#pragma unroll
+            for (int i = 0; i < r; ++i) x -= Ab[r * 65 + i] * t[i];
+            t[r] = x;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) T[(j * 16 + r) * 65 + c] = t[r];
+    } else {
+        // zero the strictly upper off-diagonal blocks: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+        for (int e = tid - 64; e < 6 * 256; e += 64) {
+            const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+            const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            T[(bi * 16 + rr) * 65 + bj * 16 + cc] = 0.f;
         }
     }
     __syncthreads();
-    // off-diagonal blocks by distance d: T_ij = -T_ii (sum_{k=j}^{i-1} A_ik T_kj)
-    for (int d = 1; d < 4; ++d) {
-        const int nent = (4 - d) * 256;
-        for (int e = tid; e < nent; e += THREADS) {
-            const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            const int bj = bi, bI = bi + d;
-            const int row = bI * 16 + rr, col = bj * 16 + cc;
-            float x = 0.f;
-            for (int k = bj * 16; k < bI * 16; ++k) x += A[row * 65 + k] * T[k * 65 + col];
-            Xb[e] = x;
+    // 16 -> 32: pairs (b1, b0) = (1, 0) and (3, 2); thread: column c, rows rg*4 .. rg*4+3
+    const int pr = tid >> 6, c16 = tid & 15, rg = (tid >> 4) & 3;
+    const int b0 = pr * 2, b1 = b0 + 1;
+    {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float tv = T[(b0 * 16 + k) * 65 + b0 * 16 + c16];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) acc[m] += A[(b1 * 16 + rg * 4 + m) * 65 + b0 * 16 + k] * tv;
         }
-        __syncthreads();
-        for (int e = tid; e < nent; e += THREADS) {
-            const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            const int bI = bi + d;
-            const int row = bI * 16 + rr, col = bi * 16 + cc;
-            float x = 0.f;
-            for (int m = 0; m <= rr; ++m) x += T[row * 65 + bI * 16 + m] * Xb[(bi << 8) + (m << 4) + cc];
-            T[row * 65 + col] = -x;
-        }
-        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < 4; ++m) Xs[pr * 256 + (rg * 4 + m) * 16 + c16] = acc[m];
     }
+    __syncthreads();
+    {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float xv = Xs[pr * 256 + k * 16 + c16];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) acc[m] += T[(b1 * 16 + rg * 4 + m) * 65 + b1 * 16 + k] * xv;
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) T[(b1 * 16 + rg * 4 + m) * 65 + b0 * 16 + c16] = -acc[m];
+    }
+    __syncthreads();
+    // 32 -> 64: thread: column c, rows rb .. rb+7 of the lower-left 32 x 32 block
+    const int c32 = tid & 31, rb = (tid >> 5) * 8;
+    {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float tv = T[k * 65 + c32];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc[m] += A[(32 + rb + m) * 65 + k] * tv;
+        }
+#pragma unroll
+        for (int m = 0; m < 8; ++m) Xs[(rb + m) * 32 + c32] = acc[m];
+    }
+    __syncthreads();
+    {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float xv = Xs[k * 32 + c32];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc[m] += T[(32 + rb + m) * 65 + 32 + k] * xv;
+        }
+#pragma unroll
+        for (int m = 0; m < 8; ++m) T[(32 + rb + m) * 65 + c32] = -acc[m];
+    }
+    __syncthreads();
 }
 
 template <int DK>
@@ -252,13 +304,13 @@ gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 if (l >= o2) run += y;
             }
             const float excl = run - a1;
-            V.G[2 * l] = excl + a0;
-            V.G[2 * l + 1] = run;
+            V.G[2 * l] = (excl + a0) * LOG2E;
+            V.G[2 * l + 1] = run * LOG2E;
         }
         __syncthreads();
         if (tid < C) {
-            V.gam[tid] = expf(V.G[tid]);
-            V.dcy[tid] = tid < L ? expf(V.G[L - 1] - V.G[tid]) : 0.f;
+            V.gam[tid] = exp2f(V.G[tid]);
+            V.dcy[tid] = tid < L ? exp2f(V.G[L - 1] - V.G[tid]) : 0.f;
         }
         ok = __syncthreads_and(ok);
         if (!ok) break;
@@ -288,14 +340,15 @@ gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const float Gr = V.G[r];
             if (tid < 64) {
                 const float sc = V.bet[r] * V.ik[r];
+#pragma unroll
                 for (int i = 0; i < 64; ++i)
-                    AF[r * 65 + i] = i < r ? sc * expf(Gr - V.G[i]) * __uint_as_float(x[i]) * V.ik[i] : 0.f;
+                    AF[r * 65 + i] = i < r ? sc * exp2f(Gr - V.G[i]) * __uint_as_float(x[i]) * V.ik[i] : 0.f;
             } else {
                 const float sc = V.iq[r];
                 float p[64];
 #pragma unroll
                 for (int i = 0; i < 64; ++i)
-                    p[i] = i <= r ? sc * expf(Gr - V.G[i]) * __uint_as_float(x[i]) * V.ik[i] : 0.f;
+                    p[i] = i <= r ? sc * exp2f(Gr - V.G[i]) * __uint_as_float(x[i]) * V.ik[i] : 0.f;
                 st_row64(sm + OFF_P, r, p);
             }
         }
@@ -434,11 +487,11 @@ gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         ok = mbar_wait(mbar, mma_par);
         mma_par ^= 1u;
         tc_fence_after();
-        // ---- E6: o_r = gam_r/|q_r| X2[:, r] + X3[:, r]
+        // ---- E6: o_r = gam_r/|q_r| X2[:, r] + X3[:, r], staged as a [64 token][128 channel]
+        // bf16 tile, then written with 16-byte coalesced stores
         {
+            __nv_bfloat16* ot = reinterpret_cast<__nv_bfloat16*>(sm + OFF_AW);
             uint32_t x2[32], x3[32];
-            __nv_bfloat16* orow = o + ((long long)b * Tn + t0) * H * dv + h * dv + c0 + tid;
-            const long long tstride = (long long)H * dv;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 tmem_ld32(tb + lane_base + TM_X2 + half * 32, x2);
@@ -447,10 +500,19 @@ gdn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int r = half * 32 + j;
-                    if (r < L)
-                        orow[r * tstride] = __float2bfloat16_rn(V.gam[r] * V.iq[r] * __uint_as_float(x2[j]) +
-                                                                __uint_as_float(x3[j]));
+                    ot[r * ROWS + tid] = __float2bfloat16_rn(V.gam[r] * V.iq[r] * __uint_as_float(x2[j]) +
+                                                             __uint_as_float(x3[j]));
                 }
+            }
+            __syncthreads();
+            const long long tstride = (long long)H * dv;
+            __nv_bfloat16* obase = o + ((long long)b * Tn + t0) * tstride + (long long)h * dv + c0;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int q = tid + m * THREADS, r = q >> 4, ch = q & 15;
+                if (r < L)
+                    *reinterpret_cast<uint4*>(obase + r * tstride + ch * 8) =
+                        *reinterpret_cast<const uint4*>(ot + r * ROWS + ch * 8);
             }
         }
         tc_fence_before();
