@@ -12,7 +12,7 @@
 #include "k_decode.cuh"
 #include "k_genconv.cuh"
 #include "k_prefill_simt.cuh"
-#include "k_prefill_tc.cuh"
+#include "k_prefill_ws.cuh"
 
 using namespace jet;
 
@@ -156,10 +156,10 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
     const long long rows = (long long)B * Tn;
     if (!tile_map(&mq, q, DK, H, rows) || !tile_map(&mk, k, DK, H, rows) || !tile_map(&mv, v, dv, H, rows))
         return JET_ERR_CUDA;
-    auto kern = pftc::gdn_prefill_tc_kernel<DK>;
-    if (smem_attr(kern, pftc::SMEM_BYTES) != JET_OK) return JET_ERR_CUDA;
-    dim3 grid(dv / pftc::ROWS, H, B);
-    kern<<<grid, pftc::THREADS, pftc::SMEM_BYTES, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv);
+    auto kern = pfws::gdn_prefill_ws_kernel<DK>;
+    if (smem_attr(kern, pfws::SMEM_BYTES) != JET_OK) return JET_ERR_CUDA;
+    dim3 grid(dv / pfws::ROWS, H, B);
+    kern<<<grid, pfws::THREADS, pfws::SMEM_BYTES, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return launch_status();
 }
@@ -258,7 +258,7 @@ jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const fl
     if (need > 0 && (!workspace || ws_bytes < need)) return JET_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dt == JET_BF16 && dv % pftc::ROWS == 0 && (long long)B * T < (1LL << 31)) {
-        // tensor-core path: bf16, 128-row state slices, dk in {64, 96, 128}
+        // tensor-core path (warp-specialised): bf16, 128-row state slices, dk in {64, 96, 128}
         if (dk == 64) return launch_prefill_tc<64>(q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
         if (dk == 96) return launch_prefill_tc<96>(q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
         if (dk == 128) return launch_prefill_tc<128>(q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
