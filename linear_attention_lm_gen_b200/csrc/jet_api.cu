@@ -257,7 +257,7 @@ jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const fl
     const size_t need = jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk, dt);
     if (need > 0 && (!workspace || ws_bytes < need)) return JET_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dt == JET_BF16 && dv % pftc::ROWS == 0 && (long long)B * T < (1LL << 31)) {
+    if (dt == JET_BF16 && dv % pfws::ROWS == 0 && (long long)B * T < (1LL << 31)) {
         // tensor-core path (warp-specialised): bf16, 128-row state slices, dk in {64, 96, 128}
         if (dk == 64) return launch_prefill_tc<64>(q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
         if (dk == 96) return launch_prefill_tc<96>(q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
