@@ -11,16 +11,19 @@
 //
 // Mapping: 4 lanes per row, each lane holding dk/16 float4 of the row in an
 // interleaved pattern (lane p reads float4 p, p+4, ...): every load
-// instruction of a warp covers 8 rows x 64 contiguous bytes. 256 threads =
-// 64 rows per CTA; grid (ceil(dv/64), H, B). State loads and stores use the
-// streaming cache policy (the state is touched once per step).
+// instruction of a warp covers 8 rows x 64 contiguous bytes. A thread owns
+// two rows (r and r + 64), so a CTA of 256 threads covers 128 rows; grid
+// (ceil(dv/128), H, B). The state loads are issued first, before the q / k
+// normalisation prologue, so they are in flight while it runs; k^ and q^ are
+// read from shared memory. State loads and stores use the streaming cache
+// policy (the state is touched once per step).
 #pragma once
 #include "common.cuh"
 
 namespace jet {
 
 constexpr int DEC_THREADS = 256;
-constexpr int DEC_ROWS = 64;    // rows of S per CTA
+constexpr int DEC_ROWS = 128;    // rows of S per CTA (two per 4-lane group)
 
 template <typename T, int NV>   // NV = dk / 16 float4 per lane
 __global__ void __launch_bounds__(DEC_THREADS)
@@ -28,11 +31,32 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
                   const float* __restrict__ g, const float* __restrict__ beta,
                   float* __restrict__ S, T* __restrict__ o, int H, int dv) {
     constexpr int DK = NV * 16;
-    __shared__ float sk[DK], sq[DK];
+    __shared__ __align__(16) float sk[DK];
+    __shared__ __align__(16) float sq[DK];
     __shared__ float red[3];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.y, b = blockIdx.z;
     const long long bh = (long long)b * H + h;
+    const int part = lane & 3;
+    const int row0 = blockIdx.x * DEC_ROWS + warp * 8 + (lane >> 2);
+    const int row1 = row0 + 64;
+    const bool ok0 = row0 < dv, ok1 = row1 < dv;
+
+    // state rows first: the loads overlap the prologue below
+    float4 s0[NV], s1[NV];
+    {
+        const float4* r0 = reinterpret_cast<const float4*>(S + (bh * dv + (ok0 ? row0 : 0)) * DK);
+        const float4* r1 = reinterpret_cast<const float4*>(S + (bh * dv + (ok1 ? row1 : 0)) * DK);
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            s0[i] = ok0 ? ld_stream_f4(r0 + part + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            s1[i] = ok1 ? ld_stream_f4(r1 + part + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    const float vi0 = ok0 ? Elem<T>::ld(v + bh * dv + row0) : 0.f;
+    const float vi1 = ok1 ? Elem<T>::ld(v + bh * dv + row1) : 0.f;
+    const float a = expf(g[bh]);
+    const float bt = beta[bh];
 
     for (int j = tid; j < DK; j += DEC_THREADS) {
         sk[j] = Elem<T>::ld(k + bh * DK + j);
@@ -50,47 +74,50 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     const float inv_k = 1.0f / sqrtf(red[0] + 1e-6f);
     const float inv_q = 1.0f / sqrtf(red[1] + 1e-6f);
     const float kq = red[2] * inv_k * inv_q;          // k^ . q^
-    const float a = expf(g[bh]);
-    const float bt = beta[bh];
 
-    const int part = lane & 3;
-    const int row = blockIdx.x * DEC_ROWS + warp * 8 + (lane >> 2);
-    if (row >= dv) return;
-
-    float4 kf[NV], qf[NV], s[NV];
-    const float4* Srow = reinterpret_cast<const float4*>(S + (bh * dv + row) * DK);
-#pragma unroll
-    for (int i = 0; i < NV; ++i) s[i] = ld_stream_f4(Srow + part + 4 * i);
+    // dot products of both rows with the raw k and q (normalised afterwards)
+    float u0 = 0.f, p0 = 0.f, u1 = 0.f, p1 = 0.f;
+    const float4* k4 = reinterpret_cast<const float4*>(sk);
+    const float4* q4 = reinterpret_cast<const float4*>(sq);
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-        const int j = 4 * (part + 4 * i);
-        kf[i] = make_float4(sk[j] * inv_k, sk[j + 1] * inv_k, sk[j + 2] * inv_k, sk[j + 3] * inv_k);
-        qf[i] = make_float4(sq[j] * inv_q, sq[j + 1] * inv_q, sq[j + 2] * inv_q, sq[j + 3] * inv_q);
+        const float4 kf = k4[part + 4 * i], qf = q4[part + 4 * i];
+        u0 += s0[i].x * kf.x + s0[i].y * kf.y + s0[i].z * kf.z + s0[i].w * kf.w;
+        p0 += s0[i].x * qf.x + s0[i].y * qf.y + s0[i].z * qf.z + s0[i].w * qf.w;
+        u1 += s1[i].x * kf.x + s1[i].y * kf.y + s1[i].z * kf.z + s1[i].w * kf.w;
+        p1 += s1[i].x * qf.x + s1[i].y * qf.y + s1[i].z * qf.z + s1[i].w * qf.w;
     }
-    float u = 0.f, p = 0.f;
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        u += s[i].x * kf[i].x + s[i].y * kf[i].y + s[i].z * kf[i].z + s[i].w * kf[i].w;
-        p += s[i].x * qf[i].x + s[i].y * qf[i].y + s[i].z * qf[i].z + s[i].w * qf[i].w;
+    for (int m = 1; m <= 2; m <<= 1) {
+        u0 += __shfl_xor_sync(0xffffffffu, u0, m);
+        p0 += __shfl_xor_sync(0xffffffffu, p0, m);
+        u1 += __shfl_xor_sync(0xffffffffu, u1, m);
+        p1 += __shfl_xor_sync(0xffffffffu, p1, m);
     }
-    u += __shfl_xor_sync(0xffffffffu, u, 1);
-    u += __shfl_xor_sync(0xffffffffu, u, 2);
-    p += __shfl_xor_sync(0xffffffffu, p, 1);
-    p += __shfl_xor_sync(0xffffffffu, p, 2);
-
-    const float vi = Elem<T>::ld(v + bh * dv + row);
-    const float c = bt * vi - a * bt * u;
-    float4* Sw = reinterpret_cast<float4*>(S + (bh * dv + row) * DK);
+    u0 *= inv_k; u1 *= inv_k; p0 *= inv_q; p1 *= inv_q;
+    const float c0 = bt * vi0 - a * bt * u0;
+    const float c1 = bt * vi1 - a * bt * u1;
+    const float ck0 = c0 * inv_k, ck1 = c1 * inv_k;   // c k^ = (c / |k|) k
+    if (ok0) {
+        float4* w = reinterpret_cast<float4*>(S + (bh * dv + row0) * DK);
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        float4 r;
-        r.x = a * s[i].x + c * kf[i].x;
-        r.y = a * s[i].y + c * kf[i].y;
-        r.z = a * s[i].z + c * kf[i].z;
-        r.w = a * s[i].w + c * kf[i].w;
-        st_stream_f4(Sw + part + 4 * i, r);
+        for (int i = 0; i < NV; ++i) {
+            const float4 kf = k4[part + 4 * i];
+            st_stream_f4(w + part + 4 * i, make_float4(a * s0[i].x + ck0 * kf.x, a * s0[i].y + ck0 * kf.y,
+                                                       a * s0[i].z + ck0 * kf.z, a * s0[i].w + ck0 * kf.w));
+        }
+        if (part == 0) Elem<T>::st(o + bh * dv + row0, a * p0 + c0 * kq);
     }
-    if (part == 0) Elem<T>::st(o + bh * dv + row, a * p + c * kq);
+    if (ok1) {
+        float4* w = reinterpret_cast<float4*>(S + (bh * dv + row1) * DK);
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const float4 kf = k4[part + 4 * i];
+            st_stream_f4(w + part + 4 * i, make_float4(a * s1[i].x + ck1 * kf.x, a * s1[i].y + ck1 * kf.y,
+                                                       a * s1[i].z + ck1 * kf.z, a * s1[i].w + ck1 * kf.w));
+        }
+        if (part == 0) Elem<T>::st(o + bh * dv + row1, a * p1 + c1 * kq);
+    }
 }
 
 }  // namespace jet
