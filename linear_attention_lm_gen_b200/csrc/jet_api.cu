@@ -13,6 +13,7 @@
 #include "k_genconv.cuh"
 #include "k_prefill_simt.cuh"
 #include "k_prefill_ws.cuh"
+#include "k_segcombine.cuh"
 
 using namespace jet;
 
@@ -149,17 +150,77 @@ bool tile_map(CUtensorMap* m, const void* base, int d, int H, long long rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Number of segments of the sequence-parallel prefill (1 = single pass):
+// the largest P that keeps both phases within one wave of 148 SMs and every
+// segment at least 8 chunks long. A function of the shapes only, so the
+// workspace size can be queried without a device.
+constexpr int kSMs = 148;
+constexpr int kMinSegChunks = 8;
+struct SegPlan { int P, seg_chunks; };
+SegPlan plan_segments(int B, int T, int H, int dv) {
+    const int nch = (T + 63) / 64, ns = dv / pfws::ROWS;
+    SegPlan best{1, nch};
+    for (int P = 2; P <= 64; ++P) {
+        const int segc = (nch + P - 1) / P;
+        if (segc < kMinSegChunks) break;
+        const int Peff = (nch + segc - 1) / segc;
+        if (Peff != P) continue;
+        const long long ctaA = (long long)B * H * ((P - 1) * ns + (P - 2));
+        const long long ctaC = (long long)B * H * ns * P;
+        if (ctaA > kSMs || ctaC > kSMs) break;
+        best = SegPlan{P, segc};
+    }
+    return best;
+}
+bool tc_prefill_ok(jet_dtype dt, int dk, int dv, long long BT) {
+    return dt == JET_BF16 && dv % pfws::ROWS == 0 && (dk == 64 || dk == 96 || dk == 128) && BT < (1LL << 31);
+}
+size_t seg_workspace_floats(int B, int H, int dk, int dv, int P) {
+    if (P <= 1) return 0;
+    return (size_t)B * (P - 1) * H * dv * dk      // E: phase A end states
+         + (size_t)B * (P - 1) * H * dk * dk      // A: transitions
+         + (size_t)B * P * H * dv * dk;           // start states
+}
+
 template <int DK>
 jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                             const float* S0, void* o, float* S_out, int B, int Tn, int H, int dv, cudaStream_t s) {
+                             const float* S0, void* o, float* S_out, float* ws, int B, int Tn, int H, int dv,
+                             cudaStream_t s) {
     CUtensorMap mq, mk, mv;
     const long long rows = (long long)B * Tn;
     if (!tile_map(&mq, q, DK, H, rows) || !tile_map(&mk, k, DK, H, rows) || !tile_map(&mv, v, dv, H, rows))
         return JET_ERR_CUDA;
     auto kern = pfws::gdn_prefill_ws_kernel<DK>;
     if (smem_attr(kern, pfws::SMEM_BYTES) != JET_OK) return JET_ERR_CUDA;
-    dim3 grid(dv / pfws::ROWS, H, B);
-    kern<<<grid, pfws::THREADS, pfws::SMEM_BYTES, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv);
+    const int ns = dv / pfws::ROWS;
+    const SegPlan plan = plan_segments(B, Tn, H, dv);
+    const int P = plan.P;
+    if (P == 1) {
+        const pfws::Seg seg{1, plan.seg_chunks, 1, 0, nullptr, nullptr, nullptr};
+        kern<<<dim3(ns, H, B), pfws::THREADS, pfws::SMEM_BYTES, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o,
+                                                                      S_out, Tn, H, dv, seg);
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return launch_status();
+    }
+    float* E = ws;
+    float* A = E + (size_t)B * (P - 1) * H * dv * DK;
+    float* Sst = A + (size_t)B * (P - 1) * H * DK * DK;
+    // phase A: segments 0 .. P-2, value slices plus the transition slice
+    const pfws::Seg segA{P, plan.seg_chunks, P - 1, 1, nullptr, E, A};
+    kern<<<dim3(ns + 1, H, B * (P - 1)), pfws::THREADS, pfws::SMEM_BYTES, s>>>(
+        mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, segA);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (launch_status() != JET_OK) return JET_ERR_CUDA;
+    // start states of every segment (S0 copied for segment 0)
+    const size_t sc_smem = sc_smem_bytes(DK);
+    if (smem_attr(seg_combine_kernel, sc_smem) != JET_OK) return JET_ERR_CUDA;
+    seg_combine_kernel<<<dim3(dv / SC_ROWS, H, B), SC_THREADS, sc_smem, s>>>(E, A, S0, Sst, P, H, dv, DK);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (launch_status() != JET_OK) return JET_ERR_CUDA;
+    // phase C: every segment from its start state, with outputs
+    const pfws::Seg segC{P, plan.seg_chunks, P, 0, Sst, nullptr, nullptr};
+    kern<<<dim3(ns, H, B * P), pfws::THREADS, pfws::SMEM_BYTES, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o,
+                                                                      S_out, Tn, H, dv, segC);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return launch_status();
 }
@@ -240,8 +301,9 @@ jet_status jet_dyn_conv_v(const void* x, const void* w1, const void* w2, const v
 }
 
 size_t jet_gdn_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt) {
-    (void)B; (void)T; (void)H; (void)dk; (void)dv; (void)chunk; (void)dt;
-    return 0;
+    if (B <= 0 || T <= 0 || H <= 0 || chunk != 64 || !tc_prefill_ok(dt, dk, dv, (long long)B * T)) return 0;
+    const SegPlan plan = plan_segments(B, T, H, dv);
+    return sizeof(float) * seg_workspace_floats(B, H, dk, dv, plan.P);
 }
 
 jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -257,11 +319,12 @@ jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const fl
     const size_t need = jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk, dt);
     if (need > 0 && (!workspace || ws_bytes < need)) return JET_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dt == JET_BF16 && dv % pfws::ROWS == 0 && (long long)B * T < (1LL << 31)) {
-        // tensor-core path (warp-specialised): bf16, 128-row state slices, dk in {64, 96, 128}
-        if (dk == 64) return launch_prefill_tc<64>(q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
-        if (dk == 96) return launch_prefill_tc<96>(q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
-        if (dk == 128) return launch_prefill_tc<128>(q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
+    if (tc_prefill_ok(dt, dk, dv, (long long)B * T)) {
+        // tensor-core path (warp-specialised, sequence-parallel when T is long)
+        float* ws = static_cast<float*>(workspace);
+        if (dk == 64) return launch_prefill_tc<64>(q, k, v, g, beta, S0, o, S_out, ws, B, T, H, dv, s);
+        if (dk == 96) return launch_prefill_tc<96>(q, k, v, g, beta, S0, o, S_out, ws, B, T, H, dv, s);
+        return launch_prefill_tc<128>(q, k, v, g, beta, S0, o, S_out, ws, B, T, H, dv, s);
     }
     if (dt == JET_BF16)
         return dispatch_prefill<__nv_bfloat16>(dk, q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);

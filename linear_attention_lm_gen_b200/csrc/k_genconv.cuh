@@ -128,38 +128,6 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
     const long long r0 = (long long)blockIdx.x * TB;
     const int nrows = (int)((N - r0) < TB ? (N - r0) : TB);
 
-    // ---- conv work items: one 16-byte channel group of one head over a run of tokens
-    using V16 = Vec16<T>;
-    constexpr int VN = V16::N;                 // channels per 16-byte group
-    const int ngrp = dv / VN;                  // groups per head row
-    const int nruns = (nrows + RUN - 1) / RUN;
-    const int cols = nh * ngrp;
-    const int items = v ? cols * nruns : 0;
-    const long long rowstride = (long long)H * dv;   // elements per token
-    // raw loads of an item: the 3 positions before its run (window) and the run itself
-    auto load_item = [&](int it, uint4* wraw, uint4* cur) {
-        const int col = it % cols, run = it / cols;
-        const int hl = col / ngrp, cg = col % ngrp;
-        const long long coff = (long long)(h0 + hl) * dv + (long long)cg * VN;
-        const int ta = run * RUN, tb = min(nrows, ta + RUN);
-        const long long rr = r0 + ta;
-        const int bseq = (int)(rr / Tn);
-        const long long tpos = rr % Tn;
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-            const long long tau = tpos - 1 - j;
-            wraw[j] = make_uint4(0, 0, 0, 0);
-            if (tau >= 0) wraw[j] = *reinterpret_cast<const uint4*>(v + (rr - 1 - j) * rowstride + coff);
-            else if (hist_in) wraw[j] = *reinterpret_cast<const uint4*>(hist_in + ((long long)bseq * 3 + (3 + tau)) * rowstride + coff);
-        }
-#pragma unroll
-        for (int i = 0; i < RUN; ++i)
-            if (ta + i < tb) cur[i] = *reinterpret_cast<const uint4*>(v + (rr + i) * rowstride + coff);
-    };
-    // the first item's loads go out now, so they are in flight during the generator
-    uint4 wraw0[3], cur0[RUN];
-    if (tid < items) load_item(tid, wraw0, cur0);
-
     for (int i = tid; i < GC_HID * CW; i += GC_THREADS) {
         const int r = i / CW, c = i % CW;
         w2s[i] = Elem<T>::ld(W2 + (long long)r * HW4 + h0 * GC_W + c);
@@ -209,21 +177,40 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
     __syncthreads();
 
     // ---- stage C: causal conv over V ----
+    using V16 = Vec16<T>;
+    constexpr int VN = V16::N;                 // channels per 16-byte group
+    const int ngrp = dv / VN;                  // groups per head row
+    const int nruns = (nrows + RUN - 1) / RUN;
+    const int cols = nh * ngrp;
+    const int items = cols * nruns;
+    const long long rowstride = (long long)H * dv;   // elements per token
     for (int it = tid; it < items; it += GC_THREADS) {
-        uint4 wraw[3], cur[RUN];
-        if (it == tid) {
-#pragma unroll
-            for (int j = 0; j < 3; ++j) wraw[j] = wraw0[j];
-#pragma unroll
-            for (int i = 0; i < RUN; ++i) cur[i] = cur0[i];
-        } else {
-            load_item(it, wraw, cur);
-        }
-        const int col = it % cols, run = it / cols;
+        const int col = it % cols;
+        const int run = it / cols;
         const int hl = col / ngrp, cg = col % ngrp;
-        const long long coff = (long long)(h0 + hl) * dv + (long long)cg * VN;
-        const int ta = run * RUN, tb = min(nrows, ta + RUN);
+        const int h = h0 + hl;
+        const long long coff = (long long)h * dv + (long long)cg * VN;
+        const int ta = run * RUN;
+        const int tb = min(nrows, ta + RUN);
+
         // window: win[0] = v_{t-1}, win[1] = v_{t-2}, win[2] = v_{t-3}
+        uint4 wraw[3];
+        uint4 cur[RUN];
+        {
+            const long long rr = r0 + ta;
+            const int bseq = (int)(rr / Tn);
+            const long long tpos = rr % Tn;
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                const long long tau = tpos - 1 - j;
+                wraw[j] = make_uint4(0, 0, 0, 0);
+                if (tau >= 0) wraw[j] = *reinterpret_cast<const uint4*>(v + (rr - 1 - j) * rowstride + coff);
+                else if (hist_in) wraw[j] = *reinterpret_cast<const uint4*>(hist_in + ((long long)bseq * 3 + (3 + tau)) * rowstride + coff);
+            }
+#pragma unroll
+            for (int i = 0; i < RUN; ++i)
+                if (ta + i < tb) cur[i] = *reinterpret_cast<const uint4*>(v + (rr + i) * rowstride + coff);
+        }
         float win[3][VN];
 #pragma unroll
         for (int j = 0; j < 3; ++j) V16::unpack(wraw[j], win[j]);

@@ -201,12 +201,33 @@ __device__ __forceinline__ uint32_t blk_chunk(int r, int ch, uint32_t bstride) {
     return (uint32_t)(ch >> 3) * bstride + sw128_off((uint32_t)r, (uint32_t)(ch & 7) * 16u);
 }
 
+// Segment decomposition of the token axis (sequence parallelism; the
+// recurrence is affine in the state, S_end = S_start A + B, so segments can
+// run concurrently once their start states are known):
+//   phase A  every segment p < P-1 runs from a zero state (p > 0) or S0
+//            (p = 0) and writes its end state B_p; an extra 128-row slice
+//            starts from the identity with zero values and yields the
+//            segment's dk x dk transition A_p;
+//   combine  S_start(p+1) = S_start(p) A_p + B_p (seg_combine_kernel);
+//   phase C  every segment runs from its true start state and writes o; the
+//            last one writes the final state.
+// P = 1 is the plain single pass.
+struct Seg {
+    int nseg;          // P
+    int seg_chunks;    // chunks per segment (the last may be shorter)
+    int zseg;          // segments covered by this launch (blockIdx.z = b * zseg + p)
+    int phaseA;        // 1: end states and transitions, no outputs
+    const float* Sst;  // phase C start states (P > 1): [B][P][H][dv][dk]
+    float* Eo;         // phase A end states: [B][P-1][H][dv][dk]
+    float* Ao;         // phase A transitions: [B][P-1][H][dk][dk]
+};
+
 template <int DK>
 __global__ void __launch_bounds__(THREADS, 1)
 gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
                       const float* __restrict__ beta, const float* S0, __nv_bfloat16* __restrict__ o,
-                      float* S_out, int Tn, int H, int dv) {
+                      float* S_out, int Tn, int H, int dv, const Seg seg) {
     static_assert(DK % 32 == 0 && DK >= 64 && DK <= 128, "DK in {64, 96, 128}");
     constexpr int NKB = (DK + 63) / 64;
     constexpr int KSTEPS = DK / 16;
@@ -218,9 +239,16 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c0 = blockIdx.x * ROWS, h = blockIdx.y, b = blockIdx.z;
+    const int ns = dv / ROWS;
+    const int h = blockIdx.y, b = blockIdx.z / seg.zseg, p_seg = blockIdx.z % seg.zseg;
+    const bool trans = blockIdx.x == ns;                  // transition slice (phase A, p >= 1)
+    if (trans && (!seg.phaseA || p_seg == 0)) return;     // whole CTA, before any barrier
+    const int c0 = blockIdx.x * ROWS;                     // transition slice: past dv, V reads as zero
     const long long bh = (long long)b * H + h;
-    const int nch = (Tn + C - 1) / C;
+    const int tbeg = p_seg * seg.seg_chunks * C;
+    const int tend = min(Tn, tbeg + seg.seg_chunks * C);
+    const int nch = (tend - tbeg + C - 1) / C;
+    const bool write_o = !seg.phaseA;
 
     if (tid == 0) {
         for (int i = 0; i < NBARS; ++i) mbar_init(&bars[i], 1);
@@ -243,17 +271,28 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int ct = tid;
         const uint32_t lb = (uint32_t)(warp * 32) << 16;
         {   // initial state (row ct of the slice)
-            const float* src = S0 ? S0 + (bh * dv + c0 + ct) * DK : nullptr;
+            const float* src = nullptr;
+            if (!seg.phaseA && seg.nseg > 1) {
+                src = seg.Sst + ((((long long)b * seg.nseg + p_seg) * H + h) * dv + c0 + ct) * DK;
+            } else if (p_seg == 0 && !trans && S0) {
+                src = S0 + (bh * dv + c0 + ct) * DK;
+            }
 #pragma unroll
             for (int cb = 0; cb < DK / 32; ++cb) {
                 uint32_t r[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) r[j] = src ? __float_as_uint(src[cb * 32 + j]) : 0u;
+                for (int j = 0; j < 32; ++j)
+                    r[j] = trans ? (cb * 32 + j == ct ? 0x3f800000u : 0u) : (src ? __float_as_uint(src[cb * 32 + j]) : 0u);
                 tmem_st32(tb + lb + TM_S + cb * 32, r);
             }
             tmem_st_wait();
         }
         auto emit_output = [&](int cc) {   // E6 for chunk cc: X2 -> staging -> global
+            if (!write_o) {
+                named_sync(2, NCHAIN);
+                if (ct == 0) arrive(&bars[B_X2FREE + (cc & 1)]);
+                return;
+            }
             __nv_bfloat16* ot = reinterpret_cast<__nv_bfloat16*>(sm + OFF_AWD);
             const uint32_t x2 = TM_X2 + (uint32_t)(cc & 1) * 64;
 #pragma unroll
@@ -267,7 +306,7 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_before();
             named_sync(2, NCHAIN);
             if (ct == 0) arrive(&bars[B_X2FREE + (cc & 1)]);
-            const int t0 = cc * C, L = min(C, Tn - t0);
+            const int t0 = tbeg + cc * C, L = min(C, tend - t0);
             const long long tstride = (long long)H * dv;
             __nv_bfloat16* obase = o + ((long long)b * Tn + t0) * tstride + (long long)h * dv + c0;
 #pragma unroll
@@ -288,7 +327,7 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_after();
             // ---- E4: S -> bf16 copy, S <- gam_L S
             {
-                const int L = min(C, Tn - c * C);
+                const int L = min(C, tend - (tbeg + c * C));
                 const float gL = V.gam[L - 1];
 #pragma unroll
                 for (int cb = 0; cb < DK / 32; ++cb) {
@@ -354,9 +393,17 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (group_all(2, NCHAIN, fin)) {
             tc_fence_after();
             emit_output(nch - 1);
-            float* dst = S_out + (bh * dv + c0 + ct) * DK;
+            float* dst = nullptr;
+            if (seg.phaseA) {
+                const long long bp = (long long)b * (seg.nseg - 1) + p_seg;
+                if (trans) { if (ct < DK) dst = seg.Ao + ((bp * H + h) * DK + ct) * DK; }
+                else dst = seg.Eo + ((bp * H + h) * dv + c0 + ct) * DK;
+            } else if (p_seg == seg.nseg - 1) {
+                dst = S_out + (bh * dv + c0 + ct) * DK;
+            }
 #pragma unroll
             for (int cb = 0; cb < DK / 32; ++cb) {
+                if (!dst) break;
                 uint32_t x[32];
                 tmem_ld32(tb + lb + TM_S + cb * 32, x);
                 tmem_ld_wait();
@@ -380,7 +427,7 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // or beta (64 <= pt < 128), loaded one chunk ahead
         auto vec_phase = [&](int cv, float gb) -> bool {
             const int pv = cv & 1;
-            const int t0 = cv * C, L = min(C, Tn - t0);
+            const int t0 = tbeg + cv * C, L = min(C, tend - t0);
             uint8_t* KQ = sm + OFF_KQ + pv * 32768;
             Vec V = vec_at(sm, pv);
             // vec[pv] is free once E5 of chunk cv-2 has read it
@@ -432,8 +479,8 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             float v = 0.f;
             if (cv < nch && pt < 128) {
                 const int r = pt & 63;
-                if (r < min(C, Tn - cv * C)) {
-                    const long long off = ((long long)b * Tn + cv * C + r) * H + h;
+                if (r < min(C, tend - (tbeg + cv * C))) {
+                    const long long off = ((long long)b * Tn + tbeg + cv * C + r) * H + h;
                     v = pt < 64 ? g[off] : beta[off];
                 }
             }
@@ -687,7 +734,7 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         auto load_kq = [&](int c) {
             const int sb = c & 1;
             uint8_t* dst = sm + OFF_KQ + sb * 32768;
-            const int z = (int)((long long)b * Tn + (long long)c * C);
+            const int z = (int)((long long)b * Tn + tbeg + (long long)c * C);
             mbar_expect_tx(&bars[B_KFULL + sb], tx_kq);
 #pragma unroll
             for (int kb = 0; kb < NKB; ++kb) {
@@ -696,7 +743,7 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
         };
         auto load_v = [&](int c) {
-            const int z = (int)((long long)b * Tn + (long long)c * C);
+            const int z = (int)((long long)b * Tn + tbeg + (long long)c * C);
             mbar_expect_tx(&bars[B_VFULL], 16384);
             tma_load_3d(sm + OFF_V, &tm_v, &bars[B_VFULL], c0, h, z);
             tma_load_3d(sm + OFF_V + 8192, &tm_v, &bars[B_VFULL], c0 + 64, h, z);
@@ -745,6 +792,7 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 mma_bf16_ss(tb + x1, dAS + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
                             dWT + (uint64_t)(kk * 2048 >> 4), ID_NEG, 1);
             mma_commit(&bars[B_P3]);        // the chain waits for Wt^T only
+            if (!write_o) return;           // phase A: no output products
 #pragma unroll
             for (int kk = 0; kk < KSTEPS; ++kk) {
                 const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
@@ -758,9 +806,11 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ss(tb + TM_S, dAWD + (uint64_t)(kk * 32 >> 4), kmn + (uint64_t)(kk * 2048 >> 4), ID_S, 1);
+            if (write_o) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), pp + (uint64_t)(kk * 32 >> 4), ID_KK, 1);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), pp + (uint64_t)(kk * 32 >> 4), ID_KK, 1);
+            }
             mma_commit(&bars[B_SDONE + (c & 1)]);
         };
         int n1 = 0, n2 = 0, n3 = 0, n4 = 0, nK = 0, nV = 0;      // actions issued

@@ -139,6 +139,38 @@ def test_prefill_long_memory_gates(orc, dtype, dk):
     assert_close(host64(S_out), rS, dtype, "S")
 
 
+@pytest.mark.parametrize("B,T,dk,s0,gate_scale", [(1, 1553, 96, True, 0.01), (2, 1600, 64, False, 0.01),
+                                                  (1, 4096 + 64 * 9 + 5, 128, True, 1.0)])
+def test_prefill_sequence_parallel_segments(orc, B, T, dk, s0, gate_scale):
+    # long enough for the segmented path (phase A, combine, phase C); long-memory
+    # gates make the carried segment states matter
+    import linear_attention_lm_gen_b200 as m
+    assert m.jet_gdn_prefill_workspace_size(B, T, 2, dk, 256) > 0
+    s = shape("bf16", B=B, T=T, H=2, dk=dk, dv=256, D=64)
+    inp = synth.prefill_inputs(s, seed=21, gate_scale=gate_scale, s0_std=0.2 if s0 else None)
+    d = gpu_inputs(inp)
+    ref = to_oracle(inp)
+    o = nan_like(d["v"])
+    S_out = torch.full((B, 2, 256, dk), float("nan"), device="cuda")
+    jet.jet_gdn_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d.get("S0"), o, S_out)
+    ro, rS = orc.gdn_sequential(ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"],
+                                inp["S0"].astype(np.float64) if s0 else None)
+    assert_close(host64(o), ro, "bf16", "o")
+    assert_close(host64(S_out), rS, "bf16", "S")
+
+
+def test_prefill_segments_final_state_may_alias_initial_state(orc):
+    s = shape("bf16", B=1, T=2000, H=2, dk=96, dv=256, D=64)
+    inp = synth.prefill_inputs(s, seed=22, gate_scale=0.01, s0_std=0.2)
+    d = gpu_inputs(inp)
+    ref = to_oracle(inp)
+    S = d["S0"].clone()
+    o, _ = jet.jet_gdn_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], S, None, S)
+    ro, rS = orc.gdn_sequential(ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"], inp["S0"].astype(np.float64))
+    assert_close(host64(o), ro, "bf16", "o")
+    assert_close(host64(S), rS, "bf16", "S")
+
+
 def test_prefill_state_alias_and_continuation(orc):
     # S_out may alias S0; prefill(T1) then prefill(T2) from its state = prefill(T1+T2)
     s = shape("bf16", B=2, T=200, H=2, dk=64, dv=64, D=64)
