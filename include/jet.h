@@ -60,7 +60,8 @@ typedef enum {
     JET_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
     JET_ERR_TIMEOUT = 5,       /* a bounded in-kernel wait ran out (via jet_device_error) */
     JET_ERR_DEVICE = 6,        /* a kernel flagged bad data (via jet_device_error) */
-    JET_ERR_WORKSPACE = 7      /* workspace pointer null or smaller than required */
+    JET_ERR_WORKSPACE = 7,     /* workspace pointer null or smaller than required */
+    JET_ERR_TOO_LARGE = 8      /* sizes need more scratch than jet_gdn_prefill_noalloc's fixed buffer */
 } jet_status;
 
 typedef enum { JET_F32 = 0, JET_BF16 = 1 } jet_dtype;
@@ -120,6 +121,36 @@ jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const fl
 jet_status jet_gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, float* S, void* o,
                                int B, int H, int dk, int dv, jet_dtype dt, void* stream);
+
+/*
+ * jet_gdn_prefill for callers that cannot allocate device memory. It has no
+ * counterpart in the paper; it exists for code that must not call an
+ * allocator on its hot path: work recorded into a CUDA graph (allocation is
+ * not allowed during stream capture), latency-bound serving loops where an
+ * allocation would stall or synchronise the device, and embedders that own a
+ * fixed memory budget and hand the library only their input and output
+ * buffers.
+ *
+ * Same operation, arguments and errors as jet_gdn_prefill, minus the
+ * workspace: the scratch it needs comes from one fixed array of
+ * JET_NOALLOC_SCRATCH_BYTES (16 MiB) inside the library, present on every
+ * GPU that loads the library until the process exits. Sizes that need more
+ * (jet_gdn_prefill_workspace_size > JET_NOALLOC_SCRATCH_BYTES) return
+ * JET_ERR_TOO_LARGE before anything is launched; the 2B shapes fit at any
+ * length (12.4 MB), 16-head dk = 128 shapes longer than 1792 tokens do not
+ * (17.8 MB).
+ * The first call on a device looks the array's device address up (no
+ * allocation); make that first call before any stream capture. The array is
+ * shared by all calls on a device and keeps the last call's contents (every
+ * element a call reads is written by that call first): calls whose work
+ * overlaps on the GPU, e.g. on two streams, race on it and must be ordered
+ * by the caller. Never calls cudaMalloc, cudaFree or any allocating routine.
+ */
+#define JET_NOALLOC_SCRATCH_BYTES (16u << 20)
+jet_status jet_gdn_prefill_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const float* S0, void* o, float* S_out,
+                                   int B, int T, int H, int dk, int dv, int chunk,
+                                   jet_dtype dt, void* stream);
 
 /*
  * Synchronises `stream`, then returns and clears the current device's error

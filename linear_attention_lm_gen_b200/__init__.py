@@ -7,8 +7,8 @@ no CUDA device is present, the calls raise.
 
 Function names match the C entry points:
   jet_kernel_gen, jet_dyn_conv_v, jet_gdn_prefill_workspace_size,
-  jet_gdn_prefill, jet_gdn_decode_step, jet_device_error, jet_status_string,
-  jet_launch_count.
+  jet_gdn_prefill, jet_gdn_prefill_noalloc, jet_gdn_decode_step,
+  jet_device_error, jet_status_string, jet_launch_count.
 """
 from __future__ import annotations
 
@@ -22,9 +22,12 @@ LIB_PATH = os.path.join(PKG, "libjet.so")
 
 JET_F32, JET_BF16 = 0, 1
 STATUS = {0: "JET_OK", 1: "JET_ERR_INVALID_ARG", 2: "JET_ERR_UNSUPPORTED", 3: "JET_ERR_MISALIGNED",
-          4: "JET_ERR_CUDA", 5: "JET_ERR_TIMEOUT", 6: "JET_ERR_DEVICE", 7: "JET_ERR_WORKSPACE"}
+          4: "JET_ERR_CUDA", 5: "JET_ERR_TIMEOUT", 6: "JET_ERR_DEVICE", 7: "JET_ERR_WORKSPACE",
+          8: "JET_ERR_TOO_LARGE"}
 EXPORTS = ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill_workspace_size", "jet_gdn_prefill",
-           "jet_gdn_decode_step", "jet_device_error", "jet_status_string", "jet_launch_count")
+           "jet_gdn_prefill_noalloc", "jet_gdn_decode_step", "jet_device_error", "jet_status_string",
+           "jet_launch_count")
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class JetError(RuntimeError):
@@ -50,13 +53,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.jet_gdn_prefill_workspace_size.argtypes = [I] * 7
     L.jet_gdn_prefill_workspace_size.restype = Z
     L.jet_gdn_prefill.argtypes = [P] * 9 + [Z] + [I] * 7 + [P]
+    L.jet_gdn_prefill_noalloc.argtypes = [P] * 8 + [I] * 7 + [P]
     L.jet_gdn_decode_step.argtypes = [P] * 7 + [I] * 5 + [P]
     L.jet_device_error.argtypes = [P]
     L.jet_status_string.argtypes = [I]
     L.jet_status_string.restype = ctypes.c_char_p
     L.jet_launch_count.argtypes = []
     L.jet_launch_count.restype = U
-    for f in ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill", "jet_gdn_decode_step", "jet_device_error"):
+    for f in ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill", "jet_gdn_prefill_noalloc",
+              "jet_gdn_decode_step", "jet_device_error"):
         getattr(L, f).restype = I
     _lib = L
     return L
@@ -156,6 +161,23 @@ def jet_gdn_prefill(q, k, v, g, beta, S0=None, o=None, S_out=None, workspace=Non
                            _ptr(S_out, "S_out", torch.float32, (B, H, dv, dk)), _ptr(workspace, "workspace"),
                            ws_bytes, B, T, H, dk, dv, 64, dt, _stream(stream))
     _check("jet_gdn_prefill", st)
+    return o, S_out
+
+
+def jet_gdn_prefill_noalloc(q, k, v, g, beta, S0, o, S_out, *, stream=None):
+    """jet_gdn_prefill without a workspace argument, for callers that cannot
+    allocate: the library uses its own fixed scratch array (16 MiB per GPU).
+    o and S_out must be given (nothing is allocated here either). Calls whose
+    work overlaps on the GPU share that array and must be ordered by the caller."""
+    L = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    st = L.jet_gdn_prefill_noalloc(_ptr(q, "q"), _ptr(k, "k", q.dtype, q.shape), _ptr(v, "v", q.dtype, (B, T, H, dv)),
+                                   _ptr(g, "g", torch.float32, (B, T, H)), _ptr(beta, "beta", torch.float32, (B, T, H)),
+                                   _ptr(S0, "S0", torch.float32, (B, H, dv, dk)), _ptr(o, "o", q.dtype, (B, T, H, dv)),
+                                   _ptr(S_out, "S_out", torch.float32, (B, H, dv, dk)),
+                                   B, T, H, dk, dv, 64, _dt(q), _stream(stream))
+    _check("jet_gdn_prefill_noalloc", st)
     return o, S_out
 
 

@@ -7,6 +7,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "k_decode.cuh"
@@ -367,6 +368,7 @@ const char* jet_status_string(jet_status s) {
         case JET_ERR_TIMEOUT: return "JET_ERR_TIMEOUT";
         case JET_ERR_DEVICE: return "JET_ERR_DEVICE";
         case JET_ERR_WORKSPACE: return "JET_ERR_WORKSPACE";
+        case JET_ERR_TOO_LARGE: return "JET_ERR_TOO_LARGE";
     }
     return "JET_ERR_UNKNOWN";
 }
@@ -374,3 +376,48 @@ const char* jet_status_string(jet_status s) {
 uint64_t jet_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- prefill without a caller workspace
+// Scratch for jet_gdn_prefill_noalloc: one fixed device array per GPU that
+// loads this library (held until the process exits). Host code cannot use
+// the array's name as a device address; the address is looked up per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[JET_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// device address of the scratch array on the current device (looked up once)
+jet_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return JET_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return JET_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return JET_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return JET_OK;
+}
+}  // namespace
+
+extern "C" jet_status jet_gdn_prefill_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                              const float* beta, const float* S0, void* o, float* S_out, int B,
+                                              int T, int H, int dk, int dv, int chunk, jet_dtype dt, void* stream) {
+    // same argument checks as jet_gdn_prefill, before anything else
+    if (!q || !k || !v || !g || !beta || !o || !S_out) return JET_ERR_INVALID_ARG;
+    if (!dtype_ok(dt)) return JET_ERR_INVALID_ARG;
+    if (elems({B, T, H, dk}) < 0 || elems({B, T, H, dv}) < 0 || elems({B, H, dv, dk}) < 0) return JET_ERR_INVALID_ARG;
+    if (!shape_ok(dk, dv) || chunk != 64 || B > 65535 || H > 65535) return JET_ERR_UNSUPPORTED;
+    const size_t need = jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk, dt);
+    if (need > (size_t)JET_NOALLOC_SCRATCH_BYTES) return JET_ERR_TOO_LARGE;
+    void* ws = nullptr;
+    if (need > 0) {
+        const jet_status st = noalloc_scratch(&ws);
+        if (st != JET_OK) return st;
+    }
+    return jet_gdn_prefill(q, k, v, g, beta, S0, o, S_out, ws, need, B, T, H, dk, dv, chunk, dt, stream);
+}
