@@ -214,8 +214,8 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
     if (launch_status() != JET_OK) return JET_ERR_CUDA;
     // start states of every segment (S0 copied for segment 0)
     const size_t sc_smem = sc_smem_bytes(DK);
-    if (smem_attr(seg_combine_kernel, sc_smem) != JET_OK) return JET_ERR_CUDA;
-    seg_combine_kernel<<<dim3(dv / SC_ROWS, H, B), SC_THREADS, sc_smem, s>>>(E, A, S0, Sst, P, H, dv, DK);
+    if (smem_attr(seg_combine_kernel<DK>, sc_smem) != JET_OK) return JET_ERR_CUDA;
+    seg_combine_kernel<DK><<<dim3(dv / SC_ROWS, H, B), sc_threads(DK), sc_smem, s>>>(E, A, S0, Sst, P, H, dv);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     if (launch_status() != JET_OK) return JET_ERR_CUDA;
     // phase C: every segment from its start state, with outputs
