@@ -91,9 +91,18 @@ jet_status jet_dyn_conv_v(const void* x, const void* w1, const void* w2, const v
                           jet_dtype dt, void* stream);
 
 /*
- * Bytes of device workspace jet_gdn_prefill needs for these sizes (may be 0).
+ * Device workspace of jet_gdn_prefill for these sizes, in bytes (either may
+ * be 0). With at least jet_gdn_prefill_workspace_size bytes the prefill runs
+ * its fastest plan: every chunk's state-independent part is prepared at once
+ * into per-chunk tiles (about 45 KB per chunk of 64 tokens and head at
+ * dk = 96, so this grows with B * T * H), then the state chain runs. With
+ * at least jet_gdn_prefill_workspace_min bytes (the sequence-parallel
+ * segment buffers only, at most a few tens of MB and independent of T beyond
+ * a few thousand tokens) it runs a plan that prepares each chunk inside the
+ * chain kernel; the results agree within the bf16 tolerance, not bit for bit.
  */
 size_t jet_gdn_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt);
+size_t jet_gdn_prefill_workspace_min(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt);
 
 /*
  * Gated DeltaNet prefill over T tokens per sequence (step 3; paper section
@@ -102,8 +111,9 @@ size_t jet_gdn_prefill_workspace_size(int B, int T, int H, int dk, int dv, int c
  *   q, k [B,T,H,dk]; v [B,T,H,dv] (normally v' from jet_dyn_conv_v); g, beta [B,T,H] float32.
  *   S0 [B,H,dv,dk] float32 or NULL (zeros). o [B,T,H,dv] out.
  *   S_out [B,H,dv,dk] float32 out: the state after token T-1; may alias S0.
- *   workspace / ws_bytes: at least jet_gdn_prefill_workspace_size(...) bytes
- *   (may be NULL when that is 0). Contents on entry are ignored.
+ *   workspace / ws_bytes: at least jet_gdn_prefill_workspace_min(...) bytes,
+ *   jet_gdn_prefill_workspace_size(...) for the fastest plan (may be NULL
+ *   when the minimum is 0). Contents on entry are ignored.
  * A prefill can be continued: pass its S_out as the next call's S0.
  */
 jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const float* g,
@@ -134,9 +144,10 @@ jet_status jet_gdn_decode_step(const void* q, const void* k, const void* v, cons
  * Same operation, arguments and errors as jet_gdn_prefill, minus the
  * workspace: the scratch it needs comes from one fixed array of
  * JET_NOALLOC_SCRATCH_BYTES (16 MiB) inside the library, present on every
- * GPU that loads the library until the process exits. Sizes that need more
- * (jet_gdn_prefill_workspace_size > JET_NOALLOC_SCRATCH_BYTES) return
- * JET_ERR_TOO_LARGE before anything is launched; the 2B shapes fit at any
+ * GPU that loads the library until the process exits. The fastest plan
+ * whose scratch fits is used; sizes whose smallest plan needs more
+ * (jet_gdn_prefill_workspace_min > JET_NOALLOC_SCRATCH_BYTES) return
+ * JET_ERR_TOO_LARGE before anything is launched: the 2B shapes fit at any
  * length (12.4 MB), 16-head dk = 128 shapes longer than 1792 tokens do not
  * (17.8 MB).
  * The first call on a device looks the array's device address up (no

@@ -7,7 +7,7 @@ no CUDA device is present, the calls raise.
 
 Function names match the C entry points:
   jet_kernel_gen, jet_dyn_conv_v, jet_gdn_prefill_workspace_size,
-  jet_gdn_prefill, jet_gdn_prefill_noalloc, jet_gdn_decode_step,
+  jet_gdn_prefill_workspace_min, jet_gdn_prefill, jet_gdn_prefill_noalloc, jet_gdn_decode_step,
   jet_device_error, jet_status_string, jet_launch_count.
 """
 from __future__ import annotations
@@ -24,7 +24,8 @@ JET_F32, JET_BF16 = 0, 1
 STATUS = {0: "JET_OK", 1: "JET_ERR_INVALID_ARG", 2: "JET_ERR_UNSUPPORTED", 3: "JET_ERR_MISALIGNED",
           4: "JET_ERR_CUDA", 5: "JET_ERR_TIMEOUT", 6: "JET_ERR_DEVICE", 7: "JET_ERR_WORKSPACE",
           8: "JET_ERR_TOO_LARGE"}
-EXPORTS = ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill_workspace_size", "jet_gdn_prefill",
+EXPORTS = ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill_workspace_size", "jet_gdn_prefill_workspace_min",
+           "jet_gdn_prefill",
            "jet_gdn_prefill_noalloc", "jet_gdn_decode_step", "jet_device_error", "jet_status_string",
            "jet_launch_count")
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -52,6 +53,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.jet_dyn_conv_v.argtypes = [P] * 8 + [I] * 8 + [P]
     L.jet_gdn_prefill_workspace_size.argtypes = [I] * 7
     L.jet_gdn_prefill_workspace_size.restype = Z
+    L.jet_gdn_prefill_workspace_min.argtypes = [I] * 7
+    L.jet_gdn_prefill_workspace_min.restype = Z
     L.jet_gdn_prefill.argtypes = [P] * 9 + [Z] + [I] * 7 + [P]
     L.jet_gdn_prefill_noalloc.argtypes = [P] * 8 + [I] * 7 + [P]
     L.jet_gdn_decode_step.argtypes = [P] * 7 + [I] * 5 + [P]
@@ -135,9 +138,17 @@ def jet_dyn_conv_v(x, W1, W2, v, hist_in=None, v_out=None, hist_out=None, conv_w
 
 
 def jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
+    """Workspace bytes of the fastest prefill plan (chunk images + segment buffers)."""
     L = load_library()
     return int(L.jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk,
                                                 JET_BF16 if dtype == torch.bfloat16 else JET_F32))
+
+
+def jet_gdn_prefill_workspace_min(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
+    """Smallest workspace jet_gdn_prefill accepts (segment buffers only)."""
+    L = load_library()
+    return int(L.jet_gdn_prefill_workspace_min(B, T, H, dk, dv, chunk,
+                                               JET_BF16 if dtype == torch.bfloat16 else JET_F32))
 
 
 def jet_gdn_prefill(q, k, v, g, beta, S0=None, o=None, S_out=None, workspace=None, *, stream=None):

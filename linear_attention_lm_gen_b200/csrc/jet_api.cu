@@ -13,6 +13,7 @@
 #include "k_decode.cuh"
 #include "k_genconv.cuh"
 #include "k_prefill_simt.cuh"
+#include "k_prefill_chain.cuh"
 #include "k_prefill_ws.cuh"
 #include "k_segcombine.cuh"
 
@@ -183,35 +184,63 @@ size_t seg_workspace_floats(int B, int H, int dk, int dv, int P) {
          + (size_t)B * P * H * dv * dk;           // start states
 }
 
-template <int DK>
+// per-chunk image of the two-kernel plan (preparation + chain), bytes
+size_t img_chunk_bytes(int dk) {
+    switch (dk) {
+        case 64: return pfws::Img<64>::BYTES;
+        case 96: return pfws::Img<96>::BYTES;
+        default: return pfws::Img<128>::BYTES;
+    }
+}
+size_t split_img_bytes(int B, int T, int H, int dk) {
+    return (size_t)B * H * ((T + pfws::C - 1) / pfws::C) * img_chunk_bytes(dk);
+}
+
+// Tensor-core prefill. SPLIT: K2a prepares every chunk into an image, then
+// the chain kernel K2b runs (workspace = images + segment buffers); otherwise
+// the fused kernel prepares chunk c+1 while it runs chunk c (workspace =
+// segment buffers only). Sequence-parallel segments as planned above.
+template <int DK, bool SPLIT>
 jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                             const float* S0, void* o, float* S_out, float* ws, int B, int Tn, int H, int dv,
-                             cudaStream_t s) {
+                             const float* S0, void* o, float* S_out, void* workspace, int B, int Tn, int H,
+                             int dv, cudaStream_t s) {
     CUtensorMap mq, mk, mv;
     const long long rows = (long long)B * Tn;
     if (!tile_map(&mq, q, DK, H, rows) || !tile_map(&mk, k, DK, H, rows) || !tile_map(&mv, v, dv, H, rows))
         return JET_ERR_CUDA;
-    auto kern = pfws::gdn_prefill_ws_kernel<DK>;
-    if (smem_attr(kern, pfws::SMEM_BYTES) != JET_OK) return JET_ERR_CUDA;
+    auto fused = pfws::gdn_prefill_ws_kernel<DK>;
+    auto chain = pfch::gdn_prefill_chain_kernel<DK>;
+    const uint32_t smem = SPLIT ? pfch::ChainSmem<DK>::BYTES : pfws::SMEM_BYTES;
+    const int threads = SPLIT ? pfch::THREADS : pfws::THREADS;
+    if ((SPLIT ? smem_attr(chain, smem) : smem_attr(fused, smem)) != JET_OK) return JET_ERR_CUDA;
+    uint8_t* img = static_cast<uint8_t*>(workspace);
+    float* ws = reinterpret_cast<float*>(img + (SPLIT ? split_img_bytes(B, Tn, H, DK) : 0));
+    if (SPLIT) {   // K2a: every chunk of every (sequence, head)
+        auto prep = pfws::gdn_chunk_prep_kernel<DK>;
+        if (smem_attr(prep, pfws::PrepSmem<DK>::BYTES) != JET_OK) return JET_ERR_CUDA;
+        prep<<<dim3((Tn + pfws::C - 1) / pfws::C, H, B), pfws::PREP_THREADS, pfws::PrepSmem<DK>::BYTES, s>>>(
+            mq, mk, g, beta, img, Tn, H);
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        if (launch_status() != JET_OK) return JET_ERR_CUDA;
+    }
+    auto run = [&](dim3 grid, const pfws::Seg& seg) {
+        if (SPLIT)
+            chain<<<grid, threads, smem, s>>>(mk, mv, img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg);
+        else
+            fused<<<grid, threads, smem, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg);
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return launch_status();
+    };
     const int ns = dv / pfws::ROWS;
     const SegPlan plan = plan_segments(B, Tn, H, dv);
     const int P = plan.P;
-    if (P == 1) {
-        const pfws::Seg seg{1, plan.seg_chunks, 1, 0, nullptr, nullptr, nullptr};
-        kern<<<dim3(ns, H, B), pfws::THREADS, pfws::SMEM_BYTES, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o,
-                                                                      S_out, Tn, H, dv, seg);
-        g_launches.fetch_add(1, std::memory_order_relaxed);
-        return launch_status();
-    }
+    if (P == 1) return run(dim3(ns, H, B), pfws::Seg{1, plan.seg_chunks, 1, 0, nullptr, nullptr, nullptr});
     float* E = ws;
     float* A = E + (size_t)B * (P - 1) * H * dv * DK;
     float* Sst = A + (size_t)B * (P - 1) * H * DK * DK;
     // phase A: segments 0 .. P-2, value slices plus the transition slice
-    const pfws::Seg segA{P, plan.seg_chunks, P - 1, 1, nullptr, E, A};
-    kern<<<dim3(ns + 1, H, B * (P - 1)), pfws::THREADS, pfws::SMEM_BYTES, s>>>(
-        mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, segA);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    if (launch_status() != JET_OK) return JET_ERR_CUDA;
+    if (run(dim3(ns + 1, H, B * (P - 1)), pfws::Seg{P, plan.seg_chunks, P - 1, 1, nullptr, E, A}) != JET_OK)
+        return JET_ERR_CUDA;
     // start states of every segment (S0 copied for segment 0)
     const size_t sc_smem = sc_smem_bytes(DK);
     if (smem_attr(seg_combine_kernel<DK>, sc_smem) != JET_OK) return JET_ERR_CUDA;
@@ -219,11 +248,7 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
     g_launches.fetch_add(1, std::memory_order_relaxed);
     if (launch_status() != JET_OK) return JET_ERR_CUDA;
     // phase C: every segment from its start state, with outputs
-    const pfws::Seg segC{P, plan.seg_chunks, P, 0, Sst, nullptr, nullptr};
-    kern<<<dim3(ns, H, B * P), pfws::THREADS, pfws::SMEM_BYTES, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o,
-                                                                      S_out, Tn, H, dv, segC);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return launch_status();
+    return run(dim3(ns, H, B * P), pfws::Seg{P, plan.seg_chunks, P, 0, Sst, nullptr, nullptr});
 }
 
 template <typename T>
@@ -301,10 +326,15 @@ jet_status jet_dyn_conv_v(const void* x, const void* w1, const void* w2, const v
     return launch_genconv<float>(x, w1, w2, v, hist_in, v_out, hist_out, conv_w_out, B, T, D, H, dv, s);
 }
 
-size_t jet_gdn_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt) {
+size_t jet_gdn_prefill_workspace_min(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt) {
     if (B <= 0 || T <= 0 || H <= 0 || chunk != 64 || !tc_prefill_ok(dt, dk, dv, (long long)B * T)) return 0;
     const SegPlan plan = plan_segments(B, T, H, dv);
     return sizeof(float) * seg_workspace_floats(B, H, dk, dv, plan.P);
+}
+
+size_t jet_gdn_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt) {
+    if (B <= 0 || T <= 0 || H <= 0 || chunk != 64 || !tc_prefill_ok(dt, dk, dv, (long long)B * T)) return 0;
+    return split_img_bytes(B, T, H, dk) + jet_gdn_prefill_workspace_min(B, T, H, dk, dv, chunk, dt);
 }
 
 jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -317,15 +347,20 @@ jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const fl
     for (const void* p : {q, k, v, (const void*)S0, (const void*)o, (const void*)S_out, (const void*)workspace})
         if (p && !aligned16(p)) return JET_ERR_MISALIGNED;
     if (!aligned_to(g, 4) || !aligned_to(beta, 4)) return JET_ERR_MISALIGNED;
-    const size_t need = jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk, dt);
-    if (need > 0 && (!workspace || ws_bytes < need)) return JET_ERR_WORKSPACE;
+    if (!workspace) ws_bytes = 0;
+    const size_t need_min = jet_gdn_prefill_workspace_min(B, T, H, dk, dv, chunk, dt);
+    if (ws_bytes < need_min) return JET_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (tc_prefill_ok(dt, dk, dv, (long long)B * T)) {
-        // tensor-core path (warp-specialised, sequence-parallel when T is long)
-        float* ws = static_cast<float*>(workspace);
-        if (dk == 64) return launch_prefill_tc<64>(q, k, v, g, beta, S0, o, S_out, ws, B, T, H, dv, s);
-        if (dk == 96) return launch_prefill_tc<96>(q, k, v, g, beta, S0, o, S_out, ws, B, T, H, dv, s);
-        return launch_prefill_tc<128>(q, k, v, g, beta, S0, o, S_out, ws, B, T, H, dv, s);
+        // tensor-core path: two-kernel plan when the workspace holds the chunk images
+        const bool split = ws_bytes >= jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk, dt);
+#define JET_TC(DK)                                                                                     \
+        return split ? launch_prefill_tc<DK, true>(q, k, v, g, beta, S0, o, S_out, workspace, B, T, H, dv, s) \
+                     : launch_prefill_tc<DK, false>(q, k, v, g, beta, S0, o, S_out, workspace, B, T, H, dv, s);
+        if (dk == 64) { JET_TC(64) }
+        if (dk == 96) { JET_TC(96) }
+        JET_TC(128)
+#undef JET_TC
     }
     if (dt == JET_BF16)
         return dispatch_prefill<__nv_bfloat16>(dk, q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
@@ -412,12 +447,15 @@ extern "C" jet_status jet_gdn_prefill_noalloc(const void* q, const void* k, cons
     if (!dtype_ok(dt)) return JET_ERR_INVALID_ARG;
     if (elems({B, T, H, dk}) < 0 || elems({B, T, H, dv}) < 0 || elems({B, H, dv, dk}) < 0) return JET_ERR_INVALID_ARG;
     if (!shape_ok(dk, dv) || chunk != 64 || B > 65535 || H > 65535) return JET_ERR_UNSUPPORTED;
+    // the fastest plan whose scratch fits the array
+    const size_t need_min = jet_gdn_prefill_workspace_min(B, T, H, dk, dv, chunk, dt);
+    if (need_min > (size_t)JET_NOALLOC_SCRATCH_BYTES) return JET_ERR_TOO_LARGE;
     const size_t need = jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk, dt);
-    if (need > (size_t)JET_NOALLOC_SCRATCH_BYTES) return JET_ERR_TOO_LARGE;
+    const size_t use = need <= (size_t)JET_NOALLOC_SCRATCH_BYTES ? need : need_min;
     void* ws = nullptr;
-    if (need > 0) {
+    if (use > 0) {
         const jet_status st = noalloc_scratch(&ws);
         if (st != JET_OK) return st;
     }
-    return jet_gdn_prefill(q, k, v, g, beta, S0, o, S_out, ws, need, B, T, H, dk, dv, chunk, dt, stream);
+    return jet_gdn_prefill(q, k, v, g, beta, S0, o, S_out, ws, use, B, T, H, dk, dv, chunk, dt, stream);
 }

@@ -1,0 +1,379 @@
+// K2b: the state chain of the chunked Gated DeltaNet prefill (Jet-Nemotron
+// paper, section 2.3), fed by the per-chunk images of K2a.
+//
+// With T1, W^T, P, Q~ and the decay vectors of every chunk already in global
+// memory, what remains per chunk is the part that depends on the state
+// (same notation as the preparation kernel):
+//   U^T  = V^T T1^T                    P2a  (state-independent, runs ahead)
+//   Wt^T = U^T - S W^T                 P3
+//   O^T  = S Q~^T + Wt^T P^T           P5a / P5b (output products)
+//   S   <- gam_{L-1} S + Wt^T diag(d/|k|) K   (E4 scales S in TMEM, then P4)
+// One CTA = (sequence, head, 128 state rows) of one segment; the float32
+// state lives in TMEM, its bf16 copy is the A operand of P3 / P5a.
+//
+//   warps 0-3  CHAIN  E4: S -> bf16 copy and S <- gam_L S;  E5: Wt^T -> bf16
+//                     (plain and scaled by d/|k|)
+//   warps 4-7  OUT    E6: O^T (TMEM) -> staging -> global, off the chain
+//   warp  8    CTRL   one thread: bulk copies of the images, TMA of K and V,
+//                     every tcgen05 MMA, in a fixed dependency order
+//
+// Buffers: images double-buffered (the copy of chunk c+2 starts once chunk c
+// is finished), K and V single (K(c+1) once P4(c) is done, V(c+1) once P2a(c)
+// is done). TMEM: S, X1[2] (U^T then Wt^T), X2[2] (O^T) = 384 of 512 columns.
+// Segments (sequence parallelism) work as in the fused kernel: see Seg.
+#pragma once
+#include "k_prefill_chunkprep.cuh"
+
+namespace jet {
+namespace pfch {
+
+using namespace pfws;
+
+constexpr int NCH_T = 128, NOUT = 128;
+constexpr int THREADS = NCH_T + NOUT + 32;            // 288
+constexpr int OUT0 = NCH_T, CTRL0 = NCH_T + NOUT;
+
+template <int DK>
+struct ChainSmem {
+    static constexpr int NKB = (DK + 63) / 64;
+    static constexpr uint32_t IB = ((Img<DK>::BYTES + 1023) / 1024) * 1024;
+    static constexpr uint32_t IMG = 0;                       // [2] images
+    static constexpr uint32_t K = IMG + 2 * IB;              // NKB x [64 tok][64 feat]
+    static constexpr uint32_t V = K + NKB * 8192;            // 2 x [64 tok][64 ch]
+    static constexpr uint32_t AS = V + 16384;                // NKB x [128 rows][64 feat] bf16 S
+    static constexpr uint32_t AW = AS + NKB * 16384;         // Wt^T
+    static constexpr uint32_t AWD = AW + 16384;              // Wt^T diag(d/|k|)
+    static constexpr uint32_t OUT = AWD + 16384;             // [64 tok][128 ch] bf16 output staging
+    static constexpr uint32_t BAR = OUT + 16384;
+    static constexpr uint32_t TSLOT = BAR + 256;
+    static constexpr uint32_t ABORT = TSLOT + 16;
+    static constexpr uint32_t BYTES = ABORT + 16 + 1024;
+    static_assert(BYTES <= 232448, "shared memory budget");
+};
+
+constexpr uint32_t TM_S = 0, TM_X1 = 128, TM_X2 = 256, TM_COLS = 512;
+
+enum {
+    B_IMG = 0,        // [2] image landed
+    B_K = 2,          // K tile landed
+    B_V = 3,          // V tile landed
+    B_P2 = 4,         // P2a complete
+    B_P3 = 5,         // P3 (and P5a) complete
+    B_SDONE = 6,      // [2] P4 / P5b complete
+    B_AS = 8,         // bf16 S written, S scaled (chain)
+    B_AW = 9,         // Wt^T copies written (chain)
+    B_X2FREE = 10,    // [2] O^T read (out)
+    NBARS = 12
+};
+
+template <int DK>
+__global__ void __launch_bounds__(THREADS, 1)
+gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                         const uint8_t* __restrict__ img, const float* S0, __nv_bfloat16* __restrict__ o,
+                         float* S_out, int Tn, int H, int dv, const Seg seg) {
+    static_assert(DK % 32 == 0 && DK >= 64 && DK <= 128, "DK in {64, 96, 128}");
+    using SM = ChainSmem<DK>;
+    using IM = Img<DK>;
+    constexpr int NKB = SM::NKB;
+    constexpr int KSTEPS = DK / 16;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM::BAR);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + SM::TSLOT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM::ABORT);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int ns = dv / ROWS;
+    const int h = blockIdx.y, b = blockIdx.z / seg.zseg, p_seg = blockIdx.z % seg.zseg;
+    const bool trans = blockIdx.x == ns;                  // transition slice (phase A, p >= 1)
+    if (trans && (!seg.phaseA || p_seg == 0)) return;     // whole CTA, before any barrier
+    const int c0 = blockIdx.x * ROWS;                     // transition slice: past dv, V reads as zero
+    const long long bh = (long long)b * H + h;
+    const int nct = (Tn + C - 1) / C;                     // chunks per sequence (image index)
+    const int cbeg = p_seg * seg.seg_chunks;
+    const int tbeg = cbeg * C;
+    const int tend = min(Tn, tbeg + seg.seg_chunks * C);
+    const int nch = (tend - tbeg + C - 1) / C;
+    const bool write_o = !seg.phaseA;
+    const uint8_t* img_bh = img + (size_t)bh * nct * IM::BYTES;
+    auto img_at = [&](int c) -> const uint8_t* { return sm + SM::IMG + (uint32_t)(c & 1) * SM::IB; };
+
+    if (tid == 0) {
+        for (int i = 0; i < NBARS; ++i) mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (tid == CTRL0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (warp == 0) tmem_alloc(tslot, TM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = *tslot;
+
+    if (warp < 4) {
+        // =============================================================== CHAIN
+        const int ct = tid;
+        const uint32_t lb = (uint32_t)(warp * 32) << 16;
+        {   // initial state (row ct of the slice)
+            const float* src = nullptr;
+            if (!seg.phaseA && seg.nseg > 1) {
+                src = seg.Sst + ((((long long)b * seg.nseg + p_seg) * H + h) * dv + c0 + ct) * DK;
+            } else if (p_seg == 0 && !trans && S0) {
+                src = S0 + (bh * dv + c0 + ct) * DK;
+            }
+#pragma unroll
+            for (int cb = 0; cb < DK / 32; ++cb) {
+                uint32_t r[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    r[j] = trans ? (cb * 32 + j == ct ? 0x3f800000u : 0u) : (src ? __float_as_uint(src[cb * 32 + j]) : 0u);
+                tmem_st32(tb + lb + TM_S + cb * 32, r);
+            }
+            tmem_st_wait();
+        }
+        for (int c = 0; c < nch; ++c) {
+            const int p = c & 1;
+            const float* iv = reinterpret_cast<const float*>(img_at(c) + IM::VEC);   // dik[64], gam_{L-1}
+            bool okw = c < 1 || wait_bar(&bars[B_SDONE + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag);
+            okw = okw && wait_bar(&bars[B_IMG + p], (c >> 1) & 1, abort_flag);
+            if (!group_all(2, NCH_T, okw)) break;
+            tc_fence_after();
+            // ---- E4: S -> bf16 copy, S <- gam_L S
+            {
+                const float gL = iv[64];
+#pragma unroll
+                for (int cb = 0; cb < DK / 32; ++cb) {
+                    uint32_t x[32];
+                    tmem_ld32(tb + lb + TM_S + cb * 32, x);
+                    tmem_ld_wait();
+                    uint8_t* tile = sm + SM::AS + (cb >> 1) * 16384;
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(x[8 * ch + e]);
+                        *reinterpret_cast<uint4*>(tile + sw128_off(ct, ((cb & 1) * 32 + ch * 8) * 2)) = pack8(f);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) x[j] = __float_as_uint(gL * __uint_as_float(x[j]));
+                    tmem_st32(tb + lb + TM_S + cb * 32, x);
+                }
+                tmem_st_wait();
+            }
+            fence_async_smem();
+            tc_fence_before();
+            named_sync(2, NCH_T);
+            if (ct == 0) arrive(&bars[B_AS]);
+            // ---- E5: Wt^T -> bf16 (plain and scaled by d/|k|)
+            if (!group_all(2, NCH_T, wait_bar(&bars[B_P3], c & 1, abort_flag))) break;
+            tc_fence_after();
+            {
+                const uint32_t x1 = TM_X1 + (uint32_t)p * 64;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t x[32];
+                    tmem_ld32(tb + lb + x1 + half * 32, x);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        float f[8], fd[8];
+                        const float4 d0 = *reinterpret_cast<const float4*>(iv + half * 32 + ch * 8);
+                        const float4 d1 = *reinterpret_cast<const float4*>(iv + half * 32 + ch * 8 + 4);
+                        const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            f[e] = __uint_as_float(x[ch * 8 + e]);
+                            fd[e] = f[e] * dd[e];
+                        }
+                        const uint32_t off = sw128_off(ct, (half * 32 + ch * 8) * 2);
+                        *reinterpret_cast<uint4*>(sm + SM::AW + off) = pack8(f);
+                        *reinterpret_cast<uint4*>(sm + SM::AWD + off) = pack8(fd);
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            named_sync(2, NCH_T);
+            if (ct == 0) arrive(&bars[B_AW]);
+        }
+        // final state of the segment (after the last P4)
+        const bool fin = !*abort_flag && nch > 0 &&
+                         wait_bar(&bars[B_SDONE + ((nch - 1) & 1)], ((nch - 1) >> 1) & 1, abort_flag);
+        if (group_all(2, NCH_T, fin)) {
+            tc_fence_after();
+            float* dst = nullptr;
+            if (seg.phaseA) {
+                const long long bp = (long long)b * (seg.nseg - 1) + p_seg;
+                if (trans) { if (ct < DK) dst = seg.Ao + ((bp * H + h) * DK + ct) * DK; }
+                else dst = seg.Eo + ((bp * H + h) * dv + c0 + ct) * DK;
+            } else if (p_seg == seg.nseg - 1) {
+                dst = S_out + (bh * dv + c0 + ct) * DK;
+            }
+#pragma unroll
+            for (int cb = 0; cb < DK / 32; ++cb) {
+                if (!dst) break;
+                uint32_t x[32];
+                tmem_ld32(tb + lb + TM_S + cb * 32, x);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4*>(dst + cb * 32 + j) =
+                        make_float4(__uint_as_float(x[j]), __uint_as_float(x[j + 1]), __uint_as_float(x[j + 2]),
+                                    __uint_as_float(x[j + 3]));
+            }
+        }
+    } else if (warp < 8) {
+        // =============================================================== OUT
+        if (write_o) {
+            const int ot = tid - OUT0;                       // channel of the slice
+            const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
+            __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sm + SM::OUT);
+            const long long tstride = (long long)H * dv;
+            for (int c = 0; c < nch; ++c) {
+                if (!group_all(3, NOUT, wait_bar(&bars[B_SDONE + (c & 1)], (c >> 1) & 1, abort_flag))) break;
+                tc_fence_after();
+                const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t x[32];
+                    tmem_ld32(tb + lb + x2 + half * 32, x);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) st[(half * 32 + j) * ROWS + ot] = __float2bfloat16_rn(__uint_as_float(x[j]));
+                }
+                tc_fence_before();
+                named_sync(3, NOUT);
+                if (ot == 0) arrive(&bars[B_X2FREE + (c & 1)]);
+                const int t0 = tbeg + c * C, L = min(C, tend - t0);
+                __nv_bfloat16* obase = o + ((long long)b * Tn + t0) * tstride + (long long)h * dv + c0;
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const int qd = ot + m * NOUT, r = qd >> 4, ch = qd & 15;
+                    if (r < L)
+                        *reinterpret_cast<uint4*>(obase + r * tstride + ch * 8) =
+                            *reinterpret_cast<const uint4*>(st + r * ROWS + ch * 8);
+                }
+                named_sync(3, NOUT);                         // staging free again
+            }
+        }
+    } else if (tid == CTRL0) {
+        // =============================================================== CTRL
+        // Fixed order (every awaited event depends only on actions issued
+        // earlier in this order):
+        //   prologue: IMG(0) K(0) V(0) IMG(1) P2a(0)
+        //   chunk c:  P3(c) [P5a(c)]  V(c+1)  P4(c) [P5b(c)]  P2a(c+1)  K(c+1) IMG(c+2)
+        const uint32_t img_bytes = write_o ? IM::BYTES : IM::A_BYTES;
+        bool ok = true;
+        auto W = [&](int bar, int phase) {
+            if (!ok) return false;
+            for (uint32_t i = 0; i < 4u * kWaitPolls; ++i) {
+                if (mbar_test_wait(&bars[bar], (uint32_t)phase & 1u)) return true;
+                if ((i & 1023u) == 1023u && *abort_flag) { ok = false; return false; }
+                __nanosleep(32);
+            }
+            *abort_flag = 1;
+            flag_error(DEVERR_TIMEOUT);
+            ok = false;
+            return false;
+        };
+        auto zrow = [&](int c) { return (int)((long long)b * Tn + tbeg + (long long)c * C); };
+        auto load_img = [&](int c) {
+            uint64_t* bar = &bars[B_IMG + (c & 1)];
+            mbar_expect_tx(bar, img_bytes);
+            bulk_load(const_cast<uint8_t*>(img_at(c)), img_bh + (size_t)(cbeg + c) * IM::BYTES, img_bytes, bar);
+        };
+        auto load_k = [&](int c) {
+            mbar_expect_tx(&bars[B_K], (uint32_t)(NKB * 8192));
+#pragma unroll
+            for (int kb = 0; kb < NKB; ++kb) tma_load_3d(sm + SM::K + kb * 8192, &tm_k, &bars[B_K], kb * 64, h, zrow(c));
+        };
+        auto load_v = [&](int c) {
+            mbar_expect_tx(&bars[B_V], 16384);
+            tma_load_3d(sm + SM::V, &tm_v, &bars[B_V], c0, h, zrow(c));
+            tma_load_3d(sm + SM::V + 8192, &tm_v, &bars[B_V], c0 + 64, h, zrow(c));
+        };
+        const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
+        const uint64_t dImgMN = sw128_desc(smem_u32(sm + SM::IMG), 8192, 1024);   // W^T (MN-major)
+        const uint64_t dKmn = sw128_desc(smem_u32(sm + SM::K), 8192, 1024);       // K as MN-major
+        const uint64_t dV = sw128_desc(smem_u32(sm + SM::V), 8192, 1024);
+        const uint64_t dAS = sw128_desc(smem_u32(sm + SM::AS), 16, 1024);
+        const uint64_t dAW = sw128_desc(smem_u32(sm + SM::AW), 16, 1024);
+        const uint64_t dAWD = sw128_desc(smem_u32(sm + SM::AWD), 16, 1024);
+        constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
+        constexpr uint32_t ID_MNK = idesc_bf16(128, 64, true, false);
+        constexpr uint32_t ID_NEG = idesc_bf16(128, 64, false, true, true);
+        constexpr uint32_t ID_S = idesc_bf16(128, DK, false, true);
+        auto ioff = [&](int c, uint32_t off) { return (uint64_t)((((uint32_t)(c & 1) * SM::IB) + off) >> 4); };
+        auto mma_p2a = [&](int c) {
+            const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tb + x1, dV + (uint64_t)(kk * 2048 >> 4), dImg + ioff(c, IM::T1 + kk * 32), ID_MNK, kk > 0);
+            mma_commit(&bars[B_P2]);
+        };
+        auto mma_p3 = [&](int c) {
+            const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64, x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk)
+                mma_bf16_ss(tb + x1, dAS + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                            dImgMN + ioff(c, IM::WT + kk * 2048), ID_NEG, 1);
+            mma_commit(&bars[B_P3]);        // the chain waits for Wt^T only
+            if (!write_o) return;
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk)
+                mma_bf16_ss(tb + x2, dAS + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                            dImg + ioff(c, IM::Q + (kk >> 2) * 8192 + (kk & 3) * 32), ID_KK, kk > 0);
+        };
+        auto mma_p4 = [&](int c) {
+            const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tb + TM_S, dAWD + (uint64_t)(kk * 32 >> 4), dKmn + (uint64_t)(kk * 2048 >> 4), ID_S, 1);
+            if (write_o) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), dImg + ioff(c, IM::P + kk * 32), ID_KK, 1);
+            }
+            mma_commit(&bars[B_SDONE + (c & 1)]);
+        };
+        int n2 = 0, n3 = 0, n4 = 0, nK = 0, nV = 0, nI = 0;      // actions issued
+        if (nch > 0) { load_img(0); ++nI; load_k(0); ++nK; load_v(0); ++nV; }
+        if (nch > 1) { load_img(1); ++nI; }
+        if (nch > 0 && W(B_IMG, 0) && W(B_V, 0)) { tc_fence_after(); mma_p2a(0); ++n2; }
+        for (int c = 0; c < nch && ok; ++c) {
+            if (W(B_AS, c) && (!write_o || c < 2 || W(B_X2FREE + (c & 1), (c - 2) >> 1))) {
+                tc_fence_after(); mma_p3(c); ++n3;
+            }
+            if (c + 1 < nch && W(B_P2, c)) { load_v(c + 1); ++nV; }
+            if (W(B_AW, c) && W(B_K, c)) { tc_fence_after(); mma_p4(c); ++n4; }
+            if (c + 1 < nch && W(B_IMG + ((c + 1) & 1), (c + 1) >> 1) && W(B_V, c + 1)) {
+                tc_fence_after(); mma_p2a(c + 1); ++n2;
+            }
+            if (c + 1 < nch && W(B_SDONE + (c & 1), c >> 1)) {
+                load_k(c + 1); ++nK;
+                if (c + 2 < nch) { load_img(c + 2); ++nI; }
+            }
+        }
+        // drain: every issued commit group and load completes before TMEM is freed
+        if (!ok) {
+            *abort_flag = 1;
+            if (n2 > 0) mbar_wait(&bars[B_P2], (n2 - 1) & 1);
+            if (n3 > 0) mbar_wait(&bars[B_P3], (n3 - 1) & 1);
+            if (n4 > 0) mbar_wait(&bars[B_SDONE + ((n4 - 1) & 1)], ((n4 - 1) >> 1) & 1);
+            if (nK > 0) mbar_wait(&bars[B_K], (nK - 1) & 1);
+            if (nV > 0) mbar_wait(&bars[B_V], (nV - 1) & 1);
+            if (nI > 0) mbar_wait(&bars[B_IMG + ((nI - 1) & 1)], ((nI - 1) >> 1) & 1);
+            if (nI > 1) mbar_wait(&bars[B_IMG + ((nI - 2) & 1)], ((nI - 2) >> 1) & 1);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tb, TM_COLS);
+}
+
+}  // namespace pfch
+}  // namespace jet

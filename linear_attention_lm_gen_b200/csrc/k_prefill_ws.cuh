@@ -40,23 +40,14 @@
 // the others stop waiting, then the control thread drains its commits and
 // TMEM is freed.
 #pragma once
-#include <cuda.h>
-#include "common.cuh"
-#include "sm100.cuh"
+#include "k_prefill_common.cuh"
 
 namespace jet {
 namespace pfws {
 
-using namespace sm100;
-
-constexpr int C = 64;
-constexpr int ROWS = 128;
-constexpr int NCHAIN = 128, NPREP = 256;
+constexpr int NCHAIN = 128;
 constexpr int THREADS = NCHAIN + NPREP + 32;          // 416
 constexpr int PREP0 = NCHAIN, CTRL0 = NCHAIN + NPREP;
-constexpr float EPS = 1e-6f;
-constexpr float LOG2E = 1.4426950408889634f;
-constexpr int LDA = 68;                                // fp32 row stride of A / T
 
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_KQ = 0;                         // [2] x 32K: per 64-col block [K 8K | Q 8K]
@@ -69,8 +60,6 @@ constexpr uint32_t OFF_AW = 163840;                    // 16K  Wt^T
 constexpr uint32_t OFF_AWD = 180224;                   // 16K  Wt^T diag(d/|k|); output staging alias
 constexpr uint32_t OFF_AF = 196608;                    // 64 x 68 fp32, A then T in place
 constexpr uint32_t OFF_XS = OFF_AF + 64 * LDA * 4;     // 32 x 40 fp32 block products
-constexpr int LDX = 40;                                // row stride of XS (32 x 32 products)
-constexpr int LDX1 = 24;                               // row stride of XS (16 x 16 products)
 constexpr uint32_t OFF_VEC = OFF_XS + 32 * LDX * 4;    // [2] x 8 x 64 fp32
 constexpr uint32_t OFF_PN = OFF_VEC + 4096;            // 2 x 128 fp32 partial norms
 constexpr uint32_t OFF_BAR = OFF_PN + 1024;            // mbarriers
@@ -100,127 +89,9 @@ enum {
     NBARS = 18
 };
 
-struct Vec {       // per-token vectors of one chunk (64 floats each)
-    float* G;      // cumulative gate, log2 units
-    float* gam;    // exp(G)
-    float* dcy;    // exp(G_{L-1} - G_i), 0 past the chunk end
-    float* bet;
-    float* ik;     // 1/|k|
-    float* iq;     // 1/|q|
-    float* graw;
-    float* F;      // exp(G_31 - G_i) for i < 32 (the lower-left block factor)
-};
 __device__ __forceinline__ Vec vec_at(uint8_t* sm, int p) {
-    float* v = reinterpret_cast<float*>(sm + OFF_VEC) + p * 512;
-    return Vec{v, v + 64, v + 128, v + 192, v + 256, v + 320, v + 384, v + 448};
+    return vec_from(reinterpret_cast<float*>(sm + OFF_VEC) + p * 512);
 }
-
-// 2^x via the MUFU ex2 instruction (relative error ~2^-22; results below
-// 2^-126 flush to zero, which only ever affects decays that are negligible)
-__device__ __forceinline__ float fast_exp2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ void named_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory");
-}
-
-// bounded wait that also gives up when another thread raised the abort flag
-// (a short sleep between polls keeps idle waiters from taking issue slots
-// from the warps that are computing)
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-    for (uint32_t i = 0; i < kWaitPolls; ++i) {
-        if (mbar_test_wait(bar, parity)) return true;
-        if ((i & 255u) == 255u && *abort_flag) return false;
-        __nanosleep(64);
-    }
-    *abort_flag = 1;
-    flag_error(DEVERR_TIMEOUT);
-    return false;
-}
-// true on every thread of named barrier `id` iff `ok` holds on all of them
-__device__ __forceinline__ bool group_all(int id, int n, bool ok) {
-    uint32_t r;
-    asm volatile(
-        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
-        " bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-        : "=r"(r) : "r"((uint32_t)ok), "r"(id), "r"(n) : "memory");
-    return r != 0;
-}
-__device__ __forceinline__ void arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&h);
-}
-__device__ __forceinline__ uint4 pack8(const float* v) {
-    return make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]), pack2(v[6], v[7]));
-}
-__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-}
-// warp-level m16n8k8 tf32 MMA (float32 accumulate); operands rounded to tf32
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-__device__ __forceinline__ void mma_tf32(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-// D[16 x 8] += A[16 x 8k] B[8k x 8] over ksteps steps of 8; A and B in shared
-// memory (row strides lda, ldb); fragment layout of m16n8k8: lane = 4 g + t,
-// A rows g, g+8 / cols t, t+4; B rows t, t+4 / col g; D rows g, g+8 / cols 2t, 2t+1
-__device__ __forceinline__ void warp_mm_tf32(float* d, const float* A, int lda, const float* B, int ldb,
-                                             int ksteps, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-    for (int ks = 0; ks < ksteps; ++ks) {
-        const float* a = A + ks * 8;
-        const float* bb = B + ks * 8 * ldb;
-        mma_tf32(d, to_tf32(a[g * lda + t]), to_tf32(a[(g + 8) * lda + t]), to_tf32(a[g * lda + t + 4]),
-                 to_tf32(a[(g + 8) * lda + t + 4]), to_tf32(bb[t * ldb + g]), to_tf32(bb[(t + 4) * ldb + g]));
-    }
-}
-// byte offset of 16-byte chunk `ch` (8 bf16 columns) of row `r` in a K/Q tile
-// stored as 64-column SW128 blocks of stride `bstride`
-__device__ __forceinline__ uint32_t blk_chunk(int r, int ch, uint32_t bstride) {
-    return (uint32_t)(ch >> 3) * bstride + sw128_off((uint32_t)r, (uint32_t)(ch & 7) * 16u);
-}
-
-// Segment decomposition of the token axis (sequence parallelism; the
-// recurrence is affine in the state, S_end = S_start A + B, so segments can
-// run concurrently once their start states are known):
-//   phase A  every segment p < P-1 runs from a zero state (p > 0) or S0
-//            (p = 0) and writes its end state B_p; an extra 128-row slice
-//            starts from the identity with zero values and yields the
-//            segment's dk x dk transition A_p;
-//   combine  S_start(p+1) = S_start(p) A_p + B_p (seg_combine_kernel);
-//   phase C  every segment runs from its true start state and writes o; the
-//            last one writes the final state.
-// P = 1 is the plain single pass.
-struct Seg {
-    int nseg;          // P
-    int seg_chunks;    // chunks per segment (the last may be shorter)
-    int zseg;          // segments covered by this launch (blockIdx.z = b * zseg + p)
-    int phaseA;        // 1: end states and transitions, no outputs
-    const float* Sst;  // phase C start states (P > 1): [B][P][H][dv][dk]
-    float* Eo;         // phase A end states: [B][P-1][H][dv][dk]
-    float* Ao;         // phase A transitions: [B][P-1][H][dk][dk]
-};
 
 template <int DK>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -231,14 +102,13 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     static_assert(DK % 32 == 0 && DK >= 64 && DK <= 128, "DK in {64, 96, 128}");
     constexpr int NKB = (DK + 63) / 64;
     constexpr int KSTEPS = DK / 16;
-    constexpr int NCH = DK / 8;                          // 16-byte chunks per q/k row
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + OFF_TSLOT);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, warp = tid >> 5;
     const int ns = dv / ROWS;
     const int h = blockIdx.y, b = blockIdx.z / seg.zseg, p_seg = blockIdx.z % seg.zseg;
     const bool trans = blockIdx.x == ns;                  // transition slice (phase A, p >= 1)
@@ -416,10 +286,7 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
     } else if (warp < 12) {
         // =============================================================== PREP
-        const int pt = tid - PREP0;                 // 0..255
-        const int pw = pt >> 5;                     // 0..7
-        const int q4 = pw & 3, hh = pw >> 2;        // TMEM lane quarter, column half
-        const uint32_t lb = (uint32_t)(q4 * 32) << 16;
+        const int pt = tid - PREP0;                 // 0..255 (warps 4-11: lane quarter = warp & 3)
         float* AF = reinterpret_cast<float*>(sm + OFF_AF);
         float* XS = reinterpret_cast<float*>(sm + OFF_XS);
         float* PN = reinterpret_cast<float*>(sm + OFF_PN);
@@ -434,44 +301,7 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             bool okw = cv < 2 || wait_bar(&bars[B_X1FREE + pv], ((cv - 2) >> 1) & 1, abort_flag);
             okw = okw && wait_bar(&bars[B_KFULL + pv], (cv >> 1) & 1, abort_flag);
             if (!group_all(1, NPREP, okw)) return false;
-            if (pt < 64) V.graw[pt] = gb; else if (pt < 128) V.bet[pt - 64] = gb;
-            {   // L2 norms: row = pt & 127 (k rows then q rows), half of the columns
-                const int row = pt & 127, half = pt >> 7;
-                const uint32_t qoff = row < 64 ? 0u : 8192u;
-                float ss = 0.f;
-#pragma unroll
-                for (int j = 0; j < NCH / 2; ++j) {
-                    float f[8];
-                    unpack8(*reinterpret_cast<const uint4*>(KQ + qoff + blk_chunk(row & 63, half * (NCH / 2) + j, 16384)), f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) ss += f[e] * f[e];
-                }
-                PN[half * 128 + row] = ss;
-            }
-            named_sync(1, NPREP);
-            if (pt < 128) {
-                const float inv = 1.0f / sqrtf(PN[pt] + PN[128 + pt] + EPS);
-                if (pt < 64) V.ik[pt] = inv; else V.iq[pt - 64] = inv;
-            }
-            if (pw == 0) {   // inclusive scan of the gates, two per lane, in log2 units
-                const float a0 = V.graw[2 * lane], a1 = a0 + V.graw[2 * lane + 1];
-                float run = a1;
-#pragma unroll
-                for (int o2 = 1; o2 < 32; o2 <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, run, o2);
-                    if (lane >= o2) run += y;
-                }
-                V.G[2 * lane] = (run - a1 + a0) * LOG2E;
-                V.G[2 * lane + 1] = run * LOG2E;
-            }
-            named_sync(1, NPREP);
-            if (pt < 64) {
-                V.gam[pt] = fast_exp2(V.G[pt]);
-                V.dcy[pt] = pt < L ? fast_exp2(V.G[L - 1] - V.G[pt]) : 0.f;
-            } else if (pt < 96) {
-                V.F[pt - 64] = fast_exp2(V.G[31] - V.G[pt - 64]);
-            }
-            named_sync(1, NPREP);
+            prep_vectors<DK>(KQ, V, PN, gb, L, pt, 1);
             if (pt == 0) arrive(&bars[B_VEC + pv]);
             return true;
         };
@@ -497,183 +327,18 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             okw = okw && wait_bar(&bars[B_P1], c & 1, abort_flag);
             if (!group_all(1, NPREP, okw)) break;
             tc_fence_after();
-            {
-                uint32_t x[32];
-                tmem_ld32(tb + lb + TM_XP + hh * 32, x);
-                tmem_ld_wait();
-                const int rb = q4 & 1;                    // 32-row block of the thread's row
-                const int r = rb * 32 + lane;
-                const float Gr = V.G[r];
-                // lower-left block (rb = 1, hh = 0): exp(G_r - G_i) = exp(G_r - G_31) exp(G_31 - G_i),
-                // both factors <= 1; upper-right block (rb = 0, hh = 1) is all zero (i > r)
-                const bool zero_blk = rb == 0 && hh == 1;
-                const bool fact_blk = rb == 1 && hh == 0;
-                const float Rr = fact_blk ? fast_exp2(Gr - V.G[31]) : 0.f;
-                const float4* G4 = reinterpret_cast<const float4*>(V.G + hh * 32);
-                const float4* K4 = reinterpret_cast<const float4*>(V.ik + hh * 32);
-                const float4* F4 = reinterpret_cast<const float4*>(V.F);
-                float e[32];
-#pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
-                    const float4 gg = G4[i4], kk = K4[i4];
-                    const float gv[4] = {gg.x, gg.y, gg.z, gg.w}, kv[4] = {kk.x, kk.y, kk.z, kk.w};
-                    float fv[4] = {0.f, 0.f, 0.f, 0.f};
-                    if (fact_blk) { const float4 ff = F4[i4]; fv[0] = ff.x; fv[1] = ff.y; fv[2] = ff.z; fv[3] = ff.w; }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int j = i4 * 4 + u;
-                        const float dec = zero_blk ? 0.f : (fact_blk ? Rr * fv[u] : fast_exp2(Gr - gv[u]));
-                        e[j] = dec * __uint_as_float(x[j]) * kv[u];
-                    }
-                }
-                if (q4 < 2) {
-                    const float sc = V.bet[r] * V.ik[r];
-#pragma unroll
-                    for (int i4 = 0; i4 < 8; ++i4) {
-                        const int i = hh * 32 + i4 * 4;
-                        float4 a;
-                        a.x = i + 0 < r ? sc * e[i4 * 4 + 0] : 0.f;
-                        a.y = i + 1 < r ? sc * e[i4 * 4 + 1] : 0.f;
-                        a.z = i + 2 < r ? sc * e[i4 * 4 + 2] : 0.f;
-                        a.w = i + 3 < r ? sc * e[i4 * 4 + 3] : 0.f;
-                        *reinterpret_cast<float4*>(AF + r * LDA + i) = a;
-                    }
-                } else {
-                    const float sc = V.iq[r];
-                    uint8_t* Pt = sm + OFF_P + p * 8192;
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        float f[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int i = hh * 32 + ch * 8 + u;
-                            f[u] = i <= r ? sc * e[ch * 8 + u] : 0.f;
-                        }
-                        *reinterpret_cast<uint4*>(Pt + sw128_off(r, (hh * 32 + ch * 8) * 2)) = pack8(f);
-                    }
-                }
-            }
+            prep_e1(tb + TM_XP, V, AF, sm + OFF_P + p * 8192, pt);
             named_sync(1, NPREP);
             // ---- UT inverse in place: 16x16 diagonal blocks, then 16 -> 32 -> 64 doubling
-            {
-                float t[16];
-                if (pt < 64) {
-                    const int cc = pt, j = cc >> 4, cl = cc & 15;
-                    const float* Ab = AF + (j * 16) * LDA + j * 16;
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        float xv = (r == cl) ? 1.f : 0.f;
-#pragma unroll
-                        for (int i = 0; i < r; ++i) xv -= Ab[r * LDA + i] * t[i];
-                        t[r] = xv;
-                    }
-                }
-                named_sync(1, NPREP);
-                if (pt < 64) {
-                    const int cc = pt, j = cc >> 4;
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) AF[(j * 16 + r) * LDA + cc] = t[r];
-                }
-                named_sync(1, NPREP);
-                // 16 -> 32 for pairs (1,0) and (3,2): X = A_10 T_00, T_10 = -T_11 X
-                // (warps 0-3: pair = pw >> 1, 8-column half = pw & 1)
-                const int g8 = lane >> 2, t4 = lane & 3;
-                if (pw < 4) {
-                    const int pr = pw >> 1, nh = pw & 1;
-                    const int b0 = pr * 2, b1 = b0 + 1;
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    warp_mm_tf32(d, AF + (b1 * 16) * LDA + b0 * 16, LDA, AF + (b0 * 16) * LDA + b0 * 16 + nh * 8, LDA,
-                                 2, lane);
-                    float* xo = XS + pr * 16 * LDX1 + nh * 8;
-                    xo[g8 * LDX1 + 2 * t4] = d[0];
-                    xo[g8 * LDX1 + 2 * t4 + 1] = d[1];
-                    xo[(g8 + 8) * LDX1 + 2 * t4] = d[2];
-                    xo[(g8 + 8) * LDX1 + 2 * t4 + 1] = d[3];
-                }
-                named_sync(1, NPREP);
-                if (pw < 4) {
-                    const int pr = pw >> 1, nh = pw & 1;
-                    const int b0 = pr * 2, b1 = b0 + 1;
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    warp_mm_tf32(d, AF + (b1 * 16) * LDA + b1 * 16, LDA, XS + pr * 16 * LDX1 + nh * 8, LDX1, 2, lane);
-                    float* to = AF + (b1 * 16) * LDA + b0 * 16 + nh * 8;
-                    to[g8 * LDA + 2 * t4] = -d[0];
-                    to[g8 * LDA + 2 * t4 + 1] = -d[1];
-                    to[(g8 + 8) * LDA + 2 * t4] = -d[2];
-                    to[(g8 + 8) * LDA + 2 * t4 + 1] = -d[3];
-                }
-                named_sync(1, NPREP);
-                // 32 -> 64: X = A[32:64][0:32] T[0:32][0:32], T[32:64][0:32] = -T[32:64][32:64] X
-                // (warp pw: 16-row half mt = pw >> 2, 8-column quarter nq = pw & 3)
-                {
-                    const int mt = pw >> 2, nq = pw & 3;
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    warp_mm_tf32(d, AF + (32 + mt * 16) * LDA, LDA, AF + nq * 8, LDA, 4, lane);
-                    float* xo = XS + (mt * 16) * LDX + nq * 8;
-                    xo[g8 * LDX + 2 * t4] = d[0];
-                    xo[g8 * LDX + 2 * t4 + 1] = d[1];
-                    xo[(g8 + 8) * LDX + 2 * t4] = d[2];
-                    xo[(g8 + 8) * LDX + 2 * t4 + 1] = d[3];
-                }
-                named_sync(1, NPREP);
-                {
-                    const int mt = pw >> 2, nq = pw & 3;
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    warp_mm_tf32(d, AF + (32 + mt * 16) * LDA + 32, LDA, XS + nq * 8, LDX, 4, lane);
-                    float* to = AF + (32 + mt * 16) * LDA + nq * 8;
-                    to[g8 * LDA + 2 * t4] = -d[0];
-                    to[g8 * LDA + 2 * t4 + 1] = -d[1];
-                    to[(g8 + 8) * LDA + 2 * t4] = -d[2];
-                    to[(g8 + 8) * LDA + 2 * t4 + 1] = -d[3];
-                }
-                named_sync(1, NPREP);
-            }
+            ut_inverse(AF, XS, pt, 1);
             // ---- T1 = T diag(b), T2 = T diag(b gam / |k|): row r = pt >> 2, 16 columns
-            {
-                const int r = pt >> 2, qc = pt & 3;
-#pragma unroll
-                for (int hc = 0; hc < 2; ++hc) {
-                    const int i0 = qc * 16 + hc * 8;
-                    float f1[8], f2[8];
-#pragma unroll
-                    for (int h4 = 0; h4 < 2; ++h4) {
-                        const float4 tv = *reinterpret_cast<const float4*>(AF + r * LDA + i0 + h4 * 4);
-                        const float4 bv = *reinterpret_cast<const float4*>(V.bet + i0 + h4 * 4);
-                        const float4 gv = *reinterpret_cast<const float4*>(V.gam + i0 + h4 * 4);
-                        const float4 kv = *reinterpret_cast<const float4*>(V.ik + i0 + h4 * 4);
-                        const float t_[4] = {tv.x, tv.y, tv.z, tv.w}, b_[4] = {bv.x, bv.y, bv.z, bv.w};
-                        const float g_[4] = {gv.x, gv.y, gv.z, gv.w}, k_[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i = i0 + h4 * 4 + e;
-                            const float t1v = i <= r ? t_[e] * b_[e] : 0.f;
-                            f1[h4 * 4 + e] = t1v;
-                            f2[h4 * 4 + e] = t1v * g_[e] * k_[e];
-                        }
-                    }
-                    const uint32_t off = sw128_off(r, i0 * 2);
-                    *reinterpret_cast<uint4*>(sm + OFF_T1 + off) = pack8(f1);
-                    *reinterpret_cast<uint4*>(sm + OFF_T2 + off) = pack8(f2);
-                }
-            }
+            prep_t1t2(AF, V, sm + OFF_T1, sm + OFF_T2, pt);
             fence_async_smem();
             tc_fence_before();
             named_sync(1, NPREP);
             if (pt == 0) arrive(&bars[B_TREADY]);
             // ---- Q~ = diag(gam / |q|) Q, in place (P1 has consumed Q)
-            {
-                const int r = pt >> 2, qc = pt & 3;
-                const float sq = V.gam[r] * V.iq[r];
-#pragma unroll
-                for (int j = qc; j < NCH; j += 4) {
-                    uint4* pq = reinterpret_cast<uint4*>(KQ + 8192 + blk_chunk(r, j, 16384));
-                    float f[8];
-                    unpack8(*pq, f);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) f[u] *= sq;
-                    *pq = pack8(f);
-                }
-            }
+            prep_qtilde<DK>(KQ, V, pt);
             // ---- next chunk's per-token vectors while P2 runs
             if (c + 1 < nch) {
                 const float gbn = gb_next;
@@ -685,21 +350,7 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             okw = okw && wait_bar(&bars[B_P2], c & 1, abort_flag);
             if (!group_all(1, NPREP, okw)) break;
             tc_fence_after();
-            {
-                uint32_t x[32];
-                tmem_ld32(tb + lb + TM_XW + hh * 32, x);
-                tmem_ld_wait();
-                const int j = q4 * 32 + lane;
-                if (j < DK) {
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        float f[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(x[ch * 8 + u]);
-                        *reinterpret_cast<uint4*>(sm + OFF_WT + sw128_off(j, (hh * 32 + ch * 8) * 2)) = pack8(f);
-                    }
-                }
-            }
+            prep_wt<DK>(tb + TM_XW, sm + OFF_WT, pt);
             fence_async_smem();
             tc_fence_before();
             named_sync(1, NPREP);

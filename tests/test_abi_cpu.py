@@ -126,6 +126,27 @@ def test_workspace_query_is_host_only(lib):
         assert prefill(lib, B=1, T=4096, H=12, dk=96, dv=256, ws=None, wsb=0) == WORKSPACE
 
 
+@pytest.mark.parametrize("B,T,H,dk,dv,img", [(1, 4096, 12, 96, 256, 46080), (2, 1553, 2, 64, 128, 33792),
+                                             (1, 65536, 16, 128, 256, 50176), (3, 100, 2, 96, 256, 46080)])
+def test_workspace_sizes(lib, B, T, H, dk, dv, img):
+    # fastest plan = one image per (sequence, head, 64-token chunk) + the segment buffers
+    lo = jet.jet_gdn_prefill_workspace_min(B, T, H, dk, dv)
+    hi = jet.jet_gdn_prefill_workspace_size(B, T, H, dk, dv)
+    assert hi == lo + B * H * ((T + 63) // 64) * img
+    assert lo % 256 == 0 and (hi - lo) % 1024 == 0
+    # a workspace below the minimum is refused before anything runs
+    if lo > 0:
+        assert prefill(lib, B=B, T=T, H=H, dk=dk, dv=dv, ws=A, wsb=lo - 16) == WORKSPACE
+
+
+def test_workspace_is_zero_off_the_tensor_core_path():
+    import torch
+    # float32 inputs and key dims other than 64 / 96 / 128 run the FFMA kernel, which needs none
+    for args, dt in (((1, 4096, 12, 96, 256), torch.float32), ((1, 4096, 2, 48, 64), torch.bfloat16)):
+        assert jet.jet_gdn_prefill_workspace_min(*args, 64, dt) == 0
+        assert jet.jet_gdn_prefill_workspace_size(*args, 64, dt) == 0
+
+
 def test_python_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(1, 4, 64, dtype=torch.bfloat16)

@@ -42,6 +42,20 @@ def nan_like(t):
     return torch.full_like(t, float("nan"))
 
 
+def prefill(plan, q, k, v, g, beta, S0=None, o=None, S_out=None):
+    """jet_gdn_prefill with the fastest plan ("split": chunk images, then the
+    chain kernel) or, given only the minimum workspace, the fused plan."""
+    ws = None
+    if plan == "fused":
+        B, T, H, dk = q.shape
+        n = jet.jet_gdn_prefill_workspace_min(B, T, H, dk, v.shape[-1], 64, q.dtype)
+        ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+    return jet.jet_gdn_prefill(q, k, v, g, beta, S0, o, S_out, workspace=ws)
+
+
+PLANS = ["split", "fused"]
+
+
 def shape(dtype, **kw):
     base = dict(name="t", B=1, T=64, H=2, dk=16, dv=32, D=64, dtype=dtype)
     base.update(kw)
@@ -112,14 +126,15 @@ def test_identity_taps_via_conv_stage(orc):
                                            ("bf16", 3, 32, 64), ("f32", 2, 64, 64), ("bf16", 2, 64, 128)])
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 130, 333])
 @pytest.mark.parametrize("s0", [False, True])
-def test_prefill_gdn_stage(orc, dtype, H, dk, dv, T, s0):
+@pytest.mark.parametrize("plan", PLANS)
+def test_prefill_gdn_stage(orc, dtype, H, dk, dv, T, s0, plan):
     s = shape(dtype, B=2, T=T, H=H, dk=dk, dv=dv, D=64)
     inp = synth.prefill_inputs(s, seed=T, s0_std=0.3 if s0 else None)
     d = gpu_inputs(inp)
     ref = to_oracle(inp)
     o = nan_like(d["v"])
     S_out = torch.full((2, H, dv, dk), float("nan"), device="cuda")
-    jet.jet_gdn_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d.get("S0"), o, S_out)
+    prefill(plan, d["q"], d["k"], d["v"], d["g"], d["beta"], d.get("S0"), o, S_out)
     ro, rS = orc.gdn_sequential(ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"],
                                 inp["S0"].astype(np.float64) if s0 else None)
     assert_close(host64(o), ro, dtype, "o")
@@ -127,13 +142,14 @@ def test_prefill_gdn_stage(orc, dtype, H, dk, dv, T, s0):
 
 
 @pytest.mark.parametrize("dtype,dk", [("bf16", 96), ("f32", 16)])
-def test_prefill_long_memory_gates(orc, dtype, dk):
+@pytest.mark.parametrize("plan", PLANS)
+def test_prefill_long_memory_gates(orc, dtype, dk, plan):
     # g = -0.01 softplus(N(0,1)): a ~ 0.99, so the state carries across many chunks
     s = shape(dtype, B=1, T=400, H=2, dk=dk, dv=64, D=64)
     inp = synth.prefill_inputs(s, seed=9, gate_scale=0.01, s0_std=0.1)
     d = gpu_inputs(inp)
     ref = to_oracle(inp)
-    o, S_out = jet.jet_gdn_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    o, S_out = prefill(plan, d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
     ro, rS = orc.gdn_sequential(ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"], inp["S0"].astype(np.float64))
     assert_close(host64(o), ro, dtype, "o")
     assert_close(host64(S_out), rS, dtype, "S")
@@ -141,31 +157,33 @@ def test_prefill_long_memory_gates(orc, dtype, dk):
 
 @pytest.mark.parametrize("B,T,dk,s0,gate_scale", [(1, 1553, 96, True, 0.01), (2, 1600, 64, False, 0.01),
                                                   (1, 4096 + 64 * 9 + 5, 128, True, 1.0)])
-def test_prefill_sequence_parallel_segments(orc, B, T, dk, s0, gate_scale):
+@pytest.mark.parametrize("plan", PLANS)
+def test_prefill_sequence_parallel_segments(orc, B, T, dk, s0, gate_scale, plan):
     # long enough for the segmented path (phase A, combine, phase C); long-memory
     # gates make the carried segment states matter
     import linear_attention_lm_gen_b200 as m
-    assert m.jet_gdn_prefill_workspace_size(B, T, 2, dk, 256) > 0
+    assert m.jet_gdn_prefill_workspace_min(B, T, 2, dk, 256) > 0
     s = shape("bf16", B=B, T=T, H=2, dk=dk, dv=256, D=64)
     inp = synth.prefill_inputs(s, seed=21, gate_scale=gate_scale, s0_std=0.2 if s0 else None)
     d = gpu_inputs(inp)
     ref = to_oracle(inp)
     o = nan_like(d["v"])
     S_out = torch.full((B, 2, 256, dk), float("nan"), device="cuda")
-    jet.jet_gdn_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d.get("S0"), o, S_out)
+    prefill(plan, d["q"], d["k"], d["v"], d["g"], d["beta"], d.get("S0"), o, S_out)
     ro, rS = orc.gdn_sequential(ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"],
                                 inp["S0"].astype(np.float64) if s0 else None)
     assert_close(host64(o), ro, "bf16", "o")
     assert_close(host64(S_out), rS, "bf16", "S")
 
 
-def test_prefill_segments_final_state_may_alias_initial_state(orc):
+@pytest.mark.parametrize("plan", PLANS)
+def test_prefill_segments_final_state_may_alias_initial_state(orc, plan):
     s = shape("bf16", B=1, T=2000, H=2, dk=96, dv=256, D=64)
     inp = synth.prefill_inputs(s, seed=22, gate_scale=0.01, s0_std=0.2)
     d = gpu_inputs(inp)
     ref = to_oracle(inp)
     S = d["S0"].clone()
-    o, _ = jet.jet_gdn_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], S, None, S)
+    o, _ = prefill(plan, d["q"], d["k"], d["v"], d["g"], d["beta"], S, None, S)
     ro, rS = orc.gdn_sequential(ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"], inp["S0"].astype(np.float64))
     assert_close(host64(o), ro, "bf16", "o")
     assert_close(host64(S), rS, "bf16", "S")
