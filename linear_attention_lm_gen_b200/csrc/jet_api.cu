@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -68,16 +69,29 @@ bool dtype_ok(jet_dtype dt) { return dt == JET_F32 || dt == JET_BF16; }
 // ---------------------------------------------------------------- K1
 template <typename T, int TB, int RUN>
 jet_status launch_genconv_t(const void* x, const void* w1, const void* w2, const void* v, const void* hin,
-                            void* vout, void* hout, float* cw, int B, int Tn, int D, int H, int dv, int hpc,
-                            cudaStream_t s) {
+                            void* vout, void* hout, float* cw, int B, int Tn, int D, int H, int dv, int groups,
+                            int hpc, cudaStream_t s) {
     const long long N = (long long)B * Tn;
     const size_t smem = sizeof(float) * gc_smem_floats(TB, hpc * GC_W);
     auto kern = genconv_kernel<T, TB, RUN>;
     if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
-    dim3 grid((unsigned)((N + TB - 1) / TB), (unsigned)((H + hpc - 1) / hpc));
-    kern<<<grid, GC_THREADS, smem, s>>>((const T*)x, (const T*)w1, (const T*)w2, (const T*)v, (const T*)hin,
-                                        (T*)vout, (T*)hout, cw, B, Tn, D, H, dv, hpc);
+    // the head-group CTAs of a token block form one cluster
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((N + TB - 1) / TB), (unsigned)groups);
+    cfg.blockDim = dim3(GC_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = (unsigned)groups;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, (const T*)x, (const T*)w1, (const T*)w2, (const T*)v,
+                                             (const T*)hin, (T*)vout, (T*)hout, cw, B, Tn, D, H, dv, hpc);
     g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (e != cudaSuccess) return JET_ERR_CUDA;
     return launch_status();
 }
 
@@ -87,13 +101,15 @@ jet_status launch_genconv(const void* x, const void* w1, const void* w2, const v
                           cudaStream_t s) {
     constexpr int TB = 16;
     const long long nblk = ((long long)B * Tn + TB - 1) / TB;
-    // split heads across CTAs until the grid covers the SMs about twice
+    // head groups (= cluster size, at most 8): enough CTAs to cover the SMs
+    // about twice, then as few groups as give every group a head
     int groups = 1;
-    while (groups < H && nblk * groups < 296) ++groups;
+    while (groups < H && groups < 8 && nblk * groups < 296) ++groups;
     const int hpc = (H + groups - 1) / groups;
+    groups = (H + hpc - 1) / hpc;
     if (Tn >= 8)
-        return launch_genconv_t<T, TB, 8>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, hpc, s);
-    return launch_genconv_t<T, TB, 1>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, hpc, s);
+        return launch_genconv_t<T, TB, 8>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, groups, hpc, s);
+    return launch_genconv_t<T, TB, 1>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, groups, hpc, s);
 }
 
 jet_status check_gen(const void* x, const void* w1, const void* w2, int B, int T, int D, int H,
@@ -218,8 +234,11 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
     if (SPLIT) {   // K2a: every chunk of every (sequence, head)
         auto prep = pfws::gdn_chunk_prep_kernel<DK>;
         if (smem_attr(prep, pfws::PrepSmem<DK>::BYTES) != JET_OK) return JET_ERR_CUDA;
-        prep<<<dim3((Tn + pfws::C - 1) / pfws::C, H, B), pfws::PREP_THREADS, pfws::PrepSmem<DK>::BYTES, s>>>(
-            mq, mk, g, beta, img, Tn, H);
+        const int nct = (Tn + pfws::C - 1) / pfws::C;
+        const long long items = (long long)B * H * nct;
+        const int grid = (int)std::min<long long>(items, 2LL * kSMs);   // two resident CTAs per SM
+        prep<<<grid, pfws::PREP_THREADS, pfws::PrepSmem<DK>::BYTES, s>>>(mq, mk, g, beta, img, Tn, H, nct,
+                                                                         (int)items);
         g_launches.fetch_add(1, std::memory_order_relaxed);
         if (launch_status() != JET_OK) return JET_ERR_CUDA;
     }

@@ -7,10 +7,14 @@
 // with positions before token 0 taken from the history (or zero).
 //
 // One CTA owns TB consecutive tokens of the flattened [B*T] token axis and a
-// group of heads:
-//   stage A  x[TB,D] . W1[D,32]: bf16 tensor-core mma (m16n8k16, fp32
-//            accumulate), the D reduction split over the 8 warps, partial
-//            sums reduced in shared memory; float32 inputs use FFMA.
+// group of heads; the G head-group CTAs of a token block form a thread-block
+// cluster:
+//   stage A  x[TB,D] . W1[D,32] split over the cluster: CTA g reduces the
+//            g-th slice of D (bf16 tensor-core mma m16n8k16 with fp32
+//            accumulate, the slice split again over the 8 warps; float32
+//            inputs use FFMA), the partial sums meet in distributed shared
+//            memory, and every CTA adds the G partials in the same order, so
+//            x and W1 are read once per token block.
 //   stage B  SiLU, then h[TB,32] . W2[32,H*4] in FFMA -> taps in shared memory
 //            (and optionally to global).
 //   stage C  conv: each work item is one 16-byte channel group of one head
@@ -31,6 +35,7 @@ constexpr int GC_W = 4;         // conv width
 // shared-memory layout (floats), TB tokens, CW = tap columns per CTA
 __host__ __device__ constexpr int gc_smem_floats(int TB, int CW) {
     return 8 * TB * GC_HID      // partial sums of the 8 warps (bf16 path)
+         + TB * GC_HID          // the CTA's partial sum (read by the cluster)
          + TB * (GC_HID + 1)    // hidden activations
          + GC_HID * CW          // W2 columns of the CTA's heads, as float
          + TB * CW;             // taps
@@ -38,6 +43,29 @@ __host__ __device__ constexpr int gc_smem_floats(int TB, int CW) {
 
 __device__ __forceinline__ uint32_t ld_u32(const void* p) { return *reinterpret_cast<const uint32_t*>(p); }
 __device__ __forceinline__ uint32_t pack_u16(uint16_t lo, uint16_t hi) { return (uint32_t)lo | ((uint32_t)hi << 16); }
+
+// ---- thread-block cluster helpers (distributed shared memory)
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+    uint32_t n;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+    return n;
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// the float at the same shared-memory offset in cluster CTA `rank`
+__device__ __forceinline__ float ld_peer_f32(const float* p, uint32_t rank) {
+    uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p)), ra;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+    return v;
+}
 
 __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, const uint32_t* b) {
     asm volatile(
@@ -47,11 +75,12 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, cons
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// Stage A for bf16: z_part[warp][t][r] over the warp's share of the D axis.
+// Stage A for bf16: z_part[warp][t][r] over the warp's share of the k-steps
+// [ks0, ks1) (16 D-columns each).
 template <int TB>
 __device__ __forceinline__ void gen_stageA_bf16(const __nv_bfloat16* __restrict__ x,
                                                 const __nv_bfloat16* __restrict__ W1,
-                                                long long r0, long long N, int D, float* zpart) {
+                                                long long r0, long long N, int D, int ks0, int ks1, float* zpart) {
     constexpr int MT = TB / 16;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, t4 = lane & 3;
@@ -65,9 +94,8 @@ __device__ __forceinline__ void gen_stageA_bf16(const __nv_bfloat16* __restrict_
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[m][n][e] = 0.f;
 
-    const int nks = D / 16;
 #pragma unroll 4
-    for (int ks = warp; ks < nks; ks += 8) {
+    for (int ks = ks0 + warp; ks < ks1; ks += 8) {
         const int k0 = ks * 16 + t4 * 2;
         uint32_t bfr[4][2];
 #pragma unroll
@@ -101,14 +129,15 @@ __device__ __forceinline__ void gen_stageA_bf16(const __nv_bfloat16* __restrict_
         }
 }
 
-// Grid: x = blocks of TB tokens, y = head groups of `hpc` heads. Every CTA of
-// a token block computes the (cheap) hidden activations of its tokens; the
-// taps and the conv are split across the head groups so that small token
-// counts (decode: one token per sequence) still spread over many SMs.
+// Grid: x = blocks of TB tokens, y = G head groups of `hpc` heads, launched
+// as clusters of (1, G, 1): the G CTAs of a token block split the x . W1
+// reduction and share the result, and the taps and the conv are split across
+// the head groups so that small token counts (decode: one token per
+// sequence) still spread over many SMs.
 // RUN = tokens per conv work item (8 keeps a sliding window in registers;
 // 1 makes every token an independent item with its 4 loads in flight).
 template <typename T, int TB, int RUN>
-__global__ void __launch_bounds__(GC_THREADS)
+__global__ void __launch_bounds__(GC_THREADS, 2)
 genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __restrict__ W2,
                const T* __restrict__ v, const T* __restrict__ hist_in, T* __restrict__ v_out,
                T* __restrict__ hist_out, float* __restrict__ conv_w_out,
@@ -116,52 +145,65 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
     extern __shared__ float smem[];
     const int HW4 = H * GC_W;
     const int h0 = blockIdx.y * hpc;
-    const int nh = min(hpc, H - h0);
+    const int nh = max(0, min(hpc, H - h0));
     const int CW = nh * GC_W;                     // tap columns of this CTA
     float* zpart = smem;                          // [8][TB][32]
-    float* hs = zpart + 8 * TB * GC_HID;          // [TB][33]
+    float* zc = zpart + 8 * TB * GC_HID;          // [TB][32] this CTA's partial sum
+    float* hs = zc + TB * GC_HID;                 // [TB][33]
     float* w2s = hs + TB * (GC_HID + 1);          // [32][CW]
-    float* taps = w2s + GC_HID * CW;              // [TB][CW]
+    float* taps = w2s + GC_HID * hpc * GC_W;      // [TB][CW]
 
     const int tid = threadIdx.x;
     const long long N = (long long)Bn * Tn;
     const long long r0 = (long long)blockIdx.x * TB;
     const int nrows = (int)((N - r0) < TB ? (N - r0) : TB);
+    const int G = (int)cluster_size(), g = (int)cluster_rank();
 
     for (int i = tid; i < GC_HID * CW; i += GC_THREADS) {
         const int r = i / CW, c = i % CW;
         w2s[i] = Elem<T>::ld(W2 + (long long)r * HW4 + h0 * GC_W + c);
     }
 
-    // ---- stage A: z = x . W1, SiLU ----
+    // ---- stage A: this CTA's slice of z = x . W1 ----
+    const int nks = D / 16, per = (nks + G - 1) / G;
+    const int ks0 = min(nks, g * per), ks1 = min(nks, ks0 + per);
     if constexpr (sizeof(T) == 2) {
         gen_stageA_bf16<TB>(reinterpret_cast<const __nv_bfloat16*>(x),
-                            reinterpret_cast<const __nv_bfloat16*>(W1), r0, N, D, zpart);
+                            reinterpret_cast<const __nv_bfloat16*>(W1), r0, N, D, ks0, ks1, zpart);
         __syncthreads();
         for (int i = tid; i < TB * GC_HID; i += GC_THREADS) {
             const int t = i / GC_HID, r = i % GC_HID;
             float z = 0.f;
 #pragma unroll
             for (int w = 0; w < 8; ++w) z += zpart[(w * TB + t) * GC_HID + r];
-            hs[t * (GC_HID + 1) + r] = z / (1.0f + expf(-z));
+            zc[i] = z;
         }
     } else {
-        // float32: thread (t, 4 hidden units) in FFMA
+        // float32: thread (t, 4 hidden units) in FFMA over the slice
         for (int i = tid; i < TB * (GC_HID / 4); i += GC_THREADS) {
             const int t = i / (GC_HID / 4), r4 = (i % (GC_HID / 4)) * 4;
             float z[4] = {0.f, 0.f, 0.f, 0.f};
             if (t < nrows) {
                 const T* xr = x + (r0 + t) * D;
-                for (int d = 0; d < D; ++d) {
+                for (int d = ks0 * 16; d < ks1 * 16; ++d) {
                     const float xv = Elem<T>::ld(xr + d);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) z[e] += xv * Elem<T>::ld(W1 + (long long)d * GC_HID + r4 + e);
                 }
             }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) hs[t * (GC_HID + 1) + r4 + e] = z[e] / (1.0f + expf(-z[e]));
+            for (int e = 0; e < 4; ++e) zc[t * GC_HID + r4 + e] = z[e];
         }
     }
+    // ---- the cluster's partial sums, added in rank order by every CTA; SiLU ----
+    cluster_sync_all();
+    for (int i = tid; i < TB * GC_HID; i += GC_THREADS) {
+        const int t = i / GC_HID, r = i % GC_HID;
+        float z = 0.f;
+        for (int q = 0; q < G; ++q) z += ld_peer_f32(zc + i, (uint32_t)q);
+        hs[t * (GC_HID + 1) + r] = z / (1.0f + expf(-z));
+    }
+    cluster_sync_all();                           // peers have read this CTA's partial
     __syncthreads();
 
     // ---- stage B: taps of this CTA's heads = h . W2 ----

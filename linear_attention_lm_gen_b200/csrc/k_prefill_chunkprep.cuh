@@ -1,6 +1,6 @@
 // K2a: state-independent preparation of every chunk of the chunked Gated
 // DeltaNet prefill (Jet-Nemotron paper, section 2.3, gated delta rule in
-// chunked WY / UT form), one CTA per (sequence, head, chunk), all at once.
+// chunked WY / UT form), for all (sequence, head, chunk) items at once.
 //
 // Everything in a chunk that does not depend on the running state is a
 // function of that chunk's q, k, g and b alone, so it is computed here in
@@ -16,11 +16,14 @@
 //   Q~   [64 r][dk]      diag(gam / |q|) Q, 64-column blocks (outputs only)
 // T1, W^T and vec come first, so a pass without outputs copies a prefix.
 //
-// Flow of one CTA (256 threads, named barrier 1 = the whole CTA): TMA of the
-// K / Q tile; P1 = [K; Q] K^T on tcgen05 while the per-token vectors are
-// formed; A and P; the UT inverse; T1 / T2; P2b = K^T T2^T on tcgen05 while
-// Q~ is formed; W^T. Tiles are staged in shared memory and written with bulk
-// copies.
+// A CTA (256 threads, named barrier 1 = the whole CTA) walks items
+// blockIdx.x, blockIdx.x + gridDim.x, ... with the K / Q tiles of the next
+// two items in flight (TMA, double buffer). Per item: P1 = [K; Q] K^T on
+// tcgen05 while the per-token vectors are formed; A and P; the UT inverse;
+// T1 / T2; P2b = K^T T2^T on tcgen05 while Q~ is formed; W^T. T1, P, W^T and
+// the vectors are stored straight from registers (each warp store covers
+// whole 128-byte rows or 16-byte pieces of them), Q~ by a bulk copy from
+// its shared-memory tile.
 #pragma once
 #include "k_prefill_common.cuh"
 
@@ -47,45 +50,38 @@ struct Img {
 template <int DK>
 struct PrepSmem {
     static constexpr int NKB = (DK + 63) / 64;
-    static constexpr uint32_t KQ = 0;                              // per 64-col block [K 8K | Q 8K]
-    static constexpr uint32_t T2 = KQ + NKB * 16384;
-    static constexpr uint32_t T1 = T2 + 8192;                      // staging of the image tiles
-    static constexpr uint32_t P = T1 + 8192;
-    static constexpr uint32_t WT = P + 8192;
-    static constexpr uint32_t AF = WT + ((DK * 128 + 1023) / 1024) * 1024;
+    static constexpr uint32_t KQB = NKB * 16384;                   // one K / Q tile: [K 8K | Q 8K] per block
+    static constexpr uint32_t KQ = 0;                              // [2] tiles
+    static constexpr uint32_t T2 = KQ + 2 * KQB;
+    static constexpr uint32_t AF = T2 + 8192;
     static constexpr uint32_t XS = AF + AF_BYTES;
     static constexpr uint32_t VEC = XS + XS_BYTES;                 // 8 x 64 fp32
     static constexpr uint32_t PN = VEC + 2048;
-    static constexpr uint32_t IV = PN + 1024;                      // vec image staging
-    static constexpr uint32_t BAR = IV + 1024;
+    static constexpr uint32_t BAR = PN + 1024;
     static constexpr uint32_t TSLOT = BAR + 64;
     static constexpr uint32_t BYTES = TSLOT + 16 + 1024;           // + alignment slack
     static_assert(2 * BYTES <= 232448, "two CTAs per SM");
 };
 
+// items = B * H * nct, item = (b * H + h) * nct + c (also the image index)
 template <int DK>
 __global__ void __launch_bounds__(PREP_THREADS, 2)
 gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const float* __restrict__ g, const float* __restrict__ beta, uint8_t* __restrict__ img,
-                      int Tn, int H) {
+                      int Tn, int H, int nct, int n_items) {
     using SM = PrepSmem<DK>;
     using IM = Img<DK>;
     constexpr int NKB = SM::NKB;
     constexpr int KSTEPS = DK / 16;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM::BAR);     // 0: K/Q landed, 1: P1, 2: P2b
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM::BAR);     // 0, 1: K/Q landed; 2: P1; 3: P2b
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + SM::TSLOT);
     const int tid = threadIdx.x;
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int nct = gridDim.x;
-    const int t0 = c * C, L = min(C, Tn - t0);
-    const int z = (int)((long long)b * Tn + t0);
-    uint8_t* out = img + (((size_t)b * H + h) * nct + c) * IM::BYTES;
     constexpr uint32_t TM_XP = 0, TM_XW = 64;
 
     if (tid == 0) {
-        for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
@@ -95,96 +91,110 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = *tslot;
-    if (tid == 0) {
-        mbar_expect_tx(&bars[0], (uint32_t)(NKB * 16384));
+
+    auto z_of = [&](int item) {                      // first token row of the item in the [B*T] axis
+        const int c = item % nct, b = item / nct / H;
+        return (int)((long long)b * Tn + (long long)c * C);
+    };
+    auto issue_load = [&](int item, int buf) {       // thread 0
+        const int h = (item / nct) % H, z = z_of(item);
+        uint8_t* dst = sm + SM::KQ + buf * SM::KQB;
+        mbar_expect_tx(&bars[buf], (uint32_t)(NKB * 16384));
 #pragma unroll
         for (int kb = 0; kb < NKB; ++kb) {
-            tma_load_3d(sm + SM::KQ + kb * 16384, &tm_k, &bars[0], kb * 64, h, z);
-            tma_load_3d(sm + SM::KQ + kb * 16384 + 8192, &tm_q, &bars[0], kb * 64, h, z);
+            tma_load_3d(dst + kb * 16384, &tm_k, &bars[buf], kb * 64, h, z);
+            tma_load_3d(dst + kb * 16384 + 8192, &tm_q, &bars[buf], kb * 64, h, z);
         }
-    }
-    float gb = 0.f;
-    if (tid < 128 && (tid & 63) < L) {
-        const long long off = ((long long)z + (tid & 63)) * H + h;
-        gb = tid < 64 ? g[off] : beta[off];
+    };
+    int nld[2] = {0, 0}, ndone[2] = {0, 0};          // loads issued / consumed per buffer (thread 0)
+    int n1 = 0, n2 = 0;                               // MMA groups issued (thread 0)
+    if (tid == 0) {
+        if (blockIdx.x < n_items) { issue_load(blockIdx.x, 0); ++nld[0]; }
+        if (blockIdx.x + gridDim.x < n_items) { issue_load(blockIdx.x + gridDim.x, 1); ++nld[1]; }
     }
     Vec V = vec_from(reinterpret_cast<float*>(sm + SM::VEC));
     float* AF = reinterpret_cast<float*>(sm + SM::AF);
     float* XS = reinterpret_cast<float*>(sm + SM::XS);
     float* PN = reinterpret_cast<float*>(sm + SM::PN);
-    float* IV = reinterpret_cast<float*>(sm + SM::IV);
-    const uint64_t dK16 = sw128_desc(smem_u32(sm + SM::KQ), 16, 1024);       // [K; Q] K-major
-    const uint64_t dKmn = sw128_desc(smem_u32(sm + SM::KQ), 16384, 1024);    // K as MN-major
-    const uint64_t dT2 = sw128_desc(smem_u32(sm + SM::T2), 16, 1024);
     constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
     constexpr uint32_t ID_MNK = idesc_bf16(128, 64, true, false);
+    const uint64_t dT2 = sw128_desc(smem_u32(sm + SM::T2), 16, 1024);
 
-    bool issued1 = false, issued2 = false;           // MMA groups in flight (thread 0)
-    bool ok = mbar_wait(&bars[0], 0);
-    if ((ok = __syncthreads_and(ok))) {
+    bool ok = true;
+    int k = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
+        const int buf = k & 1;
+        uint8_t* KQ = sm + SM::KQ + buf * SM::KQB;
+        const int c = item % nct, h = (item / nct) % H;
+        const int L = min(C, Tn - c * C);
+        const int z = z_of(item);
+        uint8_t* out = img + (size_t)item * IM::BYTES;
+        float gb = 0.f;
+        if (tid < 128 && (tid & 63) < L) {
+            const long long off = ((long long)z + (tid & 63)) * H + h;
+            gb = tid < 64 ? g[off] : beta[off];
+        }
+        if (!(ok = __syncthreads_and(mbar_wait(&bars[buf], (uint32_t)(k >> 1) & 1)))) break;
         if (tid == 0) {   // P1: [K; Q] K^T -> XP
+            ++ndone[buf];
             tc_fence_after();
+            const uint64_t dK16 = sw128_desc(smem_u32(KQ), 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < KSTEPS; ++kk) {
                 const uint64_t d = dK16 + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
                 mma_bf16_ss(tb + TM_XP, d, d, ID_KK, kk > 0);
             }
-            mma_commit(&bars[1]);
-            issued1 = true;
+            mma_commit(&bars[2]);
+            ++n1;
         }
-        prep_vectors<DK>(sm + SM::KQ, V, PN, gb, L, tid, 1);
-        ok = mbar_wait(&bars[1], 0);
-    }
-    if ((ok = __syncthreads_and(ok))) {
+        prep_vectors<DK>(KQ, V, PN, gb, L, tid, 1);
+        if (!(ok = __syncthreads_and(mbar_wait(&bars[2], (uint32_t)k & 1)))) break;
         tc_fence_after();
-        prep_e1(tb + TM_XP, V, AF, sm + SM::P, tid);
+        prep_e1(tb + TM_XP, V, AF, out + IM::P, tid);
         named_sync(1, PREP_THREADS);
         ut_inverse(AF, XS, tid, 1);
-        prep_t1t2(AF, V, sm + SM::T1, sm + SM::T2, tid);
-        if (tid < 64) IV[tid] = V.dcy[tid] * V.ik[tid];
-        else if (tid == 64) IV[64] = V.gam[L - 1];
+        prep_t1t2(AF, V, out + IM::T1, sm + SM::T2, tid);
+        if (tid < 64) reinterpret_cast<float*>(out + IM::VEC)[tid] = V.dcy[tid] * V.ik[tid];
+        else if (tid == 64) reinterpret_cast<float*>(out + IM::VEC)[64] = V.gam[L - 1];
         fence_async_smem();
         tc_fence_before();
         named_sync(1, PREP_THREADS);
-        if (tid == 0) {   // P2b: K^T T2^T -> XW; the finished tiles go out
+        if (tid == 0) {   // P2b: K^T T2^T -> XW
             tc_fence_after();
+            const uint64_t dKmn = sw128_desc(smem_u32(KQ), 16384, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ss(tb + TM_XW, dKmn + (uint64_t)(kk * 2048 >> 4), dT2 + (uint64_t)(kk * 32 >> 4), ID_MNK,
                             kk > 0);
-            mma_commit(&bars[2]);
-            issued2 = true;
-            bulk_store(out + IM::T1, sm + SM::T1, 8192);
-            bulk_store(out + IM::VEC, sm + SM::IV, 1024);
-            bulk_store(out + IM::P, sm + SM::P, 8192);
-            bulk_commit();
+            mma_commit(&bars[3]);
+            ++n2;
         }
-        prep_qtilde<DK>(sm + SM::KQ, V, tid);           // P1 has read Q; P2b reads only K
+        prep_qtilde<DK>(KQ, V, tid);                    // P1 has read Q; P2b reads only K
         fence_async_smem();
         named_sync(1, PREP_THREADS);
         if (tid == 0) {
 #pragma unroll
-            for (int kb = 0; kb < NKB; ++kb) bulk_store(out + IM::Q + kb * 8192, sm + SM::KQ + kb * 16384 + 8192, 8192);
+            for (int kb = 0; kb < NKB; ++kb) bulk_store(out + IM::Q + kb * 8192, KQ + kb * 16384 + 8192, 8192);
             bulk_commit();
         }
-        ok = mbar_wait(&bars[2], 0);
-        if ((ok = __syncthreads_and(ok))) {
-            tc_fence_after();
-            prep_wt<DK>(tb + TM_XW, sm + SM::WT, tid);
-            fence_async_smem();
-            named_sync(1, PREP_THREADS);
-            if (tid == 0) {
-                bulk_store(out + IM::WT, sm + SM::WT, DK * 128);
-                bulk_commit();
-            }
+        if (!(ok = __syncthreads_and(mbar_wait(&bars[3], (uint32_t)k & 1)))) break;
+        tc_fence_after();
+        prep_wt<DK>(tb + TM_XW, out + IM::WT, tid);
+        tc_fence_before();
+        named_sync(1, PREP_THREADS);                    // XP, XW, T2 and KQ[buf] free (but for the Q~ copy)
+        if (tid == 0 && item + 2 * (int)gridDim.x < n_items) {
+            bulk_wait_read_all();                       // the Q~ copy has read KQ[buf]
+            issue_load(item + 2 * gridDim.x, buf);
+            ++nld[buf];
         }
     }
     if (tid == 0) {
         bulk_wait_all();             // shared memory stays valid until the copies have read it
         if (!ok) {                   // a wait ran out: let issued loads / MMAs finish (bounded)
-            mbar_wait(&bars[0], 0);
-            if (issued1) mbar_wait(&bars[1], 0);
-            if (issued2) mbar_wait(&bars[2], 0);
+            for (int q = 0; q < 2; ++q)
+                if (nld[q] > ndone[q]) mbar_wait(&bars[q], (uint32_t)(nld[q] - 1) & 1);
+            if (n1 > 0) mbar_wait(&bars[2], (uint32_t)(n1 - 1) & 1);
+            if (n2 > 0) mbar_wait(&bars[3], (uint32_t)(n2 - 1) & 1);
         }
     }
     tc_fence_before();
