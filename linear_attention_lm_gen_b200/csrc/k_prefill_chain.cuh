@@ -14,12 +14,16 @@
 //   warps 0-3  CHAIN  E4: S -> bf16 copy and S <- gam_L S;  E5: Wt^T -> bf16
 //                     (plain and scaled by d/|k|)
 //   warps 4-7  OUT    E6: O^T (TMEM) -> staging -> global, off the chain
-//   warp  8    CTRL   one thread: bulk copies of the images, TMA of K and V,
-//                     every tcgen05 MMA, in a fixed dependency order
+//   warp  8    MMA    one thread issues every tcgen05 MMA in a fixed order
+//   warp  9    LOAD   one thread issues the bulk copies of the images and the
+//                     TMA loads of K and V as soon as their buffers are free
 //
 // Buffers: images double-buffered (the copy of chunk c+2 starts once chunk c
-// is finished), K and V single (K(c+1) once P4(c) is done, V(c+1) once P2a(c)
-// is done). TMEM: S, X1[2] (U^T then Wt^T), X2[2] (O^T) = 384 of 512 columns.
+// is finished), V single (V(c+1) once P2a(c) is done), K double-buffered for
+// dk <= 96 (K(c+2) once P4(c) is done) and single for dk = 128 (K(c+1) once
+// P4(c) is done; shared memory is full). TMEM: S, X1[2] (U^T then Wt^T),
+// X2[2] (O^T) = 384 of 512 columns. Waits spin on the mbarrier before they
+// start to sleep between polls, so a waiter wakes within tens of cycles.
 // Segments (sequence parallelism) work as in the fused kernel: see Seg.
 #pragma once
 #include "k_prefill_chunkprep.cuh"
@@ -30,16 +34,26 @@ namespace pfch {
 using namespace pfws;
 
 constexpr int NCH_T = 128, NOUT = 128;
-constexpr int THREADS = NCH_T + NOUT + 32;            // 288
-constexpr int OUT0 = NCH_T, CTRL0 = NCH_T + NOUT;
+constexpr int THREADS = NCH_T + NOUT + 64;            // 320
+constexpr int OUT0 = NCH_T, MMA0 = NCH_T + NOUT, LOAD0 = MMA0 + 32;
+
+// bounded wait: spin on the phase first, then poll with short sleeps; gives up
+// (error word + CTA abort flag) when the poll budget runs out or another
+// thread raised the abort flag
+__device__ __forceinline__ bool wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    for (uint32_t i = 0; i < 2048; ++i)
+        if (mbar_test_wait(bar, parity)) return true;
+    return wait_bar(bar, parity, abort_flag);
+}
 
 template <int DK>
 struct ChainSmem {
     static constexpr int NKB = (DK + 63) / 64;
+    static constexpr int NKBUF = DK <= 96 ? 2 : 1;           // K tiles in flight
     static constexpr uint32_t IB = ((Img<DK>::BYTES + 1023) / 1024) * 1024;
     static constexpr uint32_t IMG = 0;                       // [2] images
-    static constexpr uint32_t K = IMG + 2 * IB;              // NKB x [64 tok][64 feat]
-    static constexpr uint32_t V = K + NKB * 8192;            // 2 x [64 tok][64 ch]
+    static constexpr uint32_t K = IMG + 2 * IB;              // [NKBUF] x NKB x [64 tok][64 feat]
+    static constexpr uint32_t V = K + NKBUF * NKB * 8192;    // 2 x [64 tok][64 ch]
     static constexpr uint32_t AS = V + 16384;                // NKB x [128 rows][64 feat] bf16 S
     static constexpr uint32_t AW = AS + NKB * 16384;         // Wt^T
     static constexpr uint32_t AWD = AW + 16384;              // Wt^T diag(d/|k|)
@@ -55,15 +69,15 @@ constexpr uint32_t TM_S = 0, TM_X1 = 128, TM_X2 = 256, TM_COLS = 512;
 
 enum {
     B_IMG = 0,        // [2] image landed
-    B_K = 2,          // K tile landed
-    B_V = 3,          // V tile landed
-    B_P2 = 4,         // P2a complete
-    B_P3 = 5,         // P3 (and P5a) complete
-    B_SDONE = 6,      // [2] P4 / P5b complete
-    B_AS = 8,         // bf16 S written, S scaled (chain)
-    B_AW = 9,         // Wt^T copies written (chain)
-    B_X2FREE = 10,    // [2] O^T read (out)
-    NBARS = 12
+    B_K = 2,          // [NKBUF] K tile landed
+    B_V = 4,          // V tile landed
+    B_P2 = 5,         // P2a complete
+    B_P3 = 6,         // P3 (and P5a) complete
+    B_SDONE = 7,      // [2] P4 / P5b complete
+    B_AS = 9,         // bf16 S written, S scaled (chain)
+    B_AW = 10,        // Wt^T copies written (chain)
+    B_X2FREE = 11,    // [2] O^T read (out)
+    NBARS = 13
 };
 
 template <int DK>
@@ -103,7 +117,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (tid == CTRL0) {
+    if (tid == LOAD0) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
@@ -137,8 +151,8 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         for (int c = 0; c < nch; ++c) {
             const int p = c & 1;
             const float* iv = reinterpret_cast<const float*>(img_at(c) + IM::VEC);   // dik[64], gam_{L-1}
-            bool okw = c < 1 || wait_bar(&bars[B_SDONE + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag);
-            okw = okw && wait_bar(&bars[B_IMG + p], (c >> 1) & 1, abort_flag);
+            bool okw = c < 1 || wait_spin(&bars[B_SDONE + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag);
+            okw = okw && wait_spin(&bars[B_IMG + p], (c >> 1) & 1, abort_flag);
             if (!group_all(2, NCH_T, okw)) break;
             tc_fence_after();
             // ---- E4: S -> bf16 copy, S <- gam_L S
@@ -168,7 +182,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             named_sync(2, NCH_T);
             if (ct == 0) arrive(&bars[B_AS]);
             // ---- E5: Wt^T -> bf16 (plain and scaled by d/|k|)
-            if (!group_all(2, NCH_T, wait_bar(&bars[B_P3], c & 1, abort_flag))) break;
+            if (!group_all(2, NCH_T, wait_spin(&bars[B_P3], c & 1, abort_flag))) break;
             tc_fence_after();
             {
                 const uint32_t x1 = TM_X1 + (uint32_t)p * 64;
@@ -201,7 +215,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         }
         // final state of the segment (after the last P4)
         const bool fin = !*abort_flag && nch > 0 &&
-                         wait_bar(&bars[B_SDONE + ((nch - 1) & 1)], ((nch - 1) >> 1) & 1, abort_flag);
+                         wait_spin(&bars[B_SDONE + ((nch - 1) & 1)], ((nch - 1) >> 1) & 1, abort_flag);
         if (group_all(2, NCH_T, fin)) {
             tc_fence_after();
             float* dst = nullptr;
@@ -233,7 +247,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sm + SM::OUT);
             const long long tstride = (long long)H * dv;
             for (int c = 0; c < nch; ++c) {
-                if (!group_all(3, NOUT, wait_bar(&bars[B_SDONE + (c & 1)], (c >> 1) & 1, abort_flag))) break;
+                if (!group_all(3, NOUT, wait_spin(&bars[B_SDONE + (c & 1)], (c >> 1) & 1, abort_flag))) break;
                 tc_fence_after();
                 const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
 #pragma unroll
@@ -259,16 +273,19 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 named_sync(3, NOUT);                         // staging free again
             }
         }
-    } else if (tid == CTRL0) {
-        // =============================================================== CTRL
-        // Fixed order (every awaited event depends only on actions issued
-        // earlier in this order):
-        //   prologue: IMG(0) K(0) V(0) IMG(1) P2a(0)
-        //   chunk c:  P3(c) [P5a(c)]  V(c+1)  P4(c) [P5b(c)]  P2a(c+1)  K(c+1) IMG(c+2)
-        const uint32_t img_bytes = write_o ? IM::BYTES : IM::A_BYTES;
+    } else if (tid == MMA0 || tid == LOAD0) {
+        // =============================================================== MMA / LOAD
+        // Fixed orders (every awaited event depends only on actions issued
+        // earlier in these orders or by the other warps):
+        //   MMA:   P2a(0);  chunk c: P3(c) [P5a(c)]  P4(c) [P5b(c)]  P2a(c+1)
+        //   LOAD:  IMG(0) K(0) V(0) IMG(1) [K(1)];  chunk c: V(c+1) after P2a(c),
+        //          K(c+NKBUF) and IMG(c+2) after P4(c)
+        constexpr int NKBUF = SM::NKBUF;
         bool ok = true;
         auto W = [&](int bar, int phase) {
             if (!ok) return false;
+            for (uint32_t i = 0; i < 4096u; ++i)
+                if (mbar_test_wait(&bars[bar], (uint32_t)phase & 1u)) return true;
             for (uint32_t i = 0; i < 4u * kWaitPolls; ++i) {
                 if (mbar_test_wait(&bars[bar], (uint32_t)phase & 1u)) return true;
                 if ((i & 1023u) == 1023u && *abort_flag) { ok = false; return false; }
@@ -279,94 +296,108 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             ok = false;
             return false;
         };
-        auto zrow = [&](int c) { return (int)((long long)b * Tn + tbeg + (long long)c * C); };
-        auto load_img = [&](int c) {
-            uint64_t* bar = &bars[B_IMG + (c & 1)];
-            mbar_expect_tx(bar, img_bytes);
-            bulk_load(const_cast<uint8_t*>(img_at(c)), img_bh + (size_t)(cbeg + c) * IM::BYTES, img_bytes, bar);
-        };
-        auto load_k = [&](int c) {
-            mbar_expect_tx(&bars[B_K], (uint32_t)(NKB * 8192));
+        if (tid == LOAD0) {
+            const uint32_t img_bytes = write_o ? IM::BYTES : IM::A_BYTES;
+            auto zrow = [&](int c) { return (int)((long long)b * Tn + tbeg + (long long)c * C); };
+            auto load_img = [&](int c) {
+                uint64_t* bar = &bars[B_IMG + (c & 1)];
+                mbar_expect_tx(bar, img_bytes);
+                bulk_load(const_cast<uint8_t*>(img_at(c)), img_bh + (size_t)(cbeg + c) * IM::BYTES, img_bytes, bar);
+            };
+            auto load_k = [&](int c) {
+                const int kb_ = c % NKBUF;
+                uint64_t* bar = &bars[B_K + kb_];
+                mbar_expect_tx(bar, (uint32_t)(NKB * 8192));
 #pragma unroll
-            for (int kb = 0; kb < NKB; ++kb) tma_load_3d(sm + SM::K + kb * 8192, &tm_k, &bars[B_K], kb * 64, h, zrow(c));
-        };
-        auto load_v = [&](int c) {
-            mbar_expect_tx(&bars[B_V], 16384);
-            tma_load_3d(sm + SM::V, &tm_v, &bars[B_V], c0, h, zrow(c));
-            tma_load_3d(sm + SM::V + 8192, &tm_v, &bars[B_V], c0 + 64, h, zrow(c));
-        };
-        const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
-        const uint64_t dImgMN = sw128_desc(smem_u32(sm + SM::IMG), 8192, 1024);   // W^T (MN-major)
-        const uint64_t dKmn = sw128_desc(smem_u32(sm + SM::K), 8192, 1024);       // K as MN-major
-        const uint64_t dV = sw128_desc(smem_u32(sm + SM::V), 8192, 1024);
-        const uint64_t dAS = sw128_desc(smem_u32(sm + SM::AS), 16, 1024);
-        const uint64_t dAW = sw128_desc(smem_u32(sm + SM::AW), 16, 1024);
-        const uint64_t dAWD = sw128_desc(smem_u32(sm + SM::AWD), 16, 1024);
-        constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
-        constexpr uint32_t ID_MNK = idesc_bf16(128, 64, true, false);
-        constexpr uint32_t ID_NEG = idesc_bf16(128, 64, false, true, true);
-        constexpr uint32_t ID_S = idesc_bf16(128, DK, false, true);
-        auto ioff = [&](int c, uint32_t off) { return (uint64_t)((((uint32_t)(c & 1) * SM::IB) + off) >> 4); };
-        auto mma_p2a = [&](int c) {
-            const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tb + x1, dV + (uint64_t)(kk * 2048 >> 4), dImg + ioff(c, IM::T1 + kk * 32), ID_MNK, kk > 0);
-            mma_commit(&bars[B_P2]);
-        };
-        auto mma_p3 = [&](int c) {
-            const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64, x2 = TM_X2 + (uint32_t)(c & 1) * 64;
-#pragma unroll
-            for (int kk = 0; kk < KSTEPS; ++kk)
-                mma_bf16_ss(tb + x1, dAS + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                            dImgMN + ioff(c, IM::WT + kk * 2048), ID_NEG, 1);
-            mma_commit(&bars[B_P3]);        // the chain waits for Wt^T only
-            if (!write_o) return;
-#pragma unroll
-            for (int kk = 0; kk < KSTEPS; ++kk)
-                mma_bf16_ss(tb + x2, dAS + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                            dImg + ioff(c, IM::Q + (kk >> 2) * 8192 + (kk & 3) * 32), ID_KK, kk > 0);
-        };
-        auto mma_p4 = [&](int c) {
-            const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tb + TM_S, dAWD + (uint64_t)(kk * 32 >> 4), dKmn + (uint64_t)(kk * 2048 >> 4), ID_S, 1);
-            if (write_o) {
+                for (int kb = 0; kb < NKB; ++kb)
+                    tma_load_3d(sm + SM::K + (kb_ * NKB + kb) * 8192, &tm_k, bar, kb * 64, h, zrow(c));
+            };
+            auto load_v = [&](int c) {
+                mbar_expect_tx(&bars[B_V], 16384);
+                tma_load_3d(sm + SM::V, &tm_v, &bars[B_V], c0, h, zrow(c));
+                tma_load_3d(sm + SM::V + 8192, &tm_v, &bars[B_V], c0 + 64, h, zrow(c));
+            };
+            int nK = 0, nV = 0, nI = 0;                      // loads issued
+            if (nch > 0) { load_img(0); ++nI; load_k(0); ++nK; load_v(0); ++nV; }
+            if (nch > 1) { load_img(1); ++nI; }
+            if (NKBUF == 2 && nch > 1) { load_k(1); ++nK; }
+            for (int c = 0; c < nch && ok; ++c) {
+                if (c + 1 < nch && W(B_P2, c)) { load_v(c + 1); ++nV; }
+                if ((c + NKBUF < nch || c + 2 < nch) && W(B_SDONE + (c & 1), c >> 1)) {
+                    if (c + NKBUF < nch) { load_k(c + NKBUF); ++nK; }
+                    if (c + 2 < nch) { load_img(c + 2); ++nI; }
+                }
+            }
+            // every issued load has landed before the CTA can exit (the last
+            // load on each barrier; immediate unless a wait ran out)
+            if (!ok) *abort_flag = 1;
+            for (int j = max(0, nK - NKBUF); j < nK; ++j) mbar_wait(&bars[B_K + j % NKBUF], (j / NKBUF) & 1);
+            if (nV > 0) mbar_wait(&bars[B_V], (nV - 1) & 1);
+            for (int j = max(0, nI - 2); j < nI; ++j) mbar_wait(&bars[B_IMG + (j & 1)], (j >> 1) & 1);
+        } else {
+            const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
+            const uint64_t dImgMN = sw128_desc(smem_u32(sm + SM::IMG), 8192, 1024);   // W^T (MN-major)
+            const uint64_t dKmn = sw128_desc(smem_u32(sm + SM::K), 8192, 1024);       // K as MN-major
+            const uint64_t dV = sw128_desc(smem_u32(sm + SM::V), 8192, 1024);
+            const uint64_t dAS = sw128_desc(smem_u32(sm + SM::AS), 16, 1024);
+            const uint64_t dAW = sw128_desc(smem_u32(sm + SM::AW), 16, 1024);
+            const uint64_t dAWD = sw128_desc(smem_u32(sm + SM::AWD), 16, 1024);
+            constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
+            constexpr uint32_t ID_MNK = idesc_bf16(128, 64, true, false);
+            constexpr uint32_t ID_NEG = idesc_bf16(128, 64, false, true, true);
+            constexpr uint32_t ID_S = idesc_bf16(128, DK, false, true);
+            auto ioff = [&](int c, uint32_t off) { return (uint64_t)((((uint32_t)(c & 1) * SM::IB) + off) >> 4); };
+            auto mma_p2a = [&](int c) {
+                const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), dImg + ioff(c, IM::P + kk * 32), ID_KK, 1);
+                    mma_bf16_ss(tb + x1, dV + (uint64_t)(kk * 2048 >> 4), dImg + ioff(c, IM::T1 + kk * 32), ID_MNK,
+                                kk > 0);
+                mma_commit(&bars[B_P2]);
+            };
+            auto mma_p3 = [&](int c) {
+                const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64, x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+                for (int kk = 0; kk < KSTEPS; ++kk)
+                    mma_bf16_ss(tb + x1, dAS + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                                dImgMN + ioff(c, IM::WT + kk * 2048), ID_NEG, 1);
+                mma_commit(&bars[B_P3]);        // the chain waits for Wt^T only
+                if (!write_o) return;
+#pragma unroll
+                for (int kk = 0; kk < KSTEPS; ++kk)
+                    mma_bf16_ss(tb + x2, dAS + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                                dImg + ioff(c, IM::Q + (kk >> 2) * 8192 + (kk & 3) * 32), ID_KK, kk > 0);
+            };
+            auto mma_p4 = [&](int c) {
+                const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+                const uint64_t dk_ = dKmn + (uint64_t)(((uint32_t)(c % NKBUF) * NKB * 8192) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tb + TM_S, dAWD + (uint64_t)(kk * 32 >> 4), dk_ + (uint64_t)(kk * 2048 >> 4), ID_S, 1);
+                if (write_o) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), dImg + ioff(c, IM::P + kk * 32), ID_KK, 1);
+                }
+                mma_commit(&bars[B_SDONE + (c & 1)]);
+            };
+            int n2 = 0, n3 = 0, n4 = 0;                      // commit groups issued
+            if (nch > 0 && W(B_IMG, 0) && W(B_V, 0)) { tc_fence_after(); mma_p2a(0); ++n2; }
+            for (int c = 0; c < nch && ok; ++c) {
+                if (W(B_AS, c) && (!write_o || c < 2 || W(B_X2FREE + (c & 1), (c - 2) >> 1))) {
+                    tc_fence_after(); mma_p3(c); ++n3;
+                }
+                if (W(B_AW, c) && W(B_K + c % NKBUF, (c / NKBUF) & 1)) { tc_fence_after(); mma_p4(c); ++n4; }
+                if (c + 1 < nch && W(B_IMG + ((c + 1) & 1), (c + 1) >> 1) && W(B_V, c + 1)) {
+                    tc_fence_after(); mma_p2a(c + 1); ++n2;
+                }
             }
-            mma_commit(&bars[B_SDONE + (c & 1)]);
-        };
-        int n2 = 0, n3 = 0, n4 = 0, nK = 0, nV = 0, nI = 0;      // actions issued
-        if (nch > 0) { load_img(0); ++nI; load_k(0); ++nK; load_v(0); ++nV; }
-        if (nch > 1) { load_img(1); ++nI; }
-        if (nch > 0 && W(B_IMG, 0) && W(B_V, 0)) { tc_fence_after(); mma_p2a(0); ++n2; }
-        for (int c = 0; c < nch && ok; ++c) {
-            if (W(B_AS, c) && (!write_o || c < 2 || W(B_X2FREE + (c & 1), (c - 2) >> 1))) {
-                tc_fence_after(); mma_p3(c); ++n3;
-            }
-            if (c + 1 < nch && W(B_P2, c)) { load_v(c + 1); ++nV; }
-            if (W(B_AW, c) && W(B_K, c)) { tc_fence_after(); mma_p4(c); ++n4; }
-            if (c + 1 < nch && W(B_IMG + ((c + 1) & 1), (c + 1) >> 1) && W(B_V, c + 1)) {
-                tc_fence_after(); mma_p2a(c + 1); ++n2;
-            }
-            if (c + 1 < nch && W(B_SDONE + (c & 1), c >> 1)) {
-                load_k(c + 1); ++nK;
-                if (c + 2 < nch) { load_img(c + 2); ++nI; }
-            }
-        }
-        // drain: every issued commit group and load completes before TMEM is freed
-        if (!ok) {
-            *abort_flag = 1;
+            // every issued commit group has completed before TMEM is freed (the
+            // last group on each barrier; immediate unless a wait ran out)
+            if (!ok) *abort_flag = 1;
             if (n2 > 0) mbar_wait(&bars[B_P2], (n2 - 1) & 1);
             if (n3 > 0) mbar_wait(&bars[B_P3], (n3 - 1) & 1);
-            if (n4 > 0) mbar_wait(&bars[B_SDONE + ((n4 - 1) & 1)], ((n4 - 1) >> 1) & 1);
-            if (nK > 0) mbar_wait(&bars[B_K], (nK - 1) & 1);
-            if (nV > 0) mbar_wait(&bars[B_V], (nV - 1) & 1);
-            if (nI > 0) mbar_wait(&bars[B_IMG + ((nI - 1) & 1)], ((nI - 1) >> 1) & 1);
-            if (nI > 1) mbar_wait(&bars[B_IMG + ((nI - 2) & 1)], ((nI - 2) >> 1) & 1);
+            for (int j = max(0, n4 - 2); j < n4; ++j) mbar_wait(&bars[B_SDONE + (j & 1)], (j >> 1) & 1);
         }
     }
     tc_fence_before();
