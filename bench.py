@@ -148,27 +148,33 @@ class Workload:
         d = synth.decode_inputs(DECODE, seed=seed + 1)
         self.host_p = {k: T(v).pin_memory() for k, v in p.items() if isinstance(v, np.ndarray)}
         self.host_d = {k: T(v).pin_memory() for k, v in d.items() if isinstance(v, np.ndarray)}
-        self.p = {k: v.to(device) for k, v in self.host_p.items()}
+        # two device copies of the prefill inputs (the end-to-end pass copies the
+        # next step's inputs in while the current step runs)
+        self.pb = [{k: v.to(device) for k, v in self.host_p.items()} for _ in range(2)]
+        self.p = self.pb[0]
         self.d = {k: v.to(device) for k, v in self.host_d.items()}
         P, Dc = PREFILL, DECODE
         bf = torch.bfloat16
         self.vc = torch.empty((P.B, P.T, P.H, P.dv), device=device, dtype=bf)
-        self.o = torch.empty_like(self.vc)
+        self.ob = [torch.empty_like(self.vc) for _ in range(2)]
+        self.o = self.ob[0]
         self.S_out = torch.empty((P.B, P.H, P.dv, P.dk), device=device, dtype=torch.float32)
         self.S = self.d["S0"].clone()
         self.hist = [self.d["hist"].clone(), torch.empty_like(self.d["hist"])]
         self.vc_d = torch.empty((Dc.B, 1, Dc.H, Dc.dv), device=device, dtype=bf)
-        self.o_d = torch.empty((Dc.B, Dc.H, Dc.dv), device=device, dtype=bf)
+        self.odb = [torch.empty((Dc.B, Dc.H, Dc.dv), device=device, dtype=bf) for _ in range(2)]
+        self.o_d = self.odb[0]
         ws = jet.jet_gdn_prefill_workspace_size(P.B, P.T, P.H, P.dk, P.dv)
         self.ws = torch.empty(max(ws, 16), device=device, dtype=torch.uint8)
         # pinned host buffers for the end-to-end pass
-        self.h_o = torch.empty(self.o.shape, dtype=bf).pin_memory()
-        self.h_o_d = torch.empty(self.o_d.shape, dtype=bf).pin_memory()
+        self.h_o = [torch.empty(self.o.shape, dtype=bf).pin_memory() for _ in range(2)]
+        self.h_o_d = [torch.empty(self.o_d.shape, dtype=bf).pin_memory() for _ in range(2)]
         self.steps_done = 0
 
     # four calls: K1 prefill, K2 prefill (prep + chain phases), K1 decode, K3 decode
-    def step(self, stream, i: int, ev=None, counts=None):
-        jet, p, d = self.jet, self.p, self.d
+    def step(self, stream, i: int, ev=None, counts=None, buf: int = 0):
+        jet, p, d = self.jet, self.pb[buf], self.d
+        o, o_d = self.ob[buf], self.odb[buf]
 
         def mark(j):
             if ev is not None:
@@ -178,7 +184,7 @@ class Workload:
         mark(0)
         jet.jet_dyn_conv_v(p["x"], p["W1"], p["W2"], p["v"], None, self.vc, stream=stream)
         mark(1)
-        jet.jet_gdn_prefill(p["q"], p["k"], self.vc, p["g"], p["beta"], None, self.o, self.S_out, self.ws,
+        jet.jet_gdn_prefill(p["q"], p["k"], self.vc, p["g"], p["beta"], None, o, self.S_out, self.ws,
                             stream=stream)
         mark(2)
         s = i % DECODE.steps
@@ -186,26 +192,28 @@ class Workload:
         jet.jet_dyn_conv_v(d["x"][s][:, None], d["W1"], d["W2"], d["v"][s][:, None], hin, self.vc_d, hout,
                            stream=stream)
         mark(3)
-        jet.jet_gdn_decode_step(d["q"][s], d["k"][s], self.vc_d[:, 0], d["g"][s], d["beta"][s], self.S, self.o_d,
+        jet.jet_gdn_decode_step(d["q"][s], d["k"][s], self.vc_d[:, 0], d["g"][s], d["beta"][s], self.S, o_d,
                                 stream=stream)
         mark(4)
 
-    def h2d(self, stream, i: int) -> int:
-        """Copy one step's inputs from pinned host memory; returns bytes."""
+    def h2d(self, i: int, buf: int) -> int:
+        """Copy one step's inputs from pinned host memory (current stream); returns bytes."""
         n = 0
+        p = self.pb[buf]
         for k in ("x", "q", "k", "v", "g", "beta"):
-            self.p[k].copy_(self.host_p[k], non_blocking=True)
-            n += self.p[k].numel() * self.p[k].element_size()
+            p[k].copy_(self.host_p[k], non_blocking=True)
+            n += p[k].numel() * p[k].element_size()
         s = i % DECODE.steps
         for k in ("x", "q", "k", "v", "g", "beta"):
             self.d[k][s].copy_(self.host_d[k][s], non_blocking=True)
             n += self.d[k][s].numel() * self.d[k][s].element_size()
         return n
 
-    def d2h(self, stream) -> int:
-        self.h_o.copy_(self.o, non_blocking=True)
-        self.h_o_d.copy_(self.o_d, non_blocking=True)
-        return self.o.numel() * 2 + self.o_d.numel() * 2
+    def d2h(self, buf: int) -> int:
+        """Read one step's outputs back into pinned host memory (current stream); returns bytes."""
+        self.h_o[buf].copy_(self.ob[buf], non_blocking=True)
+        self.h_o_d[buf].copy_(self.odb[buf], non_blocking=True)
+        return self.ob[buf].numel() * 2 + self.odb[buf].numel() * 2
 
 
 # ------------------------------------------------------------------ CPU oracle leg
@@ -350,17 +358,39 @@ def run_jet(args):
     if jet.jet_device_error(stream) != 0:
         raise RuntimeError("device error word set in the timed region")
 
-    # ---- end-to-end pass: host inputs in, results out, through the same calls
+    # ---- end-to-end pass: host inputs in, results out, through the same calls.
+    # Every step copies its own inputs from pinned host memory and reads its
+    # outputs back; the copies of step i+1's inputs and of step i-1's outputs
+    # run on their own streams while step i computes (double-buffered).
     barrier()
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
     h2d = d2h = 0
-    with torch.cuda.stream(stream):
-        e_start.record(stream)
-        for i in range(args.steps):
-            h2d = wl.h2d(stream, i)
-            wl.step(stream, args.warmup + args.steps + i)
-            d2h = wl.d2h(stream)
-        e_stop.record(stream)
+    e_start.record(stream)
+    s_in.wait_event(e_start)
+    for i in range(args.steps):
+        j = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(comp_done[j])          # step i-2 has consumed buffer j
+            h2d = wl.h2d(args.warmup + args.steps + i, j)
+            in_ready[j].record(s_in)
+        stream.wait_event(in_ready[j])
+        if i >= 2:
+            stream.wait_event(out_done[j])             # step i-2's outputs have been read back
+        with torch.cuda.stream(stream):
+            wl.step(stream, args.warmup + args.steps + i, buf=j)
+        comp_done[j].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[j])
+            d2h = wl.d2h(j)
+            out_done[j].record(s_out)
+    for j in range(min(2, args.steps)):
+        stream.wait_event(out_done[j])
+    e_stop.record(stream)
     barrier()
     e_ms = max_over_ranks(e_start.elapsed_time(e_stop))
 

@@ -120,20 +120,24 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     constexpr uint32_t ID_MNK = idesc_bf16(128, 64, true, false);
     const uint64_t dT2 = sw128_desc(smem_u32(sm + SM::T2), 16, 1024);
 
+    // g (tid < 64) or b (64 <= tid < 128) of one token of an item, 0 past the sequence end
+    auto load_gb = [&](int item) -> float {
+        if (item >= n_items || tid >= 128) return 0.f;
+        const int c = item % nct, h = (item / nct) % H;
+        if ((tid & 63) >= min(C, Tn - c * C)) return 0.f;
+        const long long off = ((long long)z_of(item) + (tid & 63)) * H + h;
+        return tid < 64 ? g[off] : beta[off];
+    };
     bool ok = true;
     int k = 0;
+    float gb_next = load_gb(blockIdx.x);
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
         const int buf = k & 1;
         uint8_t* KQ = sm + SM::KQ + buf * SM::KQB;
-        const int c = item % nct, h = (item / nct) % H;
-        const int L = min(C, Tn - c * C);
-        const int z = z_of(item);
+        const int L = min(C, Tn - (item % nct) * C);
         uint8_t* out = img + (size_t)item * IM::BYTES;
-        float gb = 0.f;
-        if (tid < 128 && (tid & 63) < L) {
-            const long long off = ((long long)z + (tid & 63)) * H + h;
-            gb = tid < 64 ? g[off] : beta[off];
-        }
+        const float gb = gb_next;
+        gb_next = load_gb(item + gridDim.x);            // in flight during this item
         if (!(ok = __syncthreads_and(mbar_wait(&bars[buf], (uint32_t)(k >> 1) & 1)))) break;
         if (tid == 0) {   // P1: [K; Q] K^T -> XP
             ++ndone[buf];

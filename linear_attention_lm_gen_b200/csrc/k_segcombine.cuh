@@ -10,9 +10,9 @@
 // in float32. It also copies S0 (or zeros) to S_start(0), so that phase C never
 // reads S0 while the last segment may be writing a final state that aliases it.
 //
-// Rows of S are independent: a CTA owns 32 rows of one (sequence, head) and
-// walks p sequentially. Thread (j, g) owns column j of rows 8g .. 8g+7, so its
-// eight accumulators are independent FMA chains; the 32 running rows sit in
+// Rows of S are independent: a CTA owns 16 rows of one (sequence, head) and
+// walks p sequentially. Thread (j, g) owns column j of rows 4g .. 4g+3, so its
+// four accumulators are independent FMA chains; the 16 running rows sit in
 // shared memory (read as broadcast float4), and A_p arrives by one bulk copy
 // into a double buffer, the copy of A_{p+1} in flight while step p computes.
 #pragma once
@@ -21,8 +21,8 @@
 
 namespace jet {
 
-constexpr int SC_ROWS = 32;      // state rows per CTA
-constexpr int SC_RPT = 8;        // rows per thread
+constexpr int SC_ROWS = 16;      // state rows per CTA
+constexpr int SC_RPT = 4;        // rows per thread
 constexpr int SC_GROUPS = SC_ROWS / SC_RPT;
 
 __host__ __device__ constexpr int sc_threads(int dk) { return SC_GROUPS * dk; }
@@ -31,14 +31,14 @@ __host__ __device__ constexpr size_t sc_smem_bytes(int dk) {
 }
 
 // E [B][P-1][H][dv][dk], A [B][P-1][H][dk][dk], Sst [B][P][H][dv][dk];
-// grid (dv / 32, H, B), sc_threads(DK) threads, sc_smem_bytes(DK) shared.
+// grid (dv / 16, H, B), sc_threads(DK) threads, sc_smem_bytes(DK) shared.
 template <int DK>
 __global__ void __launch_bounds__(SC_GROUPS * DK)
 seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, const float* S0,
                    float* __restrict__ Sst, int P, int H, int dv) {
     extern __shared__ __align__(128) float scm[];
     float* As = scm;                                  // [2][DK][DK]
-    float* Es = As + 2 * DK * DK;                     // [32][DK] running rows
+    float* Es = As + 2 * DK * DK;                     // [16][DK] running rows
     uint64_t* bar = reinterpret_cast<uint64_t*>(Es + SC_ROWS * DK);
     constexpr uint32_t ABYTES = DK * DK * sizeof(float);
     const int tid = threadIdx.x, j = tid % DK, grp = tid / DK;
