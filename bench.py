@@ -71,24 +71,24 @@ def model_bytes():
     }
 
 
-def csrc_digest():
+def csrc_digest(files):
+    """Digest of the kernel sources a measurement depends on."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "linear_attention_lm_gen_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in sorted(files):
         h.update(f.encode())
         h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, only if it was taken
-    on the current kernel sources."""
+    """DRAM bytes per launch (read + write) from a committed ncu summary, only
+    if it was taken on the current sources of that kernel."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    ent = d.get(kernel)
-    if not ent or ent.get("csrc_sha") != csrc_digest():
+    ent = json.load(open(p)).get(kernel)
+    if not ent or ent.get("sources_sha") != csrc_digest(ent.get("sources", [])):
         return None
     return ent.get("dram_bytes_per_launch")
 
