@@ -238,31 +238,32 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
         // window: win[0] = v_{t-1}, win[1] = v_{t-2}, win[2] = v_{t-3}
         uint4 wraw[3];
         uint4 cur[RUN];
+        const long long rr0 = r0 + ta;
+        int bseq = (int)(rr0 / Tn);                    // one division per item; then stepped
+        int tpos0 = (int)(rr0 - (long long)bseq * Tn);
         {
-            const long long rr = r0 + ta;
-            const int bseq = (int)(rr / Tn);
-            const long long tpos = rr % Tn;
 #pragma unroll
             for (int j = 0; j < 3; ++j) {
-                const long long tau = tpos - 1 - j;
+                const int tau = tpos0 - 1 - j;
                 wraw[j] = make_uint4(0, 0, 0, 0);
-                if (tau >= 0) wraw[j] = *reinterpret_cast<const uint4*>(v + (rr - 1 - j) * rowstride + coff);
+                if (tau >= 0) wraw[j] = *reinterpret_cast<const uint4*>(v + (rr0 - 1 - j) * rowstride + coff);
                 else if (hist_in) wraw[j] = *reinterpret_cast<const uint4*>(hist_in + ((long long)bseq * 3 + (3 + tau)) * rowstride + coff);
             }
 #pragma unroll
             for (int i = 0; i < RUN; ++i)
-                if (ta + i < tb) cur[i] = *reinterpret_cast<const uint4*>(v + (rr + i) * rowstride + coff);
+                if (ta + i < tb) cur[i] = *reinterpret_cast<const uint4*>(v + (rr0 + i) * rowstride + coff);
         }
         float win[3][VN];
 #pragma unroll
         for (int j = 0; j < 3; ++j) V16::unpack(wraw[j], win[j]);
+        int tpos = tpos0;
 #pragma unroll
         for (int i = 0; i < RUN; ++i) {
             if (ta + i >= tb) break;
-            const long long rr = r0 + ta + i;
-            const long long tpos = rr % Tn;
-            const int bseq = (int)(rr / Tn);
-            if (RUN > 1 && tpos == 0 && i > 0) {   // a new sequence starts inside the run
+            const long long rr = rr0 + i;
+            if (RUN > 1 && i > 0 && tpos == Tn) {      // a new sequence starts inside the run
+                tpos = 0;
+                ++bseq;
 #pragma unroll
                 for (int j = 0; j < 3; ++j) {
                     uint4 u = make_uint4(0, 0, 0, 0);
@@ -285,6 +286,7 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
                 for (int j = 0; j < 3; ++j)
                     *reinterpret_cast<uint4*>(hist_out + ((long long)bseq * 3 + (2 - j)) * rowstride + coff) = V16::pack(win[j]);
             }
+            ++tpos;
         }
     }
 }
