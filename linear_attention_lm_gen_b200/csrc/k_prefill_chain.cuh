@@ -14,16 +14,20 @@
 //   warps 0-3  CHAIN  E4: S -> bf16 copy and S <- gam_L S;  E5: Wt^T -> bf16
 //                     (plain and scaled by d/|k|)
 //   warps 4-7  OUT    E6: O^T (TMEM) -> staging -> global, off the chain
-//   warp  8    MMA    one thread issues every tcgen05 MMA in a fixed order
-//   warp  9    LOAD   one thread issues the bulk copies of the images and the
-//                     TMA loads of K and V as soon as their buffers are free
+//   warp  8    MMA    one thread issues the MMAs on the state chain (P3, P4)
+//   warp  9    LOAD   one thread issues the bulk copies of the images, the TMA
+//                     loads of K and V as soon as their buffers are free, and
+//                     the MMAs off the chain (P2a, P5a, P5b)
 //
 // Buffers: images double-buffered (the copy of chunk c+2 starts once chunk c
-// is finished), V single (V(c+1) once P2a(c) is done), K double-buffered for
-// dk <= 96 (K(c+2) once P4(c) is done) and single for dk = 128 (K(c+1) once
-// P4(c) is done; shared memory is full). TMEM: S, X1[2] (U^T then Wt^T),
-// X2[2] (O^T) = 384 of 512 columns. Waits spin on the mbarrier before they
-// start to sleep between polls, so a waiter wakes within tens of cycles.
+// is finished), V double-buffered (V(c+2) once P2a(c) is done), K
+// double-buffered for dk <= 96 (K(c+2) once P4(c) is done) and single for
+// dk = 128 (K(c+1) once P4(c) is done; shared memory is full); outputs are
+// staged 32 tokens at a time. TMEM: S, X1[2] (U^T then Wt^T), X2[2] (O^T) =
+// 384 of 512 columns. The roles on the critical path (chain warps, MMA
+// thread) spin on the mbarrier before they start to sleep between polls, so
+// they wake within tens of cycles; the others sleep between polls and leave
+// the issue slots to them.
 // Segments (sequence parallelism) work as in the fused kernel: see Seg.
 #pragma once
 #include "k_prefill_chunkprep.cuh"
@@ -45,6 +49,16 @@ __device__ __forceinline__ bool wait_spin(uint64_t* bar, uint32_t parity, volati
         if (mbar_test_wait(bar, parity)) return true;
     return wait_bar(bar, parity, abort_flag);
 }
+// A group waits for one mbarrier phase: its first thread polls (spinning when
+// `spin`), the others wait at the group's named barrier, which costs no issue
+// slots and keeps the shared-memory pipe free for the MMA-issuing thread.
+// True on every thread of the group iff the wait succeeded.
+__device__ __forceinline__ bool group_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int bid, int n,
+                                           bool poller, bool spin) {
+    bool ok = true;
+    if (poller) ok = spin ? wait_spin(bar, parity, abort_flag) : wait_bar(bar, parity, abort_flag);
+    return group_all(bid, n, ok);
+}
 
 template <int DK>
 struct ChainSmem {
@@ -53,15 +67,18 @@ struct ChainSmem {
     static constexpr uint32_t IB = ((Img<DK>::BYTES + 1023) / 1024) * 1024;
     static constexpr uint32_t IMG = 0;                       // [2] images
     static constexpr uint32_t K = IMG + 2 * IB;              // [NKBUF] x NKB x [64 tok][64 feat]
-    static constexpr uint32_t V = K + NKBUF * NKB * 8192;    // 2 x [64 tok][64 ch]
-    static constexpr uint32_t AS = V + 16384;                // NKB x [128 rows][64 feat] bf16 S
+    static constexpr uint32_t V = K + NKBUF * NKB * 8192;    // [2] x 2 x [64 tok][64 ch]
+    static constexpr uint32_t AS = V + 2 * 16384;            // NKB x [128 rows][64 feat] bf16 S
     static constexpr uint32_t AW = AS + NKB * 16384;         // Wt^T
     static constexpr uint32_t AWD = AW + 16384;              // Wt^T diag(d/|k|)
-    static constexpr uint32_t OUT = AWD + 16384;             // [64 tok][128 ch] bf16 output staging
-    static constexpr uint32_t BAR = OUT + 16384;
+    static constexpr uint32_t OUT = AWD + 16384;             // [32 tok][128 ch] bf16 output staging
+    static constexpr uint32_t BAR = OUT + 8192;
     static constexpr uint32_t TSLOT = BAR + 256;
     static constexpr uint32_t ABORT = TSLOT + 16;
-    static constexpr uint32_t BYTES = ABORT + 16 + 1024;
+    // no alignment slack: the kernel checks that dynamic shared memory starts
+    // on a 1024-byte boundary (the swizzled tiles need it) and flags an error
+    // instead of running otherwise
+    static constexpr uint32_t BYTES = ABORT + 16;
     static_assert(BYTES <= 232448, "shared memory budget");
 };
 
@@ -70,14 +87,15 @@ constexpr uint32_t TM_S = 0, TM_X1 = 128, TM_X2 = 256, TM_COLS = 512;
 enum {
     B_IMG = 0,        // [2] image landed
     B_K = 2,          // [NKBUF] K tile landed
-    B_V = 4,          // V tile landed
-    B_P2 = 5,         // P2a complete
-    B_P3 = 6,         // P3 (and P5a) complete
-    B_SDONE = 7,      // [2] P4 / P5b complete
-    B_AS = 9,         // bf16 S written, S scaled (chain)
-    B_AW = 10,        // Wt^T copies written (chain)
-    B_X2FREE = 11,    // [2] O^T read (out)
-    NBARS = 13
+    B_V = 4,          // [2] V tile landed
+    B_P2 = 6,         // [2] P2a complete (per V buffer, so no waiter lags two phases)
+    B_P3 = 8,         // P3 (and P5a) complete
+    B_SDONE = 9,      // [2] P4 complete
+    B_AS = 11,        // bf16 S written, S scaled (chain)
+    B_AW = 12,        // Wt^T copies written (chain)
+    B_X2FREE = 13,    // [2] O^T read (out)
+    B_ODONE = 15,     // [2] P5a / P5b complete (O^T ready, S copy and Wt^T free)
+    NBARS = 17
 };
 
 template <int DK>
@@ -90,13 +108,17 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
     using IM = Img<DK>;
     constexpr int NKB = SM::NKB;
     constexpr int KSTEPS = DK / 16;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = smem_raw;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM::BAR);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + SM::TSLOT);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SM::ABORT);
 
     const int tid = threadIdx.x, warp = tid >> 5;
+    if (smem_u32(sm) & 1023u) {                           // whole CTA, before any barrier
+        if (tid == 0) flag_error(DEVERR_DATA);
+        return;
+    }
     const int ns = dv / ROWS;
     const int h = blockIdx.y, b = blockIdx.z / seg.zseg, p_seg = blockIdx.z % seg.zseg;
     const bool trans = blockIdx.x == ns;                  // transition slice (phase A, p >= 1)
@@ -151,8 +173,14 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         for (int c = 0; c < nch; ++c) {
             const int p = c & 1;
             const float* iv = reinterpret_cast<const float*>(img_at(c) + IM::VEC);   // dik[64], gam_{L-1}
-            bool okw = c < 1 || wait_spin(&bars[B_SDONE + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag);
-            okw = okw && wait_spin(&bars[B_IMG + p], (c >> 1) & 1, abort_flag);
+            bool okw = true;
+            if (ct == 0) {
+                // S updated (P4), the bf16 S copy and Wt^T no longer read (P5a / P5b), image landed
+                okw = c < 1 || wait_spin(&bars[B_SDONE + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag);
+                okw = okw && (c < 1 || !write_o ||
+                              wait_spin(&bars[B_ODONE + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag));
+                okw = okw && wait_spin(&bars[B_IMG + p], (c >> 1) & 1, abort_flag);
+            }
             if (!group_all(2, NCH_T, okw)) break;
             tc_fence_after();
             // ---- E4: S -> bf16 copy, S <- gam_L S
@@ -182,7 +210,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             named_sync(2, NCH_T);
             if (ct == 0) arrive(&bars[B_AS]);
             // ---- E5: Wt^T -> bf16 (plain and scaled by d/|k|)
-            if (!group_all(2, NCH_T, wait_spin(&bars[B_P3], c & 1, abort_flag))) break;
+            if (!group_wait(&bars[B_P3], c & 1, abort_flag, 2, NCH_T, ct == 0, true)) break;
             tc_fence_after();
             {
                 const uint32_t x1 = TM_X1 + (uint32_t)p * 64;
@@ -214,8 +242,10 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             if (ct == 0) arrive(&bars[B_AW]);
         }
         // final state of the segment (after the last P4)
-        const bool fin = !*abort_flag && nch > 0 &&
-                         wait_spin(&bars[B_SDONE + ((nch - 1) & 1)], ((nch - 1) >> 1) & 1, abort_flag);
+        bool fin = true;
+        if (ct == 0)
+            fin = !*abort_flag && nch > 0 &&
+                  wait_spin(&bars[B_SDONE + ((nch - 1) & 1)], ((nch - 1) >> 1) & 1, abort_flag);
         if (group_all(2, NCH_T, fin)) {
             tc_fence_after();
             float* dst = nullptr;
@@ -247,56 +277,55 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sm + SM::OUT);
             const long long tstride = (long long)H * dv;
             for (int c = 0; c < nch; ++c) {
-                if (!group_all(3, NOUT, wait_spin(&bars[B_SDONE + (c & 1)], (c >> 1) & 1, abort_flag))) break;
+                if (!group_wait(&bars[B_ODONE + (c & 1)], (c >> 1) & 1, abort_flag, 3, NOUT, ot == 0, false)) break;
                 tc_fence_after();
                 const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+                const int t0 = tbeg + c * C, L = min(C, tend - t0);
+                __nv_bfloat16* obase = o + ((long long)b * Tn + t0) * tstride + (long long)h * dv + c0;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
+                for (int half = 0; half < 2; ++half) {       // 32 tokens at a time
                     uint32_t x[32];
                     tmem_ld32(tb + lb + x2 + half * 32, x);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) st[(half * 32 + j) * ROWS + ot] = __float2bfloat16_rn(__uint_as_float(x[j]));
-                }
-                tc_fence_before();
-                named_sync(3, NOUT);
-                if (ot == 0) arrive(&bars[B_X2FREE + (c & 1)]);
-                const int t0 = tbeg + c * C, L = min(C, tend - t0);
-                __nv_bfloat16* obase = o + ((long long)b * Tn + t0) * tstride + (long long)h * dv + c0;
+                    for (int j = 0; j < 32; ++j) st[j * ROWS + ot] = __float2bfloat16_rn(__uint_as_float(x[j]));
+                    if (half == 1) tc_fence_before();
+                    named_sync(3, NOUT);
+                    if (half == 1 && ot == 0) arrive(&bars[B_X2FREE + (c & 1)]);
 #pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const int qd = ot + m * NOUT, r = qd >> 4, ch = qd & 15;
-                    if (r < L)
-                        *reinterpret_cast<uint4*>(obase + r * tstride + ch * 8) =
-                            *reinterpret_cast<const uint4*>(st + r * ROWS + ch * 8);
+                    for (int m = 0; m < 4; ++m) {
+                        const int qd = ot + m * NOUT, r = qd >> 4, ch = qd & 15;
+                        if (half * 32 + r < L)
+                            *reinterpret_cast<uint4*>(obase + (half * 32 + r) * tstride + ch * 8) =
+                                *reinterpret_cast<const uint4*>(st + r * ROWS + ch * 8);
+                    }
+                    named_sync(3, NOUT);                     // staging free again
                 }
-                named_sync(3, NOUT);                         // staging free again
             }
         }
     } else if (tid == MMA0 || tid == LOAD0) {
         // =============================================================== MMA / LOAD
-        // Fixed orders (every awaited event depends only on actions issued
-        // earlier in these orders or by the other warps):
-        //   MMA:   P2a(0);  chunk c: P3(c) [P5a(c)]  P4(c) [P5b(c)]  P2a(c+1)
-        //   LOAD:  IMG(0) K(0) V(0) IMG(1) [K(1)];  chunk c: V(c+1) after P2a(c),
-        //          K(c+NKBUF) and IMG(c+2) after P4(c)
+        // Two issuing threads, each in a fixed order (every awaited event
+        // depends only on actions issued earlier in these orders or by the
+        // other roles; a tcgen05 commit covers the issuing thread's MMAs):
+        //   MMA  (critical path):  chunk c: P3(c) after AS(c) and P2a(c);
+        //                          P4(c) after AW(c) and K(c)
+        //   LOAD (everything else): IMG(0) V(0) K(0) IMG(1) V(1) [K(1)] P2a(0);
+        //        chunk c: P5a(c) after AS(c) and X2 free, P5b(c) after AW(c);
+        //        P2a(c+1) after IMG(c+1) and V(c+1); V(c+2) after P2a(c);
+        //        K(c+NKBUF) and IMG(c+2) after P4(c) and P5b(c)
         constexpr int NKBUF = SM::NKBUF;
+        const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
+        auto ioff = [&](int c, uint32_t off) { return (uint64_t)((((uint32_t)(c & 1) * SM::IB) + off) >> 4); };
+        const uint64_t dAS = sw128_desc(smem_u32(sm + SM::AS), 16, 1024);
+        auto as_off = [&](int kk) { return (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4); };
         bool ok = true;
-        auto W = [&](int bar, int phase) {
-            if (!ok) return false;
-            for (uint32_t i = 0; i < 4096u; ++i)
-                if (mbar_test_wait(&bars[bar], (uint32_t)phase & 1u)) return true;
-            for (uint32_t i = 0; i < 4u * kWaitPolls; ++i) {
-                if (mbar_test_wait(&bars[bar], (uint32_t)phase & 1u)) return true;
-                if ((i & 1023u) == 1023u && *abort_flag) { ok = false; return false; }
-                __nanosleep(32);
-            }
-            *abort_flag = 1;
-            flag_error(DEVERR_TIMEOUT);
-            ok = false;
-            return false;
-        };
         if (tid == LOAD0) {
+            // waits off the critical path sleep between polls
+            auto WL = [&](int bar, int phase) {
+                if (ok && !wait_bar(&bars[bar], (uint32_t)phase & 1u, abort_flag)) ok = false;
+                return ok;
+            };
             const uint32_t img_bytes = write_o ? IM::BYTES : IM::A_BYTES;
             auto zrow = [&](int c) { return (int)((long long)b * Tn + tbeg + (long long)c * C); };
             auto load_img = [&](int c) {
@@ -313,89 +342,104 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                     tma_load_3d(sm + SM::K + (kb_ * NKB + kb) * 8192, &tm_k, bar, kb * 64, h, zrow(c));
             };
             auto load_v = [&](int c) {
-                mbar_expect_tx(&bars[B_V], 16384);
-                tma_load_3d(sm + SM::V, &tm_v, &bars[B_V], c0, h, zrow(c));
-                tma_load_3d(sm + SM::V + 8192, &tm_v, &bars[B_V], c0 + 64, h, zrow(c));
+                uint64_t* bar = &bars[B_V + (c & 1)];
+                uint8_t* dst = sm + SM::V + (uint32_t)(c & 1) * 16384;
+                mbar_expect_tx(bar, 16384);
+                tma_load_3d(dst, &tm_v, bar, c0, h, zrow(c));
+                tma_load_3d(dst + 8192, &tm_v, bar, c0 + 64, h, zrow(c));
             };
-            int nK = 0, nV = 0, nI = 0;                      // loads issued
-            if (nch > 0) { load_img(0); ++nI; load_k(0); ++nK; load_v(0); ++nV; }
-            if (nch > 1) { load_img(1); ++nI; }
+            const uint64_t dV = sw128_desc(smem_u32(sm + SM::V), 8192, 1024);
+            const uint64_t dAW = sw128_desc(smem_u32(sm + SM::AW), 16, 1024);
+            constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
+            constexpr uint32_t ID_MNK = idesc_bf16(128, 64, true, false);
+            auto mma_p2a = [&](int c) {      // X1[c&1] = V^T T1^T
+                const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64;
+                const uint64_t dv_ = dV + (uint64_t)(((uint32_t)(c & 1) * 16384) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tb + x1, dv_ + (uint64_t)(kk * 2048 >> 4), dImg + ioff(c, IM::T1 + kk * 32), ID_MNK,
+                                kk > 0);
+                mma_commit(&bars[B_P2 + (c & 1)]);
+            };
+            auto mma_p5a = [&](int c) {      // X2[c&1] = S Q~^T
+                const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+                for (int kk = 0; kk < KSTEPS; ++kk)
+                    mma_bf16_ss(tb + x2, dAS + as_off(kk), dImg + ioff(c, IM::Q + (kk >> 2) * 8192 + (kk & 3) * 32),
+                                ID_KK, kk > 0);
+            };
+            auto mma_p5b = [&](int c) {      // X2[c&1] += Wt^T P^T
+                const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), dImg + ioff(c, IM::P + kk * 32), ID_KK, 1);
+                mma_commit(&bars[B_ODONE + (c & 1)]);
+            };
+            int nK = 0, nV = 0, nI = 0, n2 = 0, n5 = 0;      // loads / commit groups issued
+            if (nch > 0) { load_img(0); ++nI; load_v(0); ++nV; load_k(0); ++nK; }
+            if (nch > 1) { load_img(1); ++nI; load_v(1); ++nV; }
             if (NKBUF == 2 && nch > 1) { load_k(1); ++nK; }
+            if (nch > 0 && WL(B_IMG, 0) && WL(B_V, 0)) { tc_fence_after(); mma_p2a(0); ++n2; }
             for (int c = 0; c < nch && ok; ++c) {
-                if (c + 1 < nch && W(B_P2, c)) { load_v(c + 1); ++nV; }
-                if ((c + NKBUF < nch || c + 2 < nch) && W(B_SDONE + (c & 1), c >> 1)) {
+                if (write_o) {
+                    if (WL(B_AS, c) && (c < 2 || WL(B_X2FREE + (c & 1), (c - 2) >> 1))) { tc_fence_after(); mma_p5a(c); }
+                    if (WL(B_AW, c)) { tc_fence_after(); mma_p5b(c); ++n5; }
+                }
+                if (c + 1 < nch && WL(B_IMG + ((c + 1) & 1), (c + 1) >> 1) && WL(B_V + ((c + 1) & 1), (c + 1) >> 1)) {
+                    tc_fence_after(); mma_p2a(c + 1); ++n2;
+                }
+                if (c + 2 < nch && WL(B_P2 + (c & 1), c >> 1)) { load_v(c + 2); ++nV; }
+                if ((c + NKBUF < nch || c + 2 < nch) && WL(B_SDONE + (c & 1), c >> 1) &&
+                    (!write_o || WL(B_ODONE + (c & 1), c >> 1))) {
                     if (c + NKBUF < nch) { load_k(c + NKBUF); ++nK; }
                     if (c + 2 < nch) { load_img(c + 2); ++nI; }
                 }
             }
-            // every issued load has landed before the CTA can exit (the last
-            // load on each barrier; immediate unless a wait ran out)
+            // every issued load and commit group has completed before the CTA
+            // frees its memory (the last one on each barrier; immediate unless
+            // a wait ran out)
             if (!ok) *abort_flag = 1;
             for (int j = max(0, nK - NKBUF); j < nK; ++j) mbar_wait(&bars[B_K + j % NKBUF], (j / NKBUF) & 1);
-            if (nV > 0) mbar_wait(&bars[B_V], (nV - 1) & 1);
+            for (int j = max(0, nV - 2); j < nV; ++j) mbar_wait(&bars[B_V + (j & 1)], (j >> 1) & 1);
             for (int j = max(0, nI - 2); j < nI; ++j) mbar_wait(&bars[B_IMG + (j & 1)], (j >> 1) & 1);
+            for (int j = max(0, n2 - 2); j < n2; ++j) mbar_wait(&bars[B_P2 + (j & 1)], (j >> 1) & 1);
+            for (int j = max(0, n5 - 2); j < n5; ++j) mbar_wait(&bars[B_ODONE + (j & 1)], (j >> 1) & 1);
         } else {
-            const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
+            // the critical path: spin first
+            auto W = [&](int bar, int phase) {
+                if (!ok) return false;
+                for (uint32_t i = 0; i < 4096u; ++i)
+                    if (mbar_test_wait(&bars[bar], (uint32_t)phase & 1u)) return true;
+                if (!wait_bar(&bars[bar], (uint32_t)phase & 1u, abort_flag)) ok = false;
+                return ok;
+            };
             const uint64_t dImgMN = sw128_desc(smem_u32(sm + SM::IMG), 8192, 1024);   // W^T (MN-major)
             const uint64_t dKmn = sw128_desc(smem_u32(sm + SM::K), 8192, 1024);       // K as MN-major
-            const uint64_t dV = sw128_desc(smem_u32(sm + SM::V), 8192, 1024);
-            const uint64_t dAS = sw128_desc(smem_u32(sm + SM::AS), 16, 1024);
-            const uint64_t dAW = sw128_desc(smem_u32(sm + SM::AW), 16, 1024);
             const uint64_t dAWD = sw128_desc(smem_u32(sm + SM::AWD), 16, 1024);
-            constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
-            constexpr uint32_t ID_MNK = idesc_bf16(128, 64, true, false);
             constexpr uint32_t ID_NEG = idesc_bf16(128, 64, false, true, true);
             constexpr uint32_t ID_S = idesc_bf16(128, DK, false, true);
-            auto ioff = [&](int c, uint32_t off) { return (uint64_t)((((uint32_t)(c & 1) * SM::IB) + off) >> 4); };
-            auto mma_p2a = [&](int c) {
-                const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64;
+            int n3 = 0, n4 = 0;                              // commit groups issued
+            for (int c = 0; c < nch && ok; ++c) {
+                if (W(B_AS, c) && W(B_P2 + (c & 1), c >> 1)) {      // X1[c&1] -= S W^T  (= Wt^T)
+                    tc_fence_after();
+                    const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tb + x1, dV + (uint64_t)(kk * 2048 >> 4), dImg + ioff(c, IM::T1 + kk * 32), ID_MNK,
-                                kk > 0);
-                mma_commit(&bars[B_P2]);
-            };
-            auto mma_p3 = [&](int c) {
-                const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64, x2 = TM_X2 + (uint32_t)(c & 1) * 64;
-#pragma unroll
-                for (int kk = 0; kk < KSTEPS; ++kk)
-                    mma_bf16_ss(tb + x1, dAS + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                                dImgMN + ioff(c, IM::WT + kk * 2048), ID_NEG, 1);
-                mma_commit(&bars[B_P3]);        // the chain waits for Wt^T only
-                if (!write_o) return;
-#pragma unroll
-                for (int kk = 0; kk < KSTEPS; ++kk)
-                    mma_bf16_ss(tb + x2, dAS + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                                dImg + ioff(c, IM::Q + (kk >> 2) * 8192 + (kk & 3) * 32), ID_KK, kk > 0);
-            };
-            auto mma_p4 = [&](int c) {
-                const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
-                const uint64_t dk_ = dKmn + (uint64_t)(((uint32_t)(c % NKBUF) * NKB * 8192) >> 4);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tb + TM_S, dAWD + (uint64_t)(kk * 32 >> 4), dk_ + (uint64_t)(kk * 2048 >> 4), ID_S, 1);
-                if (write_o) {
+                    for (int kk = 0; kk < KSTEPS; ++kk)
+                        mma_bf16_ss(tb + x1, dAS + as_off(kk), dImgMN + ioff(c, IM::WT + kk * 2048), ID_NEG, 1);
+                    mma_commit(&bars[B_P3]);
+                    ++n3;
+                }
+                if (W(B_AW, c) && W(B_K + c % NKBUF, (c / NKBUF) & 1)) {   // S += Wt^T diag(d/|k|) K
+                    tc_fence_after();
+                    const uint64_t dk_ = dKmn + (uint64_t)(((uint32_t)(c % NKBUF) * NKB * 8192) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), dImg + ioff(c, IM::P + kk * 32), ID_KK, 1);
-                }
-                mma_commit(&bars[B_SDONE + (c & 1)]);
-            };
-            int n2 = 0, n3 = 0, n4 = 0;                      // commit groups issued
-            if (nch > 0 && W(B_IMG, 0) && W(B_V, 0)) { tc_fence_after(); mma_p2a(0); ++n2; }
-            for (int c = 0; c < nch && ok; ++c) {
-                if (W(B_AS, c) && (!write_o || c < 2 || W(B_X2FREE + (c & 1), (c - 2) >> 1))) {
-                    tc_fence_after(); mma_p3(c); ++n3;
-                }
-                if (W(B_AW, c) && W(B_K + c % NKBUF, (c / NKBUF) & 1)) { tc_fence_after(); mma_p4(c); ++n4; }
-                if (c + 1 < nch && W(B_IMG + ((c + 1) & 1), (c + 1) >> 1) && W(B_V, c + 1)) {
-                    tc_fence_after(); mma_p2a(c + 1); ++n2;
+                        mma_bf16_ss(tb + TM_S, dAWD + (uint64_t)(kk * 32 >> 4), dk_ + (uint64_t)(kk * 2048 >> 4), ID_S, 1);
+                    mma_commit(&bars[B_SDONE + (c & 1)]);
+                    ++n4;
                 }
             }
-            // every issued commit group has completed before TMEM is freed (the
-            // last group on each barrier; immediate unless a wait ran out)
             if (!ok) *abort_flag = 1;
-            if (n2 > 0) mbar_wait(&bars[B_P2], (n2 - 1) & 1);
             if (n3 > 0) mbar_wait(&bars[B_P3], (n3 - 1) & 1);
             for (int j = max(0, n4 - 2); j < n4; ++j) mbar_wait(&bars[B_SDONE + (j & 1)], (j >> 1) & 1);
         }
