@@ -7,45 +7,77 @@
 // E_0 the true end state of segment 0) and A_p for p = 1 .. P-2; this kernel
 // chains them:
 //   S_start(1) = E_0,   S_start(p + 1) = S_start(p) A_p + E_p   (p = 1 .. P-2)
-// in float32. It also copies S0 (or zeros) to S_start(0), so that phase C never
-// reads S0 while the last segment may be writing a final state that aliases it.
+// It also copies S0 (or zeros) to S_start(0), so that phase C never reads S0
+// while the last segment may be writing a final state that aliases it.
 //
 // Rows of S are independent: a CTA owns 16 rows of one (sequence, head) and
-// walks p sequentially. Thread (j, g) owns column j of rows 4g .. 4g+3, so its
-// four accumulators are independent FMA chains; the 16 running rows sit in
-// shared memory (read as broadcast float4), and A_p arrives by one bulk copy
-// into a double buffer, the copy of A_{p+1} in flight while step p computes.
+// walks p sequentially. Each step is a 16 x dk by dk x dk product on the
+// tensor cores (mma.sync m16n8k8, tf32 in, float32 accumulate), with every
+// operand split as x = hi + lo (both tf32) and the product formed as
+// lo*hi + hi*lo + hi*hi, which keeps float32 accuracy (the dropped lo*lo
+// term is below 2^-22 relative). Warp w owns output columns 8w .. 8w+7. A_p
+// arrives by one bulk copy into a double buffer (the copy of A_{p+1} in
+// flight while step p computes); E_p of the next step is loaded during the
+// current one.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
 
 namespace jet {
 
-constexpr int SC_ROWS = 16;      // state rows per CTA
-constexpr int SC_RPT = 4;        // rows per thread
-constexpr int SC_GROUPS = SC_ROWS / SC_RPT;
+constexpr int SC_ROWS = 16;      // state rows per CTA (the MMA's M)
 
-__host__ __device__ constexpr int sc_threads(int dk) { return SC_GROUPS * dk; }
+__host__ __device__ constexpr int sc_threads(int dk) { return 4 * dk; }     // one warp per 8 columns
+__host__ __device__ constexpr int sc_lde(int dk) { return dk + 4; }          // padded row stride of the rows
 __host__ __device__ constexpr size_t sc_smem_bytes(int dk) {
-    return sizeof(float) * (2 * (size_t)dk * dk + (size_t)SC_ROWS * dk) + 2 * sizeof(uint64_t);
+    return sizeof(float) * (2 * (size_t)dk * dk + 2 * (size_t)SC_ROWS * sc_lde(dk)) + 2 * sizeof(uint64_t);
 }
+
+namespace sc {
+__device__ __forceinline__ uint32_t tf32_of(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+// x = hi + lo, both representable in tf32
+__device__ __forceinline__ void split(float x, uint32_t& hi, uint32_t& lo) {
+    hi = tf32_of(x);
+    lo = tf32_of(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma(float* d, const uint32_t* a, const uint32_t* b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+}  // namespace sc
 
 // E [B][P-1][H][dv][dk], A [B][P-1][H][dk][dk], Sst [B][P][H][dv][dk];
 // grid (dv / 16, H, B), sc_threads(DK) threads, sc_smem_bytes(DK) shared.
 template <int DK>
-__global__ void __launch_bounds__(SC_GROUPS * DK)
+__global__ void __launch_bounds__(4 * DK)
 seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, const float* S0,
                    float* __restrict__ Sst, int P, int H, int dv) {
+    static_assert(DK % 8 == 0 && DK <= 128, "dk");
+    constexpr int LDE = sc_lde(DK);
     extern __shared__ __align__(128) float scm[];
     float* As = scm;                                  // [2][DK][DK]
-    float* Es = As + 2 * DK * DK;                     // [16][DK] running rows
-    uint64_t* bar = reinterpret_cast<uint64_t*>(Es + SC_ROWS * DK);
+    float* Es = As + 2 * DK * DK;                     // [2][16][LDE] running rows
+    uint64_t* bar = reinterpret_cast<uint64_t*>(Es + 2 * SC_ROWS * LDE);
     constexpr uint32_t ABYTES = DK * DK * sizeof(float);
-    const int tid = threadIdx.x, j = tid % DK, grp = tid / DK;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t = lane & 3, n0 = warp * 8;
     const int r0 = blockIdx.x * SC_ROWS, h = blockIdx.y, b = blockIdx.z;
     auto e_at = [&](int p) { return E + ((((long long)b * (P - 1) + p) * H + h) * dv + r0) * DK; };
     auto s_at = [&](int p) { return Sst + ((((long long)b * P + p) * H + h) * dv + r0) * DK; };
     auto a_at = [&](int p) { return A + (((long long)b * (P - 1) + p) * H + h) * DK * DK; };
+    // this thread's accumulator entries: rows g and g+8, columns n0+2t and n0+2t+1
+    auto load_frag = [&](const float* src, float* d) {
+        const float2 x = *reinterpret_cast<const float2*>(src + g * DK + n0 + 2 * t);
+        const float2 y = *reinterpret_cast<const float2*>(src + (g + 8) * DK + n0 + 2 * t);
+        d[0] = x.x; d[1] = x.y; d[2] = y.x; d[3] = y.y;
+    };
 
     if (tid == 0) {
         sm100::mbar_init(&bar[0], 1);
@@ -58,52 +90,55 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
             sm100::mbar_expect_tx(&bar[p - 1], ABYTES);
             sm100::bulk_load(As + (p - 1) * DK * DK, a_at(p), ABYTES, &bar[p - 1]);
         }
-    // S_start(0) = S0 (or zeros), S_start(1) = E_0
+    // S_start(0) = S0 (or zeros); S_start(1) = E_0, also the running rows of step 1
     const float* s0 = S0 ? S0 + (((long long)b * H + h) * dv + r0) * DK : nullptr;
-#pragma unroll
-    for (int i = 0; i < SC_RPT; ++i) {
-        const int r = grp * SC_RPT + i;
-        s_at(0)[r * DK + j] = s0 ? s0[r * DK + j] : 0.f;
-        const float x = e_at(0)[r * DK + j];
-        Es[r * DK + j] = x;
-        s_at(1)[r * DK + j] = x;
+    for (int i = tid; i < SC_ROWS * DK; i += 4 * DK) {
+        const int r = i / DK, j = i % DK;
+        s_at(0)[i] = s0 ? s0[i] : 0.f;
+        const float x = e_at(0)[i];
+        Es[1 * SC_ROWS * LDE + r * LDE + j] = x;
+        s_at(1)[i] = x;
     }
+    float e_next[4] = {0.f, 0.f, 0.f, 0.f};
+    if (P > 2) load_frag(e_at(1), e_next);
     __syncthreads();
 
     for (int p = 1; p + 1 < P; ++p) {
         const int buf = (p - 1) & 1;
         const uint32_t parity = ((p - 1) >> 1) & 1;
-        float acc[SC_RPT];
-        const float* ep = e_at(p);
-#pragma unroll
-        for (int i = 0; i < SC_RPT; ++i) acc[i] = __ldcs(ep + (grp * SC_RPT + i) * DK + j);
+        float d[4] = {e_next[0], e_next[1], e_next[2], e_next[3]};
+        if (p + 2 < P) load_frag(e_at(p + 1), e_next);      // in flight during this step
         const bool ok = sm100::mbar_wait(&bar[buf], parity);
-        if (!__syncthreads_and(ok)) return;           // timed out: error word already set
+        if (!__syncthreads_and(ok)) return;                  // timed out: error word already set
         const float* Ab = As + buf * DK * DK;
-        const float* Eg = Es + grp * SC_RPT * DK;
+        const float* Ec = Es + (p & 1) * SC_ROWS * LDE;      // S_start(p) rows
 #pragma unroll 4
-        for (int q = 0; q < DK; q += 4) {
-            const float a0 = Ab[q * DK + j], a1 = Ab[(q + 1) * DK + j];
-            const float a2 = Ab[(q + 2) * DK + j], a3 = Ab[(q + 3) * DK + j];
-#pragma unroll
-            for (int i = 0; i < SC_RPT; ++i) {
-                const float4 e = *reinterpret_cast<const float4*>(Eg + i * DK + q);
-                acc[i] = fmaf(e.x, a0, fmaf(e.y, a1, fmaf(e.z, a2, fmaf(e.w, a3, acc[i]))));
-            }
+        for (int k0 = 0; k0 < DK; k0 += 8) {
+            uint32_t ah[4], al[4], bh[2], bl[2];
+            sc::split(Ec[g * LDE + k0 + t], ah[0], al[0]);
+            sc::split(Ec[(g + 8) * LDE + k0 + t], ah[1], al[1]);
+            sc::split(Ec[g * LDE + k0 + t + 4], ah[2], al[2]);
+            sc::split(Ec[(g + 8) * LDE + k0 + t + 4], ah[3], al[3]);
+            sc::split(Ab[(k0 + t) * DK + n0 + g], bh[0], bl[0]);
+            sc::split(Ab[(k0 + t + 4) * DK + n0 + g], bh[1], bl[1]);
+            sc::mma(d, al, bh);
+            sc::mma(d, ah, bl);
+            sc::mma(d, ah, bh);
         }
-        __syncthreads();                              // every read of Es and As[buf] done
-        if (tid == 0 && p + 3 < P) {          // A_{p+2} is used by step p + 2 <= P - 2
+        // S_start(p+1): to the next running-row buffer and to global
+        float* En = Es + ((p + 1) & 1) * SC_ROWS * LDE;
+        En[g * LDE + n0 + 2 * t] = d[0];
+        En[g * LDE + n0 + 2 * t + 1] = d[1];
+        En[(g + 8) * LDE + n0 + 2 * t] = d[2];
+        En[(g + 8) * LDE + n0 + 2 * t + 1] = d[3];
+        float* sp = s_at(p + 1);
+        *reinterpret_cast<float2*>(sp + g * DK + n0 + 2 * t) = make_float2(d[0], d[1]);
+        *reinterpret_cast<float2*>(sp + (g + 8) * DK + n0 + 2 * t) = make_float2(d[2], d[3]);
+        __syncthreads();                              // every read of As[buf] and of the old rows done
+        if (tid == 0 && p + 3 < P) {                  // A_{p+2} is used by step p + 2 <= P - 2
             sm100::mbar_expect_tx(&bar[buf], ABYTES);
             sm100::bulk_load(As + buf * DK * DK, a_at(p + 2), ABYTES, &bar[buf]);
         }
-        float* sp = s_at(p + 1);
-#pragma unroll
-        for (int i = 0; i < SC_RPT; ++i) {
-            const int r = grp * SC_RPT + i;
-            Es[r * DK + j] = acc[i];
-            sp[r * DK + j] = acc[i];
-        }
-        __syncthreads();
     }
 }
 
