@@ -257,9 +257,38 @@ def cpu_baseline(seed: int, budget_s: float = 15.0):
                       f"for each of 256 sequences) on the float64 oracle, {dt:.1f} s"}
 
 
+# ------------------------------------------------------------------ multi-rank plumbing
+class Ranks:
+    """One process per GPU (torchrun sets RANK / LOCAL_RANK / WORLD_SIZE). The
+    path shards without any exchange: every rank runs the same per-GPU
+    workload on its own inputs (weak scaling); the only collectives are the
+    barriers around the timed region and the max over ranks of its duration."""
+
+    def __init__(self, env=None):
+        env = os.environ if env is None else env
+        self.world = int(env.get("WORLD_SIZE", "1"))
+        self.rank = int(env.get("RANK", "0"))
+        self.local = int(env.get("LOCAL_RANK", "0"))
+
+    def seed(self, base: int) -> int:
+        return base + 17 * self.rank              # distinct synthetic inputs per rank
+
+    def max_over_ranks(self, x: float, device=None) -> float:
+        if self.world == 1:
+            return x
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def value(self, tokens_per_rank_per_step: int, steps: int, ms_max: float) -> float:
+        """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+        return tokens_per_rank_per_step * self.world * steps / (ms_max * 1e-3)
+
+
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    if Ranks().rank != 0:                       # rank 0 alone runs the oracle; the others exit
         return 0
     import oracle
     orc = oracle.get()
@@ -295,9 +324,8 @@ def run_jet(args):
     import torch.distributed as dist
     from linear_attention_lm_gen_b200 import build as jbuild
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rk = Ranks()
+    world, rank, local = rk.world, rk.rank, rk.local
     if world != args.gpus:
         print(f"WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
     torch.cuda.set_device(local)
@@ -309,7 +337,7 @@ def run_jet(args):
     jbuild.build()
     import linear_attention_lm_gen_b200 as jet
     jet.load_library()
-    wl = Workload(device, seed=args.seed + 17 * rank)
+    wl = Workload(device, seed=rk.seed(args.seed))
     stream = torch.cuda.Stream(device)
 
     def barrier():
@@ -318,11 +346,7 @@ def run_jet(args):
         torch.cuda.synchronize(device)
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return rk.max_over_ranks(x, device)
 
     counts = []
     with torch.cuda.stream(stream):
@@ -418,7 +442,7 @@ def run_jet(args):
     dom = names[int(np.argmax(per_kernel / np.maximum(per_call_launches, 1)))]
     ach = kern[dom]["achieved_gbs"]
     tokens = TOKENS_PER_STEP * world
-    value = tokens * args.steps / (ms * 1e-3)
+    value = rk.value(TOKENS_PER_STEP, args.steps, ms)
     prefill_ms = per_kernel[0] + per_kernel[1]
     decode_ms = per_kernel[2] + per_kernel[3]
     roof_step_us = sum(k["roofline_us"] for k in kern.values())
