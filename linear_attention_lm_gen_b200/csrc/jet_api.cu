@@ -236,7 +236,7 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
         if (smem_attr(prep, pfws::PrepSmem<DK>::BYTES) != JET_OK) return JET_ERR_CUDA;
         const int nct = (Tn + pfws::C - 1) / pfws::C;
         const long long items = (long long)B * H * nct;
-        const int grid = (int)std::min<long long>(items, 2LL * kSMs);   // two resident CTAs per SM
+        const int grid = (int)std::min<long long>(items, (long long)pfws::PREP_CTAS * kSMs);   // resident CTAs
         prep<<<grid, pfws::PREP_THREADS, pfws::PrepSmem<DK>::BYTES, s>>>(mq, mk, g, beta, img, Tn, H, nct,
                                                                          (int)items);
         g_launches.fetch_add(1, std::memory_order_relaxed);

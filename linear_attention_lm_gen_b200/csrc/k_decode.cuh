@@ -26,7 +26,7 @@ constexpr int DEC_THREADS = 256;
 constexpr int DEC_ROWS = 128;    // rows of S per CTA (two per 4-lane group)
 
 template <typename T, int NV>   // NV = dk / 16 float4 per lane
-__global__ void __launch_bounds__(DEC_THREADS)
+__global__ void __launch_bounds__(DEC_THREADS, NV <= 6 ? 3 : 2)   // 3 CTAs per SM where the registers allow
 gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const float* __restrict__ g, const float* __restrict__ beta,
                   float* __restrict__ S, T* __restrict__ o, int H, int dv) {

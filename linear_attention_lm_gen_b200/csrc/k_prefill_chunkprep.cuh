@@ -17,8 +17,9 @@
 // T1, W^T and vec come first, so a pass without outputs copies a prefix.
 //
 // A CTA (256 threads, named barrier 1 = the whole CTA) walks items
-// blockIdx.x, blockIdx.x + gridDim.x, ... with the K / Q tiles of the next
-// two items in flight (TMA, double buffer). Per item: P1 = [K; Q] K^T on
+// blockIdx.x, blockIdx.x + gridDim.x, ...; three CTAs share an SM, so three
+// items are in flight per SM, and the K / Q tile of a CTA's next item is
+// loaded (TMA) as soon as the current one has been consumed. Per item: P1 = [K; Q] K^T on
 // tcgen05 while the per-token vectors are formed; A and P; the UT inverse;
 // T1 / T2; P2b = K^T T2^T on tcgen05 while Q~ is formed; W^T. T1, P, W^T and
 // the vectors are stored straight from registers (each warp store covers
@@ -31,6 +32,8 @@ namespace jet {
 namespace pfws {
 
 constexpr int PREP_THREADS = 256;
+constexpr int PREP_KQBUF = 1;        // K / Q tiles in flight per CTA
+constexpr int PREP_CTAS = 3;         // resident CTAs per SM (items in flight per SM)
 
 // per-chunk image layout (bytes; every tile 1024-aligned)
 template <int DK>
@@ -51,8 +54,8 @@ template <int DK>
 struct PrepSmem {
     static constexpr int NKB = (DK + 63) / 64;
     static constexpr uint32_t KQB = NKB * 16384;                   // one K / Q tile: [K 8K | Q 8K] per block
-    static constexpr uint32_t KQ = 0;                              // [2] tiles
-    static constexpr uint32_t T2 = KQ + 2 * KQB;
+    static constexpr uint32_t KQ = 0;                              // [PREP_KQBUF] tiles
+    static constexpr uint32_t T2 = KQ + PREP_KQBUF * KQB;
     static constexpr uint32_t AF = T2 + 8192;
     static constexpr uint32_t XS = AF + AF_BYTES;
     static constexpr uint32_t VEC = XS + XS_BYTES;                 // 8 x 64 fp32
@@ -60,12 +63,12 @@ struct PrepSmem {
     static constexpr uint32_t BAR = PN + 1024;
     static constexpr uint32_t TSLOT = BAR + 64;
     static constexpr uint32_t BYTES = TSLOT + 16 + 1024;           // + alignment slack
-    static_assert(2 * BYTES <= 232448, "two CTAs per SM");
+    static_assert(PREP_CTAS * (BYTES + 1024) <= 233472, "resident CTAs per SM");
 };
 
 // items = B * H * nct, item = (b * H + h) * nct + c (also the image index)
 template <int DK>
-__global__ void __launch_bounds__(PREP_THREADS, 2)
+__global__ void __launch_bounds__(PREP_THREADS, PREP_CTAS)
 gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const float* __restrict__ g, const float* __restrict__ beta, uint8_t* __restrict__ img,
                       int Tn, int H, int nct, int n_items) {
@@ -108,10 +111,9 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     };
     int nld[2] = {0, 0}, ndone[2] = {0, 0};          // loads issued / consumed per buffer (thread 0)
     int n1 = 0, n2 = 0;                               // MMA groups issued (thread 0)
-    if (tid == 0) {
-        if (blockIdx.x < n_items) { issue_load(blockIdx.x, 0); ++nld[0]; }
-        if (blockIdx.x + gridDim.x < n_items) { issue_load(blockIdx.x + gridDim.x, 1); ++nld[1]; }
-    }
+    if (tid == 0)
+        for (int j = 0; j < PREP_KQBUF; ++j)
+            if (blockIdx.x + j * (int)gridDim.x < n_items) { issue_load(blockIdx.x + j * gridDim.x, j); ++nld[j]; }
     Vec V = vec_from(reinterpret_cast<float*>(sm + SM::VEC));
     float* AF = reinterpret_cast<float*>(sm + SM::AF);
     float* XS = reinterpret_cast<float*>(sm + SM::XS);
@@ -132,13 +134,13 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     int k = 0;
     float gb_next = load_gb(blockIdx.x);
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
-        const int buf = k & 1;
+        const int buf = k % PREP_KQBUF;
         uint8_t* KQ = sm + SM::KQ + buf * SM::KQB;
         const int L = min(C, Tn - (item % nct) * C);
         uint8_t* out = img + (size_t)item * IM::BYTES;
         const float gb = gb_next;
         gb_next = load_gb(item + gridDim.x);            // in flight during this item
-        if (!(ok = __syncthreads_and(mbar_wait(&bars[buf], (uint32_t)(k >> 1) & 1)))) break;
+        if (!(ok = __syncthreads_and(mbar_wait(&bars[buf], (uint32_t)(k / PREP_KQBUF) & 1)))) break;
         if (tid == 0) {   // P1: [K; Q] K^T -> XP
             ++ndone[buf];
             tc_fence_after();
@@ -186,16 +188,16 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         prep_wt<DK>(tb + TM_XW, out + IM::WT, tid);
         tc_fence_before();
         named_sync(1, PREP_THREADS);                    // XP, XW, T2 and KQ[buf] free (but for the Q~ copy)
-        if (tid == 0 && item + 2 * (int)gridDim.x < n_items) {
+        if (tid == 0 && item + PREP_KQBUF * (int)gridDim.x < n_items) {
             bulk_wait_read_all();                       // the Q~ copy has read KQ[buf]
-            issue_load(item + 2 * gridDim.x, buf);
+            issue_load(item + PREP_KQBUF * gridDim.x, buf);
             ++nld[buf];
         }
     }
     if (tid == 0) {
         bulk_wait_all();             // shared memory stays valid until the copies have read it
         if (!ok) {                   // a wait ran out: let issued loads / MMAs finish (bounded)
-            for (int q = 0; q < 2; ++q)
+            for (int q = 0; q < PREP_KQBUF; ++q)
                 if (nld[q] > ndone[q]) mbar_wait(&bars[q], (uint32_t)(nld[q] - 1) & 1);
             if (n1 > 0) mbar_wait(&bars[2], (uint32_t)(n1 - 1) & 1);
             if (n2 > 0) mbar_wait(&bars[3], (uint32_t)(n2 - 1) & 1);
