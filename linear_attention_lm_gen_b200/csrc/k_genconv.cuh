@@ -164,6 +164,87 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
         w2s[i] = Elem<T>::ld(W2 + (long long)r * HW4 + h0 * GC_W + c);
     }
 
+    // ---- conv work items (stage C): one 16-byte channel group of one head
+    // over a run of tokens. Their loads do not depend on the taps, so with one
+    // token per item (decode) the first items' loads go out before stage A.
+    using V16 = Vec16<T>;
+    constexpr int VN = V16::N;                 // channels per 16-byte group
+    constexpr int PF = RUN == 1 ? 2 : 0;       // items prefetched per thread
+    const int ngrp = dv / VN;                  // groups per head row
+    const int nruns = (nrows + RUN - 1) / RUN;
+    const int cols = nh * ngrp;
+    const int items = v ? cols * nruns : 0;
+    const long long rowstride = (long long)H * dv;   // elements per token
+    struct ItemGeo { long long rr0, coff; int hl, ta, tb, bseq, tpos0; };
+    auto item_load = [&](int it, uint4* wraw, uint4* cur, ItemGeo& gi) {
+        const int col = it % cols;
+        const int run = it / cols;
+        const int hl = col / ngrp, cg = col % ngrp;
+        gi.hl = hl;
+        gi.coff = (long long)(h0 + hl) * dv + (long long)cg * VN;
+        gi.ta = run * RUN;
+        gi.tb = min(nrows, gi.ta + RUN);
+        gi.rr0 = r0 + gi.ta;
+        gi.bseq = (int)(gi.rr0 / Tn);               // one division per item; then stepped
+        gi.tpos0 = (int)(gi.rr0 - (long long)gi.bseq * Tn);
+        // window: wraw[0] = v_{t-1}, wraw[1] = v_{t-2}, wraw[2] = v_{t-3}
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            const int tau = gi.tpos0 - 1 - j;
+            wraw[j] = make_uint4(0, 0, 0, 0);
+            if (tau >= 0) wraw[j] = *reinterpret_cast<const uint4*>(v + (gi.rr0 - 1 - j) * rowstride + gi.coff);
+            else if (hist_in)
+                wraw[j] = *reinterpret_cast<const uint4*>(hist_in + ((long long)gi.bseq * 3 + (3 + tau)) * rowstride + gi.coff);
+        }
+#pragma unroll
+        for (int i = 0; i < RUN; ++i)
+            if (gi.ta + i < gi.tb) cur[i] = *reinterpret_cast<const uint4*>(v + (gi.rr0 + i) * rowstride + gi.coff);
+    };
+    auto item_compute = [&](const uint4* wraw, const uint4* cur, const ItemGeo& gi) {
+        const long long coff = gi.coff;
+        int bseq = gi.bseq;
+        float win[3][VN];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) V16::unpack(wraw[j], win[j]);
+        int tpos = gi.tpos0;
+#pragma unroll
+        for (int i = 0; i < RUN; ++i) {
+            if (gi.ta + i >= gi.tb) break;
+            const long long rr = gi.rr0 + i;
+            if (RUN > 1 && i > 0 && tpos == Tn) {      // a new sequence starts inside the run
+                tpos = 0;
+                ++bseq;
+#pragma unroll
+                for (int j = 0; j < 3; ++j) {
+                    uint4 u = make_uint4(0, 0, 0, 0);
+                    if (hist_in) u = *reinterpret_cast<const uint4*>(hist_in + ((long long)bseq * 3 + (2 - j)) * rowstride + coff);
+                    V16::unpack(u, win[j]);
+                }
+            }
+            float cv[VN];
+            V16::unpack(cur[i], cv);
+            const float4 w4 = *reinterpret_cast<const float4*>(taps + (gi.ta + i) * CW + gi.hl * GC_W);
+            float out[VN];
+#pragma unroll
+            for (int e = 0; e < VN; ++e)
+                out[e] = w4.x * cv[e] + w4.y * win[0][e] + w4.z * win[1][e] + w4.w * win[2][e];
+            *reinterpret_cast<uint4*>(v_out + rr * rowstride + coff) = V16::pack(out);
+#pragma unroll
+            for (int e = 0; e < VN; ++e) { win[2][e] = win[1][e]; win[1][e] = win[0][e]; win[0][e] = cv[e]; }
+            if (hist_out && tpos == Tn - 1) {
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    *reinterpret_cast<uint4*>(hist_out + ((long long)bseq * 3 + (2 - j)) * rowstride + coff) = V16::pack(win[j]);
+            }
+            ++tpos;
+        }
+    };
+    uint4 pw[PF > 0 ? PF : 1][3], pc[PF > 0 ? PF : 1][RUN];
+    ItemGeo pg[PF > 0 ? PF : 1];
+#pragma unroll
+    for (int q = 0; q < PF; ++q)
+        if (tid + q * GC_THREADS < items) item_load(tid + q * GC_THREADS, pw[q], pc[q], pg[q]);
+
     // ---- stage A: this CTA's slice of z = x . W1 ----
     const int nks = D / 16, per = (nks + G - 1) / G;
     const int ks0 = min(nks, g * per), ks1 = min(nks, ks0 + per);
@@ -219,75 +300,14 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
     __syncthreads();
 
     // ---- stage C: causal conv over V ----
-    using V16 = Vec16<T>;
-    constexpr int VN = V16::N;                 // channels per 16-byte group
-    const int ngrp = dv / VN;                  // groups per head row
-    const int nruns = (nrows + RUN - 1) / RUN;
-    const int cols = nh * ngrp;
-    const int items = cols * nruns;
-    const long long rowstride = (long long)H * dv;   // elements per token
-    for (int it = tid; it < items; it += GC_THREADS) {
-        const int col = it % cols;
-        const int run = it / cols;
-        const int hl = col / ngrp, cg = col % ngrp;
-        const int h = h0 + hl;
-        const long long coff = (long long)h * dv + (long long)cg * VN;
-        const int ta = run * RUN;
-        const int tb = min(nrows, ta + RUN);
-
-        // window: win[0] = v_{t-1}, win[1] = v_{t-2}, win[2] = v_{t-3}
-        uint4 wraw[3];
-        uint4 cur[RUN];
-        const long long rr0 = r0 + ta;
-        int bseq = (int)(rr0 / Tn);                    // one division per item; then stepped
-        int tpos0 = (int)(rr0 - (long long)bseq * Tn);
-        {
 #pragma unroll
-            for (int j = 0; j < 3; ++j) {
-                const int tau = tpos0 - 1 - j;
-                wraw[j] = make_uint4(0, 0, 0, 0);
-                if (tau >= 0) wraw[j] = *reinterpret_cast<const uint4*>(v + (rr0 - 1 - j) * rowstride + coff);
-                else if (hist_in) wraw[j] = *reinterpret_cast<const uint4*>(hist_in + ((long long)bseq * 3 + (3 + tau)) * rowstride + coff);
-            }
-#pragma unroll
-            for (int i = 0; i < RUN; ++i)
-                if (ta + i < tb) cur[i] = *reinterpret_cast<const uint4*>(v + (rr0 + i) * rowstride + coff);
-        }
-        float win[3][VN];
-#pragma unroll
-        for (int j = 0; j < 3; ++j) V16::unpack(wraw[j], win[j]);
-        int tpos = tpos0;
-#pragma unroll
-        for (int i = 0; i < RUN; ++i) {
-            if (ta + i >= tb) break;
-            const long long rr = rr0 + i;
-            if (RUN > 1 && i > 0 && tpos == Tn) {      // a new sequence starts inside the run
-                tpos = 0;
-                ++bseq;
-#pragma unroll
-                for (int j = 0; j < 3; ++j) {
-                    uint4 u = make_uint4(0, 0, 0, 0);
-                    if (hist_in) u = *reinterpret_cast<const uint4*>(hist_in + ((long long)bseq * 3 + (2 - j)) * rowstride + coff);
-                    V16::unpack(u, win[j]);
-                }
-            }
-            float cv[VN];
-            V16::unpack(cur[i], cv);
-            const float4 w4 = *reinterpret_cast<const float4*>(taps + (ta + i) * CW + hl * GC_W);
-            float out[VN];
-#pragma unroll
-            for (int e = 0; e < VN; ++e)
-                out[e] = w4.x * cv[e] + w4.y * win[0][e] + w4.z * win[1][e] + w4.w * win[2][e];
-            *reinterpret_cast<uint4*>(v_out + rr * rowstride + coff) = V16::pack(out);
-#pragma unroll
-            for (int e = 0; e < VN; ++e) { win[2][e] = win[1][e]; win[1][e] = win[0][e]; win[0][e] = cv[e]; }
-            if (hist_out && tpos == Tn - 1) {
-#pragma unroll
-                for (int j = 0; j < 3; ++j)
-                    *reinterpret_cast<uint4*>(hist_out + ((long long)bseq * 3 + (2 - j)) * rowstride + coff) = V16::pack(win[j]);
-            }
-            ++tpos;
-        }
+    for (int q = 0; q < PF; ++q)
+        if (tid + q * GC_THREADS < items) item_compute(pw[q], pc[q], pg[q]);
+    for (int it = tid + PF * GC_THREADS; it < items; it += GC_THREADS) {
+        ItemGeo gg;
+        uint4 wraw[3], cur[RUN];
+        item_load(it, wraw, cur, gg);
+        item_compute(wraw, cur, gg);
     }
 }
 

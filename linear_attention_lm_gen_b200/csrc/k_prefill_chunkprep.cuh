@@ -184,15 +184,16 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             bulk_commit();
         }
         if (!(ok = __syncthreads_and(mbar_wait(&bars[3], (uint32_t)k & 1)))) break;
-        tc_fence_after();
-        prep_wt<DK>(tb + TM_XW, out + IM::WT, tid);
-        tc_fence_before();
-        named_sync(1, PREP_THREADS);                    // XP, XW, T2 and KQ[buf] free (but for the Q~ copy)
+        // P2b has read K: once the Q~ copy has read Q, the tile is free for a later item
         if (tid == 0 && item + PREP_KQBUF * (int)gridDim.x < n_items) {
-            bulk_wait_read_all();                       // the Q~ copy has read KQ[buf]
+            bulk_wait_read_all();
             issue_load(item + PREP_KQBUF * gridDim.x, buf);
             ++nld[buf];
         }
+        tc_fence_after();
+        prep_wt<DK>(tb + TM_XW, out + IM::WT, tid);
+        tc_fence_before();
+        named_sync(1, PREP_THREADS);                    // XP, XW and T2 free for the next item
     }
     if (tid == 0) {
         bulk_wait_all();             // shared memory stays valid until the copies have read it

@@ -13,7 +13,8 @@
 // Rows of S are independent: a CTA owns 16 rows of one (sequence, head) and
 // walks p sequentially. Each step is a 16 x dk by dk x dk product on the
 // tensor cores (mma.sync m16n8k8, tf32 in, float32 accumulate), with every
-// operand split as x = hi + lo (both tf32) and the product formed as
+// operand split as x = hi + lo (both tf32; the running rows are split once
+// when written) and the product formed as
 // lo*hi + hi*lo + hi*hi, which keeps float32 accuracy (the dropped lo*lo
 // term is below 2^-22 relative). Warp w owns output columns 8w .. 8w+7. A_p
 // arrives by one bulk copy into a double buffer (the copy of A_{p+1} in
@@ -30,7 +31,7 @@ constexpr int SC_ROWS = 16;      // state rows per CTA (the MMA's M)
 __host__ __device__ constexpr int sc_threads(int dk) { return 4 * dk; }     // one warp per 8 columns
 __host__ __device__ constexpr int sc_lde(int dk) { return dk + 4; }          // padded row stride of the rows
 __host__ __device__ constexpr size_t sc_smem_bytes(int dk) {
-    return sizeof(float) * (2 * (size_t)dk * dk + 2 * (size_t)SC_ROWS * sc_lde(dk)) + 2 * sizeof(uint64_t);
+    return sizeof(float) * (2 * (size_t)dk * dk + 4 * (size_t)SC_ROWS * sc_lde(dk)) + 2 * sizeof(uint64_t);
 }
 
 namespace sc {
@@ -63,8 +64,13 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
     constexpr int LDE = sc_lde(DK);
     extern __shared__ __align__(128) float scm[];
     float* As = scm;                                  // [2][DK][DK]
-    float* Es = As + 2 * DK * DK;                     // [2][16][LDE] running rows
-    uint64_t* bar = reinterpret_cast<uint64_t*>(Es + 2 * SC_ROWS * LDE);
+    // running rows S_start(p), split once into tf32 hi / lo parts: [2][hi, lo][16][LDE]
+    uint32_t* Es = reinterpret_cast<uint32_t*>(As + 2 * DK * DK);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(Es + 4 * SC_ROWS * LDE);
+    auto put_row = [&](int p, int r, int j, float x) {   // S_start(p)[r][j] into the running rows
+        uint32_t* e = Es + (p & 1) * 2 * SC_ROWS * LDE + r * LDE + j;
+        sc::split(x, e[0], e[SC_ROWS * LDE]);
+    };
     constexpr uint32_t ABYTES = DK * DK * sizeof(float);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3, n0 = warp * 8;
@@ -92,12 +98,22 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
         }
     // S_start(0) = S0 (or zeros); S_start(1) = E_0, also the running rows of step 1
     const float* s0 = S0 ? S0 + (((long long)b * H + h) * dv + r0) * DK : nullptr;
-    for (int i = tid; i < SC_ROWS * DK; i += 4 * DK) {
-        const int r = i / DK, j = i % DK;
-        s_at(0)[i] = s0 ? s0[i] : 0.f;
-        const float x = e_at(0)[i];
-        Es[1 * SC_ROWS * LDE + r * LDE + j] = x;
-        s_at(1)[i] = x;
+    {   // every thread owns 4 of the 16 x DK entries; all loads first, then the stores
+        constexpr int PER = SC_ROWS / 4;
+        float xs[PER], x0[PER];
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int i = tid + u * 4 * DK;
+            xs[u] = e_at(0)[i];
+            x0[u] = s0 ? s0[i] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int i = tid + u * 4 * DK;
+            s_at(0)[i] = x0[u];
+            s_at(1)[i] = xs[u];
+            put_row(1, i / DK, i % DK, xs[u]);
+        }
     }
     float e_next[4] = {0.f, 0.f, 0.f, 0.f};
     if (P > 2) load_frag(e_at(1), e_next);
@@ -111,26 +127,32 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
         const bool ok = sm100::mbar_wait(&bar[buf], parity);
         if (!__syncthreads_and(ok)) return;                  // timed out: error word already set
         const float* Ab = As + buf * DK * DK;
-        const float* Ec = Es + (p & 1) * SC_ROWS * LDE;      // S_start(p) rows
-#pragma unroll 4
+        const uint32_t* Eh = Es + (p & 1) * 2 * SC_ROWS * LDE;  // S_start(p) rows, hi parts
+        const uint32_t* El = Eh + SC_ROWS * LDE;                 // lo parts
+        // six independent accumulators (product kind x even / odd k-step) keep
+        // the dependent MMA chains short
+        float acc[2][3][4] = {};
+#pragma unroll
         for (int k0 = 0; k0 < DK; k0 += 8) {
+            const int par = (k0 >> 3) & 1;
             uint32_t ah[4], al[4], bh[2], bl[2];
-            sc::split(Ec[g * LDE + k0 + t], ah[0], al[0]);
-            sc::split(Ec[(g + 8) * LDE + k0 + t], ah[1], al[1]);
-            sc::split(Ec[g * LDE + k0 + t + 4], ah[2], al[2]);
-            sc::split(Ec[(g + 8) * LDE + k0 + t + 4], ah[3], al[3]);
+            const int i0 = g * LDE + k0 + t, i1 = (g + 8) * LDE + k0 + t;
+            ah[0] = Eh[i0]; ah[1] = Eh[i1]; ah[2] = Eh[i0 + 4]; ah[3] = Eh[i1 + 4];
+            al[0] = El[i0]; al[1] = El[i1]; al[2] = El[i0 + 4]; al[3] = El[i1 + 4];
             sc::split(Ab[(k0 + t) * DK + n0 + g], bh[0], bl[0]);
             sc::split(Ab[(k0 + t + 4) * DK + n0 + g], bh[1], bl[1]);
-            sc::mma(d, al, bh);
-            sc::mma(d, ah, bl);
-            sc::mma(d, ah, bh);
+            sc::mma(acc[par][0], al, bh);
+            sc::mma(acc[par][1], ah, bl);
+            sc::mma(acc[par][2], ah, bh);
         }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            d[e] += ((acc[0][0][e] + acc[1][0][e]) + (acc[0][1][e] + acc[1][1][e])) + (acc[0][2][e] + acc[1][2][e]);
         // S_start(p+1): to the next running-row buffer and to global
-        float* En = Es + ((p + 1) & 1) * SC_ROWS * LDE;
-        En[g * LDE + n0 + 2 * t] = d[0];
-        En[g * LDE + n0 + 2 * t + 1] = d[1];
-        En[(g + 8) * LDE + n0 + 2 * t] = d[2];
-        En[(g + 8) * LDE + n0 + 2 * t + 1] = d[3];
+        put_row(p + 1, g, n0 + 2 * t, d[0]);
+        put_row(p + 1, g, n0 + 2 * t + 1, d[1]);
+        put_row(p + 1, g + 8, n0 + 2 * t, d[2]);
+        put_row(p + 1, g + 8, n0 + 2 * t + 1, d[3]);
         float* sp = s_at(p + 1);
         *reinterpret_cast<float2*>(sp + g * DK + n0 + 2 * t) = make_float2(d[0], d[1]);
         *reinterpret_cast<float2*>(sp + (g + 8) * DK + n0 + 2 * t) = make_float2(d[2], d[3]);
