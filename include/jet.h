@@ -133,6 +133,45 @@ jet_status jet_gdn_decode_step(const void* q, const void* k, const void* v, cons
                                int B, int H, int dk, int dv, jet_dtype dt, void* stream);
 
 /*
+ * jet_gdn_decode_step with the dynamic causal conv of the new token fused in
+ * (paper sections 2.3 and 2.4): from the token's generated taps (as made by
+ * jet_kernel_gen) and the raw history, v' = w0 v_t + w1 v_{t-1} + w2 v_{t-2}
+ * + w3 v_{t-3} (rounded to the storage type), the history is shifted, and S
+ * is updated in place, in one pass over S.
+ *   q, k [B,H,dk]; v [B,H,dv] raw; hist_in [B,3,H,dv] raw, oldest first, or
+ *   NULL (zeros); hist_out [B,3,H,dv] out (must not overlap hist_in);
+ *   taps [B,H,4] float32 (16-byte aligned); g, beta [B,H] float32;
+ *   S [B,H,dv,dk] float32 in/out; o [B,H,dv] out.
+ */
+jet_status jet_conv_gdn_decode_step(const void* q, const void* k, const void* v,
+                                    const void* hist_in, void* hist_out, const float* taps,
+                                    const float* g, const float* beta, float* S, void* o,
+                                    int B, int H, int dk, int dv, jet_dtype dt, void* stream);
+
+/*
+ * The whole JetBlock mixer for one new token per sequence (steps 1-3 fused;
+ * paper sections 2.3 and 2.4): the kernel generator makes the token's taps,
+ * the dynamic causal conv is applied to v with the raw history, the history
+ * is shifted, and the gated delta rule updates S in place, all with one read
+ * and one write of S. Two launches: jet_kernel_gen, then
+ * jet_conv_gdn_decode_step.
+ *   x [B,D]; w1 [D,hidden], w2 [hidden,H*width] as in jet_kernel_gen;
+ *   q, k [B,H,dk]; v [B,H,dv] raw (before the conv); g, beta [B,H] float32;
+ *   hist_in [B,3,H,dv] raw history, oldest first, or NULL (zeros);
+ *   hist_out [B,3,H,dv] out (must not overlap hist_in);
+ *   S [B,H,dv,dk] float32 in/out; o [B,H,dv] out;
+ *   taps [B,H,width] float32 out (16-byte aligned): the generated conv taps.
+ * Equal, up to floating-point contraction, to jet_dyn_conv_v with T = 1
+ * followed by jet_gdn_decode_step on its output.
+ */
+jet_status jet_jetblock_decode_step(const void* x, const void* w1, const void* w2,
+                                    const void* q, const void* k, const void* v,
+                                    const void* hist_in, void* hist_out,
+                                    const float* g, const float* beta, float* S, void* o,
+                                    float* taps, int B, int D, int H, int dk, int dv,
+                                    int hidden, int width, jet_dtype dt, void* stream);
+
+/*
  * jet_gdn_prefill for callers that cannot allocate device memory. It has no
  * counterpart in the paper; it exists for code that must not call an
  * allocator on its hot path: work recorded into a CUDA graph (allocation is

@@ -8,6 +8,7 @@ no CUDA device is present, the calls raise.
 Function names match the C entry points:
   jet_kernel_gen, jet_dyn_conv_v, jet_gdn_prefill_workspace_size,
   jet_gdn_prefill_workspace_min, jet_gdn_prefill, jet_gdn_prefill_noalloc, jet_gdn_decode_step,
+  jet_jetblock_decode_step, jet_conv_gdn_decode_step,
   jet_device_error, jet_status_string, jet_launch_count.
 """
 from __future__ import annotations
@@ -26,8 +27,9 @@ STATUS = {0: "JET_OK", 1: "JET_ERR_INVALID_ARG", 2: "JET_ERR_UNSUPPORTED", 3: "J
           8: "JET_ERR_TOO_LARGE"}
 EXPORTS = ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill_workspace_size", "jet_gdn_prefill_workspace_min",
            "jet_gdn_prefill",
-           "jet_gdn_prefill_noalloc", "jet_gdn_decode_step", "jet_device_error", "jet_status_string",
-           "jet_launch_count")
+           "jet_gdn_prefill_noalloc", "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step",
+           "jet_device_error",
+           "jet_status_string", "jet_launch_count")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -58,13 +60,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.jet_gdn_prefill.argtypes = [P] * 9 + [Z] + [I] * 7 + [P]
     L.jet_gdn_prefill_noalloc.argtypes = [P] * 8 + [I] * 7 + [P]
     L.jet_gdn_decode_step.argtypes = [P] * 7 + [I] * 5 + [P]
+    L.jet_jetblock_decode_step.argtypes = [P] * 13 + [I] * 8 + [P]
+    L.jet_conv_gdn_decode_step.argtypes = [P] * 10 + [I] * 5 + [P]
     L.jet_device_error.argtypes = [P]
     L.jet_status_string.argtypes = [I]
     L.jet_status_string.restype = ctypes.c_char_p
     L.jet_launch_count.argtypes = []
     L.jet_launch_count.restype = U
     for f in ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill", "jet_gdn_prefill_noalloc",
-              "jet_gdn_decode_step", "jet_device_error"):
+              "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step", "jet_device_error"):
         getattr(L, f).restype = I
     _lib = L
     return L
@@ -206,6 +210,54 @@ def jet_gdn_decode_step(q, k, v, g, beta, S, o=None, *, stream=None):
                                _ptr(S, "S", torch.float32, (B, H, dv, dk)), _ptr(o, "o", q.dtype, (B, H, dv)),
                                B, H, dk, dv, dt, _stream(stream))
     _check("jet_gdn_decode_step", st)
+    return o
+
+
+def jet_jetblock_decode_step(x, W1, W2, q, k, v, hist_in, hist_out, g, beta, S, o=None, taps=None, *,
+                             stream=None):
+    """Generator + conv + history shift + decode update for one new token per
+    sequence. x [B,D], v [B,H,dv] raw, hist_in [B,3,H,dv] or None, hist_out
+    [B,3,H,dv], S [B,H,dv,dk] float32 updated in place. Returns (o, taps)."""
+    L = load_library()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    D = x.shape[-1]
+    hidden, HW = W2.shape
+    width = HW // H
+    dt = _dt(q)
+    if o is None:
+        o = torch.empty((B, H, dv), device=q.device, dtype=q.dtype)
+    if taps is None:
+        taps = torch.empty((B, H, width), device=q.device, dtype=torch.float32)
+    st = L.jet_jetblock_decode_step(
+        _ptr(x, "x", q.dtype, (B, D)), _ptr(W1, "W1", q.dtype, (D, hidden)), _ptr(W2, "W2", q.dtype, (hidden, HW)),
+        _ptr(q, "q"), _ptr(k, "k", q.dtype, q.shape), _ptr(v, "v", q.dtype, (B, H, dv)),
+        _ptr(hist_in, "hist_in", q.dtype, (B, 3, H, dv)), _ptr(hist_out, "hist_out", q.dtype, (B, 3, H, dv)),
+        _ptr(g, "g", torch.float32, (B, H)), _ptr(beta, "beta", torch.float32, (B, H)),
+        _ptr(S, "S", torch.float32, (B, H, dv, dk)), _ptr(o, "o", q.dtype, (B, H, dv)),
+        _ptr(taps, "taps", torch.float32, (B, H, width)),
+        B, D, H, dk, dv, hidden, width, dt, _stream(stream))
+    _check("jet_jetblock_decode_step", st)
+    return o, taps
+
+
+def jet_conv_gdn_decode_step(q, k, v, hist_in, hist_out, taps, g, beta, S, o=None, *, stream=None):
+    """Decode step with the conv of the new token fused in: v [B,H,dv] raw,
+    taps [B,H,4] float32 from jet_kernel_gen, hist_in [B,3,H,dv] or None,
+    hist_out [B,3,H,dv]; S updated in place. Returns o [B,H,dv]."""
+    L = load_library()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dt(q)
+    if o is None:
+        o = torch.empty((B, H, dv), device=q.device, dtype=q.dtype)
+    st = L.jet_conv_gdn_decode_step(
+        _ptr(q, "q"), _ptr(k, "k", q.dtype, q.shape), _ptr(v, "v", q.dtype, (B, H, dv)),
+        _ptr(hist_in, "hist_in", q.dtype, (B, 3, H, dv)), _ptr(hist_out, "hist_out", q.dtype, (B, 3, H, dv)),
+        _ptr(taps, "taps", torch.float32, (B, H, 4)), _ptr(g, "g", torch.float32, (B, H)),
+        _ptr(beta, "beta", torch.float32, (B, H)), _ptr(S, "S", torch.float32, (B, H, dv, dk)),
+        _ptr(o, "o", q.dtype, (B, H, dv)), B, H, dk, dv, dt, _stream(stream))
+    _check("jet_conv_gdn_decode_step", st)
     return o
 
 

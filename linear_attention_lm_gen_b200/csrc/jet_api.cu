@@ -286,19 +286,24 @@ jet_status dispatch_prefill(int dk, const void* q, const void* k, const void* v,
 // ---------------------------------------------------------------- K3
 template <typename T, int NV>
 jet_status launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                         float* S, void* o, int B, int H, int dv, cudaStream_t s) {
+                         float* S, void* o, int B, int H, int dv, const DecConv* conv, cudaStream_t s) {
     dim3 grid((dv + DEC_ROWS - 1) / DEC_ROWS, H, B);
-    gdn_decode_kernel<T, NV><<<grid, DEC_THREADS, 0, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta, S,
-                                                        (T*)o, H, dv);
+    if (conv)
+        gdn_decode_kernel<T, NV, true><<<grid, DEC_THREADS, 0, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta,
+                                                                    S, (T*)o, H, dv, *conv);
+    else
+        gdn_decode_kernel<T, NV><<<grid, DEC_THREADS, 0, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta, S,
+                                                            (T*)o, H, dv);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return launch_status();
 }
 
 template <typename T>
 jet_status dispatch_decode(int dk, const void* q, const void* k, const void* v, const float* g,
-                           const float* beta, float* S, void* o, int B, int H, int dv, cudaStream_t s) {
+                           const float* beta, float* S, void* o, int B, int H, int dv, cudaStream_t s,
+                           const DecConv* conv = nullptr) {
     switch (dk / 16) {
-#define JET_CASE(NV) case NV: return launch_decode<T, NV>(q, k, v, g, beta, S, o, B, H, dv, s);
+#define JET_CASE(NV) case NV: return launch_decode<T, NV>(q, k, v, g, beta, S, o, B, H, dv, conv, s);
         JET_CASE(1) JET_CASE(2) JET_CASE(3) JET_CASE(4) JET_CASE(5) JET_CASE(6) JET_CASE(7) JET_CASE(8)
 #undef JET_CASE
         default: return JET_ERR_UNSUPPORTED;
@@ -399,6 +404,49 @@ jet_status jet_gdn_decode_step(const void* q, const void* k, const void* v, cons
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dt == JET_BF16) return dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, B, H, dv, s);
     return dispatch_decode<float>(dk, q, k, v, g, beta, S, o, B, H, dv, s);
+}
+
+jet_status jet_conv_gdn_decode_step(const void* q, const void* k, const void* v, const void* hist_in,
+                                    void* hist_out, const float* taps, const float* g, const float* beta, float* S,
+                                    void* o, int B, int H, int dk, int dv, jet_dtype dt, void* stream) {
+    if (!q || !k || !v || !g || !beta || !S || !o || !hist_out || !taps) return JET_ERR_INVALID_ARG;
+    if (!dtype_ok(dt)) return JET_ERR_INVALID_ARG;
+    if (elems({B, H, dv, dk}) < 0 || elems({B, 3, H, dv}) < 0) return JET_ERR_INVALID_ARG;
+    if (!shape_ok(dk, dv) || B > 65535 || H > 65535) return JET_ERR_UNSUPPORTED;
+    const size_t es = esize(dt);
+    for (const void* p : {q, k, v, hist_in, (const void*)hist_out, (const void*)o})
+        if (p && !aligned_to(p, es)) return JET_ERR_MISALIGNED;
+    if (!aligned_to(g, 4) || !aligned_to(beta, 4) || !aligned16(S) || !aligned16(taps)) return JET_ERR_MISALIGNED;
+    const size_t nh = (size_t)B * 3 * H * dv * es;
+    if (hist_in && overlap(hist_in, nh, hist_out, nh)) return JET_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const DecConv conv{taps, hist_in, hist_out};
+    if (dt == JET_BF16) return dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, B, H, dv, s, &conv);
+    return dispatch_decode<float>(dk, q, k, v, g, beta, S, o, B, H, dv, s, &conv);
+}
+
+jet_status jet_jetblock_decode_step(const void* x, const void* w1, const void* w2, const void* q, const void* k,
+                                    const void* v, const void* hist_in, void* hist_out, const float* g,
+                                    const float* beta, float* S, void* o, float* taps, int B, int D, int H, int dk,
+                                    int dv, int hidden, int width, jet_dtype dt, void* stream) {
+    jet_status st = check_gen(x, w1, w2, B, 1, D, H, hidden, width, dt);
+    if (st != JET_OK) return st;
+    if (!taps) return JET_ERR_INVALID_ARG;
+    if (!aligned16(taps)) return JET_ERR_MISALIGNED;
+    // validate the decode half before launching anything (no sizes / buffers change between the two)
+    if (!q || !k || !v || !g || !beta || !S || !o || !hist_out) return JET_ERR_INVALID_ARG;
+    if (elems({B, H, dv, dk}) < 0 || elems({B, 3, H, dv}) < 0) return JET_ERR_INVALID_ARG;
+    if (!shape_ok(dk, dv) || B > 65535 || H > 65535) return JET_ERR_UNSUPPORTED;
+    const size_t es = esize(dt);
+    for (const void* p : {q, k, v, hist_in, (const void*)hist_out, (const void*)o})
+        if (p && !aligned_to(p, es)) return JET_ERR_MISALIGNED;
+    if (!aligned_to(g, 4) || !aligned_to(beta, 4) || !aligned16(S)) return JET_ERR_MISALIGNED;
+    const size_t nh = (size_t)B * 3 * H * dv * es;
+    if (hist_in && overlap(hist_in, nh, hist_out, nh)) return JET_ERR_INVALID_ARG;
+    // the taps of the new tokens, then conv + history shift + decode update in one pass over S
+    st = jet_kernel_gen(x, w1, w2, taps, B, 1, D, H, hidden, width, dt, stream);
+    if (st != JET_OK) return st;
+    return jet_conv_gdn_decode_step(q, k, v, hist_in, hist_out, taps, g, beta, S, o, B, H, dk, dv, dt, stream);
 }
 
 jet_status jet_device_error(void* stream) {

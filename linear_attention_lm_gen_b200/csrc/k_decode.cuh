@@ -9,6 +9,13 @@
 //   o_i  = S'_i . q^ = a p_i + c_i (k^ . q^)
 // so one pass over S gives both the update and the output.
 //
+// With CONV the kernel also applies the dynamic causal conv of the new token
+// (Jet-Nemotron paper, section 2.4) to the raw v it reads: with the token's
+// taps w (from the kernel generator) and the raw history v_{t-3..t-1},
+//   v'_t = w0 v_t + w1 v_{t-1} + w2 v_{t-2} + w3 v_{t-3}
+// rounded to the storage precision as the separate conv kernel stores it,
+// and it writes the shifted history (v_{t-2}, v_{t-1}, v_t) for the next step.
+//
 // Mapping: 4 lanes per row, each lane holding dk/16 float4 of the row in an
 // interleaved pattern (lane p reads float4 p, p+4, ...): every load
 // instruction of a warp covers 8 rows x 64 contiguous bytes. A thread owns
@@ -25,11 +32,18 @@ namespace jet {
 constexpr int DEC_THREADS = 256;
 constexpr int DEC_ROWS = 128;    // rows of S per CTA (two per 4-lane group)
 
-template <typename T, int NV>   // NV = dk / 16 float4 per lane
+// history [B][3][H][dv], oldest first; taps [B][H][4]
+struct DecConv {
+    const float* taps;
+    const void* hist_in;     // null: zero history
+    void* hist_out;
+};
+
+template <typename T, int NV, bool CONV = false>   // NV = dk / 16 float4 per lane
 __global__ void __launch_bounds__(DEC_THREADS, NV <= 6 ? 3 : 2)   // 3 CTAs per SM where the registers allow
 gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const float* __restrict__ g, const float* __restrict__ beta,
-                  float* __restrict__ S, T* __restrict__ o, int H, int dv) {
+                  float* __restrict__ S, T* __restrict__ o, int H, int dv, DecConv cv = {}) {
     constexpr int DK = NV * 16;
     __shared__ __align__(16) float sk[DK];
     __shared__ __align__(16) float sq[DK];
@@ -53,8 +67,25 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             s1[i] = ok1 ? ld_stream_f4(r1 + part + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
-    const float vi0 = ok0 ? Elem<T>::ld(v + bh * dv + row0) : 0.f;
-    const float vi1 = ok1 ? Elem<T>::ld(v + bh * dv + row1) : 0.f;
+    float vi0 = ok0 ? Elem<T>::ld(v + bh * dv + row0) : 0.f;
+    float vi1 = ok1 ? Elem<T>::ld(v + bh * dv + row1) : 0.f;
+    // conv inputs: the raw history of both rows (v_{t-3}, v_{t-2}, v_{t-1}), loaded
+    // now and used only after the prologue below, so their latency overlaps it
+    float hv0[3] = {0.f, 0.f, 0.f}, hv1[3] = {0.f, 0.f, 0.f};
+    const long long hb = (long long)b * 3 * H * dv + (long long)h * dv;   // history of (b, h), slot 0
+    const long long hs = (long long)H * dv;                               // slot stride
+    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+    if constexpr (CONV) {
+        w = *reinterpret_cast<const float4*>(cv.taps + bh * 4);
+        const T* hin = static_cast<const T*>(cv.hist_in);
+        if (hin) {
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                if (ok0) hv0[j] = Elem<T>::ld(hin + hb + j * hs + row0);
+                if (ok1) hv1[j] = Elem<T>::ld(hin + hb + j * hs + row1);
+            }
+        }
+    }
     const float a = expf(g[bh]);
     const float bt = beta[bh];
 
@@ -95,6 +126,19 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         p1 += __shfl_xor_sync(0xffffffffu, p1, m);
     }
     u0 *= inv_k; u1 *= inv_k; p0 *= inv_q; p1 *= inv_q;
+    if constexpr (CONV) {   // v' of both rows, and the shifted history
+        T* hout = static_cast<T*>(cv.hist_out);
+        auto conv_row = [&](int row, float raw, const float* hv) -> float {
+            if (part == 0) {
+                Elem<T>::st(hout + hb + row, hv[1]);
+                Elem<T>::st(hout + hb + hs + row, hv[2]);
+                Elem<T>::st(hout + hb + 2 * hs + row, raw);
+            }
+            return Elem<T>::round(w.x * raw + w.y * hv[2] + w.z * hv[1] + w.w * hv[0]);
+        };
+        if (ok0) vi0 = conv_row(row0, vi0, hv0);
+        if (ok1) vi1 = conv_row(row1, vi1, hv1);
+    }
     const float c0 = bt * vi0 - a * bt * u0;
     const float c1 = bt * vi1 - a * bt * u1;
     const float ck0 = c0 * inv_k, ck1 = c1 * inv_k;   // c k^ = (c / |k|) k

@@ -264,15 +264,20 @@ def test_config_long_prefill_sampled(orc, name):
         assert_close(host64(vc[:, :, h, rows]), rvc, s.dtype, f"{name} v' head {h}")
 
 
-def run_decode(d, steps, B, H, dv, dtype_t):
+def run_decode(d, steps, B, H, dv, dtype_t, fused=False):
     """Per step: generator + conv with history ping-pong (T = 1), then the GDN
-    decode step updating S in place. Returns outputs [n,B,H,dv], S, history."""
+    decode step updating S in place (fused: the same as one
+    jet_jetblock_decode_step call). Returns outputs [n,B,H,dv], S, history."""
     S = d["S0"].clone()
     ha, hb = d["hist"].clone(), torch.empty_like(d["hist"])
     outs = []
     for t in range(steps):
-        vc, _ = jet.jet_dyn_conv_v(d["x"][t][:, None], d["W1"], d["W2"], d["v"][t][:, None], ha, None, hb)
-        o = jet.jet_gdn_decode_step(d["q"][t], d["k"][t], vc[:, 0], d["g"][t], d["beta"][t], S)
+        if fused:
+            o, _ = jet.jet_jetblock_decode_step(d["x"][t], d["W1"], d["W2"], d["q"][t], d["k"][t], d["v"][t], ha, hb,
+                                                d["g"][t], d["beta"][t], S)
+        else:
+            vc, _ = jet.jet_dyn_conv_v(d["x"][t][:, None], d["W1"], d["W2"], d["v"][t][:, None], ha, None, hb)
+            o = jet.jet_gdn_decode_step(d["q"][t], d["k"][t], vc[:, 0], d["g"][t], d["beta"][t], S)
         outs.append(o)
         ha, hb = hb, ha
     return torch.stack(outs), S, ha
@@ -283,11 +288,12 @@ def run_decode(d, steps, B, H, dv, dtype_t):
     ("decode_4b_b1", 16, [0]), ("decode_4b_b16", 16, [0, 15]), ("decode_4b_b64", 8, [0, 63]),
     ("decode_4b_b256", 8, [5, 200]), ("decode_4b_b1024", 4, [0, 511, 1023]),
 ])
-def test_config_decode_sampled(orc, name, steps, seqs):
+@pytest.mark.parametrize("fused", [False, True])
+def test_config_decode_sampled(orc, name, steps, seqs, fused):
     s = synth.CONFIGS[name]
     inp = synth.decode_inputs(s, seed=0, steps=steps)
     d = gpu_inputs(inp)
-    o, S, hist = run_decode(d, steps, s.B, s.H, s.dv, d["v"].dtype)
+    o, S, hist = run_decode(d, steps, s.B, s.H, s.dv, d["v"].dtype, fused)
     sel = lambda a: np.ascontiguousarray(a[:, seqs])
     dt = s.dtype
     r = orc.jetblock_decode(synth.to_f64(sel(inp["x"]), dt), synth.to_f64(inp["W1"], dt), synth.to_f64(inp["W2"], dt),
@@ -315,3 +321,26 @@ def test_long_prefill_then_decode_continues(orc):
     r = orc.jetblock_prefill(ref["x"], ref["W1"], ref["W2"], ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"])
     assert_close(host64(o.transpose(0, 1)), r["o"][:, s.T:], "bf16", "decoded o")
     assert_close(host64(S_end), r["S"], "bf16", "S after decode")
+
+
+@pytest.mark.parametrize("dtype,H,dk,dv,hist", [("bf16", 12, 96, 256, True), ("bf16", 3, 128, 64, False),
+                                                ("f32", 2, 16, 32, True)])
+def test_fused_decode_step_equals_the_two_calls(orc, dtype, H, dk, dv, hist):
+    # jet_jetblock_decode_step = jet_dyn_conv_v (T = 1) + jet_gdn_decode_step, step after step
+    s = synth.JetShape("t", B=5, T=1, H=H, dk=dk, dv=dv, D=64, dtype=dtype)
+    inp = synth.decode_inputs(s, seed=11, steps=6)
+    d = gpu_inputs(inp)
+    if not hist:
+        d["hist"] = torch.zeros_like(d["hist"])
+    o1, S1, h1 = run_decode(d, 6, s.B, s.H, s.dv, d["v"].dtype, fused=False)
+    o2, S2, h2 = run_decode(d, 6, s.B, s.H, s.dv, d["v"].dtype, fused=True)
+    assert torch.equal(h1, h2)                              # the history is a copy: bit-exact
+    tol = 1e-5 if dtype == "f32" else 2e-3
+    assert errors(host64(o2), host64(o1))["rel_l2"] < tol
+    assert errors(host64(S2), host64(S1))["rel_l2"] < tol
+    # the taps it returns are the generator's
+    taps = torch.empty((s.B, s.H, 4), device="cuda")
+    jet.jet_jetblock_decode_step(d["x"][0], d["W1"], d["W2"], d["q"][0], d["k"][0], d["v"][0], d["hist"],
+                                 torch.empty_like(d["hist"]), d["g"][0], d["beta"][0], d["S0"].clone(), None, taps)
+    ref = jet.jet_kernel_gen(d["x"][0][:, None], d["W1"], d["W2"], H=s.H)
+    assert torch.equal(taps, ref[:, 0])
