@@ -187,8 +187,8 @@ jet_status jet_jetblock_decode_step(const void* x, const void* w1, const void* w
  * whose scratch fits is used; sizes whose smallest plan needs more
  * (jet_gdn_prefill_workspace_min > JET_NOALLOC_SCRATCH_BYTES) return
  * JET_ERR_TOO_LARGE before anything is launched: the 2B shapes fit at any
- * length (12.4 MB), 16-head dk = 128 shapes longer than 1792 tokens do not
- * (17.8 MB).
+ * length (12.5 MB), 16-head dk = 128 shapes longer than 1792 tokens do not
+ * (18.0 MB).
  * The first call on a device looks the array's device address up (no
  * allocation); make that first call before any stream capture. The array is
  * shared by all calls on a device and keeps the last call's contents (every

@@ -196,7 +196,7 @@ bool tc_prefill_ok(jet_dtype dt, int dk, int dv, long long BT) {
 size_t seg_workspace_floats(int B, int H, int dk, int dv, int P) {
     if (P <= 1) return 0;
     return (size_t)B * (P - 1) * H * dv * dk      // E: phase A end states
-         + (size_t)B * (P - 1) * H * dk * dk      // A: transitions
+         + (size_t)B * (P - 1) * H * dk * pfws::trans_ld(dk)   // A: transitions (padded rows)
          + (size_t)B * P * H * dv * dk;           // start states
 }
 
@@ -256,7 +256,7 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
     if (P == 1) return run(dim3(ns, H, B), pfws::Seg{1, plan.seg_chunks, 1, 0, nullptr, nullptr, nullptr});
     float* E = ws;
     float* A = E + (size_t)B * (P - 1) * H * dv * DK;
-    float* Sst = A + (size_t)B * (P - 1) * H * DK * DK;
+    float* Sst = A + (size_t)B * (P - 1) * H * DK * pfws::trans_ld(DK);
     // phase A: segments 0 .. P-2, value slices plus the transition slice
     if (run(dim3(ns + 1, H, B * (P - 1)), pfws::Seg{P, plan.seg_chunks, P - 1, 1, nullptr, E, A}) != JET_OK)
         return JET_ERR_CUDA;

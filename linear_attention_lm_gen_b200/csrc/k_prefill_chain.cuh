@@ -251,7 +251,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             float* dst = nullptr;
             if (seg.phaseA) {
                 const long long bp = (long long)b * (seg.nseg - 1) + p_seg;
-                if (trans) { if (ct < DK) dst = seg.Ao + ((bp * H + h) * DK + ct) * DK; }
+                if (trans) { if (ct < DK) dst = seg.Ao + ((bp * H + h) * DK + ct) * trans_ld(DK); }
                 else dst = seg.Eo + ((bp * H + h) * dv + c0 + ct) * DK;
             } else if (p_seg == seg.nseg - 1) {
                 dst = S_out + (bh * dv + c0 + ct) * DK;

@@ -33,6 +33,9 @@ constexpr int LDA = 68;                                // fp32 row stride of A /
 constexpr int LDX = 40;                                // row stride of the 32 x 32 block products
 constexpr int LDX1 = 24;                               // row stride of the 16 x 16 block products
 constexpr uint32_t AF_BYTES = 64 * LDA * 4;            // A / T scratch
+// row stride (floats) of a segment transition A_p [dk][dk] in the workspace:
+// padded so that the combine's tensor-core fragment loads hit distinct banks
+__host__ __device__ constexpr int trans_ld(int dk) { return dk + 8; }
 constexpr uint32_t XS_BYTES = 32 * LDX * 4;            // block-product scratch
 
 struct Vec {       // per-token vectors of one chunk (64 floats each)
@@ -153,7 +156,7 @@ struct Seg {
     int phaseA;        // 1: end states and transitions, no outputs
     const float* Sst;  // phase C start states (P > 1): [B][P][H][dv][dk]
     float* Eo;         // phase A end states: [B][P-1][H][dv][dk]
-    float* Ao;         // phase A transitions: [B][P-1][H][dk][dk]
+    float* Ao;         // phase A transitions: [B][P-1][H][dk][trans_ld(dk)]
 };
 
 

@@ -22,6 +22,7 @@
 // current one.
 #pragma once
 #include "common.cuh"
+#include "k_prefill_common.cuh"
 #include "sm100.cuh"
 
 namespace jet {
@@ -31,7 +32,7 @@ constexpr int SC_ROWS = 16;      // state rows per CTA (the MMA's M)
 __host__ __device__ constexpr int sc_threads(int dk) { return 4 * dk; }     // one warp per 8 columns
 __host__ __device__ constexpr int sc_lde(int dk) { return dk + 4; }          // padded row stride of the rows
 __host__ __device__ constexpr size_t sc_smem_bytes(int dk) {
-    return sizeof(float) * (2 * (size_t)dk * dk + 4 * (size_t)SC_ROWS * sc_lde(dk)) + 2 * sizeof(uint64_t);
+    return sizeof(float) * (2 * (size_t)dk * pfws::trans_ld(dk) + 4 * (size_t)SC_ROWS * sc_lde(dk)) + 2 * sizeof(uint64_t);
 }
 
 namespace sc {
@@ -54,7 +55,7 @@ __device__ __forceinline__ void mma(float* d, const uint32_t* a, const uint32_t*
 }
 }  // namespace sc
 
-// E [B][P-1][H][dv][dk], A [B][P-1][H][dk][dk], Sst [B][P][H][dv][dk];
+// E [B][P-1][H][dv][dk], A [B][P-1][H][dk][trans_ld(dk)], Sst [B][P][H][dv][dk];
 // grid (dv / 16, H, B), sc_threads(DK) threads, sc_smem_bytes(DK) shared.
 template <int DK>
 __global__ void __launch_bounds__(4 * DK)
@@ -63,21 +64,22 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
     static_assert(DK % 8 == 0 && DK <= 128, "dk");
     constexpr int LDE = sc_lde(DK);
     extern __shared__ __align__(128) float scm[];
-    float* As = scm;                                  // [2][DK][DK]
+    constexpr int LDAT = pfws::trans_ld(DK);
+    float* As = scm;                                  // [2][DK][LDAT]
     // running rows S_start(p), split once into tf32 hi / lo parts: [2][hi, lo][16][LDE]
-    uint32_t* Es = reinterpret_cast<uint32_t*>(As + 2 * DK * DK);
+    uint32_t* Es = reinterpret_cast<uint32_t*>(As + 2 * DK * LDAT);
     uint64_t* bar = reinterpret_cast<uint64_t*>(Es + 4 * SC_ROWS * LDE);
     auto put_row = [&](int p, int r, int j, float x) {   // S_start(p)[r][j] into the running rows
         uint32_t* e = Es + (p & 1) * 2 * SC_ROWS * LDE + r * LDE + j;
         sc::split(x, e[0], e[SC_ROWS * LDE]);
     };
-    constexpr uint32_t ABYTES = DK * DK * sizeof(float);
+    constexpr uint32_t ABYTES = DK * LDAT * sizeof(float);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3, n0 = warp * 8;
     const int r0 = blockIdx.x * SC_ROWS, h = blockIdx.y, b = blockIdx.z;
     auto e_at = [&](int p) { return E + ((((long long)b * (P - 1) + p) * H + h) * dv + r0) * DK; };
     auto s_at = [&](int p) { return Sst + ((((long long)b * P + p) * H + h) * dv + r0) * DK; };
-    auto a_at = [&](int p) { return A + (((long long)b * (P - 1) + p) * H + h) * DK * DK; };
+    auto a_at = [&](int p) { return A + (((long long)b * (P - 1) + p) * H + h) * DK * LDAT; };
     // this thread's accumulator entries: rows g and g+8, columns n0+2t and n0+2t+1
     auto load_frag = [&](const float* src, float* d) {
         const float2 x = *reinterpret_cast<const float2*>(src + g * DK + n0 + 2 * t);
@@ -94,7 +96,7 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
     if (tid == 0)
         for (int p = 1; p <= 2 && p + 1 < P; ++p) {
             sm100::mbar_expect_tx(&bar[p - 1], ABYTES);
-            sm100::bulk_load(As + (p - 1) * DK * DK, a_at(p), ABYTES, &bar[p - 1]);
+            sm100::bulk_load(As + (p - 1) * DK * LDAT, a_at(p), ABYTES, &bar[p - 1]);
         }
     // S_start(0) = S0 (or zeros); S_start(1) = E_0, also the running rows of step 1
     const float* s0 = S0 ? S0 + (((long long)b * H + h) * dv + r0) * DK : nullptr;
@@ -126,7 +128,7 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
         if (p + 2 < P) load_frag(e_at(p + 1), e_next);      // in flight during this step
         const bool ok = sm100::mbar_wait(&bar[buf], parity);
         if (!__syncthreads_and(ok)) return;                  // timed out: error word already set
-        const float* Ab = As + buf * DK * DK;
+        const float* Ab = As + buf * DK * LDAT;
         const uint32_t* Eh = Es + (p & 1) * 2 * SC_ROWS * LDE;  // S_start(p) rows, hi parts
         const uint32_t* El = Eh + SC_ROWS * LDE;                 // lo parts
         // six independent accumulators (product kind x even / odd k-step) keep
@@ -139,8 +141,8 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
             const int i0 = g * LDE + k0 + t, i1 = (g + 8) * LDE + k0 + t;
             ah[0] = Eh[i0]; ah[1] = Eh[i1]; ah[2] = Eh[i0 + 4]; ah[3] = Eh[i1 + 4];
             al[0] = El[i0]; al[1] = El[i1]; al[2] = El[i0 + 4]; al[3] = El[i1 + 4];
-            sc::split(Ab[(k0 + t) * DK + n0 + g], bh[0], bl[0]);
-            sc::split(Ab[(k0 + t + 4) * DK + n0 + g], bh[1], bl[1]);
+            sc::split(Ab[(k0 + t) * LDAT + n0 + g], bh[0], bl[0]);
+            sc::split(Ab[(k0 + t + 4) * LDAT + n0 + g], bh[1], bl[1]);
             sc::mma(acc[par][0], al, bh);
             sc::mma(acc[par][1], ah, bl);
             sc::mma(acc[par][2], ah, bh);
@@ -159,7 +161,7 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
         __syncthreads();                              // every read of As[buf] and of the old rows done
         if (tid == 0 && p + 3 < P) {                  // A_{p+2} is used by step p + 2 <= P - 2
             sm100::mbar_expect_tx(&bar[buf], ABYTES);
-            sm100::bulk_load(As + buf * DK * DK, a_at(p + 2), ABYTES, &bar[buf]);
+            sm100::bulk_load(As + buf * DK * LDAT, a_at(p + 2), ABYTES, &bar[buf]);
         }
     }
 }
