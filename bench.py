@@ -3,8 +3,10 @@
 
 One step = one serving iteration of the mixer on 2B shapes (H=12, dk=96,
 dv=256, d_model=1536, bf16 inputs, float32 state):
-  prefill  generator+conv (K1) and chunked GDN prefill (K2) over one new
-           4096-token sequence (zero initial state);
+  prefill  one jet_jetblock_prefill call over one new 4096-token sequence
+           (zero initial state): the kernel generator (K1 without the conv),
+           then the chunked GDN prefill (K2) with the conv applied to the raw V
+           tiles inside its state chain;
   decode   generator+conv with history (K1, T=1) and the GDN decode step (K3)
            for 256 running sequences, one token each; the state advances in
            place from step to step (64 pre-drawn token sets, cycled).
@@ -63,9 +65,14 @@ def model_bytes():
     k1d = Dc.B * (Dc.D * e + 2 * Dc.H * Dc.dv * e + 2 * 3 * Dc.H * Dc.dv * e) + (Dc.D * 32 + 32 * Dc.H * 4) * e
     k3d = Dc.B * Dc.H * (2 * Dc.dv * Dc.dk * 4 + 2 * Dc.dk * e + 2 * Dc.dv * e + 8)
     k3d_flops = Dc.B * Dc.H * 7 * Dc.dk * Dc.dv
+    # generator + conv + GDN in one call: x, q, k, raw v, g, beta read once, o and the
+    # final state written once (v' never leaves the chip); taps are on-chip-sized (4 floats per token and head)
+    kjp = T * (P.D * e + P.H * (2 * P.dk * e + 2 * P.dv * e + 8)) + P.B * P.H * P.dv * P.dk * 4 \
+        + (P.D * 32 + 32 * P.H * 4) * e
     return {
         "genconv_prefill": dict(bytes=k1p, flops=T * (2 * P.D * 32 + 2 * 32 * P.H * 4 + 8 * P.H * P.dv)),
         "gdn_prefill": dict(bytes=k2p, flops=k2p_flops),
+        "jetblock_prefill": dict(bytes=kjp, flops=T * (2 * P.D * 32 + 2 * 32 * P.H * 4 + 8 * P.H * P.dv) + k2p_flops),
         "genconv_decode": dict(bytes=k1d, flops=Dc.B * (2 * Dc.D * 32 + 8 * Dc.H * Dc.dv)),
         "gdn_decode": dict(bytes=k3d, flops=k3d_flops),
     }
@@ -155,8 +162,7 @@ class Workload:
         self.d = {k: v.to(device) for k, v in self.host_d.items()}
         P, Dc = PREFILL, DECODE
         bf = torch.bfloat16
-        self.vc = torch.empty((P.B, P.T, P.H, P.dv), device=device, dtype=bf)
-        self.ob = [torch.empty_like(self.vc) for _ in range(2)]
+        self.ob = [torch.empty((P.B, P.T, P.H, P.dv), device=device, dtype=bf) for _ in range(2)]
         self.o = self.ob[0]
         self.S_out = torch.empty((P.B, P.H, P.dv, P.dk), device=device, dtype=torch.float32)
         self.S = self.d["S0"].clone()
@@ -164,14 +170,16 @@ class Workload:
         self.vc_d = torch.empty((Dc.B, 1, Dc.H, Dc.dv), device=device, dtype=bf)
         self.odb = [torch.empty((Dc.B, Dc.H, Dc.dv), device=device, dtype=bf) for _ in range(2)]
         self.o_d = self.odb[0]
-        ws = jet.jet_gdn_prefill_workspace_size(P.B, P.T, P.H, P.dk, P.dv)
+        ws = jet.jet_jetblock_prefill_workspace_size(P.B, P.T, P.H, P.dk, P.dv)
         self.ws = torch.empty(max(ws, 16), device=device, dtype=torch.uint8)
         # pinned host buffers for the end-to-end pass
         self.h_o = [torch.empty(self.o.shape, dtype=bf).pin_memory() for _ in range(2)]
         self.h_o_d = [torch.empty(self.o_d.shape, dtype=bf).pin_memory() for _ in range(2)]
         self.steps_done = 0
 
-    # four calls: K1 prefill, K2 prefill (prep + chain phases), K1 decode, K3 decode
+    # the library calls of one step, in order (each timed between two events)
+    CALLS = ("jetblock_prefill", "genconv_decode", "gdn_decode")
+
     def step(self, stream, i: int, ev=None, counts=None, buf: int = 0):
         jet, p, d = self.jet, self.pb[buf], self.d
         o, o_d = self.ob[buf], self.odb[buf]
@@ -182,21 +190,20 @@ class Workload:
             if counts is not None:
                 counts.append(jet.jet_launch_count())
         mark(0)
-        jet.jet_dyn_conv_v(p["x"], p["W1"], p["W2"], p["v"], None, self.vc, stream=stream)
+        # prefill: generator, then the GDN prefill with the conv inside its chain (one call)
+        jet.jet_jetblock_prefill(p["x"], p["W1"], p["W2"], p["q"], p["k"], p["v"], p["g"], p["beta"], None, None,
+                                 None, o, self.S_out, self.ws, stream=stream)
         mark(1)
-        jet.jet_gdn_prefill(p["q"], p["k"], self.vc, p["g"], p["beta"], None, o, self.S_out, self.ws,
-                            stream=stream)
-        mark(2)
         s = i % DECODE.steps
         hin, hout = self.hist[i % 2], self.hist[(i + 1) % 2]
         # decode: generator + conv with the history (T = 1), then the state update. (Folding the conv
         # into the state pass, jet_conv_gdn_decode_step, measured slower on this step: 127 vs 115 us.)
         jet.jet_dyn_conv_v(d["x"][s][:, None], d["W1"], d["W2"], d["v"][s][:, None], hin, self.vc_d, hout,
                            stream=stream)
-        mark(3)
+        mark(2)
         jet.jet_gdn_decode_step(d["q"][s], d["k"][s], self.vc_d[:, 0], d["g"][s], d["beta"][s], self.S, o_d,
                                 stream=stream)
-        mark(4)
+        mark(3)
 
     def h2d(self, i: int, buf: int) -> int:
         """Copy one step's inputs from pinned host memory (current stream); returns bytes."""
@@ -354,12 +361,13 @@ def run_jet(args):
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             wl.step(stream, i, counts=counts if i == args.warmup - 1 else None)
-    per_call_launches = np.diff(np.array(counts))   # kernel launches behind each of the four calls
+    per_call_launches = np.diff(np.array(counts))   # kernel launches behind each call of a step
     if jet.jet_device_error(stream) != 0:
         raise RuntimeError("device error word set after warm-up")
 
     # ---- device-resident timed pass (per-kernel events inside it)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    ncall = len(Workload.CALLS)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(ncall + 1)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     time.sleep(0.3)
@@ -376,9 +384,9 @@ def run_jet(args):
     launches = jet.jet_launch_count() - n0
     clk = clocks.stop(t_wall0, t_wall1)
     ms = max_over_ranks(start.elapsed_time(stop))
-    per_kernel = np.zeros(4)
+    per_kernel = np.zeros(ncall)
     for e in evs:
-        for j in range(4):
+        for j in range(ncall):
             per_kernel[j] += e[j].elapsed_time(e[j + 1])
     per_kernel /= args.steps                      # ms per launch
     if jet.jet_device_error(stream) != 0:
@@ -428,7 +436,7 @@ def run_jet(args):
 
     pk = peaks()
     mb = model_bytes()
-    names = ["genconv_prefill", "gdn_prefill", "genconv_decode", "gdn_decode"]
+    names = list(Workload.CALLS)
     kern = {}
     for j, n in enumerate(names):
         t = per_kernel[j] * 1e-3
@@ -445,8 +453,8 @@ def run_jet(args):
     ach = kern[dom]["achieved_gbs"]
     tokens = TOKENS_PER_STEP * world
     value = rk.value(TOKENS_PER_STEP, args.steps, ms)
-    prefill_ms = per_kernel[0] + per_kernel[1]
-    decode_ms = per_kernel[2] + per_kernel[3]
+    prefill_ms = per_kernel[0]
+    decode_ms = per_kernel[1] + per_kernel[2]
     roof_step_us = sum(k["roofline_us"] for k in kern.values())
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -466,7 +474,7 @@ def run_jet(args):
                           "frac": roof_step_us / (1e3 * ms / args.steps)},
         "phases": {
             "prefill": {"tokens_per_s": PREFILL.T / (prefill_ms * 1e-3), "us": prefill_ms * 1e3,
-                        "roofline_us": kern["genconv_prefill"]["roofline_us"] + kern["gdn_prefill"]["roofline_us"]},
+                        "roofline_us": kern["jetblock_prefill"]["roofline_us"]},
             "decode": {"tokens_per_s": DECODE.B / (decode_ms * 1e-3), "us": decode_ms * 1e3,
                        "roofline_us": kern["genconv_decode"]["roofline_us"] + kern["gdn_decode"]["roofline_us"]}},
         "kernels": kern,

@@ -94,7 +94,7 @@ jet_status jet_dyn_conv_v(const void* x, const void* w1, const void* w2, const v
  * Device workspace of jet_gdn_prefill for these sizes, in bytes (either may
  * be 0). With at least jet_gdn_prefill_workspace_size bytes the prefill runs
  * its fastest plan: every chunk's state-independent part is prepared at once
- * into per-chunk tiles (about 45 KB per chunk of 64 tokens and head at
+ * into per-chunk tiles (about 47 KB per chunk of 64 tokens and head at
  * dk = 96, so this grows with B * T * H), then the state chain runs. With
  * at least jet_gdn_prefill_workspace_min bytes (the sequence-parallel
  * segment buffers only, at most a few tens of MB and independent of T beyond
@@ -121,6 +121,41 @@ jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const fl
                            void* workspace, size_t ws_bytes,
                            int B, int T, int H, int dk, int dv, int chunk,
                            jet_dtype dt, void* stream);
+
+/*
+ * The whole JetBlock mixer over a prompt (steps 1-3; paper sections 2.3 and
+ * 2.4): the kernel generator makes every token's taps, the dynamic causal
+ * conv is applied to the raw v, and the chunked gated delta rule runs on the
+ * result. On the tensor-core path (bf16, dk in {64, 96, 128}, dv a multiple
+ * of 128) the conv is folded into each chunk's UT transform (U = T diag(b) V'
+ * is linear in the raw V, with a three-token reach into the previous chunk),
+ * so v' is never formed; elsewhere a separate conv pass writes v' into the
+ * workspace and the SIMT prefill reads it.
+ *   x [B,T,D]; w1 [D,hidden], w2 [hidden,H*width] as in jet_kernel_gen.
+ *   q, k [B,T,H,dk]; v [B,T,H,dv] raw (before the conv); g, beta [B,T,H] float32.
+ *   hist_in [B,3,H,dv] raw V of the 3 positions before token 0, oldest first,
+ *     or NULL (zeros: the start of a sequence).
+ *   hist_out [B,3,H,dv] or NULL: the last 3 raw V positions of [hist_in, v]
+ *     (the history for the decode steps that follow). Must overlap neither
+ *     hist_in nor v.
+ *   S0, o, S_out as in jet_gdn_prefill (S_out may alias S0); o must not overlap v.
+ *   workspace / ws_bytes: at least jet_jetblock_prefill_workspace_size(...)
+ *     bytes (the taps, then the chunk images and segment buffers of the
+ *     fastest jet_gdn_prefill plan, or a v' buffer off the tensor-core path);
+ *     otherwise JET_ERR_WORKSPACE before any launch. Contents on entry are ignored.
+ * o and S_out agree with jet_dyn_conv_v followed by jet_gdn_prefill within
+ * the bf16 tolerance (the folded path never rounds v' to bf16), not bit for bit.
+ * A history containing Inf or NaN can reach the first chunk of the next
+ * sequence in the batch (its values meet zero weights there).
+ */
+size_t jet_jetblock_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt);
+jet_status jet_jetblock_prefill(const void* x, const void* w1, const void* w2,
+                                const void* q, const void* k, const void* v,
+                                const void* hist_in, void* hist_out,
+                                const float* g, const float* beta, const float* S0,
+                                void* o, float* S_out, void* workspace, size_t ws_bytes,
+                                int B, int T, int D, int H, int dk, int dv,
+                                int hidden, int width, int chunk, jet_dtype dt, void* stream);
 
 /*
  * One decode step (step 3 for a single new token per sequence), updating S in place:

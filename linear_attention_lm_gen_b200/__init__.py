@@ -8,7 +8,8 @@ no CUDA device is present, the calls raise.
 Function names match the C entry points:
   jet_kernel_gen, jet_dyn_conv_v, jet_gdn_prefill_workspace_size,
   jet_gdn_prefill_workspace_min, jet_gdn_prefill, jet_gdn_prefill_noalloc, jet_gdn_decode_step,
-  jet_jetblock_decode_step, jet_conv_gdn_decode_step,
+  jet_jetblock_decode_step, jet_conv_gdn_decode_step, jet_jetblock_prefill_workspace_size,
+  jet_jetblock_prefill,
   jet_device_error, jet_status_string, jet_launch_count.
 """
 from __future__ import annotations
@@ -28,7 +29,7 @@ STATUS = {0: "JET_OK", 1: "JET_ERR_INVALID_ARG", 2: "JET_ERR_UNSUPPORTED", 3: "J
 EXPORTS = ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill_workspace_size", "jet_gdn_prefill_workspace_min",
            "jet_gdn_prefill",
            "jet_gdn_prefill_noalloc", "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step",
-           "jet_device_error",
+           "jet_jetblock_prefill_workspace_size", "jet_jetblock_prefill", "jet_device_error",
            "jet_status_string", "jet_launch_count")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -62,13 +63,17 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.jet_gdn_decode_step.argtypes = [P] * 7 + [I] * 5 + [P]
     L.jet_jetblock_decode_step.argtypes = [P] * 13 + [I] * 8 + [P]
     L.jet_conv_gdn_decode_step.argtypes = [P] * 10 + [I] * 5 + [P]
+    L.jet_jetblock_prefill_workspace_size.argtypes = [I] * 7
+    L.jet_jetblock_prefill_workspace_size.restype = Z
+    L.jet_jetblock_prefill.argtypes = [P] * 14 + [Z] + [I] * 10 + [P]
     L.jet_device_error.argtypes = [P]
     L.jet_status_string.argtypes = [I]
     L.jet_status_string.restype = ctypes.c_char_p
     L.jet_launch_count.argtypes = []
     L.jet_launch_count.restype = U
     for f in ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill", "jet_gdn_prefill_noalloc",
-              "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step", "jet_device_error"):
+              "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step", "jet_jetblock_prefill",
+              "jet_device_error"):
         getattr(L, f).restype = I
     _lib = L
     return L
@@ -193,6 +198,45 @@ def jet_gdn_prefill_noalloc(q, k, v, g, beta, S0, o, S_out, *, stream=None):
                                    _ptr(S_out, "S_out", torch.float32, (B, H, dv, dk)),
                                    B, T, H, dk, dv, 64, _dt(q), _stream(stream))
     _check("jet_gdn_prefill_noalloc", st)
+    return o, S_out
+
+
+def jet_jetblock_prefill_workspace_size(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
+    """Workspace bytes of jet_jetblock_prefill (taps + the prefill's fastest plan)."""
+    L = load_library()
+    return int(L.jet_jetblock_prefill_workspace_size(B, T, H, dk, dv, chunk,
+                                                     JET_BF16 if dtype == torch.bfloat16 else JET_F32))
+
+
+def jet_jetblock_prefill(x, W1, W2, q, k, v, g, beta, hist_in=None, hist_out=None, S0=None, o=None, S_out=None,
+                         workspace=None, *, stream=None):
+    """Generator + dynamic conv + chunked Gated DeltaNet over a prompt. x [B,T,D],
+    q,k [B,T,H,dk], v [B,T,H,dv] raw, g,beta [B,T,H] float32, hist_in / hist_out
+    [B,3,H,dv] or None, S0 [B,H,dv,dk] float32 or None. Returns (o, S_out)."""
+    L = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    D = x.shape[-1]
+    hidden, HW = W2.shape
+    width = HW // H
+    dt = _dt(q)
+    if o is None:
+        o = torch.empty((B, T, H, dv), device=q.device, dtype=q.dtype)
+    if S_out is None:
+        S_out = torch.empty((B, H, dv, dk), device=q.device, dtype=torch.float32)
+    if workspace is None:
+        workspace = torch.empty(max(1, jet_jetblock_prefill_workspace_size(B, T, H, dk, dv, 64, q.dtype)),
+                                device=q.device, dtype=torch.uint8)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = L.jet_jetblock_prefill(
+        _ptr(x, "x", q.dtype, (B, T, D)), _ptr(W1, "W1", q.dtype, (D, hidden)), _ptr(W2, "W2", q.dtype, (hidden, HW)),
+        _ptr(q, "q"), _ptr(k, "k", q.dtype, q.shape), _ptr(v, "v", q.dtype, (B, T, H, dv)),
+        _ptr(hist_in, "hist_in", q.dtype, (B, 3, H, dv)), _ptr(hist_out, "hist_out", q.dtype, (B, 3, H, dv)),
+        _ptr(g, "g", torch.float32, (B, T, H)), _ptr(beta, "beta", torch.float32, (B, T, H)),
+        _ptr(S0, "S0", torch.float32, (B, H, dv, dk)), _ptr(o, "o", q.dtype, (B, T, H, dv)),
+        _ptr(S_out, "S_out", torch.float32, (B, H, dv, dk)), _ptr(workspace, "workspace"), ws_bytes,
+        B, T, D, H, dk, dv, hidden, width, 64, dt, _stream(stream))
+    _check("jet_jetblock_prefill", st)
     return o, S_out
 
 

@@ -64,6 +64,14 @@ template <> struct Vec16<__nv_bfloat16> {
 __device__ __forceinline__ float4 ld_stream_f4(const float4* p) { return __ldcs(p); }
 __device__ __forceinline__ void st_stream_f4(float4* p, const float4& v) { __stcs(p, v); }
 
+// One output of the width-4 dynamic causal conv (Jet-Nemotron paper, section
+// 2.4): v'_t = w0 v_t + w1 v_{t-1} + w2 v_{t-2} + w3 v_{t-3}, always evaluated
+// in this order, so that every kernel that applies the conv (the generator /
+// conv pass, the fused decode and the prefill chain) rounds identically.
+__device__ __forceinline__ float conv4(const float4& w, float v0, float v1, float v2, float v3) {
+    return fmaf(w.w, v3, fmaf(w.z, v2, fmaf(w.y, v1, w.x * v0)));
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -155,13 +155,13 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// bf16 tensor [rows][H][d] viewed as 3-D (d, H, rows); box (64, 1, 64), 128-byte swizzle
-bool tile_map(CUtensorMap* m, const void* base, int d, int H, long long rows) {
+// bf16 tensor [rows][H][d] viewed as 3-D (d, H, rows); box (64, 1, box_rows), 128-byte swizzle
+bool tile_map(CUtensorMap* m, const void* base, int d, int H, long long rows, int box_rows = 64) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)rows};
     const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * H * 2};
-    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
     const cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -216,16 +216,28 @@ size_t split_img_bytes(int B, int T, int H, int dk) {
 // the chain kernel K2b runs (workspace = images + segment buffers); otherwise
 // the fused kernel prepares chunk c+1 while it runs chunk c (workspace =
 // segment buffers only). Sequence-parallel segments as planned above.
-template <int DK, bool SPLIT>
+// CONV (split plan only): v is the raw V; the preparation folds the dynamic
+// conv with `taps` into the chunk images and the chain reads the values
+// before each segment (and the history of `cv`) for it.
+template <int DK, bool SPLIT, bool CONV = false>
 jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const float* g, const float* beta,
                              const float* S0, void* o, float* S_out, void* workspace, int B, int Tn, int H,
-                             int dv, cudaStream_t s) {
-    CUtensorMap mq, mk, mv;
+                             int dv, cudaStream_t s, const float* taps = nullptr,
+                             const pfch::ChainConv& cv = pfch::ChainConv{}) {
+    static_assert(SPLIT || !CONV, "the conv is folded in by the preparation kernel of the split plan");
+    CUtensorMap mq, mk, mv, mvh, mhh;
     const long long rows = (long long)B * Tn;
     if (!tile_map(&mq, q, DK, H, rows) || !tile_map(&mk, k, DK, H, rows) || !tile_map(&mv, v, dv, H, rows))
         return JET_ERR_CUDA;
+    // 16-row boxes of V and of the history (the values before a segment)
+    mvh = mv;
+    mhh = mv;
+    if (CONV && (!tile_map(&mvh, v, dv, H, rows, 16) ||
+                 (cv.hist_in && !tile_map(&mhh, cv.hist_in, dv, H, (long long)B * 3, 16))))
+        return JET_ERR_CUDA;
+    if (CONV && !cv.hist_in) mhh = mvh;
     auto fused = pfws::gdn_prefill_ws_kernel<DK>;
-    auto chain = pfch::gdn_prefill_chain_kernel<DK>;
+    auto chain = pfch::gdn_prefill_chain_kernel<DK, CONV>;
     const uint32_t smem = SPLIT ? pfch::ChainSmem<DK>::BYTES : pfws::SMEM_BYTES;
     const int threads = SPLIT ? pfch::THREADS : pfws::THREADS;
     if ((SPLIT ? smem_attr(chain, smem) : smem_attr(fused, smem)) != JET_OK) return JET_ERR_CUDA;
@@ -237,14 +249,15 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
         const int nct = (Tn + pfws::C - 1) / pfws::C;
         const long long items = (long long)B * H * nct;
         const int grid = (int)std::min<long long>(items, (long long)pfws::PREP_CTAS * kSMs);   // resident CTAs
-        prep<<<grid, pfws::PREP_THREADS, pfws::PrepSmem<DK>::BYTES, s>>>(mq, mk, g, beta, img, Tn, H, nct,
-                                                                         (int)items);
+        prep<<<grid, pfws::PREP_THREADS, pfws::PrepSmem<DK>::BYTES, s>>>(
+            mq, mk, g, beta, CONV ? taps : nullptr, cv.hist_in != nullptr, img, Tn, H, nct, (int)items);
         g_launches.fetch_add(1, std::memory_order_relaxed);
         if (launch_status() != JET_OK) return JET_ERR_CUDA;
     }
     auto run = [&](dim3 grid, const pfws::Seg& seg) {
         if (SPLIT)
-            chain<<<grid, threads, smem, s>>>(mk, mv, img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg);
+            chain<<<grid, threads, smem, s>>>(mk, mv, mvh, mhh, img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg,
+                                              cv);
         else
             fused<<<grid, threads, smem, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg);
         g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -389,6 +402,68 @@ jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const fl
     if (dt == JET_BF16)
         return dispatch_prefill<__nv_bfloat16>(dk, q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
     return dispatch_prefill<float>(dk, q, k, v, g, beta, S0, o, S_out, B, T, H, dv, s);
+}
+
+// ---- generator + conv + GDN prefill in one call
+// workspace: [taps B*T*H*4 float32 | rest], each part 1024-byte aligned; rest =
+// the split-plan workspace of the tensor-core path (the chain applies the
+// conv), else a v' buffer for the separate conv pass and the SIMT prefill
+size_t jet_jetblock_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt) {
+    if (B <= 0 || T <= 0 || H <= 0 || dv <= 0 || chunk != 64 || !dtype_ok(dt)) return 0;
+    const long long nt = elems({B, T, H, 4}), nv = elems({B, T, H, dv});
+    if (nt < 0 || nv < 0) return 0;
+    auto up = [](size_t x) { return (x + 1023) & ~size_t(1023); };
+    const size_t taps = up((size_t)nt * sizeof(float));
+    if (tc_prefill_ok(dt, dk, dv, (long long)B * T))
+        return taps + jet_gdn_prefill_workspace_size(B, T, H, dk, dv, chunk, dt);
+    return taps + up((size_t)nv * esize(dt));
+}
+
+jet_status jet_jetblock_prefill(const void* x, const void* w1, const void* w2, const void* q, const void* k,
+                                const void* v, const void* hist_in, void* hist_out, const float* g,
+                                const float* beta, const float* S0, void* o, float* S_out, void* workspace,
+                                size_t ws_bytes, int B, int T, int D, int H, int dk, int dv, int hidden, int width,
+                                int chunk, jet_dtype dt, void* stream) {
+    jet_status st = check_gen(x, w1, w2, B, T, D, H, hidden, width, dt);
+    if (st != JET_OK) return st;
+    if (!q || !k || !v || !g || !beta || !o || !S_out) return JET_ERR_INVALID_ARG;
+    const long long nv = elems({B, T, H, dv}), nh = elems({B, 3, H, dv});
+    if (elems({B, T, H, dk}) < 0 || nv < 0 || nh < 0 || elems({B, H, dv, dk}) < 0) return JET_ERR_INVALID_ARG;
+    if (!shape_ok(dk, dv) || chunk != 64 || B > 65535 || H > 65535) return JET_ERR_UNSUPPORTED;
+    for (const void* p : {q, k, v, hist_in, (const void*)hist_out, (const void*)S0, (const void*)o,
+                          (const void*)S_out, (const void*)workspace})
+        if (p && !aligned16(p)) return JET_ERR_MISALIGNED;
+    if (!aligned_to(g, 4) || !aligned_to(beta, 4)) return JET_ERR_MISALIGNED;
+    const size_t es = esize(dt), vb = (size_t)nv * es, hb = (size_t)nh * es;
+    // v is read (raw, and around segment starts) while o and the new history are written
+    if (overlap(v, vb, o, vb)) return JET_ERR_INVALID_ARG;
+    if (hist_out && (overlap(v, vb, hist_out, hb) || (hist_in && overlap(hist_in, hb, hist_out, hb))))
+        return JET_ERR_INVALID_ARG;
+    if (!workspace) ws_bytes = 0;
+    if (ws_bytes < jet_jetblock_prefill_workspace_size(B, T, H, dk, dv, chunk, dt)) return JET_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* taps = static_cast<float*>(workspace);
+    uint8_t* rest = static_cast<uint8_t*>(workspace) + ((elems({B, T, H, 4}) * sizeof(float) + 1023) & ~size_t(1023));
+    if (tc_prefill_ok(dt, dk, dv, (long long)B * T)) {
+        st = launch_genconv<__nv_bfloat16>(x, w1, w2, nullptr, nullptr, nullptr, nullptr, taps, B, T, D, H, dv, s);
+        if (st != JET_OK) return st;
+        const pfch::ChainConv cv{static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(hist_in),
+                                 static_cast<__nv_bfloat16*>(hist_out)};
+#define JET_TC(DK) \
+        return launch_prefill_tc<DK, true, true>(q, k, v, g, beta, S0, o, S_out, rest, B, T, H, dv, s, taps, cv);
+        if (dk == 64) { JET_TC(64) }
+        if (dk == 96) { JET_TC(96) }
+        JET_TC(128)
+#undef JET_TC
+    }
+    // other shapes and float32: the conv pass writes v' into the workspace, then the SIMT prefill
+    st = dt == JET_BF16
+             ? launch_genconv<__nv_bfloat16>(x, w1, w2, v, hist_in, rest, hist_out, taps, B, T, D, H, dv, s)
+             : launch_genconv<float>(x, w1, w2, v, hist_in, rest, hist_out, taps, B, T, D, H, dv, s);
+    if (st != JET_OK) return st;
+    if (dt == JET_BF16)
+        return dispatch_prefill<__nv_bfloat16>(dk, q, k, rest, g, beta, S0, o, S_out, B, T, H, dv, s);
+    return dispatch_prefill<float>(dk, q, k, rest, g, beta, S0, o, S_out, B, T, H, dv, s);
 }
 
 jet_status jet_gdn_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,

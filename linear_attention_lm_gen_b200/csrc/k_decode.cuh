@@ -134,7 +134,7 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
                 Elem<T>::st(hout + hb + hs + row, hv[2]);
                 Elem<T>::st(hout + hb + 2 * hs + row, raw);
             }
-            return Elem<T>::round(w.x * raw + w.y * hv[2] + w.z * hv[1] + w.w * hv[0]);
+            return Elem<T>::round(conv4(w, raw, hv[2], hv[1], hv[0]));
         };
         if (ok0) vi0 = conv_row(row0, vi0, hv0);
         if (ok1) vi1 = conv_row(row1, vi1, hv1);

@@ -227,7 +227,7 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
             float out[VN];
 #pragma unroll
             for (int e = 0; e < VN; ++e)
-                out[e] = w4.x * cv[e] + w4.y * win[0][e] + w4.z * win[1][e] + w4.w * win[2][e];
+                out[e] = conv4(w4, cv[e], win[0][e], win[1][e], win[2][e]);
             *reinterpret_cast<uint4*>(v_out + rr * rowstride + coff) = V16::pack(out);
 #pragma unroll
             for (int e = 0; e < VN; ++e) { win[2][e] = win[1][e]; win[1][e] = win[0][e]; win[0][e] = cv[e]; }

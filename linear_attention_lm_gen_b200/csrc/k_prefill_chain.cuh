@@ -29,6 +29,16 @@
 // they wake within tens of cycles; the others sleep between polls and leave
 // the issue slots to them.
 // Segments (sequence parallelism) work as in the fused kernel: see Seg.
+//
+// CONV: the V tiles hold the raw values and the images were prepared with
+// the dynamic causal conv (Jet-Nemotron paper, section 2.4) folded into T1:
+// U^T = V^T M^T + Vh^T MH, where Vh = the 16 tokens before the chunk (only the
+// last three have non-zero weights). Vh is the tail of the previous chunk's V
+// tile, still in shared memory: V(c+1) is loaded once P2a(c) is done (one
+// chunk ahead instead of two), and the tail before a segment's first chunk
+// is loaded on its own (from V, or from the history at a sequence start).
+// So v' is never formed at all; the last segment writes the new history (the
+// last three raw values) from global memory.
 #pragma once
 #include "k_prefill_chunkprep.cuh"
 
@@ -71,8 +81,9 @@ struct ChainSmem {
     static constexpr uint32_t AS = V + 2 * 16384;            // NKB x [128 rows][64 feat] bf16 S
     static constexpr uint32_t AW = AS + NKB * 16384;         // Wt^T
     static constexpr uint32_t AWD = AW + 16384;              // Wt^T diag(d/|k|)
-    static constexpr uint32_t OUT = AWD + 16384;             // [32 tok][128 ch] bf16 output staging
-    static constexpr uint32_t BAR = OUT + 8192;
+    static constexpr uint32_t OUT = AWD + 16384;             // [OUT_TOK tok][128 ch] bf16 output staging
+    static constexpr int OUT_TOK = OUT + 8192 + 256 + 32 <= 232448 ? 32 : 16;
+    static constexpr uint32_t BAR = OUT + OUT_TOK * 256;
     static constexpr uint32_t TSLOT = BAR + 256;
     static constexpr uint32_t ABORT = TSLOT + 16;
     // no alignment slack: the kernel checks that dynamic shared memory starts
@@ -83,6 +94,13 @@ struct ChainSmem {
 };
 
 constexpr uint32_t TM_S = 0, TM_X1 = 128, TM_X2 = 256, TM_COLS = 512;
+
+// raw-V conv inputs of the CONV instantiation
+struct ChainConv {
+    const __nv_bfloat16* v;          // raw v [B*T][H][dv] (the tensor map's tensor)
+    const __nv_bfloat16* hist_in;    // [B][3][H][dv] raw v_{-3..-1}, or null (zeros)
+    __nv_bfloat16* hist_out;         // [B][3][H][dv] last three raw tokens, or null
+};
 
 enum {
     B_IMG = 0,        // [2] image landed
@@ -95,14 +113,18 @@ enum {
     B_AW = 12,        // Wt^T copies written (chain)
     B_X2FREE = 13,    // [2] O^T read (out)
     B_ODONE = 15,     // [2] P5a / P5b complete (O^T ready, S copy and Wt^T free)
-    NBARS = 17
+    B_H0 = 17,        // the values before a segment's first chunk landed (CONV)
+    NBARS = 18
 };
 
-template <int DK>
+// tm_vh / tm_hh (CONV): 16-row boxes of V ([B*T][H][dv]) and of the history
+// ([B*3][H][dv]; tm_vh again without one) for the values before a segment
+template <int DK, bool CONV>
 __global__ void __launch_bounds__(THREADS, 1)
 gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ CUtensorMap tm_hh,
                          const uint8_t* __restrict__ img, const float* S0, __nv_bfloat16* __restrict__ o,
-                         float* S_out, int Tn, int H, int dv, const Seg seg) {
+                         float* S_out, int Tn, int H, int dv, const Seg seg, const ChainConv cv) {
     static_assert(DK % 32 == 0 && DK >= 64 && DK <= 128, "DK in {64, 96, 128}");
     using SM = ChainSmem<DK>;
     using IM = Img<DK>;
@@ -142,6 +164,10 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
     if (tid == LOAD0) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
+        if (CONV) {
+            tma_prefetch_desc(&tm_vh);
+            tma_prefetch_desc(&tm_hh);
+        }
     }
     if (warp == 0) tmem_alloc(tslot, TM_COLS);
     tc_fence_before();
@@ -271,36 +297,57 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         }
     } else if (warp < 8) {
         // =============================================================== OUT
-        if (write_o) {
-            const int ot = tid - OUT0;                       // channel of the slice
-            const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
-            __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sm + SM::OUT);
-            const long long tstride = (long long)H * dv;
-            for (int c = 0; c < nch; ++c) {
-                if (!group_wait(&bars[B_ODONE + (c & 1)], (c >> 1) & 1, abort_flag, 3, NOUT, ot == 0, false)) break;
-                tc_fence_after();
-                const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
-                const int t0 = tbeg + c * C, L = min(C, tend - t0);
-                __nv_bfloat16* obase = o + ((long long)b * Tn + t0) * tstride + (long long)h * dv + c0;
+        constexpr int OUT_TOK = SM::OUT_TOK;                 // tokens per staging round
+        const int ot = tid - OUT0;                           // channel of the slice
+        const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
+        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(sm + SM::OUT);
+        const long long tstride = (long long)H * dv;
+        bool run = true;
+        for (int c = 0; c < nch && write_o; ++c) {
+            if (!group_wait(&bars[B_ODONE + (c & 1)], (c >> 1) & 1, abort_flag, 3, NOUT, ot == 0, false)) {
+                run = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+            const int t0 = tbeg + c * C, L = min(C, tend - t0);
+            __nv_bfloat16* obase = o + ((long long)b * Tn + t0) * tstride + (long long)h * dv + c0;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {       // 32 tokens at a time
-                    uint32_t x[32];
-                    tmem_ld32(tb + lb + x2 + half * 32, x);
-                    tmem_ld_wait();
+            for (int half = 0; half < 2; ++half) {           // 32 tokens from TMEM at a time
+                uint32_t x[32];
+                tmem_ld32(tb + lb + x2 + half * 32, x);
+                tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) st[j * ROWS + ot] = __float2bfloat16_rn(__uint_as_float(x[j]));
-                    if (half == 1) tc_fence_before();
+                for (int sub = 0; sub < 32 / OUT_TOK; ++sub) {
+#pragma unroll
+                    for (int j = 0; j < OUT_TOK; ++j)
+                        st[j * ROWS + ot] = __float2bfloat16_rn(__uint_as_float(x[sub * OUT_TOK + j]));
+                    if (half == 1 && sub == 0) tc_fence_before();
                     named_sync(3, NOUT);
-                    if (half == 1 && ot == 0) arrive(&bars[B_X2FREE + (c & 1)]);
+                    if (half == 1 && sub == 0 && ot == 0) arrive(&bars[B_X2FREE + (c & 1)]);
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const int qd = ot + m * NOUT, r = qd >> 4, ch = qd & 15;
-                        if (half * 32 + r < L)
-                            *reinterpret_cast<uint4*>(obase + (half * 32 + r) * tstride + ch * 8) =
-                                *reinterpret_cast<const uint4*>(st + r * ROWS + ch * 8);
+                    for (int m = 0; m < OUT_TOK / 8; ++m) {  // OUT_TOK rows x 16 chunks of 16 bytes
+                        const int qd = ot + m * NOUT, r = qd >> 4, cq = qd & 15;
+                        const int tok = half * 32 + sub * OUT_TOK + r;
+                        if (tok < L)
+                            *reinterpret_cast<uint4*>(obase + tok * tstride + cq * 8) =
+                                *reinterpret_cast<const uint4*>(st + r * ROWS + cq * 8);
                     }
                     named_sync(3, NOUT);                     // staging free again
                 }
+            }
+        }
+        if (!run) *abort_flag = 1;
+        // CONV: the new history, the last three raw values of the sequence (or of the old history)
+        if (CONV && run && cv.hist_out && !seg.phaseA && p_seg == seg.nseg - 1 && c0 + ot < dv) {
+            const int ch = c0 + ot;
+#pragma unroll
+            for (int k3 = 0; k3 < 3; ++k3) {
+                const int tau = Tn - 3 + k3;
+                __nv_bfloat16 val = __float2bfloat16_rn(0.f);
+                if (tau >= 0) val = cv.v[((long long)b * Tn + tau) * tstride + (long long)h * dv + ch];
+                else if (cv.hist_in) val = cv.hist_in[((long long)b * 3 + 3 + tau) * tstride + (long long)h * dv + ch];
+                cv.hist_out[((long long)b * 3 + k3) * tstride + (long long)h * dv + ch] = val;
             }
         }
     } else if (tid == MMA0 || tid == LOAD0) {
@@ -311,8 +358,9 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         //   MMA  (critical path):  chunk c: P3(c) after AS(c) and P2a(c);
         //                          P4(c) after AW(c) and K(c)
         //   LOAD (everything else): IMG(0) V(0) K(0) IMG(1) V(1) [K(1)] P2a(0);
-        //        chunk c: P5a(c) after AS(c) and X2 free, P5b(c) after AW(c);
-        //        P2a(c+1) after IMG(c+1) and V(c+1); V(c+2) after P2a(c);
+        //        chunk c: V(c+2) (CONV: V(c+1)) after P2a(c); P5a(c) after AS(c)
+        //        and X2 free, P5b(c) after AW(c); P2a(c+1) after IMG(c+1) and V(c+1);
+        //        CONV: the segment's halo with V(0), before P2a(0);
         //        K(c+NKBUF) and IMG(c+2) after P4(c) and P5b(c)
         constexpr int NKBUF = SM::NKBUF;
         const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
@@ -348,17 +396,37 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 tma_load_3d(dst, &tm_v, bar, c0, h, zrow(c));
                 tma_load_3d(dst + 8192, &tm_v, bar, c0 + 64, h, zrow(c));
             };
+            // CONV: the 16 values before a segment's first chunk, into rows 48..63 of
+            // V buffer 1 (where P2a(0) looks for the previous chunk's tail)
+            auto load_h0 = [&]() {
+                uint64_t* bar = &bars[B_H0];
+                uint8_t* dst = sm + SM::V + 16384 + 48 * 128;
+                mbar_expect_tx(bar, 2 * 16 * 128);
+                // sequence start: the history's rows 0..2 at box rows 13..15, else all-zero rows
+                // (coordinates below 0 read as zero; rows of other sequences only meet zero weights)
+                const bool from_hist = tbeg == 0 && cv.hist_in != nullptr;
+                const CUtensorMap* m = from_hist ? &tm_hh : &tm_vh;
+                const int z = from_hist ? b * 3 - 13 : (tbeg == 0 ? -16 : (int)((long long)b * Tn + tbeg - 16));
+                tma_load_3d(dst, m, bar, c0, h, z);
+                tma_load_3d(dst + 8192, m, bar, c0 + 64, h, z);
+            };
             const uint64_t dV = sw128_desc(smem_u32(sm + SM::V), 8192, 1024);
             const uint64_t dAW = sw128_desc(smem_u32(sm + SM::AW), 16, 1024);
+            const uint64_t dImgMN = sw128_desc(smem_u32(sm + SM::IMG), 8192, 1024);   // MH (MN-major)
             constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
             constexpr uint32_t ID_MNK = idesc_bf16(128, 64, true, false);
-            auto mma_p2a = [&](int c) {      // X1[c&1] = V^T T1^T
+            constexpr uint32_t ID_MNMN = idesc_bf16(128, 64, true, true);
+            auto mma_p2a = [&](int c) {      // X1[c&1] = V^T T1^T   (CONV: Vh^T MH + V^T M^T)
                 const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64;
                 const uint64_t dv_ = dV + (uint64_t)(((uint32_t)(c & 1) * 16384) >> 4);
+                if (CONV) {   // the previous chunk's rows 48..63 (buffer (c-1)&1; c = 0: the segment's halo)
+                    const uint64_t dvh = dV + (uint64_t)(((uint32_t)((c + 1) & 1) * 16384 + 48 * 128) >> 4);
+                    mma_bf16_ss(tb + x1, dvh, dImgMN + ioff(c, IM::MH), ID_MNMN, 0);
+                }
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16_ss(tb + x1, dv_ + (uint64_t)(kk * 2048 >> 4), dImg + ioff(c, IM::T1 + kk * 32), ID_MNK,
-                                kk > 0);
+                                CONV || kk > 0);
                 mma_commit(&bars[B_P2 + (c & 1)]);
             };
             auto mma_p5a = [&](int c) {      // X2[c&1] = S Q~^T
@@ -376,11 +444,18 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 mma_commit(&bars[B_ODONE + (c & 1)]);
             };
             int nK = 0, nV = 0, nI = 0, n2 = 0, n5 = 0;      // loads / commit groups issued
+            bool h0 = false;
             if (nch > 0) { load_img(0); ++nI; load_v(0); ++nV; load_k(0); ++nK; }
-            if (nch > 1) { load_img(1); ++nI; load_v(1); ++nV; }
+            if (CONV && nch > 0) { load_h0(); h0 = true; }
+            if (nch > 1) { load_img(1); ++nI; }
+            if (!CONV && nch > 1) { load_v(1); ++nV; }
             if (NKBUF == 2 && nch > 1) { load_k(1); ++nK; }
-            if (nch > 0 && WL(B_IMG, 0) && WL(B_V, 0)) { tc_fence_after(); mma_p2a(0); ++n2; }
+            if (nch > 0 && WL(B_IMG, 0) && WL(B_V, 0) && (!CONV || WL(B_H0, 0))) { tc_fence_after(); mma_p2a(0); ++n2; }
             for (int c = 0; c < nch && ok; ++c) {
+                // the next V tile into the buffer P2a(c) has read (done early in chunk c):
+                // V(c+2), or with CONV V(c+1) (its buffer held V(c-1), the halo of P2a(c))
+                if (CONV && c + 1 < nch && WL(B_P2 + (c & 1), c >> 1)) { load_v(c + 1); ++nV; }
+                if (!CONV && c + 2 < nch && WL(B_P2 + (c & 1), c >> 1)) { load_v(c + 2); ++nV; }
                 if (write_o) {
                     if (WL(B_AS, c) && (c < 2 || WL(B_X2FREE + (c & 1), (c - 2) >> 1))) { tc_fence_after(); mma_p5a(c); }
                     if (WL(B_AW, c)) { tc_fence_after(); mma_p5b(c); ++n5; }
@@ -388,7 +463,6 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 if (c + 1 < nch && WL(B_IMG + ((c + 1) & 1), (c + 1) >> 1) && WL(B_V + ((c + 1) & 1), (c + 1) >> 1)) {
                     tc_fence_after(); mma_p2a(c + 1); ++n2;
                 }
-                if (c + 2 < nch && WL(B_P2 + (c & 1), c >> 1)) { load_v(c + 2); ++nV; }
                 if ((c + NKBUF < nch || c + 2 < nch) && WL(B_SDONE + (c & 1), c >> 1) &&
                     (!write_o || WL(B_ODONE + (c & 1), c >> 1))) {
                     if (c + NKBUF < nch) { load_k(c + NKBUF); ++nK; }
@@ -404,6 +478,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             for (int j = max(0, nI - 2); j < nI; ++j) mbar_wait(&bars[B_IMG + (j & 1)], (j >> 1) & 1);
             for (int j = max(0, n2 - 2); j < n2; ++j) mbar_wait(&bars[B_P2 + (j & 1)], (j >> 1) & 1);
             for (int j = max(0, n5 - 2); j < n5; ++j) mbar_wait(&bars[B_ODONE + (j & 1)], (j >> 1) & 1);
+            if (h0) mbar_wait(&bars[B_H0], 0);
         } else {
             // the critical path: spin first
             auto W = [&](int bar, int phase) {

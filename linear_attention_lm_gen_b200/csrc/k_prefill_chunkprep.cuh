@@ -10,11 +10,14 @@
 // read (so the chain kernel copies them into shared memory unchanged) and a
 // few float vectors:
 //   T1   [64 r][64 i]    T diag(b)                       (U^T = V^T T1^T)
+//                        or, with taps, M: T1 with the dynamic conv folded in
 //   W^T  [dk j][64 r]    (T diag(b gam / |k|) K)^T         (Wt^T = U^T - S W^T)
 //   vec  dik[64] = d_i / |k_i|, then gam_{L-1}
+//   MH   [16 s][64 r]    with taps: the conv's reach into the previous
+//                        chunk's last three raw values (see prep_mconv)
 //   P    [64 r][64 i]    exp(G_r - G_i) q^_r.k^_i (i <= r) (outputs only)
 //   Q~   [64 r][dk]      diag(gam / |q|) Q, 64-column blocks (outputs only)
-// T1, W^T and vec come first, so a pass without outputs copies a prefix.
+// T1, W^T, vec and MH come first, so a pass without outputs copies a prefix.
 //
 // A CTA (256 threads, named barrier 1 = the whole CTA) walks items
 // blockIdx.x, blockIdx.x + gridDim.x, ...; three CTAs share an SM, so three
@@ -42,11 +45,13 @@ struct Img {
     static constexpr uint32_t T1 = 0;
     static constexpr uint32_t WT = 8192;
     static constexpr uint32_t VEC = WT + DK * 128;
-    static constexpr uint32_t A_BYTES = VEC + 1024;     // prefix used without outputs
+    static constexpr uint32_t MH = VEC + 1024;
+    static constexpr uint32_t A_BYTES = MH + 2048;      // prefix used without outputs
     static constexpr uint32_t P = A_BYTES;
     static constexpr uint32_t Q = P + 8192;
     static constexpr uint32_t BYTES = Q + NKB * 8192;
-    static_assert(WT % 1024 == 0 && VEC % 1024 == 0 && P % 1024 == 0 && Q % 1024 == 0, "image alignment");
+    static_assert(WT % 1024 == 0 && VEC % 1024 == 0 && MH % 1024 == 0 && P % 1024 == 0 && Q % 1024 == 0,
+                  "image alignment");
 };
 
 // shared memory of the preparation kernel (bytes from a 1024-aligned base)
@@ -60,18 +65,22 @@ struct PrepSmem {
     static constexpr uint32_t XS = AF + AF_BYTES;
     static constexpr uint32_t VEC = XS + XS_BYTES;                 // 8 x 64 fp32
     static constexpr uint32_t PN = VEC + 2048;
-    static constexpr uint32_t BAR = PN + 1024;
+    static constexpr uint32_t TP = PN + 1024;                      // taps of the chunk's tokens (float4 each)
+    static constexpr uint32_t BAR = TP + 1024;
     static constexpr uint32_t TSLOT = BAR + 64;
     static constexpr uint32_t BYTES = TSLOT + 16 + 1024;           // + alignment slack
     static_assert(PREP_CTAS * (BYTES + 1024) <= 233472, "resident CTAs per SM");
 };
 
-// items = B * H * nct, item = (b * H + h) * nct + c (also the image index)
+// items = B * H * nct, item = (b * H + h) * nct + c (also the image index).
+// taps [B*T][H][4] or null: with taps the T1 slot holds M and MH is written
+// (the chain then reads raw values); halo0: whether the values before token 0
+// are a history (else MH of each sequence's first chunk is zero).
 template <int DK>
 __global__ void __launch_bounds__(PREP_THREADS, PREP_CTAS)
 gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const float* __restrict__ g, const float* __restrict__ beta, uint8_t* __restrict__ img,
-                      int Tn, int H, int nct, int n_items) {
+                      const float* __restrict__ g, const float* __restrict__ beta, const float* __restrict__ taps,
+                      int halo0, uint8_t* __restrict__ img, int Tn, int H, int nct, int n_items) {
     using SM = PrepSmem<DK>;
     using IM = Img<DK>;
     constexpr int NKB = SM::NKB;
@@ -140,6 +149,9 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         uint8_t* out = img + (size_t)item * IM::BYTES;
         const float gb = gb_next;
         gb_next = load_gb(item + gridDim.x);            // in flight during this item
+        float4 tw = make_float4(0.f, 0.f, 0.f, 0.f);    // tap of token tid (conv folding)
+        if (taps && tid < L)
+            tw = *reinterpret_cast<const float4*>(taps + ((long long)(z_of(item) + tid) * H + (item / nct) % H) * 4);
         if (!(ok = __syncthreads_and(mbar_wait(&bars[buf], (uint32_t)(k / PREP_KQBUF) & 1)))) break;
         if (tid == 0) {   // P1: [K; Q] K^T -> XP
             ++ndone[buf];
@@ -154,12 +166,16 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             ++n1;
         }
         prep_vectors<DK>(KQ, V, PN, gb, L, tid, 1);
+        if (tid < 64) reinterpret_cast<float4*>(sm + SM::TP)[tid] = tw;   // read after the UT inverse
         if (!(ok = __syncthreads_and(mbar_wait(&bars[2], (uint32_t)k & 1)))) break;
         tc_fence_after();
         prep_e1(tb + TM_XP, V, AF, out + IM::P, tid);
         named_sync(1, PREP_THREADS);
         ut_inverse(AF, XS, tid, 1);
-        prep_t1t2(AF, V, out + IM::T1, sm + SM::T2, tid);
+        prep_t1t2(AF, V, taps ? nullptr : out + IM::T1, sm + SM::T2, tid);
+        if (taps)
+            prep_mconv(AF, V, reinterpret_cast<const float4*>(sm + SM::TP), out + IM::T1, out + IM::MH,
+                       halo0 || item % nct != 0, tid);
         if (tid < 64) reinterpret_cast<float*>(out + IM::VEC)[tid] = V.dcy[tid] * V.ik[tid];
         else if (tid == 64) reinterpret_cast<float*>(out + IM::VEC)[64] = V.gam[L - 1];
         fence_async_smem();

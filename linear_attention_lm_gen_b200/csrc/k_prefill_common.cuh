@@ -349,7 +349,7 @@ __device__ __forceinline__ void ut_inverse(float* AF, float* XS, int pt, int bid
 }
 
 // T1 = T diag(b) and T2 = T diag(b gam / |k|) as bf16 SW128 tiles (row r = pt >> 2,
-// 16 columns per thread). No barrier inside.
+// 16 columns per thread; T1 skipped when null). No barrier inside.
 __device__ __forceinline__ void prep_t1t2(const float* AF, Vec V, uint8_t* T1, uint8_t* T2, int pt) {
     const int r = pt >> 2, qc = pt & 3;
 #pragma unroll
@@ -373,9 +373,56 @@ __device__ __forceinline__ void prep_t1t2(const float* AF, Vec V, uint8_t* T1, u
             }
         }
         const uint32_t off = sw128_off(r, i0 * 2);
-        *reinterpret_cast<uint4*>(T1 + off) = pack8(f1);
+        if (T1) *reinterpret_cast<uint4*>(T1 + off) = pack8(f1);
         *reinterpret_cast<uint4*>(T2 + off) = pack8(f2);
     }
+}
+
+// T1 with the dynamic causal conv of the chunk's values folded in (Jet-Nemotron
+// paper, section 2.4: v'_i = sum_j w_i[j] v_{i-j}). U = T1 V' is linear in the
+// raw values, U = M V + MH V_prev, where
+//   M[r][s]  = sum_{j=0..3} w_{s+j}[j] T1[r][s+j]        (s = 0..63; T1[r][i] = 0 for i > r)
+//   MH[r][s] = sum_{j=-s..3} w_{s+j}[j] T1[r][s+j]        (s = -3..-1: the previous chunk's last tokens)
+// TP: the chunk's taps w_i (float4 per token, zero past the chunk end).
+// M is stored like T1 (K-major SW128, rows r); MH as the K x N = 16 x 64
+// operand of one more K-step, MN-major SW128 (row 16 + s holds MH[.][s], rows
+// 0..12 zero), all zero when `halo` is false (a sequence start with no
+// history). Row r = pt >> 2, 16 columns per thread. No barrier inside.
+__device__ __forceinline__ void prep_mconv(const float* AF, Vec V, const float4* TP, uint8_t* M, uint8_t* MH,
+                                           bool halo, int pt) {
+    const int r = pt >> 2, qc = pt & 3, i0 = qc * 16;
+    float t1[19];                                        // T1[r][i0 .. i0+18]
+#pragma unroll
+    for (int u = 0; u < 19; ++u) {
+        const int i = i0 + u;
+        t1[u] = (i <= r && i < C) ? AF[r * LDA + i] * V.bet[i] : 0.f;
+    }
+    float m[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) m[u] = 0.f;
+#pragma unroll
+    for (int u = 0; u < 19; ++u) {                       // token i = i0 + u feeds M[r][i - j] through tap j
+        const int i = i0 + u;
+        const float4 w = i < C ? TP[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float wj[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (u - j >= 0 && u - j < 16) m[u - j] = fmaf(wj[j], t1[u], m[u - j]);
+    }
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc)
+        *reinterpret_cast<uint4*>(M + sw128_off(r, (i0 + hc * 8) * 2)) = pack8(m + hc * 8);
+    if (qc == 0) {                                       // MH[r][-3..-1] from T1[r][0..2] and w_0..w_2
+        const float4 w0 = TP[0], w1 = TP[1], w2 = TP[2];
+        const float h1 = halo ? fmaf(w2.w, t1[2], fmaf(w1.z, t1[1], w0.y * t1[0])) : 0.f;   // s = -1
+        const float h2 = halo ? fmaf(w1.w, t1[1], w0.z * t1[0]) : 0.f;                        // s = -2
+        const float h3 = halo ? w0.w * t1[0] : 0.f;                                           // s = -3
+        *reinterpret_cast<__nv_bfloat16*>(MH + sw128_off(13, r * 2)) = __float2bfloat16_rn(h3);
+        *reinterpret_cast<__nv_bfloat16*>(MH + sw128_off(14, r * 2)) = __float2bfloat16_rn(h2);
+        *reinterpret_cast<__nv_bfloat16*>(MH + sw128_off(15, r * 2)) = __float2bfloat16_rn(h1);
+    }
+    if (pt < 13 * 8)                                     // rows 0..12: zero (whole rows, layout-free)
+        *reinterpret_cast<uint4*>(MH + pt * 16) = make_uint4(0u, 0u, 0u, 0u);
 }
 
 // Q~ = diag(gam / |q|) Q in place, Q the second half of each 64-column block

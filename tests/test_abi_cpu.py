@@ -126,8 +126,8 @@ def test_workspace_query_is_host_only(lib):
         assert prefill(lib, B=1, T=4096, H=12, dk=96, dv=256, ws=None, wsb=0) == WORKSPACE
 
 
-@pytest.mark.parametrize("B,T,H,dk,dv,img", [(1, 4096, 12, 96, 256, 46080), (2, 1553, 2, 64, 128, 33792),
-                                             (1, 65536, 16, 128, 256, 50176), (3, 100, 2, 96, 256, 46080)])
+@pytest.mark.parametrize("B,T,H,dk,dv,img", [(1, 4096, 12, 96, 256, 48128), (2, 1553, 2, 64, 128, 35840),
+                                             (1, 65536, 16, 128, 256, 52224), (3, 100, 2, 96, 256, 48128)])
 def test_workspace_sizes(lib, B, T, H, dk, dv, img):
     # fastest plan = one image per (sequence, head, 64-token chunk) + the segment buffers
     lo = jet.jet_gdn_prefill_workspace_min(B, T, H, dk, dv)
@@ -169,3 +169,42 @@ def fused_decode(lib, x=A, w1=A, w2=A, q=A, k=A, v=A, hin=A + (1 << 16), hout=A 
 ])
 def test_fused_decode_rejects(lib, kw, expect):
     assert fused_decode(lib, **kw) == expect
+
+
+def jetblock_prefill(lib, x=A, w1=A, w2=A, q=A, k=A, v=A, hin=None, hout=None, g=A, b=A, S0=None,
+                     o=A + (1 << 24), S_out=A, ws=A, ws_bytes=0, B=1, T=64, D=64, H=2, dk=96, dv=128, hidden=32,
+                     width=4, chunk=64, dt=BF16):
+    return lib.jet_jetblock_prefill(P(x), P(w1), P(w2), P(q), P(k), P(v), P(hin), P(hout), P(g), P(b), P(S0),
+                                    P(o), P(S_out), P(ws), ws_bytes, B, T, D, H, dk, dv, hidden, width, chunk, dt,
+                                    None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(), WORKSPACE),                                   # no workspace: refused before any launch
+    (dict(ws=None), WORKSPACE), (dict(q=None), INVALID), (dict(S_out=None), INVALID),
+    (dict(o=A + 64), INVALID),                             # o may not overlap v
+    (dict(hout=A + 128), INVALID),                         # nor may the new history
+    (dict(hin=A + (1 << 22), hout=A + (1 << 22) + 256), INVALID),
+    (dict(chunk=32), UNSUPPORTED), (dict(width=3), UNSUPPORTED), (dict(dv=48), UNSUPPORTED),
+    (dict(v=A + 8), MISALIGNED), (dict(g=A + 2), MISALIGNED), (dict(hout=A + (1 << 23) + 8), MISALIGNED),
+])
+def test_jetblock_prefill_rejects(lib, kw, expect):
+    assert jetblock_prefill(lib, **kw) == expect
+
+
+@pytest.mark.parametrize("B,T,H,dk,dv", [(1, 4096, 12, 96, 256), (2, 130, 3, 64, 128), (1, 65536, 16, 128, 256)])
+def test_jetblock_prefill_workspace_is_taps_plus_the_fastest_plan(lib, B, T, H, dk, dv):
+    taps = -(-B * T * H * 4 * 4 // 1024) * 1024
+    n = jet.jet_jetblock_prefill_workspace_size(B, T, H, dk, dv)
+    assert n == taps + jet.jet_gdn_prefill_workspace_size(B, T, H, dk, dv)
+    # one byte short is refused before anything runs
+    assert jetblock_prefill(lib, ws_bytes=n - 1, B=B, T=T, H=H, dk=dk, dv=dv, D=64,
+                            o=A + (1 << 40), hin=None) == WORKSPACE
+
+
+def test_jetblock_prefill_workspace_off_the_tensor_core_path():
+    import torch
+    # float32 (and shapes the tensor-core prefill does not take): taps + a v' buffer
+    for (B, T, H, dk, dv, dt, es) in ((1, 64, 2, 16, 32, torch.float32, 4), (2, 100, 3, 48, 64, torch.bfloat16, 2)):
+        up = lambda x: -(-x // 1024) * 1024
+        assert jet.jet_jetblock_prefill_workspace_size(B, T, H, dk, dv, 64, dt) == up(B * T * H * 16) + up(B * T * H * dv * es)

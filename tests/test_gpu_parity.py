@@ -216,16 +216,76 @@ def run_prefill(d, H, hist_out=False):
 
 
 @pytest.mark.parametrize("name", ["tiny_f32", "prefill_2b_t4096"])
-def test_config_prefill_full(orc, name):
+@pytest.mark.parametrize("one_call", [False, True])
+def test_config_prefill_full(orc, name, one_call):
     s = synth.CONFIGS[name]
     inp = synth.prefill_inputs(s, seed=0)
     d = gpu_inputs(inp)
     ref = to_oracle(inp)
-    vc, o, S, _ = run_prefill(d, s.H)
     r = orc.jetblock_prefill(ref["x"], ref["W1"], ref["W2"], ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"])
+    if one_call:     # jet_jetblock_prefill: generator, then the conv inside the prefill
+        o, S = jet.jet_jetblock_prefill(d["x"], d["W1"], d["W2"], d["q"], d["k"], d["v"], d["g"], d["beta"])
+    else:
+        vc, o, S, _ = run_prefill(d, s.H)
+        assert_close(host64(vc), r["v_conv"], s.dtype, f"{name} v'")
     assert_close(host64(o), r["o"], s.dtype, f"{name} o")
     assert_close(host64(S), r["S"], s.dtype, f"{name} S")
-    assert_close(host64(vc), r["v_conv"], s.dtype, f"{name} v'")
+
+
+# ------------------------------------------------------------------ generator + conv inside the prefill
+@pytest.mark.parametrize("dtype,B,T,H,dk,dv,D", [
+    ("f32", 1, 64, 2, 16, 32, 64),            # float32: separate conv pass into the workspace + SIMT prefill
+    ("bf16", 2, 130, 3, 64, 128, 64),
+    ("bf16", 1, 333, 12, 96, 256, 1536),
+    ("bf16", 2, 65, 2, 128, 256, 128),
+    ("bf16", 3, 2, 2, 96, 128, 64),           # shorter than the conv window: the history carries through
+    ("bf16", 2, 1553, 2, 96, 256, 64),        # sequence-parallel segments: conv halos at segment starts
+    ("bf16", 2, 100, 3, 48, 64, 64),          # dk off the tensor-core path
+])
+@pytest.mark.parametrize("hist,s0", [(False, False), (True, True)])
+def test_jetblock_prefill_matches_oracle(orc, dtype, B, T, H, dk, dv, D, hist, s0):
+    s = shape(dtype, B=B, T=T, H=H, dk=dk, dv=dv, D=D)
+    inp = synth.prefill_inputs(s, seed=T + 7, gate_scale=0.01 if T > 1000 else 1.0, s0_std=0.2 if s0 else None)
+    d = gpu_inputs(inp)
+    ref = to_oracle(inp)
+    hin_np = synth.jetblock._draw(np.random.default_rng(6), (B, 3, H, dv), dtype) if hist else None
+    hin = dev(hin_np, dtype) if hist else None
+    hout = torch.full((B, 3, H, dv), float("nan"), device="cuda", dtype=d["v"].dtype)
+    o = nan_like(d["v"])
+    S_out = torch.full((B, H, dv, dk), float("nan"), device="cuda")
+    jet.jet_jetblock_prefill(d["x"], d["W1"], d["W2"], d["q"], d["k"], d["v"], d["g"], d["beta"], hin, hout,
+                             d.get("S0"), o, S_out)
+    r = orc.jetblock_prefill(ref["x"], ref["W1"], ref["W2"], ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"],
+                             inp["S0"].astype(np.float64) if s0 else None,
+                             synth.to_f64(hin_np, dtype) if hist else None)
+    assert_close(host64(o), r["o"], dtype, "o")
+    assert_close(host64(S_out), r["S"], dtype, "S")
+    np.testing.assert_array_equal(host64(hout), r["hist"])       # raw V: bit-exact
+
+
+@pytest.mark.parametrize("B,T,H,dk,dv,D,hist,s0", [
+    (1, 4096, 12, 96, 256, 1536, False, False),   # the 2B prompt shape
+    (2, 1553, 2, 96, 256, 64, True, True),
+    (2, 130, 3, 64, 128, 64, True, False),
+    (1, 777, 2, 128, 256, 128, False, True),
+])
+def test_jetblock_prefill_agrees_with_the_two_calls(B, T, H, dk, dv, D, hist, s0):
+    # the one-call prefill folds the conv into each chunk's UT transform instead of
+    # rounding v' to bf16, so it agrees with the two-call path to bf16 accuracy
+    # (both are checked against the oracle above); the history is a copy: bit-exact
+    s = shape("bf16", B=B, T=T, H=H, dk=dk, dv=dv, D=D)
+    inp = synth.prefill_inputs(s, seed=T, gate_scale=0.05, s0_std=0.2 if s0 else None)
+    d = gpu_inputs(inp)
+    hin = dev(synth.jetblock._draw(np.random.default_rng(8), (B, 3, H, dv), "bf16"), "bf16") if hist else None
+    h1 = torch.full((B, 3, H, dv), float("nan"), device="cuda", dtype=torch.bfloat16)
+    h2 = h1.clone()
+    vc, _ = jet.jet_dyn_conv_v(d["x"], d["W1"], d["W2"], d["v"], hin, None, h1)
+    o1, S1 = jet.jet_gdn_prefill(d["q"], d["k"], vc, d["g"], d["beta"], d.get("S0"))
+    o2, S2 = jet.jet_jetblock_prefill(d["x"], d["W1"], d["W2"], d["q"], d["k"], d["v"], d["g"], d["beta"], hin, h2,
+                                      d.get("S0"))
+    assert torch.equal(h1, h2)
+    assert_close(host64(o2), host64(o1), "bf16", "o")
+    assert_close(host64(S2), host64(S1), "bf16", "S")
 
 
 def sampled_prefill_reference(orc, inp, heads, rows, block=16384):
