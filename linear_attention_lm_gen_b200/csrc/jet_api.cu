@@ -12,6 +12,7 @@
 
 #include "common.cuh"
 #include "k_decode.cuh"
+#include "k_gen.cuh"
 #include "k_genconv.cuh"
 #include "k_prefill_simt.cuh"
 #include "k_prefill_chain.cuh"
@@ -111,6 +112,21 @@ jet_status launch_genconv(const void* x, const void* w1, const void* w2, const v
         return launch_genconv_t<T, TB, 8>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, groups, hpc, s);
     return launch_genconv_t<T, TB, 1>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, groups, hpc, s);
 }
+
+// the generator alone over a prompt (bf16): one CTA per 32 tokens
+jet_status launch_gen(const void* x, const void* w1, const void* w2, float* taps, int B, int Tn, int D, int H,
+                      cudaStream_t s) {
+    const long long N = (long long)B * Tn;
+    const int HW4 = H * GC_W;
+    const size_t smem = kgen::smem_bytes(HW4);
+    if (smem_attr(kgen::gen_kernel, smem) != JET_OK) return JET_ERR_CUDA;
+    kgen::gen_kernel<<<(unsigned)((N + kgen::GT - 1) / kgen::GT), kgen::THREADS, smem, s>>>(
+        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w1, (const __nv_bfloat16*)w2, taps, N, D, HW4);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return launch_status();
+}
+// prompts long enough to fill the GPU with 32-token CTAs take the stand-alone generator
+constexpr long long kGenMinTokens = 1024;
 
 jet_status check_gen(const void* x, const void* w1, const void* w2, int B, int T, int D, int H,
                      int hidden, int width, jet_dtype dt) {
@@ -336,6 +352,7 @@ jet_status jet_kernel_gen(const void* x, const void* w1, const void* w2, float* 
     if (!conv_w) return JET_ERR_INVALID_ARG;
     if (!aligned_to(conv_w, 4)) return JET_ERR_MISALIGNED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == JET_BF16 && (long long)B * T >= kGenMinTokens) return launch_gen(x, w1, w2, conv_w, B, T, D, H, s);
     if (dt == JET_BF16)
         return launch_genconv<__nv_bfloat16>(x, w1, w2, nullptr, nullptr, nullptr, nullptr, conv_w, B, T, D, H, 32, s);
     return launch_genconv<float>(x, w1, w2, nullptr, nullptr, nullptr, nullptr, conv_w, B, T, D, H, 32, s);
@@ -445,7 +462,9 @@ jet_status jet_jetblock_prefill(const void* x, const void* w1, const void* w2, c
     float* taps = static_cast<float*>(workspace);
     uint8_t* rest = static_cast<uint8_t*>(workspace) + ((elems({B, T, H, 4}) * sizeof(float) + 1023) & ~size_t(1023));
     if (tc_prefill_ok(dt, dk, dv, (long long)B * T)) {
-        st = launch_genconv<__nv_bfloat16>(x, w1, w2, nullptr, nullptr, nullptr, nullptr, taps, B, T, D, H, dv, s);
+        st = (long long)B * T >= kGenMinTokens
+                 ? launch_gen(x, w1, w2, taps, B, T, D, H, s)
+                 : launch_genconv<__nv_bfloat16>(x, w1, w2, nullptr, nullptr, nullptr, nullptr, taps, B, T, D, H, dv, s);
         if (st != JET_OK) return st;
         const pfch::ChainConv cv{static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(hist_in),
                                  static_cast<__nv_bfloat16*>(hist_out)};

@@ -65,8 +65,8 @@ struct PrepSmem {
     static constexpr uint32_t XS = AF + AF_BYTES;
     static constexpr uint32_t VEC = XS + XS_BYTES;                 // 8 x 64 fp32
     static constexpr uint32_t PN = VEC + 2048;
-    static constexpr uint32_t TP = PN + 1024;                      // taps of the chunk's tokens (float4 each)
-    static constexpr uint32_t BAR = TP + 1024;
+    static constexpr uint32_t TP = PN + 1024;                      // [2] taps of a chunk's tokens (see tp_slot)
+    static constexpr uint32_t BAR = TP + 2 * TP_BYTES;
     static constexpr uint32_t TSLOT = BAR + 64;
     static constexpr uint32_t BYTES = TSLOT + 16 + 1024;           // + alignment slack
     static_assert(PREP_CTAS * (BYTES + 1024) <= 233472, "resident CTAs per SM");
@@ -139,8 +139,20 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const long long off = ((long long)z_of(item) + (tid & 63)) * H + h;
         return tid < 64 ? g[off] : beta[off];
     };
+    // taps of an item's tokens into TP[buf] (threads < 64; cp.async, zero past the sequence end)
+    auto load_taps = [&](int item, int buf) {
+        if (!taps || item >= n_items || tid >= 64) return;
+        const int c = item % nct, h = (item / nct) % H;
+        const bool in = tid < min(C, Tn - c * C);
+        const float* src = taps + (in ? ((long long)(z_of(item) + tid) * H + h) * 4 : 0);
+        const uint32_t dst = smem_u32(sm + SM::TP) + (uint32_t)buf * TP_BYTES + (uint32_t)tp_slot(tid) * 16u;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(in ? 16u : 0u)
+                     : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
     bool ok = true;
     int k = 0;
+    load_taps(blockIdx.x, 0);
     float gb_next = load_gb(blockIdx.x);
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
         const int buf = k % PREP_KQBUF;
@@ -149,9 +161,6 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         uint8_t* out = img + (size_t)item * IM::BYTES;
         const float gb = gb_next;
         gb_next = load_gb(item + gridDim.x);            // in flight during this item
-        float4 tw = make_float4(0.f, 0.f, 0.f, 0.f);    // tap of token tid (conv folding)
-        if (taps && tid < L)
-            tw = *reinterpret_cast<const float4*>(taps + ((long long)(z_of(item) + tid) * H + (item / nct) % H) * 4);
         if (!(ok = __syncthreads_and(mbar_wait(&bars[buf], (uint32_t)(k / PREP_KQBUF) & 1)))) break;
         if (tid == 0) {   // P1: [K; Q] K^T -> XP
             ++ndone[buf];
@@ -166,16 +175,18 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             ++n1;
         }
         prep_vectors<DK>(KQ, V, PN, gb, L, tid, 1);
-        if (tid < 64) reinterpret_cast<float4*>(sm + SM::TP)[tid] = tw;   // read after the UT inverse
+        if (taps && tid < 64) asm volatile("cp.async.wait_group 0;" ::: "memory");   // this item's taps (read later)
         if (!(ok = __syncthreads_and(mbar_wait(&bars[2], (uint32_t)k & 1)))) break;
         tc_fence_after();
         prep_e1(tb + TM_XP, V, AF, out + IM::P, tid);
         named_sync(1, PREP_THREADS);
         ut_inverse(AF, XS, tid, 1);
-        prep_t1t2(AF, V, taps ? nullptr : out + IM::T1, sm + SM::T2, tid);
         if (taps)
-            prep_mconv(AF, V, reinterpret_cast<const float4*>(sm + SM::TP), out + IM::T1, out + IM::MH,
-                       halo0 || item % nct != 0, tid);
+            prep_t1t2_conv(AF, V, reinterpret_cast<const float4*>(sm + SM::TP + (k & 1) * TP_BYTES), out + IM::T1,
+                           out + IM::MH, sm + SM::T2, halo0 || item % nct != 0, tid);
+        else
+            prep_t1t2(AF, V, out + IM::T1, sm + SM::T2, tid);
+        load_taps(item + gridDim.x, (k + 1) & 1);      // the next item's taps, in flight from here
         if (tid < 64) reinterpret_cast<float*>(out + IM::VEC)[tid] = V.dcy[tid] * V.ik[tid];
         else if (tid == 64) reinterpret_cast<float*>(out + IM::VEC)[64] = V.gam[L - 1];
         fence_async_smem();

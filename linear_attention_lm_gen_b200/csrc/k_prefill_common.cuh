@@ -378,24 +378,54 @@ __device__ __forceinline__ void prep_t1t2(const float* AF, Vec V, uint8_t* T1, u
     }
 }
 
-// T1 with the dynamic causal conv of the chunk's values folded in (Jet-Nemotron
-// paper, section 2.4: v'_i = sum_j w_i[j] v_{i-j}). U = T1 V' is linear in the
-// raw values, U = M V + MH V_prev, where
+// float4 slot of token i's taps in a shared-memory taps array: one slot of
+// padding after every 16 tokens, so the four 16-token column groups of
+// prep_t1t2_conv read distinct banks
+__host__ __device__ constexpr int tp_slot(int i) { return i + (i >> 4); }
+constexpr uint32_t TP_BYTES = 68 * 16;
+
+// prep_t1t2 with the dynamic causal conv of the chunk's values folded into T1
+// (Jet-Nemotron paper, section 2.4: v'_i = sum_j w_i[j] v_{i-j}). U = T1 V' is
+// linear in the raw values, U = M V + MH V_prev, where
 //   M[r][s]  = sum_{j=0..3} w_{s+j}[j] T1[r][s+j]        (s = 0..63; T1[r][i] = 0 for i > r)
 //   MH[r][s] = sum_{j=-s..3} w_{s+j}[j] T1[r][s+j]        (s = -3..-1: the previous chunk's last tokens)
-// TP: the chunk's taps w_i (float4 per token, zero past the chunk end).
-// M is stored like T1 (K-major SW128, rows r); MH as the K x N = 16 x 64
-// operand of one more K-step, MN-major SW128 (row 16 + s holds MH[.][s], rows
-// 0..12 zero), all zero when `halo` is false (a sequence start with no
-// history). Row r = pt >> 2, 16 columns per thread. No barrier inside.
-__device__ __forceinline__ void prep_mconv(const float* AF, Vec V, const float4* TP, uint8_t* M, uint8_t* MH,
-                                           bool halo, int pt) {
+// TP: the chunk's taps w_i (float4 at tp_slot(i), zero past the chunk end).
+// M is stored where T1 would be (K-major SW128, rows r); MH as the K x N =
+// 16 x 64 operand of one more K-step, MN-major SW128 (row 16 + s holds
+// MH[.][s], rows 0..12 zero), all zero when `halo` is false (a sequence
+// start with no history). T2 as in prep_t1t2. Row r = pt >> 2, 16 columns
+// per thread; the three T1 values past them come from the next lane (same
+// row). No barrier inside.
+__device__ __forceinline__ void prep_t1t2_conv(const float* AF, Vec V, const float4* TP, uint8_t* M, uint8_t* MH,
+                                               uint8_t* T2, bool halo, int pt) {
     const int r = pt >> 2, qc = pt & 3, i0 = qc * 16;
     float t1[19];                                        // T1[r][i0 .. i0+18]
 #pragma unroll
-    for (int u = 0; u < 19; ++u) {
-        const int i = i0 + u;
-        t1[u] = (i <= r && i < C) ? AF[r * LDA + i] * V.bet[i] : 0.f;
+    for (int hc = 0; hc < 2; ++hc) {
+        const int j0 = i0 + hc * 8;
+        float f2[8];
+#pragma unroll
+        for (int h4 = 0; h4 < 2; ++h4) {
+            const float4 tv = *reinterpret_cast<const float4*>(AF + r * LDA + j0 + h4 * 4);
+            const float4 bv = *reinterpret_cast<const float4*>(V.bet + j0 + h4 * 4);
+            const float4 gv = *reinterpret_cast<const float4*>(V.gam + j0 + h4 * 4);
+            const float4 kv = *reinterpret_cast<const float4*>(V.ik + j0 + h4 * 4);
+            const float t_[4] = {tv.x, tv.y, tv.z, tv.w}, b_[4] = {bv.x, bv.y, bv.z, bv.w};
+            const float g_[4] = {gv.x, gv.y, gv.z, gv.w}, k_[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = j0 + h4 * 4 + e;
+                const float t1v = i <= r ? t_[e] * b_[e] : 0.f;
+                t1[hc * 8 + h4 * 4 + e] = t1v;
+                f2[h4 * 4 + e] = t1v * g_[e] * k_[e];
+            }
+        }
+        *reinterpret_cast<uint4*>(T2 + sw128_off(r, j0 * 2)) = pack8(f2);
+    }
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {
+        const float nx = __shfl_down_sync(0xffffffffu, t1[u], 1);   // T1[r][i0 + 16 + u] (lane + 1: qc + 1)
+        t1[16 + u] = qc < 3 ? nx : 0.f;
     }
     float m[16];
 #pragma unroll
@@ -403,7 +433,7 @@ __device__ __forceinline__ void prep_mconv(const float* AF, Vec V, const float4*
 #pragma unroll
     for (int u = 0; u < 19; ++u) {                       // token i = i0 + u feeds M[r][i - j] through tap j
         const int i = i0 + u;
-        const float4 w = i < C ? TP[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 w = i < C ? TP[tp_slot(i)] : make_float4(0.f, 0.f, 0.f, 0.f);
         const float wj[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j)
@@ -413,7 +443,7 @@ __device__ __forceinline__ void prep_mconv(const float* AF, Vec V, const float4*
     for (int hc = 0; hc < 2; ++hc)
         *reinterpret_cast<uint4*>(M + sw128_off(r, (i0 + hc * 8) * 2)) = pack8(m + hc * 8);
     if (qc == 0) {                                       // MH[r][-3..-1] from T1[r][0..2] and w_0..w_2
-        const float4 w0 = TP[0], w1 = TP[1], w2 = TP[2];
+        const float4 w0 = TP[tp_slot(0)], w1 = TP[tp_slot(1)], w2 = TP[tp_slot(2)];
         const float h1 = halo ? fmaf(w2.w, t1[2], fmaf(w1.z, t1[1], w0.y * t1[0])) : 0.f;   // s = -1
         const float h2 = halo ? fmaf(w1.w, t1[1], w0.z * t1[0]) : 0.f;                        // s = -2
         const float h3 = halo ? w0.w * t1[0] : 0.f;                                           // s = -3

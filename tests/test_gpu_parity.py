@@ -111,6 +111,19 @@ def test_generator_and_conv_stage(orc, dtype, B, T, H, dv, D, hist):
     assert torch.equal(cw2, cw)
 
 
+@pytest.mark.parametrize("B,T,H,D", [(1, 4096, 12, 1536), (2, 1553, 16, 2048), (1, 1024, 3, 80)])
+def test_generator_long_prompt(orc, B, T, H, D):
+    # prompts of 1024+ tokens take the stand-alone generator (32 tokens per CTA, D in
+    # 128-column slices: D = 80 is one partial slice, 2 x 1553 tokens end mid-CTA)
+    s = shape("bf16", B=B, T=T, H=H, dv=32, D=D)
+    inp = synth.prefill_inputs(s, seed=4)
+    d = gpu_inputs(inp)
+    ref = to_oracle(inp)
+    cw = jet.jet_kernel_gen(d["x"], d["W1"], d["W2"], H, torch.full((B, T, H, 4), float("nan"), device="cuda"))
+    w = orc.kernel_gen(ref["x"], ref["W1"], ref["W2"], H)
+    assert_close(host64(cw), w, "bf16", "taps", tol=dict(rel_l2=1e-5, max_abs=1e-4))
+
+
 def test_identity_taps_via_conv_stage(orc):
     # W2 = 0 gives zero taps: v' = 0 whatever V is (no hidden bias or tap offset)
     s = shape("bf16", T=70, H=2, dv=64, D=128)
