@@ -23,7 +23,7 @@ constexpr int THREADS = 256;
 constexpr int GT = 32;                  // tokens per CTA
 constexpr int HID = 32;                 // generator hidden width
 constexpr int KC = 128;                 // columns of D per slice
-constexpr int NST = 6;                  // slice buffers (NST - 1 in flight)
+constexpr int NST = 10;                 // slice buffers (NST - 1 in flight)
 constexpr int XLD = KC * 2 + 16;        // x slice row stride in bytes (16-byte pad: conflict-free ldmatrix)
 constexpr int WLD = HID * 2 + 16;       // W1 slice row stride in bytes
 constexpr int XS_BYTES = GT * XLD;      // 8704
