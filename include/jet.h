@@ -207,6 +207,34 @@ jet_status jet_jetblock_decode_step(const void* x, const void* w1, const void* w
                                     int hidden, int width, jet_dtype dt, void* stream);
 
 /*
+ * jet_jetblock_decode_step over a state cache: the states and conv histories
+ * of the running sequences live in caller-owned pools, and entry b of the
+ * batch works on pool entry slots[b] in place, so a serving loop never
+ * gathers or scatters a state (each is read and written once per step).
+ * Two launches: the generator + conv of the new tokens (histories updated in
+ * place in hist_pool), then the decode update of S_pool.
+ *   x [B,D]; w1, w2 as in jet_kernel_gen; q, k [B,H,dk]; v [B,H,dv] raw;
+ *   g, beta [B,H] float32;
+ *   hist_pool [n_slots,3,H,dv] (raw histories, oldest first) in/out;
+ *   S_pool [n_slots,H,dv,dk] float32 in/out;
+ *   slots [B] int32 (device memory) with distinct values in [0, n_slots); a
+ *     value outside that range leaves that sequence's outputs and pool
+ *     entries untouched and sets the device error word (JET_ERR_DEVICE from
+ *     jet_device_error); repeated values race;
+ *   o [B,H,dv] out; v_conv [B,H,dv] scratch (the conv output, must not
+ *   overlap v); taps [B,H,width] float32 out or NULL.
+ * Same arithmetic as jet_dyn_conv_v (T = 1) followed by jet_gdn_decode_step
+ * on pool entries gathered into a batch: the results are equal bit for bit.
+ */
+jet_status jet_jetblock_decode_slots(const void* x, const void* w1, const void* w2,
+                                     const void* q, const void* k, const void* v,
+                                     const float* g, const float* beta,
+                                     void* hist_pool, float* S_pool, const int* slots, int n_slots,
+                                     void* o, void* v_conv, float* taps,
+                                     int B, int D, int H, int dk, int dv, int hidden, int width,
+                                     jet_dtype dt, void* stream);
+
+/*
  * jet_gdn_prefill for callers that cannot allocate device memory. It has no
  * counterpart in the paper; it exists for code that must not call an
  * allocator on its hot path: work recorded into a CUDA graph (allocation is

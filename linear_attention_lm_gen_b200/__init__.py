@@ -9,7 +9,7 @@ Function names match the C entry points:
   jet_kernel_gen, jet_dyn_conv_v, jet_gdn_prefill_workspace_size,
   jet_gdn_prefill_workspace_min, jet_gdn_prefill, jet_gdn_prefill_noalloc, jet_gdn_decode_step,
   jet_jetblock_decode_step, jet_conv_gdn_decode_step, jet_jetblock_prefill_workspace_size,
-  jet_jetblock_prefill,
+  jet_jetblock_prefill, jet_jetblock_decode_slots,
   jet_device_error, jet_status_string, jet_launch_count.
 """
 from __future__ import annotations
@@ -29,7 +29,8 @@ STATUS = {0: "JET_OK", 1: "JET_ERR_INVALID_ARG", 2: "JET_ERR_UNSUPPORTED", 3: "J
 EXPORTS = ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill_workspace_size", "jet_gdn_prefill_workspace_min",
            "jet_gdn_prefill",
            "jet_gdn_prefill_noalloc", "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step",
-           "jet_jetblock_prefill_workspace_size", "jet_jetblock_prefill", "jet_device_error",
+           "jet_jetblock_prefill_workspace_size", "jet_jetblock_prefill", "jet_jetblock_decode_slots",
+           "jet_device_error",
            "jet_status_string", "jet_launch_count")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -66,6 +67,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.jet_jetblock_prefill_workspace_size.argtypes = [I] * 7
     L.jet_jetblock_prefill_workspace_size.restype = Z
     L.jet_jetblock_prefill.argtypes = [P] * 14 + [Z] + [I] * 10 + [P]
+    L.jet_jetblock_decode_slots.argtypes = [P] * 11 + [I] + [P] * 3 + [I] * 8 + [P]
     L.jet_device_error.argtypes = [P]
     L.jet_status_string.argtypes = [I]
     L.jet_status_string.restype = ctypes.c_char_p
@@ -73,7 +75,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.jet_launch_count.restype = U
     for f in ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill", "jet_gdn_prefill_noalloc",
               "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step", "jet_jetblock_prefill",
-              "jet_device_error"):
+              "jet_jetblock_decode_slots", "jet_device_error"):
         getattr(L, f).restype = I
     _lib = L
     return L
@@ -283,6 +285,35 @@ def jet_jetblock_decode_step(x, W1, W2, q, k, v, hist_in, hist_out, g, beta, S, 
         B, D, H, dk, dv, hidden, width, dt, _stream(stream))
     _check("jet_jetblock_decode_step", st)
     return o, taps
+
+
+def jet_jetblock_decode_slots(x, W1, W2, q, k, v, g, beta, hist_pool, S_pool, slots, o=None, v_conv=None, taps=None,
+                              *, stream=None):
+    """One decode step for B sequences whose states and histories are pool
+    entries: x [B,D], q,k [B,H,dk], v [B,H,dv] raw, g,beta [B,H] float32,
+    hist_pool [N,3,H,dv] and S_pool [N,H,dv,dk] float32 updated in place at
+    entries slots [B] (int32, distinct). Returns o [B,H,dv]."""
+    L = load_library()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    D = x.shape[-1]
+    hidden, HW = W2.shape
+    width = HW // H
+    N = S_pool.shape[0]
+    if o is None:
+        o = torch.empty((B, H, dv), device=q.device, dtype=q.dtype)
+    if v_conv is None:
+        v_conv = torch.empty((B, H, dv), device=q.device, dtype=q.dtype)
+    st = L.jet_jetblock_decode_slots(
+        _ptr(x, "x", q.dtype, (B, D)), _ptr(W1, "W1", q.dtype, (D, hidden)), _ptr(W2, "W2", q.dtype, (hidden, HW)),
+        _ptr(q, "q"), _ptr(k, "k", q.dtype, q.shape), _ptr(v, "v", q.dtype, (B, H, dv)),
+        _ptr(g, "g", torch.float32, (B, H)), _ptr(beta, "beta", torch.float32, (B, H)),
+        _ptr(hist_pool, "hist_pool", q.dtype, (N, 3, H, dv)), _ptr(S_pool, "S_pool", torch.float32, (N, H, dv, dk)),
+        _ptr(slots, "slots", torch.int32, (B,)), N, _ptr(o, "o", q.dtype, (B, H, dv)),
+        _ptr(v_conv, "v_conv", q.dtype, (B, H, dv)), _ptr(taps, "taps", torch.float32, (B, H, width)),
+        B, D, H, dk, dv, hidden, width, _dt(q), _stream(stream))
+    _check("jet_jetblock_decode_slots", st)
+    return o
 
 
 def jet_conv_gdn_decode_step(q, k, v, hist_in, hist_out, taps, g, beta, S, o=None, *, stream=None):

@@ -71,7 +71,7 @@ bool dtype_ok(jet_dtype dt) { return dt == JET_F32 || dt == JET_BF16; }
 template <typename T, int TB, int RUN>
 jet_status launch_genconv_t(const void* x, const void* w1, const void* w2, const void* v, const void* hin,
                             void* vout, void* hout, float* cw, int B, int Tn, int D, int H, int dv, int groups,
-                            int hpc, cudaStream_t s) {
+                            int hpc, cudaStream_t s, const int* slots, int n_slots) {
     const long long N = (long long)B * Tn;
     const size_t smem = sizeof(float) * gc_smem_floats(TB, hpc * GC_W);
     auto kern = genconv_kernel<T, TB, RUN>;
@@ -90,7 +90,8 @@ jet_status launch_genconv_t(const void* x, const void* w1, const void* w2, const
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, (const T*)x, (const T*)w1, (const T*)w2, (const T*)v,
-                                             (const T*)hin, (T*)vout, (T*)hout, cw, B, Tn, D, H, dv, hpc);
+                                             (const T*)hin, (T*)vout, (T*)hout, cw, B, Tn, D, H, dv, hpc, slots,
+                                             n_slots);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     if (e != cudaSuccess) return JET_ERR_CUDA;
     return launch_status();
@@ -99,7 +100,7 @@ jet_status launch_genconv_t(const void* x, const void* w1, const void* w2, const
 template <typename T>
 jet_status launch_genconv(const void* x, const void* w1, const void* w2, const void* v, const void* hin,
                           void* vout, void* hout, float* cw, int B, int Tn, int D, int H, int dv,
-                          cudaStream_t s) {
+                          cudaStream_t s, const int* slots = nullptr, int n_slots = 0) {
     constexpr int TB = 16;
     const long long nblk = ((long long)B * Tn + TB - 1) / TB;
     // head groups (= cluster size, at most 8): enough CTAs to cover the SMs
@@ -109,8 +110,10 @@ jet_status launch_genconv(const void* x, const void* w1, const void* w2, const v
     const int hpc = (H + groups - 1) / groups;
     groups = (H + hpc - 1) / hpc;
     if (Tn >= 8)
-        return launch_genconv_t<T, TB, 8>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, groups, hpc, s);
-    return launch_genconv_t<T, TB, 1>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, groups, hpc, s);
+        return launch_genconv_t<T, TB, 8>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, groups, hpc, s,
+                                          nullptr, 0);
+    return launch_genconv_t<T, TB, 1>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, groups, hpc, s, slots,
+                                      n_slots);
 }
 
 // the generator alone over a prompt (bf16): one CTA per 32 tokens
@@ -315,14 +318,15 @@ jet_status dispatch_prefill(int dk, const void* q, const void* k, const void* v,
 // ---------------------------------------------------------------- K3
 template <typename T, int NV>
 jet_status launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                         float* S, void* o, int B, int H, int dv, const DecConv* conv, cudaStream_t s) {
+                         float* S, void* o, int B, int H, int dv, const DecConv* conv, cudaStream_t s,
+                         const int* slots, int n_slots) {
     dim3 grid((dv + DEC_ROWS - 1) / DEC_ROWS, H, B);
     if (conv)
         gdn_decode_kernel<T, NV, true><<<grid, DEC_THREADS, 0, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta,
-                                                                    S, (T*)o, H, dv, *conv);
+                                                                    S, (T*)o, H, dv, *conv, slots, n_slots);
     else
         gdn_decode_kernel<T, NV><<<grid, DEC_THREADS, 0, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta, S,
-                                                            (T*)o, H, dv);
+                                                            (T*)o, H, dv, DecConv{}, slots, n_slots);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return launch_status();
 }
@@ -330,9 +334,9 @@ jet_status launch_decode(const void* q, const void* k, const void* v, const floa
 template <typename T>
 jet_status dispatch_decode(int dk, const void* q, const void* k, const void* v, const float* g,
                            const float* beta, float* S, void* o, int B, int H, int dv, cudaStream_t s,
-                           const DecConv* conv = nullptr) {
+                           const DecConv* conv = nullptr, const int* slots = nullptr, int n_slots = 0) {
     switch (dk / 16) {
-#define JET_CASE(NV) case NV: return launch_decode<T, NV>(q, k, v, g, beta, S, o, B, H, dv, conv, s);
+#define JET_CASE(NV) case NV: return launch_decode<T, NV>(q, k, v, g, beta, S, o, B, H, dv, conv, s, slots, n_slots);
         JET_CASE(1) JET_CASE(2) JET_CASE(3) JET_CASE(4) JET_CASE(5) JET_CASE(6) JET_CASE(7) JET_CASE(8)
 #undef JET_CASE
         default: return JET_ERR_UNSUPPORTED;
@@ -541,6 +545,39 @@ jet_status jet_jetblock_decode_step(const void* x, const void* w1, const void* w
     st = jet_kernel_gen(x, w1, w2, taps, B, 1, D, H, hidden, width, dt, stream);
     if (st != JET_OK) return st;
     return jet_conv_gdn_decode_step(q, k, v, hist_in, hist_out, taps, g, beta, S, o, B, H, dk, dv, dt, stream);
+}
+
+jet_status jet_jetblock_decode_slots(const void* x, const void* w1, const void* w2, const void* q, const void* k,
+                                     const void* v, const float* g, const float* beta, void* hist_pool,
+                                     float* S_pool, const int* slots, int n_slots, void* o, void* v_conv,
+                                     float* taps, int B, int D, int H, int dk, int dv, int hidden, int width,
+                                     jet_dtype dt, void* stream) {
+    jet_status st = check_gen(x, w1, w2, B, 1, D, H, hidden, width, dt);
+    if (st != JET_OK) return st;
+    if (!q || !k || !v || !g || !beta || !hist_pool || !S_pool || !slots || !o || !v_conv) return JET_ERR_INVALID_ARG;
+    if (n_slots <= 0 || B > n_slots) return JET_ERR_INVALID_ARG;
+    const long long nv = elems({B, H, dv});
+    if (nv < 0 || elems({n_slots, H, dv, dk}) < 0 || elems({n_slots, 3, H, dv}) < 0) return JET_ERR_INVALID_ARG;
+    if (!shape_ok(dk, dv) || B > 65535 || H > 65535) return JET_ERR_UNSUPPORTED;
+    const size_t es = esize(dt);
+    for (const void* p : {q, k, (const void*)o})
+        if (!aligned_to(p, es)) return JET_ERR_MISALIGNED;
+    for (const void* p : {v, (const void*)v_conv, (const void*)hist_pool, (const void*)S_pool})
+        if (!aligned16(p)) return JET_ERR_MISALIGNED;
+    if (!aligned_to(g, 4) || !aligned_to(beta, 4) || !aligned_to(slots, 4) || (taps && !aligned_to(taps, 4)))
+        return JET_ERR_MISALIGNED;
+    if (overlap(v, (size_t)nv * es, v_conv, (size_t)nv * es)) return JET_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // generator + conv of the new tokens with the histories of their slots (updated in place)
+    st = dt == JET_BF16 ? launch_genconv<__nv_bfloat16>(x, w1, w2, v, hist_pool, v_conv, hist_pool, taps, B, 1, D, H,
+                                                       dv, s, slots, n_slots)
+                        : launch_genconv<float>(x, w1, w2, v, hist_pool, v_conv, hist_pool, taps, B, 1, D, H, dv, s,
+                                                slots, n_slots);
+    if (st != JET_OK) return st;
+    if (dt == JET_BF16)
+        return dispatch_decode<__nv_bfloat16>(dk, q, k, v_conv, g, beta, S_pool, o, B, H, dv, s, nullptr, slots,
+                                              n_slots);
+    return dispatch_decode<float>(dk, q, k, v_conv, g, beta, S_pool, o, B, H, dv, s, nullptr, slots, n_slots);
 }
 
 jet_status jet_device_error(void* stream) {

@@ -16,6 +16,11 @@
 // rounded to the storage precision as the separate conv kernel stores it,
 // and it writes the shifted history (v_{t-2}, v_{t-1}, v_t) for the next step.
 //
+// With `slots` (a state cache), sequence b's state and history are entry
+// slots[b] of the pools S [n_slots][H][dv][dk] and hist [n_slots][3][H][dv];
+// an index outside [0, n_slots) sets the device error word and the CTA
+// touches nothing.
+//
 // Mapping: 4 lanes per row, each lane holding dk/16 float4 of the row in an
 // interleaved pattern (lane p reads float4 p, p+4, ...): every load
 // instruction of a warp covers 8 rows x 64 contiguous bytes. A thread owns
@@ -43,14 +48,24 @@ template <typename T, int NV, bool CONV = false>   // NV = dk / 16 float4 per la
 __global__ void __launch_bounds__(DEC_THREADS, NV <= 6 ? 3 : 2)   // 3 CTAs per SM where the registers allow
 gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const float* __restrict__ g, const float* __restrict__ beta,
-                  float* __restrict__ S, T* __restrict__ o, int H, int dv, DecConv cv = {}) {
+                  float* __restrict__ S, T* __restrict__ o, int H, int dv, DecConv cv = {},
+                  const int* __restrict__ slots = nullptr, int n_slots = 0) {
     constexpr int DK = NV * 16;
     __shared__ __align__(16) float sk[DK];
     __shared__ __align__(16) float sq[DK];
     __shared__ float red[3];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.y, b = blockIdx.z;
-    const long long bh = (long long)b * H + h;
+    const long long bh = (long long)b * H + h;                // token inputs and outputs
+    int sb = b;                                               // state / history entry
+    if (slots) {
+        sb = slots[b];
+        if (sb < 0 || sb >= n_slots) {                        // whole CTA, before any access
+            if (tid == 0) flag_error(DEVERR_DATA);
+            return;
+        }
+    }
+    const long long sbh = (long long)sb * H + h;
     const int part = lane & 3;
     const int row0 = blockIdx.x * DEC_ROWS + warp * 8 + (lane >> 2);
     const int row1 = row0 + 64;
@@ -59,8 +74,8 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     // state rows first: the loads overlap the prologue below
     float4 s0[NV], s1[NV];
     {
-        const float4* r0 = reinterpret_cast<const float4*>(S + (bh * dv + (ok0 ? row0 : 0)) * DK);
-        const float4* r1 = reinterpret_cast<const float4*>(S + (bh * dv + (ok1 ? row1 : 0)) * DK);
+        const float4* r0 = reinterpret_cast<const float4*>(S + (sbh * dv + (ok0 ? row0 : 0)) * DK);
+        const float4* r1 = reinterpret_cast<const float4*>(S + (sbh * dv + (ok1 ? row1 : 0)) * DK);
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
             s0[i] = ok0 ? ld_stream_f4(r0 + part + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -72,7 +87,7 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     // conv inputs: the raw history of both rows (v_{t-3}, v_{t-2}, v_{t-1}), loaded
     // now and used only after the prologue below, so their latency overlaps it
     float hv0[3] = {0.f, 0.f, 0.f}, hv1[3] = {0.f, 0.f, 0.f};
-    const long long hb = (long long)b * 3 * H * dv + (long long)h * dv;   // history of (b, h), slot 0
+    const long long hb = (long long)sb * 3 * H * dv + (long long)h * dv;  // history of (b, h), position 0
     const long long hs = (long long)H * dv;                               // slot stride
     float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
     if constexpr (CONV) {
@@ -143,7 +158,7 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     const float c1 = bt * vi1 - a * bt * u1;
     const float ck0 = c0 * inv_k, ck1 = c1 * inv_k;   // c k^ = (c / |k|) k
     if (ok0) {
-        float4* w = reinterpret_cast<float4*>(S + (bh * dv + row0) * DK);
+        float4* w = reinterpret_cast<float4*>(S + (sbh * dv + row0) * DK);
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
             const float4 kf = k4[part + 4 * i];
@@ -153,7 +168,7 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         if (part == 0) Elem<T>::st(o + bh * dv + row0, a * p0 + c0 * kq);
     }
     if (ok1) {
-        float4* w = reinterpret_cast<float4*>(S + (bh * dv + row1) * DK);
+        float4* w = reinterpret_cast<float4*>(S + (sbh * dv + row1) * DK);
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
             const float4 kf = k4[part + 4 * i];

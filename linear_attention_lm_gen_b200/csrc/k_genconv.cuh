@@ -136,12 +136,17 @@ __device__ __forceinline__ void gen_stageA_bf16(const __nv_bfloat16* __restrict_
 // sequence) still spread over many SMs.
 // RUN = tokens per conv work item (8 keeps a sliding window in registers;
 // 1 makes every token an independent item with its 4 loads in flight).
+// slots (T = 1 only): sequence b's history is entry slots[b] of hist_in /
+// hist_out, which may then be the same pool: each history element is read
+// and rewritten by the one thread that owns its item. An index outside
+// [0, n_slots) sets the device error word and the item is skipped.
 template <typename T, int TB, int RUN>
 __global__ void __launch_bounds__(GC_THREADS, 2)
 genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __restrict__ W2,
-               const T* __restrict__ v, const T* __restrict__ hist_in, T* __restrict__ v_out,
-               T* __restrict__ hist_out, float* __restrict__ conv_w_out,
-               int Bn, int Tn, int D, int H, int dv, int hpc) {
+               const T* __restrict__ v, const T* hist_in, T* __restrict__ v_out,
+               T* hist_out, float* __restrict__ conv_w_out,
+               int Bn, int Tn, int D, int H, int dv, int hpc, const int* __restrict__ slots = nullptr,
+               int n_slots = 0) {
     extern __shared__ float smem[];
     const int HW4 = H * GC_W;
     const int h0 = blockIdx.y * hpc;
@@ -175,7 +180,7 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
     const int cols = nh * ngrp;
     const int items = v ? cols * nruns : 0;
     const long long rowstride = (long long)H * dv;   // elements per token
-    struct ItemGeo { long long rr0, coff; int hl, ta, tb, bseq, tpos0; };
+    struct ItemGeo { long long rr0, coff; int hl, ta, tb, bseq, tpos0, hseq; };
     auto item_load = [&](int it, uint4* wraw, uint4* cur, ItemGeo& gi) {
         const int col = it % cols;
         const int run = it / cols;
@@ -187,14 +192,23 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
         gi.rr0 = r0 + gi.ta;
         gi.bseq = (int)(gi.rr0 / Tn);               // one division per item; then stepped
         gi.tpos0 = (int)(gi.rr0 - (long long)gi.bseq * Tn);
+        gi.hseq = gi.bseq;                          // history entry of the sequence
+        if (slots) {
+            gi.hseq = slots[gi.bseq];
+            if (gi.hseq < 0 || gi.hseq >= n_slots) {
+                flag_error(DEVERR_DATA);
+                gi.tb = gi.ta;                      // nothing to do
+                gi.hseq = -1;
+            }
+        }
         // window: wraw[0] = v_{t-1}, wraw[1] = v_{t-2}, wraw[2] = v_{t-3}
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
             const int tau = gi.tpos0 - 1 - j;
             wraw[j] = make_uint4(0, 0, 0, 0);
             if (tau >= 0) wraw[j] = *reinterpret_cast<const uint4*>(v + (gi.rr0 - 1 - j) * rowstride + gi.coff);
-            else if (hist_in)
-                wraw[j] = *reinterpret_cast<const uint4*>(hist_in + ((long long)gi.bseq * 3 + (3 + tau)) * rowstride + gi.coff);
+            else if (hist_in && gi.hseq >= 0)
+                wraw[j] = *reinterpret_cast<const uint4*>(hist_in + ((long long)gi.hseq * 3 + (3 + tau)) * rowstride + gi.coff);
         }
 #pragma unroll
         for (int i = 0; i < RUN; ++i)
@@ -232,9 +246,10 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
 #pragma unroll
             for (int e = 0; e < VN; ++e) { win[2][e] = win[1][e]; win[1][e] = win[0][e]; win[0][e] = cv[e]; }
             if (hist_out && tpos == Tn - 1) {
+                const long long hq = slots ? gi.hseq : bseq;
 #pragma unroll
                 for (int j = 0; j < 3; ++j)
-                    *reinterpret_cast<uint4*>(hist_out + ((long long)bseq * 3 + (2 - j)) * rowstride + coff) = V16::pack(win[j]);
+                    *reinterpret_cast<uint4*>(hist_out + (hq * 3 + (2 - j)) * rowstride + coff) = V16::pack(win[j]);
             }
             ++tpos;
         }

@@ -1,0 +1,107 @@
+"""A chunked-prefill serving loop over the JetBlock mixer with a state and
+history cache.
+
+The recurrent state of a JetBlock layer has a fixed size per sequence (its
+H x dv x dk float32 state and the last three raw values of V for the conv),
+which is what makes the mixer cheap to serve: the Jet-Nemotron paper (section
+2.5, finding 4; the efficiency FAQ of the explainer) puts decode speed down to
+cache size. This module keeps those per-sequence states in two pools and runs
+the library's calls on them:
+
+  admit(seq)   take a free pool entry (zero state and history)
+  prefill(seq, ...)  the sequence's next prompt tokens, in pieces of at most
+               `chunk_tokens` (chunked prefill), each piece continuing from
+               the entry's state and history (jet_jetblock_prefill)
+  decode(seqs, ...)  one new token for each of a batch of sequences, in place
+               on their entries (jet_jetblock_decode_slots)
+  release(seq) return the entry
+
+All arithmetic runs in the library's kernels; this module only keeps the
+pool bookkeeping and orders the calls (torch provides device memory).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import jet_jetblock_decode_slots, jet_jetblock_prefill, jet_jetblock_prefill_workspace_size
+
+
+class JetEngine:
+    def __init__(self, W1: torch.Tensor, W2: torch.Tensor, H: int, dk: int, dv: int, max_seqs: int,
+                 chunk_tokens: int = 4096, stream=None):
+        if chunk_tokens <= 0 or max_seqs <= 0:
+            raise ValueError("chunk_tokens and max_seqs must be positive")
+        self.W1, self.W2 = W1, W2
+        self.H, self.dk, self.dv = H, dk, dv
+        self.chunk_tokens = chunk_tokens
+        self.stream = stream
+        dev, dt = W1.device, W1.dtype
+        self.S = torch.zeros((max_seqs, H, dv, dk), device=dev, dtype=torch.float32)
+        self.hist = torch.zeros((max_seqs, 3, H, dv), device=dev, dtype=dt)
+        self._hist_out = torch.empty((1, 3, H, dv), device=dev, dtype=dt)
+        self._free = list(range(max_seqs - 1, -1, -1))    # pop() hands out the lowest entry first
+        self.slot: dict = {}                               # sequence id -> pool entry
+        self.pos: dict = {}                                # sequence id -> tokens consumed
+        self._ws = None
+
+    # ---------------------------------------------------------------- pool entries
+    @property
+    def free_slots(self) -> int:
+        return len(self._free)
+
+    def admit(self, seq) -> int:
+        """Give `seq` a pool entry with a zero state and a zero history."""
+        if seq in self.slot:
+            raise KeyError(f"sequence {seq!r} is already admitted")
+        if not self._free:
+            raise RuntimeError("state cache is full")
+        s = self._free.pop()
+        self.S[s].zero_()
+        self.hist[s].zero_()
+        self.slot[seq] = s
+        self.pos[seq] = 0
+        return s
+
+    def release(self, seq) -> None:
+        self._free.append(self.slot.pop(seq))
+        del self.pos[seq]
+
+    # ---------------------------------------------------------------- the mixer
+    def pieces(self, T: int):
+        """Token ranges of a prompt of T tokens, at most chunk_tokens each."""
+        return [(t0, min(T, t0 + self.chunk_tokens)) for t0 in range(0, T, self.chunk_tokens)]
+
+    def _workspace(self, T: int):
+        n = jet_jetblock_prefill_workspace_size(1, T, self.H, self.dk, self.dv, 64, self.W1.dtype)
+        if self._ws is None or self._ws.numel() < n:
+            self._ws = torch.empty(max(n, 16), device=self.W1.device, dtype=torch.uint8)
+        return self._ws
+
+    def prefill(self, seq, x, q, k, v, g, beta) -> torch.Tensor:
+        """The next T prompt tokens of `seq`: x [T,D], q, k [T,H,dk], v [T,H,dv]
+        (raw), g, beta [T,H]. Returns o [T,H,dv]; the entry's state and history
+        advance past the tokens."""
+        s = self.slot[seq]
+        S = self.S[s:s + 1]
+        outs = []
+        for t0, t1 in self.pieces(x.shape[0]):
+            piece = lambda a: a[t0:t1].unsqueeze(0)
+            o, _ = jet_jetblock_prefill(piece(x), self.W1, self.W2, piece(q), piece(k), piece(v), piece(g),
+                                        piece(beta), self.hist[s:s + 1], self._hist_out, S, None, S,
+                                        self._workspace(t1 - t0), stream=self.stream)
+            self.hist[s].copy_(self._hist_out[0])
+            outs.append(o[0])
+            self.pos[seq] += t1 - t0
+        return torch.cat(outs) if len(outs) > 1 else outs[0]
+
+    def decode(self, seqs, x, q, k, v, g, beta) -> torch.Tensor:
+        """One new token for each sequence of `seqs` (batch order): x [B,D],
+        q, k [B,H,dk], v [B,H,dv] (raw), g, beta [B,H]. Returns o [B,H,dv]."""
+        if len(set(seqs)) != len(seqs):
+            raise ValueError("a sequence appears twice in one decode batch")
+        slots = torch.tensor([self.slot[s] for s in seqs], dtype=torch.int32).to(self.S.device, non_blocking=True)
+        o = jet_jetblock_decode_slots(x, self.W1, self.W2, q, k, v, g, beta, self.hist, self.S, slots,
+                                      stream=self.stream)
+        for s in seqs:
+            self.pos[s] += 1
+        return o

@@ -208,3 +208,20 @@ def test_jetblock_prefill_workspace_off_the_tensor_core_path():
     for (B, T, H, dk, dv, dt, es) in ((1, 64, 2, 16, 32, torch.float32, 4), (2, 100, 3, 48, 64, torch.bfloat16, 2)):
         up = lambda x: -(-x // 1024) * 1024
         assert jet.jet_jetblock_prefill_workspace_size(B, T, H, dk, dv, 64, dt) == up(B * T * H * 16) + up(B * T * H * dv * es)
+
+
+def decode_slots(lib, x=A, w1=A, w2=A, q=A, k=A, v=A, g=A, b=A, hist=A, S=A, slots=A, n_slots=8, o=A,
+                 vc=A + (1 << 22), taps=None, B=2, D=64, H=2, dk=16, dv=32, hidden=32, width=4, dt=BF16):
+    return lib.jet_jetblock_decode_slots(P(x), P(w1), P(w2), P(q), P(k), P(v), P(g), P(b), P(hist), P(S), P(slots),
+                                         n_slots, P(o), P(vc), P(taps), B, D, H, dk, dv, hidden, width, dt, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(slots=None), INVALID), (dict(hist=None), INVALID), (dict(vc=None), INVALID),
+    (dict(n_slots=0), INVALID), (dict(n_slots=1), INVALID),   # fewer pool entries than sequences
+    (dict(vc=A + 32), INVALID),                                # the conv output may not overlap v
+    (dict(dk=24), UNSUPPORTED), (dict(S=A + 8), MISALIGNED), (dict(slots=A + 2), MISALIGNED),
+    (dict(hist=A + 8), MISALIGNED),
+])
+def test_decode_slots_rejects(lib, kw, expect):
+    assert decode_slots(lib, **kw) == expect

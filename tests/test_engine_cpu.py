@@ -1,0 +1,91 @@
+"""Host logic of the serving loop (linear_attention_lm_gen_b200.engine): pool
+entries, chunked-prefill pieces and the calls it makes, checked on the CPU
+with recording stand-ins for the two library calls (no kernel runs here)."""
+import pytest
+import torch
+
+from linear_attention_lm_gen_b200 import engine as eng
+
+H, DK, DV, D = 2, 16, 32, 64
+
+
+class Calls:
+    def __init__(self):
+        self.prefill, self.decode = [], []
+
+    def fake_prefill(self, x, W1, W2, q, k, v, g, beta, hist_in, hist_out, S0, o, S_out, workspace, *, stream=None):
+        T = x.shape[1]
+        assert S0 is S_out or S0.data_ptr() == S_out.data_ptr()          # the state advances in place
+        assert hist_out.data_ptr() != hist_in.data_ptr()                  # new history into a separate buffer
+        self.prefill.append((T, S0.data_ptr(), hist_in.data_ptr()))
+        hist_out.copy_(hist_in + 1)                                       # marks: one per piece
+        S_out.add_(T)
+        return torch.full((1, T, H, DV), float(len(self.prefill))), S_out
+
+    def fake_decode(self, x, W1, W2, q, k, v, g, beta, hist_pool, S_pool, slots, *, stream=None):
+        self.decode.append(slots.tolist())
+        for b, s in enumerate(slots.tolist()):
+            S_pool[s] += 1000
+        return torch.zeros((x.shape[0], H, DV))
+
+
+@pytest.fixture
+def engine(monkeypatch):
+    c = Calls()
+    monkeypatch.setattr(eng, "jet_jetblock_prefill", c.fake_prefill)
+    monkeypatch.setattr(eng, "jet_jetblock_decode_slots", c.fake_decode)
+    monkeypatch.setattr(eng, "jet_jetblock_prefill_workspace_size", lambda *a, **k: 64)
+    e = eng.JetEngine(torch.zeros(D, 32), torch.zeros(32, 4 * H), H, DK, DV, max_seqs=3, chunk_tokens=128)
+    return e, c
+
+
+def prompt(T):
+    return (torch.zeros(T, D), torch.zeros(T, H, DK), torch.zeros(T, H, DK), torch.zeros(T, H, DV),
+            torch.zeros(T, H), torch.zeros(T, H))
+
+
+def test_pool_entries_are_handed_out_and_reused(engine):
+    e, _ = engine
+    assert [e.admit(s) for s in ("a", "b", "c")] == [0, 1, 2]
+    with pytest.raises(RuntimeError):
+        e.admit("d")
+    with pytest.raises(KeyError):
+        e.admit("a")
+    e.S[1].fill_(5.0)
+    e.hist[1].fill_(3.0)
+    e.release("b")
+    assert e.free_slots == 1
+    assert e.admit("d") == 1
+    assert float(e.S[1].abs().sum()) == 0.0 and float(e.hist[1].abs().sum()) == 0.0   # a fresh sequence
+
+
+def test_prefill_runs_in_pieces_that_continue_the_state(engine):
+    e, c = engine
+    e.admit("a")
+    s = e.admit("b")
+    assert e.pieces(333) == [(0, 128), (128, 256), (256, 333)]
+    o = e.prefill("b", *prompt(333))
+    assert [t for t, _, _ in c.prefill] == [128, 128, 77]
+    assert all(p == e.S[s].data_ptr() for _, p, _ in c.prefill)          # every piece on the same entry
+    assert all(h == e.hist[s].data_ptr() for _, _, h in c.prefill)
+    assert o.shape == (333, H, DV)
+    assert torch.equal(o[:128], torch.full((128, H, DV), 1.0)) and torch.equal(o[256:], torch.full((77, H, DV), 3.0))
+    assert float(e.S[s].flatten()[0]) == 333.0                             # each piece continued the last
+    assert float(e.hist[s].flatten()[0]) == 3.0                            # history carried piece to piece
+    assert float(e.S[0].abs().sum()) == 0.0                                # other entries untouched
+    assert e.pos["b"] == 333
+
+
+def test_decode_batches_by_pool_entry(engine):
+    e, c = engine
+    for s in ("a", "b", "c"):
+        e.admit(s)
+    e.release("a")
+    e.admit("d")                                                           # takes entry 0 again
+    e.decode(["c", "d", "b"], torch.zeros(3, D), torch.zeros(3, H, DK), torch.zeros(3, H, DK),
+             torch.zeros(3, H, DV), torch.zeros(3, H), torch.zeros(3, H))
+    assert c.decode == [[2, 0, 1]]
+    assert e.pos == {"b": 1, "c": 1, "d": 1}
+    with pytest.raises(ValueError):
+        e.decode(["b", "b"], torch.zeros(2, D), torch.zeros(2, H, DK), torch.zeros(2, H, DK), torch.zeros(2, H, DV),
+                 torch.zeros(2, H), torch.zeros(2, H))
