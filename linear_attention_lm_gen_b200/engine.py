@@ -12,12 +12,19 @@ the library's calls on them:
   prefill(seq, ...)  the sequence's next prompt tokens, in pieces of at most
                `chunk_tokens` (chunked prefill), each piece continuing from
                the entry's state and history (jet_jetblock_prefill)
+  prefill_many({seq: ...})  the same for several sequences of different
+               lengths: in every round, the pieces of equal length run as one
+               batched call
   decode(seqs, ...)  one new token for each of a batch of sequences, in place
                on their entries (jet_jetblock_decode_slots)
   release(seq) return the entry
 
-All arithmetic runs in the library's kernels; this module only keeps the
-pool bookkeeping and orders the calls (torch provides device memory).
+All arithmetic runs in the library's kernels. This module only keeps the
+pool bookkeeping and orders the calls. torch provides device memory and
+moves data: it stacks the pieces of a batched call and gathers and scatters
+their pool entries (the prefill takes its states as one [B,...] tensor).
+Everything is issued on torch's current stream, so the library calls and
+the data movement stay in order.
 """
 from __future__ import annotations
 
@@ -28,13 +35,12 @@ from . import jet_jetblock_decode_slots, jet_jetblock_prefill, jet_jetblock_pref
 
 class JetEngine:
     def __init__(self, W1: torch.Tensor, W2: torch.Tensor, H: int, dk: int, dv: int, max_seqs: int,
-                 chunk_tokens: int = 4096, stream=None):
+                 chunk_tokens: int = 4096):
         if chunk_tokens <= 0 or max_seqs <= 0:
             raise ValueError("chunk_tokens and max_seqs must be positive")
         self.W1, self.W2 = W1, W2
         self.H, self.dk, self.dv = H, dk, dv
         self.chunk_tokens = chunk_tokens
-        self.stream = stream
         dev, dt = W1.device, W1.dtype
         self.S = torch.zeros((max_seqs, H, dv, dk), device=dev, dtype=torch.float32)
         self.hist = torch.zeros((max_seqs, 3, H, dv), device=dev, dtype=dt)
@@ -71,8 +77,8 @@ class JetEngine:
         """Token ranges of a prompt of T tokens, at most chunk_tokens each."""
         return [(t0, min(T, t0 + self.chunk_tokens)) for t0 in range(0, T, self.chunk_tokens)]
 
-    def _workspace(self, T: int):
-        n = jet_jetblock_prefill_workspace_size(1, T, self.H, self.dk, self.dv, 64, self.W1.dtype)
+    def _workspace(self, T: int, B: int = 1):
+        n = jet_jetblock_prefill_workspace_size(B, T, self.H, self.dk, self.dv, 64, self.W1.dtype)
         if self._ws is None or self._ws.numel() < n:
             self._ws = torch.empty(max(n, 16), device=self.W1.device, dtype=torch.uint8)
         return self._ws
@@ -88,11 +94,40 @@ class JetEngine:
             piece = lambda a: a[t0:t1].unsqueeze(0)
             o, _ = jet_jetblock_prefill(piece(x), self.W1, self.W2, piece(q), piece(k), piece(v), piece(g),
                                         piece(beta), self.hist[s:s + 1], self._hist_out, S, None, S,
-                                        self._workspace(t1 - t0), stream=self.stream)
+                                        self._workspace(t1 - t0))
             self.hist[s].copy_(self._hist_out[0])
             outs.append(o[0])
             self.pos[seq] += t1 - t0
         return torch.cat(outs) if len(outs) > 1 else outs[0]
+
+    def prefill_many(self, prompts: dict) -> dict:
+        """Chunked prefill of several sequences at once. prompts: seq ->
+        (x, q, k, v, g, beta) as for prefill (lengths may differ). Round r
+        takes the r-th piece of every sequence that has one; pieces of equal
+        length (every full piece, and tails that happen to match) share one
+        batched jet_jetblock_prefill call. Returns seq -> o [T,H,dv]."""
+        outs = {seq: [] for seq in prompts}
+        plan = {seq: self.pieces(inp[0].shape[0]) for seq, inp in prompts.items()}
+        for r in range(max((len(p) for p in plan.values()), default=0)):
+            groups: dict = {}
+            for seq, p in plan.items():
+                if r < len(p):
+                    groups.setdefault(p[r][1] - p[r][0], []).append(seq)
+            for L, seqs in groups.items():
+                idx = torch.tensor([self.slot[sq] for sq in seqs], device=self.S.device)
+                S = self.S.index_select(0, idx)
+                hin = self.hist.index_select(0, idx)
+                hout = torch.empty_like(hin)
+                stack = [torch.stack([prompts[sq][j][plan[sq][r][0]:plan[sq][r][1]] for sq in seqs])
+                         for j in range(6)]
+                o, _ = jet_jetblock_prefill(stack[0], self.W1, self.W2, *stack[1:], hin, hout, S, None, S,
+                                            self._workspace(L, len(seqs)))
+                self.S.index_copy_(0, idx, S)
+                self.hist.index_copy_(0, idx, hout)
+                for b, sq in enumerate(seqs):
+                    outs[sq].append(o[b])
+                    self.pos[sq] += L
+        return {sq: torch.cat(v) if len(v) > 1 else v[0] for sq, v in outs.items()}
 
     def decode(self, seqs, x, q, k, v, g, beta) -> torch.Tensor:
         """One new token for each sequence of `seqs` (batch order): x [B,D],
@@ -100,8 +135,7 @@ class JetEngine:
         if len(set(seqs)) != len(seqs):
             raise ValueError("a sequence appears twice in one decode batch")
         slots = torch.tensor([self.slot[s] for s in seqs], dtype=torch.int32).to(self.S.device, non_blocking=True)
-        o = jet_jetblock_decode_slots(x, self.W1, self.W2, q, k, v, g, beta, self.hist, self.S, slots,
-                                      stream=self.stream)
+        o = jet_jetblock_decode_slots(x, self.W1, self.W2, q, k, v, g, beta, self.hist, self.S, slots)
         for s in seqs:
             self.pos[s] += 1
         return o

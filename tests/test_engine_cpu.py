@@ -13,7 +13,7 @@ class Calls:
     def __init__(self):
         self.prefill, self.decode = [], []
 
-    def fake_prefill(self, x, W1, W2, q, k, v, g, beta, hist_in, hist_out, S0, o, S_out, workspace, *, stream=None):
+    def fake_prefill(self, x, W1, W2, q, k, v, g, beta, hist_in, hist_out, S0, o, S_out, workspace):
         T = x.shape[1]
         assert S0 is S_out or S0.data_ptr() == S_out.data_ptr()          # the state advances in place
         assert hist_out.data_ptr() != hist_in.data_ptr()                  # new history into a separate buffer
@@ -22,7 +22,7 @@ class Calls:
         S_out.add_(T)
         return torch.full((1, T, H, DV), float(len(self.prefill))), S_out
 
-    def fake_decode(self, x, W1, W2, q, k, v, g, beta, hist_pool, S_pool, slots, *, stream=None):
+    def fake_decode(self, x, W1, W2, q, k, v, g, beta, hist_pool, S_pool, slots):
         self.decode.append(slots.tolist())
         for b, s in enumerate(slots.tolist()):
             S_pool[s] += 1000
@@ -89,3 +89,48 @@ def test_decode_batches_by_pool_entry(engine):
     with pytest.raises(ValueError):
         e.decode(["b", "b"], torch.zeros(2, D), torch.zeros(2, H, DK), torch.zeros(2, H, DK), torch.zeros(2, H, DV),
                  torch.zeros(2, H), torch.zeros(2, H))
+
+
+# ---------------------------------------------------------------- batched chunked prefill, numerically
+# The library call is stood in for by the float64 oracle of the whole mixer
+# (with initial state and history), so the test checks that the engine's
+# rounds, groups, gathers and scatters continue every sequence correctly.
+def oracle_prefill(orc, calls):
+    def run(x, W1, W2, q, k, v, g, beta, hist_in, hist_out, S0, o, S_out, workspace):
+        n = lambda t: t.double().numpy()
+        r = orc.jetblock_prefill(n(x), n(W1), n(W2), n(q), n(k), n(v), n(g), n(beta), n(S0), n(hist_in))
+        calls.append(tuple(x.shape[:2]))
+        S_out.copy_(torch.from_numpy(r["S"]))
+        hist_out.copy_(torch.from_numpy(r["hist"]))
+        return torch.from_numpy(r["o"]), S_out
+    return run
+
+
+def test_prefill_many_batches_equal_pieces_and_continues_every_sequence(monkeypatch):
+    import numpy as np
+    import synth
+    from oracle import get as get_oracle
+    orc = get_oracle()
+    calls = []
+    monkeypatch.setattr(eng, "jet_jetblock_prefill", oracle_prefill(orc, calls))
+    monkeypatch.setattr(eng, "jet_jetblock_prefill_workspace_size", lambda *a, **k: 64)
+    shp = synth.JetShape("t", B=1, T=1, H=H, dk=DK, dv=DV, D=D, dtype="f32")
+    lens = {"a": 300, "b": 300, "c": 77}
+    inp = {n: synth.prefill_inputs(shp, seed=30 + i, T=T) for i, (n, T) in enumerate(lens.items())}
+    W1 = torch.from_numpy(inp["a"]["W1"]).double()
+    W2 = torch.from_numpy(inp["a"]["W2"]).double()
+    e = eng.JetEngine(W1, W2, H, DK, DV, max_seqs=4, chunk_tokens=128)
+    for n in ("c", "a", "b"):
+        e.admit(n)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a[0])).double()
+    outs = e.prefill_many({n: tuple(t(inp[n][k]) for k in ("x", "q", "k", "v", "g", "beta")) for n in lens})
+    # rounds: (a, b) full + (c) tail; (a, b) full; (a, b) tails of 44
+    assert calls == [(2, 128), (1, 77), (2, 128), (2, 44)]
+    for n, T in lens.items():
+        d = {k: inp[n][k].astype(np.float64) for k in ("x", "q", "k", "v", "g", "beta")}
+        r = orc.jetblock_prefill(d["x"], inp["a"]["W1"].astype(np.float64), inp["a"]["W2"].astype(np.float64),
+                                 d["q"], d["k"], d["v"], d["g"], d["beta"])
+        np.testing.assert_allclose(outs[n].numpy(), r["o"][0], rtol=1e-5, atol=1e-5)
+        np.testing.assert_allclose(e.S[e.slot[n]].double().numpy(), r["S"][0], rtol=1e-5, atol=1e-5)
+        np.testing.assert_array_equal(e.hist[e.slot[n]].numpy(), r["hist"][0])
+        assert e.pos[n] == T

@@ -109,3 +109,30 @@ def test_engine_chunked_prefill_then_decode_matches_the_oracle(dtype, H, dk, dv,
         assert_close(host64(e.S[e.slot[n]]), r["S"][0], dtype, f"{n} S")
         np.testing.assert_array_equal(host64(e.hist[e.slot[n]]), r["hist"][0])
         assert e.pos[n] == T + steps
+
+
+def test_engine_batched_prefill_matches_the_oracle():
+    # prompts of 300, 300 and 77 tokens in 128-token pieces: equal pieces share one batched call
+    from linear_attention_lm_gen_b200.engine import JetEngine
+    orc = get_oracle()
+    H, dk, dv, D = 12, 96, 256, 1536
+    lens = {"a": 300, "b": 300, "c": 77}
+    shp = synth.JetShape("t", B=1, T=1, H=H, dk=dk, dv=dv, D=D, dtype="bf16")
+    seqs = {n: synth.prefill_inputs(shp, seed=40 + i, T=T) for i, (n, T) in enumerate(lens.items())}
+    for n in seqs:
+        seqs[n]["W1"], seqs[n]["W2"] = seqs["a"]["W1"], seqs["a"]["W2"]
+    W = gpu_inputs(seqs["a"])
+    e = JetEngine(W["W1"], W["W2"], H, dk, dv, max_seqs=4, chunk_tokens=128)
+    for n in ("b", "c", "a"):
+        e.admit(n)
+    prompts = {}
+    for n in lens:
+        d = gpu_inputs(seqs[n])
+        prompts[n] = tuple(d[k_][0] for k_ in ("x", "q", "k", "v", "g", "beta"))
+    outs = e.prefill_many(prompts)
+    for n in lens:
+        ref = to_oracle(seqs[n])
+        r = orc.jetblock_prefill(ref["x"], ref["W1"], ref["W2"], ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"])
+        assert_close(host64(outs[n]), r["o"][0], "bf16", f"{n} o")
+        assert_close(host64(e.S[e.slot[n]]), r["S"][0], "bf16", f"{n} S")
+        np.testing.assert_array_equal(host64(e.hist[e.slot[n]]), r["hist"][0])
