@@ -1,0 +1,189 @@
+"""The mbarrier protocol of the prefill state chain (csrc/k_prefill_chain.cuh),
+checked as a model under random interleavings on the CPU.
+
+Each role of the kernel is written out as the sequence of waits and
+completions it performs, in the kernel's order:
+  chain warps  per chunk c: wait P4(c-1) [and P5(c-1)], wait the image; E4
+               -> arrive AS; wait P3(c); E5 -> arrive AW; at the end wait P4(last)
+  out warps    per chunk c (outputs only): wait P5(c); read O -> arrive X2FREE
+  MMA thread   per chunk c: wait AS(c), P2a(c) -> P3; wait AW(c), K(c) -> P4
+  load thread  prologue loads; P2a(0); per chunk c: the next V load once
+               P2a(c) is done (V(c+2), or V(c+1) with the conv folded in, whose
+               halo is the previous tile); P5a(c), P5b(c); P2a(c+1); K and image
+               loads once chunk c no longer reads their buffers
+Loads and MMA commit groups complete after random delays (each issuer's
+groups in order). A waiter of phase n is released when the barrier has
+completed n + 1 phases; seeing n + 2 would make its parity wait ambiguous.
+The model checks: no deadlock, no waiter two phases behind, every issued
+operation completes, and (folded conv) no V load overwrites a tile while a
+later P2a still needs it as its halo.
+"""
+import random
+
+import pytest
+
+
+def run(nch, nkbuf, write_o, conv, seed, mutant=None):
+    """One random interleaving; raises AssertionError on a protocol fault.
+    mutant (for the tests of the model itself): "plain_v" keeps the two-ahead
+    V schedule of plain V with the conv folded in; "one_p2" shares a single
+    P2a barrier between the two V buffers."""
+    plain_v = not conv or mutant == "plain_v"
+    p2 = (lambda c: ("P2", 0)) if mutant == "one_p2" else (lambda c: ("P2", c & 1))
+    p2n = (lambda c: c) if mutant == "one_p2" else (lambda c: c >> 1)
+    rng = random.Random(seed)
+    comp = {}
+    C = lambda b: comp.get(b, 0)
+    pending, mq = [], {"M": [], "L": []}
+    last_v = {0: None, 1: None}          # buffer -> chunk of the last V load issued into it
+    nv = [0]
+
+    def load(bar):
+        if bar[0] == "V":
+            last_v[bar[1]] = nv[0]
+            nv[0] += 1
+        pending.append([rng.randint(1, 8), bar])
+
+    def mma(who, bar):
+        mq[who].append([rng.randint(1, 4), bar])
+
+    def chain():
+        for c in range(nch):
+            if c >= 1:
+                yield ("SD", (c - 1) & 1), (c - 1) >> 1
+                if write_o:
+                    yield ("OD", (c - 1) & 1), (c - 1) >> 1
+            yield ("IMG", c & 1), c >> 1
+            comp[("AS",)] = C(("AS",)) + 1
+            yield ("P3",), c
+            comp[("AW",)] = C(("AW",)) + 1
+        if nch:
+            yield ("SD", (nch - 1) & 1), (nch - 1) >> 1
+
+    def out():
+        for c in range(nch if write_o else 0):
+            yield ("OD", c & 1), c >> 1
+            comp[("X2F", c & 1)] = C(("X2F", c & 1)) + 1
+
+    def loader():
+        if nch == 0:
+            return
+        load(("IMG", 0)); load(("V", 0)); load(("K", 0))
+        if conv:
+            load(("H0",))
+        if nch > 1:
+            load(("IMG", 1))
+            if plain_v:
+                load(("V", 1))
+        if nkbuf == 2 and nch > 1:
+            load(("K", 1))
+        yield ("IMG", 0), 0
+        yield ("V", 0), 0
+        if conv:
+            yield ("H0",), 0
+        mma("L", p2(0))
+        for c in range(nch):
+            ahead = 2 if plain_v else 1
+            if c + ahead < nch:
+                yield p2(c), p2n(c)
+                load(("V", (c + ahead) & 1))
+            if write_o:
+                yield ("AS",), c
+                if c >= 2:
+                    yield ("X2F", c & 1), (c - 2) >> 1
+                yield ("AW",), c
+                mma("L", ("OD", c & 1))
+            if c + 1 < nch:
+                yield ("IMG", (c + 1) & 1), (c + 1) >> 1
+                yield ("V", (c + 1) & 1), (c + 1) >> 1
+                if conv:   # the halo of P2a(c+1) is V(c): still the last load into its buffer
+                    assert last_v[c & 1] == c, f"halo of chunk {c + 1} overwritten"
+                mma("L", p2(c + 1))
+            if c + nkbuf < nch or c + 2 < nch:
+                yield ("SD", c & 1), c >> 1
+                if write_o:
+                    yield ("OD", c & 1), c >> 1
+                if c + nkbuf < nch:
+                    load(("K", (c + nkbuf) % nkbuf))
+                if c + 2 < nch:
+                    load(("IMG", (c + 2) & 1))
+
+    def mma_thread():
+        for c in range(nch):
+            yield ("AS",), c
+            yield p2(c), p2n(c)
+            mma("M", ("P3",))
+            yield ("AW",), c
+            yield ("K", c % nkbuf), c // nkbuf
+            mma("M", ("SD", c & 1))
+
+    roles = {"chain": chain(), "out": out(), "load": loader(), "mma": mma_thread()}
+    cur = dict.fromkeys(roles)
+    slow = {k: rng.choice([0.0, 0.5, 0.9, 0.97]) for k in roles}
+    done = set()
+    for _ in range(200000):
+        if len(done) == len(roles):
+            break
+        moved = False
+        for k in rng.sample(list(roles), len(roles)):
+            if k in done:
+                continue
+            if rng.random() < slow[k]:
+                moved = True
+                continue
+            if cur[k] is None:
+                try:
+                    cur[k] = next(roles[k])
+                except StopIteration:
+                    done.add(k)
+                moved = True
+                continue
+            bar, n = cur[k]
+            assert C(bar) < n + 2, f"{k} waits phase {n} of {bar} after {C(bar)} completions"
+            if C(bar) == n + 1:
+                cur[k] = None
+                moved = True
+        for p in pending:
+            p[0] -= 1
+        for p in [p for p in pending if p[0] <= 0]:
+            comp[p[1]] = C(p[1]) + 1
+            pending.remove(p)
+            moved = True
+        for who in ("M", "L"):
+            q = mq[who]
+            if q and rng.random() < 0.7:
+                q[0][0] -= 1
+                if q[0][0] <= 0:
+                    b = q.pop(0)[1]
+                    comp[b] = C(b) + 1
+                    moved = True
+        assert moved or pending or any(mq.values()), f"deadlock: {cur}"
+    else:
+        raise AssertionError("no progress within the step budget")
+    assert not pending and not any(mq.values()), "operations left in flight"
+
+
+@pytest.mark.parametrize("conv", [False, True])
+@pytest.mark.parametrize("write_o", [False, True])
+@pytest.mark.parametrize("nkbuf", [1, 2])
+def test_chain_protocol_has_no_deadlock_and_no_two_phase_lag(conv, write_o, nkbuf):
+    for nch in range(0, 10):
+        for seed in range(40):
+            run(nch, nkbuf, write_o, conv, seed)
+
+
+def test_the_model_catches_a_halo_overwrite():
+    # with the folded conv, the plain two-ahead V schedule would overwrite the tile that the
+    # next P2a still reads as its halo: the model must see it
+    with pytest.raises(AssertionError, match="halo"):
+        for seed in range(200):
+            run(6, 2, False, True, seed, mutant="plain_v")
+
+
+def test_the_model_catches_a_lagging_waiter():
+    # one P2a barrier for both V buffers lets the load thread run two phases ahead of the
+    # MMA thread's wait (the mistake the per-buffer barriers fix)
+    with pytest.raises(AssertionError, match="completions"):
+        for seed in range(300):
+            for w in (False, True):
+                run(8, 2, w, False, seed, mutant="one_p2")
