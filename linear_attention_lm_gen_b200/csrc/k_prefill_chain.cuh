@@ -23,7 +23,8 @@
 // is finished), V double-buffered (V(c+2) once P2a(c) is done), K
 // double-buffered for dk <= 96 (K(c+2) once P4(c) is done) and single for
 // dk = 128 (K(c+1) once P4(c) is done; shared memory is full); outputs are
-// staged 32 tokens at a time. TMEM: S, X1[2] (U^T then Wt^T), X2[2] (O^T) =
+// staged 32 tokens at a time, or 16 where the images leave less room (dk = 96).
+// TMEM: S, X1[2] (U^T then Wt^T), X2[2] (O^T) =
 // 384 of 512 columns. The roles on the critical path (chain warps, MMA
 // thread) spin on the mbarrier before they start to sleep between polls, so
 // they wake within tens of cycles; the others sleep between polls and leave
