@@ -225,3 +225,27 @@ def decode_slots(lib, x=A, w1=A, w2=A, q=A, k=A, v=A, g=A, b=A, hist=A, S=A, slo
 ])
 def test_decode_slots_rejects(lib, kw, expect):
     assert decode_slots(lib, **kw) == expect
+
+
+def segments_from_workspace(B, T, H, dk, dv):
+    """The number of sequence-parallel segments P the library plans, recovered from its minimum
+    workspace: 4 * (B (P-1) H dv dk + B (P-1) H dk (dk + 8) + B P H dv dk) bytes (0 when P = 1)."""
+    n = jet.jet_gdn_prefill_workspace_min(B, T, H, dk, dv)
+    if n == 0:
+        return 1
+    per_seg = 4 * B * H * (2 * dv * dk + dk * (dk + 8))
+    P = (n // 4 + B * H * (dv * dk + dk * (dk + 8))) * 4 // per_seg
+    assert 4 * (B * (P - 1) * H * dv * dk + B * (P - 1) * H * dk * (dk + 8) + B * P * H * dv * dk) == n
+    return P
+
+
+@pytest.mark.parametrize("B,T,H,dk,dv,P", [
+    (1, 4096, 12, 96, 256, 5),       # 2B prompt: 5 segments of 13 chunks, both phases within 148 SMs
+    (1, 65536, 16, 128, 256, 4),     # 4B long prompt
+    (1, 262144, 12, 96, 256, 5),
+    (1, 64 * 14, 12, 96, 256, 1),    # segments keep at least 8 chunks: 14 chunks run in one pass
+    (1, 64 * 15, 12, 96, 256, 2),    # ... and 15 split in two
+    (8, 4096, 12, 96, 256, 1),       # a batch already fills the GPU
+])
+def test_segment_plan_of_the_stated_shapes(lib, B, T, H, dk, dv, P):
+    assert segments_from_workspace(B, T, H, dk, dv) == P
