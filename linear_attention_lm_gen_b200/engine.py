@@ -18,6 +18,10 @@ the library's calls on them:
   decode(seqs, ...)  one new token for each of a batch of sequences, in place
                on their entries (jet_jetblock_decode_slots)
   release(seq) return the entry
+  submit(seq, prompt) / step(tokens)  a serving iteration: up to
+               `chunk_tokens` queued prompt tokens (oldest prompt first; a
+               long prompt continues in later steps), then one decode token
+               for each running sequence the caller supplies a token for
 
 All arithmetic runs in the library's kernels. This module only keeps the
 pool bookkeeping and orders the calls. torch provides device memory and
@@ -49,6 +53,7 @@ class JetEngine:
         self.slot: dict = {}                               # sequence id -> pool entry
         self.pos: dict = {}                                # sequence id -> tokens consumed
         self._ws = None
+        self._queue: list = []                             # [seq, prompt tuple, tokens done]
 
     # ---------------------------------------------------------------- pool entries
     @property
@@ -128,6 +133,48 @@ class JetEngine:
                     outs[sq].append(o[b])
                     self.pos[sq] += L
         return {sq: torch.cat(v) if len(v) > 1 else v[0] for sq, v in outs.items()}
+
+    # ---------------------------------------------------------------- serving iterations
+    def submit(self, seq, prompt) -> None:
+        """Queue a prompt (x, q, k, v, g, beta as for prefill); the sequence is
+        admitted now, so the cache must have a free entry."""
+        self.admit(seq)
+        self._queue.append([seq, prompt, 0])
+
+    @property
+    def prefilling(self) -> list:
+        return [q[0] for q in self._queue]
+
+    def step(self, tokens: dict | None = None) -> dict:
+        """One serving iteration. Prefill: up to chunk_tokens tokens of the
+        queued prompts, oldest first (prefill_many batches pieces of equal
+        length). Decode: one token for every sequence in `tokens` (seq ->
+        (x, q, k, v, g, beta) of one token), which must have finished its
+        prompt. Returns seq -> outputs of this step ([n,H,dv] prompt outputs
+        for prefill, [H,dv] for a decoded token)."""
+        budget, work, took = self.chunk_tokens, {}, {}
+        for seq, prompt, done in self._queue:
+            if budget == 0:
+                break
+            n = min(budget, prompt[0].shape[0] - done)
+            work[seq] = tuple(a[done:done + n] for a in prompt)
+            took[seq] = n
+            budget -= n
+        still = {seq for seq, prompt, done in self._queue if done + took.get(seq, 0) < prompt[0].shape[0]}
+        busy = still & set(tokens or ())
+        if busy:                                   # checked before any work is issued
+            raise ValueError(f"sequences still in prefill: {sorted(map(str, busy))}")
+        out = self.prefill_many(work) if work else {}
+        for item in self._queue:
+            item[2] += took.get(item[0], 0)
+        self._queue = [q for q in self._queue if q[0] in still]
+        if tokens:
+            seqs = list(tokens)
+            stack = [torch.stack([tokens[sq][j] for sq in seqs]) for j in range(6)]
+            o = self.decode(seqs, *stack)
+            for b, sq in enumerate(seqs):
+                out[sq] = o[b]
+        return out
 
     def decode(self, seqs, x, q, k, v, g, beta) -> torch.Tensor:
         """One new token for each sequence of `seqs` (batch order): x [B,D],

@@ -134,3 +134,55 @@ def test_prefill_many_batches_equal_pieces_and_continues_every_sequence(monkeypa
         np.testing.assert_allclose(e.S[e.slot[n]].double().numpy(), r["S"][0], rtol=1e-5, atol=1e-5)
         np.testing.assert_array_equal(e.hist[e.slot[n]].numpy(), r["hist"][0])
         assert e.pos[n] == T
+
+
+def oracle_decode(orc):
+    def run(x, W1, W2, q, k, v, g, beta, hist_pool, S_pool, slots):
+        n = lambda t: t.double().numpy()
+        idx = slots.long()
+        r = orc.jetblock_decode(n(x)[None], n(W1), n(W2), n(q)[None], n(k)[None], n(v)[None], n(g)[None],
+                                n(beta)[None], n(S_pool[idx]), n(hist_pool[idx]))
+        S_pool[idx] = torch.from_numpy(r["S"]).to(S_pool.dtype)
+        hist_pool[idx] = torch.from_numpy(r["hist"]).to(hist_pool.dtype)
+        return torch.from_numpy(r["o"][0])
+    return run
+
+
+def test_serving_steps_spend_the_prefill_budget_and_decode_finished_prompts(monkeypatch):
+    import numpy as np
+    import synth
+    from oracle import get as get_oracle
+    orc = get_oracle()
+    calls = []
+    monkeypatch.setattr(eng, "jet_jetblock_prefill", oracle_prefill(orc, calls))
+    monkeypatch.setattr(eng, "jet_jetblock_decode_slots", oracle_decode(orc))
+    monkeypatch.setattr(eng, "jet_jetblock_prefill_workspace_size", lambda *a, **k: 64)
+    shp = synth.JetShape("t", B=1, T=1, H=H, dk=DK, dv=DV, D=D, dtype="f32")
+    lens, dec = {"a": 250, "b": 60}, 3
+    inp = {n: synth.prefill_inputs(shp, seed=50 + i, T=T + dec) for i, (n, T) in enumerate(lens.items())}
+    W1 = torch.from_numpy(inp["a"]["W1"]).double()
+    W2 = torch.from_numpy(inp["a"]["W2"]).double()
+    e = eng.JetEngine(W1, W2, H, DK, DV, max_seqs=2, chunk_tokens=100)
+    t = lambda n, a, b: tuple(torch.from_numpy(np.ascontiguousarray(inp[n][k][0, a:b])).double()
+                              for k in ("x", "q", "k", "v", "g", "beta"))
+    for n, T in lens.items():
+        e.submit(n, t(n, 0, T))
+    outs = {n: [] for n in lens}
+    tok = lambda n, i: tuple(a[0] for a in t(n, i, i + 1))
+    with pytest.raises(ValueError):
+        e.step({"b": tok("b", 60)})                        # b has not finished its prompt: nothing runs
+    assert calls == [] and e.pos == {"a": 0, "b": 0} and float(e.S.abs().sum()) == 0.0
+    plan = [None, None, None, {"a": 250}, {"a": 251, "b": 60}, {"a": 252, "b": 61}, {"b": 62}]
+    for want in plan:
+        r = e.step({n: tok(n, i) for n, i in want.items()} if want else None)
+        for n, o in r.items():
+            outs[n].append(o if o.dim() == 3 else o[None])
+    # prefill budget: a 100 | a 100 | a 50 + b 50 | b 10 (then decode a) | decode | decode | decode b
+    assert calls == [(1, 100), (1, 100), (2, 50), (1, 10)]
+    assert e.prefilling == []
+    for n, T in lens.items():
+        d = {k: inp[n][k].astype(np.float64) for k in ("x", "q", "k", "v", "g", "beta")}
+        r = orc.jetblock_prefill(d["x"], inp["a"]["W1"].astype(np.float64), inp["a"]["W2"].astype(np.float64),
+                                 d["q"], d["k"], d["v"], d["g"], d["beta"])
+        np.testing.assert_allclose(torch.cat(outs[n]).numpy(), r["o"][0], rtol=1e-5, atol=1e-5)
+        assert e.pos[n] == T + dec
