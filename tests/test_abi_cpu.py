@@ -249,3 +249,18 @@ def segments_from_workspace(B, T, H, dk, dv):
 ])
 def test_segment_plan_of_the_stated_shapes(lib, B, T, H, dk, dv, P):
     assert segments_from_workspace(B, T, H, dk, dv) == P
+
+
+@pytest.mark.parametrize("std,lang", [("c99", "c"), ("c++17", "c++")])
+def test_header_is_plain_c(tmp_path, std, lang):
+    # the boundary is a C ABI: the header compiles as strict C99 (and as C++) with no torch or CUDA types
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    src = tmp_path / "use_jet.c"
+    src.write_text('#include "jet.h"\nint main(void) { return (int)jet_launch_count(); }\n')
+    r = subprocess.run([cc, f"-std={std}", "-Wall", "-Wextra", "-Werror", "-pedantic", "-fsyntax-only", "-x", lang,
+                        "-I", os.path.dirname(HEADER), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
