@@ -1,20 +1,31 @@
 #!/usr/bin/env python
 """Benchmark of the JetBlock token mixer on B200.
 
-One step = one serving iteration of the mixer on 2B shapes (H=12, dk=96,
-dv=256, d_model=1536, bf16 inputs, float32 state):
+Headline step (the `value` of the JSON line): one serving iteration of the
+mixer on 2B shapes (H=12, dk=96, dv=256, d_model=1536, bf16 inputs, float32
+state):
   prefill  one jet_jetblock_prefill call over one new 4096-token sequence
-           (zero initial state): the kernel generator (K1 without the conv),
-           then the chunked GDN prefill (K2) with the conv applied to the raw V
-           tiles inside its state chain;
-  decode   generator+conv with history (K1, T=1) and the GDN decode step (K3)
-           for 256 running sequences, one token each; the state advances in
-           place from step to step (64 pre-drawn token sets, cycled).
+           (zero initial state): the kernel generator, then the chunked GDN
+           prefill with the dynamic conv folded into its chunk preparation;
+  decode   generator+conv with history (T=1) and the GDN decode step for 256
+           running sequences, one token each; the state advances in place from
+           step to step (64 pre-drawn token sets, cycled).
 Tokens per step = 4096 + 256. Every rank runs its own copy of this work
 (independent shards, no collective on the data path): weak scaling.
 
+The same line carries the other stated workloads under "configs", each
+timed on the device, end to end from pinned host buffers, against its
+roofline, and beside a bounded sample on the float64 oracle:
+  prefill_4b_t65536   one 65536-token prefill on 4B shapes (H=16, dk=128)
+  prefill_2b_t262144  one 262144-token prefill on 2B shapes
+  decode_2b_after_t262144  256 decode steps at B=1 continuing that prefill
+  decode_4b_b{1,16,64,256,1024}  the 4B decode sweep
+Their inputs use the block-seeded variant of the recipe (synth
+prefill_inputs_blocked / decode_inputs_blocked) so that multi-GB draws take
+seconds.
+
 Prints one JSON line (rank 0). `--impl reference` times the float64 CPU
-oracle on the same workload instead (bounded sample per step).
+oracle on the headline workload instead (bounded sample per step).
 """
 from __future__ import annotations
 
@@ -40,6 +51,8 @@ TOKENS_PER_STEP = PREFILL.B * PREFILL.T + DECODE.B
 METRIC = "JetBlock prefill & decode tokens/s (2B/4B shapes); % of HBM/BF16 roofline"
 WORKLOAD = ("mixed serving step on 2B JetBlock shapes: prefill of one 4096-token sequence "
             "(prefill_2b_t4096) + one decode token for each of 256 sequences (decode_2b_b256)")
+CHUNK = 64
+L2_BYTES = 126 * (1 << 20)
 
 
 def peaks():
@@ -51,30 +64,51 @@ def peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
-# ------------------------------------------------------------------ algorithmic traffic per launch
+# ------------------------------------------------------------------ algorithmic traffic
+def prefill_model(s, B=None, T=None):
+    """Algorithmic bytes and flops of a prefill of B sequences x T tokens.
+    "bytes" is the per-unit count of the scope table: K1 (x, v read, v' written)
+    + K2 (q, k, v', g, beta read, o written, final state written), every input
+    read once and every output written once. "bytes_fused" is the minimum of the
+    one-call form, where v' never leaves the chip."""
+    B = s.B if B is None else B
+    T = s.T if T is None else T
+    e = 2 if s.dtype == "bf16" else 4
+    N = B * T
+    w = (s.D * 32 + 32 * s.H * 4) * e
+    k1 = N * (s.D * e + 2 * s.H * s.dv * e) + w
+    k2 = N * s.H * (2 * s.dk * e + 2 * s.dv * e + 8) + B * s.H * s.dv * s.dk * 4
+    fused = N * (s.D * e + s.H * (2 * s.dk * e + 2 * s.dv * e + 8)) + B * s.H * s.dv * s.dk * 4 + w
+    gen_flops = N * (2 * s.D * 32 + 2 * 32 * s.H * 4 + 8 * s.H * s.dv)
+    gdn_flops = N * s.H * (2 * CHUNK * (3 * s.dk + 2 * s.dv) + 6 * s.dk * s.dv + CHUNK * CHUNK / 3)
+    return dict(bytes=k1 + k2, bytes_fused=fused, flops=gen_flops + gdn_flops,
+                bytes_k1=k1, bytes_k2=k2, flops_k1=gen_flops, flops_k2=gdn_flops)
+
+
+def decode_model(s, B=None):
+    """Algorithmic bytes and flops of one decode step of B sequences: K1 with T=1
+    (x, v read, v' written, history read and written) and K3 (state read and
+    written, token vectors)."""
+    B = s.B if B is None else B
+    e = 2 if s.dtype == "bf16" else 4
+    k1 = B * (s.D * e + 2 * s.H * s.dv * e + 2 * 3 * s.H * s.dv * e) + (s.D * 32 + 32 * s.H * 4) * e
+    k3 = B * s.H * (2 * s.dv * s.dk * 4 + 2 * s.dk * e + 2 * s.dv * e + 8)
+    return dict(bytes=k1 + k3, bytes_k1=k1, bytes_k3=k3,
+                flops=B * (2 * s.D * 32 + 8 * s.H * s.dv) + B * s.H * 7 * s.dk * s.dv,
+                flops_k1=B * (2 * s.D * 32 + 8 * s.H * s.dv), flops_k3=B * s.H * 7 * s.dk * s.dv)
+
+
+def roofline_us(nbytes, flops, pk):
+    return 1e6 * max(nbytes / (pk["hbm_gbs"] * 1e9), flops / (pk["bf16_tflops"] * 1e12))
+
+
 def model_bytes():
-    """Algorithmic HBM bytes (and flops) per launch of each kernel of a step:
-    every input read once, every output written once."""
-    P, Dc = PREFILL, DECODE
-    e = 2  # bf16
-    T = P.B * P.T
-    k1p = T * (P.D * e + 2 * P.H * P.dv * e) + (P.D * 32 + 32 * P.H * 4) * e
-    k2p = (T * P.H * (2 * P.dk * e + 2 * P.dv * e + 8) + P.B * P.H * P.dv * P.dk * 4)
-    C = 64
-    k2p_flops = T * P.H * (2 * C * (3 * P.dk + 2 * P.dv) + 6 * P.dk * P.dv + C * C / 3)
-    k1d = Dc.B * (Dc.D * e + 2 * Dc.H * Dc.dv * e + 2 * 3 * Dc.H * Dc.dv * e) + (Dc.D * 32 + 32 * Dc.H * 4) * e
-    k3d = Dc.B * Dc.H * (2 * Dc.dv * Dc.dk * 4 + 2 * Dc.dk * e + 2 * Dc.dv * e + 8)
-    k3d_flops = Dc.B * Dc.H * 7 * Dc.dk * Dc.dv
-    # generator + conv + GDN in one call: x, q, k, raw v, g, beta read once, o and the
-    # final state written once (v' never leaves the chip); taps are on-chip-sized (4 floats per token and head)
-    kjp = T * (P.D * e + P.H * (2 * P.dk * e + 2 * P.dv * e + 8)) + P.B * P.H * P.dv * P.dk * 4 \
-        + (P.D * 32 + 32 * P.H * 4) * e
+    """Algorithmic bytes (and flops) of each library call of the headline step."""
+    p, d = prefill_model(PREFILL), decode_model(DECODE)
     return {
-        "genconv_prefill": dict(bytes=k1p, flops=T * (2 * P.D * 32 + 2 * 32 * P.H * 4 + 8 * P.H * P.dv)),
-        "gdn_prefill": dict(bytes=k2p, flops=k2p_flops),
-        "jetblock_prefill": dict(bytes=kjp, flops=T * (2 * P.D * 32 + 2 * 32 * P.H * 4 + 8 * P.H * P.dv) + k2p_flops),
-        "genconv_decode": dict(bytes=k1d, flops=Dc.B * (2 * Dc.D * 32 + 8 * Dc.H * Dc.dv)),
-        "gdn_decode": dict(bytes=k3d, flops=k3d_flops),
+        "jetblock_prefill": dict(bytes=p["bytes"], bytes_fused=p["bytes_fused"], flops=p["flops"]),
+        "genconv_decode": dict(bytes=d["bytes_k1"], flops=d["flops_k1"]),
+        "gdn_decode": dict(bytes=d["bytes_k3"], flops=d["flops_k3"]),
     }
 
 
@@ -88,13 +122,13 @@ def csrc_digest(files):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str):
-    """DRAM bytes per launch (read + write) from a committed ncu summary, only
-    if it was taken on the current sources of that kernel."""
+def ncu_traffic(call: str):
+    """DRAM bytes per call (read + write, summed over its launches) from a
+    committed ncu summary, only if it was taken on the current sources."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    ent = json.load(open(p)).get(kernel)
+    ent = json.load(open(p)).get(call)
     if not ent or ent.get("sources_sha") != csrc_digest(ent.get("sources", [])):
         return None
     return ent.get("dram_bytes_per_launch")
@@ -139,43 +173,40 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside)}
 
 
-# ------------------------------------------------------------------ the GPU workload
+def as_torch(a):
+    import torch
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a))
+
+
+# ------------------------------------------------------------------ the headline workload
 class Workload:
     def __init__(self, device, seed: int):
         import torch
         import linear_attention_lm_gen_b200 as jet
         self.torch, self.jet, self.dev = torch, jet, device
-
-        def T(a):
-            if a.dtype == np.uint16:
-                return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
-            return torch.from_numpy(np.ascontiguousarray(a))
-
         p = synth.prefill_inputs(PREFILL, seed=seed)
         d = synth.decode_inputs(DECODE, seed=seed + 1)
-        self.host_p = {k: T(v).pin_memory() for k, v in p.items() if isinstance(v, np.ndarray)}
-        self.host_d = {k: T(v).pin_memory() for k, v in d.items() if isinstance(v, np.ndarray)}
+        self.host_p = {k: as_torch(v).pin_memory() for k, v in p.items() if isinstance(v, np.ndarray)}
+        self.host_d = {k: as_torch(v).pin_memory() for k, v in d.items() if isinstance(v, np.ndarray)}
         # two device copies of the prefill inputs (the end-to-end pass copies the
         # next step's inputs in while the current step runs)
         self.pb = [{k: v.to(device) for k, v in self.host_p.items()} for _ in range(2)]
-        self.p = self.pb[0]
         self.d = {k: v.to(device) for k, v in self.host_d.items()}
         P, Dc = PREFILL, DECODE
         bf = torch.bfloat16
         self.ob = [torch.empty((P.B, P.T, P.H, P.dv), device=device, dtype=bf) for _ in range(2)]
-        self.o = self.ob[0]
         self.S_out = torch.empty((P.B, P.H, P.dv, P.dk), device=device, dtype=torch.float32)
         self.S = self.d["S0"].clone()
         self.hist = [self.d["hist"].clone(), torch.empty_like(self.d["hist"])]
         self.vc_d = torch.empty((Dc.B, 1, Dc.H, Dc.dv), device=device, dtype=bf)
         self.odb = [torch.empty((Dc.B, Dc.H, Dc.dv), device=device, dtype=bf) for _ in range(2)]
-        self.o_d = self.odb[0]
         ws = jet.jet_jetblock_prefill_workspace_size(P.B, P.T, P.H, P.dk, P.dv)
         self.ws = torch.empty(max(ws, 16), device=device, dtype=torch.uint8)
         # pinned host buffers for the end-to-end pass
-        self.h_o = [torch.empty(self.o.shape, dtype=bf).pin_memory() for _ in range(2)]
-        self.h_o_d = [torch.empty(self.o_d.shape, dtype=bf).pin_memory() for _ in range(2)]
-        self.steps_done = 0
+        self.h_o = [torch.empty(self.ob[0].shape, dtype=bf).pin_memory() for _ in range(2)]
+        self.h_o_d = [torch.empty(self.odb[0].shape, dtype=bf).pin_memory() for _ in range(2)]
 
     # the library calls of one step, in order (each timed between two events)
     CALLS = ("jetblock_prefill", "genconv_decode", "gdn_decode")
@@ -190,14 +221,13 @@ class Workload:
             if counts is not None:
                 counts.append(jet.jet_launch_count())
         mark(0)
-        # prefill: generator, then the GDN prefill with the conv inside its chain (one call)
+        # prefill: generator, then the GDN prefill with the conv folded into its chunks (one call)
         jet.jet_jetblock_prefill(p["x"], p["W1"], p["W2"], p["q"], p["k"], p["v"], p["g"], p["beta"], None, None,
                                  None, o, self.S_out, self.ws, stream=stream)
         mark(1)
         s = i % DECODE.steps
         hin, hout = self.hist[i % 2], self.hist[(i + 1) % 2]
-        # decode: generator + conv with the history (T = 1), then the state update. (Folding the conv
-        # into the state pass, jet_conv_gdn_decode_step, measured slower on this step: 127 vs 115 us.)
+        # decode: generator + conv with the history (T = 1), then the state update
         jet.jet_dyn_conv_v(d["x"][s][:, None], d["W1"], d["W2"], d["v"][s][:, None], hin, self.vc_d, hout,
                            stream=stream)
         mark(2)
@@ -225,10 +255,10 @@ class Workload:
         return self.ob[buf].numel() * 2 + self.odb[buf].numel() * 2
 
 
-# ------------------------------------------------------------------ CPU oracle leg
+# ------------------------------------------------------------------ CPU oracle legs
 def oracle_step(orc, p64, d64, frac: float = 1.0, dstep: int = 0):
-    """The workload on the float64 oracle; `frac` < 1 takes the first frac of the
-    prefill tokens and of the decode sequences (same mix). Returns tokens done."""
+    """The headline workload on the float64 oracle; `frac` < 1 takes the first frac
+    of the prefill tokens and of the decode sequences (same mix). Returns tokens done."""
     Tp = max(1, int(round(PREFILL.T * frac)))
     Bd = max(1, int(round(DECODE.B * frac)))
     sl = lambda a: a[:, :Tp]
@@ -241,12 +271,14 @@ def oracle_step(orc, p64, d64, frac: float = 1.0, dstep: int = 0):
     return Tp * PREFILL.B + Bd
 
 
+def f64_inputs(inp):
+    return {k: synth.to_f64(v, inp["dtype"]) if v.dtype == np.uint16 else v.astype(np.float64)
+            for k, v in inp.items() if isinstance(v, np.ndarray)}
+
+
 def oracle_inputs(seed: int):
-    p = synth.prefill_inputs(PREFILL, seed=seed)
-    d = synth.decode_inputs(DECODE, seed=seed + 1)
-    f = lambda inp: {k: synth.to_f64(v, inp["dtype"]) if v.dtype == np.uint16 else v.astype(np.float64)
-                     for k, v in inp.items() if isinstance(v, np.ndarray)}
-    return f(p), f(d)
+    return (f64_inputs(synth.prefill_inputs(PREFILL, seed=seed)),
+            f64_inputs(synth.decode_inputs(DECODE, seed=seed + 1)))
 
 
 def cpu_baseline(seed: int, budget_s: float = 15.0):
@@ -266,12 +298,55 @@ def cpu_baseline(seed: int, budget_s: float = 15.0):
                       f"for each of 256 sequences) on the float64 oracle, {dt:.1f} s"}
 
 
+def cpu_prefill_sample(s, inp, budget_s: float):
+    """The oracle on consecutive 1024-token pieces of sequence 0 of a prefill
+    workload (each piece continues the state and history of the last), until
+    the budget is spent."""
+    import oracle
+    orc = oracle.get()
+    dt_ = inp["dtype"]
+    W1, W2 = synth.to_f64(inp["W1"], dt_), synth.to_f64(inp["W2"], dt_)
+    S, hist, done = None, None, 0
+    t0 = time.perf_counter()
+    while done < s.T and time.perf_counter() - t0 < budget_s:
+        sl = lambda k: synth.to_f64(inp[k][:1, done:done + 1024], dt_) if inp[k].dtype == np.uint16 \
+            else inp[k][:1, done:done + 1024].astype(np.float64)
+        r = orc.jetblock_prefill(sl("x"), W1, W2, sl("q"), sl("k"), sl("v"), sl("g"), sl("beta"), S, hist)
+        S, hist = r["S"], r["hist"]
+        done += sl("x").shape[1]
+    el = time.perf_counter() - t0
+    return {"value": done / el, "unit": "tokens/s", "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"the first {done} tokens of sequence 0 in 1024-token pieces on the float64 oracle, {el:.1f} s"}
+
+
+def cpu_decode_sample(s, inp, budget_s: float, seqs: int = 16):
+    """The oracle on decode steps of the first `seqs` sequences until the budget is spent."""
+    import oracle
+    orc = oracle.get()
+    d = f64_inputs({k: (v[:, :seqs] if k in ("x", "q", "k", "v", "g", "beta") else
+                        (v[:seqs] if k in ("S0", "hist") else v)) if isinstance(v, np.ndarray) else v
+                    for k, v in inp.items()})
+    B = d["x"].shape[1]
+    S, h, n = d["S0"], d["hist"], 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        st = n % d["x"].shape[0]
+        one = lambda a: a[st:st + 1]
+        r = orc.jetblock_decode(one(d["x"]), d["W1"], d["W2"], one(d["q"]), one(d["k"]), one(d["v"]), one(d["g"]),
+                                one(d["beta"]), S, h)
+        S, h = r["S"], r["hist"]
+        n += 1
+    el = time.perf_counter() - t0
+    return {"value": n * B / el, "unit": "tokens/s", "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"{n} decode step(s) of {B} sequence(s) on the float64 oracle, {el:.1f} s"}
+
+
 # ------------------------------------------------------------------ multi-rank plumbing
 class Ranks:
     """One process per GPU (torchrun sets RANK / LOCAL_RANK / WORLD_SIZE). The
     path shards without any exchange: every rank runs the same per-GPU
     workload on its own inputs (weak scaling); the only collectives are the
-    barriers around the timed region and the max over ranks of its duration."""
+    barriers around the timed regions and the max over ranks of their durations."""
 
     def __init__(self, env=None):
         env = os.environ if env is None else env
@@ -327,6 +402,214 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------ the other stated workloads
+class Timer:
+    """Per-step events on one stream, L2 flushed between steps when asked (the
+    flush runs between the events, outside the timed work)."""
+
+    def __init__(self, torch, device, stream, flush: bool):
+        self.torch, self.stream = torch, stream
+        self.scrub = torch.empty(2 * L2_BYTES // 4, device=device, dtype=torch.float32) if flush else None
+
+    def run(self, fn, steps: int, warmup: int):
+        torch = self.torch
+        with torch.cuda.stream(self.stream):
+            for i in range(warmup):
+                fn(i)
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            for i in range(steps):
+                if self.scrub is not None:
+                    self.scrub.fill_(float(i))
+                ev[i][0].record(self.stream)
+                fn(warmup + i)
+                ev[i][1].record(self.stream)
+        self.stream.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]          # ms per step
+
+
+def host_pinned(inp, keys):
+    return {k: as_torch(inp[k]).pin_memory() for k in keys}
+
+
+def measure_prefill_config(ctx, name: str, steps: int, warmup: int, keep: bool = False):
+    """One jet_jetblock_prefill call over the whole prompt per step."""
+    torch, jet, dev, stream, rk, pk = ctx["torch"], ctx["jet"], ctx["dev"], ctx["stream"], ctx["rk"], ctx["pk"]
+    s = synth.CONFIGS[name]
+    inp = synth.prefill_inputs_blocked(s, seed=ctx["seed"])
+    keys = ("x", "q", "k", "v", "g", "beta")
+    host = host_pinned(inp, keys + ("W1", "W2"))
+    d = {k: v.to(dev) for k, v in host.items()}
+    o = torch.empty((s.B, s.T, s.H, s.dv), device=dev, dtype=torch.bfloat16)
+    S = torch.empty((s.B, s.H, s.dv, s.dk), device=dev, dtype=torch.float32)
+    hist = torch.empty((s.B, 3, s.H, s.dv), device=dev, dtype=torch.bfloat16)
+    ws = torch.empty(max(16, jet.jet_jetblock_prefill_workspace_size(s.B, s.T, s.H, s.dk, s.dv)), device=dev,
+                     dtype=torch.uint8)
+    call = lambda i: jet.jet_jetblock_prefill(d["x"], d["W1"], d["W2"], d["q"], d["k"], d["v"], d["g"], d["beta"],
+                                              None, hist, None, o, S, ws, stream=stream)
+    ctx["barrier"]()
+    ms = Timer(torch, dev, stream, flush=False).run(call, steps, warmup)      # inputs are GBs: larger than L2
+    t = rk.max_over_ranks(statistics.median(ms), dev)
+    # end to end: the step's inputs copied in from pinned memory and o read back, every step
+    h_o = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+    d2h = o.numel() * 2
+
+    def e2e(i):
+        for k in keys:
+            d[k].copy_(host[k], non_blocking=True)
+        call(i)
+        h_o.copy_(o, non_blocking=True)
+    ctx["barrier"]()
+    e_ms = rk.max_over_ranks(statistics.median(Timer(torch, dev, stream, False).run(e2e, max(2, steps // 2), 1)),
+                             dev)
+    m = prefill_model(s)
+    tok = s.B * s.T
+    r_us = roofline_us(m["bytes"], m["flops"], pk)
+    out = {"workload": f"one jet_jetblock_prefill call over {s.B} x {s.T} tokens (H={s.H}, dk={s.dk}, dv={s.dv}, "
+                       f"d_model={s.D}, bf16, float32 state, zero initial state)",
+           "tokens_per_s": rk.world * tok / (t * 1e-3), "us_per_call": t * 1e3, "steps": steps, "warmup": warmup,
+           "l2": "inputs larger than L2 (no flush needed)",
+           "roofline": {"bound": "hbm" if m["bytes"] / pk["hbm_gbs"] > m["flops"] / (pk["bf16_tflops"] * 1e3)
+                        else "tensor", "algorithmic_bytes": m["bytes"], "algorithmic_flops": m["flops"],
+                        "achieved": m["bytes"] / (t * 1e-3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "roofline_us": r_us, "frac": r_us / (t * 1e3),
+                        "frac_vs_fused_bytes": 1e6 * m["bytes_fused"] / (pk["hbm_gbs"] * 1e9) / (t * 1e3)},
+           "e2e": {"value": rk.world * tok / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                   "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}}
+    kept = dict(S=S, hist=hist, W1=d["W1"], W2=d["W2"]) if keep else None
+    del d, o, ws
+    return out, inp, kept
+
+
+def measure_decode_after(ctx, name: str, kept, reps: int):
+    """s.steps decode steps at B=1 continuing the long prefill (its state and
+    history), jet_jetblock_decode_step per step, captured once in a CUDA graph
+    and replayed; a replay is one timed iteration (L2 flushed between replays)."""
+    torch, jet, dev, stream, rk, pk = ctx["torch"], ctx["jet"], ctx["dev"], ctx["stream"], ctx["rk"], ctx["pk"]
+    s = synth.CONFIGS[name]
+    n = s.steps
+    inp = synth.decode_inputs_blocked(s.with_(B=1), seed=ctx["seed"] + 5, steps=n)
+    keys = ("x", "q", "k", "v", "g", "beta")
+    host = host_pinned(inp, keys)
+    d = {k: v.to(dev) for k, v in host.items()}
+    S, W1, W2 = kept["S"], kept["W1"], kept["W2"]
+    hb = [kept["hist"], torch.empty_like(kept["hist"])]
+    o = torch.empty((n, 1, s.H, s.dv), device=dev, dtype=torch.bfloat16)
+    taps = torch.empty((n, 1, s.H, 4), device=dev, dtype=torch.float32)
+
+    def steps_fn():
+        for t in range(n):
+            jet.jet_jetblock_decode_step(d["x"][t], W1, W2, d["q"][t], d["k"][t], d["v"][t], hb[t % 2],
+                                         hb[(t + 1) % 2], d["g"][t], d["beta"][t], S, o[t], taps[t], stream=stream)
+    with torch.cuda.stream(stream):
+        steps_fn()                                   # warm-up outside the graph
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        steps_fn()
+    ctx["barrier"]()
+    ms = Timer(torch, dev, stream, flush=True).run(lambda i: graph.replay(), reps, 3)
+    t = rk.max_over_ranks(statistics.median(ms), dev)
+    h_o = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+
+    def e2e(i):
+        for k in keys:
+            d[k].copy_(host[k], non_blocking=True)
+        graph.replay()
+        h_o.copy_(o, non_blocking=True)
+    e_ms = rk.max_over_ranks(statistics.median(Timer(torch, dev, stream, True).run(e2e, max(2, reps // 2), 1)), dev)
+    del graph
+    m = decode_model(s, 1)
+    us_step = t * 1e3 / n
+    r_us = roofline_us(m["bytes"], m["flops"], pk)
+    return {"workload": f"{n} decode steps at B=1 (2 launches each: generator, then conv + history shift + update "
+                        f"in one pass over S) continuing the {s.T}-token prefill, as one CUDA graph",
+            "tokens_per_s": rk.world * n / (t * 1e-3), "us_per_step": us_step, "replays": reps,
+            "l2": "flushed between replays; within a replay the 1.2 MB state stays in L2 from step to step",
+            "roofline": {"bound": "hbm", "algorithmic_bytes_per_step": m["bytes"], "roofline_us_per_step": r_us,
+                         "frac": r_us / us_step, "achieved": m["bytes"] / (us_step * 1e-6) / 1e9,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "note": "launch-latency bound: 2.4 MB per step is 0.37 us of HBM time"},
+            "e2e": {"value": rk.world * n / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": o.numel() * 2, "ms_per_step": e_ms}}, inp
+
+
+def measure_decode_config(ctx, name: str, steps: int, warmup: int, token_sets: int = 8):
+    """One decode step for every sequence per step: the generator + conv launch
+    (T=1, with history) and the state update, the two calls of the headline step."""
+    torch, jet, dev, stream, rk, pk = ctx["torch"], ctx["jet"], ctx["dev"], ctx["stream"], ctx["rk"], ctx["pk"]
+    s = synth.CONFIGS[name]
+    inp = synth.decode_inputs_blocked(s, seed=ctx["seed"] + 3, steps=token_sets)
+    keys = ("x", "q", "k", "v", "g", "beta")
+    host = host_pinned(inp, keys + ("W1", "W2", "S0", "hist"))
+    d = {k: v.to(dev) for k, v in host.items()}
+    S = d["S0"]
+    hb = [d["hist"], torch.empty_like(d["hist"])]
+    vc = torch.empty((s.B, 1, s.H, s.dv), device=dev, dtype=torch.bfloat16)
+    o = torch.empty((s.B, s.H, s.dv), device=dev, dtype=torch.bfloat16)
+
+    def call(i):
+        st = i % token_sets
+        jet.jet_dyn_conv_v(d["x"][st][:, None], d["W1"], d["W2"], d["v"][st][:, None], hb[i % 2], vc, hb[(i + 1) % 2],
+                           stream=stream)
+        jet.jet_gdn_decode_step(d["q"][st], d["k"][st], vc[:, 0], d["g"][st], d["beta"][st], S, o, stream=stream)
+    m = decode_model(s)
+    flush = m["bytes"] < L2_BYTES
+    ctx["barrier"]()
+    ms = Timer(torch, dev, stream, flush=flush).run(call, steps, warmup)
+    t = rk.max_over_ranks(statistics.median(ms), dev)
+    h_o = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+
+    def e2e(i):
+        st = i % token_sets
+        for k in keys:
+            d[k][st].copy_(host[k][st], non_blocking=True)
+        call(i)
+        h_o.copy_(o, non_blocking=True)
+    e_ms = rk.max_over_ranks(statistics.median(Timer(torch, dev, stream, flush).run(e2e, max(3, steps // 2), 2)), dev)
+    h2d = sum(host[k][0].numel() * host[k][0].element_size() for k in keys)
+    r_us = roofline_us(m["bytes"], m["flops"], pk)
+    del d, S, hb
+    return {"workload": f"one decode token for each of {s.B} sequences on 4B shapes (H={s.H}, dk={s.dk}, "
+                        f"dv={s.dv}, d_model={s.D}); generator + conv launch, then the state update",
+            "tokens_per_s": rk.world * s.B / (t * 1e-3), "us_per_step": t * 1e3, "steps": steps, "warmup": warmup,
+            "l2": "flushed between steps" if flush else "state larger than L2 (no flush needed)",
+            "roofline": {"bound": "hbm", "algorithmic_bytes": m["bytes"], "roofline_us": r_us,
+                         "achieved": m["bytes"] / (t * 1e-3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": r_us / (t * 1e3)},
+            "e2e": {"value": rk.world * s.B / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": o.numel() * 2, "ms_per_step": e_ms}}, inp
+
+
+def run_configs(ctx, args):
+    out = {}
+    cpu = not args.no_cpu_baseline and ctx["rk"].rank == 0
+    budget = args.cpu_budget_config
+    for name in ("prefill_4b_t65536", "prefill_2b_t262144"):
+        long_ = name == "prefill_2b_t262144"
+        r, inp, kept = measure_prefill_config(ctx, name, steps=5 if long_ else 10, warmup=3, keep=long_)
+        if cpu:
+            r["cpu_baseline"] = cpu_prefill_sample(synth.CONFIGS[name], inp, budget)
+        out[name] = r
+        del inp
+        if long_:
+            r, dinp = measure_decode_after(ctx, name, kept, reps=5)
+            if cpu:
+                r["cpu_baseline"] = cpu_decode_sample(synth.CONFIGS[name].with_(B=1), dinp, budget, seqs=1)
+            out["decode_2b_after_t262144"] = r
+            del kept
+        ctx["torch"].cuda.empty_cache()
+    for b in (1, 16, 64, 256, 1024):
+        name = f"decode_4b_b{b}"
+        r, inp = measure_decode_config(ctx, name, steps=20, warmup=3)
+        if cpu:
+            r["cpu_baseline"] = cpu_decode_sample(synth.CONFIGS[name], inp, budget / 3)
+        out[name] = r
+        ctx["torch"].cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------ main GPU arm
 def run_jet(args):
     import torch
@@ -365,7 +648,7 @@ def run_jet(args):
     if jet.jet_device_error(stream) != 0:
         raise RuntimeError("device error word set after warm-up")
 
-    # ---- device-resident timed pass (per-kernel events inside it)
+    # ---- device-resident timed pass (per-call events inside it)
     ncall = len(Workload.CALLS)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(ncall + 1)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -384,11 +667,11 @@ def run_jet(args):
     launches = jet.jet_launch_count() - n0
     clk = clocks.stop(t_wall0, t_wall1)
     ms = max_over_ranks(start.elapsed_time(stop))
-    per_kernel = np.zeros(ncall)
+    per_call = np.zeros(ncall)
     for e in evs:
         for j in range(ncall):
-            per_kernel[j] += e[j].elapsed_time(e[j + 1])
-    per_kernel /= args.steps                      # ms per launch
+            per_call[j] += e[j].elapsed_time(e[j + 1])
+    per_call /= args.steps                      # ms per call
     if jet.jet_device_error(stream) != 0:
         raise RuntimeError("device error word set in the timed region")
 
@@ -427,6 +710,14 @@ def run_jet(args):
     e_stop.record(stream)
     barrier()
     e_ms = max_over_ranks(e_start.elapsed_time(e_stop))
+    del wl
+
+    pk = peaks()
+    configs = None
+    if not args.no_configs:
+        ctx = dict(torch=torch, jet=jet, dev=device, stream=stream, rk=rk, pk=pk, seed=rk.seed(args.seed + 100),
+                   barrier=barrier)
+        configs = run_configs(ctx, args)
 
     if world > 1:
         dist.barrier()
@@ -434,57 +725,65 @@ def run_jet(args):
     if rank != 0:
         return 0
 
-    pk = peaks()
     mb = model_bytes()
     names = list(Workload.CALLS)
-    kern = {}
+    calls = {}
     for j, n in enumerate(names):
-        t = per_kernel[j] * 1e-3
+        t = per_call[j] * 1e-3
         gbs = mb[n]["bytes"] / t / 1e9
-        kern[n] = {"us_per_launch": per_kernel[j] * 1e3, "kernels_per_call": int(per_call_launches[j]),
-                   "us_per_kernel_avg": per_kernel[j] * 1e3 / max(1, int(per_call_launches[j])),
-                   "algorithmic_bytes": mb[n]["bytes"],
-                   "algorithmic_flops": mb[n]["flops"], "achieved_gbs": gbs, "hbm_frac": gbs / pk["hbm_gbs"],
-                   "roofline_us": 1e6 * max(mb[n]["bytes"] / (pk["hbm_gbs"] * 1e9),
-                                            mb[n]["flops"] / (pk["bf16_tflops"] * 1e12))}
-    # dominant kernel: the call with the longest average kernel (a call of one
-    # launch is one kernel; the ncu launch list under profiles/ confirms it)
-    dom = names[int(np.argmax(per_kernel / np.maximum(per_call_launches, 1)))]
-    ach = kern[dom]["achieved_gbs"]
-    tokens = TOKENS_PER_STEP * world
+        r_us = roofline_us(mb[n]["bytes"], mb[n]["flops"], pk)
+        calls[n] = {"us_per_call": per_call[j] * 1e3, "kernels_per_call": int(per_call_launches[j]),
+                    "algorithmic_bytes": mb[n]["bytes"], "algorithmic_flops": mb[n]["flops"], "achieved_gbs": gbs,
+                    "hbm_frac": gbs / pk["hbm_gbs"], "roofline_us": r_us, "roofline_frac": r_us / (per_call[j] * 1e3)}
+    calls["jetblock_prefill"]["algorithmic_bytes_fused"] = mb["jetblock_prefill"]["bytes_fused"]
+    calls["jetblock_prefill"]["roofline_frac_vs_fused_bytes"] = \
+        roofline_us(mb["jetblock_prefill"]["bytes_fused"], 0, pk) / (per_call[0] * 1e3)
+    # the headline roofline is that of the call with the largest share of the step
+    dom = names[int(np.argmax(per_call))]
     value = rk.value(TOKENS_PER_STEP, args.steps, ms)
-    prefill_ms = per_kernel[0]
-    decode_ms = per_kernel[1] + per_kernel[2]
-    roof_step_us = sum(k["roofline_us"] for k in kern.values())
+    prefill_ms = per_call[0]
+    decode_ms = per_call[1] + per_call[2]
+    roof_step_us = sum(c["roofline_us"] for c in calls.values())
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded numpy PCG64; shapes of the 2B JetBlock)",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded numpy PCG64; shapes of the 2B/4B JetBlock)",
         "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": TOKENS_PER_STEP,
                    "prefill": {"B": PREFILL.B, "T": PREFILL.T, "H": PREFILL.H, "dk": PREFILL.dk, "dv": PREFILL.dv,
-                               "d_model": PREFILL.D, "chunk": 64, "initial_state": "zero"},
+                               "d_model": PREFILL.D, "chunk": CHUNK, "initial_state": "zero"},
                    "decode": {"B": DECODE.B, "H": DECODE.H, "dk": DECODE.dk, "dv": DECODE.dv, "d_model": DECODE.D,
                               "state": "float32, advanced in place every step", "token_sets": DECODE.steps},
                    "l2": "inputs larger than L2: 608 MB of decode state streamed per step (L2 126 MB)",
                    "parallelism": f"dp{world} (independent shard per GPU, no collective on the data path)"},
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": ach / pk["hbm_gbs"], "traffic": ncu_traffic(dom),
-                     "peak_source": f"{pk['source']} (MEASURED_PEAKS.json hbm_gbs, burst copy)"},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": calls[dom]["achieved_gbs"], "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": calls[dom]["hbm_frac"], "traffic": ncu_traffic(dom),
+                     "peak_source": f"{pk['source']} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
+                     "note": "the call with the largest share of the step; achieved = the scope table's "
+                             "algorithmic bytes of the call / its event time"},
+        "roofline_by_phase": {
+            "prefill": {"call": "jetblock_prefill", "frac": calls["jetblock_prefill"]["roofline_frac"],
+                        "frac_vs_fused_bytes": calls["jetblock_prefill"]["roofline_frac_vs_fused_bytes"]},
+            "decode": {"calls": ["genconv_decode", "gdn_decode"],
+                       "frac": (calls["genconv_decode"]["roofline_us"] + calls["gdn_decode"]["roofline_us"])
+                       / (decode_ms * 1e3),
+                       "gdn_decode_kernel_frac": calls["gdn_decode"]["roofline_frac"]}},
         "step_roofline": {"roofline_us": roof_step_us, "measured_us": 1e3 * ms / args.steps,
                           "frac": roof_step_us / (1e3 * ms / args.steps)},
         "phases": {
             "prefill": {"tokens_per_s": PREFILL.T / (prefill_ms * 1e-3), "us": prefill_ms * 1e3,
-                        "roofline_us": kern["jetblock_prefill"]["roofline_us"]},
+                        "roofline_us": calls["jetblock_prefill"]["roofline_us"]},
             "decode": {"tokens_per_s": DECODE.B / (decode_ms * 1e-3), "us": decode_ms * 1e3,
-                       "roofline_us": kern["genconv_decode"]["roofline_us"] + kern["gdn_decode"]["roofline_us"]}},
-        "kernels": kern,
+                       "roofline_us": calls["genconv_decode"]["roofline_us"] + calls["gdn_decode"]["roofline_us"]}},
+        "calls": calls,
         "gpu_launches": int(launches),
         "clocks": clk,
-        "e2e": {"value": tokens * args.steps / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps},
+        "e2e": {"value": TOKENS_PER_STEP * world * args.steps / (e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps},
     }
     for ph in line["phases"].values():
         ph["roofline_frac"] = ph["roofline_us"] / ph["us"]
+    if configs is not None:
+        line["configs"] = configs
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.seed, args.cpu_budget)
     print(json.dumps(line), flush=True)
@@ -499,7 +798,9 @@ def main():
     ap.add_argument("--impl", default="jet", choices=["jet", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="time the headline step only")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--cpu-budget-config", type=float, default=3.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)        # at least 3 untimed warm-up steps
     if args.impl == "reference":

@@ -158,7 +158,9 @@ jet_status jet_jetblock_prefill(const void* x, const void* w1, const void* w2,
                                 int hidden, int width, int chunk, jet_dtype dt, void* stream);
 
 /*
- * One decode step (step 3 for a single new token per sequence), updating S in place:
+ * One decode step (step 3 for a single new token per sequence; paper section
+ * 2.3, the gated delta rule applied to one token; section 2.5, finding 4:
+ * decode cost is set by the state's size), updating S in place:
  *   u = S k,  S' = a S + (b v - a b u) k^T,  o = S' q.
  *   q, k [B,H,dk]; v [B,H,dv] (v' of the new token); g, beta [B,H] float32;
  *   S [B,H,dv,dk] float32 in/out; o [B,H,dv] out.
@@ -253,7 +255,10 @@ jet_status jet_jetblock_decode_slots(const void* x, const void* w1, const void* 
  * length (12.5 MB), 16-head dk = 128 shapes longer than 1792 tokens do not
  * (18.0 MB).
  * The first call on a device looks the array's device address up (no
- * allocation); make that first call before any stream capture. The array is
+ * allocation) and caches it with the device's current context; the lookup is
+ * repeated when that context changes (e.g. after cudaDeviceReset), so make
+ * the first call, and the first after such a reset, before any stream
+ * capture. The array is
  * shared by all calls on a device and keeps the last call's contents (every
  * element a call reads is written by that call first): calls whose work
  * overlaps on the GPU, e.g. on two streams, race on it and must be ordered

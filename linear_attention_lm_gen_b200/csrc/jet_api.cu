@@ -102,6 +102,9 @@ jet_status launch_genconv(const void* x, const void* w1, const void* w2, const v
                           void* vout, void* hout, float* cw, int B, int Tn, int D, int H, int dv,
                           cudaStream_t s, const int* slots = nullptr, int n_slots = 0) {
     constexpr int TB = 16;
+    // a state-cache slot index applies to one token per sequence only (the
+    // one-token work items look the slot up per item)
+    if (slots && Tn != 1) return JET_ERR_UNSUPPORTED;
     const long long nblk = ((long long)B * Tn + TB - 1) / TB;
     // head groups (= cluster size, at most 8): enough CTAs to cover the SMs
     // about twice, then as few groups as give every group a head
@@ -109,7 +112,7 @@ jet_status launch_genconv(const void* x, const void* w1, const void* w2, const v
     while (groups < H && groups < 8 && nblk * groups < 296) ++groups;
     const int hpc = (H + groups - 1) / groups;
     groups = (H + hpc - 1) / hpc;
-    if (Tn >= 8)
+    if (Tn >= 8)   // (no slots here: checked above)
         return launch_genconv_t<T, TB, 8>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, groups, hpc, s,
                                           nullptr, 0);
     return launch_genconv_t<T, TB, 1>(x, w1, w2, v, hin, vout, hout, cw, B, Tn, D, H, dv, groups, hpc, s, slots,
@@ -619,20 +622,47 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[JET_NOALLOC_SCR
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+// per device: the context the address was looked up in, and the address
+struct NoallocEntry { void* ctx; void* ptr; };
+NoallocEntry g_noalloc[kMaxDevices] = {};
 
-// device address of the scratch array on the current device (looked up once)
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (CtxGetCurrentFn) nullptr;
+        return (CtxGetCurrentFn)p;
+    }();
+    return fn;
+}
+
+// Device address of the scratch array in the current device's current
+// context. The address belongs to the context the module was loaded into, so
+// it is cached together with that context and looked up again when the
+// context changes (e.g. after cudaDeviceReset made a new primary context).
 jet_status noalloc_scratch(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return JET_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return JET_ERR_UNSUPPORTED;
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (!get_ctx) return JET_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return JET_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    NoallocEntry& e = g_noalloc[dev];
+    if (ctx == nullptr || e.ptr == nullptr || e.ctx != (void*)ctx) {
+        // set-up on this device: the lookup also makes the runtime's primary
+        // context current if no context was yet (no allocation either way)
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return JET_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return JET_ERR_CUDA;
+        e.ctx = (void*)ctx;
+        e.ptr = p;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = e.ptr;
     return JET_OK;
 }
 }  // namespace

@@ -136,7 +136,8 @@ __device__ __forceinline__ void gen_stageA_bf16(const __nv_bfloat16* __restrict_
 // sequence) still spread over many SMs.
 // RUN = tokens per conv work item (8 keeps a sliding window in registers;
 // 1 makes every token an independent item with its 4 loads in flight).
-// slots (T = 1 only): sequence b's history is entry slots[b] of hist_in /
+// slots (T = 1 and RUN = 1 only; the launcher refuses anything else, and the
+// kernel ignores slots when RUN > 1): sequence b's history is entry slots[b] of hist_in /
 // hist_out, which may then be the same pool: each history element is read
 // and rewritten by the one thread that owns its item. An index outside
 // [0, n_slots) sets the device error word and the item is skipped.
@@ -193,7 +194,7 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
         gi.bseq = (int)(gi.rr0 / Tn);               // one division per item; then stepped
         gi.tpos0 = (int)(gi.rr0 - (long long)gi.bseq * Tn);
         gi.hseq = gi.bseq;                          // history entry of the sequence
-        if (slots) {
+        if (RUN == 1 && slots) {                    // slots only with one token per item (never crosses a sequence)
             gi.hseq = slots[gi.bseq];
             if (gi.hseq < 0 || gi.hseq >= n_slots) {
                 flag_error(DEVERR_DATA);
@@ -246,7 +247,7 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
 #pragma unroll
             for (int e = 0; e < VN; ++e) { win[2][e] = win[1][e]; win[1][e] = win[0][e]; win[0][e] = cv[e]; }
             if (hist_out && tpos == Tn - 1) {
-                const long long hq = slots ? gi.hseq : bseq;
+                const long long hq = (RUN == 1 && slots) ? gi.hseq : bseq;
 #pragma unroll
                 for (int j = 0; j < 3; ++j)
                     *reinterpret_cast<uint4*>(hist_out + (hq * 3 + (2 - j)) * rowstride + coff) = V16::pack(win[j]);

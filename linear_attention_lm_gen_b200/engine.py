@@ -138,6 +138,10 @@ class JetEngine:
     def submit(self, seq, prompt) -> None:
         """Queue a prompt (x, q, k, v, g, beta as for prefill); the sequence is
         admitted now, so the cache must have a free entry."""
+        if len(prompt) != 6 or prompt[0].shape[0] == 0:
+            raise ValueError("a prompt is (x, q, k, v, g, beta) of at least one token")
+        if any(a.shape[0] != prompt[0].shape[0] for a in prompt):
+            raise ValueError("the arrays of a prompt must have the same number of tokens")
         self.admit(seq)
         self._queue.append([seq, prompt, 0])
 
@@ -161,8 +165,12 @@ class JetEngine:
             took[seq] = n
             budget -= n
         still = {seq for seq, prompt, done in self._queue if done + took.get(seq, 0) < prompt[0].shape[0]}
+        # every check comes before any work is issued
+        unknown = [sq for sq in (tokens or ()) if sq not in self.slot]
+        if unknown:
+            raise KeyError(f"decode tokens for sequences that are not admitted: {sorted(map(str, unknown))}")
         busy = still & set(tokens or ())
-        if busy:                                   # checked before any work is issued
+        if busy:
             raise ValueError(f"sequences still in prefill: {sorted(map(str, busy))}")
         out = self.prefill_many(work) if work else {}
         for item in self._queue:
@@ -181,6 +189,9 @@ class JetEngine:
         q, k [B,H,dk], v [B,H,dv] (raw), g, beta [B,H]. Returns o [B,H,dv]."""
         if len(set(seqs)) != len(seqs):
             raise ValueError("a sequence appears twice in one decode batch")
+        unknown = [sq for sq in seqs if sq not in self.slot]
+        if unknown:
+            raise KeyError(f"sequences that are not admitted: {sorted(map(str, unknown))}")
         slots = torch.tensor([self.slot[s] for s in seqs], dtype=torch.int32).to(self.S.device, non_blocking=True)
         o = jet_jetblock_decode_slots(x, self.W1, self.W2, q, k, v, g, beta, self.hist, self.S, slots)
         for s in seqs:

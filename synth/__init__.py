@@ -11,6 +11,9 @@ from .jetblock import (  # noqa: F401
     bf16_bits_from_f64,
     bf16_bits_to_f64,
     prefill_inputs,
+    prefill_inputs_blocked,
     decode_inputs,
+    decode_inputs_blocked,
+    spread_qk_norms,
     to_f64,
 )

@@ -115,6 +115,22 @@ def _draw(rng, shape, dtype: str, scale: float = 1.0, unit_last: bool = False):
     return out.reshape(shape)
 
 
+def spread_qk_norms(a: np.ndarray, dtype: str, seed: int, zero_rows=()) -> np.ndarray:
+    """Rescale every row (last axis) of a stored q or k array by 10**U(-1, 1),
+    drawn from a generator of its own (PCG64 seeded with [seed, 7]), so the
+    main input stream is unchanged; then set the rows at the index tuples
+    `zero_rows` (over the leading axes) to exactly zero. Returns a new array
+    in the same storage dtype. These inputs exercise the in-kernel L2
+    normalisation, including the eps under the square root."""
+    rng = np.random.Generator(np.random.PCG64([seed, 7]))
+    lead = a.shape[:-1]
+    s = 10.0 ** rng.uniform(-1.0, 1.0, size=lead + (1,))
+    b = to_f64(a, dtype) * s
+    for idx in zero_rows:
+        b[tuple(idx)] = 0.0
+    return _store(b, dtype)
+
+
 def _gates(rng, shape, gate_scale: float):
     beta_raw = rng.standard_normal(shape)
     g_raw = rng.standard_normal(shape)
@@ -169,5 +185,91 @@ def decode_inputs(shape: JetShape, seed: int = 0, steps: int | None = None,
     out["W2"] = _draw(rng, (shape.R, H * shape.W), dt, scale=1.0 / np.sqrt(shape.R))
     out["S0"] = _draw(rng, (B, H, dv, dk), "f32", scale=state_std)
     out["hist"] = _draw(rng, (B, shape.W - 1, H, dv), dt)
+    out["dtype"] = dt
+    return out
+
+
+# --------------------------------------------------------------------------
+# block-seeded variant (benchmark inputs of the long configurations)
+# --------------------------------------------------------------------------
+def _pool_map(fn, n: int, threads: int | None):
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    threads = threads or max(1, min(32, len(os.sched_getaffinity(0))))
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(fn, range(n)))
+
+
+def prefill_inputs_blocked(shape: JetShape, seed: int = 0, T: int | None = None, block: int = 4096,
+                           threads: int | None = None, gate_scale: float = 1.0) -> dict:
+    """The prefill recipe of prefill_inputs (same arrays, layouts and
+    distributions), with the token axis drawn in blocks of `block` tokens:
+    block i of every token tensor comes from PCG64([seed, 1, i]), in the order
+    x, q, k, v, beta_raw, g_raw; the weights come from PCG64([seed, 2]).
+    Blocks are drawn in parallel threads (numpy releases the GIL while it
+    draws), so multi-GB inputs take seconds. A different stream from
+    prefill_inputs: the two are not interchangeable for stored values."""
+    T = shape.T if T is None else T
+    B, H, dk, dv, D, dt = shape.B, shape.H, shape.dk, shape.dv, shape.D, shape.dtype
+    od = _out_dtype(dt)
+    out = {"x": np.empty((B, T, D), od), "q": np.empty((B, T, H, dk), od), "k": np.empty((B, T, H, dk), od),
+           "v": np.empty((B, T, H, dv), od), "beta": np.empty((B, T, H), np.float32),
+           "g": np.empty((B, T, H), np.float32)}
+    nblk = (T + block - 1) // block
+
+    def one(j):
+        b, i = divmod(j, nblk)
+        t0, t1 = i * block, min(T, (i + 1) * block)
+        rng = np.random.Generator(np.random.PCG64([seed, 1, b, i]))
+        n = t1 - t0
+        out["x"][b, t0:t1] = _draw(rng, (n, D), dt)
+        out["q"][b, t0:t1] = _draw(rng, (n, H, dk), dt, unit_last=True)
+        out["k"][b, t0:t1] = _draw(rng, (n, H, dk), dt, unit_last=True)
+        out["v"][b, t0:t1] = _draw(rng, (n, H, dv), dt)
+        out["beta"][b, t0:t1], out["g"][b, t0:t1] = _gates(rng, (n, H), gate_scale)
+
+    _pool_map(one, B * nblk, threads)
+    rng = np.random.Generator(np.random.PCG64([seed, 2]))
+    out["W1"] = _draw(rng, (D, shape.R), dt, scale=1.0 / np.sqrt(D))
+    out["W2"] = _draw(rng, (shape.R, H * shape.W), dt, scale=1.0 / np.sqrt(shape.R))
+    out["dtype"] = dt
+    return out
+
+
+def decode_inputs_blocked(shape: JetShape, seed: int = 0, steps: int | None = None, state_std: float = 0.02,
+                          block: int = 16, threads: int | None = None, gate_scale: float = 1.0) -> dict:
+    """The decode recipe of decode_inputs (same arrays and distributions),
+    drawn in parallel: the token tensors of step s from PCG64([seed, 3, s]);
+    the state and history of sequences [i*block, (i+1)*block) from
+    PCG64([seed, 4, i]); the weights from PCG64([seed, 2])."""
+    n = shape.steps if steps is None else steps
+    B, H, dk, dv, D, dt = shape.B, shape.H, shape.dk, shape.dv, shape.D, shape.dtype
+    od = _out_dtype(dt)
+    out = {"x": np.empty((n, B, D), od), "q": np.empty((n, B, H, dk), od), "k": np.empty((n, B, H, dk), od),
+           "v": np.empty((n, B, H, dv), od), "beta": np.empty((n, B, H), np.float32),
+           "g": np.empty((n, B, H), np.float32), "S0": np.empty((B, H, dv, dk), np.float32),
+           "hist": np.empty((B, shape.W - 1, H, dv), od)}
+
+    def tok(s):
+        rng = np.random.Generator(np.random.PCG64([seed, 3, s]))
+        out["x"][s] = _draw(rng, (B, D), dt)
+        out["q"][s] = _draw(rng, (B, H, dk), dt, unit_last=True)
+        out["k"][s] = _draw(rng, (B, H, dk), dt, unit_last=True)
+        out["v"][s] = _draw(rng, (B, H, dv), dt)
+        out["beta"][s], out["g"][s] = _gates(rng, (B, H), gate_scale)
+
+    nsb = (B + block - 1) // block
+
+    def st(i):
+        b0, b1 = i * block, min(B, (i + 1) * block)
+        rng = np.random.Generator(np.random.PCG64([seed, 4, i]))
+        out["S0"][b0:b1] = _draw(rng, (b1 - b0, H, dv, dk), "f32", scale=state_std)
+        out["hist"][b0:b1] = _draw(rng, (b1 - b0, shape.W - 1, H, dv), dt)
+
+    _pool_map(tok, n, threads)
+    _pool_map(st, nsb, threads)
+    rng = np.random.Generator(np.random.PCG64([seed, 2]))
+    out["W1"] = _draw(rng, (D, shape.R), dt, scale=1.0 / np.sqrt(D))
+    out["W2"] = _draw(rng, (shape.R, H * shape.W), dt, scale=1.0 / np.sqrt(shape.R))
     out["dtype"] = dt
     return out

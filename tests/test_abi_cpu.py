@@ -264,3 +264,19 @@ def test_header_is_plain_c(tmp_path, std, lang):
     r = subprocess.run([cc, f"-std={std}", "-Wall", "-Wextra", "-Werror", "-pedantic", "-fsyntax-only", "-x", lang,
                         "-I", os.path.dirname(HEADER), str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_noalloc_prefill_refuses_sizes_beyond_its_scratch(lib):
+    # 16 heads, dk = 128, 65536 tokens: even the smallest plan's segment buffers (~18.0 MB)
+    # exceed the 16 MiB array; the check is on the host and comes before any CUDA call
+    TOO_LARGE = 8
+    B, T, H, dk, dv = 1, 65536, 16, 128, 256
+    assert jet.jet_gdn_prefill_workspace_min(B, T, H, dk, dv) > jet.NOALLOC_SCRATCH_BYTES
+    st = lib.jet_gdn_prefill_noalloc(P(A), P(A), P(A), P(A), P(A), None, P(A), P(A), B, T, H, dk, dv, 64, BF16, None)
+    assert st == TOO_LARGE
+    assert jet.jet_status_string(st) == "JET_ERR_TOO_LARGE"
+    # the 2B shapes fit at any length (segment buffers of at most 12.5 MB)
+    assert jet.jet_gdn_prefill_workspace_min(1, 262144, 12, 96, 256) <= jet.NOALLOC_SCRATCH_BYTES
+    # bad arguments are refused before the size check as well
+    assert lib.jet_gdn_prefill_noalloc(None, P(A), P(A), P(A), P(A), None, P(A), P(A), B, T, H, dk, dv, 64, BF16,
+                                       None) == INVALID

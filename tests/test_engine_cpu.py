@@ -186,3 +186,31 @@ def test_serving_steps_spend_the_prefill_budget_and_decode_finished_prompts(monk
                                  d["q"], d["k"], d["v"], d["g"], d["beta"])
         np.testing.assert_allclose(torch.cat(outs[n]).numpy(), r["o"][0], rtol=1e-5, atol=1e-5)
         assert e.pos[n] == T + dec
+
+
+def test_step_checks_every_input_before_any_work(engine):
+    e, c = engine
+    e.submit("a", prompt(40))
+    one = tuple(a[0] for a in prompt(1))
+    S_before = e.S.clone()
+    with pytest.raises(KeyError):                 # a decode token for a sequence never admitted
+        e.step({"ghost": one})
+    assert c.prefill == [] and c.decode == [] and e.prefilling == ["a"] and e.pos["a"] == 0
+    assert torch.equal(e.S, S_before)
+    e.step()                                       # the prompt (40 <= 128 tokens) finishes
+    e.release("a")
+    with pytest.raises(KeyError):                 # ... or one already released
+        e.step({"a": one})
+    with pytest.raises(KeyError):
+        e.decode(["a"], *[a[None] for a in one])
+    assert c.decode == []
+
+
+def test_submit_rejects_empty_and_ragged_prompts(engine):
+    e, _ = engine
+    with pytest.raises(ValueError):
+        e.submit("empty", prompt(0))
+    ragged = prompt(5)[:5] + (torch.zeros(4, H),)
+    with pytest.raises(ValueError):
+        e.submit("ragged", ragged)
+    assert e.free_slots == 3 and e.prefilling == []

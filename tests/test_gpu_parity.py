@@ -324,17 +324,54 @@ def sampled_prefill_reference(orc, inp, heads, rows, block=16384):
 
 @pytest.mark.parametrize("name", ["prefill_4b_t65536", "prefill_2b_t262144"])
 def test_config_long_prefill_sampled(orc, name):
+    # configs 3 and 4a through both prefill paths: the two calls (conv pass, then the GDN
+    # prefill) and the one call that the benchmark and the serving loop use (conv folded
+    # into the chunk images); sampled (head, row) chains over every token against the oracle
     s = synth.CONFIGS[name]
     inp = synth.prefill_inputs(s, seed=0)
     d = gpu_inputs(inp)
-    vc, o, S, _ = run_prefill(d, s.H)
     heads, rows = [0, s.H - 3], [0, 1, 100, 255]
     ref = sampled_prefill_reference(orc, inp, heads, rows)
+    vc, o, S, _ = run_prefill(d, s.H)
     for h in heads:
         ro, rS, rvc = ref[h]
-        assert_close(host64(o[:, :, h, rows]), ro, s.dtype, f"{name} o head {h}")
-        assert_close(host64(S[:, h, rows]), rS, s.dtype, f"{name} S head {h}")
+        assert_close(host64(o[:, :, h, rows]), ro, s.dtype, f"{name} two calls o head {h}")
+        assert_close(host64(S[:, h, rows]), rS, s.dtype, f"{name} two calls S head {h}")
         assert_close(host64(vc[:, :, h, rows]), rvc, s.dtype, f"{name} v' head {h}")
+    del vc, o, S
+    hist = torch.full((s.B, 3, s.H, s.dv), float("nan"), device="cuda", dtype=d["v"].dtype)
+    o, S = jet.jet_jetblock_prefill(d["x"], d["W1"], d["W2"], d["q"], d["k"], d["v"], d["g"], d["beta"], None, hist)
+    for h in heads:
+        ro, rS, _ = ref[h]
+        assert_close(host64(o[:, :, h, rows]), ro, s.dtype, f"{name} one call o head {h}")
+        assert_close(host64(S[:, h, rows]), rS, s.dtype, f"{name} one call S head {h}")
+    assert torch.equal(hist, d["v"][:, -3:])                          # raw V of the last tokens: bit-exact
+    if s.steps == 0:
+        return
+    # config 4b: s.steps decode steps at B = 1 (generator + conv + update fused,
+    # jet_jetblock_decode_step) continuing from the one-call prefill's state and history
+    del o
+    dec = synth.decode_inputs(s.with_(B=1), seed=1, steps=s.steps)
+    dd = gpu_inputs(dec)
+    ha, hb = hist, torch.empty_like(hist)
+    outs = []
+    for t in range(s.steps):
+        ot, _ = jet.jet_jetblock_decode_step(dd["x"][t], d["W1"], d["W2"], dd["q"][t], dd["k"][t], dd["v"][t], ha, hb,
+                                             dd["g"][t], dd["beta"][t], S)
+        outs.append(ot)
+        ha, hb = hb, ha
+    o_dec = torch.stack(outs)                                           # [n, 1, H, dv]
+    dt = s.dtype
+    f = lambda a: synth.to_f64(a, dt)
+    for h in heads:
+        _, rS, _ = ref[h]
+        hist_h = f(inp["v"][:, -3:, h:h + 1, rows])                    # raw V of the last three prompt tokens
+        r = orc.jetblock_decode(f(dec["x"]), f(inp["W1"]), f(inp["W2"][:, 4 * h:4 * h + 4]),
+                                f(dec["q"][:, :, h:h + 1]), f(dec["k"][:, :, h:h + 1]),
+                                f(dec["v"][:, :, h:h + 1, rows]), dec["g"][:, :, h:h + 1],
+                                dec["beta"][:, :, h:h + 1], rS[:, None], hist_h)
+        assert_close(host64(o_dec[:, :, h, rows]), r["o"][:, :, 0], dt, f"4b decode o head {h}")
+        assert_close(host64(S[:, h, rows]), r["S"][:, 0], dt, f"4b decode S head {h}")
 
 
 def run_decode(d, steps, B, H, dv, dtype_t, fused=False):

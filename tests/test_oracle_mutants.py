@@ -35,6 +35,7 @@ MUTANTS = {
                                    "const double a = g[bth] + 1.0, bt = beta[bth];"),
     "l2norm_squared": ("const double inv = 1.0 / sqrt(ss + eps);", "const double inv = 1.0 / (ss + eps);"),
     "l2norm_skipped": ("const double inv = 1.0 / sqrt(ss + eps);", "const double inv = 1.0;"),
+    "l2norm_eps_outside_sqrt": ("const double inv = 1.0 / sqrt(ss + eps);", "const double inv = 1.0 / (sqrt(ss) + eps);"),
     "decode_gate_on_write": ("const double c = bt * v[bh * dv + i] - a * bt * u;",
                              "const double c = a * bt * v[bh * dv + i] - a * bt * u;"),
     "chunked_decay_sign": ("a = br * exp(G[r] - G[i]) * kk;", "a = br * exp(G[i] - G[r]) * kk;"),
@@ -58,6 +59,7 @@ PINS = [
     (pins.test_gdn_chunked_equals_sequential, {"T": 65, "C": 64, "long_memory": False}),
     (pins.test_gdn_decode_steps_equal_sequential, {}),
     (pins.test_gdn_l2_normalises_q_and_k, {}),
+    (pins.test_gdn_l2_norm_eps_on_zero_and_tiny_vectors, {}),
     (pins.test_mixer_prefill_then_decode_continues, {}),
 ]
 

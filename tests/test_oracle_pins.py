@@ -323,3 +323,26 @@ def test_mixer_identity_taps_reduce_to_plain_gdn(orc):
     o2, S2 = orc.gdn_sequential(q, k, v, g, beta, S0)
     np.testing.assert_array_equal(o1, o2)
     np.testing.assert_array_equal(S1, S2)
+
+
+def test_gdn_l2_norm_eps_on_zero_and_tiny_vectors(orc):
+    # eps sits under the square root: a zero key leaves only the decay (S_t = a_t S_{t-1}),
+    # a zero query gives o_t = 0, and a key of norm 1e-3 is scaled by 1/sqrt(1e-6 + 1e-6)
+    q, k, v, g, beta, S0 = gdn_inputs(rnd(18), T=3)
+    k[0, 1, 0] = 0.0
+    q[0, 2, 1] = 0.0
+    o, S = orc.gdn_sequential(q, k, v, g, beta, S0)
+    o1, S1 = orc.gdn_sequential(q[:, :1], k[:, :1], v[:, :1], g[:, :1], beta[:, :1], S0)
+    o2, S2 = orc.gdn_sequential(q[:, :2], k[:, :2], v[:, :2], g[:, :2], beta[:, :2], S0)
+    np.testing.assert_allclose(S2[0, 0], np.exp(g[0, 1, 0]) * S1[0, 0], rtol=1e-14, atol=0)
+    np.testing.assert_array_equal(o[0, 2, 1], 0.0)
+    # one token from S0 with a tiny key: u = S0 k / sqrt(|k|^2 + eps), written out by hand
+    kt = k[:, :1].copy()
+    kt[0, 0, 0] *= 1e-3 / np.linalg.norm(kt[0, 0, 0])
+    qt = q[:, :1]
+    _, St = orc.gdn_sequential(qt, kt, v[:, :1], g[:, :1], beta[:, :1], S0)
+    kh = kt[0, 0, 0] / np.sqrt(1e-6 + 1e-6)
+    a, b = np.exp(g[0, 0, 0]), beta[0, 0, 0]
+    Sx = S0[0, 0]
+    want = a * (Sx - b * np.outer(Sx @ kh, kh)) + b * np.outer(v[0, 0, 0], kh)
+    np.testing.assert_allclose(St[0, 0], want, rtol=1e-12, atol=1e-14)

@@ -65,3 +65,18 @@ def test_config_table_matches_the_stated_shapes():
     for s in c.values():
         assert s.dv == 256 or s.name == "tiny_f32"
         assert s.R == 32 and s.W == 4
+
+
+def test_spread_qk_norms_rescales_rows_and_zeroes_the_chosen_ones():
+    shape = synth.CONFIGS["tiny_f32"].with_(T=50, dtype="bf16")
+    a = synth.prefill_inputs(shape, seed=2)
+    k = synth.spread_qk_norms(a["k"], "bf16", seed=2, zero_rows=[(0, 7, 1)])
+    assert k.dtype == np.uint16 and k.shape == a["k"].shape
+    n = np.linalg.norm(synth.to_f64(k, "bf16"), axis=-1)
+    assert n[0, 7, 1] == 0.0
+    rest = np.delete(n.ravel(), np.ravel_multi_index((0, 7, 1), n.shape))
+    assert rest.min() > 0.09 and rest.max() < 11.0              # 10**U(-1, 1) times a unit row
+    assert rest.min() < 0.2 and rest.max() > 5.0                # the range is actually spanned
+    # its own stream: the same seed gives the same rows, and the main draw is untouched
+    np.testing.assert_array_equal(k, synth.spread_qk_norms(a["k"], "bf16", seed=2, zero_rows=[(0, 7, 1)]))
+    np.testing.assert_array_equal(a["k"], synth.prefill_inputs(shape, seed=2)["k"])
