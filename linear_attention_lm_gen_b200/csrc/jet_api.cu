@@ -16,6 +16,7 @@
 #include "k_genconv.cuh"
 #include "k_prefill_simt.cuh"
 #include "k_prefill_chain.cuh"
+#include "k_prefill_correct.cuh"
 #include "k_prefill_ws.cuh"
 #include "k_segcombine.cuh"
 
@@ -190,36 +191,77 @@ bool tile_map(CUtensorMap* m, const void* base, int d, int H, long long rows, in
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Number of segments of the sequence-parallel prefill (1 = single pass):
-// the largest P that keeps both phases within one wave of 148 SMs and every
-// segment at least 8 chunks long. A function of the shapes only, so the
-// workspace size can be queried without a device.
-constexpr int kSMs = 148;
+// Segment plans of the sequence-parallel prefill (P = 1: a single segment).
+// Both keep every launch within one wave of the SMs and every segment at
+// least 8 chunks long, and are functions of the shapes and the SM count only,
+// so the workspace can be queried without a device: the queries plan for
+// kMaxSMs (a full B200); a launch plans for min(the device's SMs, kMaxSMs),
+// which never needs more workspace.
+//   two passes (the fused low-memory kernel): phase A runs segments 0..P-2
+//     with a transition slice each for p >= 1, phase C all P segments;
+//   one pass (chunk images + chain kernel): all P segments at once, each with
+//     a transition slice for p >= 1 (see k_prefill_chain.cuh).
+constexpr int kMaxSMs = 148;
 constexpr int kMinSegChunks = 8;
 struct SegPlan { int P, seg_chunks; };
-SegPlan plan_segments(int B, int T, int H, int dv) {
-    const int nch = (T + 63) / 64, ns = dv / pfws::ROWS;
+template <typename Fits>
+SegPlan plan_segments(int T, Fits fits) {
+    const int nch = (T + 63) / 64;
     SegPlan best{1, nch};
     for (int P = 2; P <= 64; ++P) {
         const int segc = (nch + P - 1) / P;
         if (segc < kMinSegChunks) break;
         const int Peff = (nch + segc - 1) / segc;
         if (Peff != P) continue;
-        const long long ctaA = (long long)B * H * ((P - 1) * ns + (P - 2));
-        const long long ctaC = (long long)B * H * ns * P;
-        if (ctaA > kSMs || ctaC > kSMs) break;
+        if (!fits(P)) break;
         best = SegPlan{P, segc};
     }
     return best;
 }
+SegPlan plan_two_pass(int B, int T, int H, int dv, int sms) {
+    const int ns = dv / pfws::ROWS;
+    return plan_segments(T, [&](int P) {
+        return (long long)B * H * ((P - 1) * ns + (P - 2)) <= sms && (long long)B * H * ns * P <= sms;
+    });
+}
+SegPlan plan_one_pass(int B, int T, int H, int dv, int sms) {
+    const int ns = dv / pfws::ROWS;
+    return plan_segments(T, [&](int P) { return (long long)B * H * ((long long)ns * P + P - 1) <= sms; });
+}
+// SMs a launch plans for (the current device's count, at most kMaxSMs)
+int launch_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess || n <= 0)
+        return kMaxSMs;
+    return std::min(n, kMaxSMs);
+}
 bool tc_prefill_ok(jet_dtype dt, int dk, int dv, long long BT) {
     return dt == JET_BF16 && dv % pfws::ROWS == 0 && (dk == 64 || dk == 96 || dk == 128) && BT < (1LL << 31);
 }
+// segment buffers of the two-pass plan: E [B][P-1][H][dv][dk] phase-A end
+// states, A [B][P-1][H][dk][dk+8] transitions, S_start [B][P][H][dv][dk]
 size_t seg_workspace_floats(int B, int H, int dk, int dv, int P) {
     if (P <= 1) return 0;
     return (size_t)B * (P - 1) * H * dv * dk      // E: phase A end states
          + (size_t)B * (P - 1) * H * dk * pfws::trans_ld(dk)   // A: transitions (padded rows)
          + (size_t)B * P * H * dv * dk;           // start states
+}
+// segment buffers of the one-pass plan, each part 1024-byte aligned:
+// E [B][P][H][dv][dk], A [B][P][H][dk][dk+8], S_start [B][P][H][dv][dk]
+// (float32), Qe [B][H][nct][64][dk] (bf16)
+struct OnePassLayout { size_t E, A, Sst, Qe, bytes; };
+OnePassLayout one_pass_layout(int B, int T, int H, int dk, int dv, int P) {
+    auto up = [](size_t x) { return (x + 1023) & ~size_t(1023); };
+    OnePassLayout l{0, 0, 0, 0, 0};
+    if (P <= 1) return l;
+    const size_t nct = (size_t)((T + 63) / 64);
+    l.E = 0;
+    l.A = l.E + up(sizeof(float) * B * P * H * (size_t)dv * dk);
+    l.Sst = l.A + up(sizeof(float) * B * P * H * (size_t)dk * pfws::trans_ld(dk));
+    l.Qe = l.Sst + up(sizeof(float) * B * P * H * (size_t)dv * dk);
+    l.bytes = l.Qe + up(sizeof(__nv_bfloat16) * B * H * nct * 64 * (size_t)dk);
+    return l;
 }
 
 // per-chunk image of the two-kernel plan (preparation + chain), bytes
@@ -235,12 +277,25 @@ size_t split_img_bytes(int B, int T, int H, int dk) {
 }
 
 // Tensor-core prefill. SPLIT: K2a prepares every chunk into an image, then
-// the chain kernel K2b runs (workspace = images + segment buffers); otherwise
-// the fused kernel prepares chunk c+1 while it runs chunk c (workspace =
-// segment buffers only). Sequence-parallel segments as planned above.
+// the chain kernel K2b runs every segment in one pass; with several segments
+// the combine chains their start states and the correction kernel adds the
+// start-state term to the outputs (workspace = images + one-pass buffers).
+// Otherwise the fused kernel prepares chunk c+1 while it runs chunk c, in two
+// passes over the segments (workspace = two-pass segment buffers only).
 // CONV (split plan only): v is the raw V; the preparation folds the dynamic
 // conv with `taps` into the chunk images and the chain reads the values
 // before each segment (and the history of `cv`) for it.
+template <int DK, int DV>
+jet_status launch_correct(const __nv_bfloat16* Qe, const float* Sst, void* o, int B, int Tn, int H, int nct,
+                          int segc, int P, cudaStream_t s) {
+    auto kern = pfcor::prefill_correct_kernel<DK, DV>;
+    const size_t smem = pfcor::smem_bytes(DK, DV);
+    if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
+    kern<<<dim3(nct - segc, H, B), pfcor::THREADS, smem, s>>>(Qe, Sst, (__nv_bfloat16*)o, Tn, H, nct, segc, P);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return launch_status();
+}
+
 template <int DK, bool SPLIT, bool CONV = false>
 jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const float* g, const float* beta,
                              const float* S0, void* o, float* S_out, void* workspace, int B, int Tn, int H,
@@ -258,35 +313,60 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
                  (cv.hist_in && !tile_map(&mhh, cv.hist_in, dv, H, (long long)B * 3, 16))))
         return JET_ERR_CUDA;
     if (CONV && !cv.hist_in) mhh = mvh;
-    auto fused = pfws::gdn_prefill_ws_kernel<DK>;
-    auto chain = pfch::gdn_prefill_chain_kernel<DK, CONV>;
-    const uint32_t smem = SPLIT ? pfch::ChainSmem<DK>::BYTES : pfws::SMEM_BYTES;
-    const int threads = SPLIT ? pfch::THREADS : pfws::THREADS;
-    if ((SPLIT ? smem_attr(chain, smem) : smem_attr(fused, smem)) != JET_OK) return JET_ERR_CUDA;
-    uint8_t* img = static_cast<uint8_t*>(workspace);
-    float* ws = reinterpret_cast<float*>(img + (SPLIT ? split_img_bytes(B, Tn, H, DK) : 0));
-    if (SPLIT) {   // K2a: every chunk of every (sequence, head)
-        auto prep = pfws::gdn_chunk_prep_kernel<DK>;
-        if (smem_attr(prep, pfws::PrepSmem<DK>::BYTES) != JET_OK) return JET_ERR_CUDA;
-        const int nct = (Tn + pfws::C - 1) / pfws::C;
-        const long long items = (long long)B * H * nct;
-        const int grid = (int)std::min<long long>(items, (long long)pfws::PREP_CTAS * kSMs);   // resident CTAs
-        prep<<<grid, pfws::PREP_THREADS, pfws::PrepSmem<DK>::BYTES, s>>>(
-            mq, mk, g, beta, CONV ? taps : nullptr, cv.hist_in != nullptr, img, Tn, H, nct, (int)items);
+    const int ns = dv / pfws::ROWS;
+    const int nct = (Tn + pfws::C - 1) / pfws::C;
+    const int sms = launch_sms();
+    if (SPLIT) {
+        auto chain = pfch::gdn_prefill_chain_kernel<DK, CONV>;
+        constexpr uint32_t smem = pfch::ChainSmem<DK>::BYTES;
+        if (smem_attr(chain, smem) != JET_OK) return JET_ERR_CUDA;
+        uint8_t* img = static_cast<uint8_t*>(workspace);
+        uint8_t* segws = img + split_img_bytes(B, Tn, H, DK);
+        {   // K2a: every chunk of every (sequence, head)
+            auto prep = pfws::gdn_chunk_prep_kernel<DK>;
+            if (smem_attr(prep, pfws::PrepSmem<DK>::BYTES) != JET_OK) return JET_ERR_CUDA;
+            const long long items = (long long)B * H * nct;
+            const int grid = (int)std::min<long long>(items, (long long)pfws::PREP_CTAS * sms);   // resident CTAs
+            prep<<<grid, pfws::PREP_THREADS, pfws::PrepSmem<DK>::BYTES, s>>>(
+                mq, mk, g, beta, CONV ? taps : nullptr, cv.hist_in != nullptr, img, Tn, H, nct, (int)items);
+            g_launches.fetch_add(1, std::memory_order_relaxed);
+            if (launch_status() != JET_OK) return JET_ERR_CUDA;
+        }
+        const SegPlan plan = plan_one_pass(B, Tn, H, dv, sms);
+        const int P = plan.P;
+        const OnePassLayout lay = one_pass_layout(B, Tn, H, DK, dv, P);
+        float* E = reinterpret_cast<float*>(segws + lay.E);
+        float* A = reinterpret_cast<float*>(segws + lay.A);
+        float* Sst = reinterpret_cast<float*>(segws + lay.Sst);
+        __nv_bfloat16* Qe = reinterpret_cast<__nv_bfloat16*>(segws + lay.Qe);
+        const pfch::ChainSeg seg = P == 1 ? pfch::ChainSeg{1, plan.seg_chunks, nullptr, nullptr, nullptr}
+                                          : pfch::ChainSeg{P, plan.seg_chunks, E, A, Qe};
+        chain<<<dim3(ns + (P > 1 ? 1 : 0), H, B * P), pfch::THREADS, smem, s>>>(
+            mk, mv, mvh, mhh, img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg, cv);
         g_launches.fetch_add(1, std::memory_order_relaxed);
         if (launch_status() != JET_OK) return JET_ERR_CUDA;
+        if (P == 1) return JET_OK;
+        // start states S*_1 .. S*_{P-1} and the final state
+        const size_t sc_smem = sc_smem_bytes(DK);
+        if (smem_attr(seg_combine_kernel<DK, true>, sc_smem) != JET_OK) return JET_ERR_CUDA;
+        seg_combine_kernel<DK, true><<<dim3(dv / SC_ROWS, H, B), sc_threads(DK), sc_smem, s>>>(E, A, nullptr, Sst,
+                                                                                              S_out, P, H, dv);
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        if (launch_status() != JET_OK) return JET_ERR_CUDA;
+        // outputs of the segments p >= 1: O += Qe S*^T
+        return dv == 256 ? launch_correct<DK, 256>(Qe, Sst, o, B, Tn, H, nct, plan.seg_chunks, P, s)
+                         : launch_correct<DK, 128>(Qe, Sst, o, B, Tn, H, nct, plan.seg_chunks, P, s);
     }
+    auto fused = pfws::gdn_prefill_ws_kernel<DK>;
+    if (smem_attr(fused, pfws::SMEM_BYTES) != JET_OK) return JET_ERR_CUDA;
+    float* ws = reinterpret_cast<float*>(workspace);
     auto run = [&](dim3 grid, const pfws::Seg& seg) {
-        if (SPLIT)
-            chain<<<grid, threads, smem, s>>>(mk, mv, mvh, mhh, img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg,
-                                              cv);
-        else
-            fused<<<grid, threads, smem, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg);
+        fused<<<grid, pfws::THREADS, pfws::SMEM_BYTES, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o, S_out, Tn, H,
+                                                            dv, seg);
         g_launches.fetch_add(1, std::memory_order_relaxed);
         return launch_status();
     };
-    const int ns = dv / pfws::ROWS;
-    const SegPlan plan = plan_segments(B, Tn, H, dv);
+    const SegPlan plan = plan_two_pass(B, Tn, H, dv, sms);
     const int P = plan.P;
     if (P == 1) return run(dim3(ns, H, B), pfws::Seg{1, plan.seg_chunks, 1, 0, nullptr, nullptr, nullptr});
     float* E = ws;
@@ -297,8 +377,9 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
         return JET_ERR_CUDA;
     // start states of every segment (S0 copied for segment 0)
     const size_t sc_smem = sc_smem_bytes(DK);
-    if (smem_attr(seg_combine_kernel<DK>, sc_smem) != JET_OK) return JET_ERR_CUDA;
-    seg_combine_kernel<DK><<<dim3(dv / SC_ROWS, H, B), sc_threads(DK), sc_smem, s>>>(E, A, S0, Sst, P, H, dv);
+    if (smem_attr(seg_combine_kernel<DK, false>, sc_smem) != JET_OK) return JET_ERR_CUDA;
+    seg_combine_kernel<DK, false><<<dim3(dv / SC_ROWS, H, B), sc_threads(DK), sc_smem, s>>>(E, A, S0, Sst, nullptr,
+                                                                                           P, H, dv);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     if (launch_status() != JET_OK) return JET_ERR_CUDA;
     // phase C: every segment from its start state, with outputs
@@ -389,13 +470,14 @@ jet_status jet_dyn_conv_v(const void* x, const void* w1, const void* w2, const v
 
 size_t jet_gdn_prefill_workspace_min(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt) {
     if (B <= 0 || T <= 0 || H <= 0 || chunk != 64 || !tc_prefill_ok(dt, dk, dv, (long long)B * T)) return 0;
-    const SegPlan plan = plan_segments(B, T, H, dv);
+    const SegPlan plan = plan_two_pass(B, T, H, dv, kMaxSMs);
     return sizeof(float) * seg_workspace_floats(B, H, dk, dv, plan.P);
 }
 
 size_t jet_gdn_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt) {
     if (B <= 0 || T <= 0 || H <= 0 || chunk != 64 || !tc_prefill_ok(dt, dk, dv, (long long)B * T)) return 0;
-    return split_img_bytes(B, T, H, dk) + jet_gdn_prefill_workspace_min(B, T, H, dk, dv, chunk, dt);
+    const SegPlan plan = plan_one_pass(B, T, H, dv, kMaxSMs);
+    return split_img_bytes(B, T, H, dk) + one_pass_layout(B, T, H, dk, dv, plan.P).bytes;
 }
 
 jet_status jet_gdn_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,

@@ -29,7 +29,18 @@
 // thread) spin on the mbarrier before they start to sleep between polls, so
 // they wake within tens of cycles; the others sleep between polls and leave
 // the issue slots to them.
-// Segments (sequence parallelism) work as in the fused kernel: see Seg.
+//
+// Segments (sequence parallelism, one pass). The recurrence is affine in the
+// state, so with P segments every segment runs at once: segment 0 from S0,
+// the others from a zero state, each writing provisional outputs O0 and its
+// end state E_p. For p >= 1 an extra "transition" slice starts from the
+// identity with zero values; its state is the product Phi_c of the per-token
+// transitions since the segment start, and its output products give
+//   Qe_c = (Q~ - P W) Phi_c^T      (64 tokens x dk, written per chunk)
+// which is exactly what the start state multiplies in the outputs:
+//   O_c = O0_c + Qe_c S*^T,  S* = the segment's true start state.
+// The segment combine then chains S*_{p+1} = S*_p A_p + E_p (A_p = Phi at the
+// segment end) and a correction kernel adds Qe_c S*^T to the outputs.
 //
 // CONV: the V tiles hold the raw values and the images were prepared with
 // the dynamic causal conv (Jet-Nemotron paper, section 2.4) folded into T1:
@@ -103,6 +114,15 @@ struct ChainConv {
     __nv_bfloat16* hist_out;         // [B][3][H][dv] last three raw tokens, or null
 };
 
+// one pass over all segments (see the header comment); P = 1 is the plain pass
+struct ChainSeg {
+    int nseg;                 // P
+    int seg_chunks;           // chunks per segment (the last may be shorter)
+    float* Eo;                // P > 1: end states [B][P][H][dv][dk] (segment 0 from S0, the others from 0)
+    float* Ao;                // P > 1: transitions [B][P][H][dk][trans_ld(dk)] (p >= 1)
+    __nv_bfloat16* Qe;        // P > 1: output corrections [B][H][nct][64][dk] (chunks of segments p >= 1)
+};
+
 enum {
     B_IMG = 0,        // [2] image landed
     B_K = 2,          // [NKBUF] K tile landed
@@ -125,7 +145,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ CUtensorMap tm_hh,
                          const uint8_t* __restrict__ img, const float* S0, __nv_bfloat16* __restrict__ o,
-                         float* S_out, int Tn, int H, int dv, const Seg seg, const ChainConv cv) {
+                         float* S_out, int Tn, int H, int dv, const ChainSeg seg, const ChainConv cv) {
     static_assert(DK % 32 == 0 && DK >= 64 && DK <= 128, "DK in {64, 96, 128}");
     using SM = ChainSmem<DK>;
     using IM = Img<DK>;
@@ -143,9 +163,9 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         return;
     }
     const int ns = dv / ROWS;
-    const int h = blockIdx.y, b = blockIdx.z / seg.zseg, p_seg = blockIdx.z % seg.zseg;
-    const bool trans = blockIdx.x == ns;                  // transition slice (phase A, p >= 1)
-    if (trans && (!seg.phaseA || p_seg == 0)) return;     // whole CTA, before any barrier
+    const int h = blockIdx.y, b = blockIdx.z / seg.nseg, p_seg = blockIdx.z % seg.nseg;
+    const bool trans = blockIdx.x == ns;                  // transition slice (p >= 1)
+    if (trans && p_seg == 0) return;                      // whole CTA, before any barrier
     const int c0 = blockIdx.x * ROWS;                     // transition slice: past dv, V reads as zero
     const long long bh = (long long)b * H + h;
     const int nct = (Tn + C - 1) / C;                     // chunks per sequence (image index)
@@ -153,7 +173,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
     const int tbeg = cbeg * C;
     const int tend = min(Tn, tbeg + seg.seg_chunks * C);
     const int nch = (tend - tbeg + C - 1) / C;
-    const bool write_o = !seg.phaseA;
+    constexpr bool write_o = true;                        // every slice has output products (trans: Qe)
     const uint8_t* img_bh = img + (size_t)bh * nct * IM::BYTES;
     auto img_at = [&](int c) -> const uint8_t* { return sm + SM::IMG + (uint32_t)(c & 1) * SM::IB; };
 
@@ -181,12 +201,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         const int ct = tid;
         const uint32_t lb = (uint32_t)(warp * 32) << 16;
         {   // initial state (row ct of the slice)
-            const float* src = nullptr;
-            if (!seg.phaseA && seg.nseg > 1) {
-                src = seg.Sst + ((((long long)b * seg.nseg + p_seg) * H + h) * dv + c0 + ct) * DK;
-            } else if (p_seg == 0 && !trans && S0) {
-                src = S0 + (bh * dv + c0 + ct) * DK;
-            }
+            const float* src = (p_seg == 0 && !trans && S0) ? S0 + (bh * dv + c0 + ct) * DK : nullptr;
 #pragma unroll
             for (int cb = 0; cb < DK / 32; ++cb) {
                 uint32_t r[32];
@@ -276,12 +291,12 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         if (group_all(2, NCH_T, fin)) {
             tc_fence_after();
             float* dst = nullptr;
-            if (seg.phaseA) {
-                const long long bp = (long long)b * (seg.nseg - 1) + p_seg;
+            if (seg.nseg == 1) {
+                dst = S_out + (bh * dv + c0 + ct) * DK;
+            } else {
+                const long long bp = (long long)b * seg.nseg + p_seg;
                 if (trans) { if (ct < DK) dst = seg.Ao + ((bp * H + h) * DK + ct) * trans_ld(DK); }
                 else dst = seg.Eo + ((bp * H + h) * dv + c0 + ct) * DK;
-            } else if (p_seg == seg.nseg - 1) {
-                dst = S_out + (bh * dv + c0 + ct) * DK;
             }
 #pragma unroll
             for (int cb = 0; cb < DK / 32; ++cb) {
@@ -312,7 +327,12 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             tc_fence_after();
             const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
             const int t0 = tbeg + c * C, L = min(C, tend - t0);
-            __nv_bfloat16* obase = o + ((long long)b * Tn + t0) * tstride + (long long)h * dv + c0;
+            // value slices: o rows of this chunk; transition slice: Qe of the chunk
+            // ([64 tokens][dk], rows of the slice = key features, only the first dk exist)
+            __nv_bfloat16* obase = trans ? seg.Qe + ((size_t)bh * nct + cbeg + c) * C * DK
+                                         : o + ((long long)b * Tn + t0) * tstride + (long long)h * dv + c0;
+            const long long rstride = trans ? (long long)DK : tstride;
+            const int nchunk16 = trans ? DK / 8 : 16;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {           // 32 tokens from TMEM at a time
                 uint32_t x[32];
@@ -330,8 +350,8 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                     for (int m = 0; m < OUT_TOK / 8; ++m) {  // OUT_TOK rows x 16 chunks of 16 bytes
                         const int qd = ot + m * NOUT, r = qd >> 4, cq = qd & 15;
                         const int tok = half * 32 + sub * OUT_TOK + r;
-                        if (tok < L)
-                            *reinterpret_cast<uint4*>(obase + tok * tstride + cq * 8) =
+                        if (tok < L && cq < nchunk16)
+                            *reinterpret_cast<uint4*>(obase + tok * rstride + cq * 8) =
                                 *reinterpret_cast<const uint4*>(st + r * ROWS + cq * 8);
                     }
                     named_sync(3, NOUT);                     // staging free again
@@ -340,7 +360,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         }
         if (!run) *abort_flag = 1;
         // CONV: the new history, the last three raw values of the sequence (or of the old history)
-        if (CONV && run && cv.hist_out && !seg.phaseA && p_seg == seg.nseg - 1 && c0 + ot < dv) {
+        if (CONV && run && cv.hist_out && !trans && p_seg == seg.nseg - 1 && c0 + ot < dv) {
             const int ch = c0 + ot;
 #pragma unroll
             for (int k3 = 0; k3 < 3; ++k3) {

@@ -1,0 +1,149 @@
+// Output correction of the one-pass sequence-parallel prefill.
+//
+// The chunked gated delta rule (Jet-Nemotron paper, section 2.3) gives a
+// chunk's outputs as an affine function of the state S_c at the chunk start:
+//   O_c = (Q~ - P W) S_c^T + P U.
+// Inside a segment that started from a zero state instead of its true start
+// state S*, the state at chunk c differs by S* Phi_c (Phi_c: the product of
+// the transitions since the segment start), so the true outputs are
+//   O_c = O0_c + Qe_c S*^T,   Qe_c = (Q~ - P W) Phi_c^T   [64 tokens x dk],
+// where O0_c are the outputs the segment pass wrote and Qe_c is what its
+// transition slice wrote. This kernel adds Qe_c S*^T for every chunk of the
+// segments p >= 1.
+//
+// One CTA per (sequence, head, chunk): a 64 x dv by dk product on the tensor
+// cores (bf16 mma.sync m16n8k16, float32 accumulate; 2 x 1.6 Mflop per chunk
+// is far too small a tile for tcgen05, and the kernel is bound by moving the
+// 32 KB output tile). The Qe tile, S* (float32, rounded to bf16 on the way
+// into shared memory) and the output tile are staged in shared memory with
+// padded rows (conflict-free ldmatrix), then the output is written back with
+// 16-byte stores. Warp w owns output columns [w dv/8, (w+1) dv/8).
+#pragma once
+#include "common.cuh"
+
+namespace jet {
+namespace pfcor {
+
+constexpr int THREADS = 256;
+constexpr int C = 64;
+
+__host__ __device__ constexpr int lda(int dk) { return dk + 8; }      // bf16 row stride of Qe and S*
+__host__ __device__ constexpr int ldo(int dv) { return dv + 8; }      // bf16 row stride of the output tile
+__host__ __device__ constexpr size_t smem_bytes(int dk, int dv) {
+    return 2 * ((size_t)C * lda(dk) + (size_t)dv * lda(dk) + (size_t)C * ldo(dv));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t* r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint32_t* b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Qe [B][H][nct][64][DK] bf16; Sst [B][P][H][dv][DK] float32 (entries p >= 1);
+// o [B*T][H][dv] bf16 (updated in place). grid (nct - seg_chunks, H, B).
+template <int DK, int DV>
+__global__ void __launch_bounds__(THREADS)
+prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const float* __restrict__ Sst,
+                       __nv_bfloat16* __restrict__ o, int Tn, int H, int nct, int seg_chunks, int P) {
+    static_assert(DK % 16 == 0 && DK <= 128 && DV % 64 == 0 && DV <= 256, "shapes");
+    constexpr int LDA = lda(DK), LDO = ldo(DV);
+    constexpr int NT = DV / 64;                    // n8 tiles per warp (DV / 8 columns)
+    constexpr int KS = DK / 16;
+    extern __shared__ __align__(16) uint8_t smem[];
+    __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem);          // [64][LDA]
+    __nv_bfloat16* ss = qs + C * LDA;                                    // [DV][LDA]
+    __nv_bfloat16* os = ss + DV * LDA;                                   // [64][LDO]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gc = seg_chunks + blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    if (gc >= nct) return;
+    const int p = gc / seg_chunks;
+    const int t0 = gc * C, L = min(C, Tn - t0);
+    const long long bh = (long long)b * H + h;
+    const long long tstride = (long long)H * DV;
+
+    {   // Qe rows (zero past the sequence end), 16-byte pieces
+        const uint4* src = reinterpret_cast<const uint4*>(Qe + ((size_t)bh * nct + gc) * C * DK);
+        for (int i = tid; i < C * DK / 8; i += THREADS) {
+            const int r = i / (DK / 8), cc = i % (DK / 8);
+            const uint4 v = r < L ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(qs + r * LDA + cc * 8) = v;
+        }
+    }
+    {   // S* of the segment, float32 -> bf16
+        const float4* src = reinterpret_cast<const float4*>(Sst + ((((long long)b * P + p) * H + h) * DV) * DK);
+        for (int i = tid; i < DV * DK / 8; i += THREADS) {
+            const int r = i / (DK / 8), cc = i % (DK / 8);
+            const float4 a = src[2 * i], c = src[2 * i + 1];
+            const float f[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+            *reinterpret_cast<uint4*>(ss + r * LDA + cc * 8) = Vec16<__nv_bfloat16>::pack(f);
+        }
+    }
+    {   // the provisional outputs of the chunk
+        for (int i = tid; i < C * DV / 8; i += THREADS) {
+            const int r = i / (DV / 8), cc = i % (DV / 8);
+            if (r < L)
+                *reinterpret_cast<uint4*>(os + r * LDO + cc * 8) =
+                    *reinterpret_cast<const uint4*>(o + ((long long)b * Tn + t0 + r) * tstride + h * DV + cc * 8);
+        }
+    }
+    __syncthreads();
+
+    // acc[m][n]: rows 16 m + (g, g + 8), columns n0 + 8 n + (2 t, 2 t + 1)
+    float acc[4][NT][4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[m][n][e] = 0.f;
+    const int n0 = warp * (DV / 8);
+    const uint32_t qbase = static_cast<uint32_t>(__cvta_generic_to_shared(qs));
+    const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(ss));
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+        uint32_t a[4][4], bb[NT][2];
+#pragma unroll
+        for (int m = 0; m < 4; ++m)     // A rows 16 m + (lane & 15), k-offset 8 (lane >> 4)
+            ldsm_x4(qbase + (uint32_t)(((16 * m + (lane & 15)) * LDA + ks * 16 + (lane >> 4) * 8) * 2), a[m]);
+#pragma unroll
+        for (int n = 0; n < NT; ++n)    // B (S* rows = output columns) n0 + 8 n + (lane & 7), k-offset 8 ((lane >> 3) & 1)
+            ldsm_x2(sbase + (uint32_t)(((n0 + 8 * n + (lane & 7)) * LDA + ks * 16 + ((lane >> 3) & 1) * 8) * 2),
+                    bb[n]);
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int n = 0; n < NT; ++n) mma16816(acc[m][n], a[m], bb[n]);
+    }
+    // add into the staged outputs (each element is owned by one thread)
+    const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int r = 16 * m + g + 8 * hr, col = n0 + 8 * n + 2 * t4;
+                __nv_bfloat162* op = reinterpret_cast<__nv_bfloat162*>(os + r * LDO + col);
+                const float2 cur = __bfloat1622float2(*op);
+                *op = __floats2bfloat162_rn(cur.x + acc[m][n][2 * hr], cur.y + acc[m][n][2 * hr + 1]);
+            }
+    __syncthreads();
+    for (int i = tid; i < C * DV / 8; i += THREADS) {
+        const int r = i / (DV / 8), cc = i % (DV / 8);
+        if (r < L)
+            *reinterpret_cast<uint4*>(o + ((long long)b * Tn + t0 + r) * tstride + h * DV + cc * 8) =
+                *reinterpret_cast<const uint4*>(os + r * LDO + cc * 8);
+    }
+}
+
+}  // namespace pfcor
+}  // namespace jet

@@ -3,23 +3,19 @@
 // The gated delta rule is affine in the state (Jet-Nemotron paper, section
 // 2.3): over a segment, S_end = S_start A + B, with A (dk x dk) the product of
 // the per-token transitions a_t (I - b_t k^_t k^_t^T) and B the end state
-// reached from a zero start. Phase A of the prefill writes B_p (E below, with
-// E_0 the true end state of segment 0) and A_p for p = 1 .. P-2; this kernel
-// chains them:
-//   S_start(1) = E_0,   S_start(p + 1) = S_start(p) A_p + E_p   (p = 1 .. P-2)
-// It also copies S0 (or zeros) to S_start(0), so that phase C never reads S0
-// while the last segment may be writing a final state that aliases it.
-//
-// Rows of S are independent: a CTA owns 16 rows of one (sequence, head) and
-// walks p sequentially. Each step is a 16 x dk by dk x dk product on the
-// tensor cores (mma.sync m16n8k8, tf32 in, float32 accumulate), with every
-// operand split as x = hi + lo (both tf32; the running rows are split once
-// when written) and the product formed as
-// lo*hi + hi*lo + hi*hi, which keeps float32 accuracy (the dropped lo*lo
-// term is below 2^-22 relative). Warp w owns output columns 8w .. 8w+7. A_p
-// arrives by one bulk copy into a double buffer (the copy of A_{p+1} in
-// flight while step p computes); E_p of the next step is loaded during the
-// current one.
+// reached from a zero start. The segment passes write the end states E_p
+// (E_0 is the true end state of segment 0, which starts from S0) and the
+// transitions A_p (p >= 1); this kernel chains them:
+//   S_start(1) = E_0,   S_start(p + 1) = S_start(p) A_p + E_p.
+// Two layouts:
+//   one pass (FINAL): E and A hold all P segments; the kernel writes
+//     S_start(1 .. P-1) (the start states the output correction needs) and
+//     the final state S_start(P) to S_out (which may alias S0: segment 0 has
+//     read S0 before this kernel runs);
+//   two passes: E and A hold segments 0 .. P-2 (the pass without outputs);
+//     the kernel writes S_start(0 .. P-1), S_start(0) being a copy of S0 (or
+//     zeros), so that the pass with outputs never reads S0 while the last
+//     segment may be writing a final state that aliases it.
 #pragma once
 #include "common.cuh"
 #include "k_prefill_common.cuh"
@@ -55,13 +51,16 @@ __device__ __forceinline__ void mma(float* d, const uint32_t* a, const uint32_t*
 }
 }  // namespace sc
 
-// E [B][P-1][H][dv][dk], A [B][P-1][H][dk][trans_ld(dk)], Sst [B][P][H][dv][dk];
-// grid (dv / 16, H, B), sc_threads(DK) threads, sc_smem_bytes(DK) shared.
-template <int DK>
+// E [B][NE][H][dv][dk], A [B][NE][H][dk][trans_ld(dk)], Sst [B][P][H][dv][dk],
+// NE = P (FINAL) or P - 1; grid (dv / 16, H, B), sc_threads(DK) threads,
+// sc_smem_bytes(DK) shared.
+template <int DK, bool FINAL>
 __global__ void __launch_bounds__(4 * DK)
 seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, const float* S0,
-                   float* __restrict__ Sst, int P, int H, int dv) {
+                   float* __restrict__ Sst, float* S_out, int P, int H, int dv) {
     static_assert(DK % 8 == 0 && DK <= 128, "dk");
+    const int NE = FINAL ? P : P - 1;            // segments with an end state / transition
+    const int last = FINAL ? P - 1 : P - 2;      // the last step p computes S_start(p + 1)
     constexpr int LDE = sc_lde(DK);
     extern __shared__ __align__(128) float scm[];
     constexpr int LDAT = pfws::trans_ld(DK);
@@ -77,9 +76,12 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3, n0 = warp * 8;
     const int r0 = blockIdx.x * SC_ROWS, h = blockIdx.y, b = blockIdx.z;
-    auto e_at = [&](int p) { return E + ((((long long)b * (P - 1) + p) * H + h) * dv + r0) * DK; };
-    auto s_at = [&](int p) { return Sst + ((((long long)b * P + p) * H + h) * dv + r0) * DK; };
-    auto a_at = [&](int p) { return A + (((long long)b * (P - 1) + p) * H + h) * DK * LDAT; };
+    auto e_at = [&](int p) { return E + ((((long long)b * NE + p) * H + h) * dv + r0) * DK; };
+    auto s_at = [&](int p) {                     // S_start(p); S_start(P) is the final state (FINAL)
+        return (FINAL && p == P) ? S_out + (((long long)b * H + h) * dv + r0) * DK
+                                 : Sst + ((((long long)b * P + p) * H + h) * dv + r0) * DK;
+    };
+    auto a_at = [&](int p) { return A + (((long long)b * NE + p) * H + h) * DK * LDAT; };
     // this thread's accumulator entries: rows g and g+8, columns n0+2t and n0+2t+1
     auto load_frag = [&](const float* src, float* d) {
         const float2 x = *reinterpret_cast<const float2*>(src + g * DK + n0 + 2 * t);
@@ -94,12 +96,12 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
     }
     __syncthreads();
     if (tid == 0)
-        for (int p = 1; p <= 2 && p + 1 < P; ++p) {
+        for (int p = 1; p <= 2 && p <= last; ++p) {
             sm100::mbar_expect_tx(&bar[p - 1], ABYTES);
             sm100::bulk_load(As + (p - 1) * DK * LDAT, a_at(p), ABYTES, &bar[p - 1]);
         }
-    // S_start(0) = S0 (or zeros); S_start(1) = E_0, also the running rows of step 1
-    const float* s0 = S0 ? S0 + (((long long)b * H + h) * dv + r0) * DK : nullptr;
+    // two passes: S_start(0) = S0 (or zeros); both: S_start(1) = E_0, also the running rows of step 1
+    const float* s0 = (!FINAL && S0) ? S0 + (((long long)b * H + h) * dv + r0) * DK : nullptr;
     {   // every thread owns 4 of the 16 x DK entries; all loads first, then the stores
         constexpr int PER = SC_ROWS / 4;
         float xs[PER], x0[PER];
@@ -112,20 +114,20 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
 #pragma unroll
         for (int u = 0; u < PER; ++u) {
             const int i = tid + u * 4 * DK;
-            s_at(0)[i] = x0[u];
+            if (!FINAL) s_at(0)[i] = x0[u];
             s_at(1)[i] = xs[u];
             put_row(1, i / DK, i % DK, xs[u]);
         }
     }
     float e_next[4] = {0.f, 0.f, 0.f, 0.f};
-    if (P > 2) load_frag(e_at(1), e_next);
+    if (1 <= last) load_frag(e_at(1), e_next);
     __syncthreads();
 
-    for (int p = 1; p + 1 < P; ++p) {
+    for (int p = 1; p <= last; ++p) {
         const int buf = (p - 1) & 1;
         const uint32_t parity = ((p - 1) >> 1) & 1;
         float d[4] = {e_next[0], e_next[1], e_next[2], e_next[3]};
-        if (p + 2 < P) load_frag(e_at(p + 1), e_next);      // in flight during this step
+        if (p + 1 <= last) load_frag(e_at(p + 1), e_next);  // in flight during this step
         const bool ok = sm100::mbar_wait(&bar[buf], parity);
         if (!__syncthreads_and(ok)) return;                  // timed out: error word already set
         const float* Ab = As + buf * DK * LDAT;
@@ -159,7 +161,7 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
         *reinterpret_cast<float2*>(sp + g * DK + n0 + 2 * t) = make_float2(d[0], d[1]);
         *reinterpret_cast<float2*>(sp + (g + 8) * DK + n0 + 2 * t) = make_float2(d[2], d[3]);
         __syncthreads();                              // every read of As[buf] and of the old rows done
-        if (tid == 0 && p + 3 < P) {                  // A_{p+2} is used by step p + 2 <= P - 2
+        if (tid == 0 && p + 2 <= last) {              // A_{p+2} is used by step p + 2
             sm100::mbar_expect_tx(&bar[buf], ABYTES);
             sm100::bulk_load(As + buf * DK * LDAT, a_at(p + 2), ABYTES, &bar[buf]);
         }

@@ -126,14 +126,30 @@ def test_workspace_query_is_host_only(lib):
         assert prefill(lib, B=1, T=4096, H=12, dk=96, dv=256, ws=None, wsb=0) == WORKSPACE
 
 
-@pytest.mark.parametrize("B,T,H,dk,dv,img", [(1, 4096, 12, 96, 256, 48128), (2, 1553, 2, 64, 128, 35840),
-                                             (1, 65536, 16, 128, 256, 52224), (3, 100, 2, 96, 256, 48128)])
-def test_workspace_sizes(lib, B, T, H, dk, dv, img):
-    # fastest plan = one image per (sequence, head, 64-token chunk) + the segment buffers
+def one_pass_bytes(B, T, H, dk, dv, P):
+    """Segment buffers of the one-pass plan: end states E and start states [B][P][H][dv][dk] and
+    transitions [B][P][H][dk][dk+8] (float32), output corrections [B][H][chunks][64][dk] (bf16),
+    each part rounded up to 1024 bytes (none when P = 1)."""
+    if P == 1:
+        return 0
+    up = lambda x: -(-x // 1024) * 1024
+    nct = -(-T // 64)
+    return 2 * up(4 * B * P * H * dv * dk) + up(4 * B * P * H * dk * (dk + 8)) + up(2 * B * H * nct * 64 * dk)
+
+
+@pytest.mark.parametrize("B,T,H,dk,dv,img,P", [(1, 4096, 12, 96, 256, 48128, 4), (2, 1553, 2, 64, 128, 35840, 3),
+                                               (1, 65536, 16, 128, 256, 52224, 3), (3, 100, 2, 96, 256, 48128, 1)])
+def test_workspace_sizes(lib, B, T, H, dk, dv, img, P):
+    # fastest plan = one image per (sequence, head, 64-token chunk) + the one-pass segment buffers,
+    # P segments in one launch of B H (2 P - 1 + ...) CTAs within 148 SMs (value slices of every
+    # segment + a transition slice for each segment after the first)
     lo = jet.jet_gdn_prefill_workspace_min(B, T, H, dk, dv)
     hi = jet.jet_gdn_prefill_workspace_size(B, T, H, dk, dv)
-    assert hi == lo + B * H * ((T + 63) // 64) * img
-    assert lo % 256 == 0 and (hi - lo) % 1024 == 0
+    assert hi == B * H * ((T + 63) // 64) * img + one_pass_bytes(B, T, H, dk, dv, P)
+    ns = dv // 128
+    assert B * H * (ns * P + P - 1) <= 148 and (P == 1 or B * H * (ns * (P + 1) + P) > 148 or
+                                                 -(-T // 64) // (P + 1) < 8)
+    assert lo % 256 == 0 and hi % 1024 == 0
     # a workspace below the minimum is refused before anything runs
     if lo > 0:
         assert prefill(lib, B=B, T=T, H=H, dk=dk, dv=dv, ws=A, wsb=lo - 16) == WORKSPACE
