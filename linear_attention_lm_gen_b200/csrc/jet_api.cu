@@ -248,9 +248,9 @@ size_t seg_workspace_floats(int B, int H, int dk, int dv, int P) {
          + (size_t)B * P * H * dv * dk;           // start states
 }
 // segment buffers of the one-pass plan, each part 1024-byte aligned:
-// E [B][P][H][dv][dk], A [B][P][H][dk][dk+8], S_start [B][P][H][dv][dk]
-// (float32), Qe [B][H][nct][64][dk] (bf16)
-struct OnePassLayout { size_t E, A, Sst, Qe, bytes; };
+// E [B][P][H][dv][dk], A [B][P][H][dk][dk+8] (float32), start states Sb
+// [B][P][H][dv][dk] and Qe [B][H][nct][64][dk] (bf16)
+struct OnePassLayout { size_t E, A, Sb, Qe, bytes; };
 OnePassLayout one_pass_layout(int B, int T, int H, int dk, int dv, int P) {
     auto up = [](size_t x) { return (x + 1023) & ~size_t(1023); };
     OnePassLayout l{0, 0, 0, 0, 0};
@@ -258,8 +258,8 @@ OnePassLayout one_pass_layout(int B, int T, int H, int dk, int dv, int P) {
     const size_t nct = (size_t)((T + 63) / 64);
     l.E = 0;
     l.A = l.E + up(sizeof(float) * B * P * H * (size_t)dv * dk);
-    l.Sst = l.A + up(sizeof(float) * B * P * H * (size_t)dk * pfws::trans_ld(dk));
-    l.Qe = l.Sst + up(sizeof(float) * B * P * H * (size_t)dv * dk);
+    l.Sb = l.A + up(sizeof(float) * B * P * H * (size_t)dk * pfws::trans_ld(dk));
+    l.Qe = l.Sb + up(sizeof(__nv_bfloat16) * B * P * H * (size_t)dv * dk);
     l.bytes = l.Qe + up(sizeof(__nv_bfloat16) * B * H * nct * 64 * (size_t)dk);
     return l;
 }
@@ -286,12 +286,12 @@ size_t split_img_bytes(int B, int T, int H, int dk) {
 // conv with `taps` into the chunk images and the chain reads the values
 // before each segment (and the history of `cv`) for it.
 template <int DK, int DV>
-jet_status launch_correct(const __nv_bfloat16* Qe, const float* Sst, void* o, int B, int Tn, int H, int nct,
+jet_status launch_correct(const __nv_bfloat16* Qe, const __nv_bfloat16* Sb, void* o, int B, int Tn, int H, int nct,
                           int segc, int P, cudaStream_t s) {
     auto kern = pfcor::prefill_correct_kernel<DK, DV>;
     const size_t smem = pfcor::smem_bytes(DK, DV);
     if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
-    kern<<<dim3(nct - segc, H, B), pfcor::THREADS, smem, s>>>(Qe, Sst, (__nv_bfloat16*)o, Tn, H, nct, segc, P);
+    kern<<<dim3(nct - segc, H, B), pfcor::THREADS, smem, s>>>(Qe, Sb, (__nv_bfloat16*)o, Tn, H, nct, segc, P);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return launch_status();
 }
@@ -337,7 +337,7 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
         const OnePassLayout lay = one_pass_layout(B, Tn, H, DK, dv, P);
         float* E = reinterpret_cast<float*>(segws + lay.E);
         float* A = reinterpret_cast<float*>(segws + lay.A);
-        float* Sst = reinterpret_cast<float*>(segws + lay.Sst);
+        __nv_bfloat16* Sb = reinterpret_cast<__nv_bfloat16*>(segws + lay.Sb);
         __nv_bfloat16* Qe = reinterpret_cast<__nv_bfloat16*>(segws + lay.Qe);
         const pfch::ChainSeg seg = P == 1 ? pfch::ChainSeg{1, plan.seg_chunks, nullptr, nullptr, nullptr}
                                           : pfch::ChainSeg{P, plan.seg_chunks, E, A, Qe};
@@ -349,13 +349,13 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
         // start states S*_1 .. S*_{P-1} and the final state
         const size_t sc_smem = sc_smem_bytes(DK);
         if (smem_attr(seg_combine_kernel<DK, true>, sc_smem) != JET_OK) return JET_ERR_CUDA;
-        seg_combine_kernel<DK, true><<<dim3(dv / SC_ROWS, H, B), sc_threads(DK), sc_smem, s>>>(E, A, nullptr, Sst,
-                                                                                              S_out, P, H, dv);
+        seg_combine_kernel<DK, true><<<dim3(dv / SC_ROWS, H, B), sc_threads(DK), sc_smem, s>>>(
+            E, A, nullptr, nullptr, Sb, S_out, P, H, dv);
         g_launches.fetch_add(1, std::memory_order_relaxed);
         if (launch_status() != JET_OK) return JET_ERR_CUDA;
         // outputs of the segments p >= 1: O += Qe S*^T
-        return dv == 256 ? launch_correct<DK, 256>(Qe, Sst, o, B, Tn, H, nct, plan.seg_chunks, P, s)
-                         : launch_correct<DK, 128>(Qe, Sst, o, B, Tn, H, nct, plan.seg_chunks, P, s);
+        return dv == 256 ? launch_correct<DK, 256>(Qe, Sb, o, B, Tn, H, nct, plan.seg_chunks, P, s)
+                         : launch_correct<DK, 128>(Qe, Sb, o, B, Tn, H, nct, plan.seg_chunks, P, s);
     }
     auto fused = pfws::gdn_prefill_ws_kernel<DK>;
     if (smem_attr(fused, pfws::SMEM_BYTES) != JET_OK) return JET_ERR_CUDA;
@@ -379,7 +379,7 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
     const size_t sc_smem = sc_smem_bytes(DK);
     if (smem_attr(seg_combine_kernel<DK, false>, sc_smem) != JET_OK) return JET_ERR_CUDA;
     seg_combine_kernel<DK, false><<<dim3(dv / SC_ROWS, H, B), sc_threads(DK), sc_smem, s>>>(E, A, S0, Sst, nullptr,
-                                                                                           P, H, dv);
+                                                                                           nullptr, P, H, dv);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     if (launch_status() != JET_OK) return JET_ERR_CUDA;
     // phase C: every segment from its start state, with outputs

@@ -14,10 +14,13 @@
 //   warps 0-3  CHAIN  E4: S -> bf16 copy and S <- gam_L S;  E5: Wt^T -> bf16
 //                     (plain and scaled by d/|k|)
 //   warps 4-7  OUT    E6: O^T (TMEM) -> staging -> global, off the chain
-//   warp  8    MMA    one thread issues the MMAs on the state chain (P3, P4)
-//   warp  9    LOAD   one thread issues the bulk copies of the images, the TMA
+//   warp 10    MMA    one thread issues the MMAs on the state chain (P3, P4)
+//   warp 11    LOAD   one thread issues the bulk copies of the images, the TMA
 //                     loads of K and V as soon as their buffers are free, and
 //                     the MMAs off the chain (P2a, P5a, P5b)
+//   (warps 8 and 9 have no role: the issuing threads sit on the schedulers of
+//   warps 2 and 3, away from the group pollers of warps 0 and 4, so that a
+//   spinning poller does not take issue slots from the MMA issue)
 //
 // Buffers: images double-buffered (the copy of chunk c+2 starts once chunk c
 // is finished), V double-buffered (V(c+2) once P2a(c) is done), K
@@ -60,8 +63,8 @@ namespace pfch {
 using namespace pfws;
 
 constexpr int NCH_T = 128, NOUT = 128;
-constexpr int THREADS = NCH_T + NOUT + 64;            // 320
-constexpr int OUT0 = NCH_T, MMA0 = NCH_T + NOUT, LOAD0 = MMA0 + 32;
+constexpr int THREADS = NCH_T + NOUT + 128;           // 384
+constexpr int OUT0 = NCH_T, MMA0 = NCH_T + NOUT + 64, LOAD0 = MMA0 + 32;   // warps 10 and 11
 
 // bounded wait: spin on the phase first, then poll with short sleeps; gives up
 // (error word + CTA abort flag) when the poll budget runs out or another

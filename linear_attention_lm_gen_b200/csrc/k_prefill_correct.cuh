@@ -14,10 +14,11 @@
 // One CTA per (sequence, head, chunk): a 64 x dv by dk product on the tensor
 // cores (bf16 mma.sync m16n8k16, float32 accumulate; 2 x 1.6 Mflop per chunk
 // is far too small a tile for tcgen05, and the kernel is bound by moving the
-// 32 KB output tile). The Qe tile, S* (float32, rounded to bf16 on the way
-// into shared memory) and the output tile are staged in shared memory with
-// padded rows (conflict-free ldmatrix), then the output is written back with
-// 16-byte stores. Warp w owns output columns [w dv/8, (w+1) dv/8).
+// 32 KB output tile). The Qe tile, S* (in bf16, as the segment combine wrote
+// it) and the output tile are copied into shared memory by 16-byte cp.async
+// all at once (padded rows: conflict-free ldmatrix), then the output is
+// written back with 16-byte stores. Warp w owns output columns
+// [w dv/8, (w+1) dv/8).
 #pragma once
 #include "common.cuh"
 
@@ -40,6 +41,10 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
 __device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t* r) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
 }
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                 :: "r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))), "l"(src), "r"(src_bytes) : "memory");
+}
 __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint32_t* b) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
@@ -48,11 +53,11 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// Qe [B][H][nct][64][DK] bf16; Sst [B][P][H][dv][DK] float32 (entries p >= 1);
+// Qe [B][H][nct][64][DK] bf16; Sb [B][P][H][dv][DK] bf16 (entries p >= 1);
 // o [B*T][H][dv] bf16 (updated in place). grid (nct - seg_chunks, H, B).
 template <int DK, int DV>
 __global__ void __launch_bounds__(THREADS)
-prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const float* __restrict__ Sst,
+prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16* __restrict__ Sb,
                        __nv_bfloat16* __restrict__ o, int Tn, int H, int nct, int seg_chunks, int P) {
     static_assert(DK % 16 == 0 && DK <= 128 && DV % 64 == 0 && DV <= 256, "shapes");
     constexpr int LDA = lda(DK), LDO = ldo(DV);
@@ -70,31 +75,31 @@ prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const float* __rest
     const long long bh = (long long)b * H + h;
     const long long tstride = (long long)H * DV;
 
-    {   // Qe rows (zero past the sequence end), 16-byte pieces
-        const uint4* src = reinterpret_cast<const uint4*>(Qe + ((size_t)bh * nct + gc) * C * DK);
+    // every copy of the three tiles in flight at once
+    {   // Qe rows (zero past the sequence end: a 0-byte source fills zeros)
+        const __nv_bfloat16* src = Qe + ((size_t)bh * nct + gc) * C * DK;
+#pragma unroll
         for (int i = tid; i < C * DK / 8; i += THREADS) {
             const int r = i / (DK / 8), cc = i % (DK / 8);
-            const uint4 v = r < L ? src[i] : make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(qs + r * LDA + cc * 8) = v;
+            cp_async16(qs + r * LDA + cc * 8, src + (r < L ? i * 8 : 0), r < L ? 16u : 0u);
         }
     }
-    {   // S* of the segment, float32 -> bf16
-        const float4* src = reinterpret_cast<const float4*>(Sst + ((((long long)b * P + p) * H + h) * DV) * DK);
+    {   // S* of the segment
+        const __nv_bfloat16* src = Sb + ((((long long)b * P + p) * H + h) * DV) * DK;
+#pragma unroll
         for (int i = tid; i < DV * DK / 8; i += THREADS) {
             const int r = i / (DK / 8), cc = i % (DK / 8);
-            const float4 a = src[2 * i], c = src[2 * i + 1];
-            const float f[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-            *reinterpret_cast<uint4*>(ss + r * LDA + cc * 8) = Vec16<__nv_bfloat16>::pack(f);
+            cp_async16(ss + r * LDA + cc * 8, src + i * 8, 16u);
         }
     }
-    {   // the provisional outputs of the chunk
+    {   // the provisional outputs of the chunk (rows past the sequence end are never stored)
+#pragma unroll
         for (int i = tid; i < C * DV / 8; i += THREADS) {
             const int r = i / (DV / 8), cc = i % (DV / 8);
-            if (r < L)
-                *reinterpret_cast<uint4*>(os + r * LDO + cc * 8) =
-                    *reinterpret_cast<const uint4*>(o + ((long long)b * Tn + t0 + r) * tstride + h * DV + cc * 8);
+            if (r < L) cp_async16(os + r * LDO + cc * 8, o + ((long long)b * Tn + t0 + r) * tstride + h * DV + cc * 8, 16u);
         }
     }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
     __syncthreads();
 
     // acc[m][n]: rows 16 m + (g, g + 8), columns n0 + 8 n + (2 t, 2 t + 1)

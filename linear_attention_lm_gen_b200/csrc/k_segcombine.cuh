@@ -9,9 +9,9 @@
 //   S_start(1) = E_0,   S_start(p + 1) = S_start(p) A_p + E_p.
 // Two layouts:
 //   one pass (FINAL): E and A hold all P segments; the kernel writes
-//     S_start(1 .. P-1) (the start states the output correction needs) and
-//     the final state S_start(P) to S_out (which may alias S0: segment 0 has
-//     read S0 before this kernel runs);
+//     S_start(1 .. P-1) in bf16 (the operand of the output correction, Sb)
+//     and the final state S_start(P) in float32 to S_out (which may alias S0:
+//     segment 0 has read S0 before this kernel runs);
 //   two passes: E and A hold segments 0 .. P-2 (the pass without outputs);
 //     the kernel writes S_start(0 .. P-1), S_start(0) being a copy of S0 (or
 //     zeros), so that the pass with outputs never reads S0 while the last
@@ -51,13 +51,14 @@ __device__ __forceinline__ void mma(float* d, const uint32_t* a, const uint32_t*
 }
 }  // namespace sc
 
-// E [B][NE][H][dv][dk], A [B][NE][H][dk][trans_ld(dk)], Sst [B][P][H][dv][dk],
-// NE = P (FINAL) or P - 1; grid (dv / 16, H, B), sc_threads(DK) threads,
-// sc_smem_bytes(DK) shared.
+// E [B][NE][H][dv][dk], A [B][NE][H][dk][trans_ld(dk)], NE = P (FINAL) or
+// P - 1; start states Sst [B][P][H][dv][dk] float32 (two passes) or Sb
+// [B][P][H][dv][dk] bf16 (FINAL); grid (dv / 16, H, B), sc_threads(DK)
+// threads, sc_smem_bytes(DK) shared.
 template <int DK, bool FINAL>
 __global__ void __launch_bounds__(4 * DK)
 seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, const float* S0,
-                   float* __restrict__ Sst, float* S_out, int P, int H, int dv) {
+                   float* __restrict__ Sst, __nv_bfloat16* __restrict__ Sb, float* S_out, int P, int H, int dv) {
     static_assert(DK % 8 == 0 && DK <= 128, "dk");
     const int NE = FINAL ? P : P - 1;            // segments with an end state / transition
     const int last = FINAL ? P - 1 : P - 2;      // the last step p computes S_start(p + 1)
@@ -77,10 +78,11 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
     const int g = lane >> 2, t = lane & 3, n0 = warp * 8;
     const int r0 = blockIdx.x * SC_ROWS, h = blockIdx.y, b = blockIdx.z;
     auto e_at = [&](int p) { return E + ((((long long)b * NE + p) * H + h) * dv + r0) * DK; };
-    auto s_at = [&](int p) {                     // S_start(p); S_start(P) is the final state (FINAL)
+    auto s_at = [&](int p) {                     // S_start(p) (two passes); the final state (FINAL)
         return (FINAL && p == P) ? S_out + (((long long)b * H + h) * dv + r0) * DK
                                  : Sst + ((((long long)b * P + p) * H + h) * dv + r0) * DK;
     };
+    auto sb_at = [&](int p) { return Sb + ((((long long)b * P + p) * H + h) * dv + r0) * DK; };
     auto a_at = [&](int p) { return A + (((long long)b * NE + p) * H + h) * DK * LDAT; };
     // this thread's accumulator entries: rows g and g+8, columns n0+2t and n0+2t+1
     auto load_frag = [&](const float* src, float* d) {
@@ -114,8 +116,12 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
 #pragma unroll
         for (int u = 0; u < PER; ++u) {
             const int i = tid + u * 4 * DK;
-            if (!FINAL) s_at(0)[i] = x0[u];
-            s_at(1)[i] = xs[u];
+            if (!FINAL) {
+                s_at(0)[i] = x0[u];
+                s_at(1)[i] = xs[u];
+            } else if (P > 1) {
+                sb_at(1)[i] = __float2bfloat16_rn(xs[u]);
+            }
             put_row(1, i / DK, i % DK, xs[u]);
         }
     }
@@ -157,9 +163,15 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
         put_row(p + 1, g, n0 + 2 * t + 1, d[1]);
         put_row(p + 1, g + 8, n0 + 2 * t, d[2]);
         put_row(p + 1, g + 8, n0 + 2 * t + 1, d[3]);
-        float* sp = s_at(p + 1);
-        *reinterpret_cast<float2*>(sp + g * DK + n0 + 2 * t) = make_float2(d[0], d[1]);
-        *reinterpret_cast<float2*>(sp + (g + 8) * DK + n0 + 2 * t) = make_float2(d[2], d[3]);
+        if (FINAL && p + 1 < P) {                     // a start state: the correction's bf16 operand
+            __nv_bfloat16* sp = sb_at(p + 1);
+            *reinterpret_cast<__nv_bfloat162*>(sp + g * DK + n0 + 2 * t) = __floats2bfloat162_rn(d[0], d[1]);
+            *reinterpret_cast<__nv_bfloat162*>(sp + (g + 8) * DK + n0 + 2 * t) = __floats2bfloat162_rn(d[2], d[3]);
+        } else {                                      // float32: a start state (two passes) or the final state
+            float* sp = s_at(p + 1);
+            *reinterpret_cast<float2*>(sp + g * DK + n0 + 2 * t) = make_float2(d[0], d[1]);
+            *reinterpret_cast<float2*>(sp + (g + 8) * DK + n0 + 2 * t) = make_float2(d[2], d[3]);
+        }
         __syncthreads();                              // every read of As[buf] and of the old rows done
         if (tid == 0 && p + 2 <= last) {              // A_{p+2} is used by step p + 2
             sm100::mbar_expect_tx(&bar[buf], ABYTES);

@@ -127,14 +127,15 @@ def test_workspace_query_is_host_only(lib):
 
 
 def one_pass_bytes(B, T, H, dk, dv, P):
-    """Segment buffers of the one-pass plan: end states E and start states [B][P][H][dv][dk] and
-    transitions [B][P][H][dk][dk+8] (float32), output corrections [B][H][chunks][64][dk] (bf16),
-    each part rounded up to 1024 bytes (none when P = 1)."""
+    """Segment buffers of the one-pass plan: end states E [B][P][H][dv][dk] and transitions
+    [B][P][H][dk][dk+8] (float32), start states [B][P][H][dv][dk] and output corrections
+    [B][H][chunks][64][dk] (bf16), each part rounded up to 1024 bytes (none when P = 1)."""
     if P == 1:
         return 0
     up = lambda x: -(-x // 1024) * 1024
     nct = -(-T // 64)
-    return 2 * up(4 * B * P * H * dv * dk) + up(4 * B * P * H * dk * (dk + 8)) + up(2 * B * H * nct * 64 * dk)
+    return up(4 * B * P * H * dv * dk) + up(4 * B * P * H * dk * (dk + 8)) + up(2 * B * P * H * dv * dk) \
+        + up(2 * B * H * nct * 64 * dk)
 
 
 @pytest.mark.parametrize("B,T,H,dk,dv,img,P", [(1, 4096, 12, 96, 256, 48128, 4), (2, 1553, 2, 64, 128, 35840, 3),
