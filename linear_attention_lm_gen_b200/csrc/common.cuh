@@ -15,6 +15,18 @@ __device__ int g_dev_error;
 
 __device__ __forceinline__ void flag_error(int bits) { atomicOr(&g_dev_error, bits); }
 
+// Programmatic dependent launch. Every kernel of the library is launched with
+// programmatic stream serialization allowed, so it may be scheduled while the
+// previous kernel on the stream is still running. pdl_wait() blocks until
+// that kernel (and so all earlier work on the stream) has completed and its
+// writes are visible; a kernel calls it before its first read of global
+// memory, after its purely local set-up (barrier init, TMEM allocation,
+// descriptor prefetch). pdl_trigger() lets the next kernel be scheduled early;
+// the next kernel's own pdl_wait still waits for this one to finish. Both are
+// no-ops when the launch had no such dependency.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- element access for the two storage dtypes --------------------------
 template <typename T> struct Elem;
 template <> struct Elem<float> {

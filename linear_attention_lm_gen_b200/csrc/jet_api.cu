@@ -58,6 +58,27 @@ jet_status launch_status() {
     return e == cudaSuccess ? JET_OK : JET_ERR_CUDA;
 }
 
+// Launch with programmatic stream serialization allowed (the kernels wait
+// for the previous kernel on the stream with pdl_wait before reading global
+// memory), counting the launch.
+template <typename... KArgs, typename... Args>
+jet_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (e != cudaSuccess) return JET_ERR_CUDA;
+    return launch_status();
+}
+
 // opt a kernel into more than 48 KB of dynamic shared memory
 template <typename K>
 jet_status smem_attr(K kernel, size_t bytes) {
@@ -83,13 +104,15 @@ jet_status launch_genconv_t(const void* x, const void* w1, const void* w2, const
     cfg.blockDim = dim3(GC_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 1;
     attr[0].val.clusterDim.y = (unsigned)groups;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, (const T*)x, (const T*)w1, (const T*)w2, (const T*)v,
                                              (const T*)hin, (T*)vout, (T*)hout, cw, B, Tn, D, H, dv, hpc, slots,
                                              n_slots);
@@ -127,10 +150,8 @@ jet_status launch_gen(const void* x, const void* w1, const void* w2, float* taps
     const int HW4 = H * GC_W;
     const size_t smem = kgen::smem_bytes(HW4);
     if (smem_attr(kgen::gen_kernel, smem) != JET_OK) return JET_ERR_CUDA;
-    kgen::gen_kernel<<<(unsigned)((N + kgen::GT - 1) / kgen::GT), kgen::THREADS, smem, s>>>(
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w1, (const __nv_bfloat16*)w2, taps, N, D, HW4);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return launch_status();
+    return launch(kgen::gen_kernel, dim3((unsigned)((N + kgen::GT - 1) / kgen::GT)), dim3(kgen::THREADS), smem, s,
+                  (const __nv_bfloat16*)x, (const __nv_bfloat16*)w1, (const __nv_bfloat16*)w2, taps, N, D, HW4);
 }
 // prompts long enough to fill the GPU with 32-token CTAs take the stand-alone generator
 constexpr long long kGenMinTokens = 1024;
@@ -155,10 +176,8 @@ jet_status launch_prefill_simt(const void* q, const void* k, const void* v, cons
     const size_t smem = sizeof(float) * ps_smem_floats(DK);
     auto kern = gdn_prefill_simt_kernel<T, DK>;
     if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
-    dim3 grid(dv / PS_DVS, H, B);
-    kern<<<grid, PS_THREADS, smem, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta, S0, (T*)o, S_out, Tn, H, dv);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return launch_status();
+    return launch(kern, dim3(dv / PS_DVS, H, B), dim3(PS_THREADS), smem, s, (const T*)q, (const T*)k, (const T*)v, g,
+                  beta, S0, (T*)o, S_out, Tn, H, dv);
 }
 
 // ---- TMA descriptors (driver entry point fetched once through the runtime)
@@ -291,9 +310,8 @@ jet_status launch_correct(const __nv_bfloat16* Qe, const __nv_bfloat16* Sb, void
     auto kern = pfcor::prefill_correct_kernel<DK, DV>;
     const size_t smem = pfcor::smem_bytes(DK, DV);
     if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
-    kern<<<dim3(nct - segc, H, B), pfcor::THREADS, smem, s>>>(Qe, Sb, (__nv_bfloat16*)o, Tn, H, nct, segc, P);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return launch_status();
+    return launch(kern, dim3(nct - segc, H, B), dim3(pfcor::THREADS), smem, s, Qe, Sb, (__nv_bfloat16*)o, Tn, H, nct,
+                  segc, P);
 }
 
 template <int DK, bool SPLIT, bool CONV = false>
@@ -327,10 +345,9 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
             if (smem_attr(prep, pfws::PrepSmem<DK>::BYTES) != JET_OK) return JET_ERR_CUDA;
             const long long items = (long long)B * H * nct;
             const int grid = (int)std::min<long long>(items, (long long)pfws::PREP_CTAS * sms);   // resident CTAs
-            prep<<<grid, pfws::PREP_THREADS, pfws::PrepSmem<DK>::BYTES, s>>>(
-                mq, mk, g, beta, CONV ? taps : nullptr, cv.hist_in != nullptr, img, Tn, H, nct, (int)items);
-            g_launches.fetch_add(1, std::memory_order_relaxed);
-            if (launch_status() != JET_OK) return JET_ERR_CUDA;
+            if (launch(prep, dim3(grid), dim3(pfws::PREP_THREADS), pfws::PrepSmem<DK>::BYTES, s, mq, mk, g, beta,
+                       CONV ? taps : nullptr, (int)(cv.hist_in != nullptr), img, Tn, H, nct, (int)items) != JET_OK)
+                return JET_ERR_CUDA;
         }
         const SegPlan plan = plan_one_pass(B, Tn, H, dv, sms);
         const int P = plan.P;
@@ -341,18 +358,17 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
         __nv_bfloat16* Qe = reinterpret_cast<__nv_bfloat16*>(segws + lay.Qe);
         const pfch::ChainSeg seg = P == 1 ? pfch::ChainSeg{1, plan.seg_chunks, nullptr, nullptr, nullptr}
                                           : pfch::ChainSeg{P, plan.seg_chunks, E, A, Qe};
-        chain<<<dim3(ns + (P > 1 ? 1 : 0), H, B * P), pfch::THREADS, smem, s>>>(
-            mk, mv, mvh, mhh, img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg, cv);
-        g_launches.fetch_add(1, std::memory_order_relaxed);
-        if (launch_status() != JET_OK) return JET_ERR_CUDA;
+        if (launch(chain, dim3(ns + (P > 1 ? 1 : 0), H, B * P), dim3(pfch::THREADS), smem, s, mk, mv, mvh, mhh,
+                   (const uint8_t*)img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg, cv) != JET_OK)
+            return JET_ERR_CUDA;
         if (P == 1) return JET_OK;
         // start states S*_1 .. S*_{P-1} and the final state
         const size_t sc_smem = sc_smem_bytes(DK);
         if (smem_attr(seg_combine_kernel<DK, true>, sc_smem) != JET_OK) return JET_ERR_CUDA;
-        seg_combine_kernel<DK, true><<<dim3(dv / SC_ROWS, H, B), sc_threads(DK), sc_smem, s>>>(
-            E, A, nullptr, nullptr, Sb, S_out, P, H, dv);
-        g_launches.fetch_add(1, std::memory_order_relaxed);
-        if (launch_status() != JET_OK) return JET_ERR_CUDA;
+        if (launch(seg_combine_kernel<DK, true>, dim3(dv / SC_ROWS, H, B), dim3(sc_threads(DK)), sc_smem, s,
+                   (const float*)E, (const float*)A, (const float*)nullptr, (float*)nullptr, Sb, S_out, P, H,
+                   dv) != JET_OK)
+            return JET_ERR_CUDA;
         // outputs of the segments p >= 1: O += Qe S*^T
         return dv == 256 ? launch_correct<DK, 256>(Qe, Sb, o, B, Tn, H, nct, plan.seg_chunks, P, s)
                          : launch_correct<DK, 128>(Qe, Sb, o, B, Tn, H, nct, plan.seg_chunks, P, s);
@@ -361,10 +377,8 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
     if (smem_attr(fused, pfws::SMEM_BYTES) != JET_OK) return JET_ERR_CUDA;
     float* ws = reinterpret_cast<float*>(workspace);
     auto run = [&](dim3 grid, const pfws::Seg& seg) {
-        fused<<<grid, pfws::THREADS, pfws::SMEM_BYTES, s>>>(mq, mk, mv, g, beta, S0, (__nv_bfloat16*)o, S_out, Tn, H,
-                                                            dv, seg);
-        g_launches.fetch_add(1, std::memory_order_relaxed);
-        return launch_status();
+        return launch(fused, grid, dim3(pfws::THREADS), pfws::SMEM_BYTES, s, mq, mk, mv, g, beta, S0,
+                      (__nv_bfloat16*)o, S_out, Tn, H, dv, seg);
     };
     const SegPlan plan = plan_two_pass(B, Tn, H, dv, sms);
     const int P = plan.P;
@@ -378,10 +392,10 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
     // start states of every segment (S0 copied for segment 0)
     const size_t sc_smem = sc_smem_bytes(DK);
     if (smem_attr(seg_combine_kernel<DK, false>, sc_smem) != JET_OK) return JET_ERR_CUDA;
-    seg_combine_kernel<DK, false><<<dim3(dv / SC_ROWS, H, B), sc_threads(DK), sc_smem, s>>>(E, A, S0, Sst, nullptr,
-                                                                                           nullptr, P, H, dv);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    if (launch_status() != JET_OK) return JET_ERR_CUDA;
+    if (launch(seg_combine_kernel<DK, false>, dim3(dv / SC_ROWS, H, B), dim3(sc_threads(DK)), sc_smem, s,
+               (const float*)E, (const float*)A, S0, Sst, (__nv_bfloat16*)nullptr, (float*)nullptr, P, H,
+               dv) != JET_OK)
+        return JET_ERR_CUDA;
     // phase C: every segment from its start state, with outputs
     return run(dim3(ns, H, B * P), pfws::Seg{P, plan.seg_chunks, P, 0, Sst, nullptr, nullptr});
 }
@@ -404,15 +418,12 @@ template <typename T, int NV>
 jet_status launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float* S, void* o, int B, int H, int dv, const DecConv* conv, cudaStream_t s,
                          const int* slots, int n_slots) {
-    dim3 grid((dv + DEC_ROWS - 1) / DEC_ROWS, H, B);
+    const dim3 grid((dv + DEC_ROWS - 1) / DEC_ROWS, H, B);
     if (conv)
-        gdn_decode_kernel<T, NV, true><<<grid, DEC_THREADS, 0, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta,
-                                                                    S, (T*)o, H, dv, *conv, slots, n_slots);
-    else
-        gdn_decode_kernel<T, NV><<<grid, DEC_THREADS, 0, s>>>((const T*)q, (const T*)k, (const T*)v, g, beta, S,
-                                                            (T*)o, H, dv, DecConv{}, slots, n_slots);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return launch_status();
+        return launch(gdn_decode_kernel<T, NV, true>, grid, dim3(DEC_THREADS), 0, s, (const T*)q, (const T*)k,
+                      (const T*)v, g, beta, S, (T*)o, H, dv, *conv, slots, n_slots);
+    return launch(gdn_decode_kernel<T, NV>, grid, dim3(DEC_THREADS), 0, s, (const T*)q, (const T*)k, (const T*)v, g,
+                  beta, S, (T*)o, H, dv, DecConv{}, slots, n_slots);
 }
 
 template <typename T>

@@ -57,6 +57,8 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.y, b = blockIdx.z;
     const long long bh = (long long)b * H + h;                // token inputs and outputs
+    pdl_wait();
+    pdl_trigger();
     int sb = b;                                               // state / history entry
     if (slots) {
         sb = slots[b];

@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(THREADS)
 gen_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ W1,
            const __nv_bfloat16* __restrict__ W2, float* __restrict__ taps, long long N, int D, int HW4) {
     extern __shared__ __align__(16) uint8_t smem[];
+    pdl_wait();
+    pdl_trigger();
     float* hs = reinterpret_cast<float*>(smem + NST * ST_BYTES);          // [GT][HLD] hidden activations
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long r0 = (long long)blockIdx.x * GT;

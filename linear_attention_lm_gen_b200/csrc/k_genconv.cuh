@@ -149,6 +149,8 @@ genconv_kernel(const T* __restrict__ x, const T* __restrict__ W1, const T* __res
                int Bn, int Tn, int D, int H, int dv, int hpc, const int* __restrict__ slots = nullptr,
                int n_slots = 0) {
     extern __shared__ float smem[];
+    pdl_wait();
+    pdl_trigger();
     const int HW4 = H * GC_W;
     const int h0 = blockIdx.y * hpc;
     const int nh = max(0, min(hpc, H - h0));

@@ -12,15 +12,16 @@
 // state lives in TMEM, its bf16 copy is the A operand of P3 / P5a.
 //
 //   warps 0-3  CHAIN  E4: S -> bf16 copy and S <- gam_L S;  E5: Wt^T -> bf16
-//                     (plain and scaled by d/|k|)
+//                     (plain and scaled by d/|k|); after each of them the
+//                     group's first thread issues the MMAs on the state chain
+//                     itself (P3 after E4, P4 after E5), so no handoff to
+//                     another thread sits on the chain
 //   warps 4-7  OUT    E6: O^T (TMEM) -> staging -> global, off the chain
-//   warp 10    MMA    one thread issues the MMAs on the state chain (P3, P4)
-//   warp 11    LOAD   one thread issues the bulk copies of the images, the TMA
+//   warp 10    LOAD   one thread issues the bulk copies of the images, the TMA
 //                     loads of K and V as soon as their buffers are free, and
 //                     the MMAs off the chain (P2a, P5a, P5b)
-//   (warps 8 and 9 have no role: the issuing threads sit on the schedulers of
-//   warps 2 and 3, away from the group pollers of warps 0 and 4, so that a
-//   spinning poller does not take issue slots from the MMA issue)
+//   (warps 8 and 9 have no role: the load thread sits on the scheduler of
+//   warp 2, away from the group pollers of warps 0 and 4)
 //
 // Buffers: images double-buffered (the copy of chunk c+2 starts once chunk c
 // is finished), V double-buffered (V(c+2) once P2a(c) is done), K
@@ -63,8 +64,8 @@ namespace pfch {
 using namespace pfws;
 
 constexpr int NCH_T = 128, NOUT = 128;
-constexpr int THREADS = NCH_T + NOUT + 128;           // 384
-constexpr int OUT0 = NCH_T, MMA0 = NCH_T + NOUT + 64, LOAD0 = MMA0 + 32;   // warps 10 and 11
+constexpr int THREADS = NCH_T + NOUT + 96;            // 352
+constexpr int OUT0 = NCH_T, LOAD0 = NCH_T + NOUT + 64;   // warp 10
 
 // bounded wait: spin on the phase first, then poll with short sleeps; gives up
 // (error word + CTA abort flag) when the poll budget runs out or another
@@ -198,10 +199,24 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = *tslot;
+    pdl_wait();                                           // images, S0, K and V are read from here on
+    pdl_trigger();
+
+    const uint64_t dAS = sw128_desc(smem_u32(sm + SM::AS), 16, 1024);
+    auto as_off = [&](int kk) { return (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4); };
+    auto ioff = [&](int c, uint32_t off) { return (uint64_t)((((uint32_t)(c & 1) * SM::IB) + off) >> 4); };
 
     if (warp < 4) {
         // =============================================================== CHAIN
         const int ct = tid;
+        constexpr int NKBUF = SM::NKBUF;
+        const uint64_t dImgMN = sw128_desc(smem_u32(sm + SM::IMG), 8192, 1024);   // W^T (MN-major)
+        const uint64_t dKmn = sw128_desc(smem_u32(sm + SM::K), 8192, 1024);       // K as MN-major
+        const uint64_t dAWD = sw128_desc(smem_u32(sm + SM::AWD), 16, 1024);
+        constexpr uint32_t ID_NEG = idesc_bf16(128, 64, false, true, true);
+        constexpr uint32_t ID_S = idesc_bf16(128, DK, false, true);
+        int n3 = 0, n4 = 0;                                  // commit groups issued (thread 0)
+        bool live = true;                                    // thread 0: every wait so far succeeded
         const uint32_t lb = (uint32_t)(warp * 32) << 16;
         {   // initial state (row ct of the slice)
             const float* src = (p_seg == 0 && !trans && S0) ? S0 + (bh * dv + c0 + ct) * DK : nullptr;
@@ -221,7 +236,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             bool okw = true;
             if (ct == 0) {
                 // S updated (P4), the bf16 S copy and Wt^T no longer read (P5a / P5b), image landed
-                okw = c < 1 || wait_spin(&bars[B_SDONE + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag);
+                okw = live && (c < 1 || wait_spin(&bars[B_SDONE + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag));
                 okw = okw && (c < 1 || !write_o ||
                               wait_spin(&bars[B_ODONE + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag));
                 okw = okw && wait_spin(&bars[B_IMG + p], (c >> 1) & 1, abort_flag);
@@ -253,9 +268,25 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             fence_async_smem();
             tc_fence_before();
             named_sync(2, NCH_T);
-            if (ct == 0) arrive(&bars[B_AS]);
+            // ---- P3 (thread 0): X1[c&1] -= S W^T  (= Wt^T), once U^T of the chunk is in X1
+            bool okp = true;
+            if (ct == 0) {
+                arrive(&bars[B_AS]);                         // for the output product P5a
+                okp = wait_spin(&bars[B_P2 + (c & 1)], (c >> 1) & 1, abort_flag);
+                if (okp) {
+                    tc_fence_after();
+                    const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+                    for (int kk = 0; kk < KSTEPS; ++kk)
+                        mma_bf16_ss(tb + x1, dAS + as_off(kk), dImgMN + ioff(c, IM::WT + kk * 2048), ID_NEG, 1);
+                    mma_commit(&bars[B_P3]);
+                    ++n3;
+                    okp = wait_spin(&bars[B_P3], c & 1, abort_flag);
+                }
+                live = okp;
+            }
             // ---- E5: Wt^T -> bf16 (plain and scaled by d/|k|)
-            if (!group_wait(&bars[B_P3], c & 1, abort_flag, 2, NCH_T, ct == 0, true)) break;
+            if (!group_all(2, NCH_T, okp)) break;
             tc_fence_after();
             {
                 const uint32_t x1 = TM_X1 + (uint32_t)p * 64;
@@ -284,12 +315,25 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             fence_async_smem();
             tc_fence_before();
             named_sync(2, NCH_T);
-            if (ct == 0) arrive(&bars[B_AW]);
+            // ---- P4 (thread 0): S += Wt^T diag(d/|k|) K, once the K tile is in
+            if (ct == 0) {
+                arrive(&bars[B_AW]);                         // for the output product P5b
+                live = wait_spin(&bars[B_K + c % NKBUF], (c / NKBUF) & 1, abort_flag);
+                if (live) {
+                    tc_fence_after();
+                    const uint64_t dk_ = dKmn + (uint64_t)(((uint32_t)(c % NKBUF) * NKB * 8192) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tb + TM_S, dAWD + (uint64_t)(kk * 32 >> 4), dk_ + (uint64_t)(kk * 2048 >> 4), ID_S, 1);
+                    mma_commit(&bars[B_SDONE + (c & 1)]);
+                    ++n4;
+                }
+            }
         }
         // final state of the segment (after the last P4)
         bool fin = true;
         if (ct == 0)
-            fin = !*abort_flag && nch > 0 &&
+            fin = live && !*abort_flag && nch > 0 && n4 == nch &&
                   wait_spin(&bars[B_SDONE + ((nch - 1) & 1)], ((nch - 1) >> 1) & 1, abort_flag);
         if (group_all(2, NCH_T, fin)) {
             tc_fence_after();
@@ -313,6 +357,13 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                         make_float4(__uint_as_float(x[j]), __uint_as_float(x[j + 1]), __uint_as_float(x[j + 2]),
                                     __uint_as_float(x[j + 3]));
             }
+        }
+        if (ct == 0) {
+            // every chain MMA this thread issued has completed before TMEM is freed
+            // (immediate unless a wait ran out)
+            if (!fin) *abort_flag = 1;
+            if (n3 > 0) mbar_wait(&bars[B_P3], (n3 - 1) & 1);
+            for (int j = max(0, n4 - 2); j < n4; ++j) mbar_wait(&bars[B_SDONE + (j & 1)], (j >> 1) & 1);
         }
     } else if (warp < 8) {
         // =============================================================== OUT
@@ -374,13 +425,13 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 cv.hist_out[((long long)b * 3 + k3) * tstride + (long long)h * dv + ch] = val;
             }
         }
-    } else if (tid == MMA0 || tid == LOAD0) {
-        // =============================================================== MMA / LOAD
+    } else if (tid == LOAD0) {
+        // =============================================================== LOAD
         // Two issuing threads, each in a fixed order (every awaited event
         // depends only on actions issued earlier in these orders or by the
         // other roles; a tcgen05 commit covers the issuing thread's MMAs):
-        //   MMA  (critical path):  chunk c: P3(c) after AS(c) and P2a(c);
-        //                          P4(c) after AW(c) and K(c)
+        //   CHAIN thread 0 (critical path): chunk c: P3(c) after E4(c) and
+        //        P2a(c); P4(c) after E5(c) and K(c)
         //   LOAD (everything else): IMG(0) V(0) K(0) IMG(1) V(1) [K(1)] P2a(0);
         //        chunk c: V(c+2) (CONV: V(c+1)) after P2a(c); P5a(c) after AS(c)
         //        and X2 free, P5b(c) after AW(c); P2a(c+1) after IMG(c+1) and V(c+1);
@@ -388,11 +439,8 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         //        K(c+NKBUF) and IMG(c+2) after P4(c) and P5b(c)
         constexpr int NKBUF = SM::NKBUF;
         const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
-        auto ioff = [&](int c, uint32_t off) { return (uint64_t)((((uint32_t)(c & 1) * SM::IB) + off) >> 4); };
-        const uint64_t dAS = sw128_desc(smem_u32(sm + SM::AS), 16, 1024);
-        auto as_off = [&](int kk) { return (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4); };
         bool ok = true;
-        if (tid == LOAD0) {
+        {
             // waits off the critical path sleep between polls
             auto WL = [&](int bar, int phase) {
                 if (ok && !wait_bar(&bars[bar], (uint32_t)phase & 1u, abort_flag)) ok = false;
@@ -503,44 +551,6 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             for (int j = max(0, n2 - 2); j < n2; ++j) mbar_wait(&bars[B_P2 + (j & 1)], (j >> 1) & 1);
             for (int j = max(0, n5 - 2); j < n5; ++j) mbar_wait(&bars[B_ODONE + (j & 1)], (j >> 1) & 1);
             if (h0) mbar_wait(&bars[B_H0], 0);
-        } else {
-            // the critical path: spin first
-            auto W = [&](int bar, int phase) {
-                if (!ok) return false;
-                for (uint32_t i = 0; i < 4096u; ++i)
-                    if (mbar_test_wait(&bars[bar], (uint32_t)phase & 1u)) return true;
-                if (!wait_bar(&bars[bar], (uint32_t)phase & 1u, abort_flag)) ok = false;
-                return ok;
-            };
-            const uint64_t dImgMN = sw128_desc(smem_u32(sm + SM::IMG), 8192, 1024);   // W^T (MN-major)
-            const uint64_t dKmn = sw128_desc(smem_u32(sm + SM::K), 8192, 1024);       // K as MN-major
-            const uint64_t dAWD = sw128_desc(smem_u32(sm + SM::AWD), 16, 1024);
-            constexpr uint32_t ID_NEG = idesc_bf16(128, 64, false, true, true);
-            constexpr uint32_t ID_S = idesc_bf16(128, DK, false, true);
-            int n3 = 0, n4 = 0;                              // commit groups issued
-            for (int c = 0; c < nch && ok; ++c) {
-                if (W(B_AS, c) && W(B_P2 + (c & 1), c >> 1)) {      // X1[c&1] -= S W^T  (= Wt^T)
-                    tc_fence_after();
-                    const uint32_t x1 = TM_X1 + (uint32_t)(c & 1) * 64;
-#pragma unroll
-                    for (int kk = 0; kk < KSTEPS; ++kk)
-                        mma_bf16_ss(tb + x1, dAS + as_off(kk), dImgMN + ioff(c, IM::WT + kk * 2048), ID_NEG, 1);
-                    mma_commit(&bars[B_P3]);
-                    ++n3;
-                }
-                if (W(B_AW, c) && W(B_K + c % NKBUF, (c / NKBUF) & 1)) {   // S += Wt^T diag(d/|k|) K
-                    tc_fence_after();
-                    const uint64_t dk_ = dKmn + (uint64_t)(((uint32_t)(c % NKBUF) * NKB * 8192) >> 4);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tb + TM_S, dAWD + (uint64_t)(kk * 32 >> 4), dk_ + (uint64_t)(kk * 2048 >> 4), ID_S, 1);
-                    mma_commit(&bars[B_SDONE + (c & 1)]);
-                    ++n4;
-                }
-            }
-            if (!ok) *abort_flag = 1;
-            if (n3 > 0) mbar_wait(&bars[B_P3], (n3 - 1) & 1);
-            for (int j = max(0, n4 - 2); j < n4; ++j) mbar_wait(&bars[B_SDONE + (j & 1)], (j >> 1) & 1);
         }
     }
     tc_fence_before();

@@ -103,6 +103,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = *tslot;
+    pdl_wait();                                      // q, k, g, beta and the taps are read from here on
+    pdl_trigger();
 
     auto z_of = [&](int item) {                      // first token row of the item in the [B*T] axis
         const int c = item % nct, b = item / nct / H;

@@ -70,6 +70,8 @@ prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gc = seg_chunks + blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     if (gc >= nct) return;
+    pdl_wait();
+    pdl_trigger();
     const int p = gc / seg_chunks;
     const int t0 = gc * C, L = min(C, Tn - t0);
     const long long bh = (long long)b * H + h;

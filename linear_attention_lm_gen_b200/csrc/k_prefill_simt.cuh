@@ -40,6 +40,8 @@ gdn_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const 
                         const float* __restrict__ g, const float* __restrict__ beta,
                         const float* S0, T* __restrict__ o, float* S_out,
                         int Tn, int H, int dv) {
+    pdl_wait();
+    pdl_trigger();
     constexpr int C = PS_C, DVS = PS_DVS, LD = DK + 1, LV = DVS + 1, LC = C + 1;
     extern __shared__ float sm[];
     float* Kc = sm;

@@ -135,6 +135,8 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = *tslot;
+    pdl_wait();                                           // inputs are read from here on
+    pdl_trigger();
 
     if (warp < 4) {
         // =============================================================== CHAIN

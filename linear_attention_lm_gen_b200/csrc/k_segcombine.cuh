@@ -97,6 +97,8 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
         sm100::fence_mbar_init();
     }
     __syncthreads();
+    pdl_wait();                                   // E, A and S0 are read from here on
+    pdl_trigger();
     if (tid == 0)
         for (int p = 1; p <= 2 && p <= last; ++p) {
             sm100::mbar_expect_tx(&bar[p - 1], ABYTES);

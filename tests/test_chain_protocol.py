@@ -4,9 +4,10 @@ checked as a model under random interleavings on the CPU.
 Each role of the kernel is written out as the sequence of waits and
 completions it performs, in the kernel's order:
   chain warps  per chunk c: wait P4(c-1) [and P5(c-1)], wait the image; E4
-               -> arrive AS; wait P3(c); E5 -> arrive AW; at the end wait P4(last)
+               -> arrive AS; (first thread) wait P2a(c), issue P3, wait P3(c);
+               E5 -> arrive AW; (first thread) wait K(c), issue P4; at the
+               end wait P4(last)
   out warps    per chunk c (outputs only): wait P5(c); read O -> arrive X2FREE
-  MMA thread   per chunk c: wait AS(c), P2a(c) -> P3; wait AW(c), K(c) -> P4
   load thread  prologue loads; P2a(0); per chunk c: the next V load once
                P2a(c) is done (V(c+2), or V(c+1) with the conv folded in, whose
                halo is the previous tile); P5a(c), P5b(c); P2a(c+1); K and image
@@ -55,8 +56,12 @@ def run(nch, nkbuf, write_o, conv, seed, mutant=None):
                     yield ("OD", (c - 1) & 1), (c - 1) >> 1
             yield ("IMG", c & 1), c >> 1
             comp[("AS",)] = C(("AS",)) + 1
+            yield p2(c), p2n(c)
+            mma("M", ("P3",))
             yield ("P3",), c
             comp[("AW",)] = C(("AW",)) + 1
+            yield ("K", c % nkbuf), c // nkbuf
+            mma("M", ("SD", c & 1))
         if nch:
             yield ("SD", (nch - 1) & 1), (nch - 1) >> 1
 
@@ -108,16 +113,7 @@ def run(nch, nkbuf, write_o, conv, seed, mutant=None):
                 if c + 2 < nch:
                     load(("IMG", (c + 2) & 1))
 
-    def mma_thread():
-        for c in range(nch):
-            yield ("AS",), c
-            yield p2(c), p2n(c)
-            mma("M", ("P3",))
-            yield ("AW",), c
-            yield ("K", c % nkbuf), c // nkbuf
-            mma("M", ("SD", c & 1))
-
-    roles = {"chain": chain(), "out": out(), "load": loader(), "mma": mma_thread()}
+    roles = {"chain": chain(), "out": out(), "load": loader()}
     cur = dict.fromkeys(roles)
     slow = {k: rng.choice([0.0, 0.5, 0.9, 0.97]) for k in roles}
     done = set()
