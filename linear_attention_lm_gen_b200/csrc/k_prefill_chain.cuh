@@ -17,11 +17,15 @@
 //                     itself (P3 after E4, P4 after E5), so no handoff to
 //                     another thread sits on the chain
 //   warps 4-7  OUT    E6: O^T (TMEM) -> staging -> global, off the chain
+//   warp 9     OMMA   one thread issues the output products (P5a once the bf16
+//                     S copy is written, P5b once Wt^T is), so that they are
+//                     done by the time the next chunk's E4 overwrites their
+//                     operands
 //   warp 10    LOAD   one thread issues the bulk copies of the images, the TMA
 //                     loads of K and V as soon as their buffers are free, and
-//                     the MMAs off the chain (P2a, P5a, P5b)
-//   (warps 8 and 9 have no role: the load thread sits on the scheduler of
-//   warp 2, away from the group pollers of warps 0 and 4)
+//                     P2a (U^T, state-independent, runs ahead)
+//   (warp 8 has no role: the issuing threads sit on the schedulers of warps 1
+//   and 2, away from the group pollers of warps 0 and 4)
 //
 // Buffers: images double-buffered (the copy of chunk c+2 starts once chunk c
 // is finished), V double-buffered (V(c+2) once P2a(c) is done), K
@@ -65,7 +69,7 @@ using namespace pfws;
 
 constexpr int NCH_T = 128, NOUT = 128;
 constexpr int THREADS = NCH_T + NOUT + 96;            // 352
-constexpr int OUT0 = NCH_T, LOAD0 = NCH_T + NOUT + 64;   // warp 10
+constexpr int OUT0 = NCH_T, OMMA0 = NCH_T + NOUT + 32, LOAD0 = NCH_T + NOUT + 64;   // warps 9 and 10
 
 // bounded wait: spin on the phase first, then poll with short sleeps; gives up
 // (error word + CTA abort flag) when the poll budget runs out or another
@@ -244,24 +248,32 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             if (!group_all(2, NCH_T, okw)) break;
             tc_fence_after();
             // ---- E4: S -> bf16 copy, S <- gam_L S
-            {
+            {   // 64 columns (one SW128 block of the copy) per TMEM load wait
                 const float gL = iv[64];
 #pragma unroll
-                for (int cb = 0; cb < DK / 32; ++cb) {
-                    uint32_t x[32];
-                    tmem_ld32(tb + lb + TM_S + cb * 32, x);
+                for (int c2 = 0; c2 < DK / 32; c2 += 2) {
+                    constexpr int NB = 2;
+                    const int nb = min(NB, DK / 32 - c2);
+                    uint32_t x[NB][32];
+#pragma unroll
+                    for (int u = 0; u < NB; ++u)
+                        if (u < nb) tmem_ld32(tb + lb + TM_S + (c2 + u) * 32, x[u]);
                     tmem_ld_wait();
-                    uint8_t* tile = sm + SM::AS + (cb >> 1) * 16384;
+                    uint8_t* tile = sm + SM::AS + (c2 >> 1) * 16384;
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        float f[8];
+                    for (int u = 0; u < NB; ++u) {
+                        if (u >= nb) break;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(x[8 * ch + e]);
-                        *reinterpret_cast<uint4*>(tile + sw128_off(ct, ((cb & 1) * 32 + ch * 8) * 2)) = pack8(f);
+                        for (int ch = 0; ch < 4; ++ch) {
+                            float f[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(x[u][8 * ch + e]);
+                            *reinterpret_cast<uint4*>(tile + sw128_off(ct, (u * 32 + ch * 8) * 2)) = pack8(f);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) x[u][j] = __float_as_uint(gL * __uint_as_float(x[u][j]));
+                        tmem_st32(tb + lb + TM_S + (c2 + u) * 32, x[u]);
                     }
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) x[j] = __float_as_uint(gL * __uint_as_float(x[j]));
-                    tmem_st32(tb + lb + TM_S + cb * 32, x);
                 }
                 tmem_st_wait();
             }
@@ -290,11 +302,13 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             tc_fence_after();
             {
                 const uint32_t x1 = TM_X1 + (uint32_t)p * 64;
+                uint32_t xx[2][32];
+                tmem_ld32(tb + lb + x1, xx[0]);
+                tmem_ld32(tb + lb + x1 + 32, xx[1]);
+                tmem_ld_wait();
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    uint32_t x[32];
-                    tmem_ld32(tb + lb + x1 + half * 32, x);
-                    tmem_ld_wait();
+                    const uint32_t* x = xx[half];
 #pragma unroll
                     for (int ch = 0; ch < 4; ++ch) {
                         float f[8], fd[8];
@@ -425,18 +439,58 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 cv.hist_out[((long long)b * 3 + k3) * tstride + (long long)h * dv + ch] = val;
             }
         }
+    } else if (tid == OMMA0) {
+        // =============================================================== OMMA
+        // chunk c: P5a(c) after AS(c) (the image has landed before it) and X2[c&1]
+        // read by the out warps (chunk c-2); P5b(c) after AW(c); commit ODONE(c)
+        const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
+        const uint64_t dAW = sw128_desc(smem_u32(sm + SM::AW), 16, 1024);
+        constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
+        bool ok = true, pending = false;                  // pending: a P5a issued without its commit
+        int n5 = 0;
+        for (int c = 0; c < nch && ok; ++c) {
+            ok = wait_spin(&bars[B_AS], (uint32_t)c & 1u, abort_flag) &&
+                 wait_spin(&bars[B_IMG + (c & 1)], (uint32_t)(c >> 1) & 1u, abort_flag) &&
+                 (c < 2 || wait_spin(&bars[B_X2FREE + (c & 1)], (uint32_t)((c - 2) >> 1) & 1u, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk)          // X2[c&1] = S Q~^T
+                mma_bf16_ss(tb + x2, dAS + as_off(kk), dImg + ioff(c, IM::Q + (kk >> 2) * 8192 + (kk & 3) * 32),
+                            ID_KK, kk > 0);
+            pending = true;
+            if (!(ok = wait_spin(&bars[B_AW], (uint32_t)c & 1u, abort_flag))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)               // X2[c&1] += Wt^T P^T
+                mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), dImg + ioff(c, IM::P + kk * 32), ID_KK, 1);
+            mma_commit(&bars[B_ODONE + (c & 1)]);
+            pending = false;
+            ++n5;
+        }
+        // a P5a issued without its commit (the AW wait ran out) gets one, so
+        // that every MMA of this thread completes before TMEM is freed
+        if (!ok) {
+            *abort_flag = 1;
+            if (pending) {
+                mma_commit(&bars[B_ODONE + (n5 & 1)]);
+                ++n5;
+            }
+        }
+        for (int j = max(0, n5 - 2); j < n5; ++j) mbar_wait(&bars[B_ODONE + (j & 1)], (j >> 1) & 1);
     } else if (tid == LOAD0) {
         // =============================================================== LOAD
-        // Two issuing threads, each in a fixed order (every awaited event
+        // Three issuing threads, each in a fixed order (every awaited event
         // depends only on actions issued earlier in these orders or by the
         // other roles; a tcgen05 commit covers the issuing thread's MMAs):
         //   CHAIN thread 0 (critical path): chunk c: P3(c) after E4(c) and
         //        P2a(c); P4(c) after E5(c) and K(c)
+        //   OMMA: chunk c: P5a(c) after AS(c) and X2 free; P5b(c) after AW(c)
         //   LOAD (everything else): IMG(0) V(0) K(0) IMG(1) V(1) [K(1)] P2a(0);
-        //        chunk c: V(c+2) (CONV: V(c+1)) after P2a(c); P5a(c) after AS(c)
-        //        and X2 free, P5b(c) after AW(c); P2a(c+1) after IMG(c+1) and V(c+1);
-        //        CONV: the segment's halo with V(0), before P2a(0);
-        //        K(c+NKBUF) and IMG(c+2) after P4(c) and P5b(c)
+        //        chunk c: V(c+2) (CONV: V(c+1)) after P2a(c); P2a(c+1) after
+        //        IMG(c+1) and V(c+1); CONV: the segment's halo with V(0), before
+        //        P2a(0); K(c+NKBUF) and IMG(c+2) after P4(c) and P5b(c)
         constexpr int NKBUF = SM::NKBUF;
         const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
         bool ok = true;
@@ -483,9 +537,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 tma_load_3d(dst + 8192, m, bar, c0 + 64, h, z);
             };
             const uint64_t dV = sw128_desc(smem_u32(sm + SM::V), 8192, 1024);
-            const uint64_t dAW = sw128_desc(smem_u32(sm + SM::AW), 16, 1024);
             const uint64_t dImgMN = sw128_desc(smem_u32(sm + SM::IMG), 8192, 1024);   // MH (MN-major)
-            constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
             constexpr uint32_t ID_MNK = idesc_bf16(128, 64, true, false);
             constexpr uint32_t ID_MNMN = idesc_bf16(128, 64, true, true);
             auto mma_p2a = [&](int c) {      // X1[c&1] = V^T T1^T   (CONV: Vh^T MH + V^T M^T)
@@ -501,21 +553,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                                 CONV || kk > 0);
                 mma_commit(&bars[B_P2 + (c & 1)]);
             };
-            auto mma_p5a = [&](int c) {      // X2[c&1] = S Q~^T
-                const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
-#pragma unroll
-                for (int kk = 0; kk < KSTEPS; ++kk)
-                    mma_bf16_ss(tb + x2, dAS + as_off(kk), dImg + ioff(c, IM::Q + (kk >> 2) * 8192 + (kk & 3) * 32),
-                                ID_KK, kk > 0);
-            };
-            auto mma_p5b = [&](int c) {      // X2[c&1] += Wt^T P^T
-                const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), dImg + ioff(c, IM::P + kk * 32), ID_KK, 1);
-                mma_commit(&bars[B_ODONE + (c & 1)]);
-            };
-            int nK = 0, nV = 0, nI = 0, n2 = 0, n5 = 0;      // loads / commit groups issued
+            int nK = 0, nV = 0, nI = 0, n2 = 0;              // loads / commit groups issued
             bool h0 = false;
             if (nch > 0) { load_img(0); ++nI; load_v(0); ++nV; load_k(0); ++nK; }
             if (CONV && nch > 0) { load_h0(); h0 = true; }
@@ -528,10 +566,6 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 // V(c+2), or with CONV V(c+1) (its buffer held V(c-1), the halo of P2a(c))
                 if (CONV && c + 1 < nch && WL(B_P2 + (c & 1), c >> 1)) { load_v(c + 1); ++nV; }
                 if (!CONV && c + 2 < nch && WL(B_P2 + (c & 1), c >> 1)) { load_v(c + 2); ++nV; }
-                if (write_o) {
-                    if (WL(B_AS, c) && (c < 2 || WL(B_X2FREE + (c & 1), (c - 2) >> 1))) { tc_fence_after(); mma_p5a(c); }
-                    if (WL(B_AW, c)) { tc_fence_after(); mma_p5b(c); ++n5; }
-                }
                 if (c + 1 < nch && WL(B_IMG + ((c + 1) & 1), (c + 1) >> 1) && WL(B_V + ((c + 1) & 1), (c + 1) >> 1)) {
                     tc_fence_after(); mma_p2a(c + 1); ++n2;
                 }
@@ -549,7 +583,6 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             for (int j = max(0, nV - 2); j < nV; ++j) mbar_wait(&bars[B_V + (j & 1)], (j >> 1) & 1);
             for (int j = max(0, nI - 2); j < nI; ++j) mbar_wait(&bars[B_IMG + (j & 1)], (j >> 1) & 1);
             for (int j = max(0, n2 - 2); j < n2; ++j) mbar_wait(&bars[B_P2 + (j & 1)], (j >> 1) & 1);
-            for (int j = max(0, n5 - 2); j < n5; ++j) mbar_wait(&bars[B_ODONE + (j & 1)], (j >> 1) & 1);
             if (h0) mbar_wait(&bars[B_H0], 0);
         }
     }

@@ -8,9 +8,11 @@ completions it performs, in the kernel's order:
                E5 -> arrive AW; (first thread) wait K(c), issue P4; at the
                end wait P4(last)
   out warps    per chunk c (outputs only): wait P5(c); read O -> arrive X2FREE
+  output MMA   per chunk c (outputs only): wait AS(c), the image and X2FREE(c-2)
+               -> P5a; wait AW(c) -> P5b, commit P5(c)
   load thread  prologue loads; P2a(0); per chunk c: the next V load once
                P2a(c) is done (V(c+2), or V(c+1) with the conv folded in, whose
-               halo is the previous tile); P5a(c), P5b(c); P2a(c+1); K and image
+               halo is the previous tile); P2a(c+1); K and image
                loads once chunk c no longer reads their buffers
 Loads and MMA commit groups complete after random delays (each issuer's
 groups in order). A waiter of phase n is released when the barrier has
@@ -35,7 +37,7 @@ def run(nch, nkbuf, write_o, conv, seed, mutant=None):
     rng = random.Random(seed)
     comp = {}
     C = lambda b: comp.get(b, 0)
-    pending, mq = [], {"M": [], "L": []}
+    pending, mq = [], {"M": [], "L": [], "O": []}
     last_v = {0: None, 1: None}          # buffer -> chunk of the last V load issued into it
     nv = [0]
 
@@ -92,12 +94,6 @@ def run(nch, nkbuf, write_o, conv, seed, mutant=None):
             if c + ahead < nch:
                 yield p2(c), p2n(c)
                 load(("V", (c + ahead) & 1))
-            if write_o:
-                yield ("AS",), c
-                if c >= 2:
-                    yield ("X2F", c & 1), (c - 2) >> 1
-                yield ("AW",), c
-                mma("L", ("OD", c & 1))
             if c + 1 < nch:
                 yield ("IMG", (c + 1) & 1), (c + 1) >> 1
                 yield ("V", (c + 1) & 1), (c + 1) >> 1
@@ -113,7 +109,16 @@ def run(nch, nkbuf, write_o, conv, seed, mutant=None):
                 if c + 2 < nch:
                     load(("IMG", (c + 2) & 1))
 
-    roles = {"chain": chain(), "out": out(), "load": loader()}
+    def out_mma():
+        for c in range(nch if write_o else 0):
+            yield ("AS",), c
+            yield ("IMG", c & 1), c >> 1
+            if c >= 2:
+                yield ("X2F", c & 1), (c - 2) >> 1
+            yield ("AW",), c
+            mma("O", ("OD", c & 1))
+
+    roles = {"chain": chain(), "out": out(), "load": loader(), "omma": out_mma()}
     cur = dict.fromkeys(roles)
     slow = {k: rng.choice([0.0, 0.5, 0.9, 0.97]) for k in roles}
     done = set()
@@ -145,7 +150,7 @@ def run(nch, nkbuf, write_o, conv, seed, mutant=None):
             comp[p[1]] = C(p[1]) + 1
             pending.remove(p)
             moved = True
-        for who in ("M", "L"):
+        for who in ("M", "L", "O"):
             q = mq[who]
             if q and rng.random() < 0.7:
                 q[0][0] -= 1
