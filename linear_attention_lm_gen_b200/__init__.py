@@ -51,7 +51,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         return _lib
     if not os.path.exists(path):
         raise ImportError(f"libjet.so not built at {path}: run linear_attention_lm_gen_b200/build.py")
-    L = ctypes.CDLL(path)
+    _lib = declare(ctypes.CDLL(path))
+    return _lib
+
+
+def declare(L: ctypes.CDLL) -> ctypes.CDLL:
+    """Set the argument and result types of the C entry points on a loaded library."""
     P, I, Z, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
     L.jet_kernel_gen.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P]
     L.jet_dyn_conv_v.argtypes = [P] * 8 + [I] * 8 + [P]
@@ -77,7 +82,6 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
               "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step", "jet_jetblock_prefill",
               "jet_jetblock_decode_slots", "jet_device_error"):
         getattr(L, f).restype = I
-    _lib = L
     return L
 
 

@@ -28,19 +28,20 @@ def sources():
     return out
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    """Compile csrc/jet_api.cu (which includes every kernel) into libjet.so."""
-    if not force and os.path.exists(LIB):
-        mt = os.path.getmtime(LIB)
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None, out: str = LIB) -> str:
+    """Compile csrc/jet_api.cu (which includes every kernel) into libjet.so
+    (or, for a test build with extra defines, into `out`)."""
+    if not force and os.path.exists(out):
+        mt = os.path.getmtime(out)
         if all(os.path.getmtime(s) <= mt for s in sources()):
-            return LIB
+            return out
     cmd = [NVCC, *FLAGS, *(extra or []), "-I", INCLUDE, "-I", CSRC,
-           "-o", LIB + ".tmp", os.path.join(CSRC, "jet_api.cu")]
+           "-o", out + ".tmp", os.path.join(CSRC, "jet_api.cu")]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":

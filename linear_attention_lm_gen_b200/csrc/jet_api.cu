@@ -780,3 +780,10 @@ extern "C" jet_status jet_gdn_prefill_noalloc(const void* q, const void* k, cons
     }
     return jet_gdn_prefill(q, k, v, g, beta, S0, o, S_out, ws, use, B, T, H, dk, dv, chunk, dt, stream);
 }
+
+#ifdef JET_TEST_WAIT_EXPIRY
+// test builds only: see g_test_skip_p2a
+extern "C" int jet_test_skip_p2a(int on) {
+    return cudaMemcpyToSymbol(jet::pfch::g_test_skip_p2a, &on, sizeof(int)) == cudaSuccess ? 0 : 1;
+}
+#endif

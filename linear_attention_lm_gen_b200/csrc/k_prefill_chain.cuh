@@ -13,19 +13,19 @@
 //
 //   warps 0-3  CHAIN  E4: S -> bf16 copy and S <- gam_L S;  E5: Wt^T -> bf16
 //                     (plain and scaled by d/|k|); after each of them the
-//                     group's first thread issues the MMAs on the state chain
-//                     itself (P3 after E4, P4 after E5), so no handoff to
-//                     another thread sits on the chain
+//                     group's first thread issues the MMAs itself, so no
+//                     handoff to another thread sits on the chain: after E4
+//                     P3 (on the chain) then P5a, after E5 P4 (on the chain)
+//                     then P5b. Each output product is queued right behind
+//                     the state product it follows, so its issue overlaps that
+//                     product's execution and it never delays the next state
+//                     product in the tensor pipe
 //   warps 4-7  OUT    E6: O^T (TMEM) -> staging -> global, off the chain
-//   warp 9     OMMA   one thread issues the output products (P5a once the bf16
-//                     S copy is written, P5b once Wt^T is), so that they are
-//                     done by the time the next chunk's E4 overwrites their
-//                     operands
 //   warp 10    LOAD   one thread issues the bulk copies of the images, the TMA
 //                     loads of K and V as soon as their buffers are free, and
 //                     P2a (U^T, state-independent, runs ahead)
-//   (warp 8 has no role: the issuing threads sit on the schedulers of warps 1
-//   and 2, away from the group pollers of warps 0 and 4)
+//   (warps 8 and 9 have no role: the load thread sits on the scheduler of
+//   warp 2, away from the group pollers of warps 0 and 4)
 //
 // Buffers: images double-buffered (the copy of chunk c+2 starts once chunk c
 // is finished), V double-buffered (V(c+2) once P2a(c) is done), K
@@ -69,7 +69,7 @@ using namespace pfws;
 
 constexpr int NCH_T = 128, NOUT = 128;
 constexpr int THREADS = NCH_T + NOUT + 96;            // 352
-constexpr int OUT0 = NCH_T, OMMA0 = NCH_T + NOUT + 32, LOAD0 = NCH_T + NOUT + 64;   // warps 9 and 10
+constexpr int OUT0 = NCH_T, LOAD0 = NCH_T + NOUT + 64;   // warp 10
 
 // bounded wait: spin on the phase first, then poll with short sleeps; gives up
 // (error word + CTA abort flag) when the poll budget runs out or another
@@ -122,6 +122,13 @@ struct ChainConv {
     __nv_bfloat16* hist_out;         // [B][3][H][dv] last three raw tokens, or null
 };
 
+#ifdef JET_TEST_WAIT_EXPIRY
+// Test builds only (never in the library): while set, the load thread leaves
+// out P2a of chunk 1, so the chain's bounded wait for it runs out and the
+// kernel winds down with JET_ERR_TIMEOUT.
+__device__ int g_test_skip_p2a = 0;
+#endif
+
 // one pass over all segments (see the header comment); P = 1 is the plain pass
 struct ChainSeg {
     int nseg;                 // P
@@ -136,10 +143,8 @@ enum {
     B_K = 2,          // [NKBUF] K tile landed
     B_V = 4,          // [2] V tile landed
     B_P2 = 6,         // [2] P2a complete (per V buffer, so no waiter lags two phases)
-    B_P3 = 8,         // P3 (and P5a) complete
+    B_P3 = 8,         // P3 complete
     B_SDONE = 9,      // [2] P4 complete
-    B_AS = 11,        // bf16 S written, S scaled (chain)
-    B_AW = 12,        // Wt^T copies written (chain)
     B_X2FREE = 13,    // [2] O^T read (out)
     B_ODONE = 15,     // [2] P5a / P5b complete (O^T ready, S copy and Wt^T free)
     B_H0 = 17,        // the values before a segment's first chunk landed (CONV)
@@ -217,9 +222,13 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         const uint64_t dImgMN = sw128_desc(smem_u32(sm + SM::IMG), 8192, 1024);   // W^T (MN-major)
         const uint64_t dKmn = sw128_desc(smem_u32(sm + SM::K), 8192, 1024);       // K as MN-major
         const uint64_t dAWD = sw128_desc(smem_u32(sm + SM::AWD), 16, 1024);
+        const uint64_t dAW = sw128_desc(smem_u32(sm + SM::AW), 16, 1024);
+        const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
         constexpr uint32_t ID_NEG = idesc_bf16(128, 64, false, true, true);
         constexpr uint32_t ID_S = idesc_bf16(128, DK, false, true);
-        int n3 = 0, n4 = 0;                                  // commit groups issued (thread 0)
+        constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
+        int n3 = 0, n4 = 0, n5 = 0;                          // commit groups issued (thread 0)
+        bool p5a = false;                                    // thread 0: a P5a issued without its commit
         bool live = true;                                    // thread 0: every wait so far succeeded
         const uint32_t lb = (uint32_t)(warp * 32) << 16;
         {   // initial state (row ct of the slice)
@@ -248,27 +257,28 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             if (!group_all(2, NCH_T, okw)) break;
             tc_fence_after();
             // ---- E4: S -> bf16 copy, S <- gam_L S
-            {   // 64 columns (one SW128 block of the copy) per TMEM load wait
+            {   // 64 columns (one SW128 block of the copy) per TMEM load wait (32 at dk = 128: registers)
                 const float gL = iv[64];
+                constexpr int NB = DK <= 96 ? 2 : 1;
 #pragma unroll
-                for (int c2 = 0; c2 < DK / 32; c2 += 2) {
-                    constexpr int NB = 2;
+                for (int c2 = 0; c2 < DK / 32; c2 += NB) {
                     const int nb = min(NB, DK / 32 - c2);
                     uint32_t x[NB][32];
 #pragma unroll
                     for (int u = 0; u < NB; ++u)
                         if (u < nb) tmem_ld32(tb + lb + TM_S + (c2 + u) * 32, x[u]);
                     tmem_ld_wait();
-                    uint8_t* tile = sm + SM::AS + (c2 >> 1) * 16384;
 #pragma unroll
                     for (int u = 0; u < NB; ++u) {
                         if (u >= nb) break;
+                        const int cb = c2 + u;
+                        uint8_t* tile = sm + SM::AS + (cb >> 1) * 16384;
 #pragma unroll
                         for (int ch = 0; ch < 4; ++ch) {
                             float f[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(x[u][8 * ch + e]);
-                            *reinterpret_cast<uint4*>(tile + sw128_off(ct, (u * 32 + ch * 8) * 2)) = pack8(f);
+                            *reinterpret_cast<uint4*>(tile + sw128_off(ct, ((cb & 1) * 32 + ch * 8) * 2)) = pack8(f);
                         }
 #pragma unroll
                         for (int j = 0; j < 32; ++j) x[u][j] = __float_as_uint(gL * __uint_as_float(x[u][j]));
@@ -283,7 +293,6 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             // ---- P3 (thread 0): X1[c&1] -= S W^T  (= Wt^T), once U^T of the chunk is in X1
             bool okp = true;
             if (ct == 0) {
-                arrive(&bars[B_AS]);                         // for the output product P5a
                 okp = wait_spin(&bars[B_P2 + (c & 1)], (c >> 1) & 1, abort_flag);
                 if (okp) {
                     tc_fence_after();
@@ -293,7 +302,18 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                         mma_bf16_ss(tb + x1, dAS + as_off(kk), dImgMN + ioff(c, IM::WT + kk * 2048), ID_NEG, 1);
                     mma_commit(&bars[B_P3]);
                     ++n3;
-                    okp = wait_spin(&bars[B_P3], c & 1, abort_flag);
+                    // P5a: X2[c&1] = S Q~^T, once the out warps have read X2[c&1] (chunk c-2)
+                    okp = c < 2 || wait_spin(&bars[B_X2FREE + (c & 1)], ((c - 2) >> 1) & 1, abort_flag);
+                    if (okp) {
+                        tc_fence_after();
+                        const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+                        for (int kk = 0; kk < KSTEPS; ++kk)
+                            mma_bf16_ss(tb + x2, dAS + as_off(kk),
+                                        dImg + ioff(c, IM::Q + (kk >> 2) * 8192 + (kk & 3) * 32), ID_KK, kk > 0);
+                        p5a = true;
+                        okp = wait_spin(&bars[B_P3], c & 1, abort_flag);
+                    }
                 }
                 live = okp;
             }
@@ -331,7 +351,6 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             named_sync(2, NCH_T);
             // ---- P4 (thread 0): S += Wt^T diag(d/|k|) K, once the K tile is in
             if (ct == 0) {
-                arrive(&bars[B_AW]);                         // for the output product P5b
                 live = wait_spin(&bars[B_K + c % NKBUF], (c / NKBUF) & 1, abort_flag);
                 if (live) {
                     tc_fence_after();
@@ -341,6 +360,14 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                         mma_bf16_ss(tb + TM_S, dAWD + (uint64_t)(kk * 32 >> 4), dk_ + (uint64_t)(kk * 2048 >> 4), ID_S, 1);
                     mma_commit(&bars[B_SDONE + (c & 1)]);
                     ++n4;
+                    // P5b: X2[c&1] += Wt^T P^T, then the outputs of the chunk are complete
+                    const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), dImg + ioff(c, IM::P + kk * 32), ID_KK, 1);
+                    mma_commit(&bars[B_ODONE + (c & 1)]);
+                    p5a = false;
+                    ++n5;
                 }
             }
         }
@@ -376,8 +403,13 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             // every chain MMA this thread issued has completed before TMEM is freed
             // (immediate unless a wait ran out)
             if (!fin) *abort_flag = 1;
+            if (p5a) {                                        // a P5a without its commit: give it one
+                mma_commit(&bars[B_ODONE + (n5 & 1)]);
+                ++n5;
+            }
             if (n3 > 0) mbar_wait(&bars[B_P3], (n3 - 1) & 1);
             for (int j = max(0, n4 - 2); j < n4; ++j) mbar_wait(&bars[B_SDONE + (j & 1)], (j >> 1) & 1);
+            for (int j = max(0, n5 - 2); j < n5; ++j) mbar_wait(&bars[B_ODONE + (j & 1)], (j >> 1) & 1);
         }
     } else if (warp < 8) {
         // =============================================================== OUT
@@ -439,54 +471,13 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 cv.hist_out[((long long)b * 3 + k3) * tstride + (long long)h * dv + ch] = val;
             }
         }
-    } else if (tid == OMMA0) {
-        // =============================================================== OMMA
-        // chunk c: P5a(c) after AS(c) (the image has landed before it) and X2[c&1]
-        // read by the out warps (chunk c-2); P5b(c) after AW(c); commit ODONE(c)
-        const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
-        const uint64_t dAW = sw128_desc(smem_u32(sm + SM::AW), 16, 1024);
-        constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
-        bool ok = true, pending = false;                  // pending: a P5a issued without its commit
-        int n5 = 0;
-        for (int c = 0; c < nch && ok; ++c) {
-            ok = wait_spin(&bars[B_AS], (uint32_t)c & 1u, abort_flag) &&
-                 wait_spin(&bars[B_IMG + (c & 1)], (uint32_t)(c >> 1) & 1u, abort_flag) &&
-                 (c < 2 || wait_spin(&bars[B_X2FREE + (c & 1)], (uint32_t)((c - 2) >> 1) & 1u, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
-#pragma unroll
-            for (int kk = 0; kk < KSTEPS; ++kk)          // X2[c&1] = S Q~^T
-                mma_bf16_ss(tb + x2, dAS + as_off(kk), dImg + ioff(c, IM::Q + (kk >> 2) * 8192 + (kk & 3) * 32),
-                            ID_KK, kk > 0);
-            pending = true;
-            if (!(ok = wait_spin(&bars[B_AW], (uint32_t)c & 1u, abort_flag))) break;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)               // X2[c&1] += Wt^T P^T
-                mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), dImg + ioff(c, IM::P + kk * 32), ID_KK, 1);
-            mma_commit(&bars[B_ODONE + (c & 1)]);
-            pending = false;
-            ++n5;
-        }
-        // a P5a issued without its commit (the AW wait ran out) gets one, so
-        // that every MMA of this thread completes before TMEM is freed
-        if (!ok) {
-            *abort_flag = 1;
-            if (pending) {
-                mma_commit(&bars[B_ODONE + (n5 & 1)]);
-                ++n5;
-            }
-        }
-        for (int j = max(0, n5 - 2); j < n5; ++j) mbar_wait(&bars[B_ODONE + (j & 1)], (j >> 1) & 1);
     } else if (tid == LOAD0) {
         // =============================================================== LOAD
-        // Three issuing threads, each in a fixed order (every awaited event
+        // Two issuing threads, each in a fixed order (every awaited event
         // depends only on actions issued earlier in these orders or by the
         // other roles; a tcgen05 commit covers the issuing thread's MMAs):
-        //   CHAIN thread 0 (critical path): chunk c: P3(c) after E4(c) and
-        //        P2a(c); P4(c) after E5(c) and K(c)
-        //   OMMA: chunk c: P5a(c) after AS(c) and X2 free; P5b(c) after AW(c)
+        //   CHAIN thread 0: chunk c: P3(c) after E4(c) and P2a(c), then P5a(c)
+        //        after X2[c&1] free; P4(c) after E5(c) and K(c), then P5b(c)
         //   LOAD (everything else): IMG(0) V(0) K(0) IMG(1) V(1) [K(1)] P2a(0);
         //        chunk c: V(c+2) (CONV: V(c+1)) after P2a(c); P2a(c+1) after
         //        IMG(c+1) and V(c+1); CONV: the segment's halo with V(0), before
@@ -567,7 +558,10 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 if (CONV && c + 1 < nch && WL(B_P2 + (c & 1), c >> 1)) { load_v(c + 1); ++nV; }
                 if (!CONV && c + 2 < nch && WL(B_P2 + (c & 1), c >> 1)) { load_v(c + 2); ++nV; }
                 if (c + 1 < nch && WL(B_IMG + ((c + 1) & 1), (c + 1) >> 1) && WL(B_V + ((c + 1) & 1), (c + 1) >> 1)) {
-                    tc_fence_after(); mma_p2a(c + 1); ++n2;
+#ifdef JET_TEST_WAIT_EXPIRY
+                    if (!(c == 0 && *reinterpret_cast<volatile int*>(&g_test_skip_p2a)))
+#endif
+                    { tc_fence_after(); mma_p2a(c + 1); ++n2; }
                 }
                 if ((c + NKBUF < nch || c + 2 < nch) && WL(B_SDONE + (c & 1), c >> 1) &&
                     (!write_o || WL(B_ODONE + (c & 1), c >> 1))) {

@@ -66,11 +66,16 @@ __device__ __forceinline__ void named_sync(int id, int n) {
 
 // bounded wait that also gives up when another thread raised the abort flag
 // (a short sleep between polls keeps idle waiters from taking issue slots
-// from the warps that are computing)
+// from the warps that are computing); on running out of time it raises the
+// abort flag itself and sets the device error word
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0;; ++i) {
         if (mbar_test_wait(bar, parity)) return true;
-        if ((i & 255u) == 255u && *abort_flag) return false;
+        if ((i & 255u) == 255u) {
+            if (*abort_flag) return false;
+            if (global_ns() - t0 > kWaitLimitNs) break;
+        }
         __nanosleep(64);
     }
     *abort_flag = 1;

@@ -374,9 +374,13 @@ gdn_prefill_ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // short sleep between polls (a woken try_wait costs ~300 cycles here)
         auto W = [&](int bar, int phase) {
             if (!ok) return false;
-            for (uint32_t i = 0; i < 4u * kWaitPolls; ++i) {
+            const uint64_t t0 = global_ns();
+            for (uint32_t i = 0;; ++i) {
                 if (mbar_test_wait(&bars[bar], (uint32_t)phase & 1u)) return true;
-                if ((i & 1023u) == 1023u && *abort_flag) { ok = false; return false; }
+                if ((i & 1023u) == 1023u) {
+                    if (*abort_flag) { ok = false; return false; }
+                    if (global_ns() - t0 > kWaitLimitNs) break;
+                }
                 __nanosleep(32);
             }
             *abort_flag = 1;

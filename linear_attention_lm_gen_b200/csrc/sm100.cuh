@@ -23,8 +23,20 @@
 namespace jet {
 namespace sm100 {
 
-// poll budget of every bounded wait (each try_wait may itself suspend briefly)
-constexpr uint32_t kWaitPolls = 1u << 24;
+// Time limit of every bounded wait, in nanoseconds of the global timer: a
+// wait that has not seen its phase complete after this long sets the device
+// error word (JET_ERR_TIMEOUT from jet_device_error) and gives up, and the
+// kernel winds down. 1 s in the library; a test build may shorten it.
+#ifndef JET_WAIT_LIMIT_NS
+#define JET_WAIT_LIMIT_NS 1000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = JET_WAIT_LIMIT_NS;
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -60,11 +72,16 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
         : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
     return ok != 0;
 }
-// Wait for the phase with this parity to complete; on running out of polls
+// Wait for the phase with this parity to complete; on running out of time
 // set the device error word and return false (the caller winds down).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitPolls; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitLimitNs) break;
+    }
     flag_error(DEVERR_TIMEOUT);
     return false;
 }

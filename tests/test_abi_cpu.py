@@ -297,3 +297,8 @@ def test_noalloc_prefill_refuses_sizes_beyond_its_scratch(lib):
     # bad arguments are refused before the size check as well
     assert lib.jet_gdn_prefill_noalloc(None, P(A), P(A), P(A), P(A), None, P(A), P(A), B, T, H, dk, dv, 64, BF16,
                                        None) == INVALID
+
+
+def test_the_library_has_no_test_hooks(lib):
+    # the hook that makes a wait run out exists only in test builds
+    assert not hasattr(lib, "jet_test_skip_p2a")
