@@ -13,17 +13,17 @@
 //
 //   warps 0-3  CHAIN  E4: S -> bf16 copy and S <- gam_L S;  E5: Wt^T -> bf16
 //                     (plain and scaled by d/|k|); after each of them the
-//                     group's first thread issues the MMAs itself, so no
-//                     handoff to another thread sits on the chain: after E4
-//                     P3 (on the chain) then P5a, after E5 P4 (on the chain)
-//                     then P5b. Each output product is queued right behind
-//                     the state product it follows, so its issue overlaps that
-//                     product's execution and it never delays the next state
-//                     product in the tensor pipe
+//                     group's first thread issues the state product itself
+//                     (P3 after E4, P4 after E5), so no handoff to another
+//                     thread sits on the chain
 //   warps 4-7  OUT    E6: O^T (TMEM) -> staging -> global, off the chain
 //   warp 10    LOAD   one thread issues the bulk copies of the images, the TMA
 //                     loads of K and V as soon as their buffers are free, and
-//                     P2a (U^T, state-independent, runs ahead)
+//                     the products off the chain: P2a (U^T, state-independent,
+//                     runs ahead), P5a and P5b (outputs). P5a and P5b complete
+//                     on barriers of their own, so the next chunk's E4 waits
+//                     only for P5a (which reads the bf16 S copy) and its E5
+//                     only for P5b (which reads Wt^T), long done by then
 //   (warps 8 and 9 have no role: the load thread sits on the scheduler of
 //   warp 2, away from the group pollers of warps 0 and 4)
 //
@@ -145,10 +145,13 @@ enum {
     B_P2 = 6,         // [2] P2a complete (per V buffer, so no waiter lags two phases)
     B_P3 = 8,         // P3 complete
     B_SDONE = 9,      // [2] P4 complete
+    B_P5A = 11,       // [2] P5a complete (the bf16 S copy free)
     B_X2FREE = 13,    // [2] O^T read (out)
-    B_ODONE = 15,     // [2] P5a / P5b complete (O^T ready, S copy and Wt^T free)
+    B_ODONE = 15,     // [2] P5b complete (O^T ready, Wt^T free)
     B_H0 = 17,        // the values before a segment's first chunk landed (CONV)
-    NBARS = 18
+    B_AS = 18,        // bf16 S written, S scaled (chain)
+    B_AW = 19,        // Wt^T copies written (chain)
+    NBARS = 20
 };
 
 // tm_vh / tm_hh (CONV): 16-row boxes of V ([B*T][H][dv]) and of the history
@@ -222,13 +225,9 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         const uint64_t dImgMN = sw128_desc(smem_u32(sm + SM::IMG), 8192, 1024);   // W^T (MN-major)
         const uint64_t dKmn = sw128_desc(smem_u32(sm + SM::K), 8192, 1024);       // K as MN-major
         const uint64_t dAWD = sw128_desc(smem_u32(sm + SM::AWD), 16, 1024);
-        const uint64_t dAW = sw128_desc(smem_u32(sm + SM::AW), 16, 1024);
-        const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
         constexpr uint32_t ID_NEG = idesc_bf16(128, 64, false, true, true);
         constexpr uint32_t ID_S = idesc_bf16(128, DK, false, true);
-        constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
-        int n3 = 0, n4 = 0, n5 = 0;                          // commit groups issued (thread 0)
-        bool p5a = false;                                    // thread 0: a P5a issued without its commit
+        int n3 = 0, n4 = 0;                                  // commit groups issued (thread 0)
         bool live = true;                                    // thread 0: every wait so far succeeded
         const uint32_t lb = (uint32_t)(warp * 32) << 16;
         {   // initial state (row ct of the slice)
@@ -248,10 +247,10 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             const float* iv = reinterpret_cast<const float*>(img_at(c) + IM::VEC);   // dik[64], gam_{L-1}
             bool okw = true;
             if (ct == 0) {
-                // S updated (P4), the bf16 S copy and Wt^T no longer read (P5a / P5b), image landed
+                // S updated (P4), the bf16 S copy no longer read (P5a), image landed
                 okw = live && (c < 1 || wait_spin(&bars[B_SDONE + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag));
                 okw = okw && (c < 1 || !write_o ||
-                              wait_spin(&bars[B_ODONE + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag));
+                              wait_spin(&bars[B_P5A + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag));
                 okw = okw && wait_spin(&bars[B_IMG + p], (c >> 1) & 1, abort_flag);
             }
             if (!group_all(2, NCH_T, okw)) break;
@@ -293,6 +292,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             // ---- P3 (thread 0): X1[c&1] -= S W^T  (= Wt^T), once U^T of the chunk is in X1
             bool okp = true;
             if (ct == 0) {
+                arrive(&bars[B_AS]);                         // for the output product P5a
                 okp = wait_spin(&bars[B_P2 + (c & 1)], (c >> 1) & 1, abort_flag);
                 if (okp) {
                     tc_fence_after();
@@ -302,19 +302,11 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                         mma_bf16_ss(tb + x1, dAS + as_off(kk), dImgMN + ioff(c, IM::WT + kk * 2048), ID_NEG, 1);
                     mma_commit(&bars[B_P3]);
                     ++n3;
-                    // P5a: X2[c&1] = S Q~^T, once the out warps have read X2[c&1] (chunk c-2)
-                    okp = c < 2 || wait_spin(&bars[B_X2FREE + (c & 1)], ((c - 2) >> 1) & 1, abort_flag);
-                    if (okp) {
-                        tc_fence_after();
-                        const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
-#pragma unroll
-                        for (int kk = 0; kk < KSTEPS; ++kk)
-                            mma_bf16_ss(tb + x2, dAS + as_off(kk),
-                                        dImg + ioff(c, IM::Q + (kk >> 2) * 8192 + (kk & 3) * 32), ID_KK, kk > 0);
-                        p5a = true;
-                        okp = wait_spin(&bars[B_P3], c & 1, abort_flag);
-                    }
+                    okp = wait_spin(&bars[B_P3], c & 1, abort_flag);
                 }
+                // E5 overwrites Wt^T: the previous chunk's P5b has read it
+                okp = okp && (c < 1 || !write_o ||
+                              wait_spin(&bars[B_ODONE + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag));
                 live = okp;
             }
             // ---- E5: Wt^T -> bf16 (plain and scaled by d/|k|)
@@ -351,6 +343,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             named_sync(2, NCH_T);
             // ---- P4 (thread 0): S += Wt^T diag(d/|k|) K, once the K tile is in
             if (ct == 0) {
+                arrive(&bars[B_AW]);                         // for the output product P5b
                 live = wait_spin(&bars[B_K + c % NKBUF], (c / NKBUF) & 1, abort_flag);
                 if (live) {
                     tc_fence_after();
@@ -360,14 +353,6 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                         mma_bf16_ss(tb + TM_S, dAWD + (uint64_t)(kk * 32 >> 4), dk_ + (uint64_t)(kk * 2048 >> 4), ID_S, 1);
                     mma_commit(&bars[B_SDONE + (c & 1)]);
                     ++n4;
-                    // P5b: X2[c&1] += Wt^T P^T, then the outputs of the chunk are complete
-                    const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), dImg + ioff(c, IM::P + kk * 32), ID_KK, 1);
-                    mma_commit(&bars[B_ODONE + (c & 1)]);
-                    p5a = false;
-                    ++n5;
                 }
             }
         }
@@ -403,13 +388,8 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             // every chain MMA this thread issued has completed before TMEM is freed
             // (immediate unless a wait ran out)
             if (!fin) *abort_flag = 1;
-            if (p5a) {                                        // a P5a without its commit: give it one
-                mma_commit(&bars[B_ODONE + (n5 & 1)]);
-                ++n5;
-            }
             if (n3 > 0) mbar_wait(&bars[B_P3], (n3 - 1) & 1);
             for (int j = max(0, n4 - 2); j < n4; ++j) mbar_wait(&bars[B_SDONE + (j & 1)], (j >> 1) & 1);
-            for (int j = max(0, n5 - 2); j < n5; ++j) mbar_wait(&bars[B_ODONE + (j & 1)], (j >> 1) & 1);
         }
     } else if (warp < 8) {
         // =============================================================== OUT
@@ -476,12 +456,13 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         // Two issuing threads, each in a fixed order (every awaited event
         // depends only on actions issued earlier in these orders or by the
         // other roles; a tcgen05 commit covers the issuing thread's MMAs):
-        //   CHAIN thread 0: chunk c: P3(c) after E4(c) and P2a(c), then P5a(c)
-        //        after X2[c&1] free; P4(c) after E5(c) and K(c), then P5b(c)
+        //   CHAIN thread 0: chunk c: P3(c) after E4(c) and P2a(c); P4(c) after
+        //        E5(c) and K(c)
         //   LOAD (everything else): IMG(0) V(0) K(0) IMG(1) V(1) [K(1)] P2a(0);
-        //        chunk c: V(c+2) (CONV: V(c+1)) after P2a(c); P2a(c+1) after
-        //        IMG(c+1) and V(c+1); CONV: the segment's halo with V(0), before
-        //        P2a(0); K(c+NKBUF) and IMG(c+2) after P4(c) and P5b(c)
+        //        chunk c: V(c+2) (CONV: V(c+1)) after P2a(c); P5a(c) after AS(c)
+        //        and X2[c&1] free; P5b(c) after AW(c); P2a(c+1) after IMG(c+1)
+        //        and V(c+1); CONV: the segment's halo with V(0), before P2a(0);
+        //        K(c+NKBUF) and IMG(c+2) after P4(c) and P5b(c)
         constexpr int NKBUF = SM::NKBUF;
         const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
         bool ok = true;
@@ -528,7 +509,9 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 tma_load_3d(dst + 8192, m, bar, c0 + 64, h, z);
             };
             const uint64_t dV = sw128_desc(smem_u32(sm + SM::V), 8192, 1024);
+            const uint64_t dAW = sw128_desc(smem_u32(sm + SM::AW), 16, 1024);
             const uint64_t dImgMN = sw128_desc(smem_u32(sm + SM::IMG), 8192, 1024);   // MH (MN-major)
+            constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);
             constexpr uint32_t ID_MNK = idesc_bf16(128, 64, true, false);
             constexpr uint32_t ID_MNMN = idesc_bf16(128, 64, true, true);
             auto mma_p2a = [&](int c) {      // X1[c&1] = V^T T1^T   (CONV: Vh^T MH + V^T M^T)
@@ -544,7 +527,22 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                                 CONV || kk > 0);
                 mma_commit(&bars[B_P2 + (c & 1)]);
             };
-            int nK = 0, nV = 0, nI = 0, n2 = 0;              // loads / commit groups issued
+            auto mma_p5a = [&](int c) {      // X2[c&1] = S Q~^T
+                const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+                for (int kk = 0; kk < KSTEPS; ++kk)
+                    mma_bf16_ss(tb + x2, dAS + as_off(kk), dImg + ioff(c, IM::Q + (kk >> 2) * 8192 + (kk & 3) * 32),
+                                ID_KK, kk > 0);
+                mma_commit(&bars[B_P5A + (c & 1)]);
+            };
+            auto mma_p5b = [&](int c) {      // X2[c&1] += Wt^T P^T
+                const uint32_t x2 = TM_X2 + (uint32_t)(c & 1) * 64;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tb + x2, dAW + (uint64_t)(kk * 32 >> 4), dImg + ioff(c, IM::P + kk * 32), ID_KK, 1);
+                mma_commit(&bars[B_ODONE + (c & 1)]);
+            };
+            int nK = 0, nV = 0, nI = 0, n2 = 0, n5a = 0, n5 = 0;   // loads / commit groups issued
             bool h0 = false;
             if (nch > 0) { load_img(0); ++nI; load_v(0); ++nV; load_k(0); ++nK; }
             if (CONV && nch > 0) { load_h0(); h0 = true; }
@@ -557,6 +555,12 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 // V(c+2), or with CONV V(c+1) (its buffer held V(c-1), the halo of P2a(c))
                 if (CONV && c + 1 < nch && WL(B_P2 + (c & 1), c >> 1)) { load_v(c + 1); ++nV; }
                 if (!CONV && c + 2 < nch && WL(B_P2 + (c & 1), c >> 1)) { load_v(c + 2); ++nV; }
+                if (write_o) {
+                    if (WL(B_AS, c) && (c < 2 || WL(B_X2FREE + (c & 1), (c - 2) >> 1))) {
+                        tc_fence_after(); mma_p5a(c); ++n5a;
+                    }
+                    if (WL(B_AW, c)) { tc_fence_after(); mma_p5b(c); ++n5; }
+                }
                 if (c + 1 < nch && WL(B_IMG + ((c + 1) & 1), (c + 1) >> 1) && WL(B_V + ((c + 1) & 1), (c + 1) >> 1)) {
 #ifdef JET_TEST_WAIT_EXPIRY
                     if (!(c == 0 && *reinterpret_cast<volatile int*>(&g_test_skip_p2a)))
@@ -577,6 +581,8 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             for (int j = max(0, nV - 2); j < nV; ++j) mbar_wait(&bars[B_V + (j & 1)], (j >> 1) & 1);
             for (int j = max(0, nI - 2); j < nI; ++j) mbar_wait(&bars[B_IMG + (j & 1)], (j >> 1) & 1);
             for (int j = max(0, n2 - 2); j < n2; ++j) mbar_wait(&bars[B_P2 + (j & 1)], (j >> 1) & 1);
+            for (int j = max(0, n5a - 2); j < n5a; ++j) mbar_wait(&bars[B_P5A + (j & 1)], (j >> 1) & 1);
+            for (int j = max(0, n5 - 2); j < n5; ++j) mbar_wait(&bars[B_ODONE + (j & 1)], (j >> 1) & 1);
             if (h0) mbar_wait(&bars[B_H0], 0);
         }
     }

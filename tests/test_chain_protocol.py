@@ -3,14 +3,16 @@ checked as a model under random interleavings on the CPU.
 
 Each role of the kernel is written out as the sequence of waits and
 completions it performs, in the kernel's order:
-  chain warps  per chunk c: wait P4(c-1) [and P5(c-1)], wait the image; E4;
-               (first thread) wait P2a(c), issue P3, [wait X2FREE(c-2), issue
-               P5a], wait P3(c); E5; (first thread) wait K(c), issue P4, [issue
-               P5b, commit P5(c)]; at the end wait P4(last)
-  out warps    per chunk c (outputs only): wait P5(c); read O -> arrive X2FREE
+  chain warps  per chunk c: wait P4(c-1) [and P5a(c-1)], wait the image; E4
+               -> arrive AS; (first thread) wait P2a(c), issue P3, wait P3(c),
+               [wait P5b(c-1)]; E5 -> arrive AW; (first thread) wait K(c),
+               issue P4; at the end wait P4(last)
+  out warps    per chunk c (outputs only): wait P5b(c); read O -> arrive X2FREE
   load thread  prologue loads; P2a(0); per chunk c: the next V load once
                P2a(c) is done (V(c+2), or V(c+1) with the conv folded in, whose
-               halo is the previous tile); P2a(c+1); K and image
+               halo is the previous tile); [P5a(c) after AS(c) and
+               X2FREE(c-2), commit P5a(c); P5b(c) after AW(c), commit P5b(c)];
+               P2a(c+1); K and image
                loads once chunk c no longer reads their buffers
 Loads and MMA commit groups complete after random delays (each issuer's
 groups in order). A waiter of phase n is released when the barrier has
@@ -56,17 +58,17 @@ def run(nch, nkbuf, write_o, conv, seed, mutant=None, patience=None):
             if c >= 1:
                 yield ("SD", (c - 1) & 1), (c - 1) >> 1
                 if write_o:
-                    yield ("OD", (c - 1) & 1), (c - 1) >> 1
+                    yield ("PA", (c - 1) & 1), (c - 1) >> 1
             yield ("IMG", c & 1), c >> 1
+            comp[("AS",)] = C(("AS",)) + 1
             yield p2(c), p2n(c)
             mma("M", ("P3",))
-            if write_o and c >= 2:
-                yield ("X2F", c & 1), (c - 2) >> 1
             yield ("P3",), c
+            if write_o and c >= 1:
+                yield ("OD", (c - 1) & 1), (c - 1) >> 1
+            comp[("AW",)] = C(("AW",)) + 1
             yield ("K", c % nkbuf), c // nkbuf
             mma("M", ("SD", c & 1))
-            if write_o:
-                mma("M", ("OD", c & 1))
         if nch:
             yield ("SD", (nch - 1) & 1), (nch - 1) >> 1
 
@@ -97,6 +99,13 @@ def run(nch, nkbuf, write_o, conv, seed, mutant=None, patience=None):
             if c + ahead < nch:
                 yield p2(c), p2n(c)
                 load(("V", (c + ahead) & 1))
+            if write_o:
+                yield ("AS",), c
+                if c >= 2:
+                    yield ("X2F", c & 1), (c - 2) >> 1
+                mma("L", ("PA", c & 1))
+                yield ("AW",), c
+                mma("L", ("OD", c & 1))
             if c + 1 < nch:
                 yield ("IMG", (c + 1) & 1), (c + 1) >> 1
                 yield ("V", (c + 1) & 1), (c + 1) >> 1
