@@ -20,10 +20,15 @@
 //   warp 10    LOAD   one thread issues the bulk copies of the images, the TMA
 //                     loads of K and V as soon as their buffers are free, and
 //                     the products off the chain: P2a (U^T, state-independent,
-//                     runs ahead), P5a and P5b (outputs). P5a and P5b complete
-//                     on barriers of their own, so the next chunk's E4 waits
-//                     only for P5a (which reads the bf16 S copy) and its E5
-//                     only for P5b (which reads Wt^T), long done by then
+//                     one chunk ahead), P5a and P5b (outputs). They are issued
+//                     into the chain's conversion windows, where the tensor
+//                     pipe has nothing of the chain's: P5a(c) and P2a(c+1) once
+//                     P3(c) has completed (they run during E5(c)), P5b(c) once
+//                     P4(c) has completed (it runs during E4(c+1)), so they
+//                     never queue in front of a state product. P5a and P5b
+//                     complete on barriers of their own: the next chunk's E4
+//                     waits only for P5a (which reads the bf16 S copy), its E5
+//                     only for P5b (which reads Wt^T)
 //   (warps 8 and 9 have no role: the load thread sits on the scheduler of
 //   warp 2, away from the group pollers of warps 0 and 4)
 //
@@ -149,9 +154,7 @@ enum {
     B_X2FREE = 13,    // [2] O^T read (out)
     B_ODONE = 15,     // [2] P5b complete (O^T ready, Wt^T free)
     B_H0 = 17,        // the values before a segment's first chunk landed (CONV)
-    B_AS = 18,        // bf16 S written, S scaled (chain)
-    B_AW = 19,        // Wt^T copies written (chain)
-    NBARS = 20
+    NBARS = 18
 };
 
 // tm_vh / tm_hh (CONV): 16-row boxes of V ([B*T][H][dv]) and of the history
@@ -292,7 +295,6 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             // ---- P3 (thread 0): X1[c&1] -= S W^T  (= Wt^T), once U^T of the chunk is in X1
             bool okp = true;
             if (ct == 0) {
-                arrive(&bars[B_AS]);                         // for the output product P5a
                 okp = wait_spin(&bars[B_P2 + (c & 1)], (c >> 1) & 1, abort_flag);
                 if (okp) {
                     tc_fence_after();
@@ -343,7 +345,6 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             named_sync(2, NCH_T);
             // ---- P4 (thread 0): S += Wt^T diag(d/|k|) K, once the K tile is in
             if (ct == 0) {
-                arrive(&bars[B_AW]);                         // for the output product P5b
                 live = wait_spin(&bars[B_K + c % NKBUF], (c / NKBUF) & 1, abort_flag);
                 if (live) {
                     tc_fence_after();
@@ -459,10 +460,10 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         //   CHAIN thread 0: chunk c: P3(c) after E4(c) and P2a(c); P4(c) after
         //        E5(c) and K(c)
         //   LOAD (everything else): IMG(0) V(0) K(0) IMG(1) V(1) [K(1)] P2a(0);
-        //        chunk c: V(c+2) (CONV: V(c+1)) after P2a(c); P5a(c) after AS(c)
-        //        and X2[c&1] free; P5b(c) after AW(c); P2a(c+1) after IMG(c+1)
-        //        and V(c+1); CONV: the segment's halo with V(0), before P2a(0);
-        //        K(c+NKBUF) and IMG(c+2) after P4(c) and P5b(c)
+        //        chunk c: V(c+2) (CONV: V(c+1)) after P2a(c); P5a(c) after P3(c)
+        //        and X2[c&1] free; P2a(c+1) after IMG(c+1) and V(c+1); P5b(c)
+        //        after P4(c); CONV: the segment's halo with V(0), before P2a(0);
+        //        K(c+NKBUF) and IMG(c+2) after P5b(c)
         constexpr int NKBUF = SM::NKBUF;
         const uint64_t dImg = sw128_desc(smem_u32(sm + SM::IMG), 16, 1024);       // K-major tiles of the image
         bool ok = true;
@@ -555,22 +556,26 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 // V(c+2), or with CONV V(c+1) (its buffer held V(c-1), the halo of P2a(c))
                 if (CONV && c + 1 < nch && WL(B_P2 + (c & 1), c >> 1)) { load_v(c + 1); ++nV; }
                 if (!CONV && c + 2 < nch && WL(B_P2 + (c & 1), c >> 1)) { load_v(c + 2); ++nV; }
-                if (write_o) {
-                    if (WL(B_AS, c) && (c < 2 || WL(B_X2FREE + (c & 1), (c - 2) >> 1))) {
+                // E5(c) window: P3(c) has completed (E4(c) wrote the S copy before it)
+                if (WL(B_P3, c)) {
+                    if (write_o && (c < 2 || WL(B_X2FREE + (c & 1), (c - 2) >> 1))) {
                         tc_fence_after(); mma_p5a(c); ++n5a;
                     }
-                    if (WL(B_AW, c)) { tc_fence_after(); mma_p5b(c); ++n5; }
-                }
-                if (c + 1 < nch && WL(B_IMG + ((c + 1) & 1), (c + 1) >> 1) && WL(B_V + ((c + 1) & 1), (c + 1) >> 1)) {
+                    if (c + 1 < nch && WL(B_IMG + ((c + 1) & 1), (c + 1) >> 1) &&
+                        WL(B_V + ((c + 1) & 1), (c + 1) >> 1)) {
 #ifdef JET_TEST_WAIT_EXPIRY
-                    if (!(c == 0 && *reinterpret_cast<volatile int*>(&g_test_skip_p2a)))
+                        if (!(c == 0 && *reinterpret_cast<volatile int*>(&g_test_skip_p2a)))
 #endif
-                    { tc_fence_after(); mma_p2a(c + 1); ++n2; }
+                        { tc_fence_after(); mma_p2a(c + 1); ++n2; }
+                    }
                 }
-                if ((c + NKBUF < nch || c + 2 < nch) && WL(B_SDONE + (c & 1), c >> 1) &&
-                    (!write_o || WL(B_ODONE + (c & 1), c >> 1))) {
-                    if (c + NKBUF < nch) { load_k(c + NKBUF); ++nK; }
-                    if (c + 2 < nch) { load_img(c + 2); ++nI; }
+                // E4(c+1) window: P4(c) has completed (E5(c) wrote Wt^T before it)
+                if (WL(B_SDONE + (c & 1), c >> 1)) {
+                    if (write_o) { tc_fence_after(); mma_p5b(c); ++n5; }
+                    if ((c + NKBUF < nch || c + 2 < nch) && (!write_o || WL(B_ODONE + (c & 1), c >> 1))) {
+                        if (c + NKBUF < nch) { load_k(c + NKBUF); ++nK; }
+                        if (c + 2 < nch) { load_img(c + 2); ++nI; }
+                    }
                 }
             }
             // every issued load and commit group has completed before the CTA

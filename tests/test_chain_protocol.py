@@ -3,16 +3,16 @@ checked as a model under random interleavings on the CPU.
 
 Each role of the kernel is written out as the sequence of waits and
 completions it performs, in the kernel's order:
-  chain warps  per chunk c: wait P4(c-1) [and P5a(c-1)], wait the image; E4
-               -> arrive AS; (first thread) wait P2a(c), issue P3, wait P3(c),
-               [wait P5b(c-1)]; E5 -> arrive AW; (first thread) wait K(c),
-               issue P4; at the end wait P4(last)
+  chain warps  per chunk c: wait P4(c-1) [and P5a(c-1)], wait the image; E4;
+               (first thread) wait P2a(c), issue P3, wait P3(c), [wait
+               P5b(c-1)]; E5; (first thread) wait K(c), issue P4; at the end
+               wait P4(last)
   out warps    per chunk c (outputs only): wait P5b(c); read O -> arrive X2FREE
   load thread  prologue loads; P2a(0); per chunk c: the next V load once
                P2a(c) is done (V(c+2), or V(c+1) with the conv folded in, whose
-               halo is the previous tile); [P5a(c) after AS(c) and
-               X2FREE(c-2), commit P5a(c); P5b(c) after AW(c), commit P5b(c)];
-               P2a(c+1); K and image
+               halo is the previous tile); wait P3(c): [P5a(c) after
+               X2FREE(c-2)], P2a(c+1) after its image and V; wait P4(c):
+               [P5b(c)], K and image
                loads once chunk c no longer reads their buffers
 Loads and MMA commit groups complete after random delays (each issuer's
 groups in order). A waiter of phase n is released when the barrier has
@@ -30,7 +30,8 @@ def run(nch, nkbuf, write_o, conv, seed, mutant=None, patience=None):
     """One random interleaving; raises AssertionError on a protocol fault.
     mutant (for the tests of the model itself): "plain_v" keeps the two-ahead
     V schedule of plain V with the conv folded in; "one_p2" shares a single
-    P2a barrier between the two V buffers; "skip_p2a1" leaves out P2a of
+    P2a barrier between the two V buffers; "e4_early" lets E4 start without
+    waiting for the previous chunk's P5a; "skip_p2a1" leaves out P2a of
     chunk 1 (the test build's hook), with `patience` the number of rounds a
     wait may block before it gives up and raises the abort flag (after which
     every blocked wait gives up). Returns whether the abort flag was raised."""
@@ -57,16 +58,18 @@ def run(nch, nkbuf, write_o, conv, seed, mutant=None, patience=None):
         for c in range(nch):
             if c >= 1:
                 yield ("SD", (c - 1) & 1), (c - 1) >> 1
-                if write_o:
+                if write_o and mutant != "e4_early":
                     yield ("PA", (c - 1) & 1), (c - 1) >> 1
             yield ("IMG", c & 1), c >> 1
-            comp[("AS",)] = C(("AS",)) + 1
+            if write_o and c >= 1:   # E4 overwrites the S copy that P5a(c-1) reads
+                assert C(("PA", (c - 1) & 1)) > (c - 1) >> 1, f"S copy of chunk {c - 1} overwritten"
             yield p2(c), p2n(c)
             mma("M", ("P3",))
             yield ("P3",), c
             if write_o and c >= 1:
                 yield ("OD", (c - 1) & 1), (c - 1) >> 1
-            comp[("AW",)] = C(("AW",)) + 1
+                # E5 overwrites the Wt^T copy that P5b(c-1) reads
+                assert C(("OD", (c - 1) & 1)) > (c - 1) >> 1, f"Wt copy of chunk {c - 1} overwritten"
             yield ("K", c % nkbuf), c // nkbuf
             mma("M", ("SD", c & 1))
         if nch:
@@ -99,13 +102,11 @@ def run(nch, nkbuf, write_o, conv, seed, mutant=None, patience=None):
             if c + ahead < nch:
                 yield p2(c), p2n(c)
                 load(("V", (c + ahead) & 1))
+            yield ("P3",), c
             if write_o:
-                yield ("AS",), c
                 if c >= 2:
                     yield ("X2F", c & 1), (c - 2) >> 1
                 mma("L", ("PA", c & 1))
-                yield ("AW",), c
-                mma("L", ("OD", c & 1))
             if c + 1 < nch:
                 yield ("IMG", (c + 1) & 1), (c + 1) >> 1
                 yield ("V", (c + 1) & 1), (c + 1) >> 1
@@ -113,8 +114,10 @@ def run(nch, nkbuf, write_o, conv, seed, mutant=None, patience=None):
                     assert last_v[c & 1] == c, f"halo of chunk {c + 1} overwritten"
                 if not (mutant == "skip_p2a1" and c == 0):
                     mma("L", p2(c + 1))
+            yield ("SD", c & 1), c >> 1
+            if write_o:
+                mma("L", ("OD", c & 1))
             if c + nkbuf < nch or c + 2 < nch:
-                yield ("SD", c & 1), c >> 1
                 if write_o:
                     yield ("OD", c & 1), c >> 1
                 if c + nkbuf < nch:
@@ -197,13 +200,12 @@ def test_the_model_catches_a_halo_overwrite():
             run(6, 2, False, True, seed, mutant="plain_v")
 
 
-def test_the_model_catches_a_lagging_waiter():
-    # one P2a barrier for both V buffers lets the load thread run two phases ahead of the
-    # MMA thread's wait (the mistake the per-buffer barriers fix)
-    with pytest.raises(AssertionError, match="completions"):
+def test_the_model_catches_an_early_overwrite():
+    # E4 of chunk c+1 rewrites the bf16 S copy: starting it before P5a(c) has read the copy
+    # (dropping that wait) must be caught
+    with pytest.raises(AssertionError, match="overwritten"):
         for seed in range(300):
-            for w in (False, True):
-                run(8, 2, w, False, seed, mutant="one_p2")
+            run(8, 2, True, False, seed, mutant="e4_early")
 
 
 @pytest.mark.parametrize("conv", [False, True])
