@@ -20,6 +20,8 @@ roofline, and beside a bounded sample on the float64 oracle:
   prefill_2b_t262144  one 262144-token prefill on 2B shapes
   decode_2b_after_t262144  256 decode steps at B=1 continuing that prefill
   decode_4b_b{1,16,64,256,1024}  the 4B decode sweep
+  prefill_2b_t262144_seqpar  (N > 1 only) the 262144-token prompt split into
+                      N token ranges, one per GPU (strong scaling)
 Their inputs use the block-seeded variant of the recipe (synth
 prefill_inputs_blocked / decode_inputs_blocked) so that multi-GB draws take
 seconds.
@@ -582,8 +584,38 @@ def measure_decode_config(ctx, name: str, steps: int, warmup: int, token_sets: i
                     "d2h_bytes_per_step": o.numel() * 2, "ms_per_step": e_ms}}, inp
 
 
+def measure_seqpar(ctx, name: str, steps: int, warmup: int):
+    """One prompt split into N token ranges, one per rank (strong scaling):
+    each rank runs its range, the ranks all-gather the conv halos and the
+    (end state, transition) pairs over NCCL, compose the start states and
+    correct their outputs (seqpar.sequence_parallel_prefill)."""
+    torch, jet, dev, stream, rk, pk = ctx["torch"], ctx["jet"], ctx["dev"], ctx["stream"], ctx["rk"], ctx["pk"]
+    from linear_attention_lm_gen_b200 import seqpar
+    s = synth.CONFIGS[name]
+    Tr = s.T // rk.world
+    inp = synth.prefill_inputs_blocked(s.with_(T=Tr), seed=ctx["seed"] + 1000 * rk.rank)
+    d = {k: as_torch(v).to(dev) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    call = lambda i: seqpar.sequence_parallel_prefill(d["x"], d["W1"], d["W2"], d["q"], d["k"], d["v"], d["g"],
+                                                      d["beta"])
+    ctx["barrier"]()
+    ms = Timer(torch, dev, stream, flush=False).run(call, steps, warmup)
+    t = rk.max_over_ranks(statistics.median(ms), dev)
+    m = prefill_model(s)
+    r_us = roofline_us(m["bytes"], m["flops"], pk) / rk.world
+    return {"workload": f"one {s.T}-token prefill on 2B shapes split into {rk.world} ranges of {Tr} tokens, one per "
+                        f"GPU: range pass, all-gather of the conv halos and the (E, A) pairs over NCCL, compose, "
+                        f"output correction",
+            "scaling": "strong", "tokens_per_s": s.T / (t * 1e-3), "us_per_call": t * 1e3, "steps": steps,
+            "warmup": warmup, "exchange_bytes_per_rank": (s.H * s.dv * s.dk + s.H * s.dk * s.dk) * 4 + 3 * s.H * s.dv * 2,
+            "roofline": {"bound": "hbm", "roofline_us": r_us, "frac": r_us / (t * 1e3),
+                         "note": "the whole prompt's algorithmic bytes over N GPUs' HBM"}}
+
+
 def run_configs(ctx, args):
     out = {}
+    if ctx["rk"].world > 1:
+        out["prefill_2b_t262144_seqpar"] = measure_seqpar(ctx, "prefill_2b_t262144", steps=5, warmup=3)
+        ctx["torch"].cuda.empty_cache()
     cpu = not args.no_cpu_baseline and ctx["rk"].rank == 0
     budget = args.cpu_budget_config
     for name in ("prefill_4b_t65536", "prefill_2b_t262144"):

@@ -158,6 +158,69 @@ jet_status jet_jetblock_prefill(const void* x, const void* w1, const void* w2,
                                 int hidden, int width, int chunk, jet_dtype dt, void* stream);
 
 /*
+ * Sequence parallelism over token ranges: one long prompt split into R
+ * consecutive ranges, one per GPU. The gated delta rule is affine in the
+ * state (paper section 2.3): over a range, S_end = S_start A + E with A the
+ * product of the range's per-token transitions and E the end state reached
+ * from a zero start, and the range's outputs are affine in S_start too. So
+ * every range runs at once from a zero start, the (E, A) pairs are exchanged
+ * (all-gather, a few MB per GPU), each range's true start state is composed
+ * from them, and a correction adds its term to the outputs. The pages run
+ * chunked prefill on one GPU (paper section 3.1 and appendix A.3); the split
+ * across GPUs is this library's, built on that affine form.
+ *
+ * jet_jetblock_prefill_range: the whole mixer over one range (as
+ * jet_jetblock_prefill, tensor-core path only: bf16, dk in {64, 96, 128},
+ * dv a multiple of 128; else JET_ERR_UNSUPPORTED).
+ *   hist_in [B,3,H,dv]: the last three raw V tokens of the previous range (the
+ *     conv's halo), or NULL at the start of the sequence.
+ *   S0 [B,H,dv,dk] float32 or NULL: the range's start state when known (the
+ *     first range), else NULL (zero).
+ *   o [B,T,H,dv] out: the outputs for that start state (provisional for
+ *     ranges after the first until jet_gdn_range_correct).
+ *   E_out [B,H,dv,dk] float32 out: the end state reached from that start.
+ *   A_out [B,H,dk,dk] float32 out and Qe_out [B,H,ceil(T/64),64,dk] bf16 out:
+ *     the range's transition and output-correction operand; both NULL for
+ *     the first range (which needs neither), else both given.
+ *   workspace: at least jet_jetblock_prefill_range_workspace_size(...) bytes.
+ */
+size_t jet_jetblock_prefill_range_workspace_size(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt);
+jet_status jet_jetblock_prefill_range(const void* x, const void* w1, const void* w2,
+                                      const void* q, const void* k, const void* v,
+                                      const void* hist_in, void* hist_out,
+                                      const float* g, const float* beta, const float* S0,
+                                      void* o, float* E_out, float* A_out, void* Qe_out,
+                                      void* workspace, size_t ws_bytes,
+                                      int B, int T, int D, int H, int dk, int dv,
+                                      int hidden, int width, int chunk, jet_dtype dt, void* stream);
+
+/*
+ * Start states of R ranges from their (E, A) pairs (section 2.3's affine
+ * form): S*_1 = E_0, S*_{r+1} = S*_r A_r + E_r, on the tensor cores with
+ * float32 accuracy (each operand split into two tf32 parts).
+ *   E [R,B,H,dv,dk] float32: E_0 is the first range's true end state, E_r
+ *     (r >= 1) the end state of range r from a zero start.
+ *   A [R,B,H,dk,dk] float32: the ranges' transitions (entry 0 is not read).
+ *   Sb_out [R,B,H,dv,dk] bf16 out: entries 1 .. R-1 receive S*_1 .. S*_{R-1},
+ *     the operands of jet_gdn_range_correct (entry 0 is not written).
+ *   S_out [B,H,dv,dk] float32 out: the final state S*_R.
+ * R >= 2; dk in {64, 96, 128}; dv a multiple of 16, at most 256.
+ */
+jet_status jet_gdn_range_compose(const float* E, const float* A, void* Sb_out, float* S_out,
+                                 int R, int B, int H, int dk, int dv, void* stream);
+
+/*
+ * Adds a range's start-state term to its outputs: o += Qe S*^T per chunk of
+ * 64 tokens (the outputs are affine in the start state).
+ *   Qe [B,H,ceil(T/64),64,dk] bf16: from jet_jetblock_prefill_range.
+ *   Sb [B,H,dv,dk] bf16: the range's start state (an entry of Sb_out).
+ *   o [B,T,H,dv] bf16, updated in place (must not overlap Qe or Sb).
+ * Tensor-core shapes only, as jet_jetblock_prefill_range.
+ */
+jet_status jet_gdn_range_correct(const void* Qe, const void* Sb, void* o, int B, int T, int H, int dk, int dv,
+                                 jet_dtype dt, void* stream);
+
+/*
  * One decode step (step 3 for a single new token per sequence; paper section
  * 2.3, the gated delta rule applied to one token; section 2.5, finding 4:
  * decode cost is set by the state's size), updating S in place:

@@ -9,7 +9,8 @@ Function names match the C entry points:
   jet_kernel_gen, jet_dyn_conv_v, jet_gdn_prefill_workspace_size,
   jet_gdn_prefill_workspace_min, jet_gdn_prefill, jet_gdn_prefill_noalloc, jet_gdn_decode_step,
   jet_jetblock_decode_step, jet_conv_gdn_decode_step, jet_jetblock_prefill_workspace_size,
-  jet_jetblock_prefill, jet_jetblock_decode_slots,
+  jet_jetblock_prefill, jet_jetblock_decode_slots, jet_jetblock_prefill_range_workspace_size,
+  jet_jetblock_prefill_range, jet_gdn_range_compose, jet_gdn_range_correct,
   jet_device_error, jet_status_string, jet_launch_count.
 """
 from __future__ import annotations
@@ -30,7 +31,8 @@ EXPORTS = ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill_workspace_size",
            "jet_gdn_prefill",
            "jet_gdn_prefill_noalloc", "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step",
            "jet_jetblock_prefill_workspace_size", "jet_jetblock_prefill", "jet_jetblock_decode_slots",
-           "jet_device_error",
+           "jet_jetblock_prefill_range_workspace_size", "jet_jetblock_prefill_range", "jet_gdn_range_compose",
+           "jet_gdn_range_correct", "jet_device_error",
            "jet_status_string", "jet_launch_count")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -73,6 +75,11 @@ def declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.jet_jetblock_prefill_workspace_size.restype = Z
     L.jet_jetblock_prefill.argtypes = [P] * 14 + [Z] + [I] * 10 + [P]
     L.jet_jetblock_decode_slots.argtypes = [P] * 11 + [I] + [P] * 3 + [I] * 8 + [P]
+    L.jet_jetblock_prefill_range_workspace_size.argtypes = [I] * 7
+    L.jet_jetblock_prefill_range_workspace_size.restype = Z
+    L.jet_jetblock_prefill_range.argtypes = [P] * 16 + [Z] + [I] * 10 + [P]
+    L.jet_gdn_range_compose.argtypes = [P] * 4 + [I] * 5 + [P]
+    L.jet_gdn_range_correct.argtypes = [P] * 3 + [I] * 6 + [P]
     L.jet_device_error.argtypes = [P]
     L.jet_status_string.argtypes = [I]
     L.jet_status_string.restype = ctypes.c_char_p
@@ -80,7 +87,8 @@ def declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.jet_launch_count.restype = U
     for f in ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill", "jet_gdn_prefill_noalloc",
               "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step", "jet_jetblock_prefill",
-              "jet_jetblock_decode_slots", "jet_device_error"):
+              "jet_jetblock_decode_slots", "jet_jetblock_prefill_range", "jet_gdn_range_compose",
+              "jet_gdn_range_correct", "jet_device_error"):
         getattr(L, f).restype = I
     return L
 
@@ -244,6 +252,85 @@ def jet_jetblock_prefill(x, W1, W2, q, k, v, g, beta, hist_in=None, hist_out=Non
         B, T, D, H, dk, dv, hidden, width, 64, dt, _stream(stream))
     _check("jet_jetblock_prefill", st)
     return o, S_out
+
+
+def jet_jetblock_prefill_range_workspace_size(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
+    """Workspace bytes of jet_jetblock_prefill_range (taps + chunk images)."""
+    L = load_library()
+    return int(L.jet_jetblock_prefill_range_workspace_size(B, T, H, dk, dv, chunk,
+                                                           JET_BF16 if dtype == torch.bfloat16 else JET_F32))
+
+
+def jet_jetblock_prefill_range(x, W1, W2, q, k, v, g, beta, hist_in=None, hist_out=None, S0=None, first=False,
+                               o=None, E_out=None, A_out=None, Qe_out=None, workspace=None, *, stream=None):
+    """The mixer over one token range of a sequence split across GPUs.
+    first=True: the range starts at S0 (or zero) for real and gets no
+    transition; otherwise it runs from a zero start and also returns its
+    transition A [B,H,dk,dk] and output-correction operand Qe. Returns
+    (o, E, A, Qe); A and Qe are None for a first range."""
+    L = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    D = x.shape[-1]
+    hidden, HW = W2.shape
+    width = HW // H
+    dev = q.device
+    if o is None:
+        o = torch.empty((B, T, H, dv), device=dev, dtype=q.dtype)
+    if E_out is None:
+        E_out = torch.empty((B, H, dv, dk), device=dev, dtype=torch.float32)
+    if not first:
+        if A_out is None:
+            A_out = torch.empty((B, H, dk, dk), device=dev, dtype=torch.float32)
+        if Qe_out is None:
+            Qe_out = torch.empty((B, H, (T + 63) // 64, 64, dk), device=dev, dtype=q.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(16, jet_jetblock_prefill_range_workspace_size(B, T, H, dk, dv, 64, q.dtype)),
+                                device=dev, dtype=torch.uint8)
+    st = L.jet_jetblock_prefill_range(
+        _ptr(x, "x", q.dtype, (B, T, D)), _ptr(W1, "W1", q.dtype, (D, hidden)), _ptr(W2, "W2", q.dtype, (hidden, HW)),
+        _ptr(q, "q"), _ptr(k, "k", q.dtype, q.shape), _ptr(v, "v", q.dtype, (B, T, H, dv)),
+        _ptr(hist_in, "hist_in", q.dtype, (B, 3, H, dv)), _ptr(hist_out, "hist_out", q.dtype, (B, 3, H, dv)),
+        _ptr(g, "g", torch.float32, (B, T, H)), _ptr(beta, "beta", torch.float32, (B, T, H)),
+        _ptr(S0, "S0", torch.float32, (B, H, dv, dk)), _ptr(o, "o", q.dtype, (B, T, H, dv)),
+        _ptr(E_out, "E_out", torch.float32, (B, H, dv, dk)),
+        _ptr(A_out, "A_out", torch.float32, (B, H, dk, dk)),
+        _ptr(Qe_out, "Qe_out", q.dtype, (B, H, (T + 63) // 64, 64, dk)),
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        B, T, D, H, dk, dv, hidden, width, 64, _dt(q), _stream(stream))
+    _check("jet_jetblock_prefill_range", st)
+    return o, E_out, A_out, Qe_out
+
+
+def jet_gdn_range_compose(E, A, Sb=None, S_out=None, *, stream=None):
+    """Start states of R ranges from their (E, A) pairs: E [R,B,H,dv,dk] and
+    A [R,B,H,dk,dk] float32. Returns (Sb [R,B,H,dv,dk] bf16, entries 1.. are the
+    ranges' start states; S_out [B,H,dv,dk] float32, the final state)."""
+    L = load_library()
+    R, B, H, dv, dk = E.shape
+    if Sb is None:
+        Sb = torch.empty((R, B, H, dv, dk), device=E.device, dtype=torch.bfloat16)
+    if S_out is None:
+        S_out = torch.empty((B, H, dv, dk), device=E.device, dtype=torch.float32)
+    st = L.jet_gdn_range_compose(_ptr(E, "E", torch.float32), _ptr(A, "A", torch.float32, (R, B, H, dk, dk)),
+                                 _ptr(Sb, "Sb", torch.bfloat16, (R, B, H, dv, dk)),
+                                 _ptr(S_out, "S_out", torch.float32, (B, H, dv, dk)), R, B, H, dk, dv,
+                                 _stream(stream))
+    _check("jet_gdn_range_compose", st)
+    return Sb, S_out
+
+
+def jet_gdn_range_correct(Qe, Sb, o, *, stream=None):
+    """o [B,T,H,dv] += the start-state term of a range: Qe from its range pass,
+    Sb [B,H,dv,dk] bf16 its start state. Returns o."""
+    L = load_library()
+    B, T, H, dv = o.shape
+    dk = Sb.shape[-1]
+    st = L.jet_gdn_range_correct(_ptr(Qe, "Qe", o.dtype, (B, H, (T + 63) // 64, 64, dk)),
+                                 _ptr(Sb, "Sb", torch.bfloat16, (B, H, dv, dk)), _ptr(o, "o"), B, T, H, dk, dv,
+                                 _dt(o), _stream(stream))
+    _check("jet_gdn_range_correct", st)
+    return o
 
 
 def jet_gdn_decode_step(q, k, v, g, beta, S, o=None, *, stream=None):

@@ -304,21 +304,37 @@ size_t split_img_bytes(int B, int T, int H, int dk) {
 // CONV (split plan only): v is the raw V; the preparation folds the dynamic
 // conv with `taps` into the chunk images and the chain reads the values
 // before each segment (and the history of `cv`) for it.
+// o += Qe S*^T for chunks chunk0 .. nct-1 (S* of chunk gc: entry gc / segc of Sb)
 template <int DK, int DV>
 jet_status launch_correct(const __nv_bfloat16* Qe, const __nv_bfloat16* Sb, void* o, int B, int Tn, int H, int nct,
-                          int segc, int P, cudaStream_t s) {
+                          int chunk0, int segc, int P, cudaStream_t s) {
     auto kern = pfcor::prefill_correct_kernel<DK, DV>;
     const size_t smem = pfcor::smem_bytes(DK, DV);
     if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
-    return launch(kern, dim3(nct - segc, H, B), dim3(pfcor::THREADS), smem, s, Qe, Sb, (__nv_bfloat16*)o, Tn, H, nct,
-                  segc, P);
+    return launch(kern, dim3(nct - chunk0, H, B), dim3(pfcor::THREADS), smem, s, Qe, Sb, (__nv_bfloat16*)o, Tn, H,
+                  nct, chunk0, segc, P);
 }
+template <int DK>
+jet_status dispatch_correct(const __nv_bfloat16* Qe, const __nv_bfloat16* Sb, void* o, int B, int Tn, int H, int dv,
+                            int nct, int chunk0, int segc, int P, cudaStream_t s) {
+    return dv == 256 ? launch_correct<DK, 256>(Qe, Sb, o, B, Tn, H, nct, chunk0, segc, P, s)
+                     : launch_correct<DK, 128>(Qe, Sb, o, B, Tn, H, nct, chunk0, segc, P, s);
+}
+
+// range mode of the split plan: one segment, plus its transition A [B][H][dk][dk]
+// and output corrections Qe [B][H][nct][64][dk] when A is given (S_out then
+// receives the end state reached from S0, or from zero)
+struct RangeOut {
+    float* A;
+    __nv_bfloat16* Qe;
+    bool on;
+};
 
 template <int DK, bool SPLIT, bool CONV = false>
 jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const float* g, const float* beta,
                              const float* S0, void* o, float* S_out, void* workspace, int B, int Tn, int H,
                              int dv, cudaStream_t s, const float* taps = nullptr,
-                             const pfch::ChainConv& cv = pfch::ChainConv{}) {
+                             const pfch::ChainConv& cv = pfch::ChainConv{}, const RangeOut& range = RangeOut{}) {
     static_assert(SPLIT || !CONV, "the conv is folded in by the preparation kernel of the split plan");
     CUtensorMap mq, mk, mv, mvh, mhh;
     const long long rows = (long long)B * Tn;
@@ -349,6 +365,12 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
                        CONV ? taps : nullptr, (int)(cv.hist_in != nullptr), img, Tn, H, nct, (int)items) != JET_OK)
                 return JET_ERR_CUDA;
         }
+        if (range.on) {   // one segment; the transition slice when A is wanted
+            const bool tr = range.A != nullptr;
+            const pfch::ChainSeg seg{1, nct, nullptr, range.A, range.Qe, DK, tr ? 1 : 0};
+            return launch(chain, dim3(ns + (tr ? 1 : 0), H, B), dim3(pfch::THREADS), smem, s, mk, mv, mvh, mhh,
+                          (const uint8_t*)img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg, cv);
+        }
         const SegPlan plan = plan_one_pass(B, Tn, H, dv, sms);
         const int P = plan.P;
         const OnePassLayout lay = one_pass_layout(B, Tn, H, DK, dv, P);
@@ -356,8 +378,8 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
         float* A = reinterpret_cast<float*>(segws + lay.A);
         __nv_bfloat16* Sb = reinterpret_cast<__nv_bfloat16*>(segws + lay.Sb);
         __nv_bfloat16* Qe = reinterpret_cast<__nv_bfloat16*>(segws + lay.Qe);
-        const pfch::ChainSeg seg = P == 1 ? pfch::ChainSeg{1, plan.seg_chunks, nullptr, nullptr, nullptr}
-                                          : pfch::ChainSeg{P, plan.seg_chunks, E, A, Qe};
+        const pfch::ChainSeg seg = P == 1 ? pfch::ChainSeg{1, plan.seg_chunks, nullptr, nullptr, nullptr, 0, 0}
+                                          : pfch::ChainSeg{P, plan.seg_chunks, E, A, Qe, pfws::trans_ld(DK), 0};
         if (launch(chain, dim3(ns + (P > 1 ? 1 : 0), H, B * P), dim3(pfch::THREADS), smem, s, mk, mv, mvh, mhh,
                    (const uint8_t*)img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg, cv) != JET_OK)
             return JET_ERR_CUDA;
@@ -366,12 +388,11 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
         const size_t sc_smem = sc_smem_bytes(DK);
         if (smem_attr(seg_combine_kernel<DK, true>, sc_smem) != JET_OK) return JET_ERR_CUDA;
         if (launch(seg_combine_kernel<DK, true>, dim3(dv / SC_ROWS, H, B), dim3(sc_threads(DK)), sc_smem, s,
-                   (const float*)E, (const float*)A, (const float*)nullptr, (float*)nullptr, Sb, S_out, P, H,
-                   dv) != JET_OK)
+                   (const float*)E, (const float*)A, (const float*)nullptr, (float*)nullptr, Sb, S_out, P, H, dv,
+                   CombineLayout{0, pfws::trans_ld(DK)}) != JET_OK)
             return JET_ERR_CUDA;
         // outputs of the segments p >= 1: O += Qe S*^T
-        return dv == 256 ? launch_correct<DK, 256>(Qe, Sb, o, B, Tn, H, nct, plan.seg_chunks, P, s)
-                         : launch_correct<DK, 128>(Qe, Sb, o, B, Tn, H, nct, plan.seg_chunks, P, s);
+        return dispatch_correct<DK>(Qe, Sb, o, B, Tn, H, dv, nct, plan.seg_chunks, plan.seg_chunks, P, s);
     }
     auto fused = pfws::gdn_prefill_ws_kernel<DK>;
     if (smem_attr(fused, pfws::SMEM_BYTES) != JET_OK) return JET_ERR_CUDA;
@@ -393,8 +414,8 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
     const size_t sc_smem = sc_smem_bytes(DK);
     if (smem_attr(seg_combine_kernel<DK, false>, sc_smem) != JET_OK) return JET_ERR_CUDA;
     if (launch(seg_combine_kernel<DK, false>, dim3(dv / SC_ROWS, H, B), dim3(sc_threads(DK)), sc_smem, s,
-               (const float*)E, (const float*)A, S0, Sst, (__nv_bfloat16*)nullptr, (float*)nullptr, P, H,
-               dv) != JET_OK)
+               (const float*)E, (const float*)A, S0, Sst, (__nv_bfloat16*)nullptr, (float*)nullptr, P, H, dv,
+               CombineLayout{0, pfws::trans_ld(DK)}) != JET_OK)
         return JET_ERR_CUDA;
     // phase C: every segment from its start state, with outputs
     return run(dim3(ns, H, B * P), pfws::Seg{P, plan.seg_chunks, P, 0, Sst, nullptr, nullptr});
@@ -583,6 +604,98 @@ jet_status jet_jetblock_prefill(const void* x, const void* w1, const void* w2, c
     if (dt == JET_BF16)
         return dispatch_prefill<__nv_bfloat16>(dk, q, k, rest, g, beta, S0, o, S_out, B, T, H, dv, s);
     return dispatch_prefill<float>(dk, q, k, rest, g, beta, S0, o, S_out, B, T, H, dv, s);
+}
+
+// ---- sequence parallelism over token ranges (one range per GPU)
+size_t jet_jetblock_prefill_range_workspace_size(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt) {
+    if (B <= 0 || T <= 0 || H <= 0 || chunk != 64 || !tc_prefill_ok(dt, dk, dv, (long long)B * T)) return 0;
+    const long long nt = elems({B, T, H, 4});
+    if (nt < 0) return 0;
+    return (((size_t)nt * sizeof(float) + 1023) & ~size_t(1023)) + split_img_bytes(B, T, H, dk);
+}
+
+jet_status jet_jetblock_prefill_range(const void* x, const void* w1, const void* w2, const void* q, const void* k,
+                                      const void* v, const void* hist_in, void* hist_out, const float* g,
+                                      const float* beta, const float* S0, void* o, float* E_out, float* A_out,
+                                      void* Qe_out, void* workspace, size_t ws_bytes, int B, int T, int D, int H,
+                                      int dk, int dv, int hidden, int width, int chunk, jet_dtype dt, void* stream) {
+    jet_status st = check_gen(x, w1, w2, B, T, D, H, hidden, width, dt);
+    if (st != JET_OK) return st;
+    if (!q || !k || !v || !g || !beta || !o || !E_out) return JET_ERR_INVALID_ARG;
+    if ((A_out == nullptr) != (Qe_out == nullptr)) return JET_ERR_INVALID_ARG;
+    const long long nv = elems({B, T, H, dv}), nh = elems({B, 3, H, dv});
+    if (elems({B, T, H, dk}) < 0 || nv < 0 || nh < 0 || elems({B, H, dv, dk}) < 0) return JET_ERR_INVALID_ARG;
+    if (!shape_ok(dk, dv) || chunk != 64 || B > 65535 || H > 65535) return JET_ERR_UNSUPPORTED;
+    if (!tc_prefill_ok(dt, dk, dv, (long long)B * T)) return JET_ERR_UNSUPPORTED;
+    for (const void* p : {q, k, v, hist_in, (const void*)hist_out, (const void*)S0, (const void*)o,
+                          (const void*)E_out, (const void*)A_out, (const void*)Qe_out, (const void*)workspace})
+        if (p && !aligned16(p)) return JET_ERR_MISALIGNED;
+    if (!aligned_to(g, 4) || !aligned_to(beta, 4)) return JET_ERR_MISALIGNED;
+    const size_t es = esize(dt), vb = (size_t)nv * es, hb = (size_t)nh * es;
+    if (overlap(v, vb, o, vb)) return JET_ERR_INVALID_ARG;
+    if (hist_out && (overlap(v, vb, hist_out, hb) || (hist_in && overlap(hist_in, hb, hist_out, hb))))
+        return JET_ERR_INVALID_ARG;
+    if (!workspace) ws_bytes = 0;
+    if (ws_bytes < jet_jetblock_prefill_range_workspace_size(B, T, H, dk, dv, chunk, dt)) return JET_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* taps = static_cast<float*>(workspace);
+    uint8_t* rest = static_cast<uint8_t*>(workspace) + ((elems({B, T, H, 4}) * sizeof(float) + 1023) & ~size_t(1023));
+    st = (long long)B * T >= kGenMinTokens
+             ? launch_gen(x, w1, w2, taps, B, T, D, H, s)
+             : launch_genconv<__nv_bfloat16>(x, w1, w2, nullptr, nullptr, nullptr, nullptr, taps, B, T, D, H, dv, s);
+    if (st != JET_OK) return st;
+    const pfch::ChainConv cv{static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(hist_in),
+                             static_cast<__nv_bfloat16*>(hist_out)};
+    const RangeOut range{A_out, static_cast<__nv_bfloat16*>(Qe_out), true};
+#define JET_TC(DK) \
+    return launch_prefill_tc<DK, true, true>(q, k, v, g, beta, S0, o, E_out, rest, B, T, H, dv, s, taps, cv, range);
+    if (dk == 64) { JET_TC(64) }
+    if (dk == 96) { JET_TC(96) }
+    JET_TC(128)
+#undef JET_TC
+}
+
+jet_status jet_gdn_range_compose(const float* E, const float* A, void* Sb_out, float* S_out, int R, int B, int H,
+                                 int dk, int dv, void* stream) {
+    if (!E || !A || !Sb_out || !S_out) return JET_ERR_INVALID_ARG;
+    if (R < 2 || elems({R, B, H, dv, dk}) < 0 || elems({R, B, H, dk, dk}) < 0) return JET_ERR_INVALID_ARG;
+    if (!(dk == 64 || dk == 96 || dk == 128) || dv % SC_ROWS != 0 || dv > 256 || B > 65535 || H > 65535)
+        return JET_ERR_UNSUPPORTED;
+    for (const void* p : {(const void*)E, (const void*)A, (const void*)Sb_out, (const void*)S_out})
+        if (!aligned16(p)) return JET_ERR_MISALIGNED;
+    const size_t sb = (size_t)R * B * H * dv * dk;
+    if (overlap(E, sb * 4, S_out, (size_t)B * H * dv * dk * 4) || overlap(E, sb * 4, Sb_out, sb * 2))
+        return JET_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto run = [&](auto kern, int DK) {
+        const size_t smem = sc_smem_bytes(DK);
+        if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
+        return launch(kern, dim3(dv / SC_ROWS, H, B), dim3(sc_threads(DK)), smem, s, E, A, (const float*)nullptr,
+                      (float*)nullptr, static_cast<__nv_bfloat16*>(Sb_out), S_out, R, H, dv, CombineLayout{1, DK});
+    };
+    if (dk == 64) return run(seg_combine_kernel<64, true>, 64);
+    if (dk == 96) return run(seg_combine_kernel<96, true>, 96);
+    return run(seg_combine_kernel<128, true>, 128);
+}
+
+jet_status jet_gdn_range_correct(const void* Qe, const void* Sb, void* o, int B, int T, int H, int dk, int dv,
+                                 jet_dtype dt, void* stream) {
+    if (!Qe || !Sb || !o) return JET_ERR_INVALID_ARG;
+    if (!dtype_ok(dt)) return JET_ERR_INVALID_ARG;
+    if (elems({B, T, H, dv}) < 0 || elems({B, H, dv, dk}) < 0 || elems({B, H, T, dk}) < 0) return JET_ERR_INVALID_ARG;
+    if (!tc_prefill_ok(dt, dk, dv, (long long)B * T) || B > 65535 || H > 65535) return JET_ERR_UNSUPPORTED;
+    for (const void* p : {Qe, Sb, (const void*)o})
+        if (!aligned16(p)) return JET_ERR_MISALIGNED;
+    const size_t ob = (size_t)B * T * H * dv * 2;
+    if (overlap(o, ob, Qe, (size_t)B * H * ((T + 63) / 64) * 64 * dk * 2) || overlap(o, ob, Sb, (size_t)B * H * dv * dk * 2))
+        return JET_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int nct = (T + 63) / 64;
+    const __nv_bfloat16* qe = static_cast<const __nv_bfloat16*>(Qe);
+    const __nv_bfloat16* sb = static_cast<const __nv_bfloat16*>(Sb);
+    if (dk == 64) return dispatch_correct<64>(qe, sb, o, B, T, H, dv, nct, 0, nct, 1, s);
+    if (dk == 96) return dispatch_correct<96>(qe, sb, o, B, T, H, dv, nct, 0, nct, 1, s);
+    return dispatch_correct<128>(qe, sb, o, B, T, H, dv, nct, 0, nct, 1, s);
 }
 
 jet_status jet_gdn_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,

@@ -139,8 +139,10 @@ struct ChainSeg {
     int nseg;                 // P
     int seg_chunks;           // chunks per segment (the last may be shorter)
     float* Eo;                // P > 1: end states [B][P][H][dv][dk] (segment 0 from S0, the others from 0)
-    float* Ao;                // P > 1: transitions [B][P][H][dk][trans_ld(dk)] (p >= 1)
+    float* Ao;                // P > 1: transitions [B][P][H][dk][a_ld] (p >= 1)
     __nv_bfloat16* Qe;        // P > 1: output corrections [B][H][nct][64][dk] (chunks of segments p >= 1)
+    int a_ld;                 // row stride of Ao (floats)
+    int trans0;               // range mode (P = 1): segment 0 has a transition slice too, writing Ao and Qe
 };
 
 enum {
@@ -184,7 +186,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
     const int ns = dv / ROWS;
     const int h = blockIdx.y, b = blockIdx.z / seg.nseg, p_seg = blockIdx.z % seg.nseg;
     const bool trans = blockIdx.x == ns;                  // transition slice (p >= 1)
-    if (trans && p_seg == 0) return;                      // whole CTA, before any barrier
+    if (trans && p_seg == 0 && !seg.trans0) return;      // whole CTA, before any barrier
     const int c0 = blockIdx.x * ROWS;                     // transition slice: past dv, V reads as zero
     const long long bh = (long long)b * H + h;
     const int nct = (Tn + C - 1) / C;                     // chunks per sequence (image index)
@@ -365,12 +367,13 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         if (group_all(2, NCH_T, fin)) {
             tc_fence_after();
             float* dst = nullptr;
-            if (seg.nseg == 1) {
+            const long long bp = (long long)b * seg.nseg + p_seg;
+            if (trans) {                                      // the transition (p >= 1, or range mode)
+                if (ct < DK) dst = seg.Ao + ((bp * H + h) * DK + ct) * seg.a_ld;
+            } else if (seg.nseg == 1) {
                 dst = S_out + (bh * dv + c0 + ct) * DK;
             } else {
-                const long long bp = (long long)b * seg.nseg + p_seg;
-                if (trans) { if (ct < DK) dst = seg.Ao + ((bp * H + h) * DK + ct) * trans_ld(DK); }
-                else dst = seg.Eo + ((bp * H + h) * dv + c0 + ct) * DK;
+                dst = seg.Eo + ((bp * H + h) * dv + c0 + ct) * DK;
             }
 #pragma unroll
             for (int cb = 0; cb < DK / 32; ++cb) {

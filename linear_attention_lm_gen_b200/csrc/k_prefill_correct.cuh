@@ -53,12 +53,13 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// Qe [B][H][nct][64][DK] bf16; Sb [B][P][H][dv][DK] bf16 (entries p >= 1);
-// o [B*T][H][dv] bf16 (updated in place). grid (nct - seg_chunks, H, B).
+// Qe [B][H][nct][64][DK] bf16; Sb [B][P][H][dv][DK] bf16 (the start state of
+// the segment of chunk gc is entry gc / seg_chunks); o [B*T][H][dv] bf16
+// (updated in place). Chunks chunk0 .. nct-1; grid (nct - chunk0, H, B).
 template <int DK, int DV>
 __global__ void __launch_bounds__(THREADS)
 prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16* __restrict__ Sb,
-                       __nv_bfloat16* __restrict__ o, int Tn, int H, int nct, int seg_chunks, int P) {
+                       __nv_bfloat16* __restrict__ o, int Tn, int H, int nct, int chunk0, int seg_chunks, int P) {
     static_assert(DK % 16 == 0 && DK <= 128 && DV % 64 == 0 && DV <= 256, "shapes");
     constexpr int LDA = lda(DK), LDO = ldo(DV);
     constexpr int NT = DV / 64;                    // n8 tiles per warp (DV / 8 columns)
@@ -68,7 +69,7 @@ prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16
     __nv_bfloat16* ss = qs + C * LDA;                                    // [DV][LDA]
     __nv_bfloat16* os = ss + DV * LDA;                                   // [64][LDO]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gc = seg_chunks + blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int gc = chunk0 + blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     if (gc >= nct) return;
     pdl_wait();
     pdl_trigger();

@@ -51,14 +51,25 @@ __device__ __forceinline__ void mma(float* d, const uint32_t* a, const uint32_t*
 }
 }  // namespace sc
 
-// E [B][NE][H][dv][dk], A [B][NE][H][dk][trans_ld(dk)], NE = P (FINAL) or
-// P - 1; start states Sst [B][P][H][dv][dk] float32 (two passes) or Sb
-// [B][P][H][dv][dk] bf16 (FINAL); grid (dv / 16, H, B), sc_threads(DK)
+// Where segment p's end state, transition and start state of sequence b live:
+// sequence-major ([B][NE][H]...), the layout of the segment passes, or
+// segment-major ([NE][B][H]...), the layout of per-rank ranges gathered from
+// several GPUs. lda: row stride of a transition (trans_ld(dk) in the
+// workspaces; dk for dense [dk][dk] transitions, copied row by row).
+struct CombineLayout {
+    int seg_major;
+    int lda;
+};
+
+// E [B][NE][H][dv][dk], A [B][NE][H][dk][lda] (or segment-major), NE = P
+// (FINAL) or P - 1; start states Sst [B][P][H][dv][dk] float32 (two passes)
+// or Sb bf16 (FINAL, same layout as E); grid (dv / 16, H, B), sc_threads(DK)
 // threads, sc_smem_bytes(DK) shared.
 template <int DK, bool FINAL>
 __global__ void __launch_bounds__(4 * DK)
 seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, const float* S0,
-                   float* __restrict__ Sst, __nv_bfloat16* __restrict__ Sb, float* S_out, int P, int H, int dv) {
+                   float* __restrict__ Sst, __nv_bfloat16* __restrict__ Sb, float* S_out, int P, int H, int dv,
+                   const CombineLayout lay) {
     static_assert(DK % 8 == 0 && DK <= 128, "dk");
     const int NE = FINAL ? P : P - 1;            // segments with an end state / transition
     const int last = FINAL ? P - 1 : P - 2;      // the last step p computes S_start(p + 1)
@@ -74,16 +85,31 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
         sc::split(x, e[0], e[SC_ROWS * LDE]);
     };
     constexpr uint32_t ABYTES = DK * LDAT * sizeof(float);
+    const uint32_t a_bytes = lay.lda == LDAT ? ABYTES : DK * DK * (uint32_t)sizeof(float);   // per transition
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3, n0 = warp * 8;
-    const int r0 = blockIdx.x * SC_ROWS, h = blockIdx.y, b = blockIdx.z;
-    auto e_at = [&](int p) { return E + ((((long long)b * NE + p) * H + h) * dv + r0) * DK; };
+    const int r0 = blockIdx.x * SC_ROWS, h = blockIdx.y, b = blockIdx.z, nb = gridDim.z;
+    // (segment, sequence) -> index of the [H] block
+    auto sb_idx = [&](int p, int n) { return lay.seg_major ? (long long)p * nb + b : (long long)b * n + p; };
+    auto e_at = [&](int p) { return E + ((sb_idx(p, NE) * H + h) * dv + r0) * DK; };
     auto s_at = [&](int p) {                     // S_start(p) (two passes); the final state (FINAL)
         return (FINAL && p == P) ? S_out + (((long long)b * H + h) * dv + r0) * DK
                                  : Sst + ((((long long)b * P + p) * H + h) * dv + r0) * DK;
     };
-    auto sb_at = [&](int p) { return Sb + ((((long long)b * P + p) * H + h) * dv + r0) * DK; };
-    auto a_at = [&](int p) { return A + (((long long)b * NE + p) * H + h) * DK * LDAT; };
+    auto sb_at = [&](int p) { return Sb + ((sb_idx(p, NE) * H + h) * dv + r0) * DK; };
+    auto a_at = [&](int p) { return A + (sb_idx(p, NE) * H + h) * DK * (long long)lay.lda; };
+    // A_p into As[buf]: one bulk copy of the padded rows, or a copy per dense row
+    auto load_a = [&](int p, int buf) {
+        float* dst = As + buf * DK * LDAT;
+        sm100::mbar_expect_tx(&bar[buf], a_bytes);
+        if (lay.lda == LDAT) {
+            sm100::bulk_load(dst, a_at(p), ABYTES, &bar[buf]);
+        } else {
+            for (int j = 0; j < DK; ++j)
+                sm100::bulk_load(dst + j * LDAT, a_at(p) + (long long)j * lay.lda, DK * (uint32_t)sizeof(float),
+                                 &bar[buf]);
+        }
+    };
     // this thread's accumulator entries: rows g and g+8, columns n0+2t and n0+2t+1
     auto load_frag = [&](const float* src, float* d) {
         const float2 x = *reinterpret_cast<const float2*>(src + g * DK + n0 + 2 * t);
@@ -100,10 +126,7 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
     pdl_wait();                                   // E, A and S0 are read from here on
     pdl_trigger();
     if (tid == 0)
-        for (int p = 1; p <= 2 && p <= last; ++p) {
-            sm100::mbar_expect_tx(&bar[p - 1], ABYTES);
-            sm100::bulk_load(As + (p - 1) * DK * LDAT, a_at(p), ABYTES, &bar[p - 1]);
-        }
+        for (int p = 1; p <= 2 && p <= last; ++p) load_a(p, p - 1);
     // two passes: S_start(0) = S0 (or zeros); both: S_start(1) = E_0, also the running rows of step 1
     const float* s0 = (!FINAL && S0) ? S0 + (((long long)b * H + h) * dv + r0) * DK : nullptr;
     {   // every thread owns 4 of the 16 x DK entries; all loads first, then the stores
@@ -175,10 +198,7 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
             *reinterpret_cast<float2*>(sp + (g + 8) * DK + n0 + 2 * t) = make_float2(d[2], d[3]);
         }
         __syncthreads();                              // every read of As[buf] and of the old rows done
-        if (tid == 0 && p + 2 <= last) {              // A_{p+2} is used by step p + 2
-            sm100::mbar_expect_tx(&bar[buf], ABYTES);
-            sm100::bulk_load(As + buf * DK * LDAT, a_at(p + 2), ABYTES, &bar[buf]);
-        }
+        if (tid == 0 && p + 2 <= last) load_a(p + 2, buf);   // A_{p+2} is used by step p + 2
     }
 }
 

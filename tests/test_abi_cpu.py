@@ -302,3 +302,52 @@ def test_noalloc_prefill_refuses_sizes_beyond_its_scratch(lib):
 def test_the_library_has_no_test_hooks(lib):
     # the hook that makes a wait run out exists only in test builds
     assert not hasattr(lib, "jet_test_skip_p2a")
+
+
+def prefill_range(lib, x=A, w1=A, w2=A, q=A, k=A, v=A, hin=None, hout=None, g=A, b=A, S0=None, o=A + (1 << 24),
+                  E=A, Aout=A + (1 << 26), Qe=A + (1 << 27), ws=A, ws_bytes=1 << 30, B=1, T=256, D=64, H=2, dk=96,
+                  dv=128, hidden=32, width=4, chunk=64, dt=BF16):
+    return lib.jet_jetblock_prefill_range(P(x), P(w1), P(w2), P(q), P(k), P(v), P(hin), P(hout), P(g), P(b), P(S0),
+                                          P(o), P(E), P(Aout), P(Qe), P(ws), ws_bytes, B, T, D, H, dk, dv, hidden,
+                                          width, chunk, dt, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(E=None), INVALID), (dict(Aout=None), INVALID),        # A and Qe come together
+    (dict(Qe=None), INVALID), (dict(o=A + 64), INVALID),          # o may not overlap v
+    (dict(dk=48), UNSUPPORTED), (dict(dt=F32), UNSUPPORTED),      # tensor-core shapes only
+    (dict(dv=96), UNSUPPORTED), (dict(chunk=32), UNSUPPORTED),
+    (dict(E=A + 8), MISALIGNED), (dict(Qe=A + (1 << 27) + 8), MISALIGNED),
+    (dict(ws_bytes=1024), WORKSPACE), (dict(ws=None), WORKSPACE),
+])
+def test_prefill_range_rejects(lib, kw, expect):
+    assert prefill_range(lib, **kw) == expect
+
+
+def test_prefill_range_workspace_is_taps_plus_images(lib):
+    B, T, H, dk, dv = 1, 4096, 12, 96, 256
+    taps = -(-B * T * H * 16 // 1024) * 1024
+    assert jet.jet_jetblock_prefill_range_workspace_size(B, T, H, dk, dv) == taps + B * H * (T // 64) * 48128
+    assert jet.jet_jetblock_prefill_range_workspace_size(B, T, H, 48, dv) == 0    # not a tensor-core shape
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(R=1), INVALID), (dict(E=None), INVALID), (dict(dk=48), UNSUPPORTED), (dict(dv=200), UNSUPPORTED),
+    (dict(Sb=A + 8), MISALIGNED), (dict(S=A), INVALID),             # the final state may not overlap E
+])
+def test_range_compose_rejects(lib, kw, expect):
+    a = dict(E=A, Aa=A + (1 << 26), Sb=A + (1 << 27), S=A + (1 << 28), R=2, B=1, H=2, dk=96, dv=128)
+    a.update(kw)
+    assert lib.jet_gdn_range_compose(P(a["E"]), P(a["Aa"]), P(a["Sb"]), P(a["S"]), a["R"], a["B"], a["H"], a["dk"],
+                                     a["dv"], None) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(Qe=None), INVALID), (dict(dk=48), UNSUPPORTED), (dict(dt=F32), UNSUPPORTED),
+    (dict(o=A + 8), MISALIGNED), (dict(o=A), INVALID),               # o may not overlap Qe
+])
+def test_range_correct_rejects(lib, kw, expect):
+    a = dict(Qe=A, Sb=A + (1 << 26), o=A + (1 << 27), B=1, T=256, H=2, dk=96, dv=128, dt=BF16)
+    a.update(kw)
+    assert lib.jet_gdn_range_correct(P(a["Qe"]), P(a["Sb"]), P(a["o"]), a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                                     a["dt"], None) == expect
