@@ -67,8 +67,10 @@ def test_ranges_compose_to_the_whole_prompt(bounds, H, dk, dv, D):
 
 
 def test_a_single_first_range_equals_the_one_call_prefill():
-    # 900 tokens: one segment in both, so the same kernels run on the same data: bit for bit
-    s = synth.JetShape("sp", B=2, T=900, H=3, dk=96, dv=256, D=64)
+    # 500 tokens (8 chunks, fewer than two segments' minimum): one segment in both, so the
+    # same kernels run on the same data: bit for bit
+    s = synth.JetShape("sp", B=2, T=500, H=3, dk=96, dv=256, D=64)
+    assert jet.jet_gdn_prefill_workspace_min(2, 500, 3, 96, 256) == 0
     inp = synth.prefill_inputs(s, seed=82, s0_std=0.2)
     d = gpu_inputs(inp)
     h1 = torch.empty((2, 3, 3, 256), device="cuda", dtype=torch.bfloat16)
