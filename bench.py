@@ -611,6 +611,75 @@ def measure_seqpar(ctx, name: str, steps: int, warmup: int):
                          "note": "the whole prompt's algorithmic bytes over N GPUs' HBM"}}
 
 
+def varlen_lengths(n: int = 16, seed: int = 5, lo: int = 1, hi: int = 4096):
+    """A mixed serving batch: n prompt lengths drawn log-uniform in [lo, hi]
+    (seeded), the longest and shortest always present."""
+    rng = np.random.default_rng(seed)
+    lens = np.exp(rng.uniform(np.log(lo), np.log(hi), n - 2)).astype(int).clip(lo, hi).tolist()
+    return [hi] + lens + [lo]
+
+
+def measure_varlen_config(ctx, steps: int, warmup: int):
+    """A serving round of prompts of mixed lengths on 2B shapes: one
+    jet_jetblock_prefill_varlen call over the packed batch, against one
+    jet_jetblock_prefill call per prompt on the same inputs."""
+    torch, jet, dev, stream, rk, pk = ctx["torch"], ctx["jet"], ctx["dev"], ctx["stream"], ctx["rk"], ctx["pk"]
+    s = PREFILL
+    lens = varlen_lengths()
+    n, total = len(lens), sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    inp = synth.prefill_inputs_blocked(s.with_(B=1, T=total), seed=ctx["seed"] + 7)
+    keys = ("x", "q", "k", "v", "g", "beta")
+    host = {k: as_torch(inp[k][0]).pin_memory() for k in keys}
+    d = {k: v.to(dev) for k, v in host.items()}
+    W1, W2 = as_torch(inp["W1"]).to(dev), as_torch(inp["W2"]).to(dev)
+    o = torch.empty((total, s.H, s.dv), device=dev, dtype=torch.bfloat16)
+    S = torch.empty((n, s.H, s.dv, s.dk), device=dev, dtype=torch.float32)
+    hist = torch.empty((n, 3, s.H, s.dv), device=dev, dtype=torch.bfloat16)
+    ws = torch.empty(max(16, jet.jet_jetblock_prefill_varlen_workspace_size(cu, s.H, s.dk, s.dv)), device=dev,
+                     dtype=torch.uint8)
+    call = lambda i: jet.jet_jetblock_prefill_varlen(d["x"], W1, W2, d["q"], d["k"], d["v"], d["g"], d["beta"], cu,
+                                                     None, hist, None, o, S, ws, stream=stream)
+    ws1 = torch.empty(max(16, max(jet.jet_jetblock_prefill_workspace_size(1, T, s.H, s.dk, s.dv) for T in lens)),
+                      device=dev, dtype=torch.uint8)
+    one = lambda key, a, b: d[key][a:b].unsqueeze(0)
+
+    def per_prompt(i):
+        for j in range(n):
+            a, b = int(cu[j]), int(cu[j + 1])
+            jet.jet_jetblock_prefill(one("x", a, b), W1, W2, one("q", a, b), one("k", a, b), one("v", a, b),
+                                     one("g", a, b), one("beta", a, b), None, hist[j:j + 1], None,
+                                     o[a:b].unsqueeze(0), S[j:j + 1], ws1, stream=stream)
+    ctx["barrier"]()
+    timer = Timer(torch, dev, stream, flush=True)          # the batch is ~0.3 GB: flush L2 between steps
+    t = rk.max_over_ranks(statistics.median(timer.run(call, steps, warmup)), dev)
+    t_loop = rk.max_over_ranks(statistics.median(timer.run(per_prompt, steps, warmup)), dev)
+    h_o = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+
+    def e2e(i):
+        for k in keys:
+            d[k].copy_(host[k], non_blocking=True)
+        call(i)
+        h_o.copy_(o, non_blocking=True)
+    ctx["barrier"]()
+    e_ms = rk.max_over_ranks(statistics.median(timer.run(e2e, max(2, steps // 2), 1)), dev)
+    m = prefill_model(s, B=1, T=total)
+    nbytes = m["bytes"] + (n - 1) * s.H * s.dv * s.dk * 4          # one final state per prompt
+    r_us = roofline_us(nbytes, m["flops"], pk)
+    return {"workload": f"one jet_jetblock_prefill_varlen call over {n} prompts of lengths {lens} ({total} tokens) "
+                        f"packed along the token axis (2B shapes: H={s.H}, dk={s.dk}, dv={s.dv}, d_model={s.D}, "
+                        f"bf16, zero initial states)",
+            "tokens_per_s": rk.world * total / (t * 1e-3), "us_per_call": t * 1e3, "steps": steps, "warmup": warmup,
+            "l2": "flushed between steps",
+            "one_call_per_prompt": {"tokens_per_s": rk.world * total / (t_loop * 1e-3), "us_per_round": t_loop * 1e3,
+                                    "calls": n},
+            "roofline": {"bound": "hbm", "algorithmic_bytes": nbytes, "achieved": nbytes / (t * 1e-3) / 1e9,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "roofline_us": r_us, "frac": r_us / (t * 1e3)},
+            "e2e": {"value": rk.world * total / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": o.numel() * 2, "ms_per_step": e_ms}}, inp, s.with_(B=1, T=total)
+
+
 def run_configs(ctx, args):
     out = {}
     if ctx["rk"].world > 1:
@@ -618,6 +687,11 @@ def run_configs(ctx, args):
         ctx["torch"].cuda.empty_cache()
     cpu = not args.no_cpu_baseline and ctx["rk"].rank == 0
     budget = args.cpu_budget_config
+    r, inp, sp = measure_varlen_config(ctx, steps=10, warmup=3)
+    if cpu:     # the oracle's cost per token does not depend on where the prompts are cut
+        r["cpu_baseline"] = cpu_prefill_sample(sp, inp, budget / 2)
+    out["prefill_2b_varlen_mixed"] = r
+    del inp
     for name in ("prefill_4b_t65536", "prefill_2b_t262144"):
         long_ = name == "prefill_2b_t262144"
         r, inp, kept = measure_prefill_config(ctx, name, steps=5 if long_ else 10, warmup=3, keep=long_)

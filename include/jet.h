@@ -158,6 +158,36 @@ jet_status jet_jetblock_prefill(const void* x, const void* w1, const void* w2,
                                 int hidden, int width, int chunk, jet_dtype dt, void* stream);
 
 /*
+ * jet_jetblock_prefill over a batch of sequences of different lengths in one
+ * call (chunked prefill of several prompts at once: paper section 3.1 and
+ * appendix A.3, throughput measurement). The sequences are packed along the
+ * token axis: sequence i holds tokens cu_seqlens[i] .. cu_seqlens[i+1]-1.
+ *   cu_seqlens: HOST array of nseq + 1 int32 offsets, cu_seqlens[0] = 0,
+ *     strictly increasing (every sequence has at least one token); read during
+ *     the call only (the launch plan is made from it on the host).
+ *   1 <= nseq <= 256 (more returns JET_ERR_UNSUPPORTED).
+ *   x [total,D]; q, k [total,H,dk]; v [total,H,dv] raw; g, beta [total,H]
+ *     float32; o [total,H,dv] out (total = cu_seqlens[nseq]).
+ *   hist_in / hist_out [nseq,3,H,dv] or NULL; S0 / S_out [nseq,H,dv,dk]
+ *     float32 (S0 may be NULL; S_out may alias S0), per sequence as in
+ *     jet_jetblock_prefill.
+ *   workspace: at least jet_jetblock_prefill_varlen_workspace_size(...) bytes.
+ * Tensor-core shapes only (bf16, dk in {64, 96, 128}, dv a multiple of 128).
+ * Long sequences run in segments of a common length, chosen so that every
+ * segment of every sequence runs at once; the results agree with one
+ * jet_jetblock_prefill per sequence within the bf16 tolerance.
+ */
+size_t jet_jetblock_prefill_varlen_workspace_size(const int* cu_seqlens, int nseq, int H, int dk, int dv, int chunk,
+                                                  jet_dtype dt);
+jet_status jet_jetblock_prefill_varlen(const void* x, const void* w1, const void* w2,
+                                       const void* q, const void* k, const void* v,
+                                       const void* hist_in, void* hist_out,
+                                       const float* g, const float* beta, const float* S0,
+                                       void* o, float* S_out, void* workspace, size_t ws_bytes,
+                                       const int* cu_seqlens, int nseq, int D, int H, int dk, int dv,
+                                       int hidden, int width, int chunk, jet_dtype dt, void* stream);
+
+/*
  * Sequence parallelism over token ranges: one long prompt split into R
  * consecutive ranges, one per GPU. The gated delta rule is affine in the
  * state (paper section 2.3): over a range, S_end = S_start A + E with A the

@@ -9,7 +9,8 @@ Function names match the C entry points:
   jet_kernel_gen, jet_dyn_conv_v, jet_gdn_prefill_workspace_size,
   jet_gdn_prefill_workspace_min, jet_gdn_prefill, jet_gdn_prefill_noalloc, jet_gdn_decode_step,
   jet_jetblock_decode_step, jet_conv_gdn_decode_step, jet_jetblock_prefill_workspace_size,
-  jet_jetblock_prefill, jet_jetblock_decode_slots, jet_jetblock_prefill_range_workspace_size,
+  jet_jetblock_prefill, jet_jetblock_decode_slots, jet_jetblock_prefill_varlen_workspace_size,
+  jet_jetblock_prefill_varlen, jet_jetblock_prefill_range_workspace_size,
   jet_jetblock_prefill_range, jet_gdn_range_compose, jet_gdn_range_correct,
   jet_device_error, jet_status_string, jet_launch_count.
 """
@@ -31,6 +32,7 @@ EXPORTS = ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill_workspace_size",
            "jet_gdn_prefill",
            "jet_gdn_prefill_noalloc", "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step",
            "jet_jetblock_prefill_workspace_size", "jet_jetblock_prefill", "jet_jetblock_decode_slots",
+           "jet_jetblock_prefill_varlen_workspace_size", "jet_jetblock_prefill_varlen",
            "jet_jetblock_prefill_range_workspace_size", "jet_jetblock_prefill_range", "jet_gdn_range_compose",
            "jet_gdn_range_correct", "jet_device_error",
            "jet_status_string", "jet_launch_count")
@@ -75,6 +77,9 @@ def declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.jet_jetblock_prefill_workspace_size.restype = Z
     L.jet_jetblock_prefill.argtypes = [P] * 14 + [Z] + [I] * 10 + [P]
     L.jet_jetblock_decode_slots.argtypes = [P] * 11 + [I] + [P] * 3 + [I] * 8 + [P]
+    L.jet_jetblock_prefill_varlen_workspace_size.argtypes = [P, I, I, I, I, I, I]
+    L.jet_jetblock_prefill_varlen_workspace_size.restype = Z
+    L.jet_jetblock_prefill_varlen.argtypes = [P] * 14 + [Z] + [P] + [I] * 9 + [P]
     L.jet_jetblock_prefill_range_workspace_size.argtypes = [I] * 7
     L.jet_jetblock_prefill_range_workspace_size.restype = Z
     L.jet_jetblock_prefill_range.argtypes = [P] * 16 + [Z] + [I] * 10 + [P]
@@ -87,7 +92,8 @@ def declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.jet_launch_count.restype = U
     for f in ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill", "jet_gdn_prefill_noalloc",
               "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step", "jet_jetblock_prefill",
-              "jet_jetblock_decode_slots", "jet_jetblock_prefill_range", "jet_gdn_range_compose",
+              "jet_jetblock_decode_slots", "jet_jetblock_prefill_varlen", "jet_jetblock_prefill_range",
+              "jet_gdn_range_compose",
               "jet_gdn_range_correct", "jet_device_error"):
         getattr(L, f).restype = I
     return L
@@ -251,6 +257,59 @@ def jet_jetblock_prefill(x, W1, W2, q, k, v, g, beta, hist_in=None, hist_out=Non
         _ptr(S_out, "S_out", torch.float32, (B, H, dv, dk)), _ptr(workspace, "workspace"), ws_bytes,
         B, T, D, H, dk, dv, hidden, width, 64, dt, _stream(stream))
     _check("jet_jetblock_prefill", st)
+    return o, S_out
+
+
+def _cu(cu_seqlens):
+    """Sequence offsets as a host int32 array (a list, tuple or CPU tensor)."""
+    import numpy as np
+    if isinstance(cu_seqlens, torch.Tensor):
+        if cu_seqlens.is_cuda:
+            raise TypeError("cu_seqlens must be on the host: the launch plan is made from it")
+        cu_seqlens = cu_seqlens.tolist()
+    return np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+
+
+def jet_jetblock_prefill_varlen_workspace_size(cu_seqlens, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
+    """Workspace bytes of jet_jetblock_prefill_varlen for these sequence offsets."""
+    L = load_library()
+    cu = _cu(cu_seqlens)
+    return int(L.jet_jetblock_prefill_varlen_workspace_size(cu.ctypes.data_as(ctypes.c_void_p), len(cu) - 1, H, dk,
+                                                            dv, chunk, JET_BF16 if dtype == torch.bfloat16 else JET_F32))
+
+
+def jet_jetblock_prefill_varlen(x, W1, W2, q, k, v, g, beta, cu_seqlens, hist_in=None, hist_out=None, S0=None, o=None,
+                                S_out=None, workspace=None, *, stream=None):
+    """The mixer over several prompts of different lengths in one call, packed
+    along the token axis: x [total,D], q,k [total,H,dk], v [total,H,dv] raw,
+    g,beta [total,H] float32; cu_seqlens (host) the nseq + 1 offsets;
+    hist_in / hist_out [nseq,3,H,dv], S0 [nseq,H,dv,dk] or None. Returns
+    (o [total,H,dv], S_out [nseq,H,dv,dk])."""
+    L = load_library()
+    cu = _cu(cu_seqlens)
+    nseq = len(cu) - 1
+    total, H, dk = q.shape
+    dv = v.shape[-1]
+    D = x.shape[-1]
+    hidden, HW = W2.shape
+    width = HW // H
+    if o is None:
+        o = torch.empty((total, H, dv), device=q.device, dtype=q.dtype)
+    if S_out is None:
+        S_out = torch.empty((nseq, H, dv, dk), device=q.device, dtype=torch.float32)
+    if workspace is None:
+        workspace = torch.empty(max(16, jet_jetblock_prefill_varlen_workspace_size(cu, H, dk, dv, 64, q.dtype)),
+                                device=q.device, dtype=torch.uint8)
+    st = L.jet_jetblock_prefill_varlen(
+        _ptr(x, "x", q.dtype, (total, D)), _ptr(W1, "W1", q.dtype, (D, hidden)), _ptr(W2, "W2", q.dtype, (hidden, HW)),
+        _ptr(q, "q"), _ptr(k, "k", q.dtype, q.shape), _ptr(v, "v", q.dtype, (total, H, dv)),
+        _ptr(hist_in, "hist_in", q.dtype, (nseq, 3, H, dv)), _ptr(hist_out, "hist_out", q.dtype, (nseq, 3, H, dv)),
+        _ptr(g, "g", torch.float32, (total, H)), _ptr(beta, "beta", torch.float32, (total, H)),
+        _ptr(S0, "S0", torch.float32, (nseq, H, dv, dk)), _ptr(o, "o", q.dtype, (total, H, dv)),
+        _ptr(S_out, "S_out", torch.float32, (nseq, H, dv, dk)), _ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), cu.ctypes.data_as(ctypes.c_void_p), nseq, D, H, dk, dv, hidden,
+        width, 64, _dt(q), _stream(stream))
+    _check("jet_jetblock_prefill_varlen", st)
     return o, S_out
 
 

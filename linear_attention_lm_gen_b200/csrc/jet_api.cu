@@ -270,17 +270,51 @@ size_t seg_workspace_floats(int B, int H, int dk, int dv, int P) {
 // E [B][P][H][dv][dk], A [B][P][H][dk][dk+8] (float32), start states Sb
 // [B][P][H][dv][dk] and Qe [B][H][nct][64][dk] (bf16)
 struct OnePassLayout { size_t E, A, Sb, Qe, bytes; };
-OnePassLayout one_pass_layout(int B, int T, int H, int dk, int dv, int P) {
+// nsegs: segments over all sequences, nchunks: chunks over all sequences
+OnePassLayout one_pass_layout_n(size_t nsegs, size_t nchunks, int H, int dk, int dv) {
     auto up = [](size_t x) { return (x + 1023) & ~size_t(1023); };
     OnePassLayout l{0, 0, 0, 0, 0};
-    if (P <= 1) return l;
-    const size_t nct = (size_t)((T + 63) / 64);
     l.E = 0;
-    l.A = l.E + up(sizeof(float) * B * P * H * (size_t)dv * dk);
-    l.Sb = l.A + up(sizeof(float) * B * P * H * (size_t)dk * pfws::trans_ld(dk));
-    l.Qe = l.Sb + up(sizeof(__nv_bfloat16) * B * P * H * (size_t)dv * dk);
-    l.bytes = l.Qe + up(sizeof(__nv_bfloat16) * B * H * nct * 64 * (size_t)dk);
+    l.A = l.E + up(sizeof(float) * nsegs * H * (size_t)dv * dk);
+    l.Sb = l.A + up(sizeof(float) * nsegs * H * (size_t)dk * pfws::trans_ld(dk));
+    l.Qe = l.Sb + up(sizeof(__nv_bfloat16) * nsegs * H * (size_t)dv * dk);
+    l.bytes = l.Qe + up(sizeof(__nv_bfloat16) * nchunks * H * 64 * (size_t)dk);
     return l;
+}
+OnePassLayout one_pass_layout(int B, int T, int H, int dk, int dv, int P) {
+    if (P <= 1) return OnePassLayout{0, 0, 0, 0, 0};
+    return one_pass_layout_n((size_t)B * P, (size_t)B * ((T + 63) / 64), H, dk, dv);
+}
+
+// Segment plan of a variable-length batch (host cu_seqlens, already checked):
+// one segment length for all sequences, the shortest (at least 8 chunks) that
+// keeps the one-pass chain within one wave (value slices of every segment plus
+// a transition slice for every segment after a sequence's first); if none
+// does, one segment per sequence. Fills the chunk and segment offsets.
+void plan_varlen(const int* cu, int nseq, int H, int dv, int sms, pfws::SeqMap& sq) {
+    const int ns = dv / pfws::ROWS;
+    int maxc = 1;
+    sq.nseq = nseq;
+    sq.chunk[0] = 0;
+    for (int i = 0; i < nseq; ++i) {
+        sq.tok[i] = cu[i];
+        const int nci = (cu[i + 1] - cu[i] + 63) / 64;
+        sq.chunk[i + 1] = sq.chunk[i] + nci;
+        maxc = std::max(maxc, nci);
+    }
+    sq.tok[nseq] = cu[nseq];
+    int segc = maxc;
+    for (int cand = kMinSegChunks; cand < maxc; cand += std::max(1, cand / 2)) {
+        long long ctas = 0;
+        for (int i = 0; i < nseq; ++i) {
+            const int Pi = (sq.chunk[i + 1] - sq.chunk[i] + cand - 1) / cand;
+            ctas += (long long)H * ((long long)ns * Pi + Pi - 1);
+        }
+        if (ctas <= sms) { segc = cand; break; }
+    }
+    sq.seg_chunks = segc;
+    sq.seg[0] = 0;
+    for (int i = 0; i < nseq; ++i) sq.seg[i + 1] = sq.seg[i] + (sq.chunk[i + 1] - sq.chunk[i] + segc - 1) / segc;
 }
 
 // per-chunk image of the two-kernel plan (preparation + chain), bytes
@@ -304,21 +338,32 @@ size_t split_img_bytes(int B, int T, int H, int dk) {
 // CONV (split plan only): v is the raw V; the preparation folds the dynamic
 // conv with `taps` into the chunk images and the chain reads the values
 // before each segment (and the history of `cv`) for it.
-// o += Qe S*^T for chunks chunk0 .. nct-1 (S* of chunk gc: entry gc / segc of Sb)
+// o += Qe S*^T for chunks chunk0 .. nct-1 (S* of chunk gc: entry gc / segc of
+// Sb), or (variable length, vchunks > 0) for every chunk of the sequence map
 template <int DK, int DV>
 jet_status launch_correct(const __nv_bfloat16* Qe, const __nv_bfloat16* Sb, void* o, int B, int Tn, int H, int nct,
-                          int chunk0, int segc, int P, cudaStream_t s) {
+                          int chunk0, int segc, int P, cudaStream_t s, const pfws::SeqMap& sq, int vchunks) {
     auto kern = pfcor::prefill_correct_kernel<DK, DV>;
     const size_t smem = pfcor::smem_bytes(DK, DV);
     if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
-    return launch(kern, dim3(nct - chunk0, H, B), dim3(pfcor::THREADS), smem, s, Qe, Sb, (__nv_bfloat16*)o, Tn, H,
-                  nct, chunk0, segc, P);
+    const dim3 grid = vchunks > 0 ? dim3(vchunks, H, 1) : dim3(nct - chunk0, H, B);
+    return launch(kern, grid, dim3(pfcor::THREADS), smem, s, Qe, Sb, (__nv_bfloat16*)o, Tn, H, nct, chunk0, segc, P,
+                  sq);
 }
 template <int DK>
 jet_status dispatch_correct(const __nv_bfloat16* Qe, const __nv_bfloat16* Sb, void* o, int B, int Tn, int H, int dv,
-                            int nct, int chunk0, int segc, int P, cudaStream_t s) {
-    return dv == 256 ? launch_correct<DK, 256>(Qe, Sb, o, B, Tn, H, nct, chunk0, segc, P, s)
-                     : launch_correct<DK, 128>(Qe, Sb, o, B, Tn, H, nct, chunk0, segc, P, s);
+                            int nct, int chunk0, int segc, int P, cudaStream_t s, const pfws::SeqMap& sq,
+                            int vchunks) {
+    return dv == 256 ? launch_correct<DK, 256>(Qe, Sb, o, B, Tn, H, nct, chunk0, segc, P, s, sq, vchunks)
+                     : launch_correct<DK, 128>(Qe, Sb, o, B, Tn, H, nct, chunk0, segc, P, s, sq, vchunks);
+}
+const pfws::SeqMap& no_seqmap() {   // nseq = 0: the dense layout
+    static pfws::SeqMap m = [] {
+        pfws::SeqMap z;
+        memset(&z, 0, sizeof(z));
+        return z;
+    }();
+    return m;
 }
 
 // range mode of the split plan: one segment, plus its transition A [B][H][dk][dk]
@@ -334,17 +379,20 @@ template <int DK, bool SPLIT, bool CONV = false>
 jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const float* g, const float* beta,
                              const float* S0, void* o, float* S_out, void* workspace, int B, int Tn, int H,
                              int dv, cudaStream_t s, const float* taps = nullptr,
-                             const pfch::ChainConv& cv = pfch::ChainConv{}, const RangeOut& range = RangeOut{}) {
+                             const pfch::ChainConv& cv = pfch::ChainConv{}, const RangeOut& range = RangeOut{},
+                             const pfws::SeqMap* vsq = nullptr) {
     static_assert(SPLIT || !CONV, "the conv is folded in by the preparation kernel of the split plan");
+    const pfws::SeqMap& sq = vsq ? *vsq : no_seqmap();
     CUtensorMap mq, mk, mv, mvh, mhh;
-    const long long rows = (long long)B * Tn;
+    const long long rows = vsq ? (long long)vsq->tok[vsq->nseq] : (long long)B * Tn;
+    const int nseqs = vsq ? vsq->nseq : B;
     if (!tile_map(&mq, q, DK, H, rows) || !tile_map(&mk, k, DK, H, rows) || !tile_map(&mv, v, dv, H, rows))
         return JET_ERR_CUDA;
     // 16-row boxes of V and of the history (the values before a segment)
     mvh = mv;
     mhh = mv;
     if (CONV && (!tile_map(&mvh, v, dv, H, rows, 16) ||
-                 (cv.hist_in && !tile_map(&mhh, cv.hist_in, dv, H, (long long)B * 3, 16))))
+                 (cv.hist_in && !tile_map(&mhh, cv.hist_in, dv, H, (long long)nseqs * 3, 16))))
         return JET_ERR_CUDA;
     if (CONV && !cv.hist_in) mhh = mvh;
     const int ns = dv / pfws::ROWS;
@@ -354,22 +402,46 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
         auto chain = pfch::gdn_prefill_chain_kernel<DK, CONV>;
         constexpr uint32_t smem = pfch::ChainSmem<DK>::BYTES;
         if (smem_attr(chain, smem) != JET_OK) return JET_ERR_CUDA;
+        const long long nchunks = vsq ? vsq->chunk[vsq->nseq] : (long long)B * nct;   // over all sequences
         uint8_t* img = static_cast<uint8_t*>(workspace);
-        uint8_t* segws = img + split_img_bytes(B, Tn, H, DK);
+        uint8_t* segws = img + (size_t)nchunks * H * img_chunk_bytes(DK);
         {   // K2a: every chunk of every (sequence, head)
             auto prep = pfws::gdn_chunk_prep_kernel<DK>;
             if (smem_attr(prep, pfws::PrepSmem<DK>::BYTES) != JET_OK) return JET_ERR_CUDA;
-            const long long items = (long long)B * H * nct;
+            const long long items = nchunks * H;
             const int grid = (int)std::min<long long>(items, (long long)pfws::PREP_CTAS * sms);   // resident CTAs
             if (launch(prep, dim3(grid), dim3(pfws::PREP_THREADS), pfws::PrepSmem<DK>::BYTES, s, mq, mk, g, beta,
-                       CONV ? taps : nullptr, (int)(cv.hist_in != nullptr), img, Tn, H, nct, (int)items) != JET_OK)
+                       CONV ? taps : nullptr, (int)(cv.hist_in != nullptr), img, Tn, H, nct, (int)items,
+                       sq) != JET_OK)
                 return JET_ERR_CUDA;
+        }
+        if (vsq) {   // variable length: the segments of the plan in the sequence map
+            const int nsegs = vsq->seg[vsq->nseq];
+            const bool multi = nsegs > vsq->nseq;
+            const OnePassLayout lay = one_pass_layout_n(nsegs, nchunks, H, DK, dv);
+            float* E = reinterpret_cast<float*>(segws + lay.E);
+            float* A = reinterpret_cast<float*>(segws + lay.A);
+            __nv_bfloat16* Sb = reinterpret_cast<__nv_bfloat16*>(segws + lay.Sb);
+            __nv_bfloat16* Qe = reinterpret_cast<__nv_bfloat16*>(segws + lay.Qe);
+            const pfch::ChainSeg seg{1, vsq->seg_chunks, E, A, Qe, pfws::trans_ld(DK), 0};
+            if (launch(chain, dim3(ns + (multi ? 1 : 0), H, nsegs), dim3(pfch::THREADS), smem, s, mk, mv, mvh, mhh,
+                       (const uint8_t*)img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg, cv, sq) != JET_OK)
+                return JET_ERR_CUDA;
+            if (!multi) return JET_OK;
+            const size_t sc_smem = sc_smem_bytes(DK);
+            if (smem_attr(seg_combine_kernel<DK, true>, sc_smem) != JET_OK) return JET_ERR_CUDA;
+            if (launch(seg_combine_kernel<DK, true>, dim3(dv / SC_ROWS, H, vsq->nseq), dim3(sc_threads(DK)), sc_smem,
+                       s, (const float*)E, (const float*)A, (const float*)nullptr, (float*)nullptr, Sb, S_out, 0, H,
+                       dv, CombineLayout{0, pfws::trans_ld(DK)}, sq) != JET_OK)
+                return JET_ERR_CUDA;
+            return dispatch_correct<DK>(Qe, Sb, o, 1, Tn, H, dv, (int)nchunks, 0, vsq->seg_chunks, 1, s, sq,
+                                        (int)nchunks);
         }
         if (range.on) {   // one segment; the transition slice when A is wanted
             const bool tr = range.A != nullptr;
             const pfch::ChainSeg seg{1, nct, nullptr, range.A, range.Qe, DK, tr ? 1 : 0};
             return launch(chain, dim3(ns + (tr ? 1 : 0), H, B), dim3(pfch::THREADS), smem, s, mk, mv, mvh, mhh,
-                          (const uint8_t*)img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg, cv);
+                          (const uint8_t*)img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg, cv, sq);
         }
         const SegPlan plan = plan_one_pass(B, Tn, H, dv, sms);
         const int P = plan.P;
@@ -381,7 +453,7 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
         const pfch::ChainSeg seg = P == 1 ? pfch::ChainSeg{1, plan.seg_chunks, nullptr, nullptr, nullptr, 0, 0}
                                           : pfch::ChainSeg{P, plan.seg_chunks, E, A, Qe, pfws::trans_ld(DK), 0};
         if (launch(chain, dim3(ns + (P > 1 ? 1 : 0), H, B * P), dim3(pfch::THREADS), smem, s, mk, mv, mvh, mhh,
-                   (const uint8_t*)img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg, cv) != JET_OK)
+                   (const uint8_t*)img, S0, (__nv_bfloat16*)o, S_out, Tn, H, dv, seg, cv, sq) != JET_OK)
             return JET_ERR_CUDA;
         if (P == 1) return JET_OK;
         // start states S*_1 .. S*_{P-1} and the final state
@@ -389,10 +461,10 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
         if (smem_attr(seg_combine_kernel<DK, true>, sc_smem) != JET_OK) return JET_ERR_CUDA;
         if (launch(seg_combine_kernel<DK, true>, dim3(dv / SC_ROWS, H, B), dim3(sc_threads(DK)), sc_smem, s,
                    (const float*)E, (const float*)A, (const float*)nullptr, (float*)nullptr, Sb, S_out, P, H, dv,
-                   CombineLayout{0, pfws::trans_ld(DK)}) != JET_OK)
+                   CombineLayout{0, pfws::trans_ld(DK)}, sq) != JET_OK)
             return JET_ERR_CUDA;
         // outputs of the segments p >= 1: O += Qe S*^T
-        return dispatch_correct<DK>(Qe, Sb, o, B, Tn, H, dv, nct, plan.seg_chunks, plan.seg_chunks, P, s);
+        return dispatch_correct<DK>(Qe, Sb, o, B, Tn, H, dv, nct, plan.seg_chunks, plan.seg_chunks, P, s, sq, 0);
     }
     auto fused = pfws::gdn_prefill_ws_kernel<DK>;
     if (smem_attr(fused, pfws::SMEM_BYTES) != JET_OK) return JET_ERR_CUDA;
@@ -415,7 +487,7 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
     if (smem_attr(seg_combine_kernel<DK, false>, sc_smem) != JET_OK) return JET_ERR_CUDA;
     if (launch(seg_combine_kernel<DK, false>, dim3(dv / SC_ROWS, H, B), dim3(sc_threads(DK)), sc_smem, s,
                (const float*)E, (const float*)A, S0, Sst, (__nv_bfloat16*)nullptr, (float*)nullptr, P, H, dv,
-               CombineLayout{0, pfws::trans_ld(DK)}) != JET_OK)
+               CombineLayout{0, pfws::trans_ld(DK)}, sq) != JET_OK)
         return JET_ERR_CUDA;
     // phase C: every segment from its start state, with outputs
     return run(dim3(ns, H, B * P), pfws::Seg{P, plan.seg_chunks, P, 0, Sst, nullptr, nullptr});
@@ -606,6 +678,82 @@ jet_status jet_jetblock_prefill(const void* x, const void* w1, const void* w2, c
     return dispatch_prefill<float>(dk, q, k, rest, g, beta, S0, o, S_out, B, T, H, dv, s);
 }
 
+// ---- variable-length batch: sequences of different lengths packed along the token axis
+namespace {
+// host cu_seqlens: nseq + 1 offsets, 0 first, strictly increasing; the total token count
+bool varlen_ok(const int* cu, int nseq, long long* total) {
+    if (!cu || nseq < 1 || nseq > pfws::kMaxVarlenSeqs || cu[0] != 0) return false;
+    for (int i = 0; i < nseq; ++i)
+        if (cu[i + 1] <= cu[i]) return false;
+    *total = cu[nseq];
+    return *total > 0 && *total < (1LL << 31);
+}
+size_t varlen_workspace(const int* cu, int nseq, int H, int dk, int dv, int sms) {
+    pfws::SeqMap sq;
+    plan_varlen(cu, nseq, H, dv, sms, sq);
+    const long long total = cu[nseq];
+    auto up = [](size_t x) { return (x + 1023) & ~size_t(1023); };
+    const size_t nchunks = (size_t)sq.chunk[nseq];
+    const size_t nsegs = (size_t)sq.seg[nseq];
+    return up((size_t)total * H * 4 * sizeof(float)) + nchunks * H * img_chunk_bytes(dk) +
+           (nsegs > (size_t)nseq ? one_pass_layout_n(nsegs, nchunks, H, dk, dv).bytes : 0);
+}
+}  // namespace
+
+size_t jet_jetblock_prefill_varlen_workspace_size(const int* cu_seqlens, int nseq, int H, int dk, int dv, int chunk,
+                                                  jet_dtype dt) {
+    long long total = 0;
+    if (H <= 0 || chunk != 64 || !varlen_ok(cu_seqlens, nseq, &total) || !tc_prefill_ok(dt, dk, dv, total)) return 0;
+    return varlen_workspace(cu_seqlens, nseq, H, dk, dv, kMaxSMs);
+}
+
+jet_status jet_jetblock_prefill_varlen(const void* x, const void* w1, const void* w2, const void* q, const void* k,
+                                       const void* v, const void* hist_in, void* hist_out, const float* g,
+                                       const float* beta, const float* S0, void* o, float* S_out, void* workspace,
+                                       size_t ws_bytes, const int* cu_seqlens, int nseq, int D, int H, int dk, int dv,
+                                       int hidden, int width, int chunk, jet_dtype dt, void* stream) {
+    long long total = 0;
+    if (!cu_seqlens || nseq < 1) return JET_ERR_INVALID_ARG;
+    if (nseq > pfws::kMaxVarlenSeqs) return JET_ERR_UNSUPPORTED;
+    if (!varlen_ok(cu_seqlens, nseq, &total)) return JET_ERR_INVALID_ARG;
+    jet_status st = check_gen(x, w1, w2, 1, (int)total, D, H, hidden, width, dt);
+    if (st != JET_OK) return st;
+    if (!q || !k || !v || !g || !beta || !o || !S_out) return JET_ERR_INVALID_ARG;
+    const long long nv = elems({total, H, dv}), nh = elems({nseq, 3, H, dv});
+    if (elems({total, H, dk}) < 0 || nv < 0 || nh < 0 || elems({nseq, H, dv, dk}) < 0) return JET_ERR_INVALID_ARG;
+    if (!shape_ok(dk, dv) || chunk != 64 || H > 65535) return JET_ERR_UNSUPPORTED;
+    if (!tc_prefill_ok(dt, dk, dv, total)) return JET_ERR_UNSUPPORTED;
+    for (const void* p : {q, k, v, hist_in, (const void*)hist_out, (const void*)S0, (const void*)o,
+                          (const void*)S_out, (const void*)workspace})
+        if (p && !aligned16(p)) return JET_ERR_MISALIGNED;
+    if (!aligned_to(g, 4) || !aligned_to(beta, 4)) return JET_ERR_MISALIGNED;
+    const size_t es = esize(dt), vb = (size_t)nv * es, hb = (size_t)nh * es;
+    if (overlap(v, vb, o, vb)) return JET_ERR_INVALID_ARG;
+    if (hist_out && (overlap(v, vb, hist_out, hb) || (hist_in && overlap(hist_in, hb, hist_out, hb))))
+        return JET_ERR_INVALID_ARG;
+    if (!workspace) ws_bytes = 0;
+    if (ws_bytes < varlen_workspace(cu_seqlens, nseq, H, dk, dv, kMaxSMs)) return JET_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    pfws::SeqMap sq;
+    plan_varlen(cu_seqlens, nseq, H, dv, launch_sms(), sq);
+    float* taps = static_cast<float*>(workspace);
+    uint8_t* rest = static_cast<uint8_t*>(workspace) + (((size_t)total * H * 4 * sizeof(float) + 1023) & ~size_t(1023));
+    st = total >= kGenMinTokens
+             ? launch_gen(x, w1, w2, taps, 1, (int)total, D, H, s)
+             : launch_genconv<__nv_bfloat16>(x, w1, w2, nullptr, nullptr, nullptr, nullptr, taps, 1, (int)total, D, H,
+                                             dv, s);
+    if (st != JET_OK) return st;
+    const pfch::ChainConv cv{static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(hist_in),
+                             static_cast<__nv_bfloat16*>(hist_out)};
+#define JET_TC(DK)                                                                                          \
+    return launch_prefill_tc<DK, true, true>(q, k, v, g, beta, S0, o, S_out, rest, nseq, 0, H, dv, s, taps, cv, \
+                                             RangeOut{}, &sq);
+    if (dk == 64) { JET_TC(64) }
+    if (dk == 96) { JET_TC(96) }
+    JET_TC(128)
+#undef JET_TC
+}
+
 // ---- sequence parallelism over token ranges (one range per GPU)
 size_t jet_jetblock_prefill_range_workspace_size(int B, int T, int H, int dk, int dv, int chunk, jet_dtype dt) {
     if (B <= 0 || T <= 0 || H <= 0 || chunk != 64 || !tc_prefill_ok(dt, dk, dv, (long long)B * T)) return 0;
@@ -671,7 +819,8 @@ jet_status jet_gdn_range_compose(const float* E, const float* A, void* Sb_out, f
         const size_t smem = sc_smem_bytes(DK);
         if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
         return launch(kern, dim3(dv / SC_ROWS, H, B), dim3(sc_threads(DK)), smem, s, E, A, (const float*)nullptr,
-                      (float*)nullptr, static_cast<__nv_bfloat16*>(Sb_out), S_out, R, H, dv, CombineLayout{1, DK});
+                      (float*)nullptr, static_cast<__nv_bfloat16*>(Sb_out), S_out, R, H, dv, CombineLayout{1, DK},
+                      no_seqmap());
     };
     if (dk == 64) return run(seg_combine_kernel<64, true>, 64);
     if (dk == 96) return run(seg_combine_kernel<96, true>, 96);
@@ -693,9 +842,9 @@ jet_status jet_gdn_range_correct(const void* Qe, const void* Sb, void* o, int B,
     const int nct = (T + 63) / 64;
     const __nv_bfloat16* qe = static_cast<const __nv_bfloat16*>(Qe);
     const __nv_bfloat16* sb = static_cast<const __nv_bfloat16*>(Sb);
-    if (dk == 64) return dispatch_correct<64>(qe, sb, o, B, T, H, dv, nct, 0, nct, 1, s);
-    if (dk == 96) return dispatch_correct<96>(qe, sb, o, B, T, H, dv, nct, 0, nct, 1, s);
-    return dispatch_correct<128>(qe, sb, o, B, T, H, dv, nct, 0, nct, 1, s);
+    if (dk == 64) return dispatch_correct<64>(qe, sb, o, B, T, H, dv, nct, 0, nct, 1, s, no_seqmap(), 0);
+    if (dk == 96) return dispatch_correct<96>(qe, sb, o, B, T, H, dv, nct, 0, nct, 1, s, no_seqmap(), 0);
+    return dispatch_correct<128>(qe, sb, o, B, T, H, dv, nct, 0, nct, 1, s, no_seqmap(), 0);
 }
 
 jet_status jet_gdn_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,

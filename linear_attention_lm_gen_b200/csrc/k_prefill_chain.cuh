@@ -166,7 +166,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ CUtensorMap tm_hh,
                          const uint8_t* __restrict__ img, const float* S0, __nv_bfloat16* __restrict__ o,
-                         float* S_out, int Tn, int H, int dv, const ChainSeg seg, const ChainConv cv) {
+                         float* S_out, int Tn, int H, int dv, const ChainSeg seg, const ChainConv cv,
+                         const __grid_constant__ SeqMap sq) {
     static_assert(DK % 32 == 0 && DK >= 64 && DK <= 128, "DK in {64, 96, 128}");
     using SM = ChainSmem<DK>;
     using IM = Img<DK>;
@@ -184,18 +185,40 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         return;
     }
     const int ns = dv / ROWS;
-    const int h = blockIdx.y, b = blockIdx.z / seg.nseg, p_seg = blockIdx.z % seg.nseg;
+    // this CTA's sequence b and its segment p_seg of P (gs: global segment index),
+    // the sequence's tokens Tb starting at row tok0, its chunks at nctH0 + h nct_b
+    const int h = blockIdx.y, gs = blockIdx.z;
+    int b, p_seg, P, Tb, tok0, nct, nctH0, segc;
+    if (sq.nseq == 0) {
+        P = seg.nseg;
+        b = gs / P;
+        p_seg = gs % P;
+        Tb = Tn;
+        tok0 = b * Tn;
+        nct = (Tn + C - 1) / C;
+        nctH0 = b * H * nct;
+        segc = seg.seg_chunks;
+    } else {
+        b = seq_of(sq.seg, sq.nseq, gs, 1);
+        p_seg = gs - sq.seg[b];
+        P = sq.seg[b + 1] - sq.seg[b];
+        tok0 = sq.tok[b];
+        Tb = sq.tok[b + 1] - tok0;
+        nct = sq.chunk[b + 1] - sq.chunk[b];
+        nctH0 = sq.chunk[b] * H;
+        segc = sq.seg_chunks;
+    }
     const bool trans = blockIdx.x == ns;                  // transition slice (p >= 1)
     if (trans && p_seg == 0 && !seg.trans0) return;      // whole CTA, before any barrier
     const int c0 = blockIdx.x * ROWS;                     // transition slice: past dv, V reads as zero
     const long long bh = (long long)b * H + h;
-    const int nct = (Tn + C - 1) / C;                     // chunks per sequence (image index)
-    const int cbeg = p_seg * seg.seg_chunks;
+    const int cbeg = p_seg * segc;
     const int tbeg = cbeg * C;
-    const int tend = min(Tn, tbeg + seg.seg_chunks * C);
+    const int tend = min(Tb, tbeg + segc * C);
     const int nch = (tend - tbeg + C - 1) / C;
     constexpr bool write_o = true;                        // every slice has output products (trans: Qe)
-    const uint8_t* img_bh = img + (size_t)bh * nct * IM::BYTES;
+    const long long img0 = (long long)nctH0 + (long long)h * nct;   // image / Qe index of the sequence's chunk 0
+    const uint8_t* img_bh = img + (size_t)img0 * IM::BYTES;
     auto img_at = [&](int c) -> const uint8_t* { return sm + SM::IMG + (uint32_t)(c & 1) * SM::IB; };
 
     if (tid == 0) {
@@ -367,13 +390,12 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         if (group_all(2, NCH_T, fin)) {
             tc_fence_after();
             float* dst = nullptr;
-            const long long bp = (long long)b * seg.nseg + p_seg;
             if (trans) {                                      // the transition (p >= 1, or range mode)
-                if (ct < DK) dst = seg.Ao + ((bp * H + h) * DK + ct) * seg.a_ld;
-            } else if (seg.nseg == 1) {
+                if (ct < DK) dst = seg.Ao + (((long long)gs * H + h) * DK + ct) * seg.a_ld;
+            } else if (P == 1) {
                 dst = S_out + (bh * dv + c0 + ct) * DK;
             } else {
-                dst = seg.Eo + ((bp * H + h) * dv + c0 + ct) * DK;
+                dst = seg.Eo + (((long long)gs * H + h) * dv + c0 + ct) * DK;
             }
 #pragma unroll
             for (int cb = 0; cb < DK / 32; ++cb) {
@@ -413,8 +435,8 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             const int t0 = tbeg + c * C, L = min(C, tend - t0);
             // value slices: o rows of this chunk; transition slice: Qe of the chunk
             // ([64 tokens][dk], rows of the slice = key features, only the first dk exist)
-            __nv_bfloat16* obase = trans ? seg.Qe + ((size_t)bh * nct + cbeg + c) * C * DK
-                                         : o + ((long long)b * Tn + t0) * tstride + (long long)h * dv + c0;
+            __nv_bfloat16* obase = trans ? seg.Qe + ((size_t)img0 + cbeg + c) * C * DK
+                                         : o + ((long long)tok0 + t0) * tstride + (long long)h * dv + c0;
             const long long rstride = trans ? (long long)DK : tstride;
             const int nchunk16 = trans ? DK / 8 : 16;
 #pragma unroll
@@ -444,13 +466,13 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         }
         if (!run) *abort_flag = 1;
         // CONV: the new history, the last three raw values of the sequence (or of the old history)
-        if (CONV && run && cv.hist_out && !trans && p_seg == seg.nseg - 1 && c0 + ot < dv) {
+        if (CONV && run && cv.hist_out && !trans && p_seg == P - 1 && c0 + ot < dv) {
             const int ch = c0 + ot;
 #pragma unroll
             for (int k3 = 0; k3 < 3; ++k3) {
-                const int tau = Tn - 3 + k3;
+                const int tau = Tb - 3 + k3;
                 __nv_bfloat16 val = __float2bfloat16_rn(0.f);
-                if (tau >= 0) val = cv.v[((long long)b * Tn + tau) * tstride + (long long)h * dv + ch];
+                if (tau >= 0) val = cv.v[((long long)tok0 + tau) * tstride + (long long)h * dv + ch];
                 else if (cv.hist_in) val = cv.hist_in[((long long)b * 3 + 3 + tau) * tstride + (long long)h * dv + ch];
                 cv.hist_out[((long long)b * 3 + k3) * tstride + (long long)h * dv + ch] = val;
             }
@@ -477,7 +499,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 return ok;
             };
             const uint32_t img_bytes = write_o ? IM::BYTES : IM::A_BYTES;
-            auto zrow = [&](int c) { return (int)((long long)b * Tn + tbeg + (long long)c * C); };
+            auto zrow = [&](int c) { return tok0 + tbeg + c * C; };
             auto load_img = [&](int c) {
                 uint64_t* bar = &bars[B_IMG + (c & 1)];
                 mbar_expect_tx(bar, img_bytes);
@@ -508,7 +530,7 @@ gdn_prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 // (coordinates below 0 read as zero; rows of other sequences only meet zero weights)
                 const bool from_hist = tbeg == 0 && cv.hist_in != nullptr;
                 const CUtensorMap* m = from_hist ? &tm_hh : &tm_vh;
-                const int z = from_hist ? b * 3 - 13 : (tbeg == 0 ? -16 : (int)((long long)b * Tn + tbeg - 16));
+                const int z = from_hist ? b * 3 - 13 : (tbeg == 0 ? -16 : tok0 + tbeg - 16);
                 tma_load_3d(dst, m, bar, c0, h, z);
                 tma_load_3d(dst + 8192, m, bar, c0 + 64, h, z);
             };

@@ -72,15 +72,17 @@ struct PrepSmem {
     static_assert(PREP_CTAS * (BYTES + 1024) <= 233472, "resident CTAs per SM");
 };
 
-// items = B * H * nct, item = (b * H + h) * nct + c (also the image index).
-// taps [B*T][H][4] or null: with taps the T1 slot holds M and MH is written
-// (the chain then reads raw values); halo0: whether the values before token 0
+// items = B * H * nct (dense) or H * (total chunks) (variable length), see
+// item_info; the item index is also the image index. taps [tokens][H][4] or
+// null: with taps the T1 slot holds M and MH is written (the chain then reads
+// raw values); halo0: whether the values before each sequence's first token
 // are a history (else MH of each sequence's first chunk is zero).
 template <int DK>
 __global__ void __launch_bounds__(PREP_THREADS, PREP_CTAS)
 gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const float* __restrict__ g, const float* __restrict__ beta, const float* __restrict__ taps,
-                      int halo0, uint8_t* __restrict__ img, int Tn, int H, int nct, int n_items) {
+                      int halo0, uint8_t* __restrict__ img, int Tn, int H, int nct, int n_items,
+                      const __grid_constant__ SeqMap sq) {
     using SM = PrepSmem<DK>;
     using IM = Img<DK>;
     constexpr int NKB = SM::NKB;
@@ -106,18 +108,14 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     pdl_wait();                                      // q, k, g, beta and the taps are read from here on
     pdl_trigger();
 
-    auto z_of = [&](int item) {                      // first token row of the item in the [B*T] axis
-        const int c = item % nct, b = item / nct / H;
-        return (int)((long long)b * Tn + (long long)c * C);
-    };
     auto issue_load = [&](int item, int buf) {       // thread 0
-        const int h = (item / nct) % H, z = z_of(item);
+        const ItemInfo it = item_info(item, Tn, H, nct, sq);
         uint8_t* dst = sm + SM::KQ + buf * SM::KQB;
         mbar_expect_tx(&bars[buf], (uint32_t)(NKB * 16384));
 #pragma unroll
         for (int kb = 0; kb < NKB; ++kb) {
-            tma_load_3d(dst + kb * 16384, &tm_k, &bars[buf], kb * 64, h, z);
-            tma_load_3d(dst + kb * 16384 + 8192, &tm_q, &bars[buf], kb * 64, h, z);
+            tma_load_3d(dst + kb * 16384, &tm_k, &bars[buf], kb * 64, it.h, it.z);
+            tma_load_3d(dst + kb * 16384 + 8192, &tm_q, &bars[buf], kb * 64, it.h, it.z);
         }
     };
     int nld[2] = {0, 0}, ndone[2] = {0, 0};          // loads issued / consumed per buffer (thread 0)
@@ -136,17 +134,17 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // g (tid < 64) or b (64 <= tid < 128) of one token of an item, 0 past the sequence end
     auto load_gb = [&](int item) -> float {
         if (item >= n_items || tid >= 128) return 0.f;
-        const int c = item % nct, h = (item / nct) % H;
-        if ((tid & 63) >= min(C, Tn - c * C)) return 0.f;
-        const long long off = ((long long)z_of(item) + (tid & 63)) * H + h;
+        const ItemInfo it = item_info(item, Tn, H, nct, sq);
+        if ((tid & 63) >= it.L) return 0.f;
+        const long long off = ((long long)it.z + (tid & 63)) * H + it.h;
         return tid < 64 ? g[off] : beta[off];
     };
     // taps of an item's tokens into TP[buf] (threads < 64; cp.async, zero past the sequence end)
     auto load_taps = [&](int item, int buf) {
         if (!taps || item >= n_items || tid >= 64) return;
-        const int c = item % nct, h = (item / nct) % H;
-        const bool in = tid < min(C, Tn - c * C);
-        const float* src = taps + (in ? ((long long)(z_of(item) + tid) * H + h) * 4 : 0);
+        const ItemInfo it = item_info(item, Tn, H, nct, sq);
+        const bool in = tid < it.L;
+        const float* src = taps + (in ? ((long long)(it.z + tid) * H + it.h) * 4 : 0);
         const uint32_t dst = smem_u32(sm + SM::TP) + (uint32_t)buf * TP_BYTES + (uint32_t)tp_slot(tid) * 16u;
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(in ? 16u : 0u)
                      : "memory");
@@ -159,7 +157,8 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
         const int buf = k % PREP_KQBUF;
         uint8_t* KQ = sm + SM::KQ + buf * SM::KQB;
-        const int L = min(C, Tn - (item % nct) * C);
+        const ItemInfo info = item_info(item, Tn, H, nct, sq);
+        const int L = info.L;
         uint8_t* out = img + (size_t)item * IM::BYTES;
         const float gb = gb_next;
         gb_next = load_gb(item + gridDim.x);            // in flight during this item
@@ -185,7 +184,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         ut_inverse(AF, XS, tid, 1);
         if (taps)
             prep_t1t2_conv(AF, V, reinterpret_cast<const float4*>(sm + SM::TP + (k & 1) * TP_BYTES), out + IM::T1,
-                           out + IM::MH, sm + SM::T2, halo0 || item % nct != 0, tid);
+                           out + IM::MH, sm + SM::T2, halo0 || info.c != 0, tid);
         else
             prep_t1t2(AF, V, out + IM::T1, sm + SM::T2, tid);
         load_taps(item + gridDim.x, (k + 1) & 1);      // the next item's taps, in flight from here

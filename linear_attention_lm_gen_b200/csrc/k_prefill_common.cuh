@@ -165,6 +165,58 @@ struct Seg {
 };
 
 
+// Variable-length batches (one launch over sequences of different lengths,
+// packed along the token axis): sequence i holds tokens tok[i] .. tok[i+1]-1,
+// chunks chunk[i] .. chunk[i+1]-1 of the per-chunk buffers (images, output
+// corrections) and segments seg[i] .. seg[i+1]-1 (all segments seg_chunks
+// long but the last of a sequence). The table rides in the kernel parameters,
+// so no device-side copy is needed. nseq == 0: the dense layout, B sequences
+// of Tn tokens, located by arithmetic.
+constexpr int kMaxVarlenSeqs = 256;
+struct SeqMap {
+    int nseq;
+    int seg_chunks;
+    int tok[kMaxVarlenSeqs + 1];
+    int chunk[kMaxVarlenSeqs + 1];
+    int seg[kMaxVarlenSeqs + 1];
+};
+// the sequence i with off[i] * mul <= x < off[i + 1] * mul (off increasing, off[0] = 0)
+__device__ __forceinline__ int seq_of(const int* off, int nseq, long long x, int mul) {
+    int lo = 0, hi = nseq - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((long long)off[mid] * mul <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// One preparation item = one (sequence, head, chunk); item index = image index:
+// dense (b H + h) nct + c, variable-length chunk[i] H + h nct_i + c.
+struct ItemInfo {
+    int z;        // first token row of the chunk in the token axis
+    int c;        // chunk within its sequence
+    int h;        // head
+    int L;        // tokens of the chunk (64, or fewer at the sequence end)
+};
+__device__ __forceinline__ ItemInfo item_info(int item, int Tn, int H, int nct, const SeqMap& sq) {
+    ItemInfo r;
+    if (sq.nseq == 0) {
+        r.c = item % nct;
+        r.h = (item / nct) % H;
+        const int b = item / nct / H;
+        r.z = b * Tn + r.c * C;
+        r.L = min(C, Tn - r.c * C);
+    } else {
+        const int i = seq_of(sq.chunk, sq.nseq, item, H);
+        const int nci = sq.chunk[i + 1] - sq.chunk[i], rr = item - sq.chunk[i] * H;
+        r.h = rr / nci;
+        r.c = rr % nci;
+        r.z = sq.tok[i] + r.c * C;
+        r.L = min(C, sq.tok[i + 1] - r.z);
+    }
+    return r;
+}
+
 // ---------------------------------------------------------------- preparation steps
 
 // Per-token vectors of one chunk: records g and b (gb: g for pt < 64, b for

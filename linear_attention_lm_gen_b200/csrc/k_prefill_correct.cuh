@@ -21,6 +21,7 @@
 // [w dv/8, (w+1) dv/8).
 #pragma once
 #include "common.cuh"
+#include "k_prefill_common.cuh"
 
 namespace jet {
 namespace pfcor {
@@ -53,13 +54,17 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// Qe [B][H][nct][64][DK] bf16; Sb [B][P][H][dv][DK] bf16 (the start state of
-// the segment of chunk gc is entry gc / seg_chunks); o [B*T][H][dv] bf16
-// (updated in place). Chunks chunk0 .. nct-1; grid (nct - chunk0, H, B).
+// Dense: Qe [B][H][nct][64][DK] bf16; Sb [B][P][H][dv][DK] bf16 (the start
+// state of the segment of chunk gc is entry gc / seg_chunks); o [B*T][H][dv]
+// bf16 (updated in place). Chunks chunk0 .. nct-1; grid (nct - chunk0, H, B).
+// Variable length (sq.nseq > 0): blockIdx.x runs over every chunk of every
+// sequence (grid (total chunks, H, 1)); chunks of a sequence's first segment
+// have nothing to add; Qe, Sb and the token rows follow the sequence map.
 template <int DK, int DV>
 __global__ void __launch_bounds__(THREADS)
 prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16* __restrict__ Sb,
-                       __nv_bfloat16* __restrict__ o, int Tn, int H, int nct, int chunk0, int seg_chunks, int P) {
+                       __nv_bfloat16* __restrict__ o, int Tn, int H, int nct, int chunk0, int seg_chunks, int P,
+                       const __grid_constant__ pfws::SeqMap sq) {
     static_assert(DK % 16 == 0 && DK <= 128 && DV % 64 == 0 && DV <= 256, "shapes");
     constexpr int LDA = lda(DK), LDO = ldo(DV);
     constexpr int NT = DV / 64;                    // n8 tiles per warp (DV / 8 columns)
@@ -69,18 +74,37 @@ prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16
     __nv_bfloat16* ss = qs + C * LDA;                                    // [DV][LDA]
     __nv_bfloat16* os = ss + DV * LDA;                                   // [64][LDO]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gc = chunk0 + blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    if (gc >= nct) return;
+    const int h = blockIdx.y;
+    // the chunk's index within its sequence, its Qe entry, its S* entry and its first token row
+    int gc, L;
+    long long qe_idx, sb_idx, row0;
+    if (sq.nseq == 0) {
+        const int b = blockIdx.z;
+        gc = chunk0 + blockIdx.x;
+        if (gc >= nct) return;
+        const int p = gc / seg_chunks;
+        qe_idx = ((long long)b * H + h) * nct + gc;
+        sb_idx = ((long long)b * P + p) * H + h;
+        row0 = (long long)b * Tn + (long long)gc * C;
+        L = min(C, Tn - gc * C);
+    } else {
+        const int x = blockIdx.x;
+        const int i = pfws::seq_of(sq.chunk, sq.nseq, x, 1);
+        gc = x - sq.chunk[i];
+        const int p = gc / sq.seg_chunks;
+        if (p == 0) return;
+        qe_idx = (long long)sq.chunk[i] * H + (long long)h * (sq.chunk[i + 1] - sq.chunk[i]) + gc;
+        sb_idx = ((long long)sq.seg[i] + p) * H + h;
+        row0 = (long long)sq.tok[i] + (long long)gc * C;
+        L = min(C, (int)(sq.tok[i + 1] - row0));
+    }
     pdl_wait();
     pdl_trigger();
-    const int p = gc / seg_chunks;
-    const int t0 = gc * C, L = min(C, Tn - t0);
-    const long long bh = (long long)b * H + h;
     const long long tstride = (long long)H * DV;
 
     // every copy of the three tiles in flight at once
     {   // Qe rows (zero past the sequence end: a 0-byte source fills zeros)
-        const __nv_bfloat16* src = Qe + ((size_t)bh * nct + gc) * C * DK;
+        const __nv_bfloat16* src = Qe + (size_t)qe_idx * C * DK;
 #pragma unroll
         for (int i = tid; i < C * DK / 8; i += THREADS) {
             const int r = i / (DK / 8), cc = i % (DK / 8);
@@ -88,7 +112,7 @@ prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16
         }
     }
     {   // S* of the segment
-        const __nv_bfloat16* src = Sb + ((((long long)b * P + p) * H + h) * DV) * DK;
+        const __nv_bfloat16* src = Sb + (size_t)sb_idx * DV * DK;
 #pragma unroll
         for (int i = tid; i < DV * DK / 8; i += THREADS) {
             const int r = i / (DK / 8), cc = i % (DK / 8);
@@ -99,7 +123,7 @@ prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16
 #pragma unroll
         for (int i = tid; i < C * DV / 8; i += THREADS) {
             const int r = i / (DV / 8), cc = i % (DV / 8);
-            if (r < L) cp_async16(os + r * LDO + cc * 8, o + ((long long)b * Tn + t0 + r) * tstride + h * DV + cc * 8, 16u);
+            if (r < L) cp_async16(os + r * LDO + cc * 8, o + (row0 + r) * tstride + h * DV + cc * 8, 16u);
         }
     }
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
@@ -148,7 +172,7 @@ prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16
     for (int i = tid; i < C * DV / 8; i += THREADS) {
         const int r = i / (DV / 8), cc = i % (DV / 8);
         if (r < L)
-            *reinterpret_cast<uint4*>(o + ((long long)b * Tn + t0 + r) * tstride + h * DV + cc * 8) =
+            *reinterpret_cast<uint4*>(o + (row0 + r) * tstride + h * DV + cc * 8) =
                 *reinterpret_cast<const uint4*>(os + r * LDO + cc * 8);
     }
 }

@@ -65,12 +65,18 @@ struct CombineLayout {
 // (FINAL) or P - 1; start states Sst [B][P][H][dv][dk] float32 (two passes)
 // or Sb bf16 (FINAL, same layout as E); grid (dv / 16, H, B), sc_threads(DK)
 // threads, sc_smem_bytes(DK) shared.
+// Variable-length batches (FINAL, sq.nseq > 0): sequence b has segments
+// sq.seg[b] .. sq.seg[b+1]-1 of E, A and Sb ([global segment][H]...); a
+// sequence of one segment has nothing to combine (the pass wrote its final
+// state).
 template <int DK, bool FINAL>
 __global__ void __launch_bounds__(4 * DK)
 seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, const float* S0,
-                   float* __restrict__ Sst, __nv_bfloat16* __restrict__ Sb, float* S_out, int P, int H, int dv,
-                   const CombineLayout lay) {
+                   float* __restrict__ Sst, __nv_bfloat16* __restrict__ Sb, float* S_out, int Pn, int H, int dv,
+                   const CombineLayout lay, const __grid_constant__ pfws::SeqMap sq) {
     static_assert(DK % 8 == 0 && DK <= 128, "dk");
+    const int P = sq.nseq > 0 ? sq.seg[blockIdx.z + 1] - sq.seg[blockIdx.z] : Pn;
+    if (P < 2) return;                           // whole CTA, before any barrier
     const int NE = FINAL ? P : P - 1;            // segments with an end state / transition
     const int last = FINAL ? P - 1 : P - 2;      // the last step p computes S_start(p + 1)
     constexpr int LDE = sc_lde(DK);
@@ -90,7 +96,10 @@ seg_combine_kernel(const float* __restrict__ E, const float* __restrict__ A, con
     const int g = lane >> 2, t = lane & 3, n0 = warp * 8;
     const int r0 = blockIdx.x * SC_ROWS, h = blockIdx.y, b = blockIdx.z, nb = gridDim.z;
     // (segment, sequence) -> index of the [H] block
-    auto sb_idx = [&](int p, int n) { return lay.seg_major ? (long long)p * nb + b : (long long)b * n + p; };
+    auto sb_idx = [&](int p, int n) {
+        if (sq.nseq > 0) return (long long)sq.seg[b] + p;
+        return lay.seg_major ? (long long)p * nb + b : (long long)b * n + p;
+    };
     auto e_at = [&](int p) { return E + ((sb_idx(p, NE) * H + h) * dv + r0) * DK; };
     auto s_at = [&](int p) {                     // S_start(p) (two passes); the final state (FINAL)
         return (FINAL && p == P) ? S_out + (((long long)b * H + h) * dv + r0) * DK

@@ -13,8 +13,9 @@ the library's calls on them:
                `chunk_tokens` (chunked prefill), each piece continuing from
                the entry's state and history (jet_jetblock_prefill)
   prefill_many({seq: ...})  the same for several sequences of different
-               lengths: in every round, the pieces of equal length run as one
-               batched call
+               lengths: in every round, the pieces of all of them run as one
+               variable-length call (jet_jetblock_prefill_varlen; shapes off
+               the tensor-core path batch pieces of equal length instead)
   decode(seqs, ...)  one new token for each of a batch of sequences, in place
                on their entries (jet_jetblock_decode_slots)
   release(seq) return the entry
@@ -34,7 +35,10 @@ from __future__ import annotations
 
 import torch
 
-from . import jet_jetblock_decode_slots, jet_jetblock_prefill, jet_jetblock_prefill_workspace_size
+from . import (jet_jetblock_decode_slots, jet_jetblock_prefill, jet_jetblock_prefill_varlen,
+               jet_jetblock_prefill_workspace_size)
+
+MAX_VARLEN_SEQS = 256    # sequences per variable-length call
 
 
 class JetEngine:
@@ -105,16 +109,28 @@ class JetEngine:
             self.pos[seq] += t1 - t0
         return torch.cat(outs) if len(outs) > 1 else outs[0]
 
+    @property
+    def varlen(self) -> bool:
+        """Whether prefill_many can pack pieces of different lengths into one
+        call (the variable-length prefill takes the tensor-core shapes)."""
+        return self.W1.dtype == torch.bfloat16 and self.dk in (64, 96, 128) and self.dv % 128 == 0
+
     def prefill_many(self, prompts: dict) -> dict:
         """Chunked prefill of several sequences at once. prompts: seq ->
         (x, q, k, v, g, beta) as for prefill (lengths may differ). Round r
-        takes the r-th piece of every sequence that has one; pieces of equal
-        length (every full piece, and tails that happen to match) share one
-        batched jet_jetblock_prefill call. Returns seq -> o [T,H,dv]."""
+        takes the r-th piece of every sequence that has one; all of them run
+        as one variable-length call (packed along the token axis), or, off the
+        tensor-core shapes, pieces of equal length share one batched call.
+        Returns seq -> o [T,H,dv]."""
         outs = {seq: [] for seq in prompts}
         plan = {seq: self.pieces(inp[0].shape[0]) for seq, inp in prompts.items()}
         for r in range(max((len(p) for p in plan.values()), default=0)):
             groups: dict = {}
+            if self.varlen:
+                live = [seq for seq, p in plan.items() if r < len(p)]
+                for i in range(0, len(live), MAX_VARLEN_SEQS):
+                    self._prefill_packed(prompts, plan, r, live[i:i + MAX_VARLEN_SEQS], outs)
+                continue
             for seq, p in plan.items():
                 if r < len(p):
                     groups.setdefault(p[r][1] - p[r][0], []).append(seq)
@@ -133,6 +149,24 @@ class JetEngine:
                     outs[sq].append(o[b])
                     self.pos[sq] += L
         return {sq: torch.cat(v) if len(v) > 1 else v[0] for sq, v in outs.items()}
+
+    def _prefill_packed(self, prompts, plan, r, seqs, outs):
+        """Round r's pieces of `seqs` as one variable-length call."""
+        lens = [plan[sq][r][1] - plan[sq][r][0] for sq in seqs]
+        cu = [0]
+        for n in lens:
+            cu.append(cu[-1] + n)
+        idx = torch.tensor([self.slot[sq] for sq in seqs], device=self.S.device)
+        S = self.S.index_select(0, idx)
+        hin = self.hist.index_select(0, idx)
+        hout = torch.empty_like(hin)
+        packed = [torch.cat([prompts[sq][j][plan[sq][r][0]:plan[sq][r][1]] for sq in seqs]) for j in range(6)]
+        o, _ = jet_jetblock_prefill_varlen(packed[0], self.W1, self.W2, *packed[1:], cu, hin, hout, S, None, S)
+        self.S.index_copy_(0, idx, S)
+        self.hist.index_copy_(0, idx, hout)
+        for i, sq in enumerate(seqs):
+            outs[sq].append(o[cu[i]:cu[i + 1]])
+            self.pos[sq] += lens[i]
 
     # ---------------------------------------------------------------- serving iterations
     def submit(self, seq, prompt) -> None:

@@ -351,3 +351,41 @@ def test_range_correct_rejects(lib, kw, expect):
     a.update(kw)
     assert lib.jet_gdn_range_correct(P(a["Qe"]), P(a["Sb"]), P(a["o"]), a["B"], a["T"], a["H"], a["dk"], a["dv"],
                                      a["dt"], None) == expect
+
+
+def prefill_varlen(lib, x=A, w1=A, w2=A, q=A, k=A, v=A, hin=None, hout=None, g=A, b=A, S0=None, o=A + (1 << 24),
+                   S=A + (1 << 26), ws=A, ws_bytes=1 << 30, cu=(0, 100, 300), nseq=None, D=64, H=2, dk=96, dv=128,
+                   hidden=32, width=4, chunk=64, dt=BF16):
+    arr = None if cu is None else (ctypes.c_int * len(cu))(*cu)
+    n = (len(cu) - 1 if cu is not None else 2) if nseq is None else nseq
+    return lib.jet_jetblock_prefill_varlen(P(x), P(w1), P(w2), P(q), P(k), P(v), P(hin), P(hout), P(g), P(b), P(S0),
+                                           P(o), P(S), P(ws), ws_bytes, arr, n, D, H, dk, dv, hidden, width, chunk,
+                                           dt, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(cu=None), INVALID), (dict(cu=(0, 100, 100)), INVALID),     # offsets: present, strictly increasing
+    (dict(cu=(5, 100)), INVALID), (dict(cu=(0,), nseq=0), INVALID),  # from 0; at least one sequence
+    (dict(cu=tuple(range(0, 2580, 10))), UNSUPPORTED),              # 257 sequences: more than one call takes
+    (dict(dk=48), UNSUPPORTED), (dict(dt=F32), UNSUPPORTED),         # tensor-core shapes only
+    (dict(dv=96), UNSUPPORTED), (dict(chunk=32), UNSUPPORTED),
+    (dict(o=A + 64), INVALID), (dict(q=None), INVALID),              # o may not overlap v
+    (dict(S=A + (1 << 26) + 8), MISALIGNED), (dict(hout=A + (1 << 27) + 4), MISALIGNED),
+    (dict(ws_bytes=1024), WORKSPACE), (dict(ws=None), WORKSPACE),
+])
+def test_prefill_varlen_rejects(lib, kw, expect):
+    assert prefill_varlen(lib, **kw) == expect
+
+
+def test_prefill_varlen_workspace(lib):
+    # lengths 1, 62, 237, 1253, 2543: one segment each fits one wave at H = 12, so the workspace
+    # is the taps of every token plus one image per chunk (66 chunks), no one-pass buffers
+    cu = [0, 1, 63, 300, 1553, 4096]
+    H, dk, dv = 12, 96, 256
+    assert jet.jet_jetblock_prefill_varlen_workspace_size(cu, H, dk, dv) == 4096 * H * 16 + 66 * H * 48128
+    # two long prompts over two heads are split into segments: the one-pass buffers come on top
+    two = jet.jet_jetblock_prefill_varlen_workspace_size([0, 4096, 8192], 2, dk, dv)
+    assert two > -(-8192 * 2 * 16 // 1024) * 1024 + 128 * 2 * 48128
+    assert jet.jet_jetblock_prefill_varlen_workspace_size(cu, H, 48, dv) == 0      # not a tensor-core shape
+    assert jet.jet_jetblock_prefill_varlen_workspace_size([0, 10, 5], H, dk, dv) == 0
+    assert jet.jet_jetblock_prefill_varlen_workspace_size(list(range(0, 2580, 10)), H, dk, dv) == 0

@@ -214,3 +214,35 @@ def test_submit_rejects_empty_and_ragged_prompts(engine):
     with pytest.raises(ValueError):
         e.submit("ragged", ragged)
     assert e.free_slots == 3 and e.prefilling == []
+
+
+def test_prefill_many_packs_every_piece_of_a_round_into_one_call(monkeypatch):
+    # bf16 tensor-core shapes: each round is one variable-length call over all live sequences
+    calls = []
+
+    def fake_varlen(x, W1, W2, q, k, v, g, beta, cu, hist_in, hist_out, S0, o, S_out):
+        calls.append(list(cu))
+        assert S0.data_ptr() == S_out.data_ptr()
+        hist_out.copy_(hist_in + 1)
+        for i in range(len(cu) - 1):
+            S_out[i] += cu[i + 1] - cu[i]
+        return torch.full((cu[-1], 2, 128), float(len(calls))), S_out
+    monkeypatch.setattr(eng, "jet_jetblock_prefill_varlen", fake_varlen)
+    bf = torch.bfloat16
+    e = eng.JetEngine(torch.zeros(64, 32, dtype=bf), torch.zeros(32, 8, dtype=bf), 2, 64, 128, max_seqs=4,
+                      chunk_tokens=100)
+    assert e.varlen
+    lens = {"a": 250, "b": 60, "c": 100}
+    for sq in lens:
+        e.admit(sq)
+    p = lambda T: (torch.zeros(T, 64), torch.zeros(T, 2, 64), torch.zeros(T, 2, 64), torch.zeros(T, 2, 128),
+                   torch.zeros(T, 2), torch.zeros(T, 2))
+    out = e.prefill_many({sq: p(T) for sq, T in lens.items()})
+    # round 0: a 100, b 60, c 100; round 1: a 100; round 2: a 50
+    assert calls == [[0, 100, 160, 260], [0, 100], [0, 50]]
+    assert {sq: o.shape[0] for sq, o in out.items()} == lens
+    assert e.pos == lens
+    for sq, T in lens.items():
+        assert float(e.S[e.slot[sq]].flatten()[0]) == T            # every piece advanced its own state
+        rounds = (T + 99) // 100
+        assert float(e.hist[e.slot[sq]].flatten()[0]) == rounds    # and its own history, once per round
