@@ -9,11 +9,13 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "k_decode.cuh"
 #include "k_gen.cuh"
 #include "k_genconv.cuh"
+#include "k_genconv_decode.cuh"
 #include "k_prefill_simt.cuh"
 #include "k_prefill_chain.cuh"
 #include "k_prefill_correct.cuh"
@@ -121,10 +123,68 @@ jet_status launch_genconv_t(const void* x, const void* w1, const void* w2, const
     return launch_status();
 }
 
+// One new token per sequence, bf16: the decode kernel (one round trip to
+// memory). Returns JET_ERR_UNSUPPORTED, before any launch, where its
+// alignment or shared-memory needs are not met (the caller then takes the
+// general kernel).
+template <int TB>
+jet_status launch_genconv_decode_t(const void* x, const void* w1, const void* w2, const void* v, const void* hin,
+                                   void* vout, void* hout, float* cw, int B, int D, int H, int dv, int groups,
+                                   int hpc, int per, size_t smem, cudaStream_t s, const int* slots, int n_slots) {
+    auto kern = gcd::genconv_decode_kernel<TB>;
+    if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((B + TB - 1) / TB), (unsigned)groups);
+    cfg.blockDim = dim3(gcd::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = (unsigned)groups;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, (const __nv_bfloat16*)x, (const __nv_bfloat16*)w1,
+                                             (const __nv_bfloat16*)w2, (const __nv_bfloat16*)v,
+                                             (const __nv_bfloat16*)hin, (__nv_bfloat16*)vout, (__nv_bfloat16*)hout, cw,
+                                             B, D, H, dv, hpc, per, slots, n_slots);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (e != cudaSuccess) return JET_ERR_CUDA;
+    return launch_status();
+}
+
+jet_status launch_genconv_decode(const void* x, const void* w1, const void* w2, const void* v, const void* hin,
+                                 void* vout, void* hout, float* cw, int B, int D, int H, int dv, cudaStream_t s,
+                                 const int* slots, int n_slots) {
+    if (!aligned_to(w1, 16) || !aligned_to(w2, 8) || (v && dv % 8 != 0)) return JET_ERR_UNSUPPORTED;
+    const int TB = B <= 512 ? 8 : 16;
+    const long long nblk = ((long long)B + TB - 1) / TB;
+    // head groups (= cluster size, at most 8): enough CTAs to cover the SMs
+    // about twice, then as few groups as give every group a head
+    int groups = 1;
+    while (groups < H && groups < 8 && nblk * groups < 296) ++groups;
+    const int hpc = (H + groups - 1) / groups;
+    groups = (H + hpc - 1) / hpc;
+    const int per = (D / 16 + groups - 1) / groups;
+    const size_t smem = gcd::layout(per * 16, hpc * GC_W).bytes;
+    if (smem > 200 * 1024 || nblk > 0x7fffffffLL) return JET_ERR_UNSUPPORTED;
+    return TB == 8 ? launch_genconv_decode_t<8>(x, w1, w2, v, hin, vout, hout, cw, B, D, H, dv, groups, hpc, per, smem,
+                                                s, slots, n_slots)
+                   : launch_genconv_decode_t<16>(x, w1, w2, v, hin, vout, hout, cw, B, D, H, dv, groups, hpc, per,
+                                                 smem, s, slots, n_slots);
+}
+
 template <typename T>
 jet_status launch_genconv(const void* x, const void* w1, const void* w2, const void* v, const void* hin,
                           void* vout, void* hout, float* cw, int B, int Tn, int D, int H, int dv,
                           cudaStream_t s, const int* slots = nullptr, int n_slots = 0) {
+    if (std::is_same<T, __nv_bfloat16>::value && Tn == 1) {
+        const jet_status st = launch_genconv_decode(x, w1, w2, v, hin, vout, hout, cw, B, D, H, dv, s, slots, n_slots);
+        if (st != JET_ERR_UNSUPPORTED) return st;
+    }
     constexpr int TB = 16;
     // a state-cache slot index applies to one token per sequence only (the
     // one-token work items look the slot up per item)
@@ -510,21 +570,28 @@ jet_status dispatch_prefill(int dk, const void* q, const void* k, const void* v,
 template <typename T, int NV>
 jet_status launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          float* S, void* o, int B, int H, int dv, const DecConv* conv, cudaStream_t s,
-                         const int* slots, int n_slots) {
+                         const int* slots, int n_slots, int early) {
     const dim3 grid((dv + DEC_ROWS - 1) / DEC_ROWS, H, B);
+    // the state stream wants the largest L1 (it holds the loads in flight): ask for the
+    // smallest shared-memory carve-out, also while the previous launch's CTAs with a
+    // large one still share the SM
+    auto kern = conv ? gdn_decode_kernel<T, NV, true> : gdn_decode_kernel<T, NV>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 0) != cudaSuccess)
+        return JET_ERR_CUDA;
     if (conv)
         return launch(gdn_decode_kernel<T, NV, true>, grid, dim3(DEC_THREADS), 0, s, (const T*)q, (const T*)k,
-                      (const T*)v, g, beta, S, (T*)o, H, dv, *conv, slots, n_slots);
+                      (const T*)v, g, beta, S, (T*)o, H, dv, *conv, slots, n_slots, early);
     return launch(gdn_decode_kernel<T, NV>, grid, dim3(DEC_THREADS), 0, s, (const T*)q, (const T*)k, (const T*)v, g,
-                  beta, S, (T*)o, H, dv, DecConv{}, slots, n_slots);
+                  beta, S, (T*)o, H, dv, DecConv{}, slots, n_slots, early);
 }
 
 template <typename T>
 jet_status dispatch_decode(int dk, const void* q, const void* k, const void* v, const float* g,
                            const float* beta, float* S, void* o, int B, int H, int dv, cudaStream_t s,
-                           const DecConv* conv = nullptr, const int* slots = nullptr, int n_slots = 0) {
+                           const DecConv* conv = nullptr, const int* slots = nullptr, int n_slots = 0,
+                           int early = 0) {
     switch (dk / 16) {
-#define JET_CASE(NV) case NV: return launch_decode<T, NV>(q, k, v, g, beta, S, o, B, H, dv, conv, s, slots, n_slots);
+#define JET_CASE(NV) case NV: return launch_decode<T, NV>(q, k, v, g, beta, S, o, B, H, dv, conv, s, slots, n_slots, early);
         JET_CASE(1) JET_CASE(2) JET_CASE(3) JET_CASE(4) JET_CASE(5) JET_CASE(6) JET_CASE(7) JET_CASE(8)
 #undef JET_CASE
         default: return JET_ERR_UNSUPPORTED;
@@ -902,7 +969,12 @@ jet_status jet_jetblock_decode_step(const void* x, const void* w1, const void* w
     // the taps of the new tokens, then conv + history shift + decode update in one pass over S
     st = jet_kernel_gen(x, w1, w2, taps, B, 1, D, H, hidden, width, dt, stream);
     if (st != JET_OK) return st;
-    return jet_conv_gdn_decode_step(q, k, v, hist_in, hist_out, taps, g, beta, S, o, B, H, dk, dv, dt, stream);
+    // the generator writes only the taps: the decode launch reads the state before it waits for them
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const DecConv conv{taps, hist_in, hist_out};
+    if (dt == JET_BF16)
+        return dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, B, H, dv, s, &conv, nullptr, 0, 1);
+    return dispatch_decode<float>(dk, q, k, v, g, beta, S, o, B, H, dv, s, &conv, nullptr, 0, 1);
 }
 
 jet_status jet_jetblock_decode_slots(const void* x, const void* w1, const void* w2, const void* q, const void* k,
@@ -934,8 +1006,8 @@ jet_status jet_jetblock_decode_slots(const void* x, const void* w1, const void* 
     if (st != JET_OK) return st;
     if (dt == JET_BF16)
         return dispatch_decode<__nv_bfloat16>(dk, q, k, v_conv, g, beta, S_pool, o, B, H, dv, s, nullptr, slots,
-                                              n_slots);
-    return dispatch_decode<float>(dk, q, k, v_conv, g, beta, S_pool, o, B, H, dv, s, nullptr, slots, n_slots);
+                                              n_slots, 1);
+    return dispatch_decode<float>(dk, q, k, v_conv, g, beta, S_pool, o, B, H, dv, s, nullptr, slots, n_slots, 1);
 }
 
 jet_status jet_device_error(void* stream) {

@@ -43,13 +43,19 @@ struct DecConv {
     const void* hist_in;     // null: zero history
     void* hist_out;
 };
+// early != 0: the previous kernel on the stream is the same library call's
+// generator / conv launch, which writes only the taps (CONV) or the values v
+// (no CONV). Everything else the kernel reads was complete before that
+// launch began, so the state rows and the token vectors are read before the
+// wait for it, and only the taps / v after (the state stream of the first CTAs
+// then overlaps the generator).
 
 template <typename T, int NV, bool CONV = false>   // NV = dk / 16 float4 per lane
 __global__ void __launch_bounds__(DEC_THREADS, NV <= 6 ? 3 : 2)   // 3 CTAs per SM where the registers allow
 gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const float* __restrict__ g, const float* __restrict__ beta,
                   float* __restrict__ S, T* __restrict__ o, int H, int dv, DecConv cv = {},
-                  const int* __restrict__ slots = nullptr, int n_slots = 0) {
+                  const int* __restrict__ slots = nullptr, int n_slots = 0, int early = 0) {
     constexpr int DK = NV * 16;
     __shared__ __align__(16) float sk[DK];
     __shared__ __align__(16) float sq[DK];
@@ -57,7 +63,7 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.y, b = blockIdx.z;
     const long long bh = (long long)b * H + h;                // token inputs and outputs
-    pdl_wait();
+    if (!early) pdl_wait();
     pdl_trigger();
     int sb = b;                                               // state / history entry
     if (slots) {
@@ -84,8 +90,13 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             s1[i] = ok1 ? ld_stream_f4(r1 + part + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
-    float vi0 = ok0 ? Elem<T>::ld(v + bh * dv + row0) : 0.f;
-    float vi1 = ok1 ? Elem<T>::ld(v + bh * dv + row1) : 0.f;
+    // the raw v (CONV) never comes from the previous launch; a conv's output may
+    float vi0 = 0.f, vi1 = 0.f;
+    auto load_v = [&]() {
+        vi0 = ok0 ? Elem<T>::ld(v + bh * dv + row0) : 0.f;
+        vi1 = ok1 ? Elem<T>::ld(v + bh * dv + row1) : 0.f;
+    };
+    if (CONV || !early) load_v();
     // conv inputs: the raw history of both rows (v_{t-3}, v_{t-2}, v_{t-1}), loaded
     // now and used only after the prologue below, so their latency overlaps it
     float hv0[3] = {0.f, 0.f, 0.f}, hv1[3] = {0.f, 0.f, 0.f};
@@ -93,7 +104,7 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     const long long hs = (long long)H * dv;                               // slot stride
     float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
     if constexpr (CONV) {
-        w = *reinterpret_cast<const float4*>(cv.taps + bh * 4);
+        if (!early) w = *reinterpret_cast<const float4*>(cv.taps + bh * 4);
         const T* hin = static_cast<const T*>(cv.hist_in);
         if (hin) {
 #pragma unroll
@@ -143,6 +154,11 @@ gdn_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         p1 += __shfl_xor_sync(0xffffffffu, p1, m);
     }
     u0 *= inv_k; u1 *= inv_k; p0 *= inv_q; p1 *= inv_q;
+    if (early) {                                      // the previous launch's output from here on
+        pdl_wait();
+        if constexpr (CONV) w = *reinterpret_cast<const float4*>(cv.taps + bh * 4);
+        else load_v();
+    }
     if constexpr (CONV) {   // v' of both rows, and the shifted history
         T* hout = static_cast<T*>(cv.hist_out);
         auto conv_row = [&](int row, float raw, const float* hv) -> float {
