@@ -77,7 +77,7 @@ constexpr int THREADS = NCH_T + NOUT + 96;            // 352
 constexpr int OUT0 = NCH_T, LOAD0 = NCH_T + NOUT + 64;   // warp 10
 
 // bounded wait: spin on the phase first, then poll with short sleeps; gives up
-// (error word + CTA abort flag) when the poll budget runs out or another
+// (error word + CTA abort flag) when the wait time limit runs out or another
 // thread raised the abort flag
 __device__ __forceinline__ bool wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     for (uint32_t i = 0; i < 2048; ++i)

@@ -84,3 +84,27 @@ def test_varlen_prefill_agrees_with_one_call_per_prompt():
                                           S0=dev(S0[i:i + 1], "f32"))
         assert_close(host64(o[cu[i]:cu[i + 1]]), host64(o1[0]), "bf16", f"o of prompt {i}")
         assert_close(host64(S[i]), host64(S1[0]), "bf16", f"S of prompt {i}")
+
+
+def test_varlen_prefill_normalises_q_and_k():
+    # q and k rows of spread norms (10**U(-1, 1)), one key row and one query row exactly zero,
+    # in different prompts: every prompt must still match the oracle, which normalises in float64
+    lens = [70, 1, 200]
+    per, packed, W1, W2, S0 = packed_inputs(lens, 2, 96, 128, 64, seed=97)
+    packed["k"] = synth.spread_qk_norms(packed["k"], "bf16", 3, zero_rows=[(75, 1)])
+    packed["q"] = synth.spread_qk_norms(packed["q"], "bf16", 4, zero_rows=[(10, 0)])
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    d = {key: dev(val, "bf16") for key, val in packed.items() if key not in ("g", "beta")}
+    d["g"], d["beta"] = dev(packed["g"], "f32"), dev(packed["beta"], "f32")
+    o, S = jet.jet_jetblock_prefill_varlen(d["x"], dev(W1, "bf16"), dev(W2, "bf16"), d["q"], d["k"], d["v"], d["g"],
+                                           d["beta"], cu, S0=dev(S0, "f32"))
+    assert jet.jet_device_error() == 0
+    orc = get_oracle()
+    f = lambda a: synth.to_f64(a, "bf16")
+    for i in range(len(lens)):
+        a, b = cu[i], cu[i + 1]
+        r = orc.jetblock_prefill(f(packed["x"][a:b])[None], f(W1), f(W2), f(packed["q"][a:b])[None],
+                                 f(packed["k"][a:b])[None], f(packed["v"][a:b])[None], packed["g"][a:b][None],
+                                 packed["beta"][a:b][None], S0[i:i + 1].astype(np.float64))
+        assert_close(host64(o[a:b]), r["o"][0], "bf16", f"o of prompt {i}")
+        assert_close(host64(S[i]), r["S"][0], "bf16", f"S of prompt {i}")
