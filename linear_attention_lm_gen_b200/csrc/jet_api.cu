@@ -472,7 +472,7 @@ jet_status launch_prefill_tc(const void* q, const void* k, const void* v, const 
             const int grid = (int)std::min<long long>(items, (long long)pfws::PREP_CTAS * sms);   // resident CTAs
             if (launch(prep, dim3(grid), dim3(pfws::PREP_THREADS), pfws::PrepSmem<DK>::BYTES, s, mq, mk, g, beta,
                        CONV ? taps : nullptr, (int)(cv.hist_in != nullptr), img, Tn, H, nct, (int)items,
-                       sq) != JET_OK)
+                       sq, (int)CONV) != JET_OK)
                 return JET_ERR_CUDA;
         }
         if (vsq) {   // variable length: the segments of the plan in the sequence map

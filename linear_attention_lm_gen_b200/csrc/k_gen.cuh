@@ -5,7 +5,9 @@
 //
 // One CTA = GT = 32 consecutive tokens of the flattened [B*T] token axis.
 // x[GT][D] and W1[D][32] stream through shared memory in slices of KC = 128
-// columns of D (cp.async, NST - 1 slices in flight); CTA b starts at slice
+// columns of D (cp.async, NST - 1 slices in flight; four buffers, 75 KB, leave
+// room on the SM for two CTAs of the chunk preparation that follows, which
+// starts before this kernel ends); CTA b starts at slice
 // b mod (slices), so the CTAs do not all ask for the same W1 lines at once. In every slice warp w takes
 // k-step w (16 columns) of the whole 32 x 32 product: 2 x 4 bf16
 // m16n8k16 tensor-core MMAs with float32 accumulation, operands by ldmatrix
@@ -23,7 +25,7 @@ constexpr int THREADS = 256;
 constexpr int GT = 32;                  // tokens per CTA
 constexpr int HID = 32;                 // generator hidden width
 constexpr int KC = 128;                 // columns of D per slice
-constexpr int NST = 10;                 // slice buffers (NST - 1 in flight)
+constexpr int NST = 4;                  // slice buffers (NST - 1 in flight)
 constexpr int XLD = KC * 2 + 16;        // x slice row stride in bytes (16-byte pad: conflict-free ldmatrix)
 constexpr int WLD = HID * 2 + 16;       // W1 slice row stride in bytes
 constexpr int XS_BYTES = GT * XLD;      // 8704

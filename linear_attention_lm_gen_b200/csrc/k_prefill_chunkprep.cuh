@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(PREP_THREADS, PREP_CTAS)
 gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const float* __restrict__ g, const float* __restrict__ beta, const float* __restrict__ taps,
                       int halo0, uint8_t* __restrict__ img, int Tn, int H, int nct, int n_items,
-                      const __grid_constant__ SeqMap sq) {
+                      const __grid_constant__ SeqMap sq, int early) {
     using SM = PrepSmem<DK>;
     using IM = Img<DK>;
     constexpr int NKB = SM::NKB;
@@ -105,7 +105,11 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = *tslot;
-    pdl_wait();                                      // q, k, g, beta and the taps are read from here on
+    // The previous launch is waited for before the first global read, except
+    // with `early`: then it is the same call's generator, which writes only the
+    // taps, and everything else was complete before it began; q, k, g and beta
+    // are read at once and the wait comes just before the first taps are.
+    if (!early) pdl_wait();
     pdl_trigger();
 
     auto issue_load = [&](int item, int buf) {       // thread 0
@@ -152,7 +156,7 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     };
     bool ok = true;
     int k = 0;
-    load_taps(blockIdx.x, 0);
+    if (!early) load_taps(blockIdx.x, 0);
     float gb_next = load_gb(blockIdx.x);
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
         const int buf = k % PREP_KQBUF;
@@ -176,10 +180,14 @@ gdn_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             ++n1;
         }
         prep_vectors<DK>(KQ, V, PN, gb, L, tid, 1);
-        if (taps && tid < 64) asm volatile("cp.async.wait_group 0;" ::: "memory");   // this item's taps (read later)
+        if (early && k == 0) {                           // the generator's output from here on
+            pdl_wait();
+            load_taps(item, 0);
+        }
         if (!(ok = __syncthreads_and(mbar_wait(&bars[2], (uint32_t)k & 1)))) break;
         tc_fence_after();
         prep_e1(tb + TM_XP, V, AF, out + IM::P, tid);
+        if (taps && tid < 64) asm volatile("cp.async.wait_group 0;" ::: "memory");   // this item's taps (read by T1)
         named_sync(1, PREP_THREADS);
         ut_inverse(AF, XS, tid, 1);
         if (taps)
