@@ -282,17 +282,21 @@ jet_status jet_conv_gdn_decode_step(const void* q, const void* k, const void* v,
  * The whole JetBlock mixer for one new token per sequence (steps 1-3 fused;
  * paper sections 2.3 and 2.4): the kernel generator makes the token's taps,
  * the dynamic causal conv is applied to v with the raw history, the history
- * is shifted, and the gated delta rule updates S in place, all with one read
- * and one write of S. Two launches: jet_kernel_gen, then
- * jet_conv_gdn_decode_step.
+ * is shifted, and the gated delta rule updates S in place with one read and
+ * one write of S. Two launches: the generator + conv (as jet_dyn_conv_v with
+ * T = 1, its output v' written into o), then the update (as
+ * jet_gdn_decode_step, reading v' from o and writing o over it); the update
+ * starts reading its state before the first launch ends.
  *   x [B,D]; w1 [D,hidden], w2 [hidden,H*width] as in jet_kernel_gen;
  *   q, k [B,H,dk]; v [B,H,dv] raw (before the conv); g, beta [B,H] float32;
  *   hist_in [B,3,H,dv] raw history, oldest first, or NULL (zeros);
  *   hist_out [B,3,H,dv] out (must not overlap hist_in);
  *   S [B,H,dv,dk] float32 in/out; o [B,H,dv] out;
  *   taps [B,H,width] float32 out (16-byte aligned): the generated conv taps.
- * Equal, up to floating-point contraction, to jet_dyn_conv_v with T = 1
- * followed by jet_gdn_decode_step on its output.
+ * v, o and hist_out must not overlap (JET_ERR_INVALID_ARG); v, o and the
+ * histories must be 16-byte aligned (JET_ERR_MISALIGNED).
+ * Equal bit for bit to jet_dyn_conv_v with T = 1 followed by
+ * jet_gdn_decode_step on its output.
  */
 jet_status jet_jetblock_decode_step(const void* x, const void* w1, const void* w2,
                                     const void* q, const void* k, const void* v,

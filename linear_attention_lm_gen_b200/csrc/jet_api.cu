@@ -403,6 +403,15 @@ size_t split_img_bytes(int B, int T, int H, int dk) {
 template <int DK, int DV>
 jet_status launch_correct(const __nv_bfloat16* Qe, const __nv_bfloat16* Sb, void* o, int B, int Tn, int H, int nct,
                           int chunk0, int segc, int P, cudaStream_t s, const pfws::SeqMap& sq, int vchunks) {
+    if (vchunks == 0) {   // dense: groups of consecutive chunks of one segment per CTA
+        auto kern = pfcor::prefill_correct_group_kernel<DK, DV>;
+        const size_t smem = pfcor::smem_group_bytes(DK, DV);
+        if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
+        const int gps = (segc + pfcor::CH - 1) / pfcor::CH;
+        const int nseg = (nct + segc - 1) / segc - chunk0 / segc;
+        return launch(kern, dim3(nseg * gps, H, B), dim3(pfcor::GTHREADS), smem, s, Qe, Sb, (__nv_bfloat16*)o, Tn, H,
+                      nct, chunk0, segc, P);
+    }
     auto kern = pfcor::prefill_correct_kernel<DK, DV>;
     const size_t smem = pfcor::smem_bytes(DK, DV);
     if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
@@ -964,17 +973,23 @@ jet_status jet_jetblock_decode_step(const void* x, const void* w1, const void* w
     for (const void* p : {q, k, v, hist_in, (const void*)hist_out, (const void*)o})
         if (p && !aligned_to(p, es)) return JET_ERR_MISALIGNED;
     if (!aligned_to(g, 4) || !aligned_to(beta, 4) || !aligned16(S)) return JET_ERR_MISALIGNED;
-    const size_t nh = (size_t)B * 3 * H * dv * es;
+    const size_t nh = (size_t)B * 3 * H * dv * es, nvb = (size_t)B * H * dv * es;
     if (hist_in && overlap(hist_in, nh, hist_out, nh)) return JET_ERR_INVALID_ARG;
-    // the taps of the new tokens, then conv + history shift + decode update in one pass over S
-    st = jet_kernel_gen(x, w1, w2, taps, B, 1, D, H, hidden, width, dt, stream);
-    if (st != JET_OK) return st;
-    // the generator writes only the taps: the decode launch reads the state before it waits for them
+    if (overlap(v, nvb, o, nvb) || overlap(v, nvb, hist_out, nh) || overlap(o, nvb, hist_out, nh))
+        return JET_ERR_INVALID_ARG;
+    if (!aligned16(v) || !aligned16(o) || !aligned16(hist_out) || (hist_in && !aligned16(hist_in)))
+        return JET_ERR_MISALIGNED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const DecConv conv{taps, hist_in, hist_out};
+    // the generator and the conv of the new tokens, with the history shift: v' goes to o,
+    // which the update then reads (each element before the same thread overwrites it)
+    st = dt == JET_BF16 ? launch_genconv<__nv_bfloat16>(x, w1, w2, v, hist_in, o, hist_out, taps, B, 1, D, H, dv, s)
+                        : launch_genconv<float>(x, w1, w2, v, hist_in, o, hist_out, taps, B, 1, D, H, dv, s);
+    if (st != JET_OK) return st;
+    // that launch writes only v', the history and the taps: the update reads its state rows
+    // and token vectors before it waits for it
     if (dt == JET_BF16)
-        return dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, B, H, dv, s, &conv, nullptr, 0, 1);
-    return dispatch_decode<float>(dk, q, k, v, g, beta, S, o, B, H, dv, s, &conv, nullptr, 0, 1);
+        return dispatch_decode<__nv_bfloat16>(dk, q, k, o, g, beta, S, o, B, H, dv, s, nullptr, nullptr, 0, 1);
+    return dispatch_decode<float>(dk, q, k, o, g, beta, S, o, B, H, dv, s, nullptr, nullptr, 0, 1);
 }
 
 jet_status jet_jetblock_decode_slots(const void* x, const void* w1, const void* w2, const void* q, const void* k,

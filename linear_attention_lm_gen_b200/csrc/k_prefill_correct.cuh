@@ -179,3 +179,132 @@ prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16
 
 }  // namespace pfcor
 }  // namespace jet
+
+namespace jet {
+namespace pfcor {
+
+// Dense layout, CH consecutive chunks of one segment per CTA: S* is loaded
+// once and the chunks' Qe and output tiles are double-buffered, so the next
+// chunk's copies run while this one's product is formed. Segments p0 = chunk0
+// / segc .. P-1; grid (groups of the segments, H, B) with ceil(segc / CH)
+// groups per segment (a group past the sequence end returns at once).
+constexpr int CH = 4;
+constexpr int GTHREADS = 512;            // 16 warps: warp w owns output columns [w dv/16, (w+1) dv/16)
+__host__ __device__ constexpr size_t smem_group_bytes(int dk, int dv) {
+    return 2 * ((size_t)dv * lda(dk) + 2 * (size_t)C * lda(dk) + 2 * (size_t)C * ldo(dv));
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(GTHREADS)
+prefill_correct_group_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16* __restrict__ Sb,
+                             __nv_bfloat16* __restrict__ o, int Tn, int H, int nct, int chunk0, int segc, int P) {
+    static_assert(DK % 16 == 0 && DK <= 128 && DV % 64 == 0 && DV <= 256, "shapes");
+    constexpr int LDA = lda(DK), LDO = ldo(DV);
+    constexpr int NT = DV / 128;                 // n8 tiles per warp (DV / 16 columns)
+    constexpr int KS = DK / 16;
+    static_assert(NT >= 1, "dv >= 128");
+    extern __shared__ __align__(16) uint8_t smem[];
+    __nv_bfloat16* ss = reinterpret_cast<__nv_bfloat16*>(smem);          // [DV][LDA]
+    __nv_bfloat16* qs0 = ss + DV * LDA;                                  // [2][64][LDA]
+    __nv_bfloat16* os0 = qs0 + 2 * C * LDA;                              // [2][64][LDO]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int gps = (segc + CH - 1) / CH;                                // groups per segment
+    const int p = chunk0 / segc + (int)blockIdx.x / gps;
+    const int first = p * segc + ((int)blockIdx.x % gps) * CH;
+    const int last = min(min(first + CH, (p + 1) * segc), nct);          // chunks [first, last)
+    if (first >= last) return;
+    const int n = last - first;
+    pdl_wait();
+    pdl_trigger();
+    const long long tstride = (long long)H * DV;
+    const long long row_b = (long long)b * Tn;
+
+    auto issue_chunk = [&](int j) {      // Qe and output tiles of chunk first + j into buffer j & 1
+        const int gc = first + j, L = min(C, Tn - gc * C);
+        __nv_bfloat16* qs = qs0 + (j & 1) * C * LDA;
+        __nv_bfloat16* os = os0 + (j & 1) * C * LDO;
+        const __nv_bfloat16* src = Qe + (((long long)b * H + h) * nct + gc) * C * DK;
+#pragma unroll
+        for (int i = tid; i < C * DK / 8; i += GTHREADS) {
+            const int r = i / (DK / 8), cc = i % (DK / 8);
+            cp_async16(qs + r * LDA + cc * 8, src + (r < L ? i * 8 : 0), r < L ? 16u : 0u);
+        }
+        const long long row0 = row_b + (long long)gc * C;
+#pragma unroll
+        for (int i = tid; i < C * DV / 8; i += GTHREADS) {
+            const int r = i / (DV / 8), cc = i % (DV / 8);
+            if (r < L) cp_async16(os + r * LDO + cc * 8, o + (row0 + r) * tstride + h * DV + cc * 8, 16u);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    {   // S* of the segment, in the first copy group with chunk 0
+        const __nv_bfloat16* src = Sb + (((long long)b * P + p) * H + h) * DV * DK;
+#pragma unroll
+        for (int i = tid; i < DV * DK / 8; i += GTHREADS) {
+            const int r = i / (DK / 8), cc = i % (DK / 8);
+            cp_async16(ss + r * LDA + cc * 8, src + i * 8, 16u);
+        }
+    }
+    issue_chunk(0);
+    if (n > 1) issue_chunk(1);
+
+    const int n0 = warp * (DV / 16);
+    const int g = lane >> 2, t4 = lane & 3;
+    const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(ss));
+    for (int j = 0; j < n; ++j) {
+        if (j + 1 < n) asm volatile("cp.async.wait_group 1;" ::: "memory");
+        else asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();
+        __nv_bfloat16* qs = qs0 + (j & 1) * C * LDA;
+        __nv_bfloat16* os = os0 + (j & 1) * C * LDO;
+        const uint32_t qbase = static_cast<uint32_t>(__cvta_generic_to_shared(qs));
+        float acc[4][NT][4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int nn = 0; nn < NT; ++nn)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[m][nn][e] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            uint32_t a[4][4], bb[NT][2];
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                ldsm_x4(qbase + (uint32_t)(((16 * m + (lane & 15)) * LDA + ks * 16 + (lane >> 4) * 8) * 2), a[m]);
+#pragma unroll
+            for (int nn = 0; nn < NT; ++nn)
+                ldsm_x2(sbase + (uint32_t)(((n0 + 8 * nn + (lane & 7)) * LDA + ks * 16 + ((lane >> 3) & 1) * 8) * 2),
+                        bb[nn]);
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+#pragma unroll
+                for (int nn = 0; nn < NT; ++nn) mma16816(acc[m][nn], a[m], bb[nn]);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int nn = 0; nn < NT; ++nn)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int r = 16 * m + g + 8 * hr, col = n0 + 8 * nn + 2 * t4;
+                    __nv_bfloat162* op = reinterpret_cast<__nv_bfloat162*>(os + r * LDO + col);
+                    const float2 cur = __bfloat1622float2(*op);
+                    *op = __floats2bfloat162_rn(cur.x + acc[m][nn][2 * hr], cur.y + acc[m][nn][2 * hr + 1]);
+                }
+        __syncthreads();
+        const int gc = first + j, L = min(C, Tn - gc * C);
+        const long long row0 = row_b + (long long)gc * C;
+        for (int i = tid; i < C * DV / 8; i += GTHREADS) {
+            const int r = i / (DV / 8), cc = i % (DV / 8);
+            if (r < L)
+                *reinterpret_cast<uint4*>(o + (row0 + r) * tstride + h * DV + cc * 8) =
+                    *reinterpret_cast<const uint4*>(os + r * LDO + cc * 8);
+        }
+        __syncthreads();                                  // buffer j & 1 read out: free for chunk j + 2
+        if (j + 2 < n) issue_chunk(j + 2);
+    }
+}
+
+}  // namespace pfcor
+}  // namespace jet

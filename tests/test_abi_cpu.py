@@ -172,8 +172,8 @@ def test_python_binding_refuses_cpu_tensors():
                            H=2, conv_w=torch.zeros(1, 4, 2, 4))
 
 
-def fused_decode(lib, x=A, w1=A, w2=A, q=A, k=A, v=A, hin=A + (1 << 16), hout=A + (1 << 18), g=A, b=A, S=A, o=A,
-                 taps=A, B=2, D=64, H=2, dk=16, dv=32, hidden=32, width=4, dt=BF16):
+def fused_decode(lib, x=A, w1=A, w2=A, q=A, k=A, v=A, hin=A + (1 << 16), hout=A + (1 << 18), g=A, b=A, S=A,
+                 o=A + (1 << 24), taps=A, B=2, D=64, H=2, dk=16, dv=32, hidden=32, width=4, dt=BF16):
     return lib.jet_jetblock_decode_step(P(x), P(w1), P(w2), P(q), P(k), P(v), P(hin), P(hout), P(g), P(b), P(S),
                                         P(o), P(taps), B, D, H, dk, dv, hidden, width, dt, None)
 
@@ -183,6 +183,8 @@ def fused_decode(lib, x=A, w1=A, w2=A, q=A, k=A, v=A, hin=A + (1 << 16), hout=A 
     (dict(hout=A + (1 << 16) + 64), INVALID),            # the new history may not overlap the old one
     (dict(dk=24), UNSUPPORTED), (dict(dv=48), UNSUPPORTED), (dict(hidden=16), UNSUPPORTED),
     (dict(S=A + 8), MISALIGNED), (dict(taps=A + 4), MISALIGNED), (dict(x=A + 2), MISALIGNED),
+    (dict(o=A + 64), INVALID), (dict(o=A + (1 << 18)), INVALID),   # o holds v' first: it may not overlap v or hist_out
+    (dict(o=A + (1 << 24) + 2), MISALIGNED),
 ])
 def test_fused_decode_rejects(lib, kw, expect):
     assert fused_decode(lib, **kw) == expect
