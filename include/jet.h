@@ -61,7 +61,8 @@ typedef enum {
     JET_ERR_TIMEOUT = 5,       /* a bounded in-kernel wait ran out (via jet_device_error) */
     JET_ERR_DEVICE = 6,        /* a kernel flagged bad data (via jet_device_error) */
     JET_ERR_WORKSPACE = 7,     /* workspace pointer null or smaller than required */
-    JET_ERR_TOO_LARGE = 8      /* sizes need more scratch than jet_gdn_prefill_noalloc's fixed buffer */
+    JET_ERR_TOO_LARGE = 8,     /* sizes need more scratch than jet_gdn_prefill_noalloc's fixed buffer */
+    JET_ERR_LIBRARY = 9        /* a library the call needs (cuBLAS, for jet_jetblock_layer) could not be loaded */
 } jet_status;
 
 typedef enum { JET_F32 = 0, JET_BF16 = 1 } jet_dtype;
@@ -366,6 +367,40 @@ jet_status jet_gdn_prefill_noalloc(const void* q, const void* k, const void* v, 
                                    const float* beta, const float* S0, void* o, float* S_out,
                                    int B, int T, int H, int dk, int dv, int chunk,
                                    jet_dtype dt, void* stream);
+
+/*
+ * The JetBlock layer around the mixer (Jet-Nemotron paper, section 2.4: the
+ * block takes its queries, keys, values and the generator input from the
+ * shared input x; the dynamic conv acts on V alone). The paper gives no form
+ * for the gates or the output; this is the Gated DeltaNet layer without its
+ * short convolutions:
+ *   q = x Wq, k = x Wk, v = x Wv, z = x Wz                 (bf16 GEMMs, float32 accumulate)
+ *   g = -softplus(x Wg), beta = sigmoid(x Wb)             (float32)
+ *   o = the mixer (jet_jetblock_prefill; for T = 1 the decode kernels, the
+ *       state advanced in place in S_out)
+ *   y = (o / sqrt(mean_dv(o^2) + 1e-6) * gamma * SiLU(z)) Wo   (per token and head)
+ * The six projections and the output projection run on cuBLAS (loaded on the
+ * first call; JET_ERR_LIBRARY if it cannot be), the rest in this library.
+ *   x [B,T,D] bf16; wq, wk [D,H*dk]; wv, wz [D,H*dv]; wg, wb [D,H];
+ *   wo [H*dv,D] (all bf16, row-major); gamma [dv] float32;
+ *   w1, w2 the generator's weights as in jet_kernel_gen;
+ *   hist_in [B,3,H,dv] or NULL (zeros); hist_out [B,3,H,dv] or NULL (required
+ *   for T = 1); S0 [B,H,dv,dk] float32 or NULL (zeros); S_out [B,H,dv,dk]
+ *   float32 out (may alias S0); y [B,T,D] bf16 out;
+ *   workspace of jet_jetblock_layer_workspace_size bytes (16-byte aligned),
+ *   else JET_ERR_WORKSPACE before any launch.
+ * bf16 and the tensor-core shapes only (dk in {64, 96, 128}, dv a multiple
+ * of 128), D a multiple of 16; else JET_ERR_UNSUPPORTED. cuBLAS is called
+ * under a process-wide lock, so concurrent calls from several threads are
+ * serialised at their GEMMs.
+ */
+size_t jet_jetblock_layer_workspace_size(int B, int T, int D, int H, int dk, int dv);
+jet_status jet_jetblock_layer(const void* x, const void* wq, const void* wk, const void* wv,
+                              const void* wg, const void* wb, const void* wz, const void* wo,
+                              const float* gamma, const void* w1, const void* w2,
+                              const void* hist_in, void* hist_out, const float* S0, float* S_out,
+                              void* y, void* workspace, size_t ws_bytes, int B, int T, int D, int H,
+                              int dk, int dv, int hidden, int width, jet_dtype dt, void* stream);
 
 /*
  * Synchronises `stream`, then returns and clears the current device's error

@@ -27,14 +27,14 @@ LIB_PATH = os.path.join(PKG, "libjet.so")
 JET_F32, JET_BF16 = 0, 1
 STATUS = {0: "JET_OK", 1: "JET_ERR_INVALID_ARG", 2: "JET_ERR_UNSUPPORTED", 3: "JET_ERR_MISALIGNED",
           4: "JET_ERR_CUDA", 5: "JET_ERR_TIMEOUT", 6: "JET_ERR_DEVICE", 7: "JET_ERR_WORKSPACE",
-          8: "JET_ERR_TOO_LARGE"}
+          8: "JET_ERR_TOO_LARGE", 9: "JET_ERR_LIBRARY"}
 EXPORTS = ("jet_kernel_gen", "jet_dyn_conv_v", "jet_gdn_prefill_workspace_size", "jet_gdn_prefill_workspace_min",
            "jet_gdn_prefill",
            "jet_gdn_prefill_noalloc", "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step",
            "jet_jetblock_prefill_workspace_size", "jet_jetblock_prefill", "jet_jetblock_decode_slots",
            "jet_jetblock_prefill_varlen_workspace_size", "jet_jetblock_prefill_varlen",
            "jet_jetblock_prefill_range_workspace_size", "jet_jetblock_prefill_range", "jet_gdn_range_compose",
-           "jet_gdn_range_correct", "jet_device_error",
+           "jet_gdn_range_correct", "jet_jetblock_layer_workspace_size", "jet_jetblock_layer", "jet_device_error",
            "jet_status_string", "jet_launch_count")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -85,6 +85,9 @@ def declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.jet_jetblock_prefill_range.argtypes = [P] * 16 + [Z] + [I] * 10 + [P]
     L.jet_gdn_range_compose.argtypes = [P] * 4 + [I] * 5 + [P]
     L.jet_gdn_range_correct.argtypes = [P] * 3 + [I] * 6 + [P]
+    L.jet_jetblock_layer_workspace_size.argtypes = [I] * 6
+    L.jet_jetblock_layer_workspace_size.restype = Z
+    L.jet_jetblock_layer.argtypes = [P] * 17 + [Z] + [I] * 9 + [P]
     L.jet_device_error.argtypes = [P]
     L.jet_status_string.argtypes = [I]
     L.jet_status_string.restype = ctypes.c_char_p
@@ -94,7 +97,7 @@ def declare(L: ctypes.CDLL) -> ctypes.CDLL:
               "jet_gdn_decode_step", "jet_jetblock_decode_step", "jet_conv_gdn_decode_step", "jet_jetblock_prefill",
               "jet_jetblock_decode_slots", "jet_jetblock_prefill_varlen", "jet_jetblock_prefill_range",
               "jet_gdn_range_compose",
-              "jet_gdn_range_correct", "jet_device_error"):
+              "jet_gdn_range_correct", "jet_jetblock_layer", "jet_device_error"):
         getattr(L, f).restype = I
     return L
 
@@ -497,3 +500,42 @@ def jet_status_string(status: int) -> str:
 
 def jet_launch_count() -> int:
     return int(load_library().jet_launch_count())
+
+
+def jet_jetblock_layer_workspace_size(B: int, T: int, D: int, H: int, dk: int, dv: int) -> int:
+    """Workspace bytes of jet_jetblock_layer (0: not a supported shape)."""
+    return int(load_library().jet_jetblock_layer_workspace_size(B, T, D, H, dk, dv))
+
+
+def jet_jetblock_layer(x, Wq, Wk, Wv, Wg, Wb, Wz, Wo, gamma, W1, W2, hist_in=None, hist_out=None, S0=None, S_out=None,
+                       y=None, workspace=None, *, stream=None):
+    """The JetBlock layer: x [B,T,D] bf16 -> y [B,T,D] (projections, mixer,
+    per-head RMSNorm with gamma [dv] and SiLU output gate, output projection).
+    Wq, Wk [D,H*dk]; Wv, Wz [D,H*dv]; Wg, Wb [D,H]; Wo [H*dv,D]; W1, W2 the
+    generator's. S0 / S_out [B,H,dv,dk] float32 (may be the same tensor: with
+    T = 1 the state advances in place); hist_in / hist_out [B,3,H,dv].
+    Returns (y, S_out)."""
+    L = load_library()
+    B, T, D = x.shape
+    H = Wg.shape[1]
+    dk = Wq.shape[1] // H
+    dv = Wv.shape[1] // H
+    bf = torch.bfloat16
+    if y is None:
+        y = torch.empty((B, T, D), device=x.device, dtype=bf)
+    if S_out is None:
+        S_out = torch.empty((B, H, dv, dk), device=x.device, dtype=torch.float32)
+    if workspace is None:
+        workspace = torch.empty(max(16, jet_jetblock_layer_workspace_size(B, T, D, H, dk, dv)), device=x.device,
+                                dtype=torch.uint8)
+    st = L.jet_jetblock_layer(
+        _ptr(x, "x", bf), _ptr(Wq, "Wq", bf, (D, H * dk)), _ptr(Wk, "Wk", bf, (D, H * dk)),
+        _ptr(Wv, "Wv", bf, (D, H * dv)), _ptr(Wg, "Wg", bf, (D, H)), _ptr(Wb, "Wb", bf, (D, H)),
+        _ptr(Wz, "Wz", bf, (D, H * dv)), _ptr(Wo, "Wo", bf, (H * dv, D)), _ptr(gamma, "gamma", torch.float32, (dv,)),
+        _ptr(W1, "W1", bf), _ptr(W2, "W2", bf), _ptr(hist_in, "hist_in", bf, (B, 3, H, dv)),
+        _ptr(hist_out, "hist_out", bf, (B, 3, H, dv)), _ptr(S0, "S0", torch.float32, (B, H, dv, dk)),
+        _ptr(S_out, "S_out", torch.float32, (B, H, dv, dk)), _ptr(y, "y", bf, (B, T, D)), _ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), B, T, D, H, dk, dv, W1.shape[1], W2.shape[1] // H, JET_BF16,
+        _stream(stream))
+    _check("jet_jetblock_layer", st)
+    return y, S_out

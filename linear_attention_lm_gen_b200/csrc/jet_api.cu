@@ -3,12 +3,15 @@
 #include "jet.h"
 
 #include <cuda.h>
+#include <cublas_v2.h>
+#include <dlfcn.h>
 
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <tuple>
 #include <type_traits>
 
 #include "common.cuh"
@@ -16,6 +19,7 @@
 #include "k_gen.cuh"
 #include "k_genconv.cuh"
 #include "k_genconv_decode.cuh"
+#include "k_layer.cuh"
 #include "k_prefill_simt.cuh"
 #include "k_prefill_chain.cuh"
 #include "k_prefill_correct.cuh"
@@ -1047,6 +1051,7 @@ const char* jet_status_string(jet_status s) {
         case JET_ERR_DEVICE: return "JET_ERR_DEVICE";
         case JET_ERR_WORKSPACE: return "JET_ERR_WORKSPACE";
         case JET_ERR_TOO_LARGE: return "JET_ERR_TOO_LARGE";
+        case JET_ERR_LIBRARY: return "JET_ERR_LIBRARY";
     }
     return "JET_ERR_UNKNOWN";
 }
@@ -1128,6 +1133,163 @@ extern "C" jet_status jet_gdn_prefill_noalloc(const void* q, const void* k, cons
         if (st != JET_OK) return st;
     }
     return jet_gdn_prefill(q, k, v, g, beta, S0, o, S_out, ws, use, B, T, H, dk, dv, chunk, dt, stream);
+}
+
+
+// ---- the JetBlock layer around the mixer (projections, gates, output gate and norm)
+namespace {
+// cuBLAS for the layer's plain GEMMs, loaded on first use (libjet.so itself
+// does not depend on it); one handle per device
+struct Blas {
+    bool tried = false, ok = false;
+    cublasStatus_t (*create)(cublasHandle_t*) = nullptr;
+    cublasStatus_t (*set_stream)(cublasHandle_t, cudaStream_t) = nullptr;
+    cublasStatus_t (*gemm_ex)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int, const void*,
+                              const void*, cudaDataType_t, int, const void*, cudaDataType_t, int, const void*, void*,
+                              cudaDataType_t, int, cublasComputeType_t, cublasGemmAlgo_t) = nullptr;
+    cublasHandle_t handle[64] = {};
+};
+std::mutex g_blas_mu;
+Blas g_blas;
+
+// under g_blas_mu: the loaded library and this device's handle bound to stream s
+cublasHandle_t blas_handle(cudaStream_t s) {
+    Blas& b = g_blas;
+    if (!b.tried) {
+        b.tried = true;
+        void* lib = dlopen("libcublas.so.12", RTLD_NOW | RTLD_GLOBAL);
+        if (!lib) lib = dlopen("libcublas.so", RTLD_NOW | RTLD_GLOBAL);
+        if (lib) {
+            b.create = reinterpret_cast<decltype(b.create)>(dlsym(lib, "cublasCreate_v2"));
+            b.set_stream = reinterpret_cast<decltype(b.set_stream)>(dlsym(lib, "cublasSetStream_v2"));
+            b.gemm_ex = reinterpret_cast<decltype(b.gemm_ex)>(dlsym(lib, "cublasGemmEx"));
+            b.ok = b.create && b.set_stream && b.gemm_ex;
+        }
+    }
+    if (!b.ok) return nullptr;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!b.handle[dev] && b.create(&b.handle[dev]) != CUBLAS_STATUS_SUCCESS) return nullptr;
+    if (b.set_stream(b.handle[dev], s) != CUBLAS_STATUS_SUCCESS) return nullptr;
+    return b.handle[dev];
+}
+
+// row-major C[M][N] = A[M][K] B[K][N] (bf16 A and B, float32 accumulate; C bf16 or float32)
+jet_status gemm_rm(cublasHandle_t h, const void* A, const void* Bm, void* C, int M, int N, int K, bool c_f32) {
+    const float one = 1.f, zero = 0.f;
+    // column-major view: C^T[N][M] = B^T[N][K] A^T[K][M]
+    const cublasStatus_t st = g_blas.gemm_ex(h, CUBLAS_OP_N, CUBLAS_OP_N, N, M, K, &one, Bm, CUDA_R_16BF, N, A,
+                                             CUDA_R_16BF, K, &zero, C, c_f32 ? CUDA_R_32F : CUDA_R_16BF, N,
+                                             CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+    return st == CUBLAS_STATUS_SUCCESS ? JET_OK : JET_ERR_CUDA;
+}
+
+struct LayerWs {       // byte offsets in the layer's workspace
+    size_t q, k, v, z, g, b, o, mix, bytes;
+};
+LayerWs layer_ws(int B, int T, int H, int dk, int dv) {
+    auto up = [](size_t x) { return (x + 1023) & ~size_t(1023); };
+    const size_t N = (size_t)B * T;
+    LayerWs w;
+    size_t off = 0;
+    w.q = off; off += up(N * H * dk * 2);
+    w.k = off; off += up(N * H * dk * 2);
+    w.v = off; off += up(N * H * dv * 2);
+    w.z = off; off += up(N * H * dv * 2);
+    w.g = off; off += up(N * H * 4);
+    w.b = off; off += up(N * H * 4);
+    w.o = off; off += up(N * H * dv * 2);
+    w.mix = off;
+    const size_t mix = T == 1 ? up((size_t)B * H * 4 * sizeof(float))
+                              : jet_jetblock_prefill_workspace_size(B, T, H, dk, dv, 64, JET_BF16);
+    w.bytes = off + mix;
+    return w;
+}
+}  // namespace
+
+size_t jet_jetblock_layer_workspace_size(int B, int T, int D, int H, int dk, int dv) {
+    if (B <= 0 || T <= 0 || D <= 0 || H <= 0 || D % 16 != 0 || !tc_prefill_ok(JET_BF16, dk, dv, (long long)B * T))
+        return 0;
+    if (elems({B, T, H, dv}) < 0 || elems({B, T, D}) < 0) return 0;
+    return layer_ws(B, T, H, dk, dv).bytes;
+}
+
+jet_status jet_jetblock_layer(const void* x, const void* wq, const void* wk, const void* wv, const void* wg,
+                              const void* wb, const void* wz, const void* wo, const float* gamma, const void* w1,
+                              const void* w2, const void* hist_in, void* hist_out, const float* S0, float* S_out,
+                              void* y, void* workspace, size_t ws_bytes, int B, int T, int D, int H, int dk, int dv,
+                              int hidden, int width, jet_dtype dt, void* stream) {
+    jet_status st = check_gen(x, w1, w2, B, T, D, H, hidden, width, dt);
+    if (st != JET_OK) return st;
+    if (!wq || !wk || !wv || !wg || !wb || !wz || !wo || !gamma || !S_out || !y) return JET_ERR_INVALID_ARG;
+    if (elems({B, T, H, dv}) < 0 || elems({B, T, H, dk}) < 0 || elems({D, H, dv}) < 0 ||
+        elems({B, H, dv, dk}) < 0)
+        return JET_ERR_INVALID_ARG;
+    if (dt != JET_BF16 || !tc_prefill_ok(dt, dk, dv, (long long)B * T) || B > 65535 || H > 65535)
+        return JET_ERR_UNSUPPORTED;
+    for (const void* p : {wq, wk, wv, wg, wb, wz, wo, hist_in, (const void*)hist_out, (const void*)y})
+        if (p && !aligned_to(p, 2)) return JET_ERR_MISALIGNED;
+    for (const void* p : {hist_in, (const void*)hist_out, (const void*)S0, (const void*)S_out, (const void*)gamma,
+                          (const void*)workspace})
+        if (p && !aligned16(p)) return JET_ERR_MISALIGNED;
+    if (T == 1 && !hist_out) return JET_ERR_INVALID_ARG;      // a decode step shifts the history
+    if (!workspace) ws_bytes = 0;
+    const LayerWs L = layer_ws(B, T, H, dk, dv);
+    if (ws_bytes < L.bytes) return JET_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    auto* q = w + L.q;
+    auto* k = w + L.k;
+    auto* v = w + L.v;
+    auto* z = w + L.z;
+    float* g = reinterpret_cast<float*>(w + L.g);
+    float* b = reinterpret_cast<float*>(w + L.b);
+    auto* o = w + L.o;
+    const int N = B * T;
+    {   // the projections (plain GEMMs on cuBLAS)
+        std::lock_guard<std::mutex> lk(g_blas_mu);
+        cublasHandle_t h = blas_handle(s);
+        if (!h) return g_blas.ok ? JET_ERR_CUDA : JET_ERR_LIBRARY;
+        for (auto [wm, out, cols, f32] : {std::tuple<const void*, void*, int, bool>{wq, q, H * dk, false},
+                                          {wk, k, H * dk, false}, {wv, v, H * dv, false}, {wz, z, H * dv, false},
+                                          {wg, g, H, true}, {wb, b, H, true}}) {
+            st = gemm_rm(h, x, wm, out, N, cols, D, f32);
+            if (st != JET_OK) return st;
+        }
+    }
+    const long long nh = (long long)N * H;
+    st = launch(layer::gates_kernel, dim3((unsigned)std::min<long long>((nh + 255) / 256, 4096)),
+                dim3(layer::GATE_THREADS), 0, s, g, b, nh);
+    if (st != JET_OK) return st;
+    // the mixer
+    if (T == 1) {     // one new token per sequence: S advanced in place in S_out
+        if (S0 != S_out) {
+            const cudaError_t e = S0 ? cudaMemcpyAsync(S_out, S0, sizeof(float) * (size_t)B * H * dv * dk,
+                                                       cudaMemcpyDeviceToDevice, s)
+                                     : cudaMemsetAsync(S_out, 0, sizeof(float) * (size_t)B * H * dv * dk, s);
+            if (e != cudaSuccess) return JET_ERR_CUDA;
+        }
+        float* taps = reinterpret_cast<float*>(w + L.mix);
+        st = launch_genconv<__nv_bfloat16>(x, w1, w2, v, hist_in, o, hist_out, taps, B, 1, D, H, dv, s);
+        if (st != JET_OK) return st;
+        st = dispatch_decode<__nv_bfloat16>(dk, q, k, o, g, b, S_out, o, B, H, dv, s, nullptr, nullptr, 0, 1);
+    } else {
+        st = jet_jetblock_prefill(x, w1, w2, q, k, v, hist_in, hist_out, g, b, S0, o, S_out, w + L.mix,
+                                  ws_bytes - L.mix, B, T, D, H, dk, dv, hidden, width, 64, dt, stream);
+    }
+    if (st != JET_OK) return st;
+    // per-head RMSNorm, gamma and the SiLU output gate (in place over o), then the output projection
+    const long long rows = (long long)N * H;
+    const unsigned grid = (unsigned)((rows + layer::OUT_THREADS / 32 - 1) / (layer::OUT_THREADS / 32));
+    st = dv <= 256 ? launch(layer::out_gate_kernel<1>, dim3(grid), dim3(layer::OUT_THREADS), 0, s,
+                            (const __nv_bfloat16*)o, (const __nv_bfloat16*)z, gamma, (__nv_bfloat16*)o, rows, dv)
+                   : launch(layer::out_gate_kernel<2>, dim3(grid), dim3(layer::OUT_THREADS), 0, s,
+                            (const __nv_bfloat16*)o, (const __nv_bfloat16*)z, gamma, (__nv_bfloat16*)o, rows, dv);
+    if (st != JET_OK) return st;
+    std::lock_guard<std::mutex> lk(g_blas_mu);
+    cublasHandle_t h = blas_handle(s);
+    if (!h) return JET_ERR_CUDA;
+    return gemm_rm(h, o, wo, y, N, D, H * dv, false);
 }
 
 #ifdef JET_TEST_WAIT_EXPIRY

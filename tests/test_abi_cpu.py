@@ -391,3 +391,37 @@ def test_prefill_varlen_workspace(lib):
     assert jet.jet_jetblock_prefill_varlen_workspace_size(cu, H, 48, dv) == 0      # not a tensor-core shape
     assert jet.jet_jetblock_prefill_varlen_workspace_size([0, 10, 5], H, dk, dv) == 0
     assert jet.jet_jetblock_prefill_varlen_workspace_size(list(range(0, 2580, 10)), H, dk, dv) == 0
+
+
+def layer(lib, x=A, wq=A, wk=A, wv=A, wg=A, wb=A, wz=A, wo=A, gamma=A, w1=A, w2=A, hin=None, hout=A + (1 << 24),
+          S0=None, S=A + (1 << 26), y=A + (1 << 27), ws=A + (1 << 28), ws_bytes=1 << 40, B=1, T=64, D=64, H=2, dk=64,
+          dv=128, hidden=32, width=4, dt=BF16):
+    return lib.jet_jetblock_layer(P(x), P(wq), P(wk), P(wv), P(wg), P(wb), P(wz), P(wo), P(gamma), P(w1), P(w2),
+                                  P(hin), P(hout), P(S0), P(S), P(y), P(ws), ws_bytes, B, T, D, H, dk, dv, hidden,
+                                  width, dt, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(x=None), INVALID), (dict(wz=None), INVALID), (dict(gamma=None), INVALID), (dict(y=None), INVALID),
+    (dict(T=1, hout=None), INVALID),                                 # a decode step shifts the history
+    (dict(dk=48), UNSUPPORTED), (dict(dv=96), UNSUPPORTED), (dict(dt=F32), UNSUPPORTED),
+    (dict(D=72), UNSUPPORTED), (dict(hidden=16), UNSUPPORTED),
+    (dict(gamma=A + 4), MISALIGNED), (dict(S=A + (1 << 26) + 8), MISALIGNED), (dict(wo=A + 1), MISALIGNED),
+    (dict(ws_bytes=1024), WORKSPACE), (dict(ws=None), WORKSPACE),
+])
+def test_layer_rejects(lib, kw, expect):
+    assert layer(lib, **kw) == expect
+
+
+def test_layer_workspace_is_the_projections_plus_the_mixer(lib):
+    B, T, D, H, dk, dv = 1, 4096, 1536, 12, 96, 256
+    up = lambda b: -(-b // 1024) * 1024
+    N = B * T
+    own = 2 * up(N * H * dk * 2) + 3 * up(N * H * dv * 2) + 2 * up(N * H * 4)
+    assert jet.jet_jetblock_layer_workspace_size(B, T, D, H, dk, dv) == \
+        own + jet.jet_jetblock_prefill_workspace_size(B, T, H, dk, dv)
+    # one new token per sequence: the decode kernels (taps only) instead of the prefill's workspace
+    assert jet.jet_jetblock_layer_workspace_size(256, 1, D, H, dk, dv) == \
+        2 * up(256 * H * dk * 2) + 3 * up(256 * H * dv * 2) + 2 * up(256 * H * 4) + up(256 * H * 16)
+    assert jet.jet_jetblock_layer_workspace_size(B, T, D, H, 48, dv) == 0
+    assert jet.jet_jetblock_layer_workspace_size(B, T, 72, H, dk, dv) == 0

@@ -108,27 +108,27 @@ def test_decode_steps_continue_the_prefill():
 
 
 # ---- planted mistakes: each must fail at least one pin above
-def _mut_norm_over_heads(o, z, gamma, Wo, eps=L.RMS_EPS):
+def _mut_norm_over_heads(o, z, gamma, Wo, eps=L.RMS_EPS, interface=None):
     r = o / np.sqrt(np.mean(o * o, axis=-2, keepdims=True) + eps) * gamma
     return (r * L.silu(z)).reshape(o.shape[:-2] + (-1,)) @ Wo
 
 
-def _mut_gamma_before_norm(o, z, gamma, Wo, eps=L.RMS_EPS):
+def _mut_gamma_before_norm(o, z, gamma, Wo, eps=L.RMS_EPS, interface=None):
     og = o * gamma
     r = og / np.sqrt(np.mean(og * og, axis=-1, keepdims=True) + eps)
     return (r * L.silu(z)).reshape(o.shape[:-2] + (-1,)) @ Wo
 
 
-def _mut_no_silu(o, z, gamma, Wo, eps=L.RMS_EPS):
+def _mut_no_silu(o, z, gamma, Wo, eps=L.RMS_EPS, interface=None):
     r = o / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps) * gamma
     return (r * z).reshape(o.shape[:-2] + (-1,)) @ Wo
 
 
-def _mut_no_norm(o, z, gamma, Wo, eps=L.RMS_EPS):
+def _mut_no_norm(o, z, gamma, Wo, eps=L.RMS_EPS, interface=None):
     return (o * gamma * L.silu(z)).reshape(o.shape[:-2] + (-1,)) @ Wo
 
 
-def _mut_eps_outside(o, z, gamma, Wo, eps=L.RMS_EPS):
+def _mut_eps_outside(o, z, gamma, Wo, eps=L.RMS_EPS, interface=None):
     r = o / np.sqrt(np.mean(o * o, axis=-1, keepdims=True)) * gamma
     return (r * L.silu(z)).reshape(o.shape[:-2] + (-1,)) @ Wo
 
@@ -152,8 +152,8 @@ def test_a_planted_output_mistake_fails_a_pin(monkeypatch, mutant):
 def test_a_planted_projection_mistake_fails_a_pin(monkeypatch, which):
     good = L.projections
 
-    def bad(x, Wq, Wk, Wv, Wg, Wb, Wz, H):
-        q, k, v, z, g, b = good(x, Wq, Wk, Wv, Wg, Wb, Wz, H)
+    def bad(x, Wq, Wk, Wv, Wg, Wb, Wz, H, interface=None):
+        q, k, v, z, g, b = good(x, Wq, Wk, Wv, Wg, Wb, Wz, H, interface)
         if which == "g_sign":
             g = -g
         elif which == "b_as_softplus":
@@ -164,3 +164,13 @@ def test_a_planted_projection_mistake_fails_a_pin(monkeypatch, which):
     monkeypatch.setattr(L, "projections", bad)
     with pytest.raises(AssertionError):
         test_closed_forms_of_the_gates_and_projections()
+
+
+def test_bf16_rounding_of_the_interfaces():
+    # round to nearest even at bf16 (8 significand bits): exact values stay, halfway cases go to even
+    # spacing 512 at 2^16: 65536 + 256 is halfway to an odd neighbour (stays), + 768 halfway to an even one
+    np.testing.assert_array_equal(L.bf16(np.array([1.0, -2.5, 0.0, 65536 + 256, 65536 + 768])),
+                                  [1.0, -2.5, 0.0, 65536, 65536 + 1024])
+    np.testing.assert_array_equal(L.bf16(np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, 1 + 2 ** -7])),
+                                  [1.0, 1 + 2 ** -6, 1 + 2 ** -7])
+    np.testing.assert_array_equal(L.bf16(np.array([1 + 2 ** -8 + 2 ** -20])), [1 + 2 ** -7])
