@@ -685,6 +685,122 @@ def measure_varlen_config(ctx, steps: int, warmup: int):
                     "d2h_bytes_per_step": o.numel() * 2, "ms_per_step": e_ms}}, inp, s.with_(B=1, T=total)
 
 
+def layer_weights(s, seed: int):
+    """Seeded bf16 layer weights ~ N(0, 1/fan_in) on 2B/4B shapes, gamma = 1 + 0.1 N(0, 1)."""
+    rng = np.random.Generator(np.random.PCG64([seed, 11]))
+    bf = lambda *shape: synth.jetblock._draw(rng, shape, "bf16", scale=1.0 / np.sqrt(shape[0]))
+    D, H, dk, dv = s.D, s.H, s.dk, s.dv
+    w = dict(Wq=bf(D, H * dk), Wk=bf(D, H * dk), Wv=bf(D, H * dv), Wg=bf(D, H), Wb=bf(D, H), Wz=bf(D, H * dv),
+             Wo=bf(H * dv, D), W1=bf(D, 32), W2=bf(32, H * 4))
+    w["gamma"] = (1.0 + 0.1 * rng.standard_normal(dv)).astype(np.float32)
+    return w
+
+
+LAYER_ORDER = ("Wq", "Wk", "Wv", "Wg", "Wb", "Wz", "Wo", "gamma", "W1", "W2")
+
+
+def layer_model(s, B: int, T: int):
+    """Algorithmic flops and bytes of the layer over B x T tokens: the seven GEMMs and the mixer's
+    flops; bytes of the fused minimum (x in, y out, every weight once, final state and history out)."""
+    N = B * T
+    D, H, dk, dv = s.D, s.H, s.dk, s.dv
+    proj = 2 * H * dk + 2 * H * dv + 2 * H
+    flops = 2 * N * D * proj + 2 * N * H * dv * D
+    if T > 1:
+        flops += prefill_model(s, B=B, T=T)["flops"]
+    else:
+        flops += decode_model(s, B=B)["flops"]
+    weights = 2 * (D * proj + H * dv * D + D * 32 + 32 * H * 4) + 4 * dv
+    state = B * H * dv * dk * 4 * (1 if T > 1 else 2) + B * 3 * H * dv * 2 * 2
+    return dict(flops=flops, bytes=2 * N * D * 2 + weights + state)
+
+
+def measure_layer_config(ctx, name: str, T: int, steps: int, warmup: int):
+    """The JetBlock layer (jet_jetblock_layer): prefill of T tokens, or (T = 1) one decode step of B
+    sequences with the state advanced in place."""
+    torch, jet, dev, stream, rk, pk = ctx["torch"], ctx["jet"], ctx["dev"], ctx["stream"], ctx["rk"], ctx["pk"]
+    s = synth.CONFIGS[name]
+    B = s.B
+    w = layer_weights(s, ctx["seed"])
+    g = {k: as_torch(v).to(dev) for k, v in w.items()}
+    x_np = synth.jetblock._draw(np.random.Generator(np.random.PCG64([ctx["seed"], 12])), (B, T, s.D), "bf16")
+    xh = as_torch(x_np).pin_memory()
+    x = xh.to(dev)
+    S = torch.zeros((B, s.H, s.dv, s.dk), device=dev, dtype=torch.float32)
+    hist = [torch.zeros((B, 3, s.H, s.dv), device=dev, dtype=torch.bfloat16) for _ in range(2)]
+    y = torch.empty((B, T, s.D), device=dev, dtype=torch.bfloat16)
+    ws = torch.empty(max(16, jet.jet_jetblock_layer_workspace_size(B, T, s.D, s.H, s.dk, s.dv)), device=dev,
+                     dtype=torch.uint8)
+    decode = T == 1
+
+    def call(i):
+        if decode:      # one more token per sequence: the state advances in place
+            jet.jet_jetblock_layer(x, *[g[k] for k in LAYER_ORDER], hist_in=hist[i % 2], hist_out=hist[(i + 1) % 2],
+                                   S0=S, S_out=S, y=y, workspace=ws, stream=stream)
+        else:           # the same prompt from a zero state every step
+            jet.jet_jetblock_layer(x, *[g[k] for k in LAYER_ORDER], hist_out=hist[0], S_out=S, y=y, workspace=ws,
+                                   stream=stream)
+    m = layer_model(s, B, T)
+    flush = not decode              # the prefill's inputs and weights fit in L2; the decode state does not
+    ctx["barrier"]()
+    t = rk.max_over_ranks(statistics.median(Timer(torch, dev, stream, flush=flush).run(call, steps, warmup)), dev)
+    hy = torch.empty(y.shape, dtype=torch.bfloat16).pin_memory()
+
+    def e2e(i):
+        x.copy_(xh, non_blocking=True)
+        call(i)
+        hy.copy_(y, non_blocking=True)
+    e_ms = rk.max_over_ranks(statistics.median(Timer(torch, dev, stream, flush).run(e2e, max(3, steps // 2), 2)), dev)
+    tok = B * T
+    r_us = roofline_us(m["bytes"], m["flops"], pk)
+    bound = "hbm" if m["bytes"] / pk["hbm_gbs"] > m["flops"] / (pk["bf16_tflops"] * 1e3) else "tensor"
+    what = (f"one decode token for each of {B} sequences" if decode else f"a {T}-token prompt") + \
+        f" through jet_jetblock_layer on {name[:2].upper()} shapes (H={s.H}, dk={s.dk}, dv={s.dv}, d_model={s.D}): " \
+        f"projections (cuBLAS), gates, the mixer, per-head RMSNorm and SiLU gate, output projection"
+    out = {"workload": what, "tokens_per_s": rk.world * tok / (t * 1e-3), "us_per_call": t * 1e3, "steps": steps,
+           "warmup": warmup, "l2": "flushed between steps" if flush else "state larger than L2 (no flush needed)",
+           "roofline": {"bound": bound, "algorithmic_bytes": m["bytes"], "algorithmic_flops": m["flops"],
+                        "achieved": (m["flops"] / (t * 1e-3) / 1e12) if bound == "tensor"
+                        else m["bytes"] / (t * 1e-3) / 1e9,
+                        "peak": pk["bf16_tflops"] if bound == "tensor" else pk["hbm_gbs"],
+                        "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "roofline_us": r_us,
+                        "frac": r_us / (t * 1e3)},
+           "e2e": {"value": rk.world * tok / (e_ms * 1e-3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": xh.numel() * 2, "d2h_bytes_per_step": y.numel() * 2, "ms_per_step": e_ms}}
+    del g, S, ws
+    return out, w, x_np
+
+
+def cpu_layer_sample(s, w, x, budget_s: float, decode: bool):
+    """The oracle's layer on the first tokens (prefill: pieces of 256 continuing the state) or on the
+    first sequences (decode) of the workload, until the budget is spent."""
+    import oracle
+    from oracle import layer as olayer
+    orc = oracle.get()
+    f = {k: (synth.to_f64(v, "bf16") if v.dtype == np.uint16 else v.astype(np.float64)) for k, v in w.items()}
+    args = [f[k] for k in LAYER_ORDER]
+    xf = synth.to_f64(x, "bf16")
+    done, t0 = 0, time.perf_counter()
+    if decode:
+        H, dv, dk = s.H, s.dv, s.dk
+        while done < xf.shape[0] and time.perf_counter() - t0 < budget_s:
+            xs = xf[done:done + 4, 0][None]                    # [1 step, 4 sequences, D]
+            n = xs.shape[1]
+            olayer.layer_decode(orc, xs, *args, np.zeros((n, H, dv, dk)), np.zeros((n, 3, H, dv)))
+            done += n
+        what = f"one decode step of the first {done} sequences"
+    else:
+        S, hist = None, None
+        while done < xf.shape[1] and time.perf_counter() - t0 < budget_s:
+            r = olayer.layer_prefill(orc, xf[:1, done:done + 256], *args, S, hist)
+            S, hist = r["S"], r["hist"]
+            done += min(256, xf.shape[1] - done)
+        what = f"the first {done} tokens of the prompt in 256-token pieces"
+    el = time.perf_counter() - t0
+    return {"value": done / el, "unit": "tokens/s", "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"{what} on the float64 oracle of the layer, {el:.1f} s"}
+
+
 def run_configs(ctx, args):
     out = {}
     if ctx["rk"].world > 1:
@@ -692,6 +808,12 @@ def run_configs(ctx, args):
         ctx["torch"].cuda.empty_cache()
     cpu = not args.no_cpu_baseline and ctx["rk"].rank == 0
     budget = args.cpu_budget_config
+    for lname, T in (("prefill_2b_t4096", 4096), ("decode_2b_b256", 1)):
+        r, w, x = measure_layer_config(ctx, lname, T, steps=10 if T > 1 else 20, warmup=3)
+        if cpu:
+            r["cpu_baseline"] = cpu_layer_sample(synth.CONFIGS[lname], w, x, budget / 2, decode=T == 1)
+        out["jetblock_layer_" + ("2b_t4096" if T > 1 else "2b_decode_b256")] = r
+        ctx["torch"].cuda.empty_cache()
     r, inp, sp = measure_varlen_config(ctx, steps=10, warmup=3)
     if cpu:     # the oracle's cost per token does not depend on where the prompts are cut
         r["cpu_baseline"] = cpu_prefill_sample(sp, inp, budget / 2)
