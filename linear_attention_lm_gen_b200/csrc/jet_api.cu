@@ -207,11 +207,20 @@ jet_status launch_genconv(const void* x, const void* w1, const void* w2, const v
                                       n_slots);
 }
 
-// the generator alone over a prompt (bf16): one CTA per 32 tokens
+// prompts of at least this many tokens give every SM two 128-token generator CTAs
+constexpr long long kGenWideTokens = 32768;
+// the generator alone over a prompt (bf16): one CTA per 32 (or 128) tokens
 jet_status launch_gen(const void* x, const void* w1, const void* w2, float* taps, int B, int Tn, int D, int H,
                       cudaStream_t s) {
     const long long N = (long long)B * Tn;
     const int HW4 = H * GC_W;
+    if (N >= kGenWideTokens) {   // long prompts: 128-token CTAs, W1 read once per 128 tokens
+        const size_t smem = kgen::wide_smem_bytes();
+        if (smem_attr(kgen::gen_wide_kernel, smem) != JET_OK) return JET_ERR_CUDA;
+        return launch(kgen::gen_wide_kernel, dim3((unsigned)((N + kgen::WGT - 1) / kgen::WGT)), dim3(kgen::THREADS),
+                      smem, s, (const __nv_bfloat16*)x, (const __nv_bfloat16*)w1, (const __nv_bfloat16*)w2, taps, N,
+                      D, HW4);
+    }
     const size_t smem = kgen::smem_bytes(HW4);
     if (smem_attr(kgen::gen_kernel, smem) != JET_OK) return JET_ERR_CUDA;
     return launch(kgen::gen_kernel, dim3((unsigned)((N + kgen::GT - 1) / kgen::GT)), dim3(kgen::THREADS), smem, s,

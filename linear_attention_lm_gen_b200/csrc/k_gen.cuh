@@ -197,5 +197,127 @@ gen_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict_
     }
 }
 
+
+// Long prompts: one CTA = WGT = 128 tokens, and warp w owns token rows
+// [16 w, 16 w + 16) through every k-step of every slice, so W1 is read once
+// per 128 tokens instead of once per 32 (at T = 262144 that is 201 MB of W1
+// reads instead of 805, as much as the x stream itself) and no partial sums
+// meet across warps. Slices of WKC = 64 columns, WNST - 1 in flight; 89 KB
+// of shared memory, two CTAs per SM.
+constexpr int WGT = 128, WKC = 64, WNST = 3;
+constexpr int WXLD = WKC * 2 + 16;              // x row stride in a slice (bytes)
+constexpr int WXS_BYTES = WGT * WXLD;           // 18432
+constexpr int WST_BYTES = WXS_BYTES + WKC * WLD;   // + the W1 rows of the slice
+__host__ __device__ constexpr int wide_smem_bytes() { return WNST * WST_BYTES + WGT * HLD * 4; }
+
+__global__ void __launch_bounds__(THREADS, 2)
+gen_wide_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ W1,
+                const __nv_bfloat16* __restrict__ W2, float* __restrict__ taps, long long N, int D, int HW4) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    pdl_wait();
+    pdl_trigger();
+    float* hs = reinterpret_cast<float*>(smem + WNST * WST_BYTES);        // [WGT][HLD] hidden activations
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long r0 = (long long)blockIdx.x * WGT;
+    const int nsl = (D + WKC - 1) / WKC;
+    const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    // this thread's copies of a slice: x rows xr + 32 j (16 bytes at column 8 xc), W1 row wr (column 8 wc)
+    const int xr = tid >> 3, xc = tid & 7, wr = tid >> 2, wc = tid & 3;
+    int knext = (int)(blockIdx.x % (unsigned)nsl) * WKC;
+    int kcur = knext;
+    auto issue = [&](int stage) {
+        const uint32_t st = sbase + (uint32_t)stage * WST_BYTES;
+        const int k0 = knext;
+        knext = k0 + WKC >= nsl * WKC ? 0 : k0 + WKC;
+        const bool xin = k0 + xc * 8 < D;
+#pragma unroll
+        for (int j = 0; j < WGT / 32; ++j) {
+            const long long row = r0 + xr + 32 * j;
+            const bool ok = xin && row < N;
+            cp_async16(st + (uint32_t)((xr + 32 * j) * WXLD + xc * 16), ok ? x + row * D + k0 + xc * 8 : x,
+                       ok ? 16u : 0u);
+        }
+        const bool win = k0 + wr < D;
+        cp_async16(st + (uint32_t)(WXS_BYTES + wr * WLD + wc * 16),
+                   win ? W1 + (long long)(k0 + wr) * HID + wc * 8 : W1, win ? 16u : 0u);
+    };
+#pragma unroll
+    for (int s = 0; s < WNST - 1; ++s) {
+        if (s < nsl) issue(s);
+        cp_async_commit();
+    }
+    const int ng = THREADS / HW4;
+    const int col = tid % HW4, tg = tid / HW4;
+    uint32_t w2p[HID / 2];
+#pragma unroll
+    for (int r = 0; r < HID; r += 2) {
+        const uint16_t lo = tg < ng ? reinterpret_cast<const uint16_t*>(W2)[(long long)r * HW4 + col] : 0;
+        const uint16_t hi = tg < ng ? reinterpret_cast<const uint16_t*>(W2)[(long long)(r + 1) * HW4 + col] : 0;
+        w2p[r / 2] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    float acc[4][4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+    // ldmatrix rows: A (x) rows 16 warp + (lane & 15), k-offset 8 (lane >> 4); B (W1 [k][n], transposed)
+    // k-rows (lane & 15) of n-tile pair (lane >> 4)
+    const uint32_t a_off = (uint32_t)((16 * warp + (lane & 15)) * WXLD + (lane >> 4) * 16);
+    const uint32_t b_off = (uint32_t)(WXS_BYTES + (lane & 15) * WLD + (lane >> 4) * 16);
+    int stage = 0;
+    for (int s = 0; s < nsl; ++s) {
+        cp_async_wait<WNST - 2>();
+        __syncthreads();
+        if (s + WNST - 1 < nsl) issue(stage == 0 ? WNST - 1 : stage - 1);
+        cp_async_commit();
+        const uint32_t st = sbase + (uint32_t)stage * WST_BYTES;
+        const int kn = min(WKC, D - kcur) / 16;     // k-steps of this slice (D % 16 == 0)
+        for (int kk = 0; kk < kn; ++kk) {
+            uint32_t a[4], b[2][4];
+            ldsm_x4(st + a_off + (uint32_t)(kk * 32), a);
+            ldsm_x4_t(st + b_off + (uint32_t)(kk * 16 * WLD), b[0]);        // n-tiles 0, 1
+            ldsm_x4_t(st + b_off + (uint32_t)(kk * 16 * WLD) + 32, b[1]);   // n-tiles 2, 3
+#pragma unroll
+            for (int n = 0; n < 4; ++n) mma16816(acc[n], a, b[n >> 1][(n & 1) * 2], b[n >> 1][(n & 1) * 2 + 1]);
+        }
+        kcur = kcur + WKC >= nsl * WKC ? 0 : kcur + WKC;
+        stage = stage + 1 == WNST ? 0 : stage + 1;
+    }
+    cp_async_wait<0>();
+    {   // SiLU of this warp's 16 x 32 product (rows 16 warp + g and + 8, columns 8 n + 2 t4 and + 1)
+        const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+        for (int n = 0; n < 4; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = 16 * warp + g + (e >= 2 ? 8 : 0), c = 8 * n + 2 * t4 + (e & 1);
+                const float z = acc[n][e];
+                hs[r * HLD + c] = z / (1.0f + expf(-z));
+            }
+    }
+    __syncthreads();
+    if (tg >= ng) return;
+    float w2[HID];
+#pragma unroll
+    for (int r = 0; r < HID / 2; ++r) {
+        w2[2 * r] = __uint_as_float(w2p[r] << 16);
+        w2[2 * r + 1] = __uint_as_float(w2p[r] & 0xffff0000u);
+    }
+    const int nrows = (int)(N - r0 < WGT ? N - r0 : WGT);
+    for (int t = tg; t < nrows; t += ng) {
+        const float4* hr = reinterpret_cast<const float4*>(hs + t * HLD);
+        float a = 0.f;
+#pragma unroll
+        for (int r4 = 0; r4 < HID / 4; ++r4) {
+            const float4 hv = hr[r4];
+            a = fmaf(hv.x, w2[4 * r4], a);
+            a = fmaf(hv.y, w2[4 * r4 + 1], a);
+            a = fmaf(hv.z, w2[4 * r4 + 2], a);
+            a = fmaf(hv.w, w2[4 * r4 + 3], a);
+        }
+        taps[(r0 + t) * HW4 + col] = a;
+    }
+}
+
 }  // namespace kgen
 }  // namespace jet
