@@ -112,12 +112,12 @@ def test_generator_and_conv_stage(orc, dtype, B, T, H, dv, D, hist):
 
 
 @pytest.mark.parametrize("B,T,H,D", [(1, 4096, 12, 1536), (2, 1553, 16, 2048), (1, 1024, 3, 80),
-                                     (2, 16411, 12, 1536), (1, 33000, 3, 80)])
+                                     (3, 5001, 12, 1536), (2, 16411, 12, 1536), (1, 33000, 3, 80)])
 def test_generator_long_prompt(orc, B, T, H, D):
     # prompts of 1024+ tokens take the stand-alone generator (32 tokens per CTA, D in
-    # 128-column slices: D = 80 is one partial slice, 2 x 1553 tokens end mid-CTA);
-    # from 32768 tokens on, 128 tokens per CTA in 64-column slices (D = 80: a partial
-    # second slice; 2 x 16411 and 33000 tokens end mid-CTA)
+    # 128-column slices: D = 80 is one partial slice, 2 x 1553 and 3 x 5001 tokens end
+    # mid-CTA); from 32768 tokens on, 128 tokens per CTA in 64-column slices (D = 80: a
+    # partial second slice; 2 x 16411 and 33000 tokens end mid-CTA)
     s = shape("bf16", B=B, T=T, H=H, dv=32, D=D)
     inp = synth.prefill_inputs(s, seed=4)
     d = gpu_inputs(inp)
