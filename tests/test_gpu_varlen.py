@@ -108,3 +108,35 @@ def test_varlen_prefill_normalises_q_and_k():
                                  packed["beta"][a:b][None], S0[i:i + 1].astype(np.float64))
         assert_close(host64(o[a:b]), r["o"][0], "bf16", f"o of prompt {i}")
         assert_close(host64(S[i]), r["S"][0], "bf16", f"S of prompt {i}")
+
+
+def test_varlen_prefill_at_the_sequence_limit():
+    # 256 prompts (the most one call takes) of 1 to 300 tokens, seeded: every prompt against one
+    # jet_jetblock_prefill call of its own, and a sample of them against the oracle
+    rng = np.random.default_rng(5)
+    lens = rng.integers(1, 301, 256).tolist()
+    per, packed, W1, W2, S0 = packed_inputs(lens, 2, 64, 128, 64, seed=300, gate_scale=0.1)
+    d = {key: dev(val, "bf16") for key, val in packed.items() if key not in ("g", "beta")}
+    d["g"], d["beta"] = dev(packed["g"], "f32"), dev(packed["beta"], "f32")
+    w1, w2 = dev(W1, "bf16"), dev(W2, "bf16")
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    hout = torch.empty((256, 3, 2, 128), device="cuda", dtype=torch.bfloat16)
+    o, S = jet.jet_jetblock_prefill_varlen(d["x"], w1, w2, d["q"], d["k"], d["v"], d["g"], d["beta"], cu,
+                                           hist_out=hout, S0=dev(S0, "f32"))
+    assert jet.jet_device_error() == 0
+    for i in range(256):
+        sl = lambda key: d[key][cu[i]:cu[i + 1]].unsqueeze(0).contiguous()
+        h1 = torch.empty((1, 3, 2, 128), device="cuda", dtype=torch.bfloat16)
+        o1, S1 = jet.jet_jetblock_prefill(sl("x"), w1, w2, sl("q"), sl("k"), sl("v"), sl("g"), sl("beta"),
+                                          hist_out=h1, S0=dev(S0[i:i + 1], "f32"))
+        assert_close(host64(o[cu[i]:cu[i + 1]]), host64(o1[0]), "bf16", f"o of prompt {i}")
+        assert_close(host64(S[i]), host64(S1[0]), "bf16", f"S of prompt {i}")
+        assert torch.equal(hout[i], h1[0])
+    orc = get_oracle()
+    f = lambda a: synth.to_f64(a, "bf16")
+    for i in (0, 7, 100, 255):
+        p = per[i]
+        r = orc.jetblock_prefill(f(p["x"]), f(W1), f(W2), f(p["q"]), f(p["k"]), f(p["v"]), p["g"], p["beta"],
+                                 p["S0"].astype(np.float64))
+        assert_close(host64(o[cu[i]:cu[i + 1]]), r["o"][0], "bf16", f"o of prompt {i} vs the oracle")
+        assert_close(host64(S[i]), r["S"][0], "bf16", f"S of prompt {i} vs the oracle")
