@@ -420,10 +420,14 @@ jet_status launch_correct(const __nv_bfloat16* Qe, const __nv_bfloat16* Sb, void
         auto kern = pfcor::prefill_correct_group_kernel<DK, DV>;
         const size_t smem = pfcor::smem_group_bytes(DK, DV);
         if (smem_attr(kern, smem) != JET_OK) return JET_ERR_CUDA;
-        const int gps = (segc + pfcor::CH - 1) / pfcor::CH;
         const int nseg = (nct + segc - 1) / segc - chunk0 / segc;
+        // one wave: (segment, head, sequence) pairs times groups per segment within the SMs
+        const long long pairs = (long long)nseg * H * B;
+        const int gmax = (int)std::max<long long>(1, launch_sms() / std::max<long long>(1, pairs));
+        const int ch = std::max(1, (segc + gmax - 1) / gmax);
+        const int gps = (segc + ch - 1) / ch;
         return launch(kern, dim3(nseg * gps, H, B), dim3(pfcor::GTHREADS), smem, s, Qe, Sb, (__nv_bfloat16*)o, Tn, H,
-                      nct, chunk0, segc, P);
+                      nct, chunk0, segc, P, ch);
     }
     auto kern = pfcor::prefill_correct_kernel<DK, DV>;
     const size_t smem = pfcor::smem_bytes(DK, DV);

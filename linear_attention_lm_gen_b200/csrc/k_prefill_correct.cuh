@@ -183,21 +183,24 @@ prefill_correct_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16
 namespace jet {
 namespace pfcor {
 
-// Dense layout, CH consecutive chunks of one segment per CTA: S* is loaded
-// once and the chunks' Qe and output tiles are double-buffered, so the next
-// chunk's copies run while this one's product is formed. Segments p0 = chunk0
-// / segc .. P-1; grid (groups of the segments, H, B) with ceil(segc / CH)
-// groups per segment (a group past the sequence end returns at once).
-constexpr int CH = 4;
+// Dense layout, `ch` consecutive chunks of one segment per CTA (the host
+// picks ch so that the grid is one wave of the SMs): S* is loaded once and
+// the chunks' Qe and output tiles stream through NBUF buffers, NBUF - 1 chunks
+// of copies in flight while one chunk's product is formed. Segments p0 =
+// chunk0 / segc .. P-1; grid (groups of the segments, H, B) with
+// ceil(segc / ch) groups per segment (a group past the sequence end returns
+// at once).
+constexpr int NBUF = 3;
 constexpr int GTHREADS = 512;            // 16 warps: warp w owns output columns [w dv/16, (w+1) dv/16)
 __host__ __device__ constexpr size_t smem_group_bytes(int dk, int dv) {
-    return 2 * ((size_t)dv * lda(dk) + 2 * (size_t)C * lda(dk) + 2 * (size_t)C * ldo(dv));
+    return 2 * ((size_t)dv * lda(dk) + NBUF * (size_t)C * lda(dk) + NBUF * (size_t)C * ldo(dv));
 }
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(GTHREADS)
 prefill_correct_group_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bfloat16* __restrict__ Sb,
-                             __nv_bfloat16* __restrict__ o, int Tn, int H, int nct, int chunk0, int segc, int P) {
+                             __nv_bfloat16* __restrict__ o, int Tn, int H, int nct, int chunk0, int segc, int P,
+                             int ch) {
     static_assert(DK % 16 == 0 && DK <= 128 && DV % 64 == 0 && DV <= 256, "shapes");
     constexpr int LDA = lda(DK), LDO = ldo(DV);
     constexpr int NT = DV / 128;                 // n8 tiles per warp (DV / 16 columns)
@@ -205,14 +208,14 @@ prefill_correct_group_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bf
     static_assert(NT >= 1, "dv >= 128");
     extern __shared__ __align__(16) uint8_t smem[];
     __nv_bfloat16* ss = reinterpret_cast<__nv_bfloat16*>(smem);          // [DV][LDA]
-    __nv_bfloat16* qs0 = ss + DV * LDA;                                  // [2][64][LDA]
-    __nv_bfloat16* os0 = qs0 + 2 * C * LDA;                              // [2][64][LDO]
+    __nv_bfloat16* qs0 = ss + DV * LDA;                                  // [NBUF][64][LDA]
+    __nv_bfloat16* os0 = qs0 + NBUF * C * LDA;                           // [NBUF][64][LDO]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.y, b = blockIdx.z;
-    const int gps = (segc + CH - 1) / CH;                                // groups per segment
+    const int gps = (segc + ch - 1) / ch;                                // groups per segment
     const int p = chunk0 / segc + (int)blockIdx.x / gps;
-    const int first = p * segc + ((int)blockIdx.x % gps) * CH;
-    const int last = min(min(first + CH, (p + 1) * segc), nct);          // chunks [first, last)
+    const int first = p * segc + ((int)blockIdx.x % gps) * ch;
+    const int last = min(min(first + ch, (p + 1) * segc), nct);          // chunks [first, last)
     if (first >= last) return;
     const int n = last - first;
     pdl_wait();
@@ -220,10 +223,10 @@ prefill_correct_group_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bf
     const long long tstride = (long long)H * DV;
     const long long row_b = (long long)b * Tn;
 
-    auto issue_chunk = [&](int j) {      // Qe and output tiles of chunk first + j into buffer j & 1
+    auto issue_chunk = [&](int j) {      // Qe and output tiles of chunk first + j into buffer j % NBUF
         const int gc = first + j, L = min(C, Tn - gc * C);
-        __nv_bfloat16* qs = qs0 + (j & 1) * C * LDA;
-        __nv_bfloat16* os = os0 + (j & 1) * C * LDO;
+        __nv_bfloat16* qs = qs0 + (j % NBUF) * C * LDA;
+        __nv_bfloat16* os = os0 + (j % NBUF) * C * LDO;
         const __nv_bfloat16* src = Qe + (((long long)b * H + h) * nct + gc) * C * DK;
 #pragma unroll
         for (int i = tid; i < C * DK / 8; i += GTHREADS) {
@@ -246,18 +249,21 @@ prefill_correct_group_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bf
             cp_async16(ss + r * LDA + cc * 8, src + i * 8, 16u);
         }
     }
-    issue_chunk(0);
-    if (n > 1) issue_chunk(1);
+    for (int j = 0; j < NBUF - 1 && j < n; ++j) issue_chunk(j);
 
     const int n0 = warp * (DV / 16);
     const int g = lane >> 2, t4 = lane & 3;
     const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(ss));
     for (int j = 0; j < n; ++j) {
-        if (j + 1 < n) asm volatile("cp.async.wait_group 1;" ::: "memory");
+        // chunk j's copies: the groups committed after it may stay in flight
+        const int after = min(NBUF - 2, n - 1 - j);
+        if (after >= 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
         else asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncthreads();
-        __nv_bfloat16* qs = qs0 + (j & 1) * C * LDA;
-        __nv_bfloat16* os = os0 + (j & 1) * C * LDO;
+        // the buffer of chunk j - 1 is free (read out before the barrier): chunk j + NBUF - 1 into it
+        if (j + NBUF - 1 < n) issue_chunk(j + NBUF - 1);
+        __nv_bfloat16* qs = qs0 + (j % NBUF) * C * LDA;
+        __nv_bfloat16* os = os0 + (j % NBUF) * C * LDO;
         const uint32_t qbase = static_cast<uint32_t>(__cvta_generic_to_shared(qs));
         float acc[4][NT][4];
 #pragma unroll
@@ -301,8 +307,6 @@ prefill_correct_group_kernel(const __nv_bfloat16* __restrict__ Qe, const __nv_bf
                 *reinterpret_cast<uint4*>(o + (row0 + r) * tstride + h * DV + cc * 8) =
                     *reinterpret_cast<const uint4*>(os + r * LDO + cc * 8);
         }
-        __syncthreads();                                  // buffer j & 1 read out: free for chunk j + 2
-        if (j + 2 < n) issue_chunk(j + 2);
     }
 }
 
